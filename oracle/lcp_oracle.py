@@ -1,0 +1,270 @@
+"""Plain CPU oracle of the learnable-channel-permutation (LCP) hot path, in float64.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline / reference legs of ``bench.py`` may import or run this module.
+It shares no code with the CUDA path: no kernels, no helpers, no tables.
+
+Sources (the web pages the method is taken from):
+
+* [PermLLM]  "PermLLM: Learnable Channel Permutation for N:M Sparse Large
+  Language Models" (summary page of arXiv 2510.10136): section "Method",
+  subsections 1 (soft permutation relaxation: S_0(X) = exp(X),
+  S_i(X) = T_c(T_r(S_{i-1}(X))), P_hat = S_L(W_P / tau)), 3 (block-wise
+  permutation: P_B = diag(P_1, ..., P_NB), W_hat_B = W P_B), "optimization
+  objective" (L_cos(y, y~) = 1 - y.y~ / (|y| |y~|)) and "integration with
+  existing pruning methods" (the mask keeps the best N of every group of M
+  consecutive columns, straight-through estimator in the backward pass).
+* [Blog]  "PermLLM: dynamic channel permutation for N:M sparse LLMs"
+  (intelliparadigm.com): section 2.1 (plain N:M pruning: groups of M, keep the
+  N largest |w|, zero the rest) and section 2.2 (Sinkhorn in the log domain,
+  row normalisation first, then column normalisation, then exp).
+
+Readings where the pages are silent or garbled (each is restated where used):
+
+1. The forward pass uses the soft P (no Hungarian hardening).
+2. The mask score is |W'| with W' = W P_B.
+3. The mask is a constant in the backward pass (straight-through).
+4. One iteration = a row normalisation followed by a column normalisation.
+5. Z_0 = L / tau.
+6. Equal magnitudes: the lower channel index is kept first (+0 and -0 tie).
+7. Groups are M consecutive input channels of W' (permuted order).
+8. Cosine denominator max(|y_d| |y_s|, 1e-8).
+9. The loss is the mean over the T tokens (columns of Y).
+
+Notation follows the pages: W is C_out x C_in, X is the C_in x T matrix of
+calibration activations (the callers store it token-major, [T, C_in]; this
+module transposes it once at entry), L are the learnable logits of the
+C_in / B diagonal blocks of the permutation, each B x B, P_b[i, j] moving
+source channel bB+i to permuted slot bB+j.
+"""
+
+from __future__ import annotations
+
+from typing import Dict, List, Optional, Tuple
+
+import numpy as np
+
+COS_EPS = 1e-8
+
+
+# ---------------------------------------------------------------------------
+# Sinkhorn normalisation  ([PermLLM] Method 1; [Blog] 2.2)
+# ---------------------------------------------------------------------------
+
+def logsumexp(z: np.ndarray, axis: int) -> np.ndarray:
+    """log(sum(exp(z))) along ``axis`` with the maximum shifted out (kept dims)."""
+    mx = np.max(z, axis=axis, keepdims=True)
+    return mx + np.log(np.sum(np.exp(z - mx), axis=axis, keepdims=True))
+
+
+def sinkhorn(logits: np.ndarray, tau: float, n_iters: int) -> Tuple[np.ndarray, List[np.ndarray]]:
+    """Soft block permutations P_b = S_L(L_b / tau) for every block b.
+
+    ``logits`` has shape [nb, B, B].  In the log domain S_0 = exp is applied
+    last: starting from Z = L / tau, each of the ``n_iters`` iterations first
+    subtracts every row's log-sum-exp (T_r: rows sum to one) and then every
+    column's (T_c: columns sum to one); P = exp(Z).
+
+    Returns P and the trace [Z_0, Z after T_r of iteration 1, Z after T_c of
+    iteration 1, ...] (2 * n_iters + 1 arrays) that the backward pass replays.
+    """
+    Z = np.asarray(logits, dtype=np.float64) / float(tau)
+    trace = [Z]
+    for _ in range(n_iters):
+        Z = Z - logsumexp(Z, axis=2)      # T_r: normalise each row i over j
+        trace.append(Z)
+        Z = Z - logsumexp(Z, axis=1)      # T_c: normalise each column j over i
+        trace.append(Z)
+    return np.exp(Z), trace
+
+
+def sinkhorn_backward(trace: List[np.ndarray], P: np.ndarray, dP: np.ndarray, tau: float) -> np.ndarray:
+    """Gradient of a scalar loss w.r.t. the logits, given dloss/dP.
+
+    Reverse-mode through P = exp(Z_final) and each normalisation:
+    a column step Z' = Z - lse_col(Z) has Jacobian delta_ik - exp(Z'_kj), so
+    dZ = dZ' - exp(Z') * colsum(dZ'); a row step likewise with row sums.
+    Finally Z_0 = L / tau gives dL = dZ_0 / tau.
+    """
+    dZ = np.asarray(dP, np.float64) * P
+    for s in range(len(trace) - 1, 0, -1):
+        Z_after = trace[s]
+        if s % 2 == 0:   # column normalisation (T_c)
+            dZ = dZ - np.exp(Z_after) * np.sum(dZ, axis=1, keepdims=True)
+        else:            # row normalisation (T_r)
+            dZ = dZ - np.exp(Z_after) * np.sum(dZ, axis=2, keepdims=True)
+    return dZ / float(tau)
+
+
+# ---------------------------------------------------------------------------
+# Block-diagonal permutation  ([PermLLM] Method 3)
+# ---------------------------------------------------------------------------
+
+def block_diag(P: np.ndarray) -> np.ndarray:
+    """The dense C_in x C_in matrix P_B = diag(P_1, ..., P_NB)."""
+    nb, B, _ = P.shape
+    out = np.zeros((nb * B, nb * B), dtype=np.float64)
+    for b in range(nb):
+        out[b * B:(b + 1) * B, b * B:(b + 1) * B] = P[b]
+    return out
+
+
+def permute_weight(W: np.ndarray, P: np.ndarray) -> np.ndarray:
+    """W' = W P_B, one block of columns at a time (P_B is zero off the diagonal)."""
+    W = np.asarray(W, np.float64)
+    nb, B, _ = P.shape
+    Wp = np.empty_like(W)
+    for b in range(nb):
+        Wp[:, b * B:(b + 1) * B] = W[:, b * B:(b + 1) * B] @ P[b]
+    return Wp
+
+
+def permute_inputs(P: np.ndarray, Xc: np.ndarray) -> np.ndarray:
+    """Xp = P_B^T X for X given as C_in x T: permuted channel bB+k mixes sources bB+i by P_b[i, k]."""
+    nb, B, _ = P.shape
+    Xp = np.empty_like(Xc)
+    for b in range(nb):
+        Xp[b * B:(b + 1) * B, :] = P[b].T @ Xc[b * B:(b + 1) * B, :]
+    return Xp
+
+
+# ---------------------------------------------------------------------------
+# N:M magnitude mask  ([Blog] 2.1; [PermLLM] integration with pruning methods)
+# ---------------------------------------------------------------------------
+
+def nm_mask(Wp: np.ndarray, n: int, m: int) -> np.ndarray:
+    """Boolean mask keeping, in every row, the n largest |W'| of each group of m
+    consecutive columns.  Equal magnitudes keep the lower column first.
+
+    The comparison is made in the precision of the array passed in (a float32
+    W' is compared as float32).
+    """
+    rows, cols = Wp.shape
+    if cols % m:
+        raise ValueError("columns must be a multiple of m")
+    mag = np.abs(Wp).reshape(rows, cols // m, m)
+    # stable sort of -|w|: largest first, equal keys in index order
+    order = np.argsort(-mag, axis=2, kind="stable")
+    keep = np.zeros(mag.shape, dtype=bool)
+    np.put_along_axis(keep, order[:, :, :n], True, axis=2)
+    return keep.reshape(rows, cols)
+
+
+def pack_mask_bits(mask: np.ndarray) -> np.ndarray:
+    """Pack a [rows, cols] boolean mask into uint32 words: bit (j % 32) of word j // 32."""
+    rows, cols = mask.shape
+    if cols % 32:
+        raise ValueError("columns must be a multiple of 32")
+    bits = mask.reshape(rows, cols // 32, 32).astype(np.uint64)
+    weights = (np.uint64(1) << np.arange(32, dtype=np.uint64))
+    return (bits * weights).sum(axis=2).astype(np.uint32)
+
+
+def unpack_mask_bits(words: np.ndarray, cols: int) -> np.ndarray:
+    words = np.asarray(words, np.uint32)
+    rows = words.shape[0]
+    shifts = np.arange(32, dtype=np.uint32)
+    bits = (words[:, :, None] >> shifts) & np.uint32(1)
+    return bits.reshape(rows, -1)[:, :cols].astype(bool)
+
+
+# ---------------------------------------------------------------------------
+# Cosine objective  ([PermLLM] optimization objective)
+# ---------------------------------------------------------------------------
+
+def cosine_loss(Yd: np.ndarray, Ys: np.ndarray) -> Tuple[float, np.ndarray]:
+    """Mean over tokens (columns) of 1 - cos(y_d, y_s); returns (loss, cos per token)."""
+    dot = np.sum(Yd * Ys, axis=0)
+    nd = np.sqrt(np.sum(Yd * Yd, axis=0))
+    ns = np.sqrt(np.sum(Ys * Ys, axis=0))
+    cos = dot / np.maximum(nd * ns, COS_EPS)
+    return float(np.mean(1.0 - cos)), cos
+
+
+def cosine_loss_grad(Yd: np.ndarray, Ys: np.ndarray) -> np.ndarray:
+    """d loss / d Ys for the token-averaged cosine loss (same shape as Ys)."""
+    T = Ys.shape[1]
+    dot = np.sum(Yd * Ys, axis=0)
+    nd = np.sqrt(np.sum(Yd * Yd, axis=0))
+    ns = np.sqrt(np.sum(Ys * Ys, axis=0))
+    den = nd * ns
+    G = np.empty_like(Ys)
+    ok = den > COS_EPS
+    c = np.where(ok, dot / np.where(ok, den, 1.0), 0.0)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        g_ok = -(Yd / np.where(ok, den, 1.0) - c * Ys / np.where(ok, ns * ns, 1.0)) / T
+    g_clamped = -(Yd / COS_EPS) / T
+    G[:, ok] = g_ok[:, ok]
+    G[:, ~ok] = g_clamped[:, ~ok]
+    return G
+
+
+# ---------------------------------------------------------------------------
+# One forward + backward step of one layer
+# ---------------------------------------------------------------------------
+
+def forward(W: np.ndarray, X_tokens: np.ndarray, logits: np.ndarray, tau: float, n_iters: int,
+            n: int, m: int, mask: Optional[np.ndarray] = None, Wp: Optional[np.ndarray] = None,
+            P: Optional[np.ndarray] = None) -> Dict[str, object]:
+    """Forward pass in the pages' order.
+
+    ``X_tokens`` is [T, C_in]; internally X = X_tokens^T (C_in x T).
+    ``mask`` / ``Wp`` / ``P`` inject a given mask, permuted weight or soft
+    permutation in place of the computed one (used to compare with another
+    implementation on identical intermediate values).
+    """
+    W = np.asarray(W, np.float64)
+    Xc = np.asarray(X_tokens, np.float64).T
+    trace = None
+    if P is None:
+        P, trace = sinkhorn(logits, tau, n_iters)
+    else:
+        P = np.asarray(P, np.float64)
+    Wp_used = permute_weight(W, P) if Wp is None else np.asarray(Wp)
+    M = nm_mask(Wp_used, n, m) if mask is None else np.asarray(mask, bool)
+    Wp64 = np.asarray(Wp_used, np.float64)
+    A = np.where(M, Wp64, 0.0)
+    Xp = permute_inputs(P, Xc)
+    Ys = A @ Xp
+    Yd = W @ Xc
+    loss, cos = cosine_loss(Yd, Ys)
+    return dict(P=P, trace=trace, Wp=Wp64, mask=M, A=A, Xc=Xc, Xp=Xp, Yd=Yd, Ys=Ys,
+                loss=loss, cos=cos, W=W)
+
+
+def backward(fw: Dict[str, object], tau: float) -> Dict[str, np.ndarray]:
+    """Hand-written reverse pass to the logits, mask held constant (straight-through).
+
+    Ys = A Xp        ->  dA = G Xp^T,  dXp = A^T G
+    Xp = P_B^T X     ->  dP_b += X_b dXp_b^T
+    A = M * W'       ->  dW' = M * dA
+    W' = W P_B       ->  dP_b += W_b^T dW'_b
+    then back through the Sinkhorn normalisations.
+    """
+    P = fw["P"]
+    nb, B, _ = P.shape
+    G = cosine_loss_grad(fw["Yd"], fw["Ys"])
+    dA = G @ fw["Xp"].T
+    dXp = fw["A"].T @ G
+    dWp = np.where(fw["mask"], dA, 0.0)
+    W, Xc = fw["W"], fw["Xc"]
+    dP = np.empty_like(P)
+    for b in range(nb):
+        s = slice(b * B, (b + 1) * B)
+        dP[b] = Xc[s, :] @ dXp[s, :].T + W[:, s].T @ dWp[:, s]
+    out = dict(G=G, dA=dA, dWp=dWp, dP=dP)
+    if fw["trace"] is not None:
+        out["dL"] = sinkhorn_backward(fw["trace"], P, dP, tau)
+    return out
+
+
+def step(W: np.ndarray, X_tokens: np.ndarray, logits: np.ndarray, tau: float, n_iters: int,
+         n: int, m: int, mask: Optional[np.ndarray] = None) -> Dict[str, object]:
+    """Forward and backward of one layer; returns the forward dict plus G, dP, dL."""
+    fw = forward(W, X_tokens, logits, tau, n_iters, n, m, mask=mask)
+    fw.update(backward(fw, tau))
+    return fw
+
+
+def loss_of_logits(W, X_tokens, logits, tau, n_iters, n, m, mask=None) -> float:
+    return forward(W, X_tokens, logits, tau, n_iters, n, m, mask=mask)["loss"]

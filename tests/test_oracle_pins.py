@@ -1,0 +1,418 @@
+"""Pins of the CPU oracle to facts fixed by the pages and by mathematics.
+
+Each test checks the oracle against something other than itself: a closed
+form, an invariant, a textbook special case written independently, brute force
+over every permutation of a toy layer, or finite differences.  A plausible
+slip in the oracle (rows and columns swapped, iteration order reversed, tau
+dropped, P used where P^T belongs, a backward term dropped, the tie rule
+reversed) fails at least one of them.
+"""
+
+import itertools
+import math
+
+import numpy as np
+import pytest
+
+from oracle import lcp_oracle as O
+
+
+def rand(shape, seed, scale=1.0):
+    return np.random.default_rng(seed).standard_normal(shape) * scale
+
+
+# ---------------------------------------------------------------- Sinkhorn --
+
+def test_sinkhorn_zero_logits_give_uniform():
+    for B in (4, 32, 64):
+        P, _ = O.sinkhorn(np.zeros((3, B, B)), 0.5, 5)
+        assert np.allclose(P, 1.0 / B, rtol=0, atol=1e-15)
+
+
+def test_sinkhorn_additive_logits_give_uniform_after_one_iteration():
+    # L_ij = a_i + b_j: the row step removes a_i, the column step removes b_j.
+    B = 16
+    a, b = rand((B, 1), 1), rand((1, B), 2)
+    L = (a + b)[None]
+    for iters in (1, 2, 5):
+        P, _ = O.sinkhorn(L, 0.7, iters)
+        assert np.allclose(P, 1.0 / B, rtol=0, atol=1e-14)
+
+
+def test_sinkhorn_columns_sum_to_one_after_any_iteration_count():
+    L = rand((4, 32, 32), 3, 2.0)
+    for iters in (1, 2, 3, 5):
+        P, _ = O.sinkhorn(L, 0.5, iters)
+        assert np.allclose(P.sum(axis=1), 1.0, rtol=0, atol=1e-12)
+
+
+def test_sinkhorn_doubly_stochastic_at_init_scale():
+    # logits ~ N(0, 1e-3) (initialisation std of the blog page, section 6)
+    L = rand((64, 64, 64), 4, 1e-3)
+    P, _ = O.sinkhorn(L, 0.5, 5)
+    assert np.max(np.abs(P.sum(axis=1) - 1)) < 1e-12
+    assert np.max(np.abs(P.sum(axis=2) - 1)) < 1e-5
+
+
+def test_sinkhorn_peaked_logits_converge_to_doubly_stochastic():
+    rng = np.random.default_rng(5)
+    L = np.stack([np.eye(32)[rng.permutation(32)] * 3.0 + rng.standard_normal((32, 32)) * 0.5
+                  for _ in range(3)])
+    P, _ = O.sinkhorn(L, 1.0, 200)
+    assert np.max(np.abs(P.sum(axis=1) - 1)) < 1e-12
+    assert np.max(np.abs(P.sum(axis=2) - 1)) < 1e-5
+
+
+def test_sinkhorn_equals_linear_domain_sinkhorn_knopp_row_first():
+    # Textbook Sinkhorn-Knopp in the linear domain, in the order the pages fix:
+    # S_i = T_c(T_r(S_{i-1})), i.e. rows normalised before columns.
+    rng = np.random.default_rng(6)
+    L = rng.standard_normal((2, 8, 8)) * 1.5
+    tau = 0.6
+    for iters in (1, 2, 3, 7):
+        K = np.exp(L / tau)
+        for _ in range(iters):
+            for b in range(K.shape[0]):
+                for i in range(8):
+                    K[b, i, :] = K[b, i, :] / sum(K[b, i, :])
+                for j in range(8):
+                    K[b, :, j] = K[b, :, j] / sum(K[b, :, j])
+        P, _ = O.sinkhorn(L, tau, iters)
+        assert np.allclose(P, K, rtol=1e-12, atol=0)
+
+
+def test_sinkhorn_order_matters_so_the_previous_test_bites():
+    rng = np.random.default_rng(7)
+    L = rng.standard_normal((1, 8, 8))
+    P, _ = O.sinkhorn(L, 1.0, 1)
+    K = np.exp(L[0])
+    K = K / K.sum(axis=0, keepdims=True)
+    K = K / K.sum(axis=1, keepdims=True)          # column first: the wrong order
+    assert not np.allclose(P[0], K, rtol=1e-6, atol=0)
+
+
+def test_sinkhorn_2x2_limit_closed_form_with_temperature():
+    # A positive 2x2 matrix scaled to doubly stochastic form is [[p,1-p],[1-p,p]]
+    # and diagonal scaling keeps the cross ratio: p^2/(1-p)^2 = K00 K11 / (K01 K10),
+    # so p = sigmoid((Z00 + Z11 - Z01 - Z10) / 2) with Z = L / tau.
+    rng = np.random.default_rng(8)
+    for _ in range(20):
+        L = rng.standard_normal((1, 2, 2))
+        tau = float(rng.uniform(0.5, 2.0))
+        d = (L[0, 0, 0] + L[0, 1, 1] - L[0, 0, 1] - L[0, 1, 0]) / tau
+        p = 1.0 / (1.0 + math.exp(-d / 2))
+        P, _ = O.sinkhorn(L, tau, 3000)
+        assert np.allclose(P[0], [[p, 1 - p], [1 - p, p]], rtol=0, atol=1e-10)
+
+
+def test_sinkhorn_row_shift_invariance():
+    L = rand((3, 16, 16), 9)
+    shift = rand((3, 16, 1), 10, 5.0)
+    P1, _ = O.sinkhorn(L, 0.5, 4)
+    P2, _ = O.sinkhorn(L + shift, 0.5, 4)
+    assert np.allclose(P1, P2, rtol=1e-12, atol=1e-15)
+
+
+def test_sinkhorn_peaked_permutation_is_recovered_exactly():
+    rng = np.random.default_rng(11)
+    B, nb = 32, 3
+    sig = [rng.permutation(B) for _ in range(nb)]
+    L = np.zeros((nb, B, B))
+    for b in range(nb):
+        L[b, np.arange(B), sig[b]] = 60.0       # P_b[i, sigma(i)] = 1
+    P, _ = O.sinkhorn(L, 0.5, 5)
+    for b in range(nb):
+        Pi = np.zeros((B, B))
+        Pi[np.arange(B), sig[b]] = 1.0
+        assert np.array_equal(P[b], Pi) or np.max(np.abs(P[b] - Pi)) < 1e-40
+        assert np.array_equal(np.argmax(P[b], axis=1), sig[b])
+
+
+# ------------------------------------------------------- block permutation --
+
+def test_block_products_equal_dense_block_diagonal_products():
+    rng = np.random.default_rng(12)
+    W = rng.standard_normal((10, 24))
+    X = rng.standard_normal((24, 7))
+    P, _ = O.sinkhorn(rng.standard_normal((3, 8, 8)), 0.5, 3)
+    PB = O.block_diag(P)
+    assert np.allclose(O.permute_weight(W, P), W @ PB, rtol=1e-13, atol=1e-15)
+    assert np.allclose(O.permute_inputs(P, X), PB.T @ X, rtol=1e-13, atol=1e-15)
+    # block-diagonal structure
+    assert np.count_nonzero(PB) == 3 * 64
+
+
+def test_peaked_permutation_makes_wprime_an_exact_gather():
+    rng = np.random.default_rng(13)
+    B, nb = 8, 4
+    W = rng.standard_normal((5, nb * B))
+    L = np.zeros((nb, B, B))
+    sig = [rng.permutation(B) for _ in range(nb)]
+    for b in range(nb):
+        L[b, np.arange(B), sig[b]] = 80.0
+    P, _ = O.sinkhorn(L, 0.5, 5)
+    Wp = O.permute_weight(W, P)
+    for b in range(nb):
+        for i in range(B):   # source channel bB+i lands in slot bB+sigma(i)
+            assert np.array_equal(Wp[:, b * B + sig[b][i]], W[:, b * B + i])
+
+
+# ------------------------------------------------------------------ N:M mask --
+
+def _textbook_nm(W, n, m):
+    """Plain N:M magnitude pruning written with explicit loops and an explicit tie key."""
+    rows, cols = W.shape
+    keep = np.zeros((rows, cols), bool)
+    for r in range(rows):
+        for g in range(cols // m):
+            idx = list(range(g * m, (g + 1) * m))
+            best = sorted(idx, key=lambda j: (-abs(float(W[r, j])), j))[:n]
+            for j in best:
+                keep[r, j] = True
+    return keep
+
+
+@pytest.mark.parametrize("n,m", [(2, 4), (4, 8), (1, 4), (3, 4), (1, 8), (7, 8)])
+def test_mask_equals_textbook_pruning_with_ties(n, m):
+    rng = np.random.default_rng(14)
+    # quantised values give many exact ties, including +0 / -0
+    W = np.round(rng.standard_normal((12, 64)) * 2) / 2
+    W[0, :8] = [0.0, -0.0, 0.0, -0.0, 1.0, -1.0, 1.0, -1.0]
+    assert np.array_equal(O.nm_mask(W, n, m), _textbook_nm(W, n, m))
+
+
+def test_mask_characterisation_invariants():
+    rng = np.random.default_rng(15)
+    for (n, m) in ((2, 4), (4, 8)):
+        W = np.round(rng.standard_normal((40, 128)) * 3) / 3
+        M = O.nm_mask(W, n, m)
+        g = M.reshape(40, -1, m)
+        assert np.all(g.sum(axis=2) == n)
+        mag = np.abs(W).reshape(40, -1, m)
+        for r in range(40):
+            for k in range(g.shape[1]):
+                kept = [j for j in range(m) if g[r, k, j]]
+                drop = [j for j in range(m) if not g[r, k, j]]
+                for a in kept:
+                    for b in drop:
+                        assert mag[r, k, a] >= mag[r, k, b]
+                        if mag[r, k, a] == mag[r, k, b]:
+                            assert a < b
+
+
+def test_identity_logits_collapse_to_plain_nm_pruning():
+    rng = np.random.default_rng(16)
+    B, nb = 16, 4
+    W = rng.standard_normal((20, nb * B))
+    # exp(-800) underflows to 0 in float64, so P is exactly the identity
+    L = np.broadcast_to(np.eye(B) * 400.0, (nb, B, B)).copy()
+    P, _ = O.sinkhorn(L, 0.5, 5)
+    assert np.array_equal(P, np.broadcast_to(np.eye(B), P.shape))
+    Wp = O.permute_weight(W, P)
+    assert np.array_equal(Wp, W)
+    assert np.array_equal(O.nm_mask(Wp, 2, 4), _textbook_nm(W, 2, 4))
+
+
+def test_zero_logits_make_block_columns_equal_and_keep_the_first_n():
+    rng = np.random.default_rng(17)
+    B = 8
+    W = rng.standard_normal((6, 4 * B))
+    P, _ = O.sinkhorn(np.zeros((4, B, B)), 1.0, 5)
+    Wp = O.permute_weight(W, P)
+    # P = 1/B exactly, so every column of a block is the same block mean; the
+    # summation order can differ between columns only by rounding, so compare
+    # the mask on the exact block means instead.
+    means = np.repeat(W.reshape(6, 4, B).mean(axis=2), B, axis=1)
+    M = O.nm_mask(means, 2, 4)
+    assert np.all(M.reshape(6, -1, 4)[:, :, :2]) and not np.any(M.reshape(6, -1, 4)[:, :, 2:])
+    assert np.allclose(Wp, means, rtol=1e-14, atol=1e-16)
+
+
+def test_mask_bit_packing():
+    M = np.zeros((2, 64), bool)
+    M[0, 0::2] = True          # 0x55555555 in both words
+    M[1, 31] = True            # top bit of word 0
+    M[1, 32] = True            # bottom bit of word 1
+    words = O.pack_mask_bits(M)
+    assert words.dtype == np.uint32
+    assert words.tolist() == [[0x55555555, 0x55555555], [0x80000000, 0x00000001]]
+    assert np.array_equal(O.unpack_mask_bits(words, 64), M)
+
+
+# ------------------------------------------------------------------- loss --
+
+def test_cosine_loss_special_values():
+    rng = np.random.default_rng(18)
+    Yd = rng.standard_normal((9, 5))
+    assert abs(O.cosine_loss(Yd, Yd)[0]) < 1e-15
+    assert abs(O.cosine_loss(Yd, -Yd)[0] - 2.0) < 1e-15
+    assert abs(O.cosine_loss(Yd, 3.5 * Yd)[0]) < 1e-15
+    a = np.array([[1.0, 0.0], [0.0, 2.0]])
+    b = np.array([[0.0, 3.0], [1.0, 0.0]])
+    assert abs(O.cosine_loss(a, b)[0] - 1.0) < 1e-15
+    # one token at 45 degrees: 1 - 1/sqrt(2)
+    u = np.array([[1.0], [0.0]])
+    v = np.array([[1.0], [1.0]])
+    assert abs(O.cosine_loss(u, v)[0] - (1 - 1 / math.sqrt(2))) < 1e-15
+
+
+def test_cosine_loss_per_token_scale_invariance():
+    rng = np.random.default_rng(19)
+    Yd, Ys = rng.standard_normal((2, 11, 6))
+    s = rng.uniform(0.1, 10.0, size=6)
+    assert abs(O.cosine_loss(Yd * s, Ys * s)[0] - O.cosine_loss(Yd, Ys)[0]) < 1e-14
+
+
+def test_cosine_loss_gradient_by_finite_differences():
+    rng = np.random.default_rng(20)
+    Yd, Ys = rng.standard_normal((2, 7, 4))
+    G = O.cosine_loss_grad(Yd, Ys)
+    eps = 1e-6
+    num = np.zeros_like(Ys)
+    for idx in np.ndindex(Ys.shape):
+        e = np.zeros_like(Ys)
+        e[idx] = eps
+        num[idx] = (O.cosine_loss(Yd, Ys + e)[0] - O.cosine_loss(Yd, Ys - e)[0]) / (2 * eps)
+    assert np.linalg.norm(G - num) / np.linalg.norm(num) < 1e-8
+    # the gradient is orthogonal to y_s token by token (scale invariance)
+    assert np.max(np.abs(np.sum(G * Ys, axis=0))) < 1e-14
+
+
+# -------------------------------------------------------- brute force over 8! --
+
+def _hard_loss_independent(W, X_tokens, sigma, n, m):
+    """Loss of a hard permutation computed in original channel order.
+
+    Source channel i sits at permuted slot sigma[i].  Each group of m
+    consecutive slots is a set of source channels; in every row the n largest
+    |W| of that set survive (equal magnitudes: lower slot first).  The sparse
+    output is the pruned W applied to the unpermuted X.
+    """
+    rows, cols = W.shape
+    inv = np.argsort(sigma)                       # slot -> source channel
+    Ws = np.zeros_like(W)
+    for r in range(rows):
+        for g in range(cols // m):
+            slots = list(range(g * m, (g + 1) * m))
+            best = sorted(slots, key=lambda j: (-abs(W[r, inv[j]]), j))[:n]
+            for j in best:
+                Ws[r, inv[j]] = W[r, inv[j]]
+    X = X_tokens.T
+    yd, ys = W @ X, Ws @ X
+    c = np.sum(yd * ys, 0) / (np.linalg.norm(yd, axis=0) * np.linalg.norm(ys, axis=0))
+    return float(np.mean(1 - c))
+
+
+@pytest.mark.slow
+def test_brute_force_all_permutations_of_an_8_channel_toy():
+    rng = np.random.default_rng(21)
+    Cout, Cin, T, n, m = 16, 8, 32, 2, 4
+    W = rng.standard_normal((Cout, Cin)) * 0.02
+    X = rng.standard_normal((T, Cin))
+    perms = list(itertools.permutations(range(Cin)))
+    assert len(perms) == 40320
+    ind = np.array([_hard_loss_independent(W, X, np.array(s), n, m) for s in perms])
+    # only the partition of the 8 channels into two groups of 4 matters: 35 values
+    assert len(np.unique(np.round(ind, 12))) <= 35
+    # oracle forward with the hard permutation injected as P reproduces every loss
+    Pall = np.zeros((len(perms), 1, Cin, Cin))
+    for k, s in enumerate(perms):
+        Pall[k, 0, np.arange(Cin), np.array(s)] = 1.0
+    orc = np.array([O.forward(W, X, None, 1.0, 0, n, m, P=Pall[k])["loss"] for k in range(len(perms))])
+    assert np.max(np.abs(orc - ind)) < 1e-12
+    # ... and so do peaked logits through the Sinkhorn path (a sample of them)
+    for k in rng.choice(len(perms), 300, replace=False):
+        L = Pall[k] * 80.0
+        assert abs(O.forward(W, X, L, 0.5, 5, n, m)["loss"] - ind[k]) < 1e-12
+    best = np.argmin(ind)
+    assert ind[best] < ind[0] or best == 0
+
+
+def test_no_pruning_and_hard_permutation_gives_zero_loss():
+    rng = np.random.default_rng(22)
+    W = rng.standard_normal((6, 16))
+    X = rng.standard_normal((9, 16))
+    P = np.zeros((2, 8, 8))
+    for b in range(2):
+        P[b, np.arange(8), rng.permutation(8)] = 1.0
+    assert abs(O.forward(W, X, None, 1.0, 0, 4, 4, P=P)["loss"]) < 1e-14
+    # soft P: W P P^T != W, so the loss is positive even with nothing pruned
+    Ps, _ = O.sinkhorn(rng.standard_normal((2, 8, 8)), 1.0, 5)
+    assert O.forward(W, X, None, 1.0, 0, 4, 4, P=Ps)["loss"] > 1e-6
+
+
+def test_loss_invariant_to_weight_scale_and_token_scale():
+    rng = np.random.default_rng(23)
+    W = rng.standard_normal((12, 16)) * 0.02
+    X = rng.standard_normal((10, 16))
+    L = rng.standard_normal((2, 8, 8)) * 0.3
+    base = O.forward(W, X, L, 0.5, 5, 2, 4)["loss"]
+    assert abs(O.forward(3.0 * W, X, L, 0.5, 5, 2, 4)["loss"] - base) < 1e-13
+    s = rng.uniform(0.2, 5, size=(10, 1))
+    assert abs(O.forward(W, X * s, L, 0.5, 5, 2, 4)["loss"] - base) < 1e-13
+
+
+# ------------------------------------------------------------ gradient dL --
+
+def _fd_check(W, X, L, tau, iters, n, m, entries, eps=1e-6):
+    out = O.step(W, X, L, tau, iters, n, m)
+    dL = out["dL"]
+    num, ana = [], []
+    for idx in entries:
+        Lp, Lm = L.copy(), L.copy()
+        Lp[idx] += eps
+        Lm[idx] -= eps
+        fp = O.forward(W, X, Lp, tau, iters, n, m)
+        fm = O.forward(W, X, Lm, tau, iters, n, m)
+        if not (np.array_equal(fp["mask"], out["mask"]) and np.array_equal(fm["mask"], out["mask"])):
+            continue
+        num.append((fp["loss"] - fm["loss"]) / (2 * eps))
+        ana.append(dL[idx])
+    num, ana = np.array(num), np.array(ana)
+    assert len(num) >= 0.5 * len(entries)
+    return np.linalg.norm(num - ana) / np.linalg.norm(num)
+
+
+@pytest.mark.parametrize("iters,tau", [(1, 1.0), (3, 0.5), (5, 0.5)])
+def test_dL_matches_central_finite_differences(iters, tau):
+    rng = np.random.default_rng(24 + iters)
+    Cout, Cin, T, B = 24, 16, 20, 8
+    W = rng.standard_normal((Cout, Cin)) * 0.02
+    X = rng.standard_normal((T, Cin))
+    L = rng.standard_normal((Cin // B, B, B)) * 0.5
+    entries = [idx for idx in np.ndindex(L.shape)]
+    assert _fd_check(W, X, L, tau, iters, 2, 4, entries) < 1e-6
+
+
+def test_dL_finite_differences_4of8_with_outliers():
+    rng = np.random.default_rng(30)
+    Cout, Cin, T, B = 16, 32, 12, 16
+    W = rng.standard_normal((Cout, Cin)) * 0.02
+    W[:, 5] *= 10
+    X = rng.standard_normal((T, Cin))
+    X[:, 5] *= 5
+    L = rng.standard_normal((Cin // B, B, B)) * 0.5
+    entries = [tuple(int(v) for v in rng.integers(0, [2, B, B])) for _ in range(64)]
+    assert _fd_check(W, X, L, 0.5, 5, 4, 8, entries) < 1e-6
+
+
+def test_dL_rows_sum_to_zero():
+    rng = np.random.default_rng(31)
+    W = rng.standard_normal((20, 32)) * 0.02
+    X = rng.standard_normal((15, 32))
+    L = rng.standard_normal((4, 8, 8))
+    dL = O.step(W, X, L, 0.5, 5, 2, 4)["dL"]
+    assert np.max(np.abs(dL.sum(axis=2))) < 1e-12 * np.max(np.abs(dL)) * 64
+
+
+def test_token_shards_sum_to_the_full_gradient():
+    # loss is a token mean, so per-shard gradients weighted by shard size add up
+    rng = np.random.default_rng(32)
+    W = rng.standard_normal((20, 32)) * 0.02
+    X = rng.standard_normal((30, 32))
+    L = rng.standard_normal((4, 8, 8)) * 0.2
+    full = O.step(W, X, L, 0.5, 5, 2, 4)
+    a = O.step(W, X[:12], L, 0.5, 5, 2, 4)
+    b = O.step(W, X[12:], L, 0.5, 5, 2, 4)
+    assert abs((12 * a["loss"] + 18 * b["loss"]) / 30 - full["loss"]) < 1e-14
+    assert np.allclose((12 * a["dL"] + 18 * b["dL"]) / 30, full["dL"], rtol=1e-10, atol=1e-16)
