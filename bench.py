@@ -1,0 +1,393 @@
+#!/usr/bin/env python
+"""Benchmark of the learnable-channel-permutation forward+backward step.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One "step" is one pass of the whole hot path (Sinkhorn, permutation + N:M
+mask, dense and sparse calibration outputs, cosine loss, backward to the
+logits) over one layer.  The default workload is a LLaMA-7B q_proj-shaped
+layer: W 4096x4096 bf16 with 1% outlier input channels, T = 2048 calibration
+tokens, B = 64, 2:4, tau = 0.5, 5 Sinkhorn iterations (seeded synthetic data).
+
+Multi-GPU (torchrun): every rank runs its own independent layer (distinct
+seed): the work is sharded by layer, with no collective on the data path;
+``value`` is the total number of layer-steps per second over all ranks,
+timed as the maximum over ranks (weak scaling).
+
+Timing: W untimed warm-up steps, then K steps, each timed with CUDA events
+on the launching stream; the L2 cache is flushed (a 256 MiB write) between
+timed steps, outside the events.  Per-kernel durations come from events the
+library records between its stages inside the same timed steps.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "LCP fwd+bwd steps/s per layer @4096x4096 B=64 2:4; % of bf16 TC peak & HBM BW"
+UNIT = "steps/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload(name):
+    from learnable_channel_permutation_b200 import synth
+    if name == "q_proj_4096":
+        return synth.q_proj_4096()
+    if name == "toy_256":
+        return synth.toy_256()
+    raise SystemExit(f"unknown workload {name}")
+
+
+def stage_work(wl, li, splits=1):
+    """Algorithmic work of each stage for one layer: (kind, amount).
+
+    kind "flop" for the tensor-core contractions, "byte" for the HBM-bound
+    stages (compulsory bytes: every input read once, every output written once).
+    """
+    co, ci, T = li.spec.cout, li.spec.cin, li.spec.tokens
+    B, it = wl.block, wl.iters
+    nb = ci // B
+    e = 2 if wl.dtype == "bf16" else 4
+    return {
+        "sinkhorn_fwd": ("byte", nb * B * B * (4 + 4 + 3 * 2) + nb * it * 2 * B * 4),
+        "permute_mask": ("byte", co * ci * (e + e) + co * ci // 8 + 3 * nb * B * B * 2),
+        "calib_gemm": ("flop", 2 * 2 * T * co * ci),
+        "loss": ("byte", T * co * (4 + 4 + e) + T * 16),
+        "bwd_gemm": ("flop", 2 * T * co * ci),
+        "block_bwd": ("byte", co * ci * (e + e) + co * ci // 8 + splits * nb * B * B * 4),
+        "sinkhorn_bwd": ("byte", nb * B * B * (4 + 4 * splits + 4) + nb * it * 2 * B * 4),
+    }
+
+
+def src_hash(files):
+    h = hashlib.sha256()
+    for f in files:
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples taken during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
+            if self.uuid:
+                cmd.insert(1, f"--id={self.uuid}")
+            self.proc = subprocess.Popen(cmd, stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in rows for k in range(4) if r[5 + k].lower() == "active"})
+        # median over samples taken while the GPU was busy (above half of max)
+        busy = [s for s in sm if mx and s > 0.5 * max(mx)] or sm
+        return {"sm_mhz": float(np.median(busy)) if busy else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def cpu_baseline(wl, budget_s=12.0):
+    """Time the CPU oracle (as it stands) on whole steps of the same workload."""
+    from oracle import lcp_oracle as O
+    from learnable_channel_permutation_b200 import synth
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        cores = os.cpu_count()
+    li = synth.make_inputs(wl)[0]
+    n, t0 = 0, time.perf_counter()
+    while True:
+        O.step(li.W, li.X, li.L, wl.tau, wl.iters, wl.n, wl.m)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or n >= 20:
+            break
+    return {"value": n / el, "unit": UNIT, "cores": int(cores), "kind": "oracle",
+            "sample": f"{n} whole fwd+bwd steps of the {wl.name} layer (float64 numpy oracle, "
+                      f"BLAS threads = {cores}), {el:.1f} s"}
+
+
+def reference_arm(args, rank, world):
+    """The oracle timed on the host cores (only rank 0 works under torchrun)."""
+    from oracle import lcp_oracle as O
+    from learnable_channel_permutation_b200 import synth
+    if rank != 0:
+        return 0
+    wl = workload(args.workload)
+    li = synth.make_inputs(wl)[0]
+    co = li.spec.cout
+    rows = max(8, co // 8)     # bounded sample: the first C_out/8 output rows
+    W = li.W[:rows]
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        cores = os.cpu_count()
+    for _ in range(max(args.warmup, 0)):
+        O.step(W, li.X, li.L, wl.tau, wl.iters, wl.n, wl.m)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        O.step(W, li.X, li.L, wl.tau, wl.iters, wl.n, wl.m)
+    el = time.perf_counter() - t0
+    # every large term of the step is linear in C_out: scale the sample to a full layer
+    value = args.steps / el * (rows / co)
+    sample = (f"each step: the float64 oracle on the first {rows} of {co} output rows of the {wl.name} "
+              f"layer (T={li.spec.tokens}), scaled by {rows}/{co}; BLAS threads = {cores}")
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 / value, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)", "impl": "reference",
+            "config": {"workload": wl.name, "cout": co, "cin": li.spec.cin, "tokens": li.spec.tokens,
+                       "block": wl.block, "nm": f"{wl.n}:{wl.m}", "tau": wl.tau, "iters": wl.iters},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": int(cores), "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="q_proj_4096")
+    ap.add_argument("--simt", action="store_true", help="CUDA-core kernels for every contraction")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        return reference_arm(args, rank, world)
+
+    import torch
+    import torch.distributed as dist
+    from learnable_channel_permutation_b200 import binding as b
+    from learnable_channel_permutation_b200 import synth
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
+
+    wl = workload(args.workload)
+    wl.seed = rank
+    li = synth.make_inputs(wl)[0]
+    tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    W = torch.from_numpy(li.W).to(dev).to(tdt)
+    X = torch.from_numpy(li.X).to(dev).to(tdt)
+    L = torch.from_numpy(li.L).to(dev)
+    layer = b.alloc_outputs(W, X, L)
+    flags = b.FLAG_SIMT if args.simt else 0
+    step = b.Step([layer], wl.block, wl.n, wl.m, wl.iters, wl.tau, flags=flags)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    for _ in range(args.warmup):
+        step.run()
+    torch.cuda.synchronize()
+
+    K = args.steps
+    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    stages = [[torch.cuda.Event(enable_timing=True) for _ in range(b.TIMED_EVENTS)] for _ in range(K)]
+    for row in stages:            # materialise the events before handing them to the library
+        for e in row:
+            e.record()
+    props = torch.cuda.get_device_properties(dev)
+    uuid = getattr(props, "uuid", None)
+    uuid = f"GPU-{uuid}" if uuid and not str(uuid).startswith("GPU-") else (str(uuid) if uuid else None)
+    sampler = ClockSampler(uuid if world == 1 else None)
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.2)
+    for k in range(K):
+        flush.zero_()
+        ev0[k].record(stream)
+        step.run_timed(stages[k])
+        ev1[k].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+
+    total_ms = sum(ev0[k].elapsed_time(ev1[k]) for k in range(K))
+    stage_ms = {}
+    for s, name in enumerate(b.STAGES):
+        stage_ms[name] = sum(stages[k][s].elapsed_time(stages[k][s + 1]) for k in range(K)) / K
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    max_ms = float(t.item())
+    value = world * K / (max_ms / 1e3)
+
+    # end to end through the public API: pinned host inputs in, loss and dL out, every step
+    e2e = None
+    if not args.no_e2e:
+        hW = torch.from_numpy(li.W).to(tdt).pin_memory()
+        hX = torch.from_numpy(li.X).to(tdt).pin_memory()
+        hL = torch.from_numpy(li.L).pin_memory()
+        hloss = torch.empty(4, dtype=torch.float32).pin_memory()
+        hdL = torch.empty_like(hL).pin_memory()
+        Ke = max(3, min(K, 20))
+        a0 = [torch.cuda.Event(enable_timing=True) for _ in range(Ke)]
+        a1 = [torch.cuda.Event(enable_timing=True) for _ in range(Ke)]
+        for k in range(Ke + 2):
+            kk = k - 2
+            if kk >= 0:
+                a0[kk].record(stream)
+            layer["W"].copy_(hW, non_blocking=True)
+            layer["X"].copy_(hX, non_blocking=True)
+            layer["L"].copy_(hL, non_blocking=True)
+            step.run()
+            hloss.copy_(layer["loss"], non_blocking=True)
+            hdL.copy_(layer["dL"], non_blocking=True)
+            if kk >= 0:
+                a1[kk].record(stream)
+            stream.synchronize()
+        e_ms = sum(a0[k].elapsed_time(a1[k]) for k in range(Ke))
+        te = torch.tensor([e_ms / Ke], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        h2d = hW.numel() * hW.element_size() + hX.numel() * hX.element_size() + hL.numel() * 4
+        d2h = 4 * 4 + hdL.numel() * 4
+        e2e = {"value": world / (float(te.item()) / 1e3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h)}
+
+    if world > 1:
+        dist.barrier()
+    if rank != 0:
+        dist.destroy_process_group()
+        return 0
+
+    pk, pk_src = peaks()
+    work = stage_work(wl, li)
+    dom = max(stage_ms, key=lambda s: stage_ms[s])
+    kind, amount = work[dom]
+    dur_s = stage_ms[dom] / 1e3
+    if kind == "flop":
+        achieved = amount / dur_s / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / pk["bf16_tflops"]}
+    else:
+        achieved = amount / dur_s / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / pk["hbm_gbs"]}
+    roof.update({"kernel": dom, "peak_source": f"{pk_src} ({'bf16 burst' if kind == 'flop' else 'copy'})",
+                 "traffic": traffic_for(dom, args.simt), "algorithmic": amount,
+                 "algorithmic_unit": "FLOP" if kind == "flop" else "bytes"})
+    per_stage = {}
+    for s in b.STAGES:
+        kd, am = work[s]
+        ms = stage_ms[s]
+        if kd == "flop":
+            per_stage[s] = {"ms": ms, "TFLOP/s": am / (ms / 1e3) / 1e12,
+                            "frac": am / (ms / 1e3) / 1e12 / pk["bf16_tflops"]}
+        else:
+            per_stage[s] = {"ms": ms, "GB/s": am / (ms / 1e3) / 1e9, "frac": am / (ms / 1e3) / 1e9 / pk["hbm_gbs"]}
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+            "ms_per_step": max_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if wl.dtype == "bf16" else "f32", "data": "synthetic (seeded)",
+            "config": {"workload": wl.name, "cout": li.spec.cout, "cin": li.spec.cin, "tokens": li.spec.tokens,
+                       "block": wl.block, "nm": f"{wl.n}:{wl.m}", "tau": wl.tau, "iters": wl.iters,
+                       "parallelism": f"layer-sharded x{world}" if world > 1 else "single GPU",
+                       "l2": "flushed between timed steps (256 MiB write)",
+                       "path": "simt" if args.simt else "tcgen05"},
+            "roofline": roof, "stages": per_stage, "clocks": clocks, "e2e": e2e,
+            "gpu_launches": step.launches * K}
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl)
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def traffic_for(kernel, simt):
+    """DRAM bytes per launch from the committed ncu summary, if it matches the current source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if simt or not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    ent = d.get(kernel)
+    if not ent:
+        return None
+    try:
+        if ent.get("src_hash") != src_hash(ent["sources"]):
+            return None
+    except OSError:
+        return None
+    return ent.get("bytes_per_launch")
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,173 @@
+/*
+ * lcp.h -- C ABI of the B200 (sm_100a) learnable-channel-permutation hot path.
+ *
+ * The method: PermLLM, "Learnable Channel Permutation for N:M Sparse Large
+ * Language Models" (summary page of arXiv 2510.10136), section "Method".
+ * For one linear layer W (C_out x C_in) with calibration activations X
+ * (the pages' C_in x T matrix, stored here token-major as [T, C_in]):
+ *
+ *   P_b   = S_L(L_b / tau)                 block-wise log-domain Sinkhorn
+ *   W'    = W * blockdiag(P_1..P_nb)       block-wise permutation
+ *   M     = N:M magnitude mask of |W'|     (groups of M consecutive columns)
+ *   y_s   = (M (.) W') (P_B^T X),  y_d = W X
+ *   loss  = mean over tokens of 1 - cos(y_d, y_s)
+ *   dL    = d loss / d L                   (mask held constant: straight-through)
+ *
+ * Conventions for every entry point:
+ *  - Every pointer is a DEVICE pointer owned by the caller, unless stated.
+ *    The library never allocates, frees or synchronises; it enqueues kernels
+ *    on `stream` and returns.  Results are ready when the stream is.
+ *  - Arguments are validated on the host before any launch.  On error nothing
+ *    is enqueued and a status other than LCP_OK is returned; lcp_last_error()
+ *    then holds a message for the calling thread.
+ *  - A launch failure is reported as LCP_ERR_CUDA (message kept likewise).
+ *  - Matrices are row-major and densely packed:
+ *      W  [C_out, C_in]    X  [T, C_in]      (dtype of the call: f32 or bf16)
+ *      L, P, dL  [C_in/B, B, B] float32; P_b[i][j] moves source channel bB+i
+ *                to permuted slot bB+j; row sums run over j.
+ *      mask bits [C_out, C_in/32] uint32: bit (j % 32) of word j/32 of row o
+ *                is set when W'[o][j] is kept.
+ *      Yd, Ys, G [T, C_out] (token-major outputs).
+ *  - Shapes: B in {32, 64, 128, 256}; C_in % B == 0 and C_in % 32 == 0;
+ *    M in {4, 8} and 1 <= N <= M (N == M prunes nothing); B % M == 0;
+ *    C_out >= 8 and C_out % 8 == 0; T >= 1 (any value, ragged tails allowed);
+ *    1 <= iters <= 1000; tau > 0 and finite.
+ *  - The device must be compute capability 10.0 (B200); otherwise LCP_ERR_ARCH.
+ */
+#ifndef LCP_H
+#define LCP_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define LCP_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define LCP_API __attribute__((visibility("default")))
+#else
+#define LCP_API
+#endif
+
+typedef enum {
+  LCP_OK = 0,
+  LCP_ERR_NULL = 1,       /* a required pointer is NULL                         */
+  LCP_ERR_SHAPE = 2,      /* a size violates the shape rules above              */
+  LCP_ERR_DTYPE = 3,      /* unknown dtype                                      */
+  LCP_ERR_WORKSPACE = 4,  /* workspace too small or misaligned (256 B)          */
+  LCP_ERR_ARCH = 5,       /* current device is not compute capability 10.0      */
+  LCP_ERR_CUDA = 6,       /* a CUDA call or kernel launch failed                */
+  LCP_ERR_ARG = 7         /* any other invalid argument (tau, iters, flags ...) */
+} lcp_status;
+
+typedef enum { LCP_F32 = 0, LCP_BF16 = 1 } lcp_dtype;
+
+/* lcp_hparams.flags */
+#define LCP_FLAG_WRITE_WPRIME 0x1u  /* also write W' (float32, [C_out, C_in]) to layer.Wp */
+#define LCP_FLAG_SIMT         0x2u  /* run every contraction on the CUDA-core (SIMT) kernels
+                                       instead of the tensor-core kernels (bf16 only; the
+                                       f32 dtype always uses SIMT kernels)              */
+
+typedef struct {
+  int block;        /* B, the permutation block size                                */
+  int n, m;         /* N:M pattern: keep n of every m consecutive input channels     */
+  int iters;        /* Sinkhorn iterations (one = row then column normalisation)     */
+  float tau;        /* temperature: Z_0 = L / tau                                    */
+  lcp_dtype dtype;  /* element type of W and X (and of the bf16 intermediates)       */
+  unsigned flags;   /* LCP_FLAG_*                                                    */
+} lcp_hparams;
+
+typedef struct {
+  const void* W;    /* in  [C_out, C_in] dtype                                        */
+  const void* X;    /* in  [T, C_in] dtype; may alias another layer's X               */
+  const float* L;   /* in  [C_in/B, B, B] logits                                      */
+  float* P;         /* out [C_in/B, B, B] soft permutation (required)                 */
+  float* dL;        /* out [C_in/B, B, B] d loss / d L (required)                     */
+  float* loss;      /* out one float: the layer's mean cosine loss (required)         */
+  uint32_t* mask;   /* out [C_out, C_in/32] mask bits (optional, NULL = not returned) */
+  float* Wp;        /* out [C_out, C_in] W' (only with LCP_FLAG_WRITE_WPRIME)         */
+  int cout, cin, tokens;
+} lcp_layer;
+
+/* Bytes of workspace lcp_step needs for these layers (the layers run one after
+ * another on the stream, so the workspace is the maximum over layers).
+ * Cites: the whole of the "Method" section (every intermediate of the step). */
+LCP_API lcp_status lcp_workspace_size(const lcp_layer* layers, int nlayers, const lcp_hparams* hp,
+                              size_t* bytes);
+
+/* One forward + backward step for each of `nlayers` independent layers
+ * (each with its own W, L, P, dL and loss; X may be shared).  `ws` is a device
+ * buffer of at least lcp_workspace_size() bytes, 256-byte aligned, owned by the
+ * caller and not used concurrently by another call.  nlayers == 0 is a no-op. */
+LCP_API lcp_status lcp_step(const lcp_layer* layers, int nlayers, const lcp_hparams* hp, void* ws,
+                    size_t ws_bytes, cudaStream_t stream);
+
+/* As lcp_step, and records events[k] (caller-created cudaEvent_t) on `stream`
+ * at the stage boundaries of the FIRST layer: 0 before the Sinkhorn forward,
+ * then after each stage (Sinkhorn fwd, permute+mask, calibration GEMM, loss,
+ * backward GEMM, block backward, Sinkhorn bwd).  n_events must be 0 or
+ * LCP_TIMED_EVENTS.  Used to time each kernel inside a real step. */
+#define LCP_TIMED_EVENTS 8
+LCP_API lcp_status lcp_step_timed(const lcp_layer* layers, int nlayers, const lcp_hparams* hp, void* ws,
+                          size_t ws_bytes, cudaStream_t stream, cudaEvent_t* events, int n_events);
+
+/* Number of kernel launches lcp_step enqueues for these layers. */
+LCP_API lcp_status lcp_step_launches(const lcp_layer* layers, int nlayers, const lcp_hparams* hp,
+                             int* launches);
+
+/* Block-wise log-domain Sinkhorn ("Method", 1: S_0 = exp, S_i = T_c(T_r(S_{i-1})),
+ * P = S_L(L / tau); the blog page's section 2.2 fixes rows before columns).
+ * L, P: [nblocks, B, B].  ckpt (optional, may be NULL): float32
+ * [nblocks, iters, 2, B]; entry [b][k][0][i] is the row log-normaliser R_i and
+ * [b][k][1][j] the column log-normaliser C_j after iteration k+1, so that the
+ * iterate is Z = L/tau - R_i - C_j.  lcp_sinkhorn_bwd needs it. */
+LCP_API lcp_status lcp_sinkhorn_fwd(const float* L, float* P, float* ckpt, int nblocks, int B, float tau,
+                            int iters, cudaStream_t stream);
+
+/* Reverse pass of lcp_sinkhorn_fwd: dL = d loss / d L given d loss / d P.
+ * dP holds dP_splits partial gradients [dP_splits, nblocks, B, B] that are
+ * summed in index order (deterministic).  ckpt from lcp_sinkhorn_fwd with the
+ * same L, tau and iters. */
+LCP_API lcp_status lcp_sinkhorn_bwd(const float* L, const float* ckpt, const float* dP, int dP_splits,
+                            float* dL, int nblocks, int B, float tau, int iters,
+                            cudaStream_t stream);
+
+/* W' = W * blockdiag(P) ("Method", 3: W_hat_B = W P_B).  W [cout, cin] in
+ * `dtype`, P [cin/B, B, B], Wp [cout, cin] float32. */
+LCP_API lcp_status lcp_permute_weight(const void* W, const float* P, float* Wp, int cout, int cin, int B,
+                              lcp_dtype dtype, cudaStream_t stream);
+
+/* N:M magnitude mask (blog page section 2.1; "integration with existing
+ * pruning methods": the best N of each group of M consecutive columns).
+ * Keeps the n largest |Wp| of every m consecutive columns of each row; equal
+ * magnitudes keep the lower column (+0 and -0 are equal).  Wp [rows, cols] in
+ * `dtype`, compared in that precision; mask_bits [rows, cols/32].
+ * cols % 32 == 0, m in {4, 8}, 1 <= n <= m.  NaN inputs give an unspecified mask. */
+LCP_API lcp_status nm_mask(const void* Wp, uint32_t* mask_bits, int rows, int cols, int n, int m,
+                   lcp_dtype dtype, cudaStream_t stream);
+
+/* Token-averaged cosine loss ("optimization objective": 1 - y.y~ / (|y||y~|),
+ * denominator clamped at 1e-8).  Yd, Ys [tokens, cout] float32; loss: one
+ * float; stats: caller-provided scratch of 4*tokens floats that receives, per
+ * token, <y_d,y_s>, |y_d|^2, |y_s|^2 and cos (lcp_loss_bwd reads it). */
+LCP_API lcp_status lcp_loss_fwd(const float* Yd, const float* Ys, float* loss, float* stats, int cout,
+                        int tokens, cudaStream_t stream);
+
+/* G = d loss / d Ys for the loss above, written in `dtype` ([tokens, cout]);
+ * stats from lcp_loss_fwd on the same Yd, Ys. */
+LCP_API lcp_status lcp_loss_bwd(const float* Yd, const float* Ys, const float* stats, void* G, int cout,
+                        int tokens, lcp_dtype dtype, cudaStream_t stream);
+
+LCP_API const char* lcp_status_string(lcp_status s);
+/* Message of the last failed call made by this thread ("" if none). */
+LCP_API const char* lcp_last_error(void);
+LCP_API int lcp_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LCP_H */

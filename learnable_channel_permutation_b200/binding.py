@@ -1,0 +1,229 @@
+"""Python binding of liblcp (ctypes): argument marshalling only.
+
+Every operation runs in the CUDA library ``csrc/liblcp.so``; this module turns
+torch tensors into device pointers and the current torch stream into a
+``cudaStream_t``.  PyTorch is used for device memory and streams only.  If the
+library is missing, the first call raises: there is no fallback.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, List, Optional, Sequence
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "csrc", "liblcp.so")
+
+F32, BF16 = 0, 1
+FLAG_WRITE_WPRIME = 0x1
+FLAG_SIMT = 0x2
+TIMED_EVENTS = 8
+STAGES = ("sinkhorn_fwd", "permute_mask", "calib_gemm", "loss", "bwd_gemm", "block_bwd", "sinkhorn_bwd")
+
+_c_void_p, _c_int, _c_float = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+
+
+class LcpLayer(ctypes.Structure):
+    _fields_ = [("W", _c_void_p), ("X", _c_void_p), ("L", _c_void_p), ("P", _c_void_p),
+                ("dL", _c_void_p), ("loss", _c_void_p), ("mask", _c_void_p), ("Wp", _c_void_p),
+                ("cout", _c_int), ("cin", _c_int), ("tokens", _c_int)]
+
+
+class LcpHparams(ctypes.Structure):
+    _fields_ = [("block", _c_int), ("n", _c_int), ("m", _c_int), ("iters", _c_int), ("tau", _c_float),
+                ("dtype", _c_int), ("flags", ctypes.c_uint)]
+
+
+class LcpError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(msg)
+        self.status = status
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load liblcp.so (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing; build it with "
+                           "`python -m learnable_channel_permutation_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P = ctypes.POINTER
+    sig = {
+        "lcp_abi_version": ([], _c_int),
+        "lcp_last_error": ([], ctypes.c_char_p),
+        "lcp_status_string": ([_c_int], ctypes.c_char_p),
+        "lcp_workspace_size": ([P(LcpLayer), _c_int, P(LcpHparams), P(ctypes.c_size_t)], _c_int),
+        "lcp_step_launches": ([P(LcpLayer), _c_int, P(LcpHparams), P(_c_int)], _c_int),
+        "lcp_step": ([P(LcpLayer), _c_int, P(LcpHparams), _c_void_p, ctypes.c_size_t, _c_void_p], _c_int),
+        "lcp_step_timed": ([P(LcpLayer), _c_int, P(LcpHparams), _c_void_p, ctypes.c_size_t, _c_void_p,
+                            P(_c_void_p), _c_int], _c_int),
+        "lcp_sinkhorn_fwd": ([_c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_float, _c_int, _c_void_p], _c_int),
+        "lcp_sinkhorn_bwd": ([_c_void_p, _c_void_p, _c_void_p, _c_int, _c_void_p, _c_int, _c_int, _c_float,
+                              _c_int, _c_void_p], _c_int),
+        "lcp_permute_weight": ([_c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_int, _c_void_p], _c_int),
+        "nm_mask": ([_c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_int, _c_int, _c_void_p], _c_int),
+        "lcp_loss_fwd": ([_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_void_p], _c_int),
+        "lcp_loss_bwd": ([_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_void_p], _c_int),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(L, name)
+        fn.argtypes = args
+        fn.restype = res
+    _lib = L
+    return L
+
+
+def check(status: int) -> None:
+    if status != 0:
+        L = lib()
+        raise LcpError(status, f"{L.lcp_status_string(status).decode()} -- {L.lcp_last_error().decode()}")
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return F32
+    if t.dtype == torch.bfloat16:
+        return BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _ptr(t: Optional[torch.Tensor], dtype=None, name: str = "") -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name}: expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: expected a contiguous tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    return t.data_ptr()
+
+
+def _stream(stream: Optional[torch.cuda.Stream]) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def hparams(block: int, n: int, m: int, iters: int, tau: float, dtype: int, flags: int = 0) -> LcpHparams:
+    return LcpHparams(block, n, m, iters, float(tau), dtype, flags)
+
+
+def make_layer(d: Dict[str, torch.Tensor], wdtype) -> LcpLayer:
+    W, X, Lg = d["W"], d["X"], d["L"]
+    cout, cin = W.shape
+    tokens = X.shape[0]
+    if X.shape[1] != cin:
+        raise ValueError("X must be [T, C_in]")
+    return LcpLayer(_ptr(W, wdtype, "W"), _ptr(X, wdtype, "X"), _ptr(Lg, torch.float32, "L"),
+                    _ptr(d["P"], torch.float32, "P"), _ptr(d["dL"], torch.float32, "dL"),
+                    _ptr(d["loss"], torch.float32, "loss"), _ptr(d.get("mask"), torch.int32, "mask"),
+                    _ptr(d.get("Wp"), torch.float32, "Wp"), cout, cin, tokens)
+
+
+class Step:
+    """A prepared lcp_step call: the layer descriptors, hyper-parameters and
+    workspace are marshalled once; ``run()`` enqueues one step on a stream."""
+
+    def __init__(self, layers: Sequence[Dict[str, torch.Tensor]], block: int, n: int, m: int, iters: int,
+                 tau: float, flags: int = 0, workspace: Optional[torch.Tensor] = None):
+        if not layers:
+            raise ValueError("at least one layer")
+        wdtype = layers[0]["W"].dtype
+        self.hp = hparams(block, n, m, iters, tau, _dt(layers[0]["W"]), flags)
+        self.arr = (LcpLayer * len(layers))(*[make_layer(d, wdtype) for d in layers])
+        self.n = len(layers)
+        self.layers = list(layers)  # keep the tensors alive
+        nbytes = ctypes.c_size_t(0)
+        check(lib().lcp_workspace_size(self.arr, self.n, ctypes.byref(self.hp), ctypes.byref(nbytes)))
+        self.ws_bytes = int(nbytes.value)
+        if workspace is None:
+            workspace = torch.empty(max(self.ws_bytes, 256), dtype=torch.uint8, device=layers[0]["W"].device)
+        if workspace.numel() < self.ws_bytes:
+            raise ValueError("workspace too small")
+        self.ws = workspace
+        c = _c_int(0)
+        check(lib().lcp_step_launches(self.arr, self.n, ctypes.byref(self.hp), ctypes.byref(c)))
+        self.launches = int(c.value)
+
+    def run(self, stream: Optional[torch.cuda.Stream] = None) -> None:
+        check(lib().lcp_step(self.arr, self.n, ctypes.byref(self.hp), self.ws.data_ptr(), self.ws.numel(),
+                             _stream(stream)))
+
+    def run_timed(self, events: List[torch.cuda.Event], stream: Optional[torch.cuda.Stream] = None) -> None:
+        if len(events) != TIMED_EVENTS:
+            raise ValueError(f"need {TIMED_EVENTS} events")
+        for e in events:
+            if e.cuda_event == 0:
+                raise ValueError("events must be created (record once) before use")
+        arr = (_c_void_p * TIMED_EVENTS)(*[e.cuda_event for e in events])
+        check(lib().lcp_step_timed(self.arr, self.n, ctypes.byref(self.hp), self.ws.data_ptr(), self.ws.numel(),
+                                   _stream(stream), arr, TIMED_EVENTS))
+
+
+def alloc_outputs(W: torch.Tensor, X: torch.Tensor, L: torch.Tensor, with_mask: bool = True,
+                  with_wp: bool = False) -> Dict[str, torch.Tensor]:
+    dev = W.device
+    cout, cin = W.shape
+    d = dict(W=W, X=X, L=L, P=torch.empty_like(L), dL=torch.empty_like(L),
+             loss=torch.empty(4, dtype=torch.float32, device=dev))
+    if with_mask:
+        d["mask"] = torch.empty(cout, cin // 32, dtype=torch.int32, device=dev)
+    if with_wp:
+        d["Wp"] = torch.empty(cout, cin, dtype=torch.float32, device=dev)
+    return d
+
+
+def step(layers: Sequence[Dict[str, torch.Tensor]], block: int, n: int, m: int, iters: int, tau: float,
+         flags: int = 0) -> Step:
+    """Run one forward+backward step on the current stream (allocates a workspace)."""
+    s = Step(layers, block, n, m, iters, tau, flags)
+    s.run()
+    return s
+
+
+def sinkhorn_fwd(L: torch.Tensor, P: torch.Tensor, ckpt: Optional[torch.Tensor], tau: float, iters: int) -> None:
+    nb, B, _ = L.shape
+    check(lib().lcp_sinkhorn_fwd(_ptr(L, torch.float32, "L"), _ptr(P, torch.float32, "P"),
+                                 _ptr(ckpt, torch.float32, "ckpt"), nb, B, float(tau), iters, _stream(None)))
+
+
+def sinkhorn_bwd(L: torch.Tensor, ckpt: torch.Tensor, dP: torch.Tensor, dL: torch.Tensor, tau: float,
+                 iters: int) -> None:
+    nb, B, _ = L.shape
+    splits = dP.numel() // (nb * B * B)
+    check(lib().lcp_sinkhorn_bwd(_ptr(L, torch.float32, "L"), _ptr(ckpt, torch.float32, "ckpt"),
+                                 _ptr(dP, torch.float32, "dP"), splits, _ptr(dL, torch.float32, "dL"), nb, B,
+                                 float(tau), iters, _stream(None)))
+
+
+def permute_weight(W: torch.Tensor, P: torch.Tensor, Wp: torch.Tensor) -> None:
+    cout, cin = W.shape
+    check(lib().lcp_permute_weight(_ptr(W, None, "W"), _ptr(P, torch.float32, "P"), _ptr(Wp, torch.float32, "Wp"),
+                                   cout, cin, P.shape[1], _dt(W), _stream(None)))
+
+
+def nm_mask(Wp: torch.Tensor, bits: torch.Tensor, n: int, m: int) -> None:
+    rows, cols = Wp.shape
+    check(lib().nm_mask(_ptr(Wp, None, "Wp"), _ptr(bits, torch.int32, "bits"), rows, cols, n, m, _dt(Wp),
+                        _stream(None)))
+
+
+def loss_fwd(Yd: torch.Tensor, Ys: torch.Tensor, loss: torch.Tensor, stats: torch.Tensor) -> None:
+    T, cout = Yd.shape
+    check(lib().lcp_loss_fwd(_ptr(Yd, torch.float32, "Yd"), _ptr(Ys, torch.float32, "Ys"),
+                             _ptr(loss, torch.float32, "loss"), _ptr(stats, torch.float32, "stats"), cout, T,
+                             _stream(None)))
+
+
+def loss_bwd(Yd: torch.Tensor, Ys: torch.Tensor, stats: torch.Tensor, G: torch.Tensor) -> None:
+    T, cout = Yd.shape
+    check(lib().lcp_loss_bwd(_ptr(Yd, torch.float32, "Yd"), _ptr(Ys, torch.float32, "Ys"),
+                             _ptr(stats, torch.float32, "stats"), _ptr(G, None, "G"), cout, T, _dt(G),
+                             _stream(None)))

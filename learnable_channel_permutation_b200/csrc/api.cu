@@ -1,0 +1,445 @@
+// C ABI of liblcp: argument validation, workspace planning and the ordering of
+// the kernels of one learnable-channel-permutation step (see include/lcp.h).
+//
+// Step order (PermLLM summary, "Method"):
+//   Sinkhorn (Method 1)  ->  W' = W P_B (Method 3)  ->  N:M mask of |W'|
+//   (integration with pruning methods)  ->  y_d = W X, y_s = (M.W')(P_B^T X)
+//   evaluated as (M.W' P_B^T) X  ->  token-mean cosine loss (objective)
+//   ->  reverse pass to the logits with the mask held constant.
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "lcp_internal.cuh"
+
+namespace lcp {
+
+static thread_local char g_msg[512] = "";
+
+void set_error(const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+  va_end(ap);
+}
+
+lcp_status fail(lcp_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+lcp_status check_launch(const char* what) {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(LCP_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return LCP_OK;
+}
+
+namespace {
+
+#define LCP_TRY(expr)                     \
+  do {                                    \
+    const lcp_status s_ = (expr);         \
+    if (s_ != LCP_OK) return s_;          \
+  } while (0)
+
+constexpr int kMaxDim = 1 << 24;
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+lcp_status check_arch() {
+  static int cached[64];  // 0 unknown, 1 ok, 2 wrong
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(LCP_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  }
+  std::lock_guard<std::mutex> lk(mu);
+  if (dev >= 0 && dev < 64 && cached[dev]) {
+    if (cached[dev] == 1) return LCP_OK;
+    return fail(LCP_ERR_ARCH, "device %d is not compute capability 10.0 (B200)", dev);
+  }
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return fail(LCP_ERR_CUDA, "cannot query the compute capability of device %d", dev);
+  }
+  const bool ok = (major == 10 && minor == 0);
+  if (dev >= 0 && dev < 64) cached[dev] = ok ? 1 : 2;
+  if (!ok) return fail(LCP_ERR_ARCH, "device %d is sm_%d%d, this library is built for sm_100a", dev, major, minor);
+  return LCP_OK;
+}
+
+lcp_status check_hparams(const lcp_hparams* hp) {
+  if (!hp) return fail(LCP_ERR_NULL, "hparams is NULL");
+  if (hp->dtype != LCP_F32 && hp->dtype != LCP_BF16)
+    return fail(LCP_ERR_DTYPE, "unknown dtype %d", (int)hp->dtype);
+  const int B = hp->block;
+  if (B != 32 && B != 64 && B != 128 && B != 256)
+    return fail(LCP_ERR_SHAPE, "block size %d is not one of 32, 64, 128, 256", B);
+  if (hp->m != 4 && hp->m != 8) return fail(LCP_ERR_SHAPE, "m = %d is not 4 or 8", hp->m);
+  if (hp->n < 1 || hp->n > hp->m) return fail(LCP_ERR_SHAPE, "n = %d is not in [1, m]", hp->n);
+  if (B % hp->m) return fail(LCP_ERR_SHAPE, "block %d is not a multiple of m = %d", B, hp->m);
+  if (hp->iters < 1 || hp->iters > 1000)
+    return fail(LCP_ERR_ARG, "iters = %d is not in [1, 1000]", hp->iters);
+  if (!(hp->tau > 0.f) || !std::isfinite(hp->tau))
+    return fail(LCP_ERR_ARG, "tau must be positive and finite");
+  if (hp->flags & ~(LCP_FLAG_WRITE_WPRIME | LCP_FLAG_SIMT))
+    return fail(LCP_ERR_ARG, "unknown flags 0x%x", hp->flags);
+  return LCP_OK;
+}
+
+lcp_status check_layer(const lcp_layer& l, const lcp_hparams& hp, int idx) {
+  if (!l.W || !l.X || !l.L || !l.P || !l.dL || !l.loss)
+    return fail(LCP_ERR_NULL, "layer %d: W, X, L, P, dL and loss are required", idx);
+  if ((hp.flags & LCP_FLAG_WRITE_WPRIME) && !l.Wp)
+    return fail(LCP_ERR_NULL, "layer %d: LCP_FLAG_WRITE_WPRIME needs layer.Wp", idx);
+  if (l.cout < 8 || l.cout % 8 || l.cout > kMaxDim)
+    return fail(LCP_ERR_SHAPE, "layer %d: C_out = %d must be a positive multiple of 8", idx, l.cout);
+  if (l.cin < hp.block || l.cin % hp.block || l.cin % 32 || l.cin > kMaxDim)
+    return fail(LCP_ERR_SHAPE, "layer %d: C_in = %d must be a positive multiple of B = %d and of 32",
+                idx, l.cin, hp.block);
+  if (l.tokens < 1 || l.tokens > kMaxDim)
+    return fail(LCP_ERR_SHAPE, "layer %d: T = %d must be >= 1", idx, l.tokens);
+  const void* ptrs[] = {l.W, l.X, l.L, l.P, l.dL, l.mask, l.Wp};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(LCP_ERR_ARG, "layer %d: every pointer must be 16-byte aligned", idx);
+  return LCP_OK;
+}
+
+bool use_tc(const lcp_hparams& hp) {
+  return hp.dtype == LCP_BF16 && !(hp.flags & LCP_FLAG_SIMT) && tc_available();
+}
+
+size_t esize(lcp_dtype d) { return d == LCP_F32 ? 4 : 2; }
+
+struct Plan {
+  size_t ckpt, img0, img1, img2, mask, wp, amask, at, yd, ys, stats, g, dat, da, dp;
+  size_t total;
+  int splits;
+};
+
+Plan make_plan(const lcp_layer& l, const lcp_hparams& hp) {
+  const bool tc = use_tc(hp);
+  const size_t B = hp.block, nb = l.cin / hp.block;
+  const size_t oc = l.cout, ic = l.cin, T = l.tokens;
+  const size_t es = esize(hp.dtype);
+  Plan p{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off += (bytes + 1023) & ~(size_t)1023;
+    return at;
+  };
+  p.splits = tc ? block_bwd_tc_splits(l.cout, l.cin, hp.block) : 1;
+  p.ckpt = take(nb * hp.iters * 2 * B * 4);
+  p.img0 = take(tc ? nb * B * B * 2 : 0);
+  p.img1 = take(tc ? nb * B * B * 2 : 0);
+  p.img2 = take(tc ? nb * B * B * 2 : 0);
+  p.mask = take(oc * ic / 8);
+  p.wp = take(tc ? 0 : oc * ic * 4);
+  p.amask = take(tc ? 0 : oc * ic * 4);
+  p.at = take(oc * ic * es);
+  p.yd = take(T * oc * 4);
+  p.ys = take(T * oc * 4);
+  p.stats = take(T * 16);
+  p.g = take(T * oc * es);
+  p.dat = take(oc * ic * (tc ? 2 : 4));
+  p.da = take(tc ? 0 : oc * ic * 4);
+  p.dp = take((size_t)p.splits * nb * B * B * 4);
+  p.total = off;
+  return p;
+}
+
+lcp_status validate_all(const lcp_layer* layers, int nlayers, const lcp_hparams* hp) {
+  LCP_TRY(check_hparams(hp));
+  if (nlayers < 0) return fail(LCP_ERR_ARG, "nlayers = %d is negative", nlayers);
+  if (nlayers > 0 && !layers) return fail(LCP_ERR_NULL, "layers is NULL");
+  for (int i = 0; i < nlayers; ++i) LCP_TRY(check_layer(layers[i], *hp, i));
+  return LCP_OK;
+}
+
+template <typename T> T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+lcp_status record(cudaEvent_t* ev, int k, cudaStream_t st) {
+  if (!ev) return LCP_OK;
+  const cudaError_t e = cudaEventRecord(ev[k], st);
+  if (e != cudaSuccess) return fail(LCP_ERR_CUDA, "cudaEventRecord: %s", cudaGetErrorString(e));
+  return LCP_OK;
+}
+
+// ---- one layer, CUDA-core path (float32, or bf16 with LCP_FLAG_SIMT) -------
+lcp_status layer_simt(const lcp_layer& l, const lcp_hparams& hp, const Plan& p, void* ws,
+                      cudaStream_t st, cudaEvent_t* ev) {
+  const int B = hp.block, nb = l.cin / B;
+  const lcp_dtype dt = hp.dtype;
+  float* ckpt = at<float>(ws, p.ckpt);
+  uint32_t* mask = l.mask ? l.mask : at<uint32_t>(ws, p.mask);
+  float* Wp = (hp.flags & LCP_FLAG_WRITE_WPRIME) ? l.Wp : at<float>(ws, p.wp);
+  float* Am = at<float>(ws, p.amask);
+  void* At = at<void>(ws, p.at);
+  float* Yd = at<float>(ws, p.yd);
+  float* Ys = at<float>(ws, p.ys);
+  float* stats = at<float>(ws, p.stats);
+  void* G = at<void>(ws, p.g);
+  float* dAt = at<float>(ws, p.dat);
+  float* dA = at<float>(ws, p.da);
+  float* dP = at<float>(ws, p.dp);
+  const long long ic = l.cin, oc = l.cout, BB = (long long)B * B;
+
+  LCP_TRY(record(ev, 0, st));
+  LCP_TRY(launch_sinkhorn_fwd(l.L, l.P, ckpt, nullptr, nullptr, nullptr, nb, B, hp.tau, hp.iters, st));
+  LCP_TRY(record(ev, 1, st));
+  // W'_b = W_b P_b
+  LCP_TRY(launch_simt_gemm({l.cout, B, B, nb, l.W, B, ic, 1, l.P, BB, B, 1, Wp, B, ic, 1, 1.f, 0.f},
+                           dt, LCP_F32, LCP_F32, st));
+  LCP_TRY(launch_nm_mask(Wp, mask, l.cout, l.cin, hp.n, hp.m, LCP_F32, st));
+  LCP_TRY(launch_apply_mask(Wp, mask, Am, l.cout, l.cin, st));
+  // At_b = A_b P_b^T
+  LCP_TRY(launch_simt_gemm({l.cout, B, B, nb, Am, B, ic, 1, l.P, BB, 1, B, At, B, ic, 1, 1.f, 0.f},
+                           LCP_F32, LCP_F32, dt, st));
+  LCP_TRY(record(ev, 2, st));
+  // Yd = X W^T, Ys = X At^T   ([T, C_out])
+  LCP_TRY(launch_simt_gemm({l.tokens, l.cout, l.cin, 1, l.X, 0, ic, 1, l.W, 0, 1, ic, Yd, 0, oc, 1, 1.f, 0.f},
+                           dt, dt, LCP_F32, st));
+  LCP_TRY(launch_simt_gemm({l.tokens, l.cout, l.cin, 1, l.X, 0, ic, 1, At, 0, 1, ic, Ys, 0, oc, 1, 1.f, 0.f},
+                           dt, dt, LCP_F32, st));
+  LCP_TRY(record(ev, 3, st));
+  LCP_TRY(launch_loss_token(Yd, Ys, stats, G, dt, l.cout, l.tokens, st));
+  LCP_TRY(launch_loss_reduce(stats, l.loss, l.tokens, st));
+  LCP_TRY(record(ev, 4, st));
+  // dAt = G^T X   ([C_out, C_in], K = T)
+  LCP_TRY(launch_simt_gemm({l.cout, l.cin, l.tokens, 1, G, 0, 1, oc, l.X, 0, ic, 1, dAt, 0, ic, 1, 1.f, 0.f},
+                           dt, dt, LCP_F32, st));
+  LCP_TRY(record(ev, 5, st));
+  // dA_b = dAt_b P_b ; dW' = M . dA ; dP_b = dAt_b^T A_b + W_b^T dW'_b
+  LCP_TRY(launch_simt_gemm({l.cout, B, B, nb, dAt, B, ic, 1, l.P, BB, B, 1, dA, B, ic, 1, 1.f, 0.f},
+                           LCP_F32, LCP_F32, LCP_F32, st));
+  LCP_TRY(launch_apply_mask(dA, mask, dA, l.cout, l.cin, st));
+  LCP_TRY(launch_simt_gemm({B, B, l.cout, nb, dAt, B, 1, ic, Am, B, ic, 1, dP, BB, B, 1, 1.f, 0.f},
+                           LCP_F32, LCP_F32, LCP_F32, st));
+  LCP_TRY(launch_simt_gemm({B, B, l.cout, nb, l.W, B, 1, ic, dA, B, ic, 1, dP, BB, B, 1, 1.f, 1.f},
+                           dt, LCP_F32, LCP_F32, st));
+  LCP_TRY(record(ev, 6, st));
+  LCP_TRY(launch_sinkhorn_bwd(l.L, ckpt, dP, 1, l.dL, nb, B, hp.tau, hp.iters, st));
+  LCP_TRY(record(ev, 7, st));
+  return LCP_OK;
+}
+
+constexpr int kSimtLaunches = 15;
+constexpr int kTcLaunches = 8;
+
+// ---- one layer, tensor-core path (bf16 operands, float32 accumulation) -----
+lcp_status layer_tc(const lcp_layer& l, const lcp_hparams& hp, const Plan& p, void* ws,
+                    cudaStream_t st, cudaEvent_t* ev) {
+  const int B = hp.block, nb = l.cin / B;
+  float* ckpt = at<float>(ws, p.ckpt);
+  auto* pt_hi = at<__nv_bfloat16>(ws, p.img0);
+  auto* pt_lo = at<__nv_bfloat16>(ws, p.img1);
+  auto* p_hi = at<__nv_bfloat16>(ws, p.img2);
+  uint32_t* mask = l.mask ? l.mask : at<uint32_t>(ws, p.mask);
+  float* Wp = (hp.flags & LCP_FLAG_WRITE_WPRIME) ? l.Wp : nullptr;
+  auto* At = at<__nv_bfloat16>(ws, p.at);
+  float* Yd = at<float>(ws, p.yd);
+  float* Ys = at<float>(ws, p.ys);
+  float* stats = at<float>(ws, p.stats);
+  auto* G = at<__nv_bfloat16>(ws, p.g);
+  auto* dAt = at<__nv_bfloat16>(ws, p.dat);
+  float* dP = at<float>(ws, p.dp);
+  const auto* W = static_cast<const __nv_bfloat16*>(l.W);
+  const auto* X = static_cast<const __nv_bfloat16*>(l.X);
+
+  LCP_TRY(record(ev, 0, st));
+  LCP_TRY(launch_sinkhorn_fwd(l.L, l.P, ckpt, pt_hi, pt_lo, p_hi, nb, B, hp.tau, hp.iters, st));
+  LCP_TRY(record(ev, 1, st));
+  LCP_TRY(launch_permute_mask_tc(W, pt_hi, pt_lo, p_hi, mask, At, Wp, l.cout, l.cin, B, hp.n, hp.m, st));
+  LCP_TRY(record(ev, 2, st));
+  LCP_TRY(launch_calib_gemm_tc(X, W, At, Yd, Ys, l.tokens, l.cout, l.cin, st));
+  LCP_TRY(record(ev, 3, st));
+  LCP_TRY(launch_loss_token(Yd, Ys, stats, G, LCP_BF16, l.cout, l.tokens, st));
+  LCP_TRY(launch_loss_reduce(stats, l.loss, l.tokens, st));
+  LCP_TRY(record(ev, 4, st));
+  LCP_TRY(launch_bwd_gemm_tc(G, X, dAt, l.tokens, l.cout, l.cin, st));
+  LCP_TRY(record(ev, 5, st));
+  LCP_TRY(launch_block_bwd_tc(W, dAt, mask, pt_hi, pt_lo, dP, p.splits, l.cout, l.cin, B, st));
+  LCP_TRY(record(ev, 6, st));
+  LCP_TRY(launch_sinkhorn_bwd(l.L, ckpt, dP, p.splits, l.dL, nb, B, hp.tau, hp.iters, st));
+  LCP_TRY(record(ev, 7, st));
+  return LCP_OK;
+}
+
+lcp_status step_impl(const lcp_layer* layers, int nlayers, const lcp_hparams* hp, void* ws,
+                     size_t ws_bytes, cudaStream_t st, cudaEvent_t* ev, int nev) {
+  LCP_TRY(validate_all(layers, nlayers, hp));
+  if (nev != 0 && nev != LCP_TIMED_EVENTS)
+    return fail(LCP_ERR_ARG, "n_events must be 0 or %d", LCP_TIMED_EVENTS);
+  if (nev && !ev) return fail(LCP_ERR_NULL, "events is NULL");
+  if (nlayers == 0) return LCP_OK;
+  size_t need = 0;
+  for (int i = 0; i < nlayers; ++i) need = std::max(need, make_plan(layers[i], *hp).total);
+  if (!ws) return fail(LCP_ERR_NULL, "workspace is NULL");
+  if (((uintptr_t)ws & 255u) != 0) return fail(LCP_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  if (ws_bytes < need)
+    return fail(LCP_ERR_WORKSPACE, "workspace has %zu bytes, %zu needed", ws_bytes, need);
+  LCP_TRY(check_arch());
+  cudaGetLastError();  // a stale error from elsewhere must not be blamed on us
+  for (int i = 0; i < nlayers; ++i) {
+    const Plan p = make_plan(layers[i], *hp);
+    cudaEvent_t* e = (i == 0 && nev) ? ev : nullptr;
+    if (use_tc(*hp)) LCP_TRY(layer_tc(layers[i], *hp, p, ws, st, e));
+    else LCP_TRY(layer_simt(layers[i], *hp, p, ws, st, e));
+  }
+  return LCP_OK;
+}
+
+}  // namespace
+}  // namespace lcp
+
+using namespace lcp;
+
+extern "C" {
+
+int lcp_abi_version(void) { return LCP_ABI_VERSION; }
+
+const char* lcp_last_error(void) { return g_msg; }
+
+const char* lcp_status_string(lcp_status s) {
+  switch (s) {
+    case LCP_OK: return "LCP_OK";
+    case LCP_ERR_NULL: return "LCP_ERR_NULL: a required pointer is NULL";
+    case LCP_ERR_SHAPE: return "LCP_ERR_SHAPE: unsupported shape";
+    case LCP_ERR_DTYPE: return "LCP_ERR_DTYPE: unknown dtype";
+    case LCP_ERR_WORKSPACE: return "LCP_ERR_WORKSPACE: workspace too small or misaligned";
+    case LCP_ERR_ARCH: return "LCP_ERR_ARCH: device is not sm_100 (B200)";
+    case LCP_ERR_CUDA: return "LCP_ERR_CUDA: a CUDA call failed";
+    case LCP_ERR_ARG: return "LCP_ERR_ARG: invalid argument";
+  }
+  return "unknown lcp_status";
+}
+
+lcp_status lcp_workspace_size(const lcp_layer* layers, int nlayers, const lcp_hparams* hp,
+                              size_t* bytes) {
+  if (!bytes) return fail(LCP_ERR_NULL, "bytes is NULL");
+  LCP_TRY(validate_all(layers, nlayers, hp));
+  size_t need = 0;
+  for (int i = 0; i < nlayers; ++i) need = std::max(need, make_plan(layers[i], *hp).total);
+  *bytes = need;
+  return LCP_OK;
+}
+
+lcp_status lcp_step_launches(const lcp_layer* layers, int nlayers, const lcp_hparams* hp,
+                             int* launches) {
+  if (!launches) return fail(LCP_ERR_NULL, "launches is NULL");
+  LCP_TRY(validate_all(layers, nlayers, hp));
+  *launches = nlayers * (use_tc(*hp) ? kTcLaunches : kSimtLaunches);
+  return LCP_OK;
+}
+
+lcp_status lcp_step(const lcp_layer* layers, int nlayers, const lcp_hparams* hp, void* ws,
+                    size_t ws_bytes, cudaStream_t stream) {
+  return step_impl(layers, nlayers, hp, ws, ws_bytes, stream, nullptr, 0);
+}
+
+lcp_status lcp_step_timed(const lcp_layer* layers, int nlayers, const lcp_hparams* hp, void* ws,
+                          size_t ws_bytes, cudaStream_t stream, cudaEvent_t* events,
+                          int n_events) {
+  return step_impl(layers, nlayers, hp, ws, ws_bytes, stream, events, n_events);
+}
+
+lcp_status lcp_sinkhorn_fwd(const float* L, float* P, float* ckpt, int nblocks, int B, float tau,
+                            int iters, cudaStream_t stream) {
+  if (!L || !P) return fail(LCP_ERR_NULL, "L and P are required");
+  if (B != 32 && B != 64 && B != 128 && B != 256)
+    return fail(LCP_ERR_SHAPE, "block size %d is not one of 32, 64, 128, 256", B);
+  if (nblocks < 0 || nblocks > kMaxDim) return fail(LCP_ERR_SHAPE, "nblocks = %d", nblocks);
+  if (iters < 1 || iters > 1000) return fail(LCP_ERR_ARG, "iters = %d is not in [1, 1000]", iters);
+  if (!(tau > 0.f) || !std::isfinite(tau)) return fail(LCP_ERR_ARG, "tau must be positive and finite");
+  if (nblocks == 0) return LCP_OK;
+  LCP_TRY(check_arch());
+  cudaGetLastError();
+  return launch_sinkhorn_fwd(L, P, ckpt, nullptr, nullptr, nullptr, nblocks, B, tau, iters, stream);
+}
+
+lcp_status lcp_sinkhorn_bwd(const float* L, const float* ckpt, const float* dP, int dP_splits,
+                            float* dL, int nblocks, int B, float tau, int iters,
+                            cudaStream_t stream) {
+  if (!L || !ckpt || !dP || !dL) return fail(LCP_ERR_NULL, "L, ckpt, dP and dL are required");
+  if (B != 32 && B != 64 && B != 128 && B != 256)
+    return fail(LCP_ERR_SHAPE, "block size %d is not one of 32, 64, 128, 256", B);
+  if (nblocks < 0 || nblocks > kMaxDim) return fail(LCP_ERR_SHAPE, "nblocks = %d", nblocks);
+  if (dP_splits < 1 || dP_splits > 64) return fail(LCP_ERR_ARG, "dP_splits = %d is not in [1, 64]", dP_splits);
+  if (iters < 1 || iters > 1000) return fail(LCP_ERR_ARG, "iters = %d is not in [1, 1000]", iters);
+  if (!(tau > 0.f) || !std::isfinite(tau)) return fail(LCP_ERR_ARG, "tau must be positive and finite");
+  if (nblocks == 0) return LCP_OK;
+  LCP_TRY(check_arch());
+  cudaGetLastError();
+  return launch_sinkhorn_bwd(L, ckpt, dP, dP_splits, dL, nblocks, B, tau, iters, stream);
+}
+
+lcp_status lcp_permute_weight(const void* W, const float* P, float* Wp, int cout, int cin, int B,
+                              lcp_dtype dtype, cudaStream_t stream) {
+  if (!W || !P || !Wp) return fail(LCP_ERR_NULL, "W, P and Wp are required");
+  if (dtype != LCP_F32 && dtype != LCP_BF16) return fail(LCP_ERR_DTYPE, "unknown dtype %d", (int)dtype);
+  if (B != 32 && B != 64 && B != 128 && B != 256)
+    return fail(LCP_ERR_SHAPE, "block size %d is not one of 32, 64, 128, 256", B);
+  if (cout < 0 || cin < 0 || cin % B || cout > kMaxDim || cin > kMaxDim)
+    return fail(LCP_ERR_SHAPE, "C_out = %d, C_in = %d (C_in must be a multiple of B)", cout, cin);
+  if (cout == 0 || cin == 0) return LCP_OK;
+  LCP_TRY(check_arch());
+  cudaGetLastError();
+  const long long ic = cin, BB = (long long)B * B;
+  return launch_simt_gemm({cout, B, B, cin / B, W, B, ic, 1, P, BB, B, 1, Wp, B, ic, 1, 1.f, 0.f},
+                          dtype, LCP_F32, LCP_F32, stream);
+}
+
+lcp_status nm_mask(const void* Wp, uint32_t* mask_bits, int rows, int cols, int n, int m,
+                   lcp_dtype dtype, cudaStream_t stream) {
+  if (!Wp || !mask_bits) return fail(LCP_ERR_NULL, "Wp and mask_bits are required");
+  if (dtype != LCP_F32 && dtype != LCP_BF16) return fail(LCP_ERR_DTYPE, "unknown dtype %d", (int)dtype);
+  if (m != 4 && m != 8) return fail(LCP_ERR_SHAPE, "m = %d is not 4 or 8", m);
+  if (n < 1 || n > m) return fail(LCP_ERR_SHAPE, "n = %d is not in [1, m]", n);
+  if (rows < 0 || cols < 0 || cols % 32 || rows > kMaxDim || cols > kMaxDim)
+    return fail(LCP_ERR_SHAPE, "rows = %d, cols = %d (cols must be a multiple of 32)", rows, cols);
+  if (!aligned16(Wp) || !aligned16(mask_bits)) return fail(LCP_ERR_ARG, "pointers must be 16-byte aligned");
+  if (rows == 0 || cols == 0) return LCP_OK;
+  LCP_TRY(check_arch());
+  cudaGetLastError();
+  return launch_nm_mask(Wp, mask_bits, rows, cols, n, m, dtype, stream);
+}
+
+lcp_status lcp_loss_fwd(const float* Yd, const float* Ys, float* loss, float* stats, int cout,
+                        int tokens, cudaStream_t stream) {
+  if (!Yd || !Ys || !loss || !stats) return fail(LCP_ERR_NULL, "Yd, Ys, loss and stats are required");
+  if (cout < 8 || cout % 8 || cout > kMaxDim) return fail(LCP_ERR_SHAPE, "C_out = %d must be a positive multiple of 8", cout);
+  if (tokens < 1 || tokens > kMaxDim) return fail(LCP_ERR_SHAPE, "T = %d must be >= 1", tokens);
+  if (!aligned16(Yd) || !aligned16(Ys) || !aligned16(stats)) return fail(LCP_ERR_ARG, "pointers must be 16-byte aligned");
+  LCP_TRY(check_arch());
+  cudaGetLastError();
+  LCP_TRY(launch_loss_token(Yd, Ys, stats, nullptr, LCP_F32, cout, tokens, stream));
+  return launch_loss_reduce(stats, loss, tokens, stream);
+}
+
+lcp_status lcp_loss_bwd(const float* Yd, const float* Ys, const float* stats, void* G, int cout,
+                        int tokens, lcp_dtype dtype, cudaStream_t stream) {
+  if (!Yd || !Ys || !stats || !G) return fail(LCP_ERR_NULL, "Yd, Ys, stats and G are required");
+  if (dtype != LCP_F32 && dtype != LCP_BF16) return fail(LCP_ERR_DTYPE, "unknown dtype %d", (int)dtype);
+  if (cout < 8 || cout % 8 || cout > kMaxDim) return fail(LCP_ERR_SHAPE, "C_out = %d must be a positive multiple of 8", cout);
+  if (tokens < 1 || tokens > kMaxDim) return fail(LCP_ERR_SHAPE, "T = %d must be >= 1", tokens);
+  if (!aligned16(Yd) || !aligned16(Ys) || !aligned16(stats) || !aligned16(G))
+    return fail(LCP_ERR_ARG, "pointers must be 16-byte aligned");
+  LCP_TRY(check_arch());
+  cudaGetLastError();
+  return launch_loss_grad(Yd, Ys, stats, G, dtype, cout, tokens, stream);
+}
+
+}  // extern "C"

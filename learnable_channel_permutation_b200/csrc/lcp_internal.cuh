@@ -1,0 +1,86 @@
+// Internal declarations shared by the CUDA translation units of liblcp.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/lcp.h"
+
+namespace lcp {
+
+// ---- error reporting (thread-local message, see lcp_last_error) ----------
+void set_error(const char* fmt, ...);
+lcp_status fail(lcp_status s, const char* fmt, ...);
+// Checks cudaGetLastError() after a launch; returns LCP_ERR_CUDA with `what`.
+lcp_status check_launch(const char* what);
+
+// ---- element conversions -------------------------------------------------
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+template <typename T> __device__ __forceinline__ T from_f32(float v);
+template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) {
+  return __float2bfloat16_rn(v);
+}
+
+// ---- launchers (host side; each returns LCP_OK or LCP_ERR_CUDA) ----------
+
+// Sinkhorn.  img_* are optional bf16 operand images for the tensor-core path:
+//   img_pt_hi[b][j][i] = bf16(P_b[i][j])          (P_b transposed, high part)
+//   img_pt_lo[b][j][i] = bf16(P_b[i][j] - hi)     (P_b transposed, low part)
+//   img_p_hi [b][i][j] = bf16(P_b[i][j])          (P_b, high part)
+lcp_status launch_sinkhorn_fwd(const float* L, float* P, float* ckpt, __nv_bfloat16* img_pt_hi,
+                               __nv_bfloat16* img_pt_lo, __nv_bfloat16* img_p_hi, int nblocks,
+                               int B, float tau, int iters, cudaStream_t st);
+lcp_status launch_sinkhorn_bwd(const float* L, const float* ckpt, const float* dP, int splits,
+                               float* dL, int nblocks, int B, float tau, int iters,
+                               cudaStream_t st);
+
+// N:M mask of a [rows, cols] matrix (float or bf16) into packed bits.
+lcp_status launch_nm_mask(const void* Wp, uint32_t* bits, int rows, int cols, int n, int m,
+                          lcp_dtype dt, cudaStream_t st);
+// out[o][j] = mask(o, j) ? in[o][j] : 0   (float32, [rows, cols])
+lcp_status launch_apply_mask(const float* in, const uint32_t* bits, float* out, int rows,
+                             int cols, cudaStream_t st);
+
+// Generic strided batched GEMM on CUDA cores with float32 accumulation:
+//   C[z](m, n) = alpha * sum_k A[z](m, k) * B[z](k, n) + beta * C[z](m, n)
+struct SimtGemm {
+  int M, N, K, batch;
+  const void* A; long long sAz, sAm, sAk;
+  const void* B; long long sBz, sBk, sBn;
+  void* C;       long long sCz, sCm, sCn;
+  float alpha, beta;
+};
+lcp_status launch_simt_gemm(const SimtGemm& g, lcp_dtype ta, lcp_dtype tb, lcp_dtype tc,
+                            cudaStream_t st);
+
+// Loss.  stats[t] = {<yd,ys>, |yd|^2, |ys|^2, cos}.  G (optional) in dtype.
+lcp_status launch_loss_token(const float* Yd, const float* Ys, float* stats, void* G,
+                             lcp_dtype gdt, int cout, int tokens, cudaStream_t st);
+lcp_status launch_loss_grad(const float* Yd, const float* Ys, const float* stats, void* G,
+                            lcp_dtype gdt, int cout, int tokens, cudaStream_t st);
+lcp_status launch_loss_reduce(const float* stats, float* loss, int tokens, cudaStream_t st);
+
+// Tensor-core (tcgen05) kernels, bf16 operands, float32 accumulation.
+bool tc_available();
+lcp_status launch_permute_mask_tc(const __nv_bfloat16* W, const __nv_bfloat16* img_pt_hi,
+                                  const __nv_bfloat16* img_pt_lo, const __nv_bfloat16* img_p_hi,
+                                  uint32_t* mask, __nv_bfloat16* At, float* Wp_out, int cout,
+                                  int cin, int B, int n, int m, cudaStream_t st);
+lcp_status launch_calib_gemm_tc(const __nv_bfloat16* X, const __nv_bfloat16* W,
+                                const __nv_bfloat16* At, float* Yd, float* Ys, int tokens,
+                                int cout, int cin, cudaStream_t st);
+lcp_status launch_bwd_gemm_tc(const __nv_bfloat16* G, const __nv_bfloat16* X,
+                              __nv_bfloat16* dAt, int tokens, int cout, int cin,
+                              cudaStream_t st);
+lcp_status launch_block_bwd_tc(const __nv_bfloat16* W, const __nv_bfloat16* dAt,
+                               const uint32_t* mask, const __nv_bfloat16* img_pt_hi,
+                               const __nv_bfloat16* img_pt_lo, float* dP_partials, int splits,
+                               int cout, int cin, int B, cudaStream_t st);
+int block_bwd_tc_splits(int cout, int cin, int B);
+
+constexpr int kCkptPerIter = 2;  // R then C vectors per iteration
+
+}  // namespace lcp

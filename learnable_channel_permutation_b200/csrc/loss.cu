@@ -1,0 +1,156 @@
+// Token-averaged cosine loss between the dense and sparse outputs and its
+// gradient with respect to the sparse output (PermLLM summary, "optimization
+// objective": L_cos(y, y~) = 1 - y.y~ / (|y| |y~|)), averaged over tokens.
+//
+//   c_t  = <yd_t, ys_t> / max(|yd_t| |ys_t|, 1e-8)
+//   loss = (1/T) sum_t (1 - c_t)
+//   G_t  = -(1/T) (yd_t / (|yd_t||ys_t|) - c_t ys_t / |ys_t|^2)
+//
+// One CTA per token reads its two rows with 128-bit loads, reduces in a fixed
+// order (deterministic), writes the four per-token statistics and optionally
+// G; a one-CTA kernel then sums the T cosines in a fixed order.
+
+#include "lcp_internal.cuh"
+
+namespace lcp {
+namespace {
+
+constexpr float kCosEps = 1e-8f;
+constexpr int NT = 256;
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+template <typename TG>
+__device__ __forceinline__ void write_g(TG* G, size_t off, float4 g);
+template <>
+__device__ __forceinline__ void write_g<float>(float* G, size_t off, float4 g) {
+  *reinterpret_cast<float4*>(G + off) = g;
+}
+template <>
+__device__ __forceinline__ void write_g<__nv_bfloat16>(__nv_bfloat16* G, size_t off, float4 g) {
+  __nv_bfloat162 a = __floats2bfloat162_rn(g.x, g.y);
+  __nv_bfloat162 b = __floats2bfloat162_rn(g.z, g.w);
+  uint2 u;
+  u.x = *reinterpret_cast<uint32_t*>(&a);
+  u.y = *reinterpret_cast<uint32_t*>(&b);
+  *reinterpret_cast<uint2*>(G + off) = u;
+}
+
+template <typename TG>
+__device__ __forceinline__ void token_grad(const float4* yd, const float4* ys, TG* G, size_t row,
+                                           int quads, float dot, float nd2, float ns2,
+                                           float inv_T) {
+  const float den = sqrtf(nd2) * sqrtf(ns2);
+  const bool ok = den > kCosEps;
+  const float c = dot / fmaxf(den, kCosEps);
+  const float a = ok ? -inv_T / den : -inv_T / kCosEps;     // coefficient of yd
+  const float b = ok ? inv_T * c / ns2 : 0.f;               // coefficient of ys
+  for (int q = threadIdx.x; q < quads; q += NT) {
+    const float4 d = yd[q], s = ys[q];
+    float4 g;
+    g.x = a * d.x + b * s.x;
+    g.y = a * d.y + b * s.y;
+    g.z = a * d.z + b * s.z;
+    g.w = a * d.w + b * s.w;
+    write_g<TG>(G, row + 4 * (size_t)q, g);
+  }
+}
+
+template <typename TG, bool WRITE_G>
+__global__ void __launch_bounds__(NT)
+loss_token_kernel(const float* __restrict__ Yd, const float* __restrict__ Ys,
+                  float* __restrict__ stats, TG* __restrict__ G, int cout, float inv_T) {
+  __shared__ float red[3][NT / 32];
+  const int t = blockIdx.x;
+  const size_t row = (size_t)t * cout;
+  const float4* yd = reinterpret_cast<const float4*>(Yd + row);
+  const float4* ys = reinterpret_cast<const float4*>(Ys + row);
+  const int quads = cout / 4;
+  float dot = 0.f, nd = 0.f, ns = 0.f;
+  for (int q = threadIdx.x; q < quads; q += NT) {
+    const float4 a = yd[q], b = ys[q];
+    dot += a.x * b.x + a.y * b.y + a.z * b.z + a.w * b.w;
+    nd += a.x * a.x + a.y * a.y + a.z * a.z + a.w * a.w;
+    ns += b.x * b.x + b.y * b.y + b.z * b.z + b.w * b.w;
+  }
+  dot = warp_sum(dot);
+  nd = warp_sum(nd);
+  ns = warp_sum(ns);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  if (lane == 0) { red[0][warp] = dot; red[1][warp] = nd; red[2][warp] = ns; }
+  __syncthreads();
+  dot = 0.f; nd = 0.f; ns = 0.f;
+#pragma unroll
+  for (int w = 0; w < NT / 32; ++w) { dot += red[0][w]; nd += red[1][w]; ns += red[2][w]; }
+  if (threadIdx.x == 0) {
+    const float c = dot / fmaxf(sqrtf(nd) * sqrtf(ns), kCosEps);
+    float4 s;
+    s.x = dot; s.y = nd; s.z = ns; s.w = c;
+    reinterpret_cast<float4*>(stats)[t] = s;
+  }
+  if constexpr (WRITE_G) token_grad<TG>(yd, ys, G, row, quads, dot, nd, ns, inv_T);
+}
+
+template <typename TG>
+__global__ void __launch_bounds__(NT)
+loss_grad_kernel(const float* __restrict__ Yd, const float* __restrict__ Ys,
+                 const float* __restrict__ stats, TG* __restrict__ G, int cout, float inv_T) {
+  const int t = blockIdx.x;
+  const size_t row = (size_t)t * cout;
+  const float4 s = reinterpret_cast<const float4*>(stats)[t];
+  token_grad<TG>(reinterpret_cast<const float4*>(Yd + row), reinterpret_cast<const float4*>(Ys + row),
+                 G, row, cout / 4, s.x, s.y, s.z, inv_T);
+}
+
+__global__ void __launch_bounds__(1024)
+loss_reduce_kernel(const float* __restrict__ stats, float* __restrict__ loss, int tokens) {
+  __shared__ double red[32];
+  double s = 0.0;
+  for (int t = threadIdx.x; t < tokens; t += 1024) s += 1.0 - (double)stats[4 * (size_t)t + 3];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (threadIdx.x % 32 == 0) red[threadIdx.x / 32] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double tot = 0.0;
+    for (int w = 0; w < 32; ++w) tot += red[w];
+    *loss = (float)(tot / tokens);
+  }
+}
+
+}  // namespace
+
+lcp_status launch_loss_token(const float* Yd, const float* Ys, float* stats, void* G,
+                             lcp_dtype gdt, int cout, int tokens, cudaStream_t st) {
+  const float inv_T = 1.0f / (float)tokens;
+  if (!G) {
+    loss_token_kernel<float, false><<<tokens, NT, 0, st>>>(Yd, Ys, stats, nullptr, cout, inv_T);
+  } else if (gdt == LCP_F32) {
+    loss_token_kernel<float, true><<<tokens, NT, 0, st>>>(Yd, Ys, stats, (float*)G, cout, inv_T);
+  } else {
+    loss_token_kernel<__nv_bfloat16, true>
+        <<<tokens, NT, 0, st>>>(Yd, Ys, stats, (__nv_bfloat16*)G, cout, inv_T);
+  }
+  return check_launch("loss_token");
+}
+
+lcp_status launch_loss_grad(const float* Yd, const float* Ys, const float* stats, void* G,
+                            lcp_dtype gdt, int cout, int tokens, cudaStream_t st) {
+  const float inv_T = 1.0f / (float)tokens;
+  if (gdt == LCP_F32)
+    loss_grad_kernel<float><<<tokens, NT, 0, st>>>(Yd, Ys, stats, (float*)G, cout, inv_T);
+  else
+    loss_grad_kernel<__nv_bfloat16><<<tokens, NT, 0, st>>>(Yd, Ys, stats, (__nv_bfloat16*)G, cout, inv_T);
+  return check_launch("loss_grad");
+}
+
+lcp_status launch_loss_reduce(const float* stats, float* loss, int tokens, cudaStream_t st) {
+  loss_reduce_kernel<<<1, 1024, 0, st>>>(stats, loss, tokens);
+  return check_launch("loss_reduce");
+}
+
+}  // namespace lcp

@@ -1,0 +1,114 @@
+"""The C-ABI library loads on a machine without a GPU, exports every symbol the
+header declares, and rejects bad arguments on the host before touching a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from learnable_channel_permutation_b200 import binding as b
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lcp.h")
+
+pytestmark = pytest.mark.skipif(not os.path.exists(b.LIB_PATH), reason="liblcp.so not built")
+
+
+def declared_symbols():
+    txt = open(HEADER).read()
+    return sorted(set(re.findall(r"^LCP_API\s+[\w\s\*]+?\b(\w+)\s*\(", txt, flags=re.M)))
+
+
+def test_header_declares_the_entry_points():
+    syms = declared_symbols()
+    for name in ["lcp_sinkhorn_fwd", "lcp_sinkhorn_bwd", "lcp_permute_weight", "nm_mask", "lcp_loss_fwd",
+                 "lcp_loss_bwd", "lcp_step", "lcp_workspace_size", "lcp_status_string"]:
+        assert name in syms
+
+
+def test_library_exports_every_declared_symbol():
+    L = b.lib()
+    for name in declared_symbols():
+        assert hasattr(L, name), name
+    assert L.lcp_abi_version() == int(re.search(r"#define LCP_ABI_VERSION (\d+)", open(HEADER).read()).group(1))
+
+
+def _layer(cout=64, cin=128, T=32, base=0x10000000):
+    p = lambda k: base + 0x100000 * k   # fake, 16-byte aligned device addresses (never dereferenced)
+    return b.LcpLayer(p(1), p(2), p(3), p(4), p(5), p(6), None, None, cout, cin, T)
+
+
+def _ws(layers, hp):
+    arr = (b.LcpLayer * len(layers))(*layers)
+    n = ctypes.c_size_t(0)
+    st = b.lib().lcp_workspace_size(arr, len(layers), ctypes.byref(hp), ctypes.byref(n))
+    return st, n.value
+
+
+def test_workspace_size_for_valid_layers():
+    hp = b.hparams(64, 2, 4, 5, 0.5, b.BF16)
+    st, n = _ws([_layer()], hp)
+    assert st == 0 and n > 0
+    st2, n2 = _ws([_layer(), _layer(cout=128)], hp)
+    assert st2 == 0 and n2 >= n
+    st0, n0 = _ws([], hp)
+    assert st0 == 0 and n0 == 0
+
+
+@pytest.mark.parametrize("mut,code", [
+    (lambda l, h: setattr(h, "block", 48), 2),
+    (lambda l, h: setattr(h, "block", 512), 2),
+    (lambda l, h: setattr(h, "m", 6), 2),
+    (lambda l, h: setattr(h, "n", 0), 2),
+    (lambda l, h: setattr(h, "n", 5), 2),
+    (lambda l, h: setattr(h, "iters", 0), 7),
+    (lambda l, h: setattr(h, "tau", 0.0), 7),
+    (lambda l, h: setattr(h, "tau", float("inf")), 7),
+    (lambda l, h: setattr(h, "dtype", 9), 3),
+    (lambda l, h: setattr(h, "flags", 0x100), 7),
+    (lambda l, h: setattr(l, "W", None), 1),
+    (lambda l, h: setattr(l, "loss", None), 1),
+    (lambda l, h: setattr(l, "cout", 12), 2),
+    (lambda l, h: setattr(l, "cout", 0), 2),
+    (lambda l, h: setattr(l, "cin", 96), 2),       # not a multiple of B = 64
+    (lambda l, h: setattr(l, "tokens", 0), 2),
+    (lambda l, h: setattr(l, "X", 0x10000008), 7),  # misaligned
+    (lambda l, h: setattr(h, "flags", b.FLAG_WRITE_WPRIME), 1),  # needs layer.Wp
+])
+def test_host_validation_codes(mut, code):
+    l = _layer()
+    hp = b.hparams(64, 2, 4, 5, 0.5, b.BF16)
+    mut(l, hp)
+    st, _ = _ws([l], hp)
+    assert st == code
+    assert b.lib().lcp_last_error().decode() != ""
+
+
+def test_step_rejects_small_or_misaligned_workspace_without_a_gpu():
+    L = b.lib()
+    hp = b.hparams(64, 2, 4, 5, 0.5, b.BF16)
+    arr = (b.LcpLayer * 1)(_layer())
+    _, need = _ws([_layer()], hp)
+    assert L.lcp_step(arr, 1, ctypes.byref(hp), 0x20000000, need - 1, None) == 4
+    assert L.lcp_step(arr, 1, ctypes.byref(hp), 0x20000010, need, None) == 4
+    assert L.lcp_step(arr, 0, ctypes.byref(hp), None, 0, None) == 0   # no layers: a no-op
+
+
+def test_standalone_entry_points_validate_before_launch():
+    L = b.lib()
+    assert L.lcp_sinkhorn_fwd(None, 0x1000, None, 1, 64, 1.0, 5, None) == 1
+    assert L.lcp_sinkhorn_fwd(0x1000, 0x2000, None, 1, 40, 1.0, 5, None) == 2
+    assert L.lcp_sinkhorn_fwd(0x1000, 0x2000, None, 0, 64, 1.0, 5, None) == 0  # empty
+    assert L.nm_mask(0x1000, 0x2000, 4, 30, 2, 4, 0, None) == 2
+    assert L.nm_mask(0x1000, 0x2000, 4, 32, 2, 5, 0, None) == 2
+    assert L.nm_mask(0x1000, 0x2000, 0, 32, 2, 4, 0, None) == 0               # empty
+    assert L.lcp_loss_fwd(0x1000, 0x2000, 0x3000, 0x4000, 12, 5, None) == 2
+    assert L.lcp_sinkhorn_bwd(0x1000, 0x2000, 0x3000, 0, 0x4000, 1, 64, 1.0, 5, None) == 7
+
+
+def test_launch_count_reported():
+    hp = b.hparams(64, 2, 4, 5, 0.5, b.F32)
+    arr = (b.LcpLayer * 2)(_layer(), _layer())
+    c = ctypes.c_int(0)
+    assert b.lib().lcp_step_launches(arr, 2, ctypes.byref(hp), ctypes.byref(c)) == 0
+    assert c.value > 0 and c.value % 2 == 0
