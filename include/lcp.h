@@ -162,6 +162,25 @@ LCP_API lcp_status lcp_loss_fwd(const float* Yd, const float* Ys, float* loss, f
 LCP_API lcp_status lcp_loss_bwd(const float* Yd, const float* Ys, const float* stats, void* G, int cout,
                         int tokens, lcp_dtype dtype, cudaStream_t stream);
 
+/* Allocation-free variant of lcp_loss_fwd (the paper has no counterpart; this
+ * is a library convenience).  Same loss, same arguments minus the scratch
+ * buffer: the per-token scratch lives in a static __device__ array of
+ * LCP_STATIC_MAX_TOKENS * 4 floats that every GPU loading the library holds
+ * until exit.  For callers that cannot allocate device memory: code running
+ * while a stream is captured into a CUDA graph or inside a stream-ordered
+ * pipeline (cudaMalloc may synchronise the device), and embedders whose device
+ * memory belongs to another allocator or is reserved up front.
+ * - tokens > LCP_STATIC_MAX_TOKENS is rejected with LCP_ERR_SHAPE.
+ * - The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make it before any
+ *   stream capture begins.
+ * - All calls share the array (each call overwrites all of it that it reads,
+ *   so nothing must be cleared); calls that overlap on the GPU race on it.
+ * - Allocates and frees nothing, calls no allocating routine. */
+#define LCP_STATIC_MAX_TOKENS 65536
+LCP_API lcp_status lcp_loss_fwd_static(const float* Yd, const float* Ys, float* loss, int cout,
+                                       int tokens, cudaStream_t stream);
+
 LCP_API const char* lcp_status_string(lcp_status s);
 /* Message of the last failed call made by this thread ("" if none). */
 LCP_API const char* lcp_last_error(void);

@@ -71,6 +71,7 @@ def lib() -> ctypes.CDLL:
         "nm_mask": ([_c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_int, _c_int, _c_void_p], _c_int),
         "lcp_loss_fwd": ([_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_void_p], _c_int),
         "lcp_loss_bwd": ([_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_void_p], _c_int),
+        "lcp_loss_fwd_static": ([_c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_void_p], _c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -227,3 +228,14 @@ def loss_bwd(Yd: torch.Tensor, Ys: torch.Tensor, stats: torch.Tensor, G: torch.T
     check(lib().lcp_loss_bwd(_ptr(Yd, torch.float32, "Yd"), _ptr(Ys, torch.float32, "Ys"),
                              _ptr(stats, torch.float32, "stats"), _ptr(G, None, "G"), cout, T, _dt(G),
                              _stream(None)))
+
+
+STATIC_MAX_TOKENS = 65536
+
+
+def loss_fwd_static(Yd: torch.Tensor, Ys: torch.Tensor, loss: torch.Tensor) -> None:
+    """lcp_loss_fwd without a scratch argument: for callers that cannot allocate
+    device memory (see lcp_loss_fwd_static in include/lcp.h)."""
+    T, cout = Yd.shape
+    check(lib().lcp_loss_fwd_static(_ptr(Yd, torch.float32, "Yd"), _ptr(Ys, torch.float32, "Ys"),
+                                    _ptr(loss, torch.float32, "loss"), cout, T, _stream(None)))
