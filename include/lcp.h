@@ -162,6 +162,26 @@ LCP_API lcp_status lcp_loss_fwd(const float* Yd, const float* Ys, float* loss, f
 LCP_API lcp_status lcp_loss_bwd(const float* Yd, const float* Ys, const float* stats, void* G, int cout,
                         int tokens, lcp_dtype dtype, cudaStream_t stream);
 
+/* Calibration outputs on the tensor cores ("optimization objective": the dense
+ * output y = W X and the sparse output y~ = At X with At = (M.W') P_B^T):
+ * Yd = X W^T and, when At and Ys are given, Ys = X At^T.  X [T, C_in],
+ * W and At [C_out, C_in] bf16; Yd, Ys [T, C_out] float32 (float32
+ * accumulation).  C_out and C_in multiples of 8, T >= 1. */
+LCP_API lcp_status lcp_calib_gemm(const void* X, const void* W, const void* At, float* Yd, float* Ys,
+                                  int tokens, int cout, int cin, cudaStream_t stream);
+
+/* Weight gradient of the sparse output on the tensor cores: dAt = G^T X with
+ * G [T, C_out] and X [T, C_in] bf16 and dAt [C_out, C_in] bf16 (float32
+ * accumulation over the T tokens). */
+LCP_API lcp_status lcp_grad_gemm(const void* G, const void* X, void* dAt, int tokens, int cout,
+                                 int cin, cudaStream_t stream);
+
+/* Diagnostic (synchronous: reads a device word).  Every wait inside the
+ * tensor-core kernels is bounded; a wait that expires records its site here
+ * (0 = none) and the kernel returns early with incomplete results.  With
+ * reset != 0 the word is cleared after reading. */
+LCP_API lcp_status lcp_device_error(int* site, int reset);
+
 /* Allocation-free variant of lcp_loss_fwd (the paper has no counterpart; this
  * is a library convenience).  Same loss, same arguments minus the scratch
  * buffer: the per-token scratch lives in a static __device__ array of

@@ -72,6 +72,10 @@ def lib() -> ctypes.CDLL:
         "lcp_loss_fwd": ([_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_void_p], _c_int),
         "lcp_loss_bwd": ([_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_void_p], _c_int),
         "lcp_loss_fwd_static": ([_c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_void_p], _c_int),
+        "lcp_calib_gemm": ([_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_int,
+                            _c_void_p], _c_int),
+        "lcp_grad_gemm": ([_c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_void_p], _c_int),
+        "lcp_device_error": ([P(_c_int), _c_int], _c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -214,6 +218,31 @@ def nm_mask(Wp: torch.Tensor, bits: torch.Tensor, n: int, m: int) -> None:
     rows, cols = Wp.shape
     check(lib().nm_mask(_ptr(Wp, None, "Wp"), _ptr(bits, torch.int32, "bits"), rows, cols, n, m, _dt(Wp),
                         _stream(None)))
+
+
+def calib_gemm(X: torch.Tensor, W: torch.Tensor, At: Optional[torch.Tensor], Yd: torch.Tensor,
+               Ys: Optional[torch.Tensor]) -> None:
+    T, cin = X.shape
+    cout = W.shape[0]
+    bf = torch.bfloat16
+    check(lib().lcp_calib_gemm(_ptr(X, bf, "X"), _ptr(W, bf, "W"), _ptr(At, bf, "At"),
+                               _ptr(Yd, torch.float32, "Yd"), _ptr(Ys, torch.float32, "Ys"), T, cout, cin,
+                               _stream(None)))
+
+
+def grad_gemm(G: torch.Tensor, X: torch.Tensor, dAt: torch.Tensor) -> None:
+    T, cout = G.shape
+    cin = X.shape[1]
+    bf = torch.bfloat16
+    check(lib().lcp_grad_gemm(_ptr(G, bf, "G"), _ptr(X, bf, "X"), _ptr(dAt, bf, "dAt"), T, cout, cin,
+                              _stream(None)))
+
+
+def device_error(reset: bool = True) -> int:
+    """Site code of the first tensor-core wait that expired (0 = none); synchronous."""
+    v = _c_int(0)
+    check(lib().lcp_device_error(ctypes.byref(v), 1 if reset else 0))
+    return int(v.value)
 
 
 def loss_fwd(Yd: torch.Tensor, Ys: torch.Tensor, loss: torch.Tensor, stats: torch.Tensor) -> None:

@@ -97,6 +97,10 @@ lcp_status check_hparams(const lcp_hparams* hp) {
   return LCP_OK;
 }
 
+bool use_tc(const lcp_hparams& hp) {
+  return hp.dtype == LCP_BF16 && !(hp.flags & LCP_FLAG_SIMT) && tc_available();
+}
+
 lcp_status check_layer(const lcp_layer& l, const lcp_hparams& hp, int idx) {
   if (!l.W || !l.X || !l.L || !l.P || !l.dL || !l.loss)
     return fail(LCP_ERR_NULL, "layer %d: W, X, L, P, dL and loss are required", idx);
@@ -109,15 +113,16 @@ lcp_status check_layer(const lcp_layer& l, const lcp_hparams& hp, int idx) {
                 idx, l.cin, hp.block);
   if (l.tokens < 1 || l.tokens > kMaxDim)
     return fail(LCP_ERR_SHAPE, "layer %d: T = %d must be >= 1", idx, l.tokens);
+  if (use_tc(hp) && l.cin % 64)
+    return fail(LCP_ERR_SHAPE,
+                "layer %d: C_in = %d must be a multiple of 64 on the tensor-core path "
+                "(LCP_FLAG_SIMT accepts multiples of 32)", idx, l.cin);
   const void* ptrs[] = {l.W, l.X, l.L, l.P, l.dL, l.mask, l.Wp};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return fail(LCP_ERR_ARG, "layer %d: every pointer must be 16-byte aligned", idx);
   return LCP_OK;
 }
 
-bool use_tc(const lcp_hparams& hp) {
-  return hp.dtype == LCP_BF16 && !(hp.flags & LCP_FLAG_SIMT) && tc_available();
-}
 
 size_t esize(lcp_dtype d) { return d == LCP_F32 ? 4 : 2; }
 
@@ -141,19 +146,22 @@ Plan make_plan(const lcp_layer& l, const lcp_hparams& hp) {
   };
   p.splits = tc ? block_bwd_tc_splits(l.cout, l.cin, hp.block) : 1;
   p.ckpt = take(nb * hp.iters * 2 * B * 4);
-  p.img0 = take(tc ? nb * B * B * 2 : 0);
-  p.img1 = take(tc ? nb * B * B * 2 : 0);
-  p.img2 = take(tc ? nb * B * B * 2 : 0);
+  const size_t BC = B < 64 ? 64 : B;   // tile width of the operand images
+  p.img0 = take(tc ? ic * BC * 2 : 0);
+  p.img1 = take(tc ? ic * BC * 2 : 0);
+  p.img2 = take(tc ? ic * BC * 2 : 0);
   p.mask = take(oc * ic / 8);
-  p.wp = take(tc ? 0 : oc * ic * 4);
-  p.amask = take(tc ? 0 : oc * ic * 4);
+  // the CUDA-core block backward (f32, LCP_FLAG_SIMT, or B = 256) works on float32 W', A, dA
+  const bool simt_bwd = !tc || !block_bwd_tc_supported(hp.block);
+  p.wp = take(simt_bwd ? oc * ic * 4 : 0);
+  p.amask = take(simt_bwd ? oc * ic * 4 : 0);
   p.at = take(oc * ic * es);
   p.yd = take(T * oc * 4);
   p.ys = take(T * oc * 4);
   p.stats = take(T * 16);
   p.g = take(T * oc * es);
   p.dat = take(oc * ic * (tc ? 2 : 4));
-  p.da = take(tc ? 0 : oc * ic * 4);
+  p.da = take(simt_bwd ? oc * ic * 4 : 0);
   p.dp = take((size_t)p.splits * nb * B * B * 4);
   p.total = off;
   return p;
@@ -238,6 +246,12 @@ lcp_status layer_simt(const lcp_layer& l, const lcp_hparams& hp, const Plan& p, 
 
 constexpr int kSimtLaunches = 15;
 constexpr int kTcLaunches = 8;
+constexpr int kTcLaunchesSimtBwd = 13;   // B = 256: block backward on CUDA cores (6 launches)
+
+int launches_per_layer(const lcp_hparams& hp) {
+  if (!use_tc(hp)) return kSimtLaunches;
+  return block_bwd_tc_supported(hp.block) ? kTcLaunches : kTcLaunchesSimtBwd;
+}
 
 // ---- one layer, tensor-core path (bf16 operands, float32 accumulation) -----
 lcp_status layer_tc(const lcp_layer& l, const lcp_hparams& hp, const Plan& p, void* ws,
@@ -271,7 +285,26 @@ lcp_status layer_tc(const lcp_layer& l, const lcp_hparams& hp, const Plan& p, vo
   LCP_TRY(record(ev, 4, st));
   LCP_TRY(launch_bwd_gemm_tc(G, X, dAt, l.tokens, l.cout, l.cin, st));
   LCP_TRY(record(ev, 5, st));
-  LCP_TRY(launch_block_bwd_tc(W, dAt, mask, pt_hi, pt_lo, dP, p.splits, l.cout, l.cin, B, st));
+  if (block_bwd_tc_supported(B)) {
+    LCP_TRY(launch_block_bwd_tc(W, dAt, mask, pt_hi, pt_lo, dP, p.splits, l.cout, l.cin, B, st));
+  } else {
+    // B = 256: the fused kernel does not fit one SM's tensor memory; use the
+    // CUDA-core products on float32 W', A = M.W' and dA.
+    const long long ic = l.cin, BB = (long long)B * B;
+    float* Wp32 = at<float>(ws, p.wp);
+    float* Am = at<float>(ws, p.amask);
+    float* dA = at<float>(ws, p.da);
+    LCP_TRY(launch_simt_gemm({l.cout, B, B, nb, W, B, ic, 1, l.P, BB, B, 1, Wp32, B, ic, 1, 1.f, 0.f},
+                             LCP_BF16, LCP_F32, LCP_F32, st));
+    LCP_TRY(launch_apply_mask(Wp32, mask, Am, l.cout, l.cin, st));
+    LCP_TRY(launch_simt_gemm({l.cout, B, B, nb, dAt, B, ic, 1, l.P, BB, B, 1, dA, B, ic, 1, 1.f, 0.f},
+                             LCP_BF16, LCP_F32, LCP_F32, st));
+    LCP_TRY(launch_apply_mask(dA, mask, dA, l.cout, l.cin, st));
+    LCP_TRY(launch_simt_gemm({B, B, l.cout, nb, dAt, B, 1, ic, Am, B, ic, 1, dP, BB, B, 1, 1.f, 0.f},
+                             LCP_BF16, LCP_F32, LCP_F32, st));
+    LCP_TRY(launch_simt_gemm({B, B, l.cout, nb, W, B, 1, ic, dA, B, ic, 1, dP, BB, B, 1, 1.f, 1.f},
+                             LCP_BF16, LCP_F32, LCP_F32, st));
+  }
   LCP_TRY(record(ev, 6, st));
   LCP_TRY(launch_sinkhorn_bwd(l.L, ckpt, dP, p.splits, l.dL, nb, B, hp.tau, hp.iters, st));
   LCP_TRY(record(ev, 7, st));
@@ -341,7 +374,7 @@ lcp_status lcp_step_launches(const lcp_layer* layers, int nlayers, const lcp_hpa
                              int* launches) {
   if (!launches) return fail(LCP_ERR_NULL, "launches is NULL");
   LCP_TRY(validate_all(layers, nlayers, hp));
-  *launches = nlayers * (use_tc(*hp) ? kTcLaunches : kSimtLaunches);
+  *launches = nlayers * launches_per_layer(*hp);
   return LCP_OK;
 }
 
@@ -415,6 +448,35 @@ lcp_status nm_mask(const void* Wp, uint32_t* mask_bits, int rows, int cols, int 
   LCP_TRY(check_arch());
   cudaGetLastError();
   return launch_nm_mask(Wp, mask_bits, rows, cols, n, m, dtype, stream);
+}
+
+lcp_status lcp_calib_gemm(const void* X, const void* W, const void* At, float* Yd, float* Ys, int tokens,
+                          int cout, int cin, cudaStream_t stream) {
+  if (!X || !W || !Yd) return fail(LCP_ERR_NULL, "X, W and Yd are required");
+  if ((At == nullptr) != (Ys == nullptr)) return fail(LCP_ERR_NULL, "At and Ys go together");
+  if (cout < 8 || cout % 8 || cout > kMaxDim) return fail(LCP_ERR_SHAPE, "C_out = %d must be a positive multiple of 8", cout);
+  if (cin < 8 || cin % 8 || cin > kMaxDim) return fail(LCP_ERR_SHAPE, "C_in = %d must be a positive multiple of 8", cin);
+  if (tokens < 1 || tokens > kMaxDim) return fail(LCP_ERR_SHAPE, "T = %d must be >= 1", tokens);
+  const void* ptrs[] = {X, W, At, Yd, Ys};
+  for (const void* q : ptrs)
+    if (q && !aligned16(q)) return fail(LCP_ERR_ARG, "pointers must be 16-byte aligned");
+  LCP_TRY(check_arch());
+  cudaGetLastError();
+  return launch_calib_gemm_tc(static_cast<const __nv_bfloat16*>(X), static_cast<const __nv_bfloat16*>(W),
+                              static_cast<const __nv_bfloat16*>(At), Yd, Ys, tokens, cout, cin, stream);
+}
+
+lcp_status lcp_grad_gemm(const void* G, const void* X, void* dAt, int tokens, int cout, int cin,
+                         cudaStream_t stream) {
+  if (!G || !X || !dAt) return fail(LCP_ERR_NULL, "G, X and dAt are required");
+  if (cout < 8 || cout % 8 || cout > kMaxDim) return fail(LCP_ERR_SHAPE, "C_out = %d must be a positive multiple of 8", cout);
+  if (cin < 8 || cin % 8 || cin > kMaxDim) return fail(LCP_ERR_SHAPE, "C_in = %d must be a positive multiple of 8", cin);
+  if (tokens < 1 || tokens > kMaxDim) return fail(LCP_ERR_SHAPE, "T = %d must be >= 1", tokens);
+  if (!aligned16(G) || !aligned16(X) || !aligned16(dAt)) return fail(LCP_ERR_ARG, "pointers must be 16-byte aligned");
+  LCP_TRY(check_arch());
+  cudaGetLastError();
+  return launch_bwd_gemm_tc(static_cast<const __nv_bfloat16*>(G), static_cast<const __nv_bfloat16*>(X),
+                            static_cast<__nv_bfloat16*>(dAt), tokens, cout, cin, stream);
 }
 
 lcp_status lcp_loss_fwd(const float* Yd, const float* Ys, float* loss, float* stats, int cout,

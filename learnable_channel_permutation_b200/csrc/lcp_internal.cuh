@@ -26,10 +26,12 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 
 // ---- launchers (host side; each returns LCP_OK or LCP_ERR_CUDA) ----------
 
-// Sinkhorn.  img_* are optional bf16 operand images for the tensor-core path:
-//   img_pt_hi[b][j][i] = bf16(P_b[i][j])          (P_b transposed, high part)
-//   img_pt_lo[b][j][i] = bf16(P_b[i][j] - hi)     (P_b transposed, low part)
-//   img_p_hi [b][i][j] = bf16(P_b[i][j])          (P_b, high part)
+// Sinkhorn.  img_* are optional bf16 operand images for the tensor-core path,
+// stored as C_in/BC tiles of BC x BC (BC = max(B, 64)); tile t is the slice of
+// blockdiag(P) covering channels [t*BC, (t+1)*BC), so with local indices:
+//   img_pt_hi[t][j][i] = bf16(P[i][j])          (transposed, high part)
+//   img_pt_lo[t][j][i] = bf16(P[i][j] - hi)     (transposed, low part)
+//   img_p_hi [t][i][j] = bf16(P[i][j])          (high part)
 lcp_status launch_sinkhorn_fwd(const float* L, float* P, float* ckpt, __nv_bfloat16* img_pt_hi,
                                __nv_bfloat16* img_pt_lo, __nv_bfloat16* img_p_hi, int nblocks,
                                int B, float tau, int iters, cudaStream_t st);
@@ -80,6 +82,7 @@ lcp_status launch_block_bwd_tc(const __nv_bfloat16* W, const __nv_bfloat16* dAt,
                                const __nv_bfloat16* img_pt_lo, float* dP_partials, int splits,
                                int cout, int cin, int B, cudaStream_t st);
 int block_bwd_tc_splits(int cout, int cin, int B);
+bool block_bwd_tc_supported(int B);   // B <= 128 (TMEM/smem budget of the fused kernel)
 
 constexpr int kCkptPerIter = 2;  // R then C vectors per iteration
 

@@ -138,6 +138,15 @@ sinkhorn_fwd_kernel(const float* __restrict__ L, float* __restrict__ P, float* _
     __syncthreads();
   }
 
+  // Operand images for the tensor-core kernels, in tiles of BC = max(B, 64)
+  // columns: tile t holds the BC x BC block-diagonal slice of P_B covering
+  // channels [t*BC, (t+1)*BC) (for B = 32 two blocks share one tile and the
+  // off-diagonal quadrants are written as zeros).
+  constexpr int BC = B < 64 ? 64 : B;
+  const int gcol0 = blk * B;
+  const size_t tbase = (size_t)(gcol0 / BC) * BC * BC;
+  const int q0 = gcol0 % BC;
+  const __nv_bfloat16 zero = __float2bfloat16_rn(0.f);
   for (int e = tid; e < R * B; e += NT) {
     const int r = e / B, j = e % B;
     const float p = expf(z[e] - rv[r] - cv[j]);
@@ -146,9 +155,15 @@ sinkhorn_fwd_kernel(const float* __restrict__ L, float* __restrict__ P, float* _
     if (pt_hi) {
       const __nv_bfloat16 hi = __float2bfloat16_rn(p);
       const __nv_bfloat16 lo = __float2bfloat16_rn(p - __bfloat162float(hi));
-      pt_hi[base + (size_t)j * B + i] = hi;
-      pt_lo[base + (size_t)j * B + i] = lo;
-      p_hi[base + (size_t)i * B + j] = hi;
+      pt_hi[tbase + (size_t)(q0 + j) * BC + q0 + i] = hi;
+      pt_lo[tbase + (size_t)(q0 + j) * BC + q0 + i] = lo;
+      p_hi[tbase + (size_t)(q0 + i) * BC + q0 + j] = hi;
+      if constexpr (B < BC) {
+        const int zc = (q0 == 0) ? B : 0;
+        pt_hi[tbase + (size_t)(q0 + j) * BC + zc + i] = zero;
+        pt_lo[tbase + (size_t)(q0 + j) * BC + zc + i] = zero;
+        p_hi[tbase + (size_t)(q0 + i) * BC + zc + j] = zero;
+      }
     }
   }
   // keep peers' shared memory alive until every CTA of the cluster is done reading it
