@@ -8,15 +8,18 @@
 //
 // Every log-domain iterate has the form Z = Z_0 - R_i - C_j, so a row step
 // only has to compute R_i = LSE_j(Z_0[i,j] - C_j) and a column step
-// C_j = LSE_i(Z_0[i,j] - R_i).  Z_0 = L / tau stays resident in shared
-// memory; the (R, C) pair of every iteration is the checkpoint the reverse
-// pass replays (2 * iters * B floats per block instead of 2 * iters * B^2).
+// C_j = LSE_i(Z_0[i,j] - R_i).  Z_0 = L / tau never changes, so each thread
+// keeps its share of Z_0 in registers twice: a row slice (TPR adjacent lanes
+// per row, interleaved columns) for the row steps and a column slice (TPC
+// adjacent lanes per column, interleaved rows) for the column steps.  A step
+// is then register arithmetic, a read of the other side's normaliser vector
+// from shared memory and two or three shuffles; the (R, C) pair of every
+// iteration is the checkpoint the reverse pass replays.
 //
-// One CTA owns one block (B <= 128).  For B = 256 the 256 KB fp32 tile does
-// not fit one CTA's shared memory, so a cluster of CS CTAs splits the rows;
-// column reductions combine per-CTA partials through distributed shared
-// memory (fixed rank order, so every CTA gets bit-identical results).
-// All reductions run in a fixed order: results are deterministic.
+// One CTA owns one block for B <= 128.  For B = 256 a cluster of 4 CTAs
+// splits the rows; column reductions combine the per-CTA partials through
+// distributed shared memory in a fixed rank order, so every CTA gets
+// bit-identical results.  Every reduction runs in a fixed order.
 
 #include <cooperative_groups.h>
 #include <math_constants.h>
@@ -28,23 +31,19 @@ namespace cg = cooperative_groups;
 namespace lcp {
 namespace {
 
-__device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
-}
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
-
 template <int B> struct SkCfg {
-  static constexpr int CS = (B == 256) ? 4 : 1;          // CTAs per block (row split)
-  static constexpr int NT = (B <= 64) ? 256 : 512;       // threads per CTA
-  static constexpr int R = B / CS;                       // rows per CTA
-  static constexpr int G = NT / B;                       // row groups of the column pass
-  static_assert(NT % B == 0 && R % G == 0, "bad Sinkhorn configuration");
+  static constexpr int CS = (B == 256) ? 4 : 1;                   // CTAs per block
+  static constexpr int NT = (B == 32) ? 128 : (B == 64 ? 256 : 512);
+  static constexpr int R = B / CS;                                 // rows per CTA
+  static constexpr int TPR = NT / R;                               // lanes per row
+  static constexpr int EPR = B / TPR;                              // elements per row slice
+  static constexpr int TPC = NT / B;                               // lanes per column
+  static constexpr int EPC = R / TPC;                              // elements per column slice
+  static constexpr int NW = NT / 32;
+  static constexpr int LD = B + 1;                                 // padded smem tile row
+  static_assert(TPR >= 1 && TPR <= 32 && (32 % TPR) == 0, "row slices must sit inside a warp");
+  static_assert(TPC >= 1 && TPC <= 32 && (32 % TPC) == 0, "column slices must sit inside a warp");
+  static_assert(R * TPR == NT && B * TPC == NT, "bad Sinkhorn configuration");
 };
 
 template <int CS> __device__ __forceinline__ int cta_rank() {
@@ -59,133 +58,190 @@ template <int CS> __device__ __forceinline__ const float* peer(float* p, int r) 
   else return p;
 }
 
-// Forward.  Shared memory (floats): z[R*B] rv[R] cv[B] pm[G*B] ps[G*B] xm[2*B] xs[2*B]
+// reductions over `W` adjacent lanes (W a power of two)
+template <int W> __device__ __forceinline__ float group_max(float v) {
+#pragma unroll
+  for (int o = 1; o < W; o <<= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+template <int W> __device__ __forceinline__ float group_sum(float v) {
+#pragma unroll
+  for (int o = 1; o < W; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// log-sum-exp of x[0..N) combined over W adjacent lanes
+template <int N, int W> __device__ __forceinline__ void lse_parts(const float (&x)[N], float& m, float& s) {
+  float mx = x[0];
+#pragma unroll
+  for (int e = 1; e < N; ++e) mx = fmaxf(mx, x[e]);
+  m = group_max<W>(mx);
+  float acc = 0.f;
+#pragma unroll
+  for (int e = 0; e < N; ++e) acc += expf(x[e] - m);
+  s = group_sum<W>(acc);
+}
+
+// Stage a R x B row-major slab of a float32 [*, B, B] tensor into the padded tile (coalesced).
+template <int B, int NT, int R>
+__device__ __forceinline__ void load_slab(float* tile, const float* __restrict__ src, float scale) {
+  constexpr int Q = B / 4;
+  for (int q = threadIdx.x; q < R * Q; q += NT) {
+    const float4 v = reinterpret_cast<const float4*>(src)[q];
+    const int r = q / Q, j = (q % Q) * 4;
+    float* d = tile + r * (B + 1) + j;
+    d[0] = v.x * scale; d[1] = v.y * scale; d[2] = v.z * scale; d[3] = v.w * scale;
+  }
+}
+
+// Forward.  Shared memory (floats): tile[R*(B+1)] rv[R] cv[B] xm[2B] xs[2B]
 template <int B>
 __global__ void __launch_bounds__(SkCfg<B>::NT)
 sinkhorn_fwd_kernel(const float* __restrict__ L, float* __restrict__ P, float* __restrict__ ckpt,
                     __nv_bfloat16* __restrict__ pt_hi, __nv_bfloat16* __restrict__ pt_lo,
                     __nv_bfloat16* __restrict__ p_hi, float tau, int iters) {
   using C = SkCfg<B>;
-  constexpr int R = C::R, G = C::G, NT = C::NT, NW = NT / 32, CS = C::CS;
+  constexpr int R = C::R, NT = C::NT, CS = C::CS, TPR = C::TPR, EPR = C::EPR, TPC = C::TPC,
+                EPC = C::EPC, LD = C::LD;
   extern __shared__ __align__(16) float sm[];
-  float* z = sm;
-  float* rv = z + R * B;
+  float* tile = sm;
+  float* rv = tile + R * LD;
   float* cv = rv + R;
-  float* pm = cv + B;
-  float* ps = pm + G * B;
-  float* xm = ps + G * B;   // this CTA's column partials, double-buffered by iteration parity
+  float* xm = cv + B;   // this CTA's column partials, double-buffered by iteration parity
   float* xs = xm + 2 * B;
 
   const int rank = cta_rank<CS>();
   const int blk = blockIdx.x / CS;
   const int row0 = rank * R;
-  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const int tid = threadIdx.x;
   const size_t base = (size_t)blk * B * B;
+  const int r = tid / TPR, c = tid % TPR;     // row slice: row r, columns c + TPR*e
+  const int j = tid / TPC, g = tid % TPC;     // column slice: column j, rows g + TPC*e
 
-  for (int e = tid; e < R * B; e += NT) z[e] = L[base + (size_t)row0 * B + e] / tau;
-  for (int j = tid; j < B; j += NT) cv[j] = 0.f;
+  // Z_0 = L / tau.  Division kept exact (not a reciprocal multiply) on load.
+  for (int q = tid; q < R * (B / 4); q += NT) {
+    const float4 v = reinterpret_cast<const float4*>(L + base + (size_t)row0 * B)[q];
+    const int rr = q / (B / 4), jj = (q % (B / 4)) * 4;
+    float* d = tile + rr * LD + jj;
+    d[0] = v.x / tau; d[1] = v.y / tau; d[2] = v.z / tau; d[3] = v.w / tau;
+  }
+  for (int jj = tid; jj < B; jj += NT) cv[jj] = 0.f;
   __syncthreads();
+  float zr[EPR], zc[EPC];
+#pragma unroll
+  for (int e = 0; e < EPR; ++e) zr[e] = tile[r * LD + c + TPR * e];
+#pragma unroll
+  for (int e = 0; e < EPC; ++e) zc[e] = tile[(g + TPC * e) * LD + j];
 
+  float myR = 0.f;
   for (int k = 0; k < iters; ++k) {
-    // T_r: R_i = LSE_j(z_ij - C_j) -- one warp per row
-    for (int r = warp; r < R; r += NW) {
-      const float* zr = z + r * B;
-      float mx = -CUDART_INF_F;
-      for (int j = lane; j < B; j += 32) mx = fmaxf(mx, zr[j] - cv[j]);
-      mx = warp_max(mx);
-      float s = 0.f;
-      for (int j = lane; j < B; j += 32) s += expf(zr[j] - cv[j] - mx);
-      s = warp_sum(s);
-      if (lane == 0) {
-        const float v = mx + logf(s);
-        rv[r] = v;
-        if (ckpt) ckpt[((size_t)blk * iters + k) * 2 * B + row0 + r] = v;
+    // T_r: R_i = LSE_j(z_ij - C_j)
+    {
+      float x[EPR];
+#pragma unroll
+      for (int e = 0; e < EPR; ++e) x[e] = zr[e] - cv[c + TPR * e];
+      float m, s;
+      lse_parts<EPR, TPR>(x, m, s);
+      myR = m + logf(s);
+      if (c == 0) {
+        rv[r] = myR;
+        if (ckpt) ckpt[((size_t)blk * iters + k) * 2 * B + row0 + r] = myR;
       }
     }
     __syncthreads();
     // T_c: C_j = LSE_i(z_ij - R_i) over all B rows of the block
     {
-      const int j = tid % B, g = tid / B;
-      float mx = -CUDART_INF_F;
-      for (int r = g; r < R; r += G) mx = fmaxf(mx, z[r * B + j] - rv[r]);
-      float s = 0.f;
-      for (int r = g; r < R; r += G) s += expf(z[r * B + j] - rv[r] - mx);
-      pm[g * B + j] = mx;
-      ps[g * B + j] = s;
+      float x[EPC];
+#pragma unroll
+      for (int e = 0; e < EPC; ++e) x[e] = zc[e] - rv[g + TPC * e];
+      float m, s;
+      lse_parts<EPC, TPC>(x, m, s);
+      if constexpr (CS == 1) {
+        if (g == 0) {
+          const float v = m + logf(s);
+          cv[j] = v;
+          if (ckpt) ckpt[(((size_t)blk * iters + k) * 2 + 1) * B + j] = v;
+        }
+        __syncthreads();
+      } else {
+        float* bm = xm + (k & 1) * B;
+        float* bs = xs + (k & 1) * B;
+        if (g == 0) { bm[j] = m; bs[j] = s; }
+        cluster_barrier<CS>();
+        if (g == 0) {
+          float M = -CUDART_INF_F;
+#pragma unroll
+          for (int q = 0; q < CS; ++q) M = fmaxf(M, peer<CS>(bm, q)[j]);
+          float S = 0.f;
+#pragma unroll
+          for (int q = 0; q < CS; ++q) S += peer<CS>(bs, q)[j] * expf(peer<CS>(bm, q)[j] - M);
+          const float v = M + logf(S);
+          cv[j] = v;
+          if (ckpt && rank == 0) ckpt[(((size_t)blk * iters + k) * 2 + 1) * B + j] = v;
+        }
+        __syncthreads();
+      }
     }
-    __syncthreads();
-    float* bm = xm + (k & 1) * B;
-    float* bs = xs + (k & 1) * B;
-    for (int j = tid; j < B; j += NT) {
-      float mx = pm[j];
-      for (int g = 1; g < G; ++g) mx = fmaxf(mx, pm[g * B + j]);
-      float s = 0.f;
-      for (int g = 0; g < G; ++g) s += ps[g * B + j] * expf(pm[g * B + j] - mx);
-      bm[j] = mx;
-      bs[j] = s;
-    }
-    cluster_barrier<CS>();
-    if constexpr (CS == 1) __syncthreads();
-    for (int j = tid; j < B; j += NT) {
-      float mx = -CUDART_INF_F;
-      for (int q = 0; q < CS; ++q) mx = fmaxf(mx, peer<CS>(bm, q)[j]);
-      float s = 0.f;
-      for (int q = 0; q < CS; ++q) s += peer<CS>(bs, q)[j] * expf(peer<CS>(bm, q)[j] - mx);
-      const float v = mx + logf(s);
-      cv[j] = v;
-      if (ckpt && rank == 0) ckpt[(((size_t)blk * iters + k) * 2 + 1) * B + j] = v;
-    }
-    __syncthreads();
   }
 
-  // Operand images for the tensor-core kernels, in tiles of BC = max(B, 64)
-  // columns: tile t holds the BC x BC block-diagonal slice of P_B covering
-  // channels [t*BC, (t+1)*BC) (for B = 32 two blocks share one tile and the
-  // off-diagonal quadrants are written as zeros).
-  constexpr int BC = B < 64 ? 64 : B;
-  const int gcol0 = blk * B;
-  const size_t tbase = (size_t)(gcol0 / BC) * BC * BC;
-  const int q0 = gcol0 % BC;
-  const __nv_bfloat16 zero = __float2bfloat16_rn(0.f);
-  for (int e = tid; e < R * B; e += NT) {
-    const int r = e / B, j = e % B;
-    const float p = expf(z[e] - rv[r] - cv[j]);
-    const int i = row0 + r;
-    P[base + (size_t)i * B + j] = p;
-    if (pt_hi) {
+  // P = exp(Z_0 - R - C), staged through the tile for coalesced stores
+#pragma unroll
+  for (int e = 0; e < EPR; ++e) tile[r * LD + c + TPR * e] = expf(zr[e] - myR - cv[c + TPR * e]);
+  __syncthreads();
+  for (int q = tid; q < R * B; q += NT) {
+    const int rr = q / B, jj = q % B;
+    P[base + (size_t)(row0 + rr) * B + jj] = tile[rr * LD + jj];
+  }
+  if (pt_hi) {
+    // Operand images for the tensor-core kernels, in tiles of BC = max(B, 64)
+    // columns: tile t holds the BC x BC block-diagonal slice of P_B covering
+    // channels [t*BC, (t+1)*BC) (for B = 32 two blocks share one tile and the
+    // off-diagonal quadrants are written as zeros).
+    constexpr int BC = B < 64 ? 64 : B;
+    const int gcol0 = blk * B;
+    const size_t tb = (size_t)(gcol0 / BC) * BC * BC;
+    const int q0 = gcol0 % BC;
+    const __nv_bfloat16 zero = __float2bfloat16_rn(0.f);
+    // transposed images: consecutive threads take consecutive source rows i
+    for (int q = tid; q < R * B; q += NT) {
+      const int jj = q / R, rr = q % R, i = row0 + rr;
+      const float p = tile[rr * LD + jj];
       const __nv_bfloat16 hi = __float2bfloat16_rn(p);
-      const __nv_bfloat16 lo = __float2bfloat16_rn(p - __bfloat162float(hi));
-      pt_hi[tbase + (size_t)(q0 + j) * BC + q0 + i] = hi;
-      pt_lo[tbase + (size_t)(q0 + j) * BC + q0 + i] = lo;
-      p_hi[tbase + (size_t)(q0 + i) * BC + q0 + j] = hi;
+      pt_hi[tb + (size_t)(q0 + jj) * BC + q0 + i] = hi;
+      pt_lo[tb + (size_t)(q0 + jj) * BC + q0 + i] = __float2bfloat16_rn(p - __bfloat162float(hi));
       if constexpr (B < BC) {
-        const int zc = (q0 == 0) ? B : 0;
-        pt_hi[tbase + (size_t)(q0 + j) * BC + zc + i] = zero;
-        pt_lo[tbase + (size_t)(q0 + j) * BC + zc + i] = zero;
-        p_hi[tbase + (size_t)(q0 + i) * BC + zc + j] = zero;
+        const int zc0 = (q0 == 0) ? B : 0;
+        pt_hi[tb + (size_t)(q0 + jj) * BC + zc0 + i] = zero;
+        pt_lo[tb + (size_t)(q0 + jj) * BC + zc0 + i] = zero;
       }
+    }
+    for (int q = tid; q < R * B; q += NT) {
+      const int rr = q / B, jj = q % B, i = row0 + rr;
+      p_hi[tb + (size_t)(q0 + i) * BC + q0 + jj] = __float2bfloat16_rn(tile[rr * LD + jj]);
+      if constexpr (B < BC) p_hi[tb + (size_t)(q0 + i) * BC + ((q0 == 0) ? B : 0) + jj] = zero;
     }
   }
   // keep peers' shared memory alive until every CTA of the cluster is done reading it
   cluster_barrier<CS>();
 }
 
-// Reverse.  Shared memory (floats): z[R*B] d[R*B] rv[R] ck[B] ck1[B] pm[G*B] xs[2*B]
+// Reverse.  dZ lives in registers in the row layout.
+// Shared memory (floats): tile[R*(B+1)] ck[B] ck1[B] part[NW*B] cs[B] xs[2B]
 template <int B>
 __global__ void __launch_bounds__(SkCfg<B>::NT)
 sinkhorn_bwd_kernel(const float* __restrict__ L, const float* __restrict__ ckpt,
                     const float* __restrict__ dP, int splits, int nblocks,
                     float* __restrict__ dL, float tau, int iters) {
   using C = SkCfg<B>;
-  constexpr int R = C::R, G = C::G, NT = C::NT, NW = NT / 32, CS = C::CS;
+  constexpr int R = C::R, NT = C::NT, CS = C::CS, TPR = C::TPR, EPR = C::EPR, NW = C::NW, LD = C::LD;
+  constexpr int RPW = 32 / TPR;   // rows per warp
   extern __shared__ __align__(16) float sm[];
-  float* z = sm;
-  float* d = z + R * B;
-  float* rv = d + R * B;
-  float* ck = rv + R;      // C^(k)
-  float* ck1 = ck + B;     // C^(k-1)
-  float* pm = ck1 + B;
-  float* xs = pm + G * B;
+  float* tile = sm;
+  float* ck = tile + R * LD;   // C^(k+1)
+  float* ck1 = ck + B;         // C^(k)
+  float* part = ck1 + B;       // per-warp column partial sums
+  float* cs = part + NW * B;   // column sums of dZ
+  float* xs = cs + B;          // this CTA's column sums for the cluster, double-buffered
 
   const int rank = cta_rank<CS>();
   const int blk = blockIdx.x / CS;
@@ -194,73 +250,101 @@ sinkhorn_bwd_kernel(const float* __restrict__ L, const float* __restrict__ ckpt,
   const size_t base = (size_t)blk * B * B;
   const size_t split_stride = (size_t)nblocks * B * B;
   const float* ckb = ckpt + (size_t)blk * iters * 2 * B;
+  const int r = tid / TPR, c = tid % TPR;
 
-  for (int e = tid; e < R * B; e += NT) {
-    const size_t off = base + (size_t)row0 * B + e;
-    z[e] = L[off] / tau;
-    float g = dP[off];
-    for (int s = 1; s < splits; ++s) g += dP[(size_t)s * split_stride + off];
-    d[e] = g;
+  float zr[EPR], dz[EPR];
+  // Z_0 = L / tau
+  for (int q = tid; q < R * (B / 4); q += NT) {
+    const float4 v = reinterpret_cast<const float4*>(L + base + (size_t)row0 * B)[q];
+    const int rr = q / (B / 4), jj = (q % (B / 4)) * 4;
+    float* d = tile + rr * LD + jj;
+    d[0] = v.x / tau; d[1] = v.y / tau; d[2] = v.z / tau; d[3] = v.w / tau;
   }
-  for (int r = tid; r < R; r += NT) rv[r] = ckb[(size_t)(iters - 1) * 2 * B + row0 + r];
-  for (int j = tid; j < B; j += NT) ck[j] = ckb[(size_t)(iters - 1) * 2 * B + B + j];
   __syncthreads();
+#pragma unroll
+  for (int e = 0; e < EPR; ++e) zr[e] = tile[r * LD + c + TPR * e];
+  __syncthreads();
+  // dP summed over the splits in index order
+  for (int q = tid; q < R * (B / 4); q += NT) {
+    float4 a = reinterpret_cast<const float4*>(dP + base + (size_t)row0 * B)[q];
+    for (int s = 1; s < splits; ++s) {
+      const float4 b = reinterpret_cast<const float4*>(dP + (size_t)s * split_stride + base + (size_t)row0 * B)[q];
+      a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+    }
+    const int rr = q / (B / 4), jj = (q % (B / 4)) * 4;
+    float* d = tile + rr * LD + jj;
+    d[0] = a.x; d[1] = a.y; d[2] = a.z; d[3] = a.w;
+  }
+  for (int jj = tid; jj < B; jj += NT) ck[jj] = ckb[(size_t)(iters - 1) * 2 * B + B + jj];
+  __syncthreads();
+  float myR = ckb[(size_t)(iters - 1) * 2 * B + row0 + r];
   // dZ = dP (.) P with P = exp(z - R^(K) - C^(K))
-  for (int e = tid; e < R * B; e += NT) d[e] *= expf(z[e] - rv[e / B] - ck[e % B]);
-  __syncthreads();
+#pragma unroll
+  for (int e = 0; e < EPR; ++e) dz[e] = tile[r * LD + c + TPR * e] * expf(zr[e] - myR - ck[c + TPR * e]);
 
   for (int k = iters - 1; k >= 0; --k) {
-    // rv = R^(k+1), ck = C^(k+1), ck1 = C^(k) (zero before the first iteration)
-    for (int r = tid; r < R; r += NT) rv[r] = ckb[(size_t)k * 2 * B + row0 + r];
-    for (int j = tid; j < B; j += NT) {
-      ck[j] = ckb[(size_t)k * 2 * B + B + j];
-      ck1[j] = (k > 0) ? ckb[(size_t)(k - 1) * 2 * B + B + j] : 0.f;
+    __syncthreads();   // previous iteration done with ck, ck1, part, cs
+    for (int jj = tid; jj < B; jj += NT) {
+      ck[jj] = ckb[(size_t)k * 2 * B + B + jj];
+      ck1[jj] = (k > 0) ? ckb[(size_t)(k - 1) * 2 * B + B + jj] : 0.f;
     }
-    // column step: dZ -= exp(Z') * colsum(dZ), Z' = z - R^(k+1) - C^(k+1)
-    {
-      const int j = tid % B, g = tid / B;
-      float s = 0.f;
-      for (int r = g; r < R; r += G) s += d[r * B + j];
-      pm[g * B + j] = s;
+    myR = ckb[(size_t)k * 2 * B + row0 + r];
+    // column sums of dZ: over the rows of this warp (lanes with equal c), then over warps
+#pragma unroll
+    for (int e = 0; e < EPR; ++e) {
+      float v = dz[e];
+#pragma unroll
+      for (int o = TPR; o < 32; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if (lane < TPR) part[warp * B + c + TPR * e] = v;
     }
     __syncthreads();
     float* bs = xs + (k & 1) * B;
-    for (int j = tid; j < B; j += NT) {
+    for (int jj = tid; jj < B; jj += NT) {
       float s = 0.f;
-      for (int g = 0; g < G; ++g) s += pm[g * B + j];
-      bs[j] = s;
+      for (int w = 0; w < NW; ++w) s += part[w * B + jj];
+      if constexpr (CS == 1) cs[jj] = s;
+      else bs[jj] = s;
     }
-    cluster_barrier<CS>();
-    if constexpr (CS == 1) __syncthreads();
-    for (int e = tid; e < R * B; e += NT) {
-      const int r = e / B, j = e % B;
-      float cs = 0.f;
-      for (int q = 0; q < CS; ++q) cs += peer<CS>(bs, q)[j];
-      d[e] -= expf(z[e] - rv[r] - ck[j]) * cs;
+    if constexpr (CS > 1) {
+      cluster_barrier<CS>();
+      for (int jj = tid; jj < B; jj += NT) {
+        float s = 0.f;
+        for (int q = 0; q < CS; ++q) s += peer<CS>(bs, q)[jj];
+        cs[jj] = s;
+      }
     }
     __syncthreads();
-    // row step: dZ -= exp(Z') * rowsum(dZ), Z' = z - R^(k+1) - C^(k); one warp per row
-    for (int r = warp; r < R; r += NW) {
-      float* dr = d + r * B;
-      const float* zr = z + r * B;
-      float s = 0.f;
-      for (int j = lane; j < B; j += 32) s += dr[j];
-      s = warp_sum(s);
-      for (int j = lane; j < B; j += 32) dr[j] -= expf(zr[j] - rv[r] - ck1[j]) * s;
-    }
-    __syncthreads();
+    // column step: dZ -= exp(Z') colsum, Z' = z - R^(k+1) - C^(k+1)
+#pragma unroll
+    for (int e = 0; e < EPR; ++e) dz[e] -= expf(zr[e] - myR - ck[c + TPR * e]) * cs[c + TPR * e];
+    // row step: dZ -= exp(Z') rowsum, Z' = z - R^(k+1) - C^(k)
+    float rs = 0.f;
+#pragma unroll
+    for (int e = 0; e < EPR; ++e) rs += dz[e];
+    rs = group_sum<TPR>(rs);
+#pragma unroll
+    for (int e = 0; e < EPR; ++e) dz[e] -= expf(zr[e] - myR - ck1[c + TPR * e]) * rs;
   }
-  for (int e = tid; e < R * B; e += NT) dL[base + (size_t)row0 * B + e] = d[e] / tau;
+  // dL = dZ_0 / tau, staged for coalesced stores
+  __syncthreads();
+#pragma unroll
+  for (int e = 0; e < EPR; ++e) tile[r * LD + c + TPR * e] = dz[e] / tau;
+  __syncthreads();
+  for (int q = tid; q < R * B; q += NT) {
+    const int rr = q / B, jj = q % B;
+    dL[base + (size_t)(row0 + rr) * B + jj] = tile[rr * LD + jj];
+  }
   cluster_barrier<CS>();
+  (void)RPW;
 }
 
 template <int B> constexpr size_t fwd_smem() {
   using C = SkCfg<B>;
-  return sizeof(float) * (C::R * B + C::R + B + 2 * C::G * B + 4 * B);
+  return sizeof(float) * (C::R * C::LD + C::R + B + 4 * B);
 }
 template <int B> constexpr size_t bwd_smem() {
   using C = SkCfg<B>;
-  return sizeof(float) * (2 * C::R * B + C::R + 2 * B + C::G * B + 2 * B);
+  return sizeof(float) * (C::R * C::LD + 2 * B + C::NW * B + B + 2 * B);
 }
 
 template <typename K, typename... Args>
@@ -280,7 +364,7 @@ lcp_status launch_cluster(K kernel, int grid, int threads, size_t smem, int cs, 
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = cs > 1 ? 1 : 0;
   cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
   if (e != cudaSuccess) {
     cudaGetLastError();

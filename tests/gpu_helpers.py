@@ -54,6 +54,7 @@ def run_gpu(wl, inputs, flags=0, with_wp=True, L_override=None):
     s = b.Step(dev, wl.block, wl.n, wl.m, wl.iters, wl.tau, flags=f)
     s.run()
     torch.cuda.synchronize()
+    assert b.device_error() == 0, "a bounded wait inside a tensor-core kernel expired"
     out = []
     for d in dev:
         cout, cin = d["W"].shape
