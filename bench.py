@@ -361,7 +361,7 @@ def main():
                        "block": wl.block, "nm": f"{wl.n}:{wl.m}", "tau": wl.tau, "iters": wl.iters,
                        "parallelism": f"layer-sharded x{world}" if world > 1 else "single GPU",
                        "l2": "flushed between timed steps (256 MiB write)",
-                       "path": "tcgen05" if step.launches == 8 else "simt"},
+                       "path": "simt" if args.simt else "tcgen05"},
             "roofline": roof, "stages": per_stage, "clocks": clocks, "e2e": e2e,
             "gpu_launches": step.launches * K}
     if world == 1 and not args.no_cpu_baseline:

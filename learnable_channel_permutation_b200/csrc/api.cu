@@ -127,7 +127,7 @@ lcp_status check_layer(const lcp_layer& l, const lcp_hparams& hp, int idx) {
 size_t esize(lcp_dtype d) { return d == LCP_F32 ? 4 : 2; }
 
 struct Plan {
-  size_t ckpt, img0, img1, img2, mask, wp, amask, at, yd, ys, stats, g, dat, da, dp;
+  size_t ckpt, img0, img1, img2, mask, wp, amask, at, yd, ys, stats, counter, g, dat, da, dp;
   size_t total;
   int splits;
 };
@@ -159,6 +159,7 @@ Plan make_plan(const lcp_layer& l, const lcp_hparams& hp) {
   p.yd = take(T * oc * 4);
   p.ys = take(T * oc * 4);
   p.stats = take(T * 16);
+  p.counter = take(256);
   p.g = take(T * oc * es);
   p.dat = take(oc * ic * (tc ? 2 : 4));
   p.da = take(simt_bwd ? oc * ic * 4 : 0);
@@ -178,6 +179,16 @@ lcp_status validate_all(const lcp_layer* layers, int nlayers, const lcp_hparams*
 template <typename T> T* at(void* ws, size_t off) {
   return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
 }
+
+// Loss stage of a step: the fused one-launch kernel when a token row fits its
+// registers, else per-token statistics + gradient and a separate reduction.
+lcp_status launch_loss(const float* Yd, const float* Ys, float* stats, void* G, lcp_dtype gdt, float* loss,
+                       unsigned* counter, int cout, int tokens, cudaStream_t st) {
+  if (loss_fused_supported(cout)) return launch_loss_fused(Yd, Ys, stats, G, gdt, loss, counter, cout, tokens, st);
+  LCP_TRY(launch_loss_token(Yd, Ys, stats, G, gdt, cout, tokens, st));
+  return launch_loss_reduce(stats, loss, tokens, st);
+}
+int loss_launches(int cout) { return loss_fused_supported(cout) ? 1 : 2; }
 
 lcp_status record(cudaEvent_t* ev, int k, cudaStream_t st) {
   if (!ev) return LCP_OK;
@@ -223,8 +234,7 @@ lcp_status layer_simt(const lcp_layer& l, const lcp_hparams& hp, const Plan& p, 
   LCP_TRY(launch_simt_gemm({l.tokens, l.cout, l.cin, 1, l.X, 0, ic, 1, At, 0, 1, ic, Ys, 0, oc, 1, 1.f, 0.f},
                            dt, dt, LCP_F32, st));
   LCP_TRY(record(ev, 3, st));
-  LCP_TRY(launch_loss_token(Yd, Ys, stats, G, dt, l.cout, l.tokens, st));
-  LCP_TRY(launch_loss_reduce(stats, l.loss, l.tokens, st));
+  LCP_TRY(launch_loss(Yd, Ys, stats, G, dt, l.loss, at<unsigned>(ws, p.counter), l.cout, l.tokens, st));
   LCP_TRY(record(ev, 4, st));
   // dAt = G^T X   ([C_out, C_in], K = T)
   LCP_TRY(launch_simt_gemm({l.cout, l.cin, l.tokens, 1, G, 0, 1, oc, l.X, 0, ic, 1, dAt, 0, ic, 1, 1.f, 0.f},
@@ -244,13 +254,15 @@ lcp_status layer_simt(const lcp_layer& l, const lcp_hparams& hp, const Plan& p, 
   return LCP_OK;
 }
 
-constexpr int kSimtLaunches = 15;
-constexpr int kTcLaunches = 8;
-constexpr int kTcLaunchesSimtBwd = 13;   // B = 256: block backward on CUDA cores (6 launches)
+// kernel launches per layer, not counting the loss stage (1 or 2 launches)
+constexpr int kSimtLaunches = 13;
+constexpr int kTcLaunches = 6;
+constexpr int kTcLaunchesSimtBwd = 11;   // B = 256: block backward on CUDA cores (6 launches)
 
-int launches_per_layer(const lcp_hparams& hp) {
-  if (!use_tc(hp)) return kSimtLaunches;
-  return block_bwd_tc_supported(hp.block) ? kTcLaunches : kTcLaunchesSimtBwd;
+int launches_per_layer(const lcp_layer& l, const lcp_hparams& hp) {
+  const int loss = loss_launches(l.cout);
+  if (!use_tc(hp)) return kSimtLaunches + loss;
+  return (block_bwd_tc_supported(hp.block) ? kTcLaunches : kTcLaunchesSimtBwd) + loss;
 }
 
 // ---- one layer, tensor-core path (bf16 operands, float32 accumulation) -----
@@ -280,8 +292,7 @@ lcp_status layer_tc(const lcp_layer& l, const lcp_hparams& hp, const Plan& p, vo
   LCP_TRY(record(ev, 2, st));
   LCP_TRY(launch_calib_gemm_tc(X, W, At, Yd, Ys, l.tokens, l.cout, l.cin, st));
   LCP_TRY(record(ev, 3, st));
-  LCP_TRY(launch_loss_token(Yd, Ys, stats, G, LCP_BF16, l.cout, l.tokens, st));
-  LCP_TRY(launch_loss_reduce(stats, l.loss, l.tokens, st));
+  LCP_TRY(launch_loss(Yd, Ys, stats, G, LCP_BF16, l.loss, at<unsigned>(ws, p.counter), l.cout, l.tokens, st));
   LCP_TRY(record(ev, 4, st));
   LCP_TRY(launch_bwd_gemm_tc(G, X, dAt, l.tokens, l.cout, l.cin, st));
   LCP_TRY(record(ev, 5, st));
@@ -374,7 +385,9 @@ lcp_status lcp_step_launches(const lcp_layer* layers, int nlayers, const lcp_hpa
                              int* launches) {
   if (!launches) return fail(LCP_ERR_NULL, "launches is NULL");
   LCP_TRY(validate_all(layers, nlayers, hp));
-  *launches = nlayers * launches_per_layer(*hp);
+  int n = 0;
+  for (int i = 0; i < nlayers; ++i) n += launches_per_layer(layers[i], *hp);
+  *launches = n;
   return LCP_OK;
 }
 

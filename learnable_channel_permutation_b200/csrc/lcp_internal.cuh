@@ -64,6 +64,10 @@ lcp_status launch_loss_token(const float* Yd, const float* Ys, float* stats, voi
 lcp_status launch_loss_grad(const float* Yd, const float* Ys, const float* stats, void* G,
                             lcp_dtype gdt, int cout, int tokens, cudaStream_t st);
 lcp_status launch_loss_reduce(const float* stats, float* loss, int tokens, cudaStream_t st);
+// One launch (plus a 4-byte counter reset): stats, G and the loss.  cout <= 16384.
+bool loss_fused_supported(int cout);
+lcp_status launch_loss_fused(const float* Yd, const float* Ys, float* stats, void* G, lcp_dtype gdt,
+                             float* loss, unsigned* counter, int cout, int tokens, cudaStream_t st);
 
 // Tensor-core (tcgen05) kernels, bf16 operands, float32 accumulation.
 bool tc_available();

@@ -106,6 +106,90 @@ loss_grad_kernel(const float* __restrict__ Yd, const float* __restrict__ Ys,
                  G, row, cout / 4, s.x, s.y, s.z, inv_T);
 }
 
+// Fused variant used inside a step: one CTA per token keeps the token's two
+// rows in registers (QPT float4 quads per thread), so Y is read from HBM once;
+// the CTA that finishes last (a counter that the caller zeroes before the
+// launch) sums the T cosines in index order into the loss and re-zeroes the
+// counter.  Deterministic: the order of the final sum never depends on timing.
+template <typename TG, int NTH, int QPT>
+__global__ void __launch_bounds__(NTH)
+loss_fused_kernel(const float* __restrict__ Yd, const float* __restrict__ Ys, float* __restrict__ stats,
+                  TG* __restrict__ G, float* __restrict__ loss, unsigned* __restrict__ counter, int cout,
+                  int tokens, float inv_T) {
+  constexpr int NWARP = NTH / 32;
+  __shared__ float red[3][NWARP];
+  __shared__ double redd[NWARP];
+  __shared__ int is_last;
+  const int t = blockIdx.x;
+  const size_t row = (size_t)t * cout;
+  const float4* yd = reinterpret_cast<const float4*>(Yd + row);
+  const float4* ys = reinterpret_cast<const float4*>(Ys + row);
+  const int quads = cout / 4;
+  float4 a[QPT], b[QPT];
+#pragma unroll
+  for (int i = 0; i < QPT; ++i) {
+    const int q = threadIdx.x + i * NTH;
+    if (q < quads) { a[i] = yd[q]; b[i] = ys[q]; }
+    else { a[i] = make_float4(0.f, 0.f, 0.f, 0.f); b[i] = a[i]; }
+  }
+  float dot = 0.f, nd = 0.f, ns = 0.f;
+#pragma unroll
+  for (int i = 0; i < QPT; ++i) {
+    dot += a[i].x * b[i].x + a[i].y * b[i].y + a[i].z * b[i].z + a[i].w * b[i].w;
+    nd += a[i].x * a[i].x + a[i].y * a[i].y + a[i].z * a[i].z + a[i].w * a[i].w;
+    ns += b[i].x * b[i].x + b[i].y * b[i].y + b[i].z * b[i].z + b[i].w * b[i].w;
+  }
+  dot = warp_sum(dot);
+  nd = warp_sum(nd);
+  ns = warp_sum(ns);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  if (lane == 0) { red[0][warp] = dot; red[1][warp] = nd; red[2][warp] = ns; }
+  __syncthreads();
+  dot = 0.f; nd = 0.f; ns = 0.f;
+#pragma unroll
+  for (int w = 0; w < NWARP; ++w) { dot += red[0][w]; nd += red[1][w]; ns += red[2][w]; }
+  const float den = sqrtf(nd) * sqrtf(ns);
+  const float c = dot / fmaxf(den, kCosEps);
+  if (threadIdx.x == 0) {
+    float4 sv;
+    sv.x = dot; sv.y = nd; sv.z = ns; sv.w = c;
+    reinterpret_cast<float4*>(stats)[t] = sv;
+  }
+  const bool ok = den > kCosEps;
+  const float ca = ok ? -inv_T / den : -inv_T / kCosEps;
+  const float cb = ok ? inv_T * c / ns : 0.f;
+#pragma unroll
+  for (int i = 0; i < QPT; ++i) {
+    const int q = threadIdx.x + i * NTH;
+    if (q < quads) {
+      float4 g;
+      g.x = ca * a[i].x + cb * b[i].x;
+      g.y = ca * a[i].y + cb * b[i].y;
+      g.z = ca * a[i].z + cb * b[i].z;
+      g.w = ca * a[i].w + cb * b[i].w;
+      write_g<TG>(G, row + 4 * (size_t)q, g);
+    }
+  }
+  // last CTA: the loss
+  __threadfence();
+  if (threadIdx.x == 0) is_last = (atomicAdd(counter, 1u) == (unsigned)tokens - 1u);
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  double sum = 0.0;
+  for (int u = threadIdx.x; u < tokens; u += NTH) sum += 1.0 - (double)__ldcg(stats + 4 * (size_t)u + 3);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if (lane == 0) redd[warp] = sum;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double tot = 0.0;
+    for (int w = 0; w < NWARP; ++w) tot += redd[w];
+    *loss = (float)(tot / tokens);
+    *counter = 0u;
+  }
+}
+
 __global__ void __launch_bounds__(1024)
 loss_reduce_kernel(const float* __restrict__ stats, float* __restrict__ loss, int tokens) {
   __shared__ double red[32];
@@ -146,6 +230,33 @@ lcp_status launch_loss_grad(const float* Yd, const float* Ys, const float* stats
   else
     loss_grad_kernel<__nv_bfloat16><<<tokens, NT, 0, st>>>(Yd, Ys, stats, (__nv_bfloat16*)G, cout, inv_T);
   return check_launch("loss_grad");
+}
+
+bool loss_fused_supported(int cout) { return cout <= 8 * 4 * 512; }
+
+lcp_status launch_loss_fused(const float* Yd, const float* Ys, float* stats, void* G, lcp_dtype gdt,
+                             float* loss, unsigned* counter, int cout, int tokens, cudaStream_t st) {
+  const float inv_T = 1.0f / (float)tokens;
+  const cudaError_t e = cudaMemsetAsync(counter, 0, sizeof(unsigned), st);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(LCP_ERR_CUDA, "loss counter reset: %s", cudaGetErrorString(e));
+  }
+  const int quads = cout / 4;
+#define LCP_LOSS_FUSED(TG, NTH, QPT)                                                                  \
+  loss_fused_kernel<TG, NTH, QPT><<<tokens, NTH, 0, st>>>(Yd, Ys, stats, static_cast<TG*>(G), loss,   \
+                                                           counter, cout, tokens, inv_T)
+  if (gdt == LCP_F32) {
+    if (quads <= 4 * 256) LCP_LOSS_FUSED(float, 256, 4);
+    else if (quads <= 8 * 256) LCP_LOSS_FUSED(float, 256, 8);
+    else LCP_LOSS_FUSED(float, 512, 8);
+  } else {
+    if (quads <= 4 * 256) LCP_LOSS_FUSED(__nv_bfloat16, 256, 4);
+    else if (quads <= 8 * 256) LCP_LOSS_FUSED(__nv_bfloat16, 256, 8);
+    else LCP_LOSS_FUSED(__nv_bfloat16, 512, 8);
+  }
+#undef LCP_LOSS_FUSED
+  return check_launch("loss_fused");
 }
 
 lcp_status launch_loss_reduce(const float* stats, float* loss, int tokens, cudaStream_t st) {
