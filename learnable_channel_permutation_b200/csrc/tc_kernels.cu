@@ -108,6 +108,35 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
       : "memory");
 }
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// at most N committed bulk groups still reading shared memory
+template <int N> __device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// barrier over `n` threads on named barrier `id` that also ANDs a predicate
+__device__ __forceinline__ bool named_and(int id, int n, bool v) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(out)
+      : "r"(v ? 1u : 0u), "r"(id), "r"(n)
+      : "memory");
+  return out != 0;
+}
+__device__ __forceinline__ void named_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
 __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -579,6 +608,197 @@ permute_mask_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
   }
 }
 
+// ------------------------------------- permute + mask, warp-specialised ---
+// BC = 64 (B = 32 or 64).  Persistent CTAs walk a flat list of (channel tile,
+// row tile) pairs.  Warp 0 streams each tile's W block together with its P
+// images into a 3-stage ring; warp 1 issues W' = W (P_hi + P_lo) into one of
+// two TMEM buffers and, once the epilogue has written A = M.W' to shared
+// memory, At = A P_hi into the same buffer; warps 2-9 (two per TMEM lane
+// quadrant, 32 columns each) compute the mask, write A, and copy At out
+// through a swizzled staging tile with TMA stores.
+struct PwCfg {
+  static constexpr int STAGES = 3;
+  static constexpr int W_BYTES = 16384;                 // 128 rows x 64 bf16
+  static constexpr int IMG_BYTES = 8192;                // 64 x 64 bf16
+  static constexpr int STAGE = W_BYTES + 3 * IMG_BYTES; // W | Pt_hi | Pt_lo | P_hi
+  static constexpr int A_BYTES = 16384;
+  static constexpr int SMEM = STAGES * STAGE + 2 * A_BYTES + 2 * A_BYTES + 1024 + 256;
+  static constexpr int THREADS = 320;
+  static constexpr int EPI = 256;                        // epilogue threads (warps 2..9)
+};
+
+template <int MGROUP>
+__global__ void __launch_bounds__(PwCfg::THREADS, 1)
+permute_mask_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmPth,
+                       const __grid_constant__ CUtensorMap tmPtl, const __grid_constant__ CUtensorMap tmPh,
+                       const __grid_constant__ CUtensorMap tmAt, uint32_t* __restrict__ mask,
+                       float* __restrict__ Wp_out, int cout, int cin, int n) {
+  using C = PwCfg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sStage = smem;
+  uint8_t* sA = smem + C::STAGES * C::STAGE;          // 2 buffers
+  uint8_t* sO = sA + 2 * C::A_BYTES;                  // 2 staging tiles for At
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sO + 2 * C::A_BYTES);
+  // bars: full[3] empty[3] wf[2] af[2] atf[2] tme[2] drain
+  uint32_t* holder = reinterpret_cast<uint32_t*>(bars + 15);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(holder + 1);
+  auto bar = [&](int i) { return smem_u32(bars + i); };
+  const int FULL = 0, EMPTY = 3, WF = 6, AF = 8, ATF = 10, TME = 12, DRAIN = 14;
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int nrt = cdiv(cout, 128), ntc = cin / 64;
+  const int total = nrt * ntc;
+  const int words = cin / 32;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 3; ++i) { mbar_init(bar(FULL + i), 1); mbar_init(bar(EMPTY + i), 1); }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(WF + i), 1);
+      mbar_init(bar(AF + i), 8);
+      mbar_init(bar(ATF + i), 1);
+      mbar_init(bar(TME + i), 8);
+    }
+    mbar_init(bar(DRAIN), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(smem_u32(holder), 256);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *holder;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int k = 0;
+      uint32_t issued = 0, par = 0;   // per stage: outstanding load and its parity
+      for (int idx = blockIdx.x; idx < total; idx += gridDim.x, ++k) {
+        const int st = k % C::STAGES;
+        const uint32_t use = (uint32_t)(k / C::STAGES) & 1u;
+        if (!mbar_wait(bar(EMPTY + st), use ^ 1u, abort_flag, 61)) break;
+        const int t = idx / nrt, rt = idx % nrt;
+        uint8_t* sg = sStage + st * C::STAGE;
+        mbar_expect_tx(bar(FULL + st), C::STAGE);
+        tma_load_2d(smem_u32(sg), &tmW, bar(FULL + st), t * 64, rt * 128);
+        tma_load_2d(smem_u32(sg + C::W_BYTES), &tmPth, bar(FULL + st), 0, t * 64);
+        tma_load_2d(smem_u32(sg + C::W_BYTES + C::IMG_BYTES), &tmPtl, bar(FULL + st), 0, t * 64);
+        tma_load_2d(smem_u32(sg + C::W_BYTES + 2 * C::IMG_BYTES), &tmPh, bar(FULL + st), 0, t * 64);
+        issued |= 1u << st;
+        par = (par & ~(1u << st)) | (use << st);
+      }
+      for (int st = 0; st < C::STAGES; ++st)
+        if (issued & (1u << st)) mbar_wait_drain(bar(FULL + st), (par >> st) & 1u, 62);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(128, 64, false, false);
+      int k = 0;
+      for (int idx = blockIdx.x; idx < total; idx += gridDim.x, ++k) {
+        const int st = k % C::STAGES, a = k & 1;
+        const uint32_t use = (uint32_t)(k / C::STAGES) & 1u, ua = (uint32_t)(k >> 1) & 1u;
+        if (!mbar_wait(bar(FULL + st), use, abort_flag, 63)) break;
+        if (!mbar_wait(bar(TME + a), ua ^ 1u, abort_flag, 64)) break;
+        tc_fence_after();
+        const uint32_t sg = smem_u32(sStage + st * C::STAGE);
+        const uint32_t dW = tmem + a * 128, dAt = tmem + a * 128 + 64;
+#pragma unroll
+        for (int k16 = 0; k16 < 4; ++k16) {
+          const uint64_t ad = sdesc(sg + k16 * 32, 16, 1024);
+          mma_bf16(dW, ad, sdesc(sg + C::W_BYTES + k16 * 32, 16, 1024), idesc, k16 != 0);
+          mma_bf16(dW, ad, sdesc(sg + C::W_BYTES + C::IMG_BYTES + k16 * 32, 16, 1024), idesc, true);
+        }
+        mma_commit(bar(WF + a));
+        if (!mbar_wait(bar(AF + a), ua, abort_flag, 65)) break;
+        tc_fence_after();
+        const uint32_t sa = smem_u32(sA + a * C::A_BYTES);
+#pragma unroll
+        for (int k16 = 0; k16 < 4; ++k16)
+          mma_bf16(dAt, sdesc(sa + k16 * 32, 16, 1024), sdesc(sg + C::W_BYTES + 2 * C::IMG_BYTES + k16 * 32, 16, 1024),
+                   idesc, k16 != 0);
+        mma_commit(bar(ATF + a));
+        mma_commit(bar(EMPTY + st));
+      }
+      mma_commit(bar(DRAIN));
+      mbar_wait_drain(bar(DRAIN), 0, 66);
+    }
+    __syncwarp();
+  } else {
+    const int e = warp - 2, q = warp & 3, h = e >> 2;
+    const int row = q * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    const bool leader = (e == 0 && lane == 0);
+    int k = 0;
+    for (int idx = blockIdx.x; idx < total; idx += gridDim.x, ++k) {
+      const int a = k & 1;
+      const uint32_t ua = (uint32_t)(k >> 1) & 1u;
+      const int t = idx / nrt, rt = idx % nrt;
+      const int grow = rt * 128 + row;
+      if (!named_and(1, C::EPI, mbar_wait(bar(WF + a), ua, abort_flag, 67))) break;
+      tc_fence_after();
+      uint32_t v[32];
+      tmem_ld32(tmem + lane_off + a * 128 + h * 32, v);
+      tmem_ld_wait();
+      const uint32_t w = nm_word<MGROUP>(v, n);
+      if (grow < cout) {
+        mask[(size_t)grow * words + 2 * t + h] = w;
+        if (Wp_out) {
+          float4* o = reinterpret_cast<float4*>(Wp_out + (size_t)grow * cin + t * 64 + h * 32);
+#pragma unroll
+          for (int qq = 0; qq < 8; ++qq)
+            o[qq] = make_float4(__uint_as_float(v[4 * qq]), __uint_as_float(v[4 * qq + 1]),
+                                __uint_as_float(v[4 * qq + 2]), __uint_as_float(v[4 * qq + 3]));
+        }
+      }
+      uint8_t* sa = sA + a * C::A_BYTES;
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4) {
+        float f[8];
+#pragma unroll
+        for (int x = 0; x < 8; ++x) f[x] = ((w >> (8 * c4 + x)) & 1u) ? __uint_as_float(v[8 * c4 + x]) : 0.f;
+        st_sw128(sa, row, h * 4 + c4, make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                                                 pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7])));
+      }
+      fence_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(AF + a));
+      // At of this tile
+      const bool got = mbar_wait(bar(ATF + a), ua, abort_flag, 68);
+      // the staging tile of two tiles ago must have been read out by its TMA store
+      if (leader) bulk_wait_read<1>();
+      if (!named_and(1, C::EPI, got)) break;
+      tc_fence_after();
+      tmem_ld32(tmem + lane_off + a * 128 + 64 + h * 32, v);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(TME + a));
+      uint8_t* so = sO + a * C::A_BYTES;
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4)
+        st_sw128(so, row, h * 4 + c4,
+                 make_uint4(pack_bf16x2(__uint_as_float(v[8 * c4 + 0]), __uint_as_float(v[8 * c4 + 1])),
+                            pack_bf16x2(__uint_as_float(v[8 * c4 + 2]), __uint_as_float(v[8 * c4 + 3])),
+                            pack_bf16x2(__uint_as_float(v[8 * c4 + 4]), __uint_as_float(v[8 * c4 + 5])),
+                            pack_bf16x2(__uint_as_float(v[8 * c4 + 6]), __uint_as_float(v[8 * c4 + 7]))));
+      fence_async_smem();
+      named_sync(1, C::EPI);
+      if (leader) {
+        tma_store_2d(&tmAt, smem_u32(so), t * 64, rt * 128);
+        bulk_commit();
+      }
+    }
+    if (leader) bulk_wait_all();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
 // ----------------------------------------- permute + mask, row-streamed ---
 // For BC <= 128 the P images of the CTA's channel tile stay resident and the
 // CTA walks the row tiles rt = blockIdx.y, blockIdx.y + gridDim.y, ...; the W
@@ -780,6 +1000,223 @@ permute_mask_tc2_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_co
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// ---------------------------------------- block backward, warp-specialised ---
+// BC = 64 (B = 32 or 64).  One CTA per (channel tile, row segment).  Warp 0
+// streams the (dAt, W) tiles of each 128-row chunk into a 3-stage ring; warp 1
+// issues W' = W (P_hi + P_lo) and dA = dAt P_hi into one of two TMEM buffers,
+// then, once the epilogue has written A = M.W' and dW' = M.dA, the stacked
+// dP product; warps 2-9 (two per TMEM lane quadrant, 32 columns each) turn
+// W', dA and the mask into the bf16 operands.  The dP accumulator stays in
+// TMEM for the whole segment and is written once at the end.
+struct BwCfg {
+  static constexpr int STAGES = 3;
+  static constexpr int T_BYTES = 16384;                  // 128 rows x 64 bf16
+  static constexpr int STAGE = 2 * T_BYTES;              // dAt | W (adjacent: stacked A operand)
+  static constexpr int IMG_BYTES = 8192;
+  static constexpr int SMEM = STAGES * STAGE + 2 * IMG_BYTES + 2 * (2 * T_BYTES) + 1024 + 256;
+  static constexpr int THREADS = 320;
+  static constexpr int EPI = 256;
+};
+
+template <int B>
+__global__ void __launch_bounds__(BwCfg::THREADS, 1)
+block_bwd_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmDAt,
+                    const __grid_constant__ CUtensorMap tmPth, const __grid_constant__ CUtensorMap tmPtl,
+                    const uint32_t* __restrict__ mask, float* __restrict__ dP, int cout, int cin,
+                    int rows_per_split) {
+  using C = BwCfg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sStage = smem;
+  uint8_t* sPth = smem + C::STAGES * C::STAGE;
+  uint8_t* sPtl = sPth + C::IMG_BYTES;
+  uint8_t* sAB = sPtl + C::IMG_BYTES;      // buffer a at + a * 2 * T_BYTES: A | dW' (adjacent)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sAB + 2 * 2 * C::T_BYTES);
+  // bars: full[3] empty[3] wd[2] abf[2] abe[2] dpf drain img
+  uint32_t* holder = reinterpret_cast<uint32_t*>(bars + 16);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(holder + 1);
+  auto bar = [&](int i) { return smem_u32(bars + i); };
+  const int FULL = 0, EMPTY = 3, WD = 6, ABF = 8, ABE = 10, DPF = 12, DRAIN = 13, IMG = 14;
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int t = blockIdx.x, sidx = blockIdx.y, col0 = t * 64;
+  const int rbeg = sidx * rows_per_split;
+  const int rend = min(cout, rbeg + rows_per_split);
+  const int nchunk = cdiv(rend - rbeg, 128);
+  const int words = cin / 32;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 3; ++i) { mbar_init(bar(FULL + i), 1); mbar_init(bar(EMPTY + i), 1); }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(WD + i), 1);
+      mbar_init(bar(ABF + i), 8);
+      mbar_init(bar(ABE + i), 1);
+    }
+    mbar_init(bar(DPF), 1);
+    mbar_init(bar(DRAIN), 1);
+    mbar_init(bar(IMG), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(smem_u32(holder), 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *holder;
+  const uint32_t tDP = tmem + 256;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      bool img_ok = true;
+      if (nchunk > 0) {
+        mbar_expect_tx(bar(IMG), 2 * C::IMG_BYTES);
+        tma_load_2d(smem_u32(sPth), &tmPth, bar(IMG), 0, col0);
+        tma_load_2d(smem_u32(sPtl), &tmPtl, bar(IMG), 0, col0);
+      }
+      uint32_t issued = 0, par = 0;
+      for (int c = 0; c < nchunk; ++c) {
+        const int st = c % C::STAGES;
+        const uint32_t use = (uint32_t)(c / C::STAGES) & 1u;
+        if (!mbar_wait(bar(EMPTY + st), use ^ 1u, abort_flag, 71)) break;
+        uint8_t* sg = sStage + st * C::STAGE;
+        const int r0 = rbeg + c * 128;
+        mbar_expect_tx(bar(FULL + st), C::STAGE);
+        tma_load_2d(smem_u32(sg), &tmDAt, bar(FULL + st), col0, r0);
+        tma_load_2d(smem_u32(sg + C::T_BYTES), &tmW, bar(FULL + st), col0, r0);
+        issued |= 1u << st;
+        par = (par & ~(1u << st)) | (use << st);
+      }
+      for (int st = 0; st < C::STAGES; ++st)
+        if (issued & (1u << st)) mbar_wait_drain(bar(FULL + st), (par >> st) & 1u, 72);
+      if (nchunk > 0) img_ok = mbar_wait_drain(bar(IMG), 0, 73);
+      (void)img_ok;
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc_n = idesc_bf16(128, 64, false, false);
+      constexpr uint32_t idesc_dp = idesc_bf16(128, 128, true, true);
+      bool ok = nchunk == 0 || mbar_wait(bar(IMG), 0, abort_flag, 74);
+      for (int c = 0; c < nchunk && ok; ++c) {
+        const int st = c % C::STAGES, a = c & 1;
+        const uint32_t use = (uint32_t)(c / C::STAGES) & 1u, ua = (uint32_t)(c >> 1) & 1u;
+        if (!mbar_wait(bar(FULL + st), use, abort_flag, 75)) break;
+        // the epilogue has read buffer a of chunk c - 2 (it arrived on ABF after its loads)
+        if (c >= 2 && !mbar_wait(bar(ABF + a), ua ^ 1u, abort_flag, 76)) break;
+        tc_fence_after();
+        const uint32_t sg = smem_u32(sStage + st * C::STAGE);
+        const uint32_t tW = tmem + a * 128, tDA = tmem + a * 128 + 64;
+#pragma unroll
+        for (int k16 = 0; k16 < 4; ++k16) {
+          const uint64_t wdesc = sdesc(sg + C::T_BYTES + k16 * 32, 16, 1024);
+          mma_bf16(tW, wdesc, sdesc(smem_u32(sPth) + k16 * 32, 16, 1024), idesc_n, k16 != 0);
+          mma_bf16(tW, wdesc, sdesc(smem_u32(sPtl) + k16 * 32, 16, 1024), idesc_n, true);
+          mma_bf16(tDA, sdesc(sg + k16 * 32, 16, 1024), sdesc(smem_u32(sPth) + k16 * 32, 16, 1024), idesc_n,
+                   k16 != 0);
+        }
+        mma_commit(bar(WD + a));
+        if (!mbar_wait(bar(ABF + a), ua, abort_flag, 77)) break;
+        tc_fence_after();
+        const uint32_t sab = smem_u32(sAB + a * 2 * C::T_BYTES);
+        // stacked: A operand [dAt | W] (M = 128), B operand [A | dW'] (N = 128), LBO = 16 KB
+#pragma unroll
+        for (int k16 = 0; k16 < 8; ++k16)
+          mma_bf16(tDP, sdesc(sg + k16 * 2048, 16384, 1024), sdesc(sab + k16 * 2048, 16384, 1024), idesc_dp,
+                   (c | k16) != 0);
+        mma_commit(bar(ABE + a));
+        mma_commit(bar(EMPTY + st));
+      }
+      mma_commit(bar(DPF));
+      mma_commit(bar(DRAIN));
+      mbar_wait_drain(bar(DRAIN), 0, 78);
+    }
+    __syncwarp();
+  } else {
+    const int e = warp - 2, q = warp & 3, h = e >> 2;
+    const int row = q * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    bool ok = true;
+    for (int c = 0; c < nchunk; ++c) {
+      const int a = c & 1;
+      const uint32_t ua = (uint32_t)(c >> 1) & 1u;
+      const int grow = rbeg + c * 128 + row;
+      ok = named_and(1, C::EPI, mbar_wait(bar(WD + a), ua, abort_flag, 79));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t wv[32], dv[32];
+      tmem_ld32(tmem + lane_off + a * 128 + h * 32, wv);
+      tmem_ld32(tmem + lane_off + a * 128 + 64 + h * 32, dv);
+      tmem_ld_wait();
+      const uint32_t bits = grow < rend ? __ldg(mask + (size_t)grow * words + col0 / 32 + h) : 0u;
+      // buffer a was last read by the dP product of chunk c - 2
+      ok = named_and(1, C::EPI, c < 2 || mbar_wait(bar(ABE + a), ua ^ 1u, abort_flag, 80));
+      if (!ok) break;
+      uint8_t* rA = sAB + a * 2 * C::T_BYTES;
+      uint8_t* rD = rA + C::T_BYTES;
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4) {
+        float fa[8], fd[8];
+#pragma unroll
+        for (int x = 0; x < 8; ++x) {
+          const bool keep = (bits >> (8 * c4 + x)) & 1u;
+          fa[x] = keep ? __uint_as_float(wv[8 * c4 + x]) : 0.f;
+          fd[x] = keep ? __uint_as_float(dv[8 * c4 + x]) : 0.f;
+        }
+        st_sw128(rA, row, h * 4 + c4, make_uint4(pack_bf16x2(fa[0], fa[1]), pack_bf16x2(fa[2], fa[3]),
+                                                 pack_bf16x2(fa[4], fa[5]), pack_bf16x2(fa[6], fa[7])));
+        st_sw128(rD, row, h * 4 + c4, make_uint4(pack_bf16x2(fd[0], fd[1]), pack_bf16x2(fd[2], fd[3]),
+                                                 pack_bf16x2(fd[4], fd[5]), pack_bf16x2(fd[6], fd[7])));
+      }
+      fence_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(ABF + a));
+    }
+    if (ok) ok = named_and(1, C::EPI, mbar_wait(bar(DPF), 0, abort_flag, 81));
+    if (ok) {
+      tc_fence_after();
+      // rows 0..63 hold dAt^T A (columns 0..63), rows 64..127 W^T dW' (columns 64..127)
+      uint32_t v[32];
+      const uint32_t cbase = (row < 64 ? 0u : 64u) + h * 32;
+      tmem_ld32(tDP + lane_off + cbase, v);
+      tmem_ld_wait();
+      float* scratch = reinterpret_cast<float*>(sAB);   // 64 x 64 floats; every MMA is done
+      if (row >= 64) {
+#pragma unroll
+        for (int x = 0; x < 32; ++x) scratch[(row - 64) * 64 + h * 32 + x] = __uint_as_float(v[x]);
+      }
+      named_sync(1, C::EPI);
+      if (row < 64) {
+        const int nb = cin / B;
+        float* dPs = dP + (size_t)sidx * nb * B * B;
+        const float* add = scratch + row * 64 + h * 32;
+        if constexpr (B == 64) {
+          float4* o = reinterpret_cast<float4*>(dPs + ((size_t)t * 64 + row) * 64 + h * 32);
+#pragma unroll
+          for (int qq = 0; qq < 8; ++qq)
+            o[qq] = make_float4(__uint_as_float(v[4 * qq]) + add[4 * qq], __uint_as_float(v[4 * qq + 1]) + add[4 * qq + 1],
+                                __uint_as_float(v[4 * qq + 2]) + add[4 * qq + 2],
+                                __uint_as_float(v[4 * qq + 3]) + add[4 * qq + 3]);
+        } else {
+          // B = 32: the tile holds blocks 2t (rows/columns 0..31) and 2t+1 (32..63);
+          // keep only the diagonal quadrants
+          const int qb = row / 32;
+          if (h == qb) {
+            float* o = dPs + ((size_t)(2 * t + qb) * 32 + (row - 32 * qb)) * 32;
+#pragma unroll
+            for (int x = 0; x < 32; ++x) o[x] = __uint_as_float(v[x]) + add[x];
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -1330,8 +1767,8 @@ int bb_rows_per_split(int cout, int cin, int B) {
   const int BC = B < 64 ? 64 : B;
   const int tiles = cin / BC;
   const int chunks = cdiv(cout, 128);
-  const int target = (BC == 64 ? 2 : 1) * 148;
-  int S = (target + tiles - 1) / tiles;
+  // one CTA per SM: as many row segments per channel tile as fill the SMs once
+  int S = 148 / tiles;
   if (S < 1) S = 1;
   if (S > 64) S = 64;
   if (S > chunks) S = chunks;
@@ -1387,6 +1824,19 @@ lcp_status launch_permute_mask_tc(const __nv_bfloat16* W, const __nv_bfloat16* i
   TC_TRY(make_map(&mPth, img_pt_hi, BC, cin, 64, 64, "permute_mask Pt_hi"));
   TC_TRY(make_map(&mPtl, img_pt_lo, BC, cin, 64, 64, "permute_mask Pt_lo"));
   TC_TRY(make_map(&mPh, img_p_hi, BC, cin, 64, BC, "permute_mask P_hi"));
+  if (BC == 64) {
+    CUtensorMap mAt, mPth64, mPtl64, mPh64;
+    TC_TRY(make_map(&mAt, At, cin, cout, 64, 128, "permute_mask At"));
+    TC_TRY(make_map(&mPth64, img_pt_hi, 64, cin, 64, 64, "permute_mask Pt_hi"));
+    TC_TRY(make_map(&mPtl64, img_pt_lo, 64, cin, 64, 64, "permute_mask Pt_lo"));
+    TC_TRY(make_map(&mPh64, img_p_hi, 64, cin, 64, 64, "permute_mask P_hi"));
+    auto k = (m == 4) ? permute_mask_ws_kernel<4> : permute_mask_ws_kernel<8>;
+    TC_TRY(set_smem(k, PwCfg::SMEM, "permute_mask_tc"));
+    const int tiles = cdiv(cout, 128) * (cin / 64);
+    const int grid = tiles < num_sms() ? tiles : num_sms();
+    k<<<grid, PwCfg::THREADS, PwCfg::SMEM, st>>>(mW, mPth64, mPtl64, mPh64, mAt, mask, Wp_out, cout, cin, n);
+    return check_launch("permute_mask_tc");
+  }
   if (m == 4) {
     if (BC == 64) return permute_mask2_bc<64, 4>(mW, mPth, mPtl, mPh, mask, At, Wp_out, cout, cin, n, st);
     if (BC == 128) return permute_mask2_bc<128, 4>(mW, mPth, mPtl, mPh, mask, At, Wp_out, cout, cin, n, st);
@@ -1409,8 +1859,13 @@ lcp_status launch_block_bwd_tc(const __nv_bfloat16* W, const __nv_bfloat16* dAt,
   TC_TRY(make_map(&mD, dAt, cin, cout, 64, 128, "block_bwd dAt"));
   TC_TRY(make_map(&mPth, img_pt_hi, BC, cin, 64, BC, "block_bwd Pt_hi"));
   TC_TRY(make_map(&mPtl, img_pt_lo, BC, cin, 64, BC, "block_bwd Pt_lo"));
-  if (B == 32) return block_bwd2_bc<32>(mW, mD, mPth, mPtl, mask, dP_partials, splits, rows, cout, cin, st);
-  if (B == 64) return block_bwd2_bc<64>(mW, mD, mPth, mPtl, mask, dP_partials, splits, rows, cout, cin, st);
+  if (B <= 64) {
+    auto k = (B == 32) ? block_bwd_ws_kernel<32> : block_bwd_ws_kernel<64>;
+    TC_TRY(set_smem(k, BwCfg::SMEM, "block_bwd_tc"));
+    k<<<dim3(cin / 64, splits), BwCfg::THREADS, BwCfg::SMEM, st>>>(mW, mD, mPth, mPtl, mask, dP_partials, cout,
+                                                                   cin, rows);
+    return check_launch("block_bwd_tc");
+  }
   return block_bwd_bc<128, 128>(mW, mD, mPth, mPtl, mask, dP_partials, splits, rows, cout, cin, st);
 }
 
