@@ -34,6 +34,25 @@ lcp_status fail(lcp_status s, const char* fmt, ...) {
   return s;
 }
 
+lcp_status ensure_smem_limit(const void* func, int bytes, const char* what) {
+  struct Entry { const void* f; int dev; int bytes; };
+  static std::mutex mu;
+  static Entry seen[256];
+  static int nseen = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lk(mu);
+  for (int i = 0; i < nseen; ++i)
+    if (seen[i].f == func && seen[i].dev == dev && seen[i].bytes >= bytes) return LCP_OK;
+  const cudaError_t e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(LCP_ERR_CUDA, "%s: cudaFuncSetAttribute: %s", what, cudaGetErrorString(e));
+  }
+  if (nseen < 256) seen[nseen++] = Entry{func, dev, bytes};
+  return LCP_OK;
+}
+
 lcp_status check_launch(const char* what) {
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(LCP_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
@@ -190,9 +209,15 @@ lcp_status launch_loss(const float* Yd, const float* Ys, float* stats, void* G, 
 }
 int loss_launches(int cout) { return loss_fused_supported(cout) ? 1 : 2; }
 
+// Stage events.  Under stream capture they become event-record nodes of the
+// graph (external records), so a replayed graph still times every stage.
 lcp_status record(cudaEvent_t* ev, int k, cudaStream_t st) {
   if (!ev) return LCP_OK;
-  const cudaError_t e = cudaEventRecord(ev[k], st);
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  cudaStreamIsCapturing(st, &cs);
+  const cudaError_t e = (cs == cudaStreamCaptureStatusActive)
+                            ? cudaEventRecordWithFlags(ev[k], st, cudaEventRecordExternal)
+                            : cudaEventRecord(ev[k], st);
   if (e != cudaSuccess) return fail(LCP_ERR_CUDA, "cudaEventRecord: %s", cudaGetErrorString(e));
   return LCP_OK;
 }

@@ -15,6 +15,10 @@ lcp_status fail(lcp_status s, const char* fmt, ...);
 // Checks cudaGetLastError() after a launch; returns LCP_ERR_CUDA with `what`.
 lcp_status check_launch(const char* what);
 
+// Raises `func`'s dynamic shared-memory limit to `bytes` on the current device
+// unless an earlier call already did (the attribute persists for the process).
+lcp_status ensure_smem_limit(const void* func, int bytes, const char* what);
+
 // ---- element conversions -------------------------------------------------
 __device__ __forceinline__ float to_f32(float v) { return v; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }

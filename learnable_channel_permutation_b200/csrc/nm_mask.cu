@@ -15,17 +15,24 @@
 namespace lcp {
 namespace {
 
+// Each pair k < j is compared once: k ranks ahead of j exactly when
+// |a_k| >= |a_j| (ties go to the lower index), otherwise j ranks ahead of k.
 template <int M>
 __device__ __forceinline__ uint32_t group_bits(const float* a, int n) {
+  int ahead[M];
+#pragma unroll
+  for (int j = 0; j < M; ++j) ahead[j] = 0;
+#pragma unroll
+  for (int k = 0; k < M; ++k)
+#pragma unroll
+    for (int j = k + 1; j < M; ++j) {
+      const int kj = a[k] >= a[j];
+      ahead[j] += kj;
+      ahead[k] += 1 - kj;
+    }
   uint32_t bits = 0;
 #pragma unroll
-  for (int j = 0; j < M; ++j) {
-    int ahead = 0;
-#pragma unroll
-    for (int k = 0; k < M; ++k)
-      if (k != j) ahead += (a[k] > a[j]) || (a[k] == a[j] && k < j);
-    bits |= (ahead < n ? 1u : 0u) << j;
-  }
+  for (int j = 0; j < M; ++j) bits |= (ahead[j] < n ? 1u : 0u) << j;
   return bits;
 }
 

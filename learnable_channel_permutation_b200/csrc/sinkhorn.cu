@@ -35,7 +35,7 @@ namespace {
 
 template <int B> struct SkCfg {
   static constexpr int CS = (B == 256) ? 4 : 1;                   // CTAs per block
-  static constexpr int NT = (B == 32) ? 128 : (B == 64 ? 256 : 512);
+  static constexpr int NT = (B == 32) ? 256 : (B == 64 ? 512 : 1024);
   static constexpr int R = B / CS;                                 // rows per CTA
   static constexpr int TPR = NT / R;                               // lanes per row
   static constexpr int EPR = B / TPR;                              // elements per row slice
@@ -98,7 +98,7 @@ __device__ __forceinline__ void load_slab(float* tile, const float* __restrict__
 
 // Forward.  Shared memory (floats): tile[R*(B+1)] rv[R] cv[B] xm[2B] xs[2B]
 template <int B>
-__global__ void __launch_bounds__(SkCfg<B>::NT)
+__global__ void __launch_bounds__(SkCfg<B>::NT, 1)
 sinkhorn_fwd_kernel(const float* __restrict__ L, float* __restrict__ P, float* __restrict__ ckpt,
                     __nv_bfloat16* __restrict__ pt_hi, __nv_bfloat16* __restrict__ pt_lo,
                     __nv_bfloat16* __restrict__ p_hi, float tau, int iters) {
@@ -230,7 +230,7 @@ sinkhorn_fwd_kernel(const float* __restrict__ L, float* __restrict__ P, float* _
 // Reverse.  dZ lives in registers in the row layout.
 // Shared memory (floats): tile[R*(B+1)] ck[B] ck1[B] part[NW*B] cs[B] xs[2B]
 template <int B>
-__global__ void __launch_bounds__(SkCfg<B>::NT)
+__global__ void __launch_bounds__(SkCfg<B>::NT, 1)
 sinkhorn_bwd_kernel(const float* __restrict__ L, const float* __restrict__ ckpt,
                     const float* __restrict__ dP, int splits, int nblocks,
                     float* __restrict__ dL, float tau, int iters) {
@@ -352,9 +352,8 @@ template <int B> constexpr size_t bwd_smem() {
 template <typename K, typename... Args>
 lcp_status launch_cluster(K kernel, int grid, int threads, size_t smem, int cs, cudaStream_t st,
                           const char* what, Args... args) {
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-      cudaSuccess)
-    return check_launch(what);
+  const lcp_status s0 = ensure_smem_limit(reinterpret_cast<const void*>(kernel), (int)smem, what);
+  if (s0 != LCP_OK) return s0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(threads);

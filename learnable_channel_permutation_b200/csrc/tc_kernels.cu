@@ -220,23 +220,29 @@ __device__ __forceinline__ void st_sw128(uint8_t* region, int row, int ch, uint4
 }
 
 // N:M keep bits of the 32 consecutive values in v (|v| compared as float32;
-// equal magnitudes keep the lower column).
+// equal magnitudes keep the lower column).  Element k ranks ahead of j when
+// |v_k| > |v_j|, or the two are equal and k < j; j is kept when fewer than n
+// elements rank ahead of it.  Each pair k < j is compared once: k ranks ahead
+// of j exactly when |v_k| >= |v_j|, otherwise j ranks ahead of k.
 template <int M>
 __device__ __forceinline__ uint32_t nm_word(const uint32_t (&v)[32], int n) {
   uint32_t w = 0;
 #pragma unroll
   for (int g = 0; g < 32 / M; ++g) {
     float a[M];
+    int ahead[M];
 #pragma unroll
-    for (int j = 0; j < M; ++j) a[j] = fabsf(__uint_as_float(v[g * M + j]));
+    for (int j = 0; j < M; ++j) { a[j] = fabsf(__uint_as_float(v[g * M + j])); ahead[j] = 0; }
 #pragma unroll
-    for (int j = 0; j < M; ++j) {
-      int ahead = 0;
+    for (int k = 0; k < M; ++k)
 #pragma unroll
-      for (int k = 0; k < M; ++k)
-        if (k != j) ahead += (a[k] > a[j]) || (a[k] == a[j] && k < j);
-      w |= (ahead < n ? 1u : 0u) << (g * M + j);
-    }
+      for (int j = k + 1; j < M; ++j) {
+        const int kj = a[k] >= a[j];
+        ahead[j] += kj;
+        ahead[k] += 1 - kj;
+      }
+#pragma unroll
+    for (int j = 0; j < M; ++j) w |= (ahead[j] < n ? 1u : 0u) << (g * M + j);
   }
   return w;
 }
@@ -693,15 +699,16 @@ permute_mask_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16(128, 64, false, false);
-      int k = 0;
-      for (int idx = blockIdx.x; idx < total; idx += gridDim.x, ++k) {
+      const int nloc = blockIdx.x < total ? cdiv(total - blockIdx.x, gridDim.x) : 0;
+      // W' = W (P_hi + P_lo) of local tile k into TMEM buffer k & 1
+      auto mma1 = [&](int k) -> bool {
         const int st = k % C::STAGES, a = k & 1;
         const uint32_t use = (uint32_t)(k / C::STAGES) & 1u, ua = (uint32_t)(k >> 1) & 1u;
-        if (!mbar_wait(bar(FULL + st), use, abort_flag, 63)) break;
-        if (!mbar_wait(bar(TME + a), ua ^ 1u, abort_flag, 64)) break;
+        if (!mbar_wait(bar(FULL + st), use, abort_flag, 63)) return false;
+        if (!mbar_wait(bar(TME + a), ua ^ 1u, abort_flag, 64)) return false;
         tc_fence_after();
         const uint32_t sg = smem_u32(sStage + st * C::STAGE);
-        const uint32_t dW = tmem + a * 128, dAt = tmem + a * 128 + 64;
+        const uint32_t dW = tmem + a * 128;
 #pragma unroll
         for (int k16 = 0; k16 < 4; ++k16) {
           const uint64_t ad = sdesc(sg + k16 * 32, 16, 1024);
@@ -709,9 +716,20 @@ permute_mask_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
           mma_bf16(dW, ad, sdesc(sg + C::W_BYTES + C::IMG_BYTES + k16 * 32, 16, 1024), idesc, true);
         }
         mma_commit(bar(WF + a));
+        return true;
+      };
+      // the next tile's first product is issued before waiting for this tile's
+      // epilogue, so the tensor core and the epilogue warps overlap
+      bool ok = nloc == 0 || mma1(0);
+      for (int k = 0; k < nloc && ok; ++k) {
+        const int st = k % C::STAGES, a = k & 1;
+        const uint32_t ua = (uint32_t)(k >> 1) & 1u;
+        if (k + 1 < nloc && !mma1(k + 1)) break;
         if (!mbar_wait(bar(AF + a), ua, abort_flag, 65)) break;
         tc_fence_after();
+        const uint32_t sg = smem_u32(sStage + st * C::STAGE);
         const uint32_t sa = smem_u32(sA + a * C::A_BYTES);
+        const uint32_t dAt = tmem + a * 128 + 64;
 #pragma unroll
         for (int k16 = 0; k16 < 4; ++k16)
           mma_bf16(dAt, sdesc(sa + k16 * 32, 16, 1024), sdesc(sg + C::W_BYTES + 2 * C::IMG_BYTES + k16 * 32, 16, 1024),
@@ -1099,12 +1117,13 @@ block_bwd_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_consta
       constexpr uint32_t idesc_n = idesc_bf16(128, 64, false, false);
       constexpr uint32_t idesc_dp = idesc_bf16(128, 128, true, true);
       bool ok = nchunk == 0 || mbar_wait(bar(IMG), 0, abort_flag, 74);
-      for (int c = 0; c < nchunk && ok; ++c) {
+      // W' = W (P_hi + P_lo) and dA = dAt P_hi of chunk c into TMEM buffer c & 1
+      auto mma1 = [&](int c) -> bool {
         const int st = c % C::STAGES, a = c & 1;
         const uint32_t use = (uint32_t)(c / C::STAGES) & 1u, ua = (uint32_t)(c >> 1) & 1u;
-        if (!mbar_wait(bar(FULL + st), use, abort_flag, 75)) break;
-        // the epilogue has read buffer a of chunk c - 2 (it arrived on ABF after its loads)
-        if (c >= 2 && !mbar_wait(bar(ABF + a), ua ^ 1u, abort_flag, 76)) break;
+        if (!mbar_wait(bar(FULL + st), use, abort_flag, 75)) return false;
+        // the epilogue has read buffer a of chunk c - 2 (it arrives on ABF after its loads)
+        if (c >= 2 && !mbar_wait(bar(ABF + a), ua ^ 1u, abort_flag, 76)) return false;
         tc_fence_after();
         const uint32_t sg = smem_u32(sStage + st * C::STAGE);
         const uint32_t tW = tmem + a * 128, tDA = tmem + a * 128 + 64;
@@ -1117,8 +1136,16 @@ block_bwd_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_consta
                    k16 != 0);
         }
         mma_commit(bar(WD + a));
+        return true;
+      };
+      if (ok && nchunk > 0) ok = mma1(0);
+      for (int c = 0; c < nchunk && ok; ++c) {
+        const int st = c % C::STAGES, a = c & 1;
+        const uint32_t ua = (uint32_t)(c >> 1) & 1u;
+        if (c + 1 < nchunk && !mma1(c + 1)) break;
         if (!mbar_wait(bar(ABF + a), ua, abort_flag, 77)) break;
         tc_fence_after();
+        const uint32_t sg = smem_u32(sStage + st * C::STAGE);
         const uint32_t sab = smem_u32(sAB + a * 2 * C::T_BYTES);
         // stacked: A operand [dAt | W] (M = 128), B operand [A | dW'] (N = 128), LBO = 16 KB
 #pragma unroll
@@ -1142,6 +1169,8 @@ block_bwd_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_consta
       const int a = c & 1;
       const uint32_t ua = (uint32_t)(c >> 1) & 1u;
       const int grow = rbeg + c * 128 + row;
+      // the mask word is fetched before waiting for the tensor core
+      const uint32_t bits = grow < rend ? __ldg(mask + (size_t)grow * words + col0 / 32 + h) : 0u;
       ok = named_and(1, C::EPI, mbar_wait(bar(WD + a), ua, abort_flag, 79));
       if (!ok) break;
       tc_fence_after();
@@ -1149,7 +1178,6 @@ block_bwd_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_consta
       tmem_ld32(tmem + lane_off + a * 128 + h * 32, wv);
       tmem_ld32(tmem + lane_off + a * 128 + 64 + h * 32, dv);
       tmem_ld_wait();
-      const uint32_t bits = grow < rend ? __ldg(mask + (size_t)grow * words + col0 / 32 + h) : 0u;
       // buffer a was last read by the dP product of chunk c - 2
       ok = named_and(1, C::EPI, c < 2 || mbar_wait(bar(ABE + a), ua ^ 1u, abort_flag, 80));
       if (!ok) break;
@@ -1701,12 +1729,7 @@ int num_sms() {
 
 template <typename K>
 lcp_status set_smem(K kernel, int bytes, const char* what) {
-  const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e != cudaSuccess) {
-    cudaGetLastError();
-    return fail(LCP_ERR_CUDA, "%s: cudaFuncSetAttribute: %s", what, cudaGetErrorString(e));
-  }
-  return LCP_OK;
+  return ensure_smem_limit(reinterpret_cast<const void*>(kernel), bytes, what);
 }
 
 #define TC_TRY(x)                      \
