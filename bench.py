@@ -212,6 +212,7 @@ def main():
     ap.add_argument("--simt", action="store_true", help="CUDA-core kernels for every contraction")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--eager", action="store_true", help="time eager launches instead of CUDA-graph replays")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
@@ -248,46 +249,70 @@ def main():
     stream = torch.cuda.current_stream()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
-    for _ in range(args.warmup):
-        step.run()
-    torch.cuda.synchronize()
-
     K = args.steps
-    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    stages = [[torch.cuda.Event(enable_timing=True) for _ in range(b.TIMED_EVENTS)] for _ in range(K)]
-    for row in stages:            # materialise the events before handing them to the library
-        for e in row:
-            e.record()
     props = torch.cuda.get_device_properties(dev)
     uuid = getattr(props, "uuid", None)
     uuid = f"GPU-{uuid}" if uuid and not str(uuid).startswith("GPU-") else (str(uuid) if uuid else None)
     sampler = ClockSampler(uuid if world == 1 else None)
 
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
+    def timed_loop(graph_mode):
+        """K timed steps; returns (total ms of our kernels, per-stage ms averages)."""
+        if graph_mode:
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(b.TIMED_EVENTS)]
+            for e in ev:
+                e.record()
+            g = b.capture(step, ev)
+            for _ in range(args.warmup):
+                g.replay()
+        else:
+            ev = None
+            for _ in range(args.warmup):
+                step.run()
+        torch.cuda.synchronize()
+        rows = []
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        for _ in range(K):
+            flush.zero_()                      # L2 flush, outside the timed events
+            if graph_mode:
+                g.replay()
+                torch.cuda.synchronize()       # the stage events are reused by every replay
+                rows.append([ev[s].elapsed_time(ev[s + 1]) for s in range(len(b.STAGES))])
+            else:
+                e = [torch.cuda.Event(enable_timing=True) for _ in range(b.TIMED_EVENTS)]
+                for x in e:
+                    x.record()
+                step.run_timed(e)
+                rows.append(e)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        if not graph_mode:
+            rows = [[e[s].elapsed_time(e[s + 1]) for s in range(len(b.STAGES))] for e in rows]
+        total = sum(sum(r) for r in rows)
+        per_stage = {name: sum(r[i] for r in rows) / K for i, name in enumerate(b.STAGES)}
+        if graph_mode:
+            del g
+        return total, per_stage
+
     sampler.start()
     time.sleep(0.2)
-    for k in range(K):
-        flush.zero_()
-        ev0[k].record(stream)
-        step.run_timed(stages[k])
-        ev1[k].record(stream)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
+    graph_mode = not args.eager
+    total_ms, stage_ms = timed_loop(graph_mode)
     clocks = sampler.stop()
+    eager_total = None
+    if graph_mode:
+        eager_total, _ = timed_loop(False)
 
-    total_ms = sum(ev0[k].elapsed_time(ev1[k]) for k in range(K))
-    stage_ms = {}
-    for s, name in enumerate(b.STAGES):
-        stage_ms[name] = sum(stages[k][s].elapsed_time(stages[k][s + 1]) for k in range(K)) / K
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    t = torch.tensor([total_ms, eager_total or 0.0], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    max_ms = float(t.item())
+    max_ms = float(t[0].item())
     value = world * K / (max_ms / 1e3)
+    eager = None
+    if eager_total is not None:
+        eager = {"value": world * K / (float(t[1].item()) / 1e3), "ms_per_step": float(t[1].item()) / K}
 
     # end to end through the public API: pinned host inputs in, loss and dL out, every step
     e2e = None
@@ -361,8 +386,9 @@ def main():
                        "block": wl.block, "nm": f"{wl.n}:{wl.m}", "tau": wl.tau, "iters": wl.iters,
                        "parallelism": f"layer-sharded x{world}" if world > 1 else "single GPU",
                        "l2": "flushed between timed steps (256 MiB write)",
-                       "path": "simt" if args.simt else "tcgen05"},
-            "roofline": roof, "stages": per_stage, "clocks": clocks, "e2e": e2e,
+                       "path": "simt" if args.simt else "tcgen05",
+                       "launch": "cuda-graph replay per step" if graph_mode else "eager launches"},
+            "roofline": roof, "stages": per_stage, "clocks": clocks, "e2e": e2e, "eager": eager,
             "gpu_launches": step.launches * K}
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)

@@ -172,6 +172,24 @@ class Step:
                                    _stream(stream), arr, TIMED_EVENTS))
 
 
+def capture(step: "Step", events: Optional[List[torch.cuda.Event]] = None) -> "torch.cuda.CUDAGraph":
+    """Capture one lcp_step (and, with ``events``, its stage events) into a CUDA
+    graph; replaying it re-runs the step on the same buffers with one launch."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step.run(side)                     # first call outside capture (one-time set-up)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        if events is None:
+            step.run()
+        else:
+            step.run_timed(events)
+    return g
+
+
 def alloc_outputs(W: torch.Tensor, X: torch.Tensor, L: torch.Tensor, with_mask: bool = True,
                   with_wp: bool = False) -> Dict[str, torch.Tensor]:
     dev = W.device
