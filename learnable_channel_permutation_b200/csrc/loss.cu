@@ -170,9 +170,12 @@ loss_fused_kernel(const float* __restrict__ Yd, const float* __restrict__ Ys, fl
       write_g<TG>(G, row + 4 * (size_t)q, g);
     }
   }
-  // last CTA: the loss
-  __threadfence();
-  if (threadIdx.x == 0) is_last = (atomicAdd(counter, 1u) == (unsigned)tokens - 1u);
+  // last CTA: the loss.  Thread 0 wrote this token's statistics; its fence
+  // orders that write before its vote, so the last voter sees every token.
+  if (threadIdx.x == 0) {
+    __threadfence();
+    is_last = (atomicAdd(counter, 1u) == (unsigned)tokens - 1u);
+  }
   __syncthreads();
   if (!is_last) return;
   __threadfence();

@@ -152,13 +152,17 @@ __device__ __forceinline__ uint32_t mapa(uint32_t a, uint32_t rank) {
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
+// Arrivals on a barrier addressed through the cluster window (it may live in
+// the peer CTA).  No cluster-scope release: the data these arrivals announce
+// travels by TMA (counted by complete_tx) or lives in tensor memory (ordered by
+// tcgen05.fence), and a cluster-scope release would make the arriving thread
+// wait for its own outstanding bulk copies.
 __device__ __forceinline__ void mbar_expect_tx_cluster(uint32_t bar_cluster, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(bar_cluster),
-               "r"(bytes)
+  asm volatile("mbarrier.arrive.expect_tx.shared::cluster.b64 _, [%0], %1;" ::"r"(bar_cluster), "r"(bytes)
                : "memory");
 }
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
 }
 // TMA load into this CTA's shared memory whose completion is counted on a
 // barrier that may live in the peer CTA of the pair
@@ -1420,12 +1424,17 @@ block_bwd_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_consta
     const int row = q * 32 + lane;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     bool ok = true;
+    // mask words run one chunk ahead of the chunk being processed
+    auto mask_word = [&](int c) -> uint32_t {
+      const int grow = rbeg + c * 128 + row;
+      return (c < nchunk && grow < rend) ? __ldg(mask + (size_t)grow * words + col0 / 32 + h) : 0u;
+    };
+    uint32_t next_bits = mask_word(0);
     for (int c = 0; c < nchunk; ++c) {
       const int a = c & 1;
       const uint32_t ua = (uint32_t)(c >> 1) & 1u;
-      const int grow = rbeg + c * 128 + row;
-      // the mask word is fetched before waiting for the tensor core
-      const uint32_t bits = grow < rend ? __ldg(mask + (size_t)grow * words + col0 / 32 + h) : 0u;
+      const uint32_t bits = next_bits;
+      next_bits = mask_word(c + 1);
       ok = named_and(1, C::EPI, mbar_wait(bar(WD + a), ua, abort_flag, 79));
       if (!ok) break;
       tc_fence_after();
@@ -1500,218 +1509,6 @@ block_bwd_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_consta
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
-  }
-}
-
-// ---------------------------------------------- block backward, streamed ---
-// BC = 64 (B = 32 or 64): as block_bwd_tc_kernel below, with the W and dAt
-// tiles of the next 128-row chunk streaming into a second stage while the
-// current chunk is processed.  Stage s = [dAt_s | W_s] (adjacent, so that the
-// stacked MN-major A operand of the dP product spans both).
-struct Bb2Cfg {
-  static constexpr int T_BYTES = 64 * 256;        // 128 rows x 64 bf16
-  static constexpr int STAGE = 2 * T_BYTES;
-  static constexpr int P_BYTES = 64 * 64 * 2;
-  static constexpr uint32_t TMEM_COLS = 256u;     // W' 64 | dA 64 | dP 128
-  // no alignment slack (two CTAs per SM must fit in 228 KB): the kernel checks
-  // that the dynamic shared memory starts on a 1024-byte boundary instead
-  static constexpr int SMEM = 2 * STAGE + 2 * P_BYTES + 2 * T_BYTES + 128;
-};
-
-template <int B>
-__global__ void __launch_bounds__(128)
-block_bwd_tc2_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmDAt,
-                     const __grid_constant__ CUtensorMap tmPth, const __grid_constant__ CUtensorMap tmPtl,
-                     const uint32_t* __restrict__ mask, float* __restrict__ dP, int cout, int cin,
-                     int rows_per_split) {
-  using C = Bb2Cfg;
-  constexpr int BC = 64;
-  extern __shared__ uint8_t smem_raw[];
-  if (smem_u32(smem_raw) & 1023u) {   // uniform across the CTA: nothing has been started yet
-    if (threadIdx.x == 0) atomicCAS(&g_tc_error, 0, 50);
-    return;
-  }
-  uint8_t* smem = smem_raw;
-  uint8_t* sStage = smem;                       // stage s at + s * STAGE: dAt then W
-  uint8_t* sPth = smem + 2 * C::STAGE;
-  uint8_t* sPtl = sPth + C::P_BYTES;
-  uint8_t* sAb = sPtl + C::P_BYTES;
-  uint8_t* sdWb = sAb + C::T_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sdWb + C::T_BYTES);
-  uint32_t* holder = reinterpret_cast<uint32_t*>(bars + 5);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(holder + 1);
-  const uint32_t bar_full0 = smem_u32(bars + 0);
-  const uint32_t bar_mma1 = smem_u32(bars + 2), bar_mma2 = smem_u32(bars + 3), bar_drain = smem_u32(bars + 4);
-
-  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-  const int t = blockIdx.x, s = blockIdx.y, col0 = t * BC;
-  const int rbeg = s * rows_per_split;
-  const int rend = min(cout, rbeg + rows_per_split);
-  const int nchunk = cdiv(rend - rbeg, 128);
-  if (tid == 0) {
-    mbar_init(bar_full0, 1);
-    mbar_init(bar_full0 + 8, 1);
-    mbar_init(bar_mma1, 1);
-    mbar_init(bar_mma2, 1);
-    mbar_init(bar_drain, 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == 0) tmem_alloc(smem_u32(holder), C::TMEM_COLS);
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *holder;
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-  const int row = warp * 32 + lane;
-  const int words = cin / 32;
-  constexpr uint32_t idesc_n = idesc_bf16(128, BC, false, false);
-  constexpr uint32_t idesc_dp = idesc_bf16(128, 128, true, true);
-  const uint32_t tW = tmem, tDA = tmem + BC, tDP = tmem + 2 * BC;
-
-  auto load_chunk = [&](int ch, int st) {   // thread 0
-    const int r0 = rbeg + ch * 128;
-    tma_load_2d(smem_u32(sStage + st * C::STAGE), &tmDAt, bar_full0 + 8 * st, col0, r0);
-    tma_load_2d(smem_u32(sStage + st * C::STAGE + C::T_BYTES), &tmW, bar_full0 + 8 * st, col0, r0);
-  };
-  int issued = 0, consumed = 0;
-  if (tid == 0 && nchunk > 0) {
-    mbar_expect_tx(bar_full0, C::STAGE + 2 * C::P_BYTES);
-    tma_load_2d(smem_u32(sPth), &tmPth, bar_full0, 0, col0);
-    tma_load_2d(smem_u32(sPtl), &tmPtl, bar_full0, 0, col0);
-    load_chunk(0, 0);
-    issued = 1;
-    if (nchunk > 1) {
-      mbar_expect_tx(bar_full0 + 8, C::STAGE);
-      load_chunk(1, 1);
-      issued = 2;
-    }
-  }
-
-  bool ok = true;
-  for (int ch = 0; ch < nchunk && ok; ++ch) {
-    const int st = ch & 1;
-    const uint8_t* sDAt = sStage + st * C::STAGE;
-    const uint8_t* sW = sDAt + C::T_BYTES;
-    if (tid == 0) {
-      if (mbar_wait(bar_full0 + 8 * st, (uint32_t)(ch >> 1) & 1u, abort_flag, 51)) {
-        consumed = ch + 1;
-        tc_fence_after();
-#pragma unroll
-        for (int k16 = 0; k16 < 4; ++k16) {
-          const uint64_t a = sdesc(smem_u32(sW) + k16 * 32, 16, 1024);
-          mma_bf16(tW, a, sdesc(smem_u32(sPth) + k16 * 32, 16, 1024), idesc_n, k16 != 0);
-          mma_bf16(tW, a, sdesc(smem_u32(sPtl) + k16 * 32, 16, 1024), idesc_n, true);
-          mma_bf16(tDA, sdesc(smem_u32(sDAt) + k16 * 32, 16, 1024), sdesc(smem_u32(sPth) + k16 * 32, 16, 1024),
-                   idesc_n, k16 != 0);
-        }
-        mma_commit(bar_mma1);
-      } else {
-        *abort_flag = 1;
-      }
-    }
-    ok = __syncthreads_and(mbar_wait(bar_mma1, (uint32_t)ch & 1u, abort_flag, 52));
-    if (!ok) break;
-    tc_fence_after();
-    const int grow = rbeg + ch * 128 + row;
-    const bool valid = grow < rend;
-    const uint2 bw = valid ? __ldg(reinterpret_cast<const uint2*>(mask + (size_t)grow * words + col0 / 32))
-                           : make_uint2(0u, 0u);
-#pragma unroll 1
-    for (int cc = 0; cc < 2; ++cc) {
-      uint32_t wv[32], dv[32];
-      tmem_ld32(tW + lane_off + cc * 32, wv);
-      tmem_ld32(tDA + lane_off + cc * 32, dv);
-      tmem_ld_wait();
-      const uint32_t bits = cc ? bw.y : bw.x;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        float fa[8], fd[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const bool keep = (bits >> (8 * q + e)) & 1u;
-          fa[e] = keep ? __uint_as_float(wv[8 * q + e]) : 0.f;
-          fd[e] = keep ? __uint_as_float(dv[8 * q + e]) : 0.f;
-        }
-        st_sw128(sAb, row, cc * 4 + q, make_uint4(pack_bf16x2(fa[0], fa[1]), pack_bf16x2(fa[2], fa[3]),
-                                                  pack_bf16x2(fa[4], fa[5]), pack_bf16x2(fa[6], fa[7])));
-        st_sw128(sdWb, row, cc * 4 + q, make_uint4(pack_bf16x2(fd[0], fd[1]), pack_bf16x2(fd[2], fd[3]),
-                                                   pack_bf16x2(fd[4], fd[5]), pack_bf16x2(fd[6], fd[7])));
-      }
-    }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0) {
-      tc_fence_after();
-      // stacked: A = [dAt | W] (M = 128), B = [A | dW'] (N = 128), LBO = 16 KB
-#pragma unroll
-      for (int k16 = 0; k16 < 8; ++k16)
-        mma_bf16(tDP, sdesc(smem_u32(sDAt) + k16 * 2048, 16384, 1024),
-                 sdesc(smem_u32(sAb) + k16 * 2048, 16384, 1024), idesc_dp, (ch | k16) != 0);
-      mma_commit(bar_mma2);
-      if (ch + 2 < nchunk) {
-        // this stage is free once the dP product has read it: stream chunk ch + 2 in
-        if (mbar_wait(bar_mma2, (uint32_t)ch & 1u, abort_flag, 53)) {
-          mbar_expect_tx(bar_full0 + 8 * st, C::STAGE);
-          load_chunk(ch + 2, st);
-          issued = ch + 3;
-        } else {
-          *abort_flag = 1;
-        }
-      }
-    }
-  }
-  if (ok && nchunk > 0) ok = __syncthreads_and(mbar_wait(bar_mma2, (uint32_t)(nchunk - 1) & 1u, abort_flag, 54));
-  const int nb = cin / B;
-  float* dPs = dP + (size_t)s * nb * B * B;
-  if (ok) {
-    tc_fence_after();
-    // rows 0..63: dAt^T A in columns 0..63; rows 64..127: W^T dW' in columns 64..127
-    float* scratch = reinterpret_cast<float*>(sAb);   // 64 x 64 floats (free: last MMA done)
-    uint32_t r0v[32], r1v[32];
-    const uint32_t cbase = (row < 64) ? 0u : 64u;
-    tmem_ld32(tDP + lane_off + cbase, r0v);
-    tmem_ld32(tDP + lane_off + cbase + 32, r1v);
-    tmem_ld_wait();
-    if (row >= 64) {
-      float* dst = scratch + (row - 64) * 64;
-#pragma unroll
-      for (int e = 0; e < 32; ++e) { dst[e] = __uint_as_float(r0v[e]); dst[32 + e] = __uint_as_float(r1v[e]); }
-    }
-    __syncthreads();
-    if (row < 64) {
-      const float* add = scratch + row * 64;
-      if constexpr (B == 64) {
-        float4* o = reinterpret_cast<float4*>(dPs + ((size_t)t * 64 + row) * 64);
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-          o[q] = make_float4(__uint_as_float(r0v[4 * q]) + add[4 * q], __uint_as_float(r0v[4 * q + 1]) + add[4 * q + 1],
-                             __uint_as_float(r0v[4 * q + 2]) + add[4 * q + 2], __uint_as_float(r0v[4 * q + 3]) + add[4 * q + 3]);
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-          o[8 + q] = make_float4(__uint_as_float(r1v[4 * q]) + add[32 + 4 * q], __uint_as_float(r1v[4 * q + 1]) + add[33 + 4 * q],
-                                 __uint_as_float(r1v[4 * q + 2]) + add[34 + 4 * q], __uint_as_float(r1v[4 * q + 3]) + add[35 + 4 * q]);
-      } else {
-        const int qb = row / 32;            // which 32-block of the tile
-        float* o = dPs + ((size_t)(2 * t + qb) * 32 + (row - 32 * qb)) * 32;
-        const uint32_t* src = qb ? r1v : r0v;
-#pragma unroll
-        for (int e = 0; e < 32; ++e) o[e] = __uint_as_float(src[e]) + add[32 * qb + e];
-      }
-    }
-  }
-  if (tid == 0) {
-    for (int kk = consumed; kk < issued; ++kk)
-      mbar_wait_drain(bar_full0 + 8 * (kk & 1), (uint32_t)(kk >> 1) & 1u, 55);
-    mma_commit(bar_drain);
-    mbar_wait_drain(bar_drain, 0, 56);
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 0) {
-    tc_fence_after();
-    tmem_dealloc(tmem, C::TMEM_COLS);
   }
 }
 
@@ -2019,17 +1816,6 @@ lcp_status permute_mask_bc(const CUtensorMap& mW, const CUtensorMap& mPth, const
   return check_launch("permute_mask_tc");
 }
 
-template <int B>
-lcp_status block_bwd2_bc(const CUtensorMap& mW, const CUtensorMap& mD, const CUtensorMap& mPth,
-                         const CUtensorMap& mPtl, const uint32_t* mask, float* dP, int splits, int rows,
-                         int cout, int cin, cudaStream_t st) {
-  auto k = block_bwd_tc2_kernel<B>;
-  TC_TRY(set_smem(k, Bb2Cfg::SMEM, "block_bwd_tc"));
-  const dim3 grid(cin / 64, splits);
-  k<<<grid, 128, Bb2Cfg::SMEM, st>>>(mW, mD, mPth, mPtl, mask, dP, cout, cin, rows);
-  return check_launch("block_bwd_tc");
-}
-
 template <int BC, int B>
 lcp_status block_bwd_bc(const CUtensorMap& mW, const CUtensorMap& mD, const CUtensorMap& mPth,
                         const CUtensorMap& mPtl, const uint32_t* mask, float* dP, int splits, int rows,
@@ -2144,26 +1930,21 @@ lcp_status launch_permute_mask_tc(const __nv_bfloat16* W, const __nv_bfloat16* i
   TC_TRY(make_map(&mW, W, cin, cout, 64, 128, "permute_mask W"));
   TC_TRY(make_map(&mPth, img_pt_hi, BC, cin, 64, 64, "permute_mask Pt_hi"));
   TC_TRY(make_map(&mPtl, img_pt_lo, BC, cin, 64, 64, "permute_mask Pt_lo"));
-  TC_TRY(make_map(&mPh, img_p_hi, BC, cin, 64, BC, "permute_mask P_hi"));
+  TC_TRY(make_map(&mPh, img_p_hi, BC, cin, 64, BC == 64 ? 64 : BC, "permute_mask P_hi"));
   if (BC == 64) {
-    CUtensorMap mAt, mPth64, mPtl64, mPh64;
+    CUtensorMap mAt;
     TC_TRY(make_map(&mAt, At, cin, cout, 64, 128, "permute_mask At"));
-    TC_TRY(make_map(&mPth64, img_pt_hi, 64, cin, 64, 64, "permute_mask Pt_hi"));
-    TC_TRY(make_map(&mPtl64, img_pt_lo, 64, cin, 64, 64, "permute_mask Pt_lo"));
-    TC_TRY(make_map(&mPh64, img_p_hi, 64, cin, 64, 64, "permute_mask P_hi"));
     auto k = (m == 4) ? permute_mask_ws_kernel<4> : permute_mask_ws_kernel<8>;
     TC_TRY(set_smem(k, PwCfg::SMEM, "permute_mask_tc"));
     const int tiles = cdiv(cout, 128) * (cin / 64);
     const int grid = tiles < num_sms() ? tiles : num_sms();
-    k<<<grid, PwCfg::THREADS, PwCfg::SMEM, st>>>(mW, mPth64, mPtl64, mPh64, mAt, mask, Wp_out, cout, cin, n);
+    k<<<grid, PwCfg::THREADS, PwCfg::SMEM, st>>>(mW, mPth, mPtl, mPh, mAt, mask, Wp_out, cout, cin, n);
     return check_launch("permute_mask_tc");
   }
   if (m == 4) {
-    if (BC == 64) return permute_mask2_bc<64, 4>(mW, mPth, mPtl, mPh, mask, At, Wp_out, cout, cin, n, st);
     if (BC == 128) return permute_mask2_bc<128, 4>(mW, mPth, mPtl, mPh, mask, At, Wp_out, cout, cin, n, st);
     return permute_mask_bc<256, 4>(mW, mPth, mPtl, mPh, mask, At, Wp_out, cout, cin, n, st);
   }
-  if (BC == 64) return permute_mask2_bc<64, 8>(mW, mPth, mPtl, mPh, mask, At, Wp_out, cout, cin, n, st);
   if (BC == 128) return permute_mask2_bc<128, 8>(mW, mPth, mPtl, mPh, mask, At, Wp_out, cout, cin, n, st);
   return permute_mask_bc<256, 8>(mW, mPth, mPtl, mPh, mask, At, Wp_out, cout, cin, n, st);
 }
