@@ -245,6 +245,19 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
 }
+// 32 lanes x 16 consecutive 32-bit columns
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+// NV columns per epilogue thread: 32 (one tcgen05.ld x32) or 16 (x16)
+template <int NV> __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[NV]) {
+  if constexpr (NV == 32) tmem_ld32(taddr, r);
+  else tmem_ld16(taddr, r);
+}
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -286,11 +299,11 @@ __device__ __forceinline__ void st_sw128(uint8_t* region, int row, int ch, uint4
 // |v_k| > |v_j|, or the two are equal and k < j; j is kept when fewer than n
 // elements rank ahead of it.  Each pair k < j is compared once: k ranks ahead
 // of j exactly when |v_k| >= |v_j|, otherwise j ranks ahead of k.
-template <int M>
-__device__ __forceinline__ uint32_t nm_word(const uint32_t (&v)[32], int n) {
+template <int M, int NV>
+__device__ __forceinline__ uint32_t nm_bits(const uint32_t (&v)[NV], int n) {
   uint32_t w = 0;
 #pragma unroll
-  for (int g = 0; g < 32 / M; ++g) {
+  for (int g = 0; g < NV / M; ++g) {
     float a[M];
     int ahead[M];
 #pragma unroll
@@ -307,6 +320,10 @@ __device__ __forceinline__ uint32_t nm_word(const uint32_t (&v)[32], int n) {
     for (int j = 0; j < M; ++j) w |= (ahead[j] < n ? 1u : 0u) << (g * M + j);
   }
   return w;
+}
+template <int M>
+__device__ __forceinline__ uint32_t nm_word(const uint32_t (&v)[32], int n) {
+  return nm_bits<M, 32>(v, n);
 }
 
 // --------------------------------------------------------------- GEMM -----
@@ -881,24 +898,27 @@ permute_mask_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
 // memory, At = A P_hi into the same buffer; warps 2-9 (two per TMEM lane
 // quadrant, 32 columns each) compute the mask, write A, and copy At out
 // through a swizzled staging tile with TMA stores.
-struct PwCfg {
+template <int NSL> struct PwCfg {
   static constexpr int STAGES = 3;
   static constexpr int W_BYTES = 16384;                 // 128 rows x 64 bf16
   static constexpr int IMG_BYTES = 8192;                // 64 x 64 bf16
   static constexpr int STAGE = W_BYTES + 3 * IMG_BYTES; // W | Pt_hi | Pt_lo | P_hi
   static constexpr int A_BYTES = 16384;
   static constexpr int SMEM = STAGES * STAGE + 2 * A_BYTES + 2 * A_BYTES + 1024 + 256;
-  static constexpr int THREADS = 320;
-  static constexpr int EPI = 256;                        // epilogue threads (warps 2..9)
+  static constexpr int EPI_WARPS = 4 * NSL;              // NSL column slices per TMEM lane quadrant
+  static constexpr int COLS = 64 / NSL;                  // columns per epilogue thread
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+  static constexpr int EPI = 32 * EPI_WARPS;
 };
 
-template <int MGROUP>
-__global__ void __launch_bounds__(PwCfg::THREADS, 1)
+template <int MGROUP, int NSL>
+__global__ void __launch_bounds__(PwCfg<NSL>::THREADS, 1)
 permute_mask_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmPth,
                        const __grid_constant__ CUtensorMap tmPtl, const __grid_constant__ CUtensorMap tmPh,
                        const __grid_constant__ CUtensorMap tmAt, uint32_t* __restrict__ mask,
                        float* __restrict__ Wp_out, int cout, int cin, int n) {
-  using C = PwCfg;
+  using C = PwCfg<NSL>;
+  constexpr int NV = C::COLS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sStage = smem;
@@ -919,9 +939,9 @@ permute_mask_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
     for (int i = 0; i < 3; ++i) { mbar_init(bar(FULL + i), 1); mbar_init(bar(EMPTY + i), 1); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(WF + i), 1);
-      mbar_init(bar(AF + i), 8);
+      mbar_init(bar(AF + i), C::EPI_WARPS);
       mbar_init(bar(ATF + i), 1);
-      mbar_init(bar(TME + i), 8);
+      mbar_init(bar(TME + i), C::EPI_WARPS);
     }
     mbar_init(bar(DRAIN), 1);
     *abort_flag = 0;
@@ -1001,7 +1021,7 @@ permute_mask_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
     }
     __syncwarp();
   } else {
-    const int e = warp - 2, q = warp & 3, h = e >> 2;
+    const int e = warp - 2, q = warp & 3, h = e >> 2;   // h: column slice of NV columns
     const int row = q * 32 + lane;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     const bool leader = (e == 0 && lane == 0);
@@ -1013,28 +1033,32 @@ permute_mask_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
       const int grow = rt * 128 + row;
       if (!named_and(1, C::EPI, mbar_wait(bar(WF + a), ua, abort_flag, 67))) break;
       tc_fence_after();
-      uint32_t v[32];
-      tmem_ld32(tmem + lane_off + a * 128 + h * 32, v);
+      uint32_t v[NV];
+      tmem_ld_cols<NV>(tmem + lane_off + a * 128 + h * NV, v);
       tmem_ld_wait();
-      const uint32_t w = nm_word<MGROUP>(v, n);
+      const uint32_t w = nm_bits<MGROUP, NV>(v, n);
       if (grow < cout) {
-        mask[(size_t)grow * words + 2 * t + h] = w;
+        if constexpr (NV == 32) {
+          mask[(size_t)grow * words + 2 * t + h] = w;
+        } else {
+          reinterpret_cast<uint16_t*>(mask)[((size_t)grow * words + 2 * t) * 2 + h] = (uint16_t)w;
+        }
         if (Wp_out) {
-          float4* o = reinterpret_cast<float4*>(Wp_out + (size_t)grow * cin + t * 64 + h * 32);
+          float4* o = reinterpret_cast<float4*>(Wp_out + (size_t)grow * cin + t * 64 + h * NV);
 #pragma unroll
-          for (int qq = 0; qq < 8; ++qq)
+          for (int qq = 0; qq < NV / 4; ++qq)
             o[qq] = make_float4(__uint_as_float(v[4 * qq]), __uint_as_float(v[4 * qq + 1]),
                                 __uint_as_float(v[4 * qq + 2]), __uint_as_float(v[4 * qq + 3]));
         }
       }
       uint8_t* sa = sA + a * C::A_BYTES;
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
+      for (int c8 = 0; c8 < NV / 8; ++c8) {
         float f[8];
 #pragma unroll
-        for (int x = 0; x < 8; ++x) f[x] = ((w >> (8 * c4 + x)) & 1u) ? __uint_as_float(v[8 * c4 + x]) : 0.f;
-        st_sw128(sa, row, h * 4 + c4, make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
-                                                 pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7])));
+        for (int x = 0; x < 8; ++x) f[x] = ((w >> (8 * c8 + x)) & 1u) ? __uint_as_float(v[8 * c8 + x]) : 0.f;
+        st_sw128(sa, row, h * (NV / 8) + c8, make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                                                        pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7])));
       }
       fence_async_smem();
       tc_fence_before();
@@ -1046,19 +1070,19 @@ permute_mask_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
       if (leader) bulk_wait_read<1>();
       if (!named_and(1, C::EPI, got)) break;
       tc_fence_after();
-      tmem_ld32(tmem + lane_off + a * 128 + 64 + h * 32, v);
+      tmem_ld_cols<NV>(tmem + lane_off + a * 128 + 64 + h * NV, v);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(TME + a));
       uint8_t* so = sO + a * C::A_BYTES;
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4)
-        st_sw128(so, row, h * 4 + c4,
-                 make_uint4(pack_bf16x2(__uint_as_float(v[8 * c4 + 0]), __uint_as_float(v[8 * c4 + 1])),
-                            pack_bf16x2(__uint_as_float(v[8 * c4 + 2]), __uint_as_float(v[8 * c4 + 3])),
-                            pack_bf16x2(__uint_as_float(v[8 * c4 + 4]), __uint_as_float(v[8 * c4 + 5])),
-                            pack_bf16x2(__uint_as_float(v[8 * c4 + 6]), __uint_as_float(v[8 * c4 + 7]))));
+      for (int c8 = 0; c8 < NV / 8; ++c8)
+        st_sw128(so, row, h * (NV / 8) + c8,
+                 make_uint4(pack_bf16x2(__uint_as_float(v[8 * c8 + 0]), __uint_as_float(v[8 * c8 + 1])),
+                            pack_bf16x2(__uint_as_float(v[8 * c8 + 2]), __uint_as_float(v[8 * c8 + 3])),
+                            pack_bf16x2(__uint_as_float(v[8 * c8 + 4]), __uint_as_float(v[8 * c8 + 5])),
+                            pack_bf16x2(__uint_as_float(v[8 * c8 + 6]), __uint_as_float(v[8 * c8 + 7]))));
       fence_async_smem();
       named_sync(1, C::EPI);
       if (leader) {
@@ -1288,23 +1312,26 @@ permute_mask_tc2_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_co
 // dP product; warps 2-9 (two per TMEM lane quadrant, 32 columns each) turn
 // W', dA and the mask into the bf16 operands.  The dP accumulator stays in
 // TMEM for the whole segment and is written once at the end.
-struct BwCfg {
+template <int NSL> struct BwCfg {
   static constexpr int STAGES = 3;
   static constexpr int T_BYTES = 16384;                  // 128 rows x 64 bf16
   static constexpr int STAGE = 2 * T_BYTES;              // dAt | W (adjacent: stacked A operand)
   static constexpr int IMG_BYTES = 8192;
   static constexpr int SMEM = STAGES * STAGE + 2 * IMG_BYTES + 2 * (2 * T_BYTES) + 1024 + 256;
-  static constexpr int THREADS = 320;
-  static constexpr int EPI = 256;
+  static constexpr int EPI_WARPS = 4 * NSL;              // NSL column slices per TMEM lane quadrant
+  static constexpr int COLS = 64 / NSL;
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+  static constexpr int EPI = 32 * EPI_WARPS;
 };
 
-template <int B>
-__global__ void __launch_bounds__(BwCfg::THREADS, 1)
+template <int B, int NSL>
+__global__ void __launch_bounds__(BwCfg<NSL>::THREADS, 1)
 block_bwd_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmDAt,
                     const __grid_constant__ CUtensorMap tmPth, const __grid_constant__ CUtensorMap tmPtl,
                     const uint32_t* __restrict__ mask, float* __restrict__ dP, int cout, int cin,
                     int rows_per_split) {
-  using C = BwCfg;
+  using C = BwCfg<NSL>;
+  constexpr int NV = C::COLS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sStage = smem;
@@ -1328,7 +1355,7 @@ block_bwd_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_consta
     for (int i = 0; i < 3; ++i) { mbar_init(bar(FULL + i), 1); mbar_init(bar(EMPTY + i), 1); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(WD + i), 1);
-      mbar_init(bar(ABF + i), 8);
+      mbar_init(bar(ABF + i), C::EPI_WARPS);
       mbar_init(bar(ABE + i), 1);
     }
     mbar_init(bar(DPF), 1);
@@ -1420,27 +1447,29 @@ block_bwd_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_consta
     }
     __syncwarp();
   } else {
-    const int e = warp - 2, q = warp & 3, h = e >> 2;
+    const int e = warp - 2, q = warp & 3, h = e >> 2;   // h: column slice of NV columns
     const int row = q * 32 + lane;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     bool ok = true;
-    // mask words run one chunk ahead of the chunk being processed
-    auto mask_word = [&](int c) -> uint32_t {
+    // mask bits of this thread's NV columns, one chunk ahead of the chunk being processed
+    auto mask_bits = [&](int c) -> uint32_t {
       const int grow = rbeg + c * 128 + row;
-      return (c < nchunk && grow < rend) ? __ldg(mask + (size_t)grow * words + col0 / 32 + h) : 0u;
+      if (c >= nchunk || grow >= rend) return 0u;
+      const uint32_t w = __ldg(mask + (size_t)grow * words + col0 / 32 + (h * NV) / 32);
+      return NV == 32 ? w : (w >> ((h * NV) % 32)) & ((1u << NV) - 1u);
     };
-    uint32_t next_bits = mask_word(0);
+    uint32_t next_bits = mask_bits(0);
     for (int c = 0; c < nchunk; ++c) {
       const int a = c & 1;
       const uint32_t ua = (uint32_t)(c >> 1) & 1u;
       const uint32_t bits = next_bits;
-      next_bits = mask_word(c + 1);
+      next_bits = mask_bits(c + 1);
       ok = named_and(1, C::EPI, mbar_wait(bar(WD + a), ua, abort_flag, 79));
       if (!ok) break;
       tc_fence_after();
-      uint32_t wv[32], dv[32];
-      tmem_ld32(tmem + lane_off + a * 128 + h * 32, wv);
-      tmem_ld32(tmem + lane_off + a * 128 + 64 + h * 32, dv);
+      uint32_t wv[NV], dv[NV];
+      tmem_ld_cols<NV>(tmem + lane_off + a * 128 + h * NV, wv);
+      tmem_ld_cols<NV>(tmem + lane_off + a * 128 + 64 + h * NV, dv);
       tmem_ld_wait();
       // buffer a was last read by the dP product of chunk c - 2
       ok = named_and(1, C::EPI, c < 2 || mbar_wait(bar(ABE + a), ua ^ 1u, abort_flag, 80));
@@ -1448,18 +1477,19 @@ block_bwd_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_consta
       uint8_t* rA = sAB + a * 2 * C::T_BYTES;
       uint8_t* rD = rA + C::T_BYTES;
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
+      for (int c8 = 0; c8 < NV / 8; ++c8) {
         float fa[8], fd[8];
 #pragma unroll
         for (int x = 0; x < 8; ++x) {
-          const bool keep = (bits >> (8 * c4 + x)) & 1u;
-          fa[x] = keep ? __uint_as_float(wv[8 * c4 + x]) : 0.f;
-          fd[x] = keep ? __uint_as_float(dv[8 * c4 + x]) : 0.f;
+          const bool keep = (bits >> (8 * c8 + x)) & 1u;
+          fa[x] = keep ? __uint_as_float(wv[8 * c8 + x]) : 0.f;
+          fd[x] = keep ? __uint_as_float(dv[8 * c8 + x]) : 0.f;
         }
-        st_sw128(rA, row, h * 4 + c4, make_uint4(pack_bf16x2(fa[0], fa[1]), pack_bf16x2(fa[2], fa[3]),
-                                                 pack_bf16x2(fa[4], fa[5]), pack_bf16x2(fa[6], fa[7])));
-        st_sw128(rD, row, h * 4 + c4, make_uint4(pack_bf16x2(fd[0], fd[1]), pack_bf16x2(fd[2], fd[3]),
-                                                 pack_bf16x2(fd[4], fd[5]), pack_bf16x2(fd[6], fd[7])));
+        const int chunk = h * (NV / 8) + c8;
+        st_sw128(rA, row, chunk, make_uint4(pack_bf16x2(fa[0], fa[1]), pack_bf16x2(fa[2], fa[3]),
+                                            pack_bf16x2(fa[4], fa[5]), pack_bf16x2(fa[6], fa[7])));
+        st_sw128(rD, row, chunk, make_uint4(pack_bf16x2(fd[0], fd[1]), pack_bf16x2(fd[2], fd[3]),
+                                            pack_bf16x2(fd[4], fd[5]), pack_bf16x2(fd[6], fd[7])));
       }
       fence_async_smem();
       tc_fence_before();
@@ -1470,24 +1500,24 @@ block_bwd_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_consta
     if (ok) {
       tc_fence_after();
       // rows 0..63 hold dAt^T A (columns 0..63), rows 64..127 W^T dW' (columns 64..127)
-      uint32_t v[32];
-      const uint32_t cbase = (row < 64 ? 0u : 64u) + h * 32;
-      tmem_ld32(tDP + lane_off + cbase, v);
+      uint32_t v[NV];
+      const uint32_t cbase = (row < 64 ? 0u : 64u) + h * NV;
+      tmem_ld_cols<NV>(tDP + lane_off + cbase, v);
       tmem_ld_wait();
       float* scratch = reinterpret_cast<float*>(sAB);   // 64 x 64 floats; every MMA is done
       if (row >= 64) {
 #pragma unroll
-        for (int x = 0; x < 32; ++x) scratch[(row - 64) * 64 + h * 32 + x] = __uint_as_float(v[x]);
+        for (int x = 0; x < NV; ++x) scratch[(row - 64) * 64 + h * NV + x] = __uint_as_float(v[x]);
       }
       named_sync(1, C::EPI);
       if (row < 64) {
         const int nb = cin / B;
         float* dPs = dP + (size_t)sidx * nb * B * B;
-        const float* add = scratch + row * 64 + h * 32;
+        const float* add = scratch + row * 64 + h * NV;
         if constexpr (B == 64) {
-          float4* o = reinterpret_cast<float4*>(dPs + ((size_t)t * 64 + row) * 64 + h * 32);
+          float4* o = reinterpret_cast<float4*>(dPs + ((size_t)t * 64 + row) * 64 + h * NV);
 #pragma unroll
-          for (int qq = 0; qq < 8; ++qq)
+          for (int qq = 0; qq < NV / 4; ++qq)
             o[qq] = make_float4(__uint_as_float(v[4 * qq]) + add[4 * qq], __uint_as_float(v[4 * qq + 1]) + add[4 * qq + 1],
                                 __uint_as_float(v[4 * qq + 2]) + add[4 * qq + 2],
                                 __uint_as_float(v[4 * qq + 3]) + add[4 * qq + 3]);
@@ -1495,10 +1525,10 @@ block_bwd_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_consta
           // B = 32: the tile holds blocks 2t (rows/columns 0..31) and 2t+1 (32..63);
           // keep only the diagonal quadrants
           const int qb = row / 32;
-          if (h == qb) {
-            float* o = dPs + ((size_t)(2 * t + qb) * 32 + (row - 32 * qb)) * 32;
+          if ((h * NV) / 32 == qb) {
+            float* o = dPs + ((size_t)(2 * t + qb) * 32 + (row - 32 * qb)) * 32 + (h * NV) % 32;
 #pragma unroll
-            for (int x = 0; x < 32; ++x) o[x] = __uint_as_float(v[x]) + add[x];
+            for (int x = 0; x < NV; ++x) o[x] = __uint_as_float(v[x]) + add[x];
           }
         }
       }
@@ -1934,11 +1964,13 @@ lcp_status launch_permute_mask_tc(const __nv_bfloat16* W, const __nv_bfloat16* i
   if (BC == 64) {
     CUtensorMap mAt;
     TC_TRY(make_map(&mAt, At, cin, cout, 64, 128, "permute_mask At"));
-    auto k = (m == 4) ? permute_mask_ws_kernel<4> : permute_mask_ws_kernel<8>;
-    TC_TRY(set_smem(k, PwCfg::SMEM, "permute_mask_tc"));
+    constexpr int NSL = 4;
+    using C = PwCfg<NSL>;
+    auto k = (m == 4) ? permute_mask_ws_kernel<4, NSL> : permute_mask_ws_kernel<8, NSL>;
+    TC_TRY(set_smem(k, C::SMEM, "permute_mask_tc"));
     const int tiles = cdiv(cout, 128) * (cin / 64);
     const int grid = tiles < num_sms() ? tiles : num_sms();
-    k<<<grid, PwCfg::THREADS, PwCfg::SMEM, st>>>(mW, mPth, mPtl, mPh, mAt, mask, Wp_out, cout, cin, n);
+    k<<<grid, C::THREADS, C::SMEM, st>>>(mW, mPth, mPtl, mPh, mAt, mask, Wp_out, cout, cin, n);
     return check_launch("permute_mask_tc");
   }
   if (m == 4) {
@@ -1962,10 +1994,11 @@ lcp_status launch_block_bwd_tc(const __nv_bfloat16* W, const __nv_bfloat16* dAt,
   TC_TRY(make_map(&mPth, img_pt_hi, BC, cin, 64, BC, "block_bwd Pt_hi"));
   TC_TRY(make_map(&mPtl, img_pt_lo, BC, cin, 64, BC, "block_bwd Pt_lo"));
   if (B <= 64) {
-    auto k = (B == 32) ? block_bwd_ws_kernel<32> : block_bwd_ws_kernel<64>;
-    TC_TRY(set_smem(k, BwCfg::SMEM, "block_bwd_tc"));
-    k<<<dim3(cin / 64, splits), BwCfg::THREADS, BwCfg::SMEM, st>>>(mW, mD, mPth, mPtl, mask, dP_partials, cout,
-                                                                   cin, rows);
+    constexpr int NSL = 4;
+    using C = BwCfg<NSL>;
+    auto k = (B == 32) ? block_bwd_ws_kernel<32, NSL> : block_bwd_ws_kernel<64, NSL>;
+    TC_TRY(set_smem(k, C::SMEM, "block_bwd_tc"));
+    k<<<dim3(cin / 64, splits), C::THREADS, C::SMEM, st>>>(mW, mD, mPth, mPtl, mask, dP_partials, cout, cin, rows);
     return check_launch("block_bwd_tc");
   }
   return block_bwd_bc<128, 128>(mW, mD, mPth, mPtl, mask, dP_partials, splits, rows, cout, cin, st);
