@@ -236,8 +236,8 @@ def main():
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
 
-    wl = workload(args.workload)
-    wl.seed = rank
+    from learnable_channel_permutation_b200 import parallel
+    wl = parallel.rank_workload(workload(args.workload), rank)   # each rank: its own layer
     li = synth.make_inputs(wl)[0]
     tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
     W = torch.from_numpy(li.W).to(dev).to(tdt)
@@ -305,14 +305,11 @@ def main():
     if graph_mode:
         eager_total, _ = timed_loop(False)
 
-    t = torch.tensor([total_ms, eager_total or 0.0], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    max_ms = float(t[0].item())
-    value = world * K / (max_ms / 1e3)
+    max_ms, max_eager = parallel.max_over_ranks([total_ms, eager_total or 0.0], device=dev)
+    value = parallel.job_throughput(K, world, max_ms)
     eager = None
     if eager_total is not None:
-        eager = {"value": world * K / (float(t[1].item()) / 1e3), "ms_per_step": float(t[1].item()) / K}
+        eager = {"value": parallel.job_throughput(K, world, max_eager), "ms_per_step": max_eager / K}
 
     # end to end through the public API: pinned host inputs in, loss and dL out, every step
     e2e = None
@@ -339,12 +336,10 @@ def main():
                 a1[kk].record(stream)
             stream.synchronize()
         e_ms = sum(a0[k].elapsed_time(a1[k]) for k in range(Ke))
-        te = torch.tensor([e_ms / Ke], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        (te_ms,) = parallel.max_over_ranks([e_ms / Ke], device=dev)
         h2d = hW.numel() * hW.element_size() + hX.numel() * hX.element_size() + hL.numel() * 4
         d2h = 4 * 4 + hdL.numel() * 4
-        e2e = {"value": world / (float(te.item()) / 1e3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+        e2e = {"value": parallel.job_throughput(1, world, te_ms), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h)}
 
     if world > 1:

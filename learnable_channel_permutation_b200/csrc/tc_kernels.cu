@@ -1964,7 +1964,7 @@ lcp_status launch_permute_mask_tc(const __nv_bfloat16* W, const __nv_bfloat16* i
   if (BC == 64) {
     CUtensorMap mAt;
     TC_TRY(make_map(&mAt, At, cin, cout, 64, 128, "permute_mask At"));
-    constexpr int NSL = 4;
+    constexpr int NSL = 2;
     using C = PwCfg<NSL>;
     auto k = (m == 4) ? permute_mask_ws_kernel<4, NSL> : permute_mask_ws_kernel<8, NSL>;
     TC_TRY(set_smem(k, C::SMEM, "permute_mask_tc"));
@@ -1994,7 +1994,7 @@ lcp_status launch_block_bwd_tc(const __nv_bfloat16* W, const __nv_bfloat16* dAt,
   TC_TRY(make_map(&mPth, img_pt_hi, BC, cin, 64, BC, "block_bwd Pt_hi"));
   TC_TRY(make_map(&mPtl, img_pt_lo, BC, cin, 64, BC, "block_bwd Pt_lo"));
   if (B <= 64) {
-    constexpr int NSL = 4;
+    constexpr int NSL = 2;
     using C = BwCfg<NSL>;
     auto k = (B == 32) ? block_bwd_ws_kernel<32, NSL> : block_bwd_ws_kernel<64, NSL>;
     TC_TRY(set_smem(k, C::SMEM, "block_bwd_tc"));
