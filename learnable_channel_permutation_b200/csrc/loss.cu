@@ -106,75 +106,90 @@ loss_grad_kernel(const float* __restrict__ Yd, const float* __restrict__ Ys,
                  G, row, cout / 4, s.x, s.y, s.z, inv_T);
 }
 
-// Fused variant used inside a step: one CTA per token keeps the token's two
-// rows in registers (QPT float4 quads per thread), so Y is read from HBM once;
-// the CTA that finishes last (a counter that the caller zeroes before the
-// launch) sums the T cosines in index order into the loss and re-zeroes the
-// counter.  Deterministic: the order of the final sum never depends on timing.
-template <typename TG, int NTH, int QPT>
-__global__ void __launch_bounds__(NTH)
+// Fused variant used inside a step.  Persistent CTAs walk the tokens
+// t = blockIdx.x, blockIdx.x + gridDim.x, ...; each thread keeps QPT float4
+// quads of the current token's two rows in registers and already holds the
+// next token's rows (loaded while the current one is reduced), so Y is read
+// from HBM once with the loads always in flight.  The CTA that finishes last
+// (a counter zeroed by the caller before the launch) sums the T cosines in
+// index order into the loss and re-zeroes the counter: deterministic.
+template <typename TG, int NTH, int QPT, bool PREFETCH>
+__global__ void __launch_bounds__(NTH, PREFETCH ? 2 : 1)
 loss_fused_kernel(const float* __restrict__ Yd, const float* __restrict__ Ys, float* __restrict__ stats,
                   TG* __restrict__ G, float* __restrict__ loss, unsigned* __restrict__ counter, int cout,
                   int tokens, float inv_T) {
   constexpr int NWARP = NTH / 32;
-  __shared__ float red[3][NWARP];
+  __shared__ float red[2][3][NWARP];
   __shared__ double redd[NWARP];
   __shared__ int is_last;
-  const int t = blockIdx.x;
-  const size_t row = (size_t)t * cout;
-  const float4* yd = reinterpret_cast<const float4*>(Yd + row);
-  const float4* ys = reinterpret_cast<const float4*>(Ys + row);
   const int quads = cout / 4;
-  float4 a[QPT], b[QPT];
-#pragma unroll
-  for (int i = 0; i < QPT; ++i) {
-    const int q = threadIdx.x + i * NTH;
-    if (q < quads) { a[i] = yd[q]; b[i] = ys[q]; }
-    else { a[i] = make_float4(0.f, 0.f, 0.f, 0.f); b[i] = a[i]; }
-  }
-  float dot = 0.f, nd = 0.f, ns = 0.f;
-#pragma unroll
-  for (int i = 0; i < QPT; ++i) {
-    dot += a[i].x * b[i].x + a[i].y * b[i].y + a[i].z * b[i].z + a[i].w * b[i].w;
-    nd += a[i].x * a[i].x + a[i].y * a[i].y + a[i].z * a[i].z + a[i].w * a[i].w;
-    ns += b[i].x * b[i].x + b[i].y * b[i].y + b[i].z * b[i].z + b[i].w * b[i].w;
-  }
-  dot = warp_sum(dot);
-  nd = warp_sum(nd);
-  ns = warp_sum(ns);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  if (lane == 0) { red[0][warp] = dot; red[1][warp] = nd; red[2][warp] = ns; }
-  __syncthreads();
-  dot = 0.f; nd = 0.f; ns = 0.f;
+  float4 a[QPT], b[QPT], na[QPT], nb[QPT];
+  auto load = [&](int t, float4 (&x)[QPT], float4 (&y)[QPT]) {
+    const float4* yd = reinterpret_cast<const float4*>(Yd + (size_t)t * cout);
+    const float4* ys = reinterpret_cast<const float4*>(Ys + (size_t)t * cout);
 #pragma unroll
-  for (int w = 0; w < NWARP; ++w) { dot += red[0][w]; nd += red[1][w]; ns += red[2][w]; }
-  const float den = sqrtf(nd) * sqrtf(ns);
-  const float c = dot / fmaxf(den, kCosEps);
-  if (threadIdx.x == 0) {
-    float4 sv;
-    sv.x = dot; sv.y = nd; sv.z = ns; sv.w = c;
-    reinterpret_cast<float4*>(stats)[t] = sv;
-  }
-  const bool ok = den > kCosEps;
-  const float ca = ok ? -inv_T / den : -inv_T / kCosEps;
-  const float cb = ok ? inv_T * c / ns : 0.f;
+    for (int i = 0; i < QPT; ++i) {
+      const int q = threadIdx.x + i * NTH;
+      if (t < tokens && q < quads) { x[i] = __ldcs(yd + q); y[i] = __ldcs(ys + q); }
+      else { x[i] = make_float4(0.f, 0.f, 0.f, 0.f); y[i] = x[i]; }
+    }
+  };
+  int t = blockIdx.x;
+  if constexpr (PREFETCH) load(t, na, nb);
+  for (int it = 0; t < tokens; t += gridDim.x, ++it) {
+    if constexpr (PREFETCH) {
 #pragma unroll
-  for (int i = 0; i < QPT; ++i) {
-    const int q = threadIdx.x + i * NTH;
-    if (q < quads) {
-      float4 g;
-      g.x = ca * a[i].x + cb * b[i].x;
-      g.y = ca * a[i].y + cb * b[i].y;
-      g.z = ca * a[i].z + cb * b[i].z;
-      g.w = ca * a[i].w + cb * b[i].w;
-      write_g<TG>(G, row + 4 * (size_t)q, g);
+      for (int i = 0; i < QPT; ++i) { a[i] = na[i]; b[i] = nb[i]; }
+      load(t + gridDim.x, na, nb);          // next token, in flight during this one
+    } else {
+      load(t, a, b);
+    }
+    float dot = 0.f, nd = 0.f, ns = 0.f;
+#pragma unroll
+    for (int i = 0; i < QPT; ++i) {
+      dot += a[i].x * b[i].x + a[i].y * b[i].y + a[i].z * b[i].z + a[i].w * b[i].w;
+      nd += a[i].x * a[i].x + a[i].y * a[i].y + a[i].z * a[i].z + a[i].w * a[i].w;
+      ns += b[i].x * b[i].x + b[i].y * b[i].y + b[i].z * b[i].z + b[i].w * b[i].w;
+    }
+    dot = warp_sum(dot);
+    nd = warp_sum(nd);
+    ns = warp_sum(ns);
+    const int p = it & 1;   // double-buffered partials: one barrier per token
+    if (lane == 0) { red[p][0][warp] = dot; red[p][1][warp] = nd; red[p][2][warp] = ns; }
+    __syncthreads();
+    dot = 0.f; nd = 0.f; ns = 0.f;
+#pragma unroll
+    for (int w = 0; w < NWARP; ++w) { dot += red[p][0][w]; nd += red[p][1][w]; ns += red[p][2][w]; }
+    const float den = sqrtf(nd) * sqrtf(ns);
+    const float c = dot / fmaxf(den, kCosEps);
+    if (threadIdx.x == 0) {
+      float4 sv;
+      sv.x = dot; sv.y = nd; sv.z = ns; sv.w = c;
+      reinterpret_cast<float4*>(stats)[t] = sv;
+    }
+    const bool ok = den > kCosEps;
+    const float ca = ok ? -inv_T / den : -inv_T / kCosEps;
+    const float cb = ok ? inv_T * c / ns : 0.f;
+    const size_t row = (size_t)t * cout;
+#pragma unroll
+    for (int i = 0; i < QPT; ++i) {
+      const int q = threadIdx.x + i * NTH;
+      if (q < quads) {
+        float4 g;
+        g.x = ca * a[i].x + cb * b[i].x;
+        g.y = ca * a[i].y + cb * b[i].y;
+        g.z = ca * a[i].z + cb * b[i].z;
+        g.w = ca * a[i].w + cb * b[i].w;
+        write_g<TG>(G, row + 4 * (size_t)q, g);
+      }
     }
   }
-  // last CTA: the loss.  Thread 0 wrote this token's statistics; its fence
-  // orders that write before its vote, so the last voter sees every token.
+  // last CTA: the loss.  Thread 0 wrote this CTA's statistics; its fence
+  // orders those writes before its vote, so the last voter sees every token.
   if (threadIdx.x == 0) {
     __threadfence();
-    is_last = (atomicAdd(counter, 1u) == (unsigned)tokens - 1u);
+    is_last = (atomicAdd(counter, 1u) == gridDim.x - 1u);
   }
   __syncthreads();
   if (!is_last) return;
@@ -246,9 +261,13 @@ lcp_status launch_loss_fused(const float* Yd, const float* Ys, float* stats, voi
     return fail(LCP_ERR_CUDA, "loss counter reset: %s", cudaGetErrorString(e));
   }
   const int quads = cout / 4;
-#define LCP_LOSS_FUSED(TG, NTH, QPT)                                                                  \
-  loss_fused_kernel<TG, NTH, QPT><<<tokens, NTH, 0, st>>>(Yd, Ys, stats, static_cast<TG*>(G), loss,   \
-                                                           counter, cout, tokens, inv_T)
+  int sms = 148, dev = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = tokens < 2 * sms ? tokens : 2 * sms;
+#define LCP_LOSS_FUSED(TG, NTH, QPT)                                                                \
+  loss_fused_kernel<TG, NTH, QPT, (QPT <= 4)><<<grid, NTH, 0, st>>>(Yd, Ys, stats, static_cast<TG*>(G), \
+                                                                    loss, counter, cout, tokens, inv_T)
   if (gdt == LCP_F32) {
     if (quads <= 4 * 256) LCP_LOSS_FUSED(float, 256, 4);
     else if (quads <= 8 * 256) LCP_LOSS_FUSED(float, 256, 8);

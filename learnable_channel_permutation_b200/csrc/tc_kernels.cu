@@ -925,15 +925,16 @@ permute_mask_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
   uint8_t* sA = smem + C::STAGES * C::STAGE;          // 2 buffers
   uint8_t* sO = sA + 2 * C::A_BYTES;                  // 2 staging tiles for At
   uint64_t* bars = reinterpret_cast<uint64_t*>(sO + 2 * C::A_BYTES);
-  // bars: full[3] empty[3] wf[2] af[2] atf[2] tme[2] drain
-  uint32_t* holder = reinterpret_cast<uint32_t*>(bars + 15);
+  // bars: full[3] empty[3] wf[2] af[2] atf[2] tmw[2] tma[2] drain
+  uint32_t* holder = reinterpret_cast<uint32_t*>(bars + 17);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(holder + 1);
   auto bar = [&](int i) { return smem_u32(bars + i); };
-  const int FULL = 0, EMPTY = 3, WF = 6, AF = 8, ATF = 10, TME = 12, DRAIN = 14;
+  const int FULL = 0, EMPTY = 3, WF = 6, AF = 8, ATF = 10, TMW = 12, TMA = 14, DRAIN = 16;
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int nrt = cdiv(cout, 128), ntc = cin / 64;
   const int total = nrt * ntc;
+  const int nloc = (int)blockIdx.x < total ? cdiv(total - (int)blockIdx.x, (int)gridDim.x) : 0;
   const int words = cin / 32;
   if (threadIdx.x == 0) {
     for (int i = 0; i < 3; ++i) { mbar_init(bar(FULL + i), 1); mbar_init(bar(EMPTY + i), 1); }
@@ -941,7 +942,8 @@ permute_mask_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
       mbar_init(bar(WF + i), 1);
       mbar_init(bar(AF + i), C::EPI_WARPS);
       mbar_init(bar(ATF + i), 1);
-      mbar_init(bar(TME + i), C::EPI_WARPS);
+      mbar_init(bar(TMW + i), C::EPI_WARPS);
+      mbar_init(bar(TMA + i), C::EPI_WARPS);
     }
     mbar_init(bar(DRAIN), 1);
     *abort_flag = 0;
@@ -952,16 +954,21 @@ permute_mask_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *holder;
+  auto tile_of = [&](int k, int& t, int& rt) {
+    const int idx = (int)blockIdx.x + k * (int)gridDim.x;
+    t = idx / nrt;
+    rt = idx % nrt;
+  };
 
   if (warp == 0) {
     if (lane == 0) {
-      int k = 0;
       uint32_t issued = 0, par = 0;   // per stage: outstanding load and its parity
-      for (int idx = blockIdx.x; idx < total; idx += gridDim.x, ++k) {
+      for (int k = 0; k < nloc; ++k) {
         const int st = k % C::STAGES;
         const uint32_t use = (uint32_t)(k / C::STAGES) & 1u;
         if (!mbar_wait(bar(EMPTY + st), use ^ 1u, abort_flag, 61)) break;
-        const int t = idx / nrt, rt = idx % nrt;
+        int t, rt;
+        tile_of(k, t, rt);
         uint8_t* sg = sStage + st * C::STAGE;
         mbar_expect_tx(bar(FULL + st), C::STAGE);
         tma_load_2d(smem_u32(sg), &tmW, bar(FULL + st), t * 64, rt * 128);
@@ -978,13 +985,12 @@ permute_mask_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16(128, 64, false, false);
-      const int nloc = blockIdx.x < total ? cdiv(total - blockIdx.x, gridDim.x) : 0;
-      // W' = W (P_hi + P_lo) of local tile k into TMEM buffer k & 1
+      // W' = W (P_hi + P_lo) of local tile k into the W' half of TMEM buffer k & 1
       auto mma1 = [&](int k) -> bool {
         const int st = k % C::STAGES, a = k & 1;
         const uint32_t use = (uint32_t)(k / C::STAGES) & 1u, ua = (uint32_t)(k >> 1) & 1u;
         if (!mbar_wait(bar(FULL + st), use, abort_flag, 63)) return false;
-        if (!mbar_wait(bar(TME + a), ua ^ 1u, abort_flag, 64)) return false;
+        if (!mbar_wait(bar(TMW + a), ua ^ 1u, abort_flag, 64)) return false;   // W' of tile k - 2 read
         tc_fence_after();
         const uint32_t sg = smem_u32(sStage + st * C::STAGE);
         const uint32_t dW = tmem + a * 128;
@@ -1004,7 +1010,8 @@ permute_mask_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
         const int st = k % C::STAGES, a = k & 1;
         const uint32_t ua = (uint32_t)(k >> 1) & 1u;
         if (k + 1 < nloc && !mma1(k + 1)) break;
-        if (!mbar_wait(bar(AF + a), ua, abort_flag, 65)) break;
+        if (!mbar_wait(bar(AF + a), ua, abort_flag, 65)) break;        // A of tile k in shared memory
+        if (!mbar_wait(bar(TMA + a), ua ^ 1u, abort_flag, 69)) break;  // At of tile k - 2 read
         tc_fence_after();
         const uint32_t sg = smem_u32(sStage + st * C::STAGE);
         const uint32_t sa = smem_u32(sA + a * C::A_BYTES);
@@ -1021,73 +1028,86 @@ permute_mask_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
     }
     __syncwarp();
   } else {
+    // Software-pipelined epilogue: in step k the warps first turn W' of tile k
+    // into the mask and A (so the MMA warp can start At of tile k), then copy
+    // out At of tile k - 1, whose product ran meanwhile.
     const int e = warp - 2, q = warp & 3, h = e >> 2;   // h: column slice of NV columns
     const int row = q * 32 + lane;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     const bool leader = (e == 0 && lane == 0);
-    int k = 0;
-    for (int idx = blockIdx.x; idx < total; idx += gridDim.x, ++k) {
-      const int a = k & 1;
-      const uint32_t ua = (uint32_t)(k >> 1) & 1u;
-      const int t = idx / nrt, rt = idx % nrt;
-      const int grow = rt * 128 + row;
-      if (!named_and(1, C::EPI, mbar_wait(bar(WF + a), ua, abort_flag, 67))) break;
-      tc_fence_after();
-      uint32_t v[NV];
-      tmem_ld_cols<NV>(tmem + lane_off + a * 128 + h * NV, v);
-      tmem_ld_wait();
-      const uint32_t w = nm_bits<MGROUP, NV>(v, n);
-      if (grow < cout) {
-        if constexpr (NV == 32) {
-          mask[(size_t)grow * words + 2 * t + h] = w;
-        } else {
-          reinterpret_cast<uint16_t*>(mask)[((size_t)grow * words + 2 * t) * 2 + h] = (uint16_t)w;
+    for (int k = 0; k <= nloc; ++k) {
+      if (k < nloc) {
+        const int a = k & 1;
+        const uint32_t ua = (uint32_t)(k >> 1) & 1u;
+        int t, rt;
+        tile_of(k, t, rt);
+        const int grow = rt * 128 + row;
+        if (!named_and(1, C::EPI, mbar_wait(bar(WF + a), ua, abort_flag, 67))) break;
+        tc_fence_after();
+        uint32_t v[NV];
+        tmem_ld_cols<NV>(tmem + lane_off + a * 128 + h * NV, v);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(TMW + a));
+        const uint32_t w = nm_bits<MGROUP, NV>(v, n);
+        if (grow < cout) {
+          if constexpr (NV == 32) {
+            mask[(size_t)grow * words + 2 * t + h] = w;
+          } else {
+            reinterpret_cast<uint16_t*>(mask)[((size_t)grow * words + 2 * t) * 2 + h] = (uint16_t)w;
+          }
+          if (Wp_out) {
+            float4* o = reinterpret_cast<float4*>(Wp_out + (size_t)grow * cin + t * 64 + h * NV);
+#pragma unroll
+            for (int qq = 0; qq < NV / 4; ++qq)
+              o[qq] = make_float4(__uint_as_float(v[4 * qq]), __uint_as_float(v[4 * qq + 1]),
+                                  __uint_as_float(v[4 * qq + 2]), __uint_as_float(v[4 * qq + 3]));
+          }
         }
-        if (Wp_out) {
-          float4* o = reinterpret_cast<float4*>(Wp_out + (size_t)grow * cin + t * 64 + h * NV);
+        uint8_t* sa = sA + a * C::A_BYTES;
 #pragma unroll
-          for (int qq = 0; qq < NV / 4; ++qq)
-            o[qq] = make_float4(__uint_as_float(v[4 * qq]), __uint_as_float(v[4 * qq + 1]),
-                                __uint_as_float(v[4 * qq + 2]), __uint_as_float(v[4 * qq + 3]));
+        for (int c8 = 0; c8 < NV / 8; ++c8) {
+          float f[8];
+#pragma unroll
+          for (int x = 0; x < 8; ++x) f[x] = ((w >> (8 * c8 + x)) & 1u) ? __uint_as_float(v[8 * c8 + x]) : 0.f;
+          st_sw128(sa, row, h * (NV / 8) + c8, make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                                                          pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7])));
         }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(AF + a));
       }
-      uint8_t* sa = sA + a * C::A_BYTES;
+      if (k > 0) {
+        const int kp = k - 1, a = kp & 1;
+        const uint32_t ua = (uint32_t)(kp >> 1) & 1u;
+        int t, rt;
+        tile_of(kp, t, rt);
+        const bool got = mbar_wait(bar(ATF + a), ua, abort_flag, 68);
+        // the staging tile of two tiles ago must have been read out by its TMA store
+        if (leader) bulk_wait_read<1>();
+        if (!named_and(1, C::EPI, got)) break;
+        tc_fence_after();
+        uint32_t v[NV];
+        tmem_ld_cols<NV>(tmem + lane_off + a * 128 + 64 + h * NV, v);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(TMA + a));
+        uint8_t* so = sO + a * C::A_BYTES;
 #pragma unroll
-      for (int c8 = 0; c8 < NV / 8; ++c8) {
-        float f[8];
-#pragma unroll
-        for (int x = 0; x < 8; ++x) f[x] = ((w >> (8 * c8 + x)) & 1u) ? __uint_as_float(v[8 * c8 + x]) : 0.f;
-        st_sw128(sa, row, h * (NV / 8) + c8, make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
-                                                        pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7])));
-      }
-      fence_async_smem();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(AF + a));
-      // At of this tile
-      const bool got = mbar_wait(bar(ATF + a), ua, abort_flag, 68);
-      // the staging tile of two tiles ago must have been read out by its TMA store
-      if (leader) bulk_wait_read<1>();
-      if (!named_and(1, C::EPI, got)) break;
-      tc_fence_after();
-      tmem_ld_cols<NV>(tmem + lane_off + a * 128 + 64 + h * NV, v);
-      tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(TME + a));
-      uint8_t* so = sO + a * C::A_BYTES;
-#pragma unroll
-      for (int c8 = 0; c8 < NV / 8; ++c8)
-        st_sw128(so, row, h * (NV / 8) + c8,
-                 make_uint4(pack_bf16x2(__uint_as_float(v[8 * c8 + 0]), __uint_as_float(v[8 * c8 + 1])),
-                            pack_bf16x2(__uint_as_float(v[8 * c8 + 2]), __uint_as_float(v[8 * c8 + 3])),
-                            pack_bf16x2(__uint_as_float(v[8 * c8 + 4]), __uint_as_float(v[8 * c8 + 5])),
-                            pack_bf16x2(__uint_as_float(v[8 * c8 + 6]), __uint_as_float(v[8 * c8 + 7]))));
-      fence_async_smem();
-      named_sync(1, C::EPI);
-      if (leader) {
-        tma_store_2d(&tmAt, smem_u32(so), t * 64, rt * 128);
-        bulk_commit();
+        for (int c8 = 0; c8 < NV / 8; ++c8)
+          st_sw128(so, row, h * (NV / 8) + c8,
+                   make_uint4(pack_bf16x2(__uint_as_float(v[8 * c8 + 0]), __uint_as_float(v[8 * c8 + 1])),
+                              pack_bf16x2(__uint_as_float(v[8 * c8 + 2]), __uint_as_float(v[8 * c8 + 3])),
+                              pack_bf16x2(__uint_as_float(v[8 * c8 + 4]), __uint_as_float(v[8 * c8 + 5])),
+                              pack_bf16x2(__uint_as_float(v[8 * c8 + 6]), __uint_as_float(v[8 * c8 + 7]))));
+        fence_async_smem();
+        named_sync(1, C::EPI);
+        if (leader) {
+          tma_store_2d(&tmAt, smem_u32(so), t * 64, rt * 128);
+          bulk_commit();
+        }
       }
     }
     if (leader) bulk_wait_all();
