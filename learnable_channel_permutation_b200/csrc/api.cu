@@ -117,7 +117,7 @@ lcp_status check_hparams(const lcp_hparams* hp) {
 }
 
 bool use_tc(const lcp_hparams& hp) {
-  return hp.dtype == LCP_BF16 && !(hp.flags & LCP_FLAG_SIMT) && tc_available();
+  return hp.dtype == LCP_BF16 && !(hp.flags & LCP_FLAG_SIMT);
 }
 
 lcp_status check_layer(const lcp_layer& l, const lcp_hparams& hp, int idx) {
@@ -543,3 +543,18 @@ lcp_status lcp_loss_bwd(const float* Yd, const float* Ys, const float* stats, vo
 }
 
 }  // extern "C"
+
+extern "C" lcp_status lcp_device_error(int* site, int reset) {
+  using namespace lcp;
+  if (!site) return fail(LCP_ERR_NULL, "site is NULL");
+  lcp_status (*const readers[])(int*, int) = {tc_error_gemm, tc_error_permute, tc_error_block_bwd};
+  int first = 0;
+  for (auto rd : readers) {
+    int v = 0;
+    const lcp_status s = rd(&v, reset);
+    if (s != LCP_OK) return s;
+    if (!first) first = v;
+  }
+  *site = first;
+  return LCP_OK;
+}

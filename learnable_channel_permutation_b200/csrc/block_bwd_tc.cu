@@ -1,0 +1,523 @@
+// Block backward on the tensor cores: dA = dAt P_B, dW' = M.dA and the
+// gradient of every diagonal block, dP_b = dAt_b^T A_b + W_b^T dW'_b
+// (reverse of PermLLM's Method 3 product and mask).
+
+#include "tc_common.cuh"
+
+namespace lcp {
+namespace {
+
+// ---------------------------------------- block backward, warp-specialised ---
+// BC = 64 (B = 32 or 64).  One CTA per (channel tile, row segment).  Warp 0
+// streams the (dAt, W) tiles of each 128-row chunk into a 3-stage ring; warp 1
+// issues W' = W (P_hi + P_lo) and dA = dAt P_hi into one of two TMEM buffers,
+// then, once the epilogue has written A = M.W' and dW' = M.dA, the stacked
+// dP product; warps 2-9 (two per TMEM lane quadrant, 32 columns each) turn
+// W', dA and the mask into the bf16 operands.  The dP accumulator stays in
+// TMEM for the whole segment and is written once at the end.
+template <int NSL> struct BwCfg {
+  static constexpr int STAGES = 3;
+  static constexpr int T_BYTES = 16384;                  // 128 rows x 64 bf16
+  static constexpr int STAGE = 2 * T_BYTES;              // dAt | W (adjacent: stacked A operand)
+  static constexpr int IMG_BYTES = 8192;
+  static constexpr int SMEM = STAGES * STAGE + 2 * IMG_BYTES + 2 * (2 * T_BYTES) + 1024 + 256;
+  static constexpr int EPI_WARPS = 4 * NSL;              // NSL column slices per TMEM lane quadrant
+  static constexpr int COLS = 64 / NSL;
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+  static constexpr int EPI = 32 * EPI_WARPS;
+};
+
+template <int B, int NSL>
+__global__ void __launch_bounds__(BwCfg<NSL>::THREADS, 1)
+block_bwd_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmDAt,
+                    const __grid_constant__ CUtensorMap tmPth, const __grid_constant__ CUtensorMap tmPtl,
+                    const uint32_t* __restrict__ mask, float* __restrict__ dP, int cout, int cin,
+                    int rows_per_split) {
+  using C = BwCfg<NSL>;
+  constexpr int NV = C::COLS;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sStage = smem;
+  uint8_t* sPth = smem + C::STAGES * C::STAGE;
+  uint8_t* sPtl = sPth + C::IMG_BYTES;
+  uint8_t* sAB = sPtl + C::IMG_BYTES;      // buffer a at + a * 2 * T_BYTES: A | dW' (adjacent)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sAB + 2 * 2 * C::T_BYTES);
+  // bars: full[3] empty[3] wd[2] abf[2] abe[2] dpf drain img
+  uint32_t* holder = reinterpret_cast<uint32_t*>(bars + 16);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(holder + 1);
+  auto bar = [&](int i) { return smem_u32(bars + i); };
+  const int FULL = 0, EMPTY = 3, WD = 6, ABF = 8, ABE = 10, DPF = 12, DRAIN = 13, IMG = 14;
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int t = blockIdx.x, sidx = blockIdx.y, col0 = t * 64;
+  const int rbeg = sidx * rows_per_split;
+  const int rend = min(cout, rbeg + rows_per_split);
+  const int nchunk = cdiv(rend - rbeg, 128);
+  const int words = cin / 32;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 3; ++i) { mbar_init(bar(FULL + i), 1); mbar_init(bar(EMPTY + i), 1); }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(WD + i), 1);
+      mbar_init(bar(ABF + i), C::EPI_WARPS);
+      mbar_init(bar(ABE + i), 1);
+    }
+    mbar_init(bar(DPF), 1);
+    mbar_init(bar(DRAIN), 1);
+    mbar_init(bar(IMG), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(smem_u32(holder), 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *holder;
+  const uint32_t tDP = tmem + 256;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      bool img_ok = true;
+      if (nchunk > 0) {
+        mbar_expect_tx(bar(IMG), 2 * C::IMG_BYTES);
+        tma_load_2d(smem_u32(sPth), &tmPth, bar(IMG), 0, col0);
+        tma_load_2d(smem_u32(sPtl), &tmPtl, bar(IMG), 0, col0);
+      }
+      uint32_t issued = 0, par = 0;
+      for (int c = 0; c < nchunk; ++c) {
+        const int st = c % C::STAGES;
+        const uint32_t use = (uint32_t)(c / C::STAGES) & 1u;
+        if (!mbar_wait(bar(EMPTY + st), use ^ 1u, abort_flag, 71)) break;
+        uint8_t* sg = sStage + st * C::STAGE;
+        const int r0 = rbeg + c * 128;
+        mbar_expect_tx(bar(FULL + st), C::STAGE);
+        tma_load_2d(smem_u32(sg), &tmDAt, bar(FULL + st), col0, r0);
+        tma_load_2d(smem_u32(sg + C::T_BYTES), &tmW, bar(FULL + st), col0, r0);
+        issued |= 1u << st;
+        par = (par & ~(1u << st)) | (use << st);
+      }
+      for (int st = 0; st < C::STAGES; ++st)
+        if (issued & (1u << st)) mbar_wait_drain(bar(FULL + st), (par >> st) & 1u, 72);
+      if (nchunk > 0) img_ok = mbar_wait_drain(bar(IMG), 0, 73);
+      (void)img_ok;
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc_n = idesc_bf16(128, 64, false, false);
+      constexpr uint32_t idesc_dp = idesc_bf16(128, 128, true, true);
+      bool ok = nchunk == 0 || mbar_wait(bar(IMG), 0, abort_flag, 74);
+      // W' = W (P_hi + P_lo) and dA = dAt P_hi of chunk c into TMEM buffer c & 1
+      auto mma1 = [&](int c) -> bool {
+        const int st = c % C::STAGES, a = c & 1;
+        const uint32_t use = (uint32_t)(c / C::STAGES) & 1u, ua = (uint32_t)(c >> 1) & 1u;
+        if (!mbar_wait(bar(FULL + st), use, abort_flag, 75)) return false;
+        // the epilogue has read buffer a of chunk c - 2 (it arrives on ABF after its loads)
+        if (c >= 2 && !mbar_wait(bar(ABF + a), ua ^ 1u, abort_flag, 76)) return false;
+        tc_fence_after();
+        const uint32_t sg = smem_u32(sStage + st * C::STAGE);
+        const uint32_t tW = tmem + a * 128, tDA = tmem + a * 128 + 64;
+#pragma unroll
+        for (int k16 = 0; k16 < 4; ++k16) {
+          const uint64_t wdesc = sdesc(sg + C::T_BYTES + k16 * 32, 16, 1024);
+          mma_bf16(tW, wdesc, sdesc(smem_u32(sPth) + k16 * 32, 16, 1024), idesc_n, k16 != 0);
+          mma_bf16(tW, wdesc, sdesc(smem_u32(sPtl) + k16 * 32, 16, 1024), idesc_n, true);
+          mma_bf16(tDA, sdesc(sg + k16 * 32, 16, 1024), sdesc(smem_u32(sPth) + k16 * 32, 16, 1024), idesc_n,
+                   k16 != 0);
+        }
+        mma_commit(bar(WD + a));
+        return true;
+      };
+      if (ok && nchunk > 0) ok = mma1(0);
+      for (int c = 0; c < nchunk && ok; ++c) {
+        const int st = c % C::STAGES, a = c & 1;
+        const uint32_t ua = (uint32_t)(c >> 1) & 1u;
+        if (c + 1 < nchunk && !mma1(c + 1)) break;
+        if (!mbar_wait(bar(ABF + a), ua, abort_flag, 77)) break;
+        tc_fence_after();
+        const uint32_t sg = smem_u32(sStage + st * C::STAGE);
+        const uint32_t sab = smem_u32(sAB + a * 2 * C::T_BYTES);
+        // stacked: A operand [dAt | W] (M = 128), B operand [A | dW'] (N = 128), LBO = 16 KB
+#pragma unroll
+        for (int k16 = 0; k16 < 8; ++k16)
+          mma_bf16(tDP, sdesc(sg + k16 * 2048, 16384, 1024), sdesc(sab + k16 * 2048, 16384, 1024), idesc_dp,
+                   (c | k16) != 0);
+        mma_commit(bar(ABE + a));
+        mma_commit(bar(EMPTY + st));
+      }
+      mma_commit(bar(DPF));
+      mma_commit(bar(DRAIN));
+      mbar_wait_drain(bar(DRAIN), 0, 78);
+    }
+    __syncwarp();
+  } else {
+    const int e = warp - 2, q = warp & 3, h = e >> 2;   // h: column slice of NV columns
+    const int row = q * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    bool ok = true;
+    // mask bits of this thread's NV columns, one chunk ahead of the chunk being processed
+    auto mask_bits = [&](int c) -> uint32_t {
+      const int grow = rbeg + c * 128 + row;
+      if (c >= nchunk || grow >= rend) return 0u;
+      const uint32_t w = __ldg(mask + (size_t)grow * words + col0 / 32 + (h * NV) / 32);
+      return NV == 32 ? w : (w >> ((h * NV) % 32)) & ((1u << NV) - 1u);
+    };
+    uint32_t next_bits = mask_bits(0);
+    for (int c = 0; c < nchunk; ++c) {
+      const int a = c & 1;
+      const uint32_t ua = (uint32_t)(c >> 1) & 1u;
+      const uint32_t bits = next_bits;
+      next_bits = mask_bits(c + 1);
+      ok = named_and(1, C::EPI, mbar_wait(bar(WD + a), ua, abort_flag, 79));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t wv[NV], dv[NV];
+      tmem_ld_cols<NV>(tmem + lane_off + a * 128 + h * NV, wv);
+      tmem_ld_cols<NV>(tmem + lane_off + a * 128 + 64 + h * NV, dv);
+      tmem_ld_wait();
+      // buffer a was last read by the dP product of chunk c - 2
+      ok = named_and(1, C::EPI, c < 2 || mbar_wait(bar(ABE + a), ua ^ 1u, abort_flag, 80));
+      if (!ok) break;
+      uint8_t* rA = sAB + a * 2 * C::T_BYTES;
+      uint8_t* rD = rA + C::T_BYTES;
+#pragma unroll
+      for (int c8 = 0; c8 < NV / 8; ++c8) {
+        float fa[8], fd[8];
+#pragma unroll
+        for (int x = 0; x < 8; ++x) {
+          const bool keep = (bits >> (8 * c8 + x)) & 1u;
+          fa[x] = keep ? __uint_as_float(wv[8 * c8 + x]) : 0.f;
+          fd[x] = keep ? __uint_as_float(dv[8 * c8 + x]) : 0.f;
+        }
+        const int chunk = h * (NV / 8) + c8;
+        st_sw128(rA, row, chunk, make_uint4(pack_bf16x2(fa[0], fa[1]), pack_bf16x2(fa[2], fa[3]),
+                                            pack_bf16x2(fa[4], fa[5]), pack_bf16x2(fa[6], fa[7])));
+        st_sw128(rD, row, chunk, make_uint4(pack_bf16x2(fd[0], fd[1]), pack_bf16x2(fd[2], fd[3]),
+                                            pack_bf16x2(fd[4], fd[5]), pack_bf16x2(fd[6], fd[7])));
+      }
+      fence_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(ABF + a));
+    }
+    if (ok) ok = named_and(1, C::EPI, mbar_wait(bar(DPF), 0, abort_flag, 81));
+    if (ok) {
+      tc_fence_after();
+      // rows 0..63 hold dAt^T A (columns 0..63), rows 64..127 W^T dW' (columns 64..127)
+      uint32_t v[NV];
+      const uint32_t cbase = (row < 64 ? 0u : 64u) + h * NV;
+      tmem_ld_cols<NV>(tDP + lane_off + cbase, v);
+      tmem_ld_wait();
+      float* scratch = reinterpret_cast<float*>(sAB);   // 64 x 64 floats; every MMA is done
+      if (row >= 64) {
+#pragma unroll
+        for (int x = 0; x < NV; ++x) scratch[(row - 64) * 64 + h * NV + x] = __uint_as_float(v[x]);
+      }
+      named_sync(1, C::EPI);
+      if (row < 64) {
+        const int nb = cin / B;
+        float* dPs = dP + (size_t)sidx * nb * B * B;
+        const float* add = scratch + row * 64 + h * NV;
+        if constexpr (B == 64) {
+          float4* o = reinterpret_cast<float4*>(dPs + ((size_t)t * 64 + row) * 64 + h * NV);
+#pragma unroll
+          for (int qq = 0; qq < NV / 4; ++qq)
+            o[qq] = make_float4(__uint_as_float(v[4 * qq]) + add[4 * qq], __uint_as_float(v[4 * qq + 1]) + add[4 * qq + 1],
+                                __uint_as_float(v[4 * qq + 2]) + add[4 * qq + 2],
+                                __uint_as_float(v[4 * qq + 3]) + add[4 * qq + 3]);
+        } else {
+          // B = 32: the tile holds blocks 2t (rows/columns 0..31) and 2t+1 (32..63);
+          // keep only the diagonal quadrants
+          const int qb = row / 32;
+          if ((h * NV) / 32 == qb) {
+            float* o = dPs + ((size_t)(2 * t + qb) * 32 + (row - 32 * qb)) * 32 + (h * NV) % 32;
+#pragma unroll
+            for (int x = 0; x < NV; ++x) o[x] = __uint_as_float(v[x]) + add[x];
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------- block backward ---
+// One CTA: channel tile t (BC columns) x a segment of C_out rows, in chunks of
+// 128 rows o:
+//   W'  = W_tile (P_hi + P_lo)          dA = dAt_tile P_hi          (TMEM)
+//   A = M.W', dW' = M.dA  -> bf16 operand tiles in shared memory
+//   dP += dAt_tile^T A + W_tile^T dW'   (contraction over the 128 rows: the
+//         row-major tiles are read as MN-major operands)
+// For BC = 64 the two products share one M = 128 MMA: the A operand stacks the
+// dAt and W tiles (adjacent, LBO = 16 KB) and the B operand stacks A and dW',
+// so the wanted sums are the two diagonal 64 x 64 quadrants of the result.
+// The partial dP of each segment goes to dP[s] (summed by the Sinkhorn reverse).
+
+template <int BC> struct BbCfg {
+  static constexpr int NCH = BC / 64;
+  static constexpr int T_BYTES = BC * 256;   // 128 rows x BC bf16
+  static constexpr int P_BYTES = BC * BC * 2;
+  static constexpr uint32_t TMEM_COLS = (2 * BC + 128 <= 256) ? 256u : 512u;
+  // sDAt | sW | sPth | sPtl | sAb | sdWb
+  static constexpr int SMEM = 4 * T_BYTES + 2 * P_BYTES + 1024 + 128;
+};
+
+template <int BC, int B>
+__global__ void __launch_bounds__(128)
+block_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmDAt,
+                    const __grid_constant__ CUtensorMap tmPth, const __grid_constant__ CUtensorMap tmPtl,
+                    const uint32_t* __restrict__ mask, float* __restrict__ dP, int cout, int cin,
+                    int rows_per_split) {
+  using C = BbCfg<BC>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sDAt = smem;
+  uint8_t* sW = sDAt + C::T_BYTES;
+  uint8_t* sPth = sW + C::T_BYTES;
+  uint8_t* sPtl = sPth + C::P_BYTES;
+  uint8_t* sAb = sPtl + C::P_BYTES;
+  uint8_t* sdWb = sAb + C::T_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sdWb + C::T_BYTES);
+  uint32_t* holder = reinterpret_cast<uint32_t*>(bars + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(holder + 1);
+  const uint32_t bar_load = smem_u32(bars + 0), bar_mma1 = smem_u32(bars + 1), bar_mma2 = smem_u32(bars + 2);
+  const uint32_t bar_drain = smem_u32(bars + 3);
+
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const int t = blockIdx.x, s = blockIdx.y, col0 = t * BC;
+  const int rbeg = s * rows_per_split;
+  const int rend = min(cout, rbeg + rows_per_split);
+  const int nchunk = cdiv(rend - rbeg, 128);
+  if (tid == 0) {
+    mbar_init(bar_load, 1);
+    mbar_init(bar_mma1, 1);
+    mbar_init(bar_mma2, 1);
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) tmem_alloc(smem_u32(holder), C::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *holder;
+  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  const int row = warp * 32 + lane;
+  const int words = cin / 32;
+  int pending_load = -1;
+  constexpr uint32_t idesc_n = idesc_bf16(128, BC, false, false);
+  constexpr uint32_t idesc_dp = idesc_bf16(128, 128, true, true);
+  const uint32_t tW = tmem, tDA = tmem + BC, tDP = tmem + 2 * BC;
+
+  bool ok = true;
+  for (int ch = 0; ch < nchunk && ok; ++ch) {
+    const int r0 = rbeg + ch * 128;
+    if (tid == 0) {
+      bool go = (ch == 0) || mbar_wait(bar_mma2, (uint32_t)(ch - 1) & 1u, abort_flag, 31);
+      if (go) {
+        pending_load = ch & 1;
+        mbar_expect_tx(bar_load, 2 * C::T_BYTES + (ch == 0 ? 2 * C::P_BYTES : 0));
+        for (int kc = 0; kc < C::NCH; ++kc) {
+          tma_load_2d(smem_u32(sW + kc * 16384), &tmW, bar_load, col0 + kc * 64, r0);
+          tma_load_2d(smem_u32(sDAt + kc * 16384), &tmDAt, bar_load, col0 + kc * 64, r0);
+        }
+        if (ch == 0)
+          for (int kc = 0; kc < C::NCH; ++kc) {
+            tma_load_2d(smem_u32(sPth + kc * BC * 128), &tmPth, bar_load, kc * 64, col0);
+            tma_load_2d(smem_u32(sPtl + kc * BC * 128), &tmPtl, bar_load, kc * 64, col0);
+          }
+        go = mbar_wait(bar_load, (uint32_t)ch & 1u, abort_flag, 32);
+        if (go) pending_load = -1;
+      }
+      if (!go) *abort_flag = 1;
+      if (go) {
+        tc_fence_after();
+        for (int kc = 0; kc < C::NCH; ++kc)
+#pragma unroll
+          for (int k16 = 0; k16 < 4; ++k16) {
+            const uint64_t a = sdesc(smem_u32(sW + kc * 16384) + k16 * 32, 16, 1024);
+            mma_bf16(tW, a, sdesc(smem_u32(sPth + kc * BC * 128) + k16 * 32, 16, 1024), idesc_n,
+                     (kc | k16) != 0);
+            mma_bf16(tW, a, sdesc(smem_u32(sPtl + kc * BC * 128) + k16 * 32, 16, 1024), idesc_n, true);
+            mma_bf16(tDA, sdesc(smem_u32(sDAt + kc * 16384) + k16 * 32, 16, 1024),
+                     sdesc(smem_u32(sPth + kc * BC * 128) + k16 * 32, 16, 1024), idesc_n, (kc | k16) != 0);
+          }
+        mma_commit(bar_mma1);
+      }
+    }
+    ok = __syncthreads_and(mbar_wait(bar_mma1, (uint32_t)ch & 1u, abort_flag, 33));
+    if (!ok) break;
+    tc_fence_after();
+    const int grow = r0 + row;
+    const bool valid = grow < rend;
+#pragma unroll 1
+    for (int cc = 0; cc < BC / 32; ++cc) {
+      uint32_t wv[32], dv[32];
+      tmem_ld32(tW + lane_off + cc * 32, wv);
+      tmem_ld32(tDA + lane_off + cc * 32, dv);
+      tmem_ld_wait();
+      const uint32_t bits = valid ? __ldg(mask + (size_t)grow * words + col0 / 32 + cc) : 0u;
+      uint8_t* rA = sAb + (cc / 2) * 16384;
+      uint8_t* rD = sdWb + (cc / 2) * 16384;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float fa[8], fd[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const bool keep = (bits >> (8 * q + e)) & 1u;
+          fa[e] = keep ? __uint_as_float(wv[8 * q + e]) : 0.f;
+          fd[e] = keep ? __uint_as_float(dv[8 * q + e]) : 0.f;
+        }
+        const int chunk16 = (cc & 1) * 4 + q;
+        st_sw128(rA, row, chunk16, make_uint4(pack_bf16x2(fa[0], fa[1]), pack_bf16x2(fa[2], fa[3]),
+                                              pack_bf16x2(fa[4], fa[5]), pack_bf16x2(fa[6], fa[7])));
+        st_sw128(rD, row, chunk16, make_uint4(pack_bf16x2(fd[0], fd[1]), pack_bf16x2(fd[2], fd[3]),
+                                              pack_bf16x2(fd[4], fd[5]), pack_bf16x2(fd[6], fd[7])));
+      }
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      if constexpr (BC == 64) {
+        // stacked: A = [dAt | W] (M = 128), B = [A | dW'] (N = 128), LBO = 16 KB
+#pragma unroll
+        for (int k16 = 0; k16 < 8; ++k16)
+          mma_bf16(tDP, sdesc(smem_u32(sDAt) + k16 * 2048, 16384, 1024),
+                   sdesc(smem_u32(sAb) + k16 * 2048, 16384, 1024), idesc_dp, (ch | k16) != 0);
+      } else {
+#pragma unroll
+        for (int k16 = 0; k16 < 8; ++k16)
+          mma_bf16(tDP, sdesc(smem_u32(sDAt) + k16 * 2048, 16384, 1024),
+                   sdesc(smem_u32(sAb) + k16 * 2048, 16384, 1024), idesc_dp, (ch | k16) != 0);
+#pragma unroll
+        for (int k16 = 0; k16 < 8; ++k16)
+          mma_bf16(tDP, sdesc(smem_u32(sW) + k16 * 2048, 16384, 1024),
+                   sdesc(smem_u32(sdWb) + k16 * 2048, 16384, 1024), idesc_dp, true);
+      }
+      mma_commit(bar_mma2);
+    }
+  }
+  if (ok && nchunk > 0) ok = __syncthreads_and(mbar_wait(bar_mma2, (uint32_t)(nchunk - 1) & 1u, abort_flag, 34));
+  const int nb = cin / B;
+  float* dPs = dP + (size_t)s * nb * B * B;
+  if (ok) {
+    tc_fence_after();
+    if constexpr (BC == 64) {
+      // rows 0..63: dAt^T A in columns 0..63; rows 64..127: W^T dW' in columns 64..127
+      float* scratch = reinterpret_cast<float*>(sAb);   // 64 x 64 floats (free: last MMA done)
+      uint32_t r0v[32], r1v[32];
+      const uint32_t cbase = (row < 64) ? 0u : 64u;
+      tmem_ld32(tDP + lane_off + cbase, r0v);
+      tmem_ld32(tDP + lane_off + cbase + 32, r1v);
+      tmem_ld_wait();
+      if (row >= 64) {
+        float* dst = scratch + (row - 64) * 64;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) { dst[e] = __uint_as_float(r0v[e]); dst[32 + e] = __uint_as_float(r1v[e]); }
+      }
+      __syncthreads();
+      if (row < 64) {
+        const float* add = scratch + row * 64;
+        float v[64];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) { v[e] = __uint_as_float(r0v[e]) + add[e]; v[32 + e] = __uint_as_float(r1v[e]) + add[32 + e]; }
+        if constexpr (B == 64) {
+          float* o = dPs + ((size_t)t * 64 + row) * 64;
+#pragma unroll
+          for (int e = 0; e < 64; ++e) o[e] = v[e];
+        } else {
+          const int qb = row / 32;            // which 32-block of the tile
+          float* o = dPs + ((size_t)(2 * t + qb) * 32 + (row - 32 * qb)) * 32;
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = v[32 * qb + e];
+        }
+      }
+    } else {
+      float* o = dPs + ((size_t)t * BC + row) * BC;
+#pragma unroll 1
+      for (int cc = 0; cc < BC / 32; ++cc) {
+        uint32_t r[32];
+        tmem_ld32(tDP + lane_off + cc * 32, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o[cc * 32 + e] = __uint_as_float(r[e]);
+      }
+    }
+  }
+  if (tid == 0) {
+    if (pending_load >= 0) mbar_wait_drain(bar_load, (uint32_t)pending_load, 35);
+    mma_commit(bar_drain);
+    mbar_wait_drain(bar_drain, 0, 36);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+template <int BC, int B>
+lcp_status block_bwd_bc(const CUtensorMap& mW, const CUtensorMap& mD, const CUtensorMap& mPth,
+                        const CUtensorMap& mPtl, const uint32_t* mask, float* dP, int splits, int rows,
+                        int cout, int cin, cudaStream_t st) {
+  auto k = block_bwd_tc_kernel<BC, B>;
+  TC_TRY(set_smem(k, BbCfg<BC>::SMEM, "block_bwd_tc"));
+  const dim3 grid(cin / BC, splits);
+  k<<<grid, 128, BbCfg<BC>::SMEM, st>>>(mW, mD, mPth, mPtl, mask, dP, cout, cin, rows);
+  return check_launch("block_bwd_tc");
+}
+
+int bb_rows_per_split(int cout, int cin, int B) {
+  const int BC = B < 64 ? 64 : B;
+  const int tiles = cin / BC;
+  const int chunks = cdiv(cout, 128);
+  // one CTA per SM: as many row segments per channel tile as fill the SMs once
+  int S = 148 / tiles;
+  if (S < 1) S = 1;
+  if (S > 64) S = 64;
+  if (S > chunks) S = chunks;
+  return cdiv(chunks, S) * 128;
+}
+
+}  // namespace
+
+lcp_status tc_error_block_bwd(int* site, int reset) { return read_tc_error(site, reset); }
+
+bool block_bwd_tc_supported(int B) { return B <= 128; }
+
+int block_bwd_tc_splits(int cout, int cin, int B) {
+  if (!block_bwd_tc_supported(B)) return 1;
+  return cdiv(cout, bb_rows_per_split(cout, cin, B));
+}
+
+lcp_status launch_block_bwd_tc(const __nv_bfloat16* W, const __nv_bfloat16* dAt, const uint32_t* mask,
+                               const __nv_bfloat16* img_pt_hi, const __nv_bfloat16* img_pt_lo, float* dP_partials,
+                               int splits, int cout, int cin, int B, cudaStream_t st) {
+  if (!block_bwd_tc_supported(B)) return fail(LCP_ERR_SHAPE, "block_bwd_tc: B = %d is not supported", B);
+  const int BC = B < 64 ? 64 : B;
+  const int rows = bb_rows_per_split(cout, cin, B);
+  if (cdiv(cout, rows) != splits) return fail(LCP_ERR_ARG, "block_bwd_tc: split count mismatch");
+  CUtensorMap mW, mD, mPth, mPtl;
+  TC_TRY(make_map(&mW, W, cin, cout, 64, 128, "block_bwd W"));
+  TC_TRY(make_map(&mD, dAt, cin, cout, 64, 128, "block_bwd dAt"));
+  TC_TRY(make_map(&mPth, img_pt_hi, BC, cin, 64, BC, "block_bwd Pt_hi"));
+  TC_TRY(make_map(&mPtl, img_pt_lo, BC, cin, 64, BC, "block_bwd Pt_lo"));
+  if (B <= 64) {
+    constexpr int NSL = 2;
+    using C = BwCfg<NSL>;
+    auto k = (B == 32) ? block_bwd_ws_kernel<32, NSL> : block_bwd_ws_kernel<64, NSL>;
+    TC_TRY(set_smem(k, C::SMEM, "block_bwd_tc"));
+    k<<<dim3(cin / 64, splits), C::THREADS, C::SMEM, st>>>(mW, mD, mPth, mPtl, mask, dP_partials, cout, cin, rows);
+    return check_launch("block_bwd_tc");
+  }
+  return block_bwd_bc<128, 128>(mW, mD, mPth, mPtl, mask, dP_partials, splits, rows, cout, cin, st);
+}
+
+}  // namespace lcp

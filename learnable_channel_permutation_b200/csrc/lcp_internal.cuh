@@ -74,7 +74,6 @@ lcp_status launch_loss_fused(const float* Yd, const float* Ys, float* stats, voi
                              float* loss, unsigned* counter, int cout, int tokens, cudaStream_t st);
 
 // Tensor-core (tcgen05) kernels, bf16 operands, float32 accumulation.
-bool tc_available();
 lcp_status launch_permute_mask_tc(const __nv_bfloat16* W, const __nv_bfloat16* img_pt_hi,
                                   const __nv_bfloat16* img_pt_lo, const __nv_bfloat16* img_p_hi,
                                   uint32_t* mask, __nv_bfloat16* At, float* Wp_out, int cout,
@@ -91,6 +90,12 @@ lcp_status launch_block_bwd_tc(const __nv_bfloat16* W, const __nv_bfloat16* dAt,
                                int cout, int cin, int B, cudaStream_t st);
 int block_bwd_tc_splits(int cout, int cin, int B);
 bool block_bwd_tc_supported(int B);   // B <= 128 (TMEM/smem budget of the fused kernel)
+
+// Device error words of the tensor-core translation units: the first wait
+// site that timed out since the last reset, 0 if none (cleared when `reset`).
+lcp_status tc_error_gemm(int* site, int reset);
+lcp_status tc_error_permute(int* site, int reset);
+lcp_status tc_error_block_bwd(int* site, int reset);
 
 constexpr int kCkptPerIter = 2;  // R then C vectors per iteration
 

@@ -1,0 +1,681 @@
+// W' = W P_B (PermLLM, Method 3: the block-diagonal permutation applied to the
+// weight's input channels), the N:M mask of |W'| (integration with pruning
+// methods), A = M.W' and At = A P_B^T, fused per tile on the tensor cores.
+
+#include "tc_common.cuh"
+
+namespace lcp {
+namespace {
+
+// ------------------------------------------------------- permute + mask ---
+// One CTA: rows [r0, r0+128) x channels [t*BC, (t+1)*BC) with BC = max(B, 64),
+// in 64-column chunks c:
+//   W'_c  = W_tile (P_hi + P_lo)[:, chunk c]          (TMEM, 64 columns)
+//   mask bits and A_c = M.W'_c (bf16, shared memory, SW128 K-major)
+//   At   += A_c P_hi[:, chunk c]^T                      (TMEM, BC columns)
+// P enters through the tile-format images written by the Sinkhorn kernel:
+// Pt[t][j][i] = P[i][j] (B operand of the first product, rows j of chunk c),
+// Ph[t][i][j] = P[i][j] (B operand of the second product, columns of chunk c).
+
+template <int BC> struct PmCfg {
+  static constexpr int NCH = BC / 64;
+  static constexpr int W_BYTES = BC * 256;   // 128 rows x BC bf16
+  static constexpr int PT_BYTES = BC * 128;  // 64 rows x BC bf16 (NCH regions of 8 KB)
+  static constexpr int PH_BYTES = BC * 128;  // BC rows x 64 bf16
+  static constexpr int A_BYTES = 16384;      // 128 rows x 64 bf16
+  static constexpr uint32_t TMEM_COLS = (64 + BC <= 128) ? 128u : ((64 + BC <= 256) ? 256u : 512u);
+  static constexpr int SMEM = W_BYTES + 2 * PT_BYTES + PH_BYTES + A_BYTES + 1024 + 128;
+};
+
+template <int BC, int MGROUP>
+__global__ void __launch_bounds__(128)
+permute_mask_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmPth,
+                       const __grid_constant__ CUtensorMap tmPtl, const __grid_constant__ CUtensorMap tmPh,
+                       uint32_t* __restrict__ mask, __nv_bfloat16* __restrict__ At,
+                       float* __restrict__ Wp_out, int cout, int cin, int n) {
+  using C = PmCfg<BC>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sW = smem;
+  uint8_t* sPth = sW + C::W_BYTES;
+  uint8_t* sPtl = sPth + C::PT_BYTES;
+  uint8_t* sPh = sPtl + C::PT_BYTES;
+  uint8_t* sA = sPh + C::PH_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sA + C::A_BYTES);
+  uint32_t* holder = reinterpret_cast<uint32_t*>(bars + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(holder + 1);
+  const uint32_t bar_load = smem_u32(bars + 0), bar_mma1 = smem_u32(bars + 1), bar_mma2 = smem_u32(bars + 2);
+  const uint32_t bar_drain = smem_u32(bars + 3);
+
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const int r0 = blockIdx.x * 128, t = blockIdx.y, col0 = t * BC;
+  if (tid == 0) {
+    mbar_init(bar_load, 1);
+    mbar_init(bar_mma1, 1);
+    mbar_init(bar_mma2, 1);
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) tmem_alloc(smem_u32(holder), C::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *holder;
+  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  const int row = warp * 32 + lane, grow = r0 + row;
+  const int words = cin / 32;
+  constexpr uint32_t idesc1 = idesc_bf16(128, 64, false, false);
+  constexpr uint32_t idesc2 = idesc_bf16(128, BC, false, false);
+
+  bool ok = true;
+  int pending_load = -1;   // thread 0: parity of a load not yet seen complete
+  for (int c = 0; c < C::NCH && ok; ++c) {
+    if (tid == 0) {
+      bool go = (c == 0) || mbar_wait(bar_mma2, (uint32_t)(c - 1) & 1u, abort_flag, 21);
+      if (go) {
+        pending_load = c & 1;
+        mbar_expect_tx(bar_load, (c == 0 ? C::W_BYTES : 0) + 2 * C::PT_BYTES + C::PH_BYTES);
+        if (c == 0)
+          for (int kc = 0; kc < C::NCH; ++kc)
+            tma_load_2d(smem_u32(sW + kc * 16384), &tmW, bar_load, col0 + kc * 64, r0);
+        for (int kc = 0; kc < C::NCH; ++kc) {
+          tma_load_2d(smem_u32(sPth + kc * 8192), &tmPth, bar_load, kc * 64, col0 + c * 64);
+          tma_load_2d(smem_u32(sPtl + kc * 8192), &tmPtl, bar_load, kc * 64, col0 + c * 64);
+        }
+        tma_load_2d(smem_u32(sPh), &tmPh, bar_load, c * 64, col0);
+        go = mbar_wait(bar_load, (uint32_t)c & 1u, abort_flag, 22);
+        if (go) pending_load = -1;
+      }
+      if (!go) *abort_flag = 1;
+      if (go) {
+        tc_fence_after();
+#pragma unroll 1
+        for (int pass = 0; pass < 2; ++pass) {
+          const uint8_t* sB = pass ? sPtl : sPth;
+          for (int kc = 0; kc < C::NCH; ++kc)
+#pragma unroll
+            for (int k16 = 0; k16 < 4; ++k16)
+              mma_bf16(tmem, sdesc(smem_u32(sW + kc * 16384) + k16 * 32, 16, 1024),
+                       sdesc(smem_u32(sB + kc * 8192) + k16 * 32, 16, 1024), idesc1,
+                       (pass | kc | k16) != 0);
+        }
+        mma_commit(bar_mma1);
+      }
+    }
+    ok = __syncthreads_and(mbar_wait(bar_mma1, (uint32_t)c & 1u, abort_flag, 23));
+    if (!ok) break;
+    tc_fence_after();
+    uint32_t v0[32], v1[32];
+    tmem_ld32(tmem + lane_off + 0, v0);
+    tmem_ld32(tmem + lane_off + 32, v1);
+    tmem_ld_wait();
+    const uint32_t w0 = nm_word<MGROUP>(v0, n), w1 = nm_word<MGROUP>(v1, n);
+    if (grow < cout) {
+      const int wi = (col0 + c * 64) / 32;
+      mask[(size_t)grow * words + wi] = w0;
+      mask[(size_t)grow * words + wi + 1] = w1;
+      if (Wp_out) {
+        float4* o = reinterpret_cast<float4*>(Wp_out + (size_t)grow * cin + col0 + c * 64);
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          o[q] = make_float4(__uint_as_float(v0[4 * q]), __uint_as_float(v0[4 * q + 1]),
+                             __uint_as_float(v0[4 * q + 2]), __uint_as_float(v0[4 * q + 3]));
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          o[8 + q] = make_float4(__uint_as_float(v1[4 * q]), __uint_as_float(v1[4 * q + 1]),
+                                 __uint_as_float(v1[4 * q + 2]), __uint_as_float(v1[4 * q + 3]));
+      }
+    }
+    // A_c = M . W'_c as bf16 into the K-major SW128 operand tile
+#pragma unroll
+    for (int ch = 0; ch < 8; ++ch) {
+      const uint32_t* v = ch < 4 ? v0 : v1;
+      const uint32_t w = ch < 4 ? w0 : w1;
+      const int b0 = (ch & 3) * 8;
+      float f[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) f[e] = ((w >> (b0 + e)) & 1u) ? __uint_as_float(v[b0 + e]) : 0.f;
+      st_sw128(sA, row, ch, make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                                       pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7])));
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+#pragma unroll
+      for (int k16 = 0; k16 < 4; ++k16)
+        mma_bf16(tmem + 64, sdesc(smem_u32(sA) + k16 * 32, 16, 1024), sdesc(smem_u32(sPh) + k16 * 32, 16, 1024),
+                 idesc2, (c | k16) != 0);
+      mma_commit(bar_mma2);
+    }
+  }
+  if (ok) ok = __syncthreads_and(mbar_wait(bar_mma2, (uint32_t)(C::NCH - 1) & 1u, abort_flag, 24));
+  if (ok) {
+    tc_fence_after();
+#pragma unroll 1
+    for (int cc = 0; cc < BC / 32; ++cc) {
+      uint32_t r[32];
+      tmem_ld32(tmem + lane_off + 64 + cc * 32, r);
+      tmem_ld_wait();
+      if (grow < cout) {
+        uint4* o = reinterpret_cast<uint4*>(At + (size_t)grow * cin + col0 + cc * 32);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          o[q] = make_uint4(pack_bf16x2(__uint_as_float(r[8 * q]), __uint_as_float(r[8 * q + 1])),
+                            pack_bf16x2(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3])),
+                            pack_bf16x2(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5])),
+                            pack_bf16x2(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7])));
+      }
+    }
+  }
+  if (tid == 0) {
+    // no copy or MMA of ours may still be running when the CTA exits
+    if (pending_load >= 0) mbar_wait_drain(bar_load, (uint32_t)pending_load, 25);
+    mma_commit(bar_drain);
+    mbar_wait_drain(bar_drain, 0, 26);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// ------------------------------------- permute + mask, warp-specialised ---
+// BC = 64 (B = 32 or 64).  Persistent CTAs walk a flat list of (channel tile,
+// row tile) pairs.  Warp 0 streams each tile's W block together with its P
+// images into a 3-stage ring; warp 1 issues W' = W (P_hi + P_lo) into one of
+// two TMEM buffers and, once the epilogue has written A = M.W' to shared
+// memory, At = A P_hi into the same buffer; warps 2-9 (two per TMEM lane
+// quadrant, 32 columns each) compute the mask, write A, and copy At out
+// through a swizzled staging tile with TMA stores.
+template <int NSL> struct PwCfg {
+  static constexpr int STAGES = 3;
+  static constexpr int W_BYTES = 16384;                 // 128 rows x 64 bf16
+  static constexpr int IMG_BYTES = 8192;                // 64 x 64 bf16
+  static constexpr int STAGE = W_BYTES + 3 * IMG_BYTES; // W | Pt_hi | Pt_lo | P_hi
+  static constexpr int A_BYTES = 16384;
+  static constexpr int SMEM = STAGES * STAGE + 2 * A_BYTES + 2 * A_BYTES + 1024 + 256;
+  static constexpr int EPI_WARPS = 4 * NSL;              // NSL column slices per TMEM lane quadrant
+  static constexpr int COLS = 64 / NSL;                  // columns per epilogue thread
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+  static constexpr int EPI = 32 * EPI_WARPS;
+};
+
+template <int MGROUP, int NSL>
+__global__ void __launch_bounds__(PwCfg<NSL>::THREADS, 1)
+permute_mask_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmPth,
+                       const __grid_constant__ CUtensorMap tmPtl, const __grid_constant__ CUtensorMap tmPh,
+                       const __grid_constant__ CUtensorMap tmAt, uint32_t* __restrict__ mask,
+                       float* __restrict__ Wp_out, int cout, int cin, int n) {
+  using C = PwCfg<NSL>;
+  constexpr int NV = C::COLS;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sStage = smem;
+  uint8_t* sA = smem + C::STAGES * C::STAGE;          // 2 buffers
+  uint8_t* sO = sA + 2 * C::A_BYTES;                  // 2 staging tiles for At
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sO + 2 * C::A_BYTES);
+  // bars: full[3] empty[3] wf[2] af[2] atf[2] tmw[2] tma[2] drain
+  uint32_t* holder = reinterpret_cast<uint32_t*>(bars + 17);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(holder + 1);
+  auto bar = [&](int i) { return smem_u32(bars + i); };
+  const int FULL = 0, EMPTY = 3, WF = 6, AF = 8, ATF = 10, TMW = 12, TMA = 14, DRAIN = 16;
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int nrt = cdiv(cout, 128), ntc = cin / 64;
+  const int total = nrt * ntc;
+  const int nloc = (int)blockIdx.x < total ? cdiv(total - (int)blockIdx.x, (int)gridDim.x) : 0;
+  const int words = cin / 32;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 3; ++i) { mbar_init(bar(FULL + i), 1); mbar_init(bar(EMPTY + i), 1); }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(WF + i), 1);
+      mbar_init(bar(AF + i), C::EPI_WARPS);
+      mbar_init(bar(ATF + i), 1);
+      mbar_init(bar(TMW + i), C::EPI_WARPS);
+      mbar_init(bar(TMA + i), C::EPI_WARPS);
+    }
+    mbar_init(bar(DRAIN), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(smem_u32(holder), 256);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *holder;
+  auto tile_of = [&](int k, int& t, int& rt) {
+    const int idx = (int)blockIdx.x + k * (int)gridDim.x;
+    t = idx / nrt;
+    rt = idx % nrt;
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t issued = 0, par = 0;   // per stage: outstanding load and its parity
+      for (int k = 0; k < nloc; ++k) {
+        const int st = k % C::STAGES;
+        const uint32_t use = (uint32_t)(k / C::STAGES) & 1u;
+        if (!mbar_wait(bar(EMPTY + st), use ^ 1u, abort_flag, 61)) break;
+        int t, rt;
+        tile_of(k, t, rt);
+        uint8_t* sg = sStage + st * C::STAGE;
+        mbar_expect_tx(bar(FULL + st), C::STAGE);
+        tma_load_2d(smem_u32(sg), &tmW, bar(FULL + st), t * 64, rt * 128);
+        tma_load_2d(smem_u32(sg + C::W_BYTES), &tmPth, bar(FULL + st), 0, t * 64);
+        tma_load_2d(smem_u32(sg + C::W_BYTES + C::IMG_BYTES), &tmPtl, bar(FULL + st), 0, t * 64);
+        tma_load_2d(smem_u32(sg + C::W_BYTES + 2 * C::IMG_BYTES), &tmPh, bar(FULL + st), 0, t * 64);
+        issued |= 1u << st;
+        par = (par & ~(1u << st)) | (use << st);
+      }
+      for (int st = 0; st < C::STAGES; ++st)
+        if (issued & (1u << st)) mbar_wait_drain(bar(FULL + st), (par >> st) & 1u, 62);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(128, 64, false, false);
+      // W' = W (P_hi + P_lo) of local tile k into the W' half of TMEM buffer k & 1
+      auto mma1 = [&](int k) -> bool {
+        const int st = k % C::STAGES, a = k & 1;
+        const uint32_t use = (uint32_t)(k / C::STAGES) & 1u, ua = (uint32_t)(k >> 1) & 1u;
+        if (!mbar_wait(bar(FULL + st), use, abort_flag, 63)) return false;
+        if (!mbar_wait(bar(TMW + a), ua ^ 1u, abort_flag, 64)) return false;   // W' of tile k - 2 read
+        tc_fence_after();
+        const uint32_t sg = smem_u32(sStage + st * C::STAGE);
+        const uint32_t dW = tmem + a * 128;
+#pragma unroll
+        for (int k16 = 0; k16 < 4; ++k16) {
+          const uint64_t ad = sdesc(sg + k16 * 32, 16, 1024);
+          mma_bf16(dW, ad, sdesc(sg + C::W_BYTES + k16 * 32, 16, 1024), idesc, k16 != 0);
+          mma_bf16(dW, ad, sdesc(sg + C::W_BYTES + C::IMG_BYTES + k16 * 32, 16, 1024), idesc, true);
+        }
+        mma_commit(bar(WF + a));
+        return true;
+      };
+      // the next tile's first product is issued before waiting for this tile's
+      // epilogue, so the tensor core and the epilogue warps overlap
+      bool ok = nloc == 0 || mma1(0);
+      for (int k = 0; k < nloc && ok; ++k) {
+        const int st = k % C::STAGES, a = k & 1;
+        const uint32_t ua = (uint32_t)(k >> 1) & 1u;
+        if (k + 1 < nloc && !mma1(k + 1)) break;
+        if (!mbar_wait(bar(AF + a), ua, abort_flag, 65)) break;        // A of tile k in shared memory
+        if (!mbar_wait(bar(TMA + a), ua ^ 1u, abort_flag, 69)) break;  // At of tile k - 2 read
+        tc_fence_after();
+        const uint32_t sg = smem_u32(sStage + st * C::STAGE);
+        const uint32_t sa = smem_u32(sA + a * C::A_BYTES);
+        const uint32_t dAt = tmem + a * 128 + 64;
+#pragma unroll
+        for (int k16 = 0; k16 < 4; ++k16)
+          mma_bf16(dAt, sdesc(sa + k16 * 32, 16, 1024), sdesc(sg + C::W_BYTES + 2 * C::IMG_BYTES + k16 * 32, 16, 1024),
+                   idesc, k16 != 0);
+        mma_commit(bar(ATF + a));
+        mma_commit(bar(EMPTY + st));
+      }
+      mma_commit(bar(DRAIN));
+      mbar_wait_drain(bar(DRAIN), 0, 66);
+    }
+    __syncwarp();
+  } else {
+    // Software-pipelined epilogue: in step k the warps first turn W' of tile k
+    // into the mask and A (so the MMA warp can start At of tile k), then copy
+    // out At of tile k - 1, whose product ran meanwhile.
+    const int e = warp - 2, q = warp & 3, h = e >> 2;   // h: column slice of NV columns
+    const int row = q * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    const bool leader = (e == 0 && lane == 0);
+    for (int k = 0; k <= nloc; ++k) {
+      if (k < nloc) {
+        const int a = k & 1;
+        const uint32_t ua = (uint32_t)(k >> 1) & 1u;
+        int t, rt;
+        tile_of(k, t, rt);
+        const int grow = rt * 128 + row;
+        if (!named_and(1, C::EPI, mbar_wait(bar(WF + a), ua, abort_flag, 67))) break;
+        tc_fence_after();
+        uint32_t v[NV];
+        tmem_ld_cols<NV>(tmem + lane_off + a * 128 + h * NV, v);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(TMW + a));
+        const uint32_t w = nm_bits<MGROUP, NV>(v, n);
+        if (grow < cout) {
+          if constexpr (NV == 32) {
+            mask[(size_t)grow * words + 2 * t + h] = w;
+          } else {
+            reinterpret_cast<uint16_t*>(mask)[((size_t)grow * words + 2 * t) * 2 + h] = (uint16_t)w;
+          }
+          if (Wp_out) {
+            float4* o = reinterpret_cast<float4*>(Wp_out + (size_t)grow * cin + t * 64 + h * NV);
+#pragma unroll
+            for (int qq = 0; qq < NV / 4; ++qq)
+              o[qq] = make_float4(__uint_as_float(v[4 * qq]), __uint_as_float(v[4 * qq + 1]),
+                                  __uint_as_float(v[4 * qq + 2]), __uint_as_float(v[4 * qq + 3]));
+          }
+        }
+        uint8_t* sa = sA + a * C::A_BYTES;
+#pragma unroll
+        for (int c8 = 0; c8 < NV / 8; ++c8) {
+          float f[8];
+#pragma unroll
+          for (int x = 0; x < 8; ++x) f[x] = ((w >> (8 * c8 + x)) & 1u) ? __uint_as_float(v[8 * c8 + x]) : 0.f;
+          st_sw128(sa, row, h * (NV / 8) + c8, make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                                                          pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7])));
+        }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(AF + a));
+      }
+      if (k > 0) {
+        const int kp = k - 1, a = kp & 1;
+        const uint32_t ua = (uint32_t)(kp >> 1) & 1u;
+        int t, rt;
+        tile_of(kp, t, rt);
+        const bool got = mbar_wait(bar(ATF + a), ua, abort_flag, 68);
+        // the staging tile of two tiles ago must have been read out by its TMA store
+        if (leader) bulk_wait_read<1>();
+        if (!named_and(1, C::EPI, got)) break;
+        tc_fence_after();
+        uint32_t v[NV];
+        tmem_ld_cols<NV>(tmem + lane_off + a * 128 + 64 + h * NV, v);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(TMA + a));
+        uint8_t* so = sO + a * C::A_BYTES;
+#pragma unroll
+        for (int c8 = 0; c8 < NV / 8; ++c8)
+          st_sw128(so, row, h * (NV / 8) + c8,
+                   make_uint4(pack_bf16x2(__uint_as_float(v[8 * c8 + 0]), __uint_as_float(v[8 * c8 + 1])),
+                              pack_bf16x2(__uint_as_float(v[8 * c8 + 2]), __uint_as_float(v[8 * c8 + 3])),
+                              pack_bf16x2(__uint_as_float(v[8 * c8 + 4]), __uint_as_float(v[8 * c8 + 5])),
+                              pack_bf16x2(__uint_as_float(v[8 * c8 + 6]), __uint_as_float(v[8 * c8 + 7]))));
+        fence_async_smem();
+        named_sync(1, C::EPI);
+        if (leader) {
+          tma_store_2d(&tmAt, smem_u32(so), t * 64, rt * 128);
+          bulk_commit();
+        }
+      }
+    }
+    if (leader) bulk_wait_all();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+// ----------------------------------------- permute + mask, row-streamed ---
+// For BC <= 128 the P images of the CTA's channel tile stay resident and the
+// CTA walks the row tiles rt = blockIdx.y, blockIdx.y + gridDim.y, ...; the W
+// tile of the next-but-one row tile streams in (two buffers) while the current
+// one is processed, so that HBM reads stay in flight across the whole launch.
+template <int BC> struct Pm2Cfg {
+  static constexpr int NCH = BC / 64;
+  static constexpr int W_BYTES = BC * 256;        // 128 rows x BC
+  static constexpr int PT_BYTES = BC * BC * 2;    // every chunk of one transposed image
+  static constexpr int PH_BYTES = BC * BC * 2;
+  static constexpr int A_BYTES = 16384;
+  static constexpr uint32_t TMEM_COLS = (64 + BC <= 128) ? 128u : 256u;
+  static constexpr int SMEM = 2 * W_BYTES + 2 * PT_BYTES + PH_BYTES + A_BYTES + 1024 + 128;
+  static constexpr int CTAS_PER_SM = BC == 64 ? 3 : 1;
+};
+
+template <int BC, int MGROUP>
+__global__ void __launch_bounds__(128)
+permute_mask_tc2_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmPth,
+                        const __grid_constant__ CUtensorMap tmPtl, const __grid_constant__ CUtensorMap tmPh,
+                        uint32_t* __restrict__ mask, __nv_bfloat16* __restrict__ At,
+                        float* __restrict__ Wp_out, int cout, int cin, int n) {
+  using C = Pm2Cfg<BC>;
+  constexpr int NCH = C::NCH;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sW0 = smem;
+  uint8_t* sPth = sW0 + 2 * C::W_BYTES;
+  uint8_t* sPtl = sPth + C::PT_BYTES;
+  uint8_t* sPh = sPtl + C::PT_BYTES;
+  uint8_t* sA = sPh + C::PH_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sA + C::A_BYTES);
+  uint32_t* holder = reinterpret_cast<uint32_t*>(bars + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(holder + 1);
+  const uint32_t bar_full0 = smem_u32(bars + 0);          // +8 for buffer 1
+  const uint32_t bar_mma1 = smem_u32(bars + 2), bar_mma2 = smem_u32(bars + 3), bar_drain = smem_u32(bars + 4);
+
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const int t = blockIdx.x, col0 = t * BC;
+  const int nrt = cdiv(cout, 128), first = blockIdx.y, step = gridDim.y;
+  const int nloc = first < nrt ? cdiv(nrt - first, step) : 0;
+  if (tid == 0) {
+    mbar_init(bar_full0, 1);
+    mbar_init(bar_full0 + 8, 1);
+    mbar_init(bar_mma1, 1);
+    mbar_init(bar_mma2, 1);
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) tmem_alloc(smem_u32(holder), C::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *holder;
+  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  const int row = warp * 32 + lane;
+  const int words = cin / 32;
+  constexpr uint32_t idesc1 = idesc_bf16(128, 64, false, false);
+  constexpr uint32_t idesc2 = idesc_bf16(128, BC, false, false);
+
+  auto load_w = [&](int k, int b) {   // thread 0: W rows of local tile k into buffer b
+    const int r0 = (first + k * step) * 128;
+    for (int kc = 0; kc < NCH; ++kc)
+      tma_load_2d(smem_u32(sW0 + b * C::W_BYTES + kc * 16384), &tmW, bar_full0 + 8 * b, col0 + kc * 64, r0);
+  };
+  int issued = 0;   // thread 0: local tiles whose W load has been issued
+  if (tid == 0 && nloc > 0) {
+    mbar_expect_tx(bar_full0, C::W_BYTES + 2 * C::PT_BYTES + C::PH_BYTES);
+    for (int c = 0; c < NCH; ++c) {
+      for (int kc = 0; kc < NCH; ++kc) {
+        tma_load_2d(smem_u32(sPth + (c * NCH + kc) * 8192), &tmPth, bar_full0, kc * 64, col0 + c * 64);
+        tma_load_2d(smem_u32(sPtl + (c * NCH + kc) * 8192), &tmPtl, bar_full0, kc * 64, col0 + c * 64);
+      }
+      tma_load_2d(smem_u32(sPh + c * BC * 128), &tmPh, bar_full0, c * 64, col0);
+    }
+    load_w(0, 0);
+    issued = 1;
+    if (nloc > 1) {
+      mbar_expect_tx(bar_full0 + 8, C::W_BYTES);
+      load_w(1, 1);
+      issued = 2;
+    }
+  }
+
+  bool ok = true;
+  uint32_t n1 = 0, n2 = 0;   // completed phases of bar_mma1 / bar_mma2
+  int consumed = 0;          // thread 0: local tiles whose W load was seen complete
+  for (int k = 0; k < nloc && ok; ++k) {
+    const int b = k & 1;
+    const int grow = (first + k * step) * 128 + row;
+    const uint8_t* sW = sW0 + b * C::W_BYTES;
+    if (tid == 0) {
+      if (mbar_wait(bar_full0 + 8 * b, (uint32_t)(k >> 1) & 1u, abort_flag, 41)) consumed = k + 1;
+      else *abort_flag = 1;
+    }
+    for (int c = 0; c < NCH; ++c) {
+      if (tid == 0 && !*abort_flag) {
+        tc_fence_after();
+#pragma unroll 1
+        for (int pass = 0; pass < 2; ++pass) {
+          const uint8_t* sB = (pass ? sPtl : sPth) + c * NCH * 8192;
+          for (int kc = 0; kc < NCH; ++kc)
+#pragma unroll
+            for (int k16 = 0; k16 < 4; ++k16)
+              mma_bf16(tmem, sdesc(smem_u32(sW + kc * 16384) + k16 * 32, 16, 1024),
+                       sdesc(smem_u32(sB + kc * 8192) + k16 * 32, 16, 1024), idesc1, (pass | kc | k16) != 0);
+        }
+        mma_commit(bar_mma1);
+      }
+      ok = __syncthreads_and(mbar_wait(bar_mma1, n1 & 1u, abort_flag, 42));
+      ++n1;
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t v0[32], v1[32];
+      tmem_ld32(tmem + lane_off + 0, v0);
+      tmem_ld32(tmem + lane_off + 32, v1);
+      tmem_ld_wait();
+      const uint32_t w0 = nm_word<MGROUP>(v0, n), w1 = nm_word<MGROUP>(v1, n);
+      if (grow < cout) {
+        const int wi = (col0 + c * 64) / 32;
+        *reinterpret_cast<uint2*>(mask + (size_t)grow * words + wi) = make_uint2(w0, w1);
+        if (Wp_out) {
+          float4* o = reinterpret_cast<float4*>(Wp_out + (size_t)grow * cin + col0 + c * 64);
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            o[q] = make_float4(__uint_as_float(v0[4 * q]), __uint_as_float(v0[4 * q + 1]),
+                               __uint_as_float(v0[4 * q + 2]), __uint_as_float(v0[4 * q + 3]));
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            o[8 + q] = make_float4(__uint_as_float(v1[4 * q]), __uint_as_float(v1[4 * q + 1]),
+                                   __uint_as_float(v1[4 * q + 2]), __uint_as_float(v1[4 * q + 3]));
+        }
+      }
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch) {
+        const uint32_t* v = ch < 4 ? v0 : v1;
+        const uint32_t w = ch < 4 ? w0 : w1;
+        const int b0 = (ch & 3) * 8;
+        float f[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) f[e] = ((w >> (b0 + e)) & 1u) ? __uint_as_float(v[b0 + e]) : 0.f;
+        st_sw128(sA, row, ch, make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                                         pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7])));
+      }
+      fence_async_smem();
+      tc_fence_before();
+      __syncthreads();
+      if (tid == 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int k16 = 0; k16 < 4; ++k16)
+          mma_bf16(tmem + 64, sdesc(smem_u32(sA) + k16 * 32, 16, 1024),
+                   sdesc(smem_u32(sPh + c * BC * 128) + k16 * 32, 16, 1024), idesc2, (c | k16) != 0);
+        mma_commit(bar_mma2);
+      }
+    }
+    if (!ok) break;
+    n2 += NCH;
+    // the W buffer of this tile is free once its MMAs are done: stream tile k + 2 into it
+    if (tid == 0 && k + 2 < nloc) {
+      if (mbar_wait(bar_mma2, (n2 - 1) & 1u, abort_flag, 43)) {
+        mbar_expect_tx(bar_full0 + 8 * b, C::W_BYTES);
+        load_w(k + 2, b);
+        issued = k + 3;
+      } else {
+        *abort_flag = 1;
+      }
+    }
+    ok = __syncthreads_and(mbar_wait(bar_mma2, (n2 - 1) & 1u, abort_flag, 44));
+    if (!ok) break;
+    tc_fence_after();
+#pragma unroll 1
+    for (int cc = 0; cc < BC / 32; ++cc) {
+      uint32_t r[32];
+      tmem_ld32(tmem + lane_off + 64 + cc * 32, r);
+      tmem_ld_wait();
+      if (grow < cout) {
+        uint4* o = reinterpret_cast<uint4*>(At + (size_t)grow * cin + col0 + cc * 32);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          o[q] = make_uint4(pack_bf16x2(__uint_as_float(r[8 * q]), __uint_as_float(r[8 * q + 1])),
+                            pack_bf16x2(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3])),
+                            pack_bf16x2(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5])),
+                            pack_bf16x2(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7])));
+      }
+    }
+    tc_fence_before();
+    __syncthreads();   // the next tile's MMAs overwrite the accumulators just read
+  }
+  if (tid == 0) {
+    for (int kk = consumed; kk < issued; ++kk)
+      mbar_wait_drain(bar_full0 + 8 * (kk & 1), (uint32_t)(kk >> 1) & 1u, 45);
+    mma_commit(bar_drain);
+    mbar_wait_drain(bar_drain, 0, 46);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+template <int BC, int MG>
+lcp_status permute_mask2_bc(const CUtensorMap& mW, const CUtensorMap& mPth, const CUtensorMap& mPtl,
+                            const CUtensorMap& mPh, uint32_t* mask, __nv_bfloat16* At, float* Wp, int cout,
+                            int cin, int n, cudaStream_t st) {
+  using C = Pm2Cfg<BC>;
+  auto k = permute_mask_tc2_kernel<BC, MG>;
+  TC_TRY(set_smem(k, C::SMEM, "permute_mask_tc"));
+  const int ntiles = cin / BC, nrt = cdiv(cout, 128);
+  int ry = cdiv(C::CTAS_PER_SM * num_sms(), ntiles);
+  if (ry > nrt) ry = nrt;
+  if (ry < 1) ry = 1;
+  k<<<dim3(ntiles, ry), 128, C::SMEM, st>>>(mW, mPth, mPtl, mPh, mask, At, Wp, cout, cin, n);
+  return check_launch("permute_mask_tc");
+}
+
+template <int BC, int MG>
+lcp_status permute_mask_bc(const CUtensorMap& mW, const CUtensorMap& mPth, const CUtensorMap& mPtl,
+                           const CUtensorMap& mPh, uint32_t* mask, __nv_bfloat16* At, float* Wp, int cout,
+                           int cin, int n, cudaStream_t st) {
+  auto k = permute_mask_tc_kernel<BC, MG>;
+  TC_TRY(set_smem(k, PmCfg<BC>::SMEM, "permute_mask_tc"));
+  const dim3 grid(cdiv(cout, 128), cin / BC);
+  k<<<grid, 128, PmCfg<BC>::SMEM, st>>>(mW, mPth, mPtl, mPh, mask, At, Wp, cout, cin, n);
+  return check_launch("permute_mask_tc");
+}
+
+}  // namespace
+
+lcp_status tc_error_permute(int* site, int reset) { return read_tc_error(site, reset); }
+
+lcp_status launch_permute_mask_tc(const __nv_bfloat16* W, const __nv_bfloat16* img_pt_hi,
+                                  const __nv_bfloat16* img_pt_lo, const __nv_bfloat16* img_p_hi, uint32_t* mask,
+                                  __nv_bfloat16* At, float* Wp_out, int cout, int cin, int B, int n, int m,
+                                  cudaStream_t st) {
+  const int BC = B < 64 ? 64 : B;
+  CUtensorMap mW, mPth, mPtl, mPh;
+  TC_TRY(make_map(&mW, W, cin, cout, 64, 128, "permute_mask W"));
+  TC_TRY(make_map(&mPth, img_pt_hi, BC, cin, 64, 64, "permute_mask Pt_hi"));
+  TC_TRY(make_map(&mPtl, img_pt_lo, BC, cin, 64, 64, "permute_mask Pt_lo"));
+  TC_TRY(make_map(&mPh, img_p_hi, BC, cin, 64, BC == 64 ? 64 : BC, "permute_mask P_hi"));
+  if (BC == 64) {
+    CUtensorMap mAt;
+    TC_TRY(make_map(&mAt, At, cin, cout, 64, 128, "permute_mask At"));
+    constexpr int NSL = 2;
+    using C = PwCfg<NSL>;
+    auto k = (m == 4) ? permute_mask_ws_kernel<4, NSL> : permute_mask_ws_kernel<8, NSL>;
+    TC_TRY(set_smem(k, C::SMEM, "permute_mask_tc"));
+    const int tiles = cdiv(cout, 128) * (cin / 64);
+    const int grid = tiles < num_sms() ? tiles : num_sms();
+    k<<<grid, C::THREADS, C::SMEM, st>>>(mW, mPth, mPtl, mPh, mAt, mask, Wp_out, cout, cin, n);
+    return check_launch("permute_mask_tc");
+  }
+  if (m == 4) {
+    if (BC == 128) return permute_mask2_bc<128, 4>(mW, mPth, mPtl, mPh, mask, At, Wp_out, cout, cin, n, st);
+    return permute_mask_bc<256, 4>(mW, mPth, mPtl, mPh, mask, At, Wp_out, cout, cin, n, st);
+  }
+  if (BC == 128) return permute_mask2_bc<128, 8>(mW, mPth, mPtl, mPh, mask, At, Wp_out, cout, cin, n, st);
+  return permute_mask_bc<256, 8>(mW, mPth, mPtl, mPh, mask, At, Wp_out, cout, cin, n, st);
+}
+
+}  // namespace lcp
