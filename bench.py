@@ -255,55 +255,59 @@ def main():
     uuid = f"GPU-{uuid}" if uuid and not str(uuid).startswith("GPU-") else (str(uuid) if uuid else None)
     sampler = ClockSampler(uuid if world == 1 else None)
 
-    def timed_loop(graph_mode):
-        """K timed steps; returns (total ms of our kernels, per-stage ms averages)."""
-        if graph_mode:
-            ev = [torch.cuda.Event(enable_timing=True) for _ in range(b.TIMED_EVENTS)]
-            for e in ev:
-                e.record()
-            g = b.capture(step, ev)
-            for _ in range(args.warmup):
-                g.replay()
-        else:
-            ev = None
-            for _ in range(args.warmup):
-                step.run()
+    def time_steps(run_one):
+        """W warm-up calls, then K timed ones with L2 flushed before each; the
+        device time between events recorded right before and after each call."""
+        for _ in range(args.warmup):
+            run_one()
         torch.cuda.synchronize()
-        rows = []
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
-        for _ in range(K):
+        e0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        e1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        for k in range(K):
             flush.zero_()                      # L2 flush, outside the timed events
-            if graph_mode:
-                g.replay()
-                torch.cuda.synchronize()       # the stage events are reused by every replay
-                rows.append([ev[s].elapsed_time(ev[s + 1]) for s in range(len(b.STAGES))])
-            else:
-                e = [torch.cuda.Event(enable_timing=True) for _ in range(b.TIMED_EVENTS)]
-                for x in e:
-                    x.record()
-                step.run_timed(e)
-                rows.append(e)
+            e0[k].record()
+            run_one()
+            e1[k].record()
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
-        if not graph_mode:
-            rows = [[e[s].elapsed_time(e[s + 1]) for s in range(len(b.STAGES))] for e in rows]
-        total = sum(sum(r) for r in rows)
-        per_stage = {name: sum(r[i] for r in rows) / K for i, name in enumerate(b.STAGES)}
-        if graph_mode:
-            del g
-        return total, per_stage
+        return sum(e0[k].elapsed_time(e1[k]) for k in range(K))
 
+    def stage_breakdown():
+        """Per-stage averages from a graph that also records the stage events
+        (an event between two kernels keeps the second from starting early, so
+        these stages add up to a little more than the headline step time)."""
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(b.TIMED_EVENTS)]
+        for e in ev:
+            e.record()
+        g = b.capture(step, ev)
+        for _ in range(args.warmup):
+            g.replay()
+        rows = []
+        for _ in range(K):
+            flush.zero_()
+            g.replay()
+            torch.cuda.synchronize()           # the stage events are reused by every replay
+            rows.append([ev[s].elapsed_time(ev[s + 1]) for s in range(len(b.STAGES))])
+        del g
+        return {name: sum(r[i] for r in rows) / K for i, name in enumerate(b.STAGES)}
+
+    graph_mode = not args.eager
     sampler.start()
     time.sleep(0.2)
-    graph_mode = not args.eager
-    total_ms, stage_ms = timed_loop(graph_mode)
-    clocks = sampler.stop()
-    eager_total = None
     if graph_mode:
-        eager_total, _ = timed_loop(False)
+        g_step = b.capture(step)
+        total_ms = time_steps(g_step.replay)
+    else:
+        total_ms = time_steps(step.run)
+    clocks = sampler.stop()
+    eager_total = time_steps(step.run) if graph_mode else None
+    if graph_mode:
+        del g_step
+    stage_ms = stage_breakdown()
 
     max_ms, max_eager = parallel.max_over_ranks([total_ms, eager_total or 0.0], device=dev)
     value = parallel.job_throughput(K, world, max_ms)
@@ -311,7 +315,11 @@ def main():
     if eager_total is not None:
         eager = {"value": parallel.job_throughput(K, world, max_eager), "ms_per_step": max_eager / K}
 
-    # end to end through the public API: pinned host inputs in, loss and dL out, every step
+    # End to end through the public API: every step copies its inputs (W, X, L)
+    # from pinned host memory and reads its results (loss, dL) back.  Two device
+    # input sets on a copy stream keep the host-to-device copy of step k + 1 in
+    # flight while step k computes (a 2-deep pipeline); the time runs from the
+    # first copy to the last read-back.
     e2e = None
     if not args.no_e2e:
         hW = torch.from_numpy(li.W).to(tdt).pin_memory()
@@ -319,28 +327,45 @@ def main():
         hL = torch.from_numpy(li.L).pin_memory()
         hloss = torch.empty(4, dtype=torch.float32).pin_memory()
         hdL = torch.empty_like(hL).pin_memory()
-        Ke = max(3, min(K, 20))
-        a0 = [torch.cuda.Event(enable_timing=True) for _ in range(Ke)]
-        a1 = [torch.cuda.Event(enable_timing=True) for _ in range(Ke)]
-        for k in range(Ke + 2):
-            kk = k - 2
-            if kk >= 0:
-                a0[kk].record(stream)
-            layer["W"].copy_(hW, non_blocking=True)
-            layer["X"].copy_(hX, non_blocking=True)
-            layer["L"].copy_(hL, non_blocking=True)
-            step.run()
-            hloss.copy_(layer["loss"], non_blocking=True)
-            hdL.copy_(layer["dL"], non_blocking=True)
-            if kk >= 0:
-                a1[kk].record(stream)
-            stream.synchronize()
-        e_ms = sum(a0[k].elapsed_time(a1[k]) for k in range(Ke))
-        (te_ms,) = parallel.max_over_ranks([e_ms / Ke], device=dev)
+        layer2 = b.alloc_outputs(torch.empty_like(W), torch.empty_like(X), torch.empty_like(L))
+        sets = [layer, layer2]
+        steps = [step, b.Step([layer2], wl.block, wl.n, wl.m, wl.iters, wl.tau, flags=flags, workspace=step.ws)]
+        cstream = torch.cuda.Stream()
+        copied = [torch.cuda.Event(), torch.cuda.Event()]
+        freed = [torch.cuda.Event(), torch.cuda.Event()]
+
+        def issue(k):
+            j = k % 2
+            with torch.cuda.stream(cstream):
+                if k >= 2:
+                    cstream.wait_event(freed[j])          # step k - 2 is done with input set j
+                sets[j]["W"].copy_(hW, non_blocking=True)
+                sets[j]["X"].copy_(hX, non_blocking=True)
+                sets[j]["L"].copy_(hL, non_blocking=True)
+                copied[j].record(cstream)
+            stream.wait_event(copied[j])
+            steps[j].run(stream)
+            hloss.copy_(sets[j]["loss"], non_blocking=True)
+            hdL.copy_(sets[j]["dL"], non_blocking=True)
+            freed[j].record(stream)
+
+        Ke = max(4, min(K, 20))
+        for k in range(2):
+            issue(k)
+        torch.cuda.synchronize()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(cstream)
+        for k in range(Ke):
+            issue(k)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        (te_ms,) = parallel.max_over_ranks([t0.elapsed_time(t1) / Ke], device=dev)
         h2d = hW.numel() * hW.element_size() + hX.numel() * hX.element_size() + hL.numel() * 4
         d2h = 4 * 4 + hdL.numel() * 4
         e2e = {"value": parallel.job_throughput(1, world, te_ms), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
-               "d2h_bytes_per_step": int(d2h)}
+               "d2h_bytes_per_step": int(d2h), "steps": Ke,
+               "pipeline": "2 input sets: step k+1's host-to-device copy overlaps step k"}
 
     if world > 1:
         dist.barrier()
@@ -382,7 +407,8 @@ def main():
                        "parallelism": f"layer-sharded x{world}" if world > 1 else "single GPU",
                        "l2": "flushed between timed steps (256 MiB write)",
                        "path": "simt" if args.simt else "tcgen05",
-                       "launch": "cuda-graph replay per step" if graph_mode else "eager launches"},
+                       "launch": "cuda-graph replay per step" if graph_mode else "eager launches",
+                       "pdl": os.environ.get("LCP_PDL", "1") != "0"},
             "roofline": roof, "stages": per_stage, "clocks": clocks, "e2e": e2e, "eager": eager,
             "gpu_launches": step.launches * K}
     if world == 1 and not args.no_cpu_baseline:

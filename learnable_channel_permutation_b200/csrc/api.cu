@@ -7,6 +7,7 @@
 //   evaluated as (M.W' P_B^T) X  ->  token-mean cosine loss (objective)
 //   ->  reverse pass to the logits with the mask held constant.
 
+#include <cstdlib>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -51,6 +52,14 @@ lcp_status ensure_smem_limit(const void* func, int bytes, const char* what) {
   }
   if (nseen < 256) seen[nseen++] = Entry{func, dev, bytes};
   return LCP_OK;
+}
+
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* v = std::getenv("LCP_PDL");
+    return !(v && v[0] == '0');
+  }();
+  return on;
 }
 
 lcp_status check_launch(const char* what) {
@@ -242,7 +251,8 @@ lcp_status layer_simt(const lcp_layer& l, const lcp_hparams& hp, const Plan& p, 
   const long long ic = l.cin, oc = l.cout, BB = (long long)B * B;
 
   LCP_TRY(record(ev, 0, st));
-  LCP_TRY(launch_sinkhorn_fwd(l.L, l.P, ckpt, nullptr, nullptr, nullptr, nb, B, hp.tau, hp.iters, st));
+  LCP_TRY(launch_sinkhorn_fwd(l.L, l.P, ckpt, nullptr, nullptr, nullptr, at<unsigned>(ws, p.counter), nb, B, hp.tau,
+                              hp.iters, st));
   LCP_TRY(record(ev, 1, st));
   // W'_b = W_b P_b
   LCP_TRY(launch_simt_gemm({l.cout, B, B, nb, l.W, B, ic, 1, l.P, BB, B, 1, Wp, B, ic, 1, 1.f, 0.f},
@@ -311,7 +321,8 @@ lcp_status layer_tc(const lcp_layer& l, const lcp_hparams& hp, const Plan& p, vo
   const auto* X = static_cast<const __nv_bfloat16*>(l.X);
 
   LCP_TRY(record(ev, 0, st));
-  LCP_TRY(launch_sinkhorn_fwd(l.L, l.P, ckpt, pt_hi, pt_lo, p_hi, nb, B, hp.tau, hp.iters, st));
+  LCP_TRY(launch_sinkhorn_fwd(l.L, l.P, ckpt, pt_hi, pt_lo, p_hi, at<unsigned>(ws, p.counter), nb, B, hp.tau,
+                              hp.iters, st));
   LCP_TRY(record(ev, 1, st));
   LCP_TRY(launch_permute_mask_tc(W, pt_hi, pt_lo, p_hi, mask, At, Wp, l.cout, l.cin, B, hp.n, hp.m, st));
   LCP_TRY(record(ev, 2, st));
@@ -438,7 +449,7 @@ lcp_status lcp_sinkhorn_fwd(const float* L, float* P, float* ckpt, int nblocks, 
   if (nblocks == 0) return LCP_OK;
   LCP_TRY(check_arch());
   cudaGetLastError();
-  return launch_sinkhorn_fwd(L, P, ckpt, nullptr, nullptr, nullptr, nblocks, B, tau, iters, stream);
+  return launch_sinkhorn_fwd(L, P, ckpt, nullptr, nullptr, nullptr, nullptr, nblocks, B, tau, iters, stream);
 }
 
 lcp_status lcp_sinkhorn_bwd(const float* L, const float* ckpt, const float* dP, int dP_splits,

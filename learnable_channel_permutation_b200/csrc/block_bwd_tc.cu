@@ -72,6 +72,8 @@ block_bwd_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_consta
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *holder;
+  pdl_wait();
+  pdl_trigger();
   const uint32_t tDP = tmem + 256;
 
   if (warp == 0) {
@@ -305,6 +307,8 @@ block_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_consta
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *holder;
+  pdl_wait();
+  pdl_trigger();
   const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
   const int row = warp * 32 + lane;
   const int words = cin / 32;
@@ -470,8 +474,8 @@ lcp_status block_bwd_bc(const CUtensorMap& mW, const CUtensorMap& mD, const CUte
   auto k = block_bwd_tc_kernel<BC, B>;
   TC_TRY(set_smem(k, BbCfg<BC>::SMEM, "block_bwd_tc"));
   const dim3 grid(cin / BC, splits);
-  k<<<grid, 128, BbCfg<BC>::SMEM, st>>>(mW, mD, mPth, mPtl, mask, dP, cout, cin, rows);
-  return check_launch("block_bwd_tc");
+  return launch_kernel(k, grid, dim3(128), BbCfg<BC>::SMEM, st, 1, true, "block_bwd_tc", mW, mD, mPth, mPtl, mask,
+                       dP, cout, cin, rows);
 }
 
 int bb_rows_per_split(int cout, int cin, int B) {
@@ -514,8 +518,8 @@ lcp_status launch_block_bwd_tc(const __nv_bfloat16* W, const __nv_bfloat16* dAt,
     using C = BwCfg<NSL>;
     auto k = (B == 32) ? block_bwd_ws_kernel<32, NSL> : block_bwd_ws_kernel<64, NSL>;
     TC_TRY(set_smem(k, C::SMEM, "block_bwd_tc"));
-    k<<<dim3(cin / 64, splits), C::THREADS, C::SMEM, st>>>(mW, mD, mPth, mPtl, mask, dP_partials, cout, cin, rows);
-    return check_launch("block_bwd_tc");
+    return launch_kernel(k, dim3(cin / 64, splits), dim3(C::THREADS), C::SMEM, st, 1, true, "block_bwd_tc", mW, mD,
+                         mPth, mPtl, mask, dP_partials, cout, cin, rows);
   }
   return block_bwd_bc<128, 128>(mW, mD, mPth, mPtl, mask, dP_partials, splits, rows, cout, cin, st);
 }

@@ -61,6 +61,8 @@ gemm_pair_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
   cluster_sync_all();   // both CTAs' barriers exist before either touches the other's
   tc_fence_after();
   const uint32_t tmem = *holder;
+  pdl_wait();           // operands come from the previous kernel
+  pdl_trigger();
 
   const int mtiles = cdiv(M, G2_BM), ntiles = cdiv(N, G2_BN);
   const int total = mtiles * ntiles * nprob;
@@ -214,24 +216,8 @@ lcp_status launch_pair(K kernel, int tiles, const CUtensorMap& a, const CUtensor
   TC_TRY(set_smem(kernel, G2_SMEM, what));
   const int max_pairs = num_sms() / 2;
   const int pairs = tiles < max_pairs ? tiles : max_pairs;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * pairs);
-  cfg.blockDim = dim3(GM_THREADS);
-  cfg.dynamicSmemBytes = G2_SMEM;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, a, b0, b1, d0, d1, M, N, Kd, ldd, nprob);
-  if (e != cudaSuccess) {
-    cudaGetLastError();
-    return fail(LCP_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
-  }
-  return check_launch(what);
+  return launch_kernel(kernel, dim3(2 * pairs), dim3(GM_THREADS), G2_SMEM, st, 2, true, what, a, b0, b1, d0, d1, M, N,
+                       Kd, ldd, nprob);
 }
 
 }  // namespace

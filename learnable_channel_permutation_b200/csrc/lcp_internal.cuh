@@ -19,6 +19,51 @@ lcp_status check_launch(const char* what);
 // unless an earlier call already did (the attribute persists for the process).
 lcp_status ensure_smem_limit(const void* func, int bytes, const char* what);
 
+// ---- programmatic dependent launch -------------------------------------
+// A kernel launched with pdl = true (launch_kernel below) may start while the
+// kernel before it on the stream is still finishing.  It calls pdl_wait()
+// before touching any global memory that an earlier kernel writes or reads
+// (the only exception: the permute kernels prefetch the weight W, which no
+// kernel of a step writes), and pdl_trigger() after its own pdl_wait(), which
+// lets the next kernel start its prologue.  Launched without the attribute,
+// both are no-ops.  LCP_PDL=0 in the environment turns the attribute off.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+bool pdl_enabled();
+
+// Launches `kernel` with an optional cluster size (x) and the PDL attribute.
+template <typename... KArgs, typename... Args>
+lcp_status launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                         int cluster, bool pdl, const char* what, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  unsigned na = 0;
+  if (cluster > 1) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = (unsigned)cluster;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  if (pdl && pdl_enabled()) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(LCP_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  }
+  return check_launch(what);
+}
+
 // ---- element conversions -------------------------------------------------
 __device__ __forceinline__ float to_f32(float v) { return v; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
@@ -26,6 +71,36 @@ template <typename T> __device__ __forceinline__ T from_f32(float v);
 template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
 template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) {
   return __float2bfloat16_rn(v);
+}
+
+// ---- N:4 keep bits --------------------------------------------------------
+// Bit j of the result keeps element j of NV consecutive values (NV / 4 groups
+// of M = 4 consecutive columns), bit-sliced.  For each
+// element three words record whether it beats each of the other three members
+// of its group (j beats k when |v_j| > |v_k|, or the two are equal and j < k);
+// on the 31-bit magnitudes u the test is the sign of a difference:
+// u_j >= u_k exactly when u_k - u_j - 1 < 0, and u_j > u_k when u_k - u_j < 0.
+// An element is kept when it beats at least 4 - n of the others: all three
+// (n = 1, bitwise AND), two of three (n = 2, bitwise majority) or one (n = 3,
+// OR); n = 4 keeps every element.
+__device__ __forceinline__ uint32_t sign_to(uint32_t d, int pos) { return (d >> 31) << pos; }
+template <int NV>
+__device__ __forceinline__ uint32_t nm4_keep(const uint32_t (&v)[NV], int n) {
+  uint32_t X = 0, Y = 0, Z = 0;   // element j's 1st, 2nd and 3rd opponent, in index order
+#pragma unroll
+  for (int g = 0; g < NV / 4; ++g) {
+    const uint32_t u0 = v[4 * g] & 0x7fffffffu, u1 = v[4 * g + 1] & 0x7fffffffu;
+    const uint32_t u2 = v[4 * g + 2] & 0x7fffffffu, u3 = v[4 * g + 3] & 0x7fffffffu;
+    const int b = 4 * g;
+    X |= sign_to(u1 - u0 - 1, b) | sign_to(u0 - u1, b + 1) | sign_to(u0 - u2, b + 2) | sign_to(u0 - u3, b + 3);
+    Y |= sign_to(u2 - u0 - 1, b) | sign_to(u2 - u1 - 1, b + 1) | sign_to(u1 - u2, b + 2) | sign_to(u1 - u3, b + 3);
+    Z |= sign_to(u3 - u0 - 1, b) | sign_to(u3 - u1 - 1, b + 1) | sign_to(u3 - u2 - 1, b + 2) |
+         sign_to(u2 - u3, b + 3);
+  }
+  const uint32_t all3 = X & Y & Z, two = (X & Y) | (X & Z) | (Y & Z), one = X | Y | Z;
+  if (n >= 4) return 0xffffffffu;   // nothing pruned
+  if (n <= 0) return 0u;
+  return n == 1 ? all3 : (n == 2 ? two : one);
 }
 
 // ---- launchers (host side; each returns LCP_OK or LCP_ERR_CUDA) ----------
@@ -36,9 +111,11 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 //   img_pt_hi[t][j][i] = bf16(P[i][j])          (transposed, high part)
 //   img_pt_lo[t][j][i] = bf16(P[i][j] - hi)     (transposed, low part)
 //   img_p_hi [t][i][j] = bf16(P[i][j])          (high part)
+// zero_word (optional) is set to 0 by the first CTA: the counter of the
+// layer's fused loss kernel, which runs later on the same stream.
 lcp_status launch_sinkhorn_fwd(const float* L, float* P, float* ckpt, __nv_bfloat16* img_pt_hi,
-                               __nv_bfloat16* img_pt_lo, __nv_bfloat16* img_p_hi, int nblocks,
-                               int B, float tau, int iters, cudaStream_t st);
+                               __nv_bfloat16* img_pt_lo, __nv_bfloat16* img_p_hi, unsigned* zero_word,
+                               int nblocks, int B, float tau, int iters, cudaStream_t st);
 lcp_status launch_sinkhorn_bwd(const float* L, const float* ckpt, const float* dP, int splits,
                                float* dL, int nblocks, int B, float tau, int iters,
                                cudaStream_t st);
@@ -68,7 +145,8 @@ lcp_status launch_loss_token(const float* Yd, const float* Ys, float* stats, voi
 lcp_status launch_loss_grad(const float* Yd, const float* Ys, const float* stats, void* G,
                             lcp_dtype gdt, int cout, int tokens, cudaStream_t st);
 lcp_status launch_loss_reduce(const float* stats, float* loss, int tokens, cudaStream_t st);
-// One launch (plus a 4-byte counter reset): stats, G and the loss.  cout <= 16384.
+// One launch: stats, G and the loss.  cout <= 16384.  `counter` must be zero
+// at launch (an earlier kernel of the step clears it); the kernel leaves it zero.
 bool loss_fused_supported(int cout);
 lcp_status launch_loss_fused(const float* Yd, const float* Ys, float* stats, void* G, lcp_dtype gdt,
                              float* loss, unsigned* counter, int cout, int tokens, cudaStream_t st);

@@ -64,6 +64,8 @@ template <typename TG, bool WRITE_G>
 __global__ void __launch_bounds__(NT)
 loss_token_kernel(const float* __restrict__ Yd, const float* __restrict__ Ys,
                   float* __restrict__ stats, TG* __restrict__ G, int cout, float inv_T) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float red[3][NT / 32];
   const int t = blockIdx.x;
   const size_t row = (size_t)t * cout;
@@ -99,6 +101,8 @@ template <typename TG>
 __global__ void __launch_bounds__(NT)
 loss_grad_kernel(const float* __restrict__ Yd, const float* __restrict__ Ys,
                  const float* __restrict__ stats, TG* __restrict__ G, int cout, float inv_T) {
+  pdl_wait();
+  pdl_trigger();
   const int t = blockIdx.x;
   const size_t row = (size_t)t * cout;
   const float4 s = reinterpret_cast<const float4*>(stats)[t];
@@ -118,6 +122,8 @@ __global__ void __launch_bounds__(NTH, PREFETCH ? 2 : 1)
 loss_fused_kernel(const float* __restrict__ Yd, const float* __restrict__ Ys, float* __restrict__ stats,
                   TG* __restrict__ G, float* __restrict__ loss, unsigned* __restrict__ counter, int cout,
                   int tokens, float inv_T) {
+  pdl_wait();
+  pdl_trigger();
   constexpr int NWARP = NTH / 32;
   __shared__ float red[2][3][NWARP];
   __shared__ double redd[NWARP];
@@ -210,6 +216,8 @@ loss_fused_kernel(const float* __restrict__ Yd, const float* __restrict__ Ys, fl
 
 __global__ void __launch_bounds__(1024)
 loss_reduce_kernel(const float* __restrict__ stats, float* __restrict__ loss, int tokens) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ double red[32];
   double s = 0.0;
   for (int t = threadIdx.x; t < tokens; t += 1024) s += 1.0 - (double)stats[4 * (size_t)t + 3];
@@ -229,25 +237,26 @@ loss_reduce_kernel(const float* __restrict__ stats, float* __restrict__ loss, in
 lcp_status launch_loss_token(const float* Yd, const float* Ys, float* stats, void* G,
                              lcp_dtype gdt, int cout, int tokens, cudaStream_t st) {
   const float inv_T = 1.0f / (float)tokens;
-  if (!G) {
-    loss_token_kernel<float, false><<<tokens, NT, 0, st>>>(Yd, Ys, stats, nullptr, cout, inv_T);
-  } else if (gdt == LCP_F32) {
-    loss_token_kernel<float, true><<<tokens, NT, 0, st>>>(Yd, Ys, stats, (float*)G, cout, inv_T);
-  } else {
-    loss_token_kernel<__nv_bfloat16, true>
-        <<<tokens, NT, 0, st>>>(Yd, Ys, stats, (__nv_bfloat16*)G, cout, inv_T);
-  }
-  return check_launch("loss_token");
+  const dim3 grid(tokens), block(NT);
+  if (!G)
+    return launch_kernel(loss_token_kernel<float, false>, grid, block, 0, st, 1, true, "loss_token", Yd, Ys, stats,
+                         (float*)nullptr, cout, inv_T);
+  if (gdt == LCP_F32)
+    return launch_kernel(loss_token_kernel<float, true>, grid, block, 0, st, 1, true, "loss_token", Yd, Ys, stats,
+                         (float*)G, cout, inv_T);
+  return launch_kernel(loss_token_kernel<__nv_bfloat16, true>, grid, block, 0, st, 1, true, "loss_token", Yd, Ys,
+                       stats, (__nv_bfloat16*)G, cout, inv_T);
 }
 
 lcp_status launch_loss_grad(const float* Yd, const float* Ys, const float* stats, void* G,
                             lcp_dtype gdt, int cout, int tokens, cudaStream_t st) {
   const float inv_T = 1.0f / (float)tokens;
+  const dim3 grid(tokens), block(NT);
   if (gdt == LCP_F32)
-    loss_grad_kernel<float><<<tokens, NT, 0, st>>>(Yd, Ys, stats, (float*)G, cout, inv_T);
-  else
-    loss_grad_kernel<__nv_bfloat16><<<tokens, NT, 0, st>>>(Yd, Ys, stats, (__nv_bfloat16*)G, cout, inv_T);
-  return check_launch("loss_grad");
+    return launch_kernel(loss_grad_kernel<float>, grid, block, 0, st, 1, true, "loss_grad", Yd, Ys, stats,
+                         (float*)G, cout, inv_T);
+  return launch_kernel(loss_grad_kernel<__nv_bfloat16>, grid, block, 0, st, 1, true, "loss_grad", Yd, Ys, stats,
+                       (__nv_bfloat16*)G, cout, inv_T);
 }
 
 bool loss_fused_supported(int cout) { return cout <= 8 * 4 * 512; }
@@ -255,35 +264,27 @@ bool loss_fused_supported(int cout) { return cout <= 8 * 4 * 512; }
 lcp_status launch_loss_fused(const float* Yd, const float* Ys, float* stats, void* G, lcp_dtype gdt,
                              float* loss, unsigned* counter, int cout, int tokens, cudaStream_t st) {
   const float inv_T = 1.0f / (float)tokens;
-  const cudaError_t e = cudaMemsetAsync(counter, 0, sizeof(unsigned), st);
-  if (e != cudaSuccess) {
-    cudaGetLastError();
-    return fail(LCP_ERR_CUDA, "loss counter reset: %s", cudaGetErrorString(e));
-  }
   const int quads = cout / 4;
   int sms = 148, dev = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int grid = tokens < 2 * sms ? tokens : 2 * sms;
-#define LCP_LOSS_FUSED(TG, NTH, QPT)                                                                \
-  loss_fused_kernel<TG, NTH, QPT, (QPT <= 4)><<<grid, NTH, 0, st>>>(Yd, Ys, stats, static_cast<TG*>(G), \
-                                                                    loss, counter, cout, tokens, inv_T)
+  const dim3 grid(tokens < 2 * sms ? tokens : 2 * sms);
+#define LCP_LOSS_FUSED(TG, NTH, QPT)                                                                             \
+  return launch_kernel(loss_fused_kernel<TG, NTH, QPT, (QPT <= 4)>, grid, dim3(NTH), 0, st, 1, true, "loss_fused", \
+                       Yd, Ys, stats, static_cast<TG*>(G), loss, counter, cout, tokens, inv_T)
   if (gdt == LCP_F32) {
     if (quads <= 4 * 256) LCP_LOSS_FUSED(float, 256, 4);
-    else if (quads <= 8 * 256) LCP_LOSS_FUSED(float, 256, 8);
-    else LCP_LOSS_FUSED(float, 512, 8);
-  } else {
-    if (quads <= 4 * 256) LCP_LOSS_FUSED(__nv_bfloat16, 256, 4);
-    else if (quads <= 8 * 256) LCP_LOSS_FUSED(__nv_bfloat16, 256, 8);
-    else LCP_LOSS_FUSED(__nv_bfloat16, 512, 8);
+    if (quads <= 8 * 256) LCP_LOSS_FUSED(float, 256, 8);
+    LCP_LOSS_FUSED(float, 512, 8);
   }
+  if (quads <= 4 * 256) LCP_LOSS_FUSED(__nv_bfloat16, 256, 4);
+  if (quads <= 8 * 256) LCP_LOSS_FUSED(__nv_bfloat16, 256, 8);
+  LCP_LOSS_FUSED(__nv_bfloat16, 512, 8);
 #undef LCP_LOSS_FUSED
-  return check_launch("loss_fused");
 }
 
 lcp_status launch_loss_reduce(const float* stats, float* loss, int tokens, cudaStream_t st) {
-  loss_reduce_kernel<<<1, 1024, 0, st>>>(stats, loss, tokens);
-  return check_launch("loss_reduce");
+  return launch_kernel(loss_reduce_kernel, dim3(1), dim3(1024), 0, st, 1, true, "loss_reduce", stats, loss, tokens);
 }
 
 }  // namespace lcp

@@ -75,7 +75,14 @@ nm_mask_kernel(const T* __restrict__ Wp, uint32_t* __restrict__ bits, long long 
       }
     }
   }
-  bits[w] = word_bits<M>(v, n);
+  if constexpr (M == 4) {
+    uint32_t u[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(v[i]);
+    bits[w] = nm4_keep<32>(u, n);
+  } else {
+    bits[w] = word_bits<M>(v, n);
+  }
 }
 
 __global__ void __launch_bounds__(256)

@@ -62,6 +62,8 @@ permute_mask_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *holder;
+  pdl_wait();
+  pdl_trigger();
   const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
   const int row = warp * 32 + lane, grow = r0 + row;
   const int words = cin / 32;
@@ -110,7 +112,8 @@ permute_mask_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
     tmem_ld32(tmem + lane_off + 0, v0);
     tmem_ld32(tmem + lane_off + 32, v1);
     tmem_ld_wait();
-    const uint32_t w0 = nm_word<MGROUP>(v0, n), w1 = nm_word<MGROUP>(v1, n);
+    const uint32_t w0 = MGROUP == 4 ? nm4_keep<32>(v0, n) : nm_word<MGROUP>(v0, n);
+    const uint32_t w1 = MGROUP == 4 ? nm4_keep<32>(v1, n) : nm_word<MGROUP>(v1, n);
     if (grow < cout) {
       const int wi = (col0 + c * 64) / 32;
       mask[(size_t)grow * words + wi] = w0;
@@ -185,232 +188,328 @@ permute_mask_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
 }
 
 // ------------------------------------- permute + mask, warp-specialised ---
-// BC = 64 (B = 32 or 64).  Persistent CTAs walk a flat list of (channel tile,
-// row tile) pairs.  Warp 0 streams each tile's W block together with its P
-// images into a 3-stage ring; warp 1 issues W' = W (P_hi + P_lo) into one of
-// two TMEM buffers and, once the epilogue has written A = M.W' to shared
-// memory, At = A P_hi into the same buffer; warps 2-9 (two per TMEM lane
-// quadrant, 32 columns each) compute the mask, write A, and copy At out
-// through a swizzled staging tile with TMA stores.
-template <int NSL> struct PwCfg {
-  static constexpr int STAGES = 3;
+// BC = 64 (B = 32 or 64).  CTA c takes the contiguous run
+// [c * total / G, (c + 1) * total / G) of the flat (channel tile t, row tile
+// rt) list in t-major order, so a run walks down one or two channel strips
+// (more only when C_out is short) and the three P images of its current
+// channel tile stay resident in one of two shared-memory slots.  The ring then
+// carries W tiles only and a stage is free as soon as W' of its tile is
+// formed, so the loads run STAGES tiles ahead of the tensor core.
+//   warp 0: TMA producer (W ring; the images of each channel tile once)
+//   warp 1: MMA issuer: W' = W (P_hi + P_lo) of tile k + 2 into TMEM buffer
+//           (k + 2) % NB, then, once A = M.W' of tile k is in shared memory,
+//           At = A P_hi of tile k into buffer k % NB
+//   warps 2-9: mask warps (two per TMEM lane quadrant, 32 columns each): W'
+//           of tile k -> the N:M keep bits (stored to the mask) and A
+//   warps 10-13: copy-out warps (one per quadrant, 64 columns each): At of
+//           tile k -> swizzled staging tile -> TMA store
+// The two epilogue roles run side by side (the mask is ALU work, the copy-out
+// memory traffic) and meet only through mbarriers; the mask warps never wait
+// for the tensor core in steady state.
+struct PwCfg {
+  static constexpr int STAGES = 5;
+  static constexpr int NB = 4;                          // TMEM (W', At) buffers of 128 columns
+  static constexpr int NA = 3;                          // A buffers
   static constexpr int W_BYTES = 16384;                 // 128 rows x 64 bf16
   static constexpr int IMG_BYTES = 8192;                // 64 x 64 bf16
-  static constexpr int STAGE = W_BYTES + 3 * IMG_BYTES; // W | Pt_hi | Pt_lo | P_hi
+  static constexpr int SLOT = 3 * IMG_BYTES;            // Pt_hi | Pt_lo | P_hi
   static constexpr int A_BYTES = 16384;
-  static constexpr int SMEM = STAGES * STAGE + 2 * A_BYTES + 2 * A_BYTES + 1024 + 256;
-  static constexpr int EPI_WARPS = 4 * NSL;              // NSL column slices per TMEM lane quadrant
-  static constexpr int COLS = 64 / NSL;                  // columns per epilogue thread
-  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
-  static constexpr int EPI = 32 * EPI_WARPS;
+  static constexpr int NBAR = 2 * STAGES + 4 * NB + NA + 4 * 2 + 1;
+  static constexpr int SMEM = STAGES * W_BYTES + 2 * SLOT + (NA + 2) * A_BYTES + NBAR * 8 + 16 + 1024;
+  static constexpr int MASK_WARPS = 8, COPY_WARPS = 4;
+  static constexpr int MASK0 = 2, COPY0 = MASK0 + MASK_WARPS;   // first warp of each role
+  static constexpr int THREADS = 32 * (COPY0 + COPY_WARPS);
+  static_assert(SMEM <= 232448, "shared memory budget");
 };
 
-template <int MGROUP, int NSL>
-__global__ void __launch_bounds__(PwCfg<NSL>::THREADS, 1)
+// position in the flat t-major tile list, advanced one tile at a time
+struct TileIter {
+  int t, rt, nrt;
+  __device__ TileIter(int idx, int nrt_) : t(idx / nrt_), rt(idx % nrt_), nrt(nrt_) {}
+  __device__ void next() {
+    if (++rt == nrt) { rt = 0; ++t; }
+  }
+};
+
+template <int MGROUP>
+__global__ void __launch_bounds__(PwCfg::THREADS, 1)
 permute_mask_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmPth,
                        const __grid_constant__ CUtensorMap tmPtl, const __grid_constant__ CUtensorMap tmPh,
                        const __grid_constant__ CUtensorMap tmAt, uint32_t* __restrict__ mask,
                        float* __restrict__ Wp_out, int cout, int cin, int n) {
-  using C = PwCfg<NSL>;
-  constexpr int NV = C::COLS;
+  using C = PwCfg;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sStage = smem;
-  uint8_t* sA = smem + C::STAGES * C::STAGE;          // 2 buffers
-  uint8_t* sO = sA + 2 * C::A_BYTES;                  // 2 staging tiles for At
+  uint8_t* sSlot = sStage + C::STAGES * C::W_BYTES;     // 2 slots of P images
+  uint8_t* sA = sSlot + 2 * C::SLOT;                    // NA buffers of A = M.W'
+  uint8_t* sO = sA + C::NA * C::A_BYTES;                // 2 staging tiles for At
   uint64_t* bars = reinterpret_cast<uint64_t*>(sO + 2 * C::A_BYTES);
-  // bars: full[3] empty[3] wf[2] af[2] atf[2] tmw[2] tma[2] drain
-  uint32_t* holder = reinterpret_cast<uint32_t*>(bars + 17);
+  uint32_t* holder = reinterpret_cast<uint32_t*>(bars + C::NBAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(holder + 1);
   auto bar = [&](int i) { return smem_u32(bars + i); };
-  const int FULL = 0, EMPTY = 3, WF = 6, AF = 8, ATF = 10, TMW = 12, TMA = 14, DRAIN = 16;
+  constexpr int NB = C::NB, NA = C::NA;
+  constexpr int FULL = 0, EMPTY = C::STAGES, WF = 2 * C::STAGES, ATF = WF + NB, TMW = ATF + NB, TMA = TMW + NB,
+                AF = TMA + NB, PREADY = AF + NA, PFREE = PREADY + 2, SFULL = PFREE + 2, SFREE = SFULL + 2,
+                DRAIN = SFREE + 2;
+  static_assert(DRAIN + 1 == C::NBAR, "barrier count");
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int nrt = cdiv(cout, 128), ntc = cin / 64;
   const int total = nrt * ntc;
-  const int nloc = (int)blockIdx.x < total ? cdiv(total - (int)blockIdx.x, (int)gridDim.x) : 0;
+  const int first = (int)((long long)blockIdx.x * total / gridDim.x);
+  const int last = (int)((long long)(blockIdx.x + 1) * total / gridDim.x);
+  const int nloc = last - first;
+  const int t_first = first / nrt;
+  const int nt = nloc > 0 ? (last - 1) / nrt - t_first + 1 : 0;   // channel tiles met by the run
   const int words = cin / 32;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 3; ++i) { mbar_init(bar(FULL + i), 1); mbar_init(bar(EMPTY + i), 1); }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < C::STAGES; ++i) { mbar_init(bar(FULL + i), 1); mbar_init(bar(EMPTY + i), 1); }
+    for (int i = 0; i < NB; ++i) {
       mbar_init(bar(WF + i), 1);
-      mbar_init(bar(AF + i), C::EPI_WARPS);
       mbar_init(bar(ATF + i), 1);
-      mbar_init(bar(TMW + i), C::EPI_WARPS);
-      mbar_init(bar(TMA + i), C::EPI_WARPS);
+      mbar_init(bar(TMW + i), C::MASK_WARPS);
+      mbar_init(bar(TMA + i), C::COPY_WARPS);
+    }
+    for (int i = 0; i < NA; ++i) mbar_init(bar(AF + i), C::MASK_WARPS);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(PREADY + i), 1);
+      mbar_init(bar(PFREE + i), 1);
+      mbar_init(bar(SFULL + i), C::COPY_WARPS);
+      mbar_init(bar(SFREE + i), 1);
     }
     mbar_init(bar(DRAIN), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 1) tmem_alloc(smem_u32(holder), 256);
+  if (warp == 1) tmem_alloc(smem_u32(holder), 128 * NB);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *holder;
-  auto tile_of = [&](int k, int& t, int& rt) {
-    const int idx = (int)blockIdx.x + k * (int)gridDim.x;
-    t = idx / nrt;
-    rt = idx % nrt;
+  // the producer prefetches W (never written by a kernel of the step) before waiting
+  if (warp != 0) {
+    pdl_wait();
+    pdl_trigger();
+  }
+  auto wait_all = [&](int b, uint32_t parity, int site) {
+    return __all_sync(0xffffffffu, mbar_wait(bar(b), parity, abort_flag, site));
   };
 
   if (warp == 0) {
     if (lane == 0) {
       uint32_t issued = 0, par = 0;   // per stage: outstanding load and its parity
-      for (int k = 0; k < nloc; ++k) {
+      uint32_t img_issued = 0;        // per slot: images in flight
+      int img_next = 0;               // next channel tile (run-local) whose images to load
+      bool ok = true;
+      // images of run-local channel tiles up to jt, each into slot jt & 1 once
+      // the products of channel tile jt - 2 that read the slot have completed
+      auto images_upto = [&](int jt) -> bool {
+        for (; img_next <= jt && img_next < nt; ++img_next) {
+          const int s = img_next & 1;
+          if (!mbar_wait(bar(PFREE + s), ((uint32_t)(img_next >> 1) & 1u) ^ 1u, abort_flag, 60)) return false;
+          const uint32_t d = smem_u32(sSlot + s * C::SLOT);
+          const int t = t_first + img_next;
+          mbar_expect_tx(bar(PREADY + s), C::SLOT);
+          tma_load_2d(d, &tmPth, bar(PREADY + s), 0, t * 64);
+          tma_load_2d(d + C::IMG_BYTES, &tmPtl, bar(PREADY + s), 0, t * 64);
+          tma_load_2d(d + 2 * C::IMG_BYTES, &tmPh, bar(PREADY + s), 0, t * 64);
+          img_issued |= 1u << s;
+        }
+        return true;
+      };
+      // first ring fill: W tiles at once, the P images (written by the
+      // Sinkhorn kernel) once the previous kernel has completed
+      const int pre = nloc < C::STAGES ? nloc : C::STAGES;
+      TileIter it(first, nrt);
+      for (int k = 0; k < pre; ++k, it.next()) {
+        mbar_expect_tx(bar(FULL + k), C::W_BYTES);
+        tma_load_2d(smem_u32(sStage + k * C::W_BYTES), &tmW, bar(FULL + k), it.t * 64, it.rt * 128);
+        issued |= 1u << k;
+      }
+      pdl_wait();
+      pdl_trigger();
+      if (nloc > 0) {
+        const int jt_pre = (first + pre - 1) / nrt - t_first;
+        ok = images_upto(jt_pre > 1 ? jt_pre : (nt > 1 ? 1 : 0));
+      }
+      for (int k = pre; k < nloc && ok; ++k, it.next()) {
         const int st = k % C::STAGES;
         const uint32_t use = (uint32_t)(k / C::STAGES) & 1u;
         if (!mbar_wait(bar(EMPTY + st), use ^ 1u, abort_flag, 61)) break;
-        int t, rt;
-        tile_of(k, t, rt);
-        uint8_t* sg = sStage + st * C::STAGE;
-        mbar_expect_tx(bar(FULL + st), C::STAGE);
-        tma_load_2d(smem_u32(sg), &tmW, bar(FULL + st), t * 64, rt * 128);
-        tma_load_2d(smem_u32(sg + C::W_BYTES), &tmPth, bar(FULL + st), 0, t * 64);
-        tma_load_2d(smem_u32(sg + C::W_BYTES + C::IMG_BYTES), &tmPtl, bar(FULL + st), 0, t * 64);
-        tma_load_2d(smem_u32(sg + C::W_BYTES + 2 * C::IMG_BYTES), &tmPh, bar(FULL + st), 0, t * 64);
+        if (!images_upto(it.t - t_first)) break;
+        mbar_expect_tx(bar(FULL + st), C::W_BYTES);
+        tma_load_2d(smem_u32(sStage + st * C::W_BYTES), &tmW, bar(FULL + st), it.t * 64, it.rt * 128);
         issued |= 1u << st;
         par = (par & ~(1u << st)) | (use << st);
       }
+      // drain: every copy this thread started has landed before the CTA exits
       for (int st = 0; st < C::STAGES; ++st)
         if (issued & (1u << st)) mbar_wait_drain(bar(FULL + st), (par >> st) & 1u, 62);
+      for (int s = 0; s < 2; ++s)
+        if (img_issued & (1u << s)) {
+          const int lastj = (img_next - 1) - ((img_next - 1 - s) & 1);   // last run-local tile loaded into slot s
+          mbar_wait_drain(bar(PREADY + s), (uint32_t)(lastj >> 1) & 1u, 59);
+        }
     }
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16(128, 64, false, false);
-      // W' = W (P_hi + P_lo) of local tile k into the W' half of TMEM buffer k & 1
+      TileIter i1(first, nrt), i2(first, nrt);   // tiles of the W' and the At products
+      // W' = W (P_hi + P_lo) of local tile k into the W' half of TMEM buffer
+      // k % NB; the ring stage is free once these products complete
       auto mma1 = [&](int k) -> bool {
-        const int st = k % C::STAGES, a = k & 1;
-        const uint32_t use = (uint32_t)(k / C::STAGES) & 1u, ua = (uint32_t)(k >> 1) & 1u;
+        const int st = k % C::STAGES, b = k % NB, jt = i1.t - t_first;
+        const uint32_t use = (uint32_t)(k / C::STAGES) & 1u, ub = (uint32_t)(k / NB) & 1u;
+        if ((k == 0 || i1.rt == 0) &&
+            !mbar_wait(bar(PREADY + (jt & 1)), (uint32_t)(jt >> 1) & 1u, abort_flag, 58))
+          return false;                                                        // images of this channel tile
         if (!mbar_wait(bar(FULL + st), use, abort_flag, 63)) return false;
-        if (!mbar_wait(bar(TMW + a), ua ^ 1u, abort_flag, 64)) return false;   // W' of tile k - 2 read
+        if (!mbar_wait(bar(TMW + b), ub ^ 1u, abort_flag, 64)) return false;   // W' of tile k - NB read
         tc_fence_after();
-        const uint32_t sg = smem_u32(sStage + st * C::STAGE);
-        const uint32_t dW = tmem + a * 128;
+        const uint32_t sw = smem_u32(sStage + st * C::W_BYTES);
+        const uint32_t sp = smem_u32(sSlot + (jt & 1) * C::SLOT);
+        const uint32_t dW = tmem + b * 128;
 #pragma unroll
         for (int k16 = 0; k16 < 4; ++k16) {
-          const uint64_t ad = sdesc(sg + k16 * 32, 16, 1024);
-          mma_bf16(dW, ad, sdesc(sg + C::W_BYTES + k16 * 32, 16, 1024), idesc, k16 != 0);
-          mma_bf16(dW, ad, sdesc(sg + C::W_BYTES + C::IMG_BYTES + k16 * 32, 16, 1024), idesc, true);
+          const uint64_t ad = sdesc(sw + k16 * 32, 16, 1024);
+          mma_bf16(dW, ad, sdesc(sp + k16 * 32, 16, 1024), idesc, k16 != 0);
+          mma_bf16(dW, ad, sdesc(sp + C::IMG_BYTES + k16 * 32, 16, 1024), idesc, true);
         }
-        mma_commit(bar(WF + a));
+        mma_commit(bar(WF + b));
+        mma_commit(bar(EMPTY + st));
+        i1.next();
         return true;
       };
-      // the next tile's first product is issued before waiting for this tile's
-      // epilogue, so the tensor core and the epilogue warps overlap
-      bool ok = nloc == 0 || mma1(0);
-      for (int k = 0; k < nloc && ok; ++k) {
-        const int st = k % C::STAGES, a = k & 1;
-        const uint32_t ua = (uint32_t)(k >> 1) & 1u;
-        if (k + 1 < nloc && !mma1(k + 1)) break;
-        if (!mbar_wait(bar(AF + a), ua, abort_flag, 65)) break;        // A of tile k in shared memory
-        if (!mbar_wait(bar(TMA + a), ua ^ 1u, abort_flag, 69)) break;  // At of tile k - 2 read
+      // W' runs two tiles ahead of At, so the mask warps find W' ready
+      bool ok = true;
+      for (int k = 0; k < 2 && k < nloc && ok; ++k) ok = mma1(k);
+      for (int k = 0; k < nloc && ok; ++k, i2.next()) {
+        const int b = k % NB, jt = i2.t - t_first;
+        const uint32_t ub = (uint32_t)(k / NB) & 1u;
+        if (k + 2 < nloc && !mma1(k + 2)) break;
+        if (!mbar_wait(bar(AF + k % NA), (uint32_t)(k / NA) & 1u, abort_flag, 65)) break;   // A of tile k
+        if (!mbar_wait(bar(TMA + b), ub ^ 1u, abort_flag, 69)) break;   // At of tile k - NB read
         tc_fence_after();
-        const uint32_t sg = smem_u32(sStage + st * C::STAGE);
-        const uint32_t sa = smem_u32(sA + a * C::A_BYTES);
-        const uint32_t dAt = tmem + a * 128 + 64;
+        const uint32_t sa = smem_u32(sA + (k % NA) * C::A_BYTES);
+        const uint32_t sph = smem_u32(sSlot + (jt & 1) * C::SLOT + 2 * C::IMG_BYTES);
+        const uint32_t dAt = tmem + b * 128 + 64;
 #pragma unroll
         for (int k16 = 0; k16 < 4; ++k16)
-          mma_bf16(dAt, sdesc(sa + k16 * 32, 16, 1024), sdesc(sg + C::W_BYTES + 2 * C::IMG_BYTES + k16 * 32, 16, 1024),
-                   idesc, k16 != 0);
-        mma_commit(bar(ATF + a));
-        mma_commit(bar(EMPTY + st));
+          mma_bf16(dAt, sdesc(sa + k16 * 32, 16, 1024), sdesc(sph + k16 * 32, 16, 1024), idesc, k16 != 0);
+        mma_commit(bar(ATF + b));
+        if (k + 1 == nloc || i2.rt == nrt - 1) mma_commit(bar(PFREE + (jt & 1)));   // slot reusable
       }
       mma_commit(bar(DRAIN));
       mbar_wait_drain(bar(DRAIN), 0, 66);
     }
     __syncwarp();
-  } else {
-    // Software-pipelined epilogue: in step k the warps first turn W' of tile k
-    // into the mask and A (so the MMA warp can start At of tile k), then copy
-    // out At of tile k - 1, whose product ran meanwhile.
-    const int e = warp - 2, q = warp & 3, h = e >> 2;   // h: column slice of NV columns
+  } else if (warp < C::COPY0) {
+    // mask warps: A buffer k % NA was last read by At of tile k - NA, whose
+    // completion the MMA warp saw before it could issue W' of tile k
+    // (k >= NA: the W' product of tile k follows At of tile k - 2 in issue
+    // order, and WF of tile k arrives only after every earlier product)
+    const int e = warp - C::MASK0, q = warp & 3, h = e >> 2;   // h: 32-column half of the tile
     const int row = q * 32 + lane;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-    const bool leader = (e == 0 && lane == 0);
-    for (int k = 0; k <= nloc; ++k) {
-      if (k < nloc) {
-        const int a = k & 1;
-        const uint32_t ua = (uint32_t)(k >> 1) & 1u;
-        int t, rt;
-        tile_of(k, t, rt);
-        const int grow = rt * 128 + row;
-        if (!named_and(1, C::EPI, mbar_wait(bar(WF + a), ua, abort_flag, 67))) break;
-        tc_fence_after();
-        uint32_t v[NV];
-        tmem_ld_cols<NV>(tmem + lane_off + a * 128 + h * NV, v);
-        tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(TMW + a));
-        const uint32_t w = nm_bits<MGROUP, NV>(v, n);
-        if (grow < cout) {
-          if constexpr (NV == 32) {
-            mask[(size_t)grow * words + 2 * t + h] = w;
-          } else {
-            reinterpret_cast<uint16_t*>(mask)[((size_t)grow * words + 2 * t) * 2 + h] = (uint16_t)w;
-          }
-          if (Wp_out) {
-            float4* o = reinterpret_cast<float4*>(Wp_out + (size_t)grow * cin + t * 64 + h * NV);
+    TileIter it(first, nrt);
+    for (int k = 0; k < nloc; ++k, it.next()) {
+      const int b = k % NB;
+      if (!wait_all(WF + b, (uint32_t)(k / NB) & 1u, 67)) break;
+      tc_fence_after();
+      uint32_t v[32];
+      tmem_ld32(tmem + lane_off + b * 128 + h * 32, v);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(TMW + b));
+      const int grow = it.rt * 128 + row;
+      if (Wp_out && grow < cout) {
+        float4* o = reinterpret_cast<float4*>(Wp_out + (size_t)grow * cin + it.t * 64 + h * 32);
 #pragma unroll
-            for (int qq = 0; qq < NV / 4; ++qq)
-              o[qq] = make_float4(__uint_as_float(v[4 * qq]), __uint_as_float(v[4 * qq + 1]),
-                                  __uint_as_float(v[4 * qq + 2]), __uint_as_float(v[4 * qq + 3]));
-          }
-        }
-        uint8_t* sa = sA + a * C::A_BYTES;
-#pragma unroll
-        for (int c8 = 0; c8 < NV / 8; ++c8) {
-          float f[8];
-#pragma unroll
-          for (int x = 0; x < 8; ++x) f[x] = ((w >> (8 * c8 + x)) & 1u) ? __uint_as_float(v[8 * c8 + x]) : 0.f;
-          st_sw128(sa, row, h * (NV / 8) + c8, make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
-                                                          pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7])));
-        }
-        fence_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(AF + a));
+        for (int qq = 0; qq < 8; ++qq)
+          o[qq] = make_float4(__uint_as_float(v[4 * qq]), __uint_as_float(v[4 * qq + 1]),
+                              __uint_as_float(v[4 * qq + 2]), __uint_as_float(v[4 * qq + 3]));
       }
-      if (k > 0) {
-        const int kp = k - 1, a = kp & 1;
-        const uint32_t ua = (uint32_t)(kp >> 1) & 1u;
-        int t, rt;
-        tile_of(kp, t, rt);
-        const bool got = mbar_wait(bar(ATF + a), ua, abort_flag, 68);
-        // the staging tile of two tiles ago must have been read out by its TMA store
-        if (leader) bulk_wait_read<1>();
-        if (!named_and(1, C::EPI, got)) break;
-        tc_fence_after();
-        uint32_t v[NV];
-        tmem_ld_cols<NV>(tmem + lane_off + a * 128 + 64 + h * NV, v);
-        tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(TMA + a));
-        uint8_t* so = sO + a * C::A_BYTES;
+      // keep bits; v becomes A = M.W'
+      const uint32_t w = MGROUP == 4 ? nm4_keep<32>(v, n) : nm_bits<MGROUP, 32>(v, n);
 #pragma unroll
-        for (int c8 = 0; c8 < NV / 8; ++c8)
-          st_sw128(so, row, h * (NV / 8) + c8,
-                   make_uint4(pack_bf16x2(__uint_as_float(v[8 * c8 + 0]), __uint_as_float(v[8 * c8 + 1])),
-                              pack_bf16x2(__uint_as_float(v[8 * c8 + 2]), __uint_as_float(v[8 * c8 + 3])),
-                              pack_bf16x2(__uint_as_float(v[8 * c8 + 4]), __uint_as_float(v[8 * c8 + 5])),
-                              pack_bf16x2(__uint_as_float(v[8 * c8 + 6]), __uint_as_float(v[8 * c8 + 7]))));
-        fence_async_smem();
-        named_sync(1, C::EPI);
-        if (leader) {
-          tma_store_2d(&tmAt, smem_u32(so), t * 64, rt * 128);
+      for (int x = 0; x < 32; ++x) v[x] = ((w >> x) & 1u) ? v[x] : 0u;
+      if (grow < cout) mask[(size_t)grow * words + 2 * it.t + h] = w;
+      uint8_t* sa = sA + (k % NA) * C::A_BYTES;
+#pragma unroll
+      for (int c8 = 0; c8 < 4; ++c8)
+        st_sw128(sa, row, h * 4 + c8,
+                 make_uint4(pack_bf16x2(__uint_as_float(v[8 * c8 + 0]), __uint_as_float(v[8 * c8 + 1])),
+                            pack_bf16x2(__uint_as_float(v[8 * c8 + 2]), __uint_as_float(v[8 * c8 + 3])),
+                            pack_bf16x2(__uint_as_float(v[8 * c8 + 4]), __uint_as_float(v[8 * c8 + 5])),
+                            pack_bf16x2(__uint_as_float(v[8 * c8 + 6]), __uint_as_float(v[8 * c8 + 7]))));
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(AF + k % NA));
+    }
+  } else {
+    // copy-out warps: At of tile j -> staging tile j & 1 (refilled once the
+    // store of tile j - 2 has read it: SFREE) -> TMA store by the first copy
+    // warp once all four have written their rows (SFULL)
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    const bool storer = warp == C::COPY0;
+    TileIter it(first, nrt);
+    for (int j = 0; j < nloc; ++j, it.next()) {
+      const int b = j % NB, s = j & 1;
+      const uint32_t us = (uint32_t)(j >> 1) & 1u;
+      if (!wait_all(ATF + b, (uint32_t)(j / NB) & 1u, 68)) break;
+      tc_fence_after();
+      uint32_t u0[32], u1[32];
+      tmem_ld32(tmem + lane_off + b * 128 + 64, u0);
+      tmem_ld32(tmem + lane_off + b * 128 + 96, u1);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(TMA + b));
+      if (!wait_all(SFREE + s, us ^ 1u, 70)) break;
+      uint8_t* so = sO + s * C::A_BYTES;
+#pragma unroll
+      for (int c8 = 0; c8 < 4; ++c8)
+        st_sw128(so, row, c8,
+                 make_uint4(pack_bf16x2(__uint_as_float(u0[8 * c8 + 0]), __uint_as_float(u0[8 * c8 + 1])),
+                            pack_bf16x2(__uint_as_float(u0[8 * c8 + 2]), __uint_as_float(u0[8 * c8 + 3])),
+                            pack_bf16x2(__uint_as_float(u0[8 * c8 + 4]), __uint_as_float(u0[8 * c8 + 5])),
+                            pack_bf16x2(__uint_as_float(u0[8 * c8 + 6]), __uint_as_float(u0[8 * c8 + 7]))));
+#pragma unroll
+      for (int c8 = 0; c8 < 4; ++c8)
+        st_sw128(so, row, 4 + c8,
+                 make_uint4(pack_bf16x2(__uint_as_float(u1[8 * c8 + 0]), __uint_as_float(u1[8 * c8 + 1])),
+                            pack_bf16x2(__uint_as_float(u1[8 * c8 + 2]), __uint_as_float(u1[8 * c8 + 3])),
+                            pack_bf16x2(__uint_as_float(u1[8 * c8 + 4]), __uint_as_float(u1[8 * c8 + 5])),
+                            pack_bf16x2(__uint_as_float(u1[8 * c8 + 6]), __uint_as_float(u1[8 * c8 + 7]))));
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(SFULL + s));
+      if (storer) {
+        if (!wait_all(SFULL + s, us, 71)) break;
+        if (lane == 0) {
+          tma_store_2d(&tmAt, smem_u32(so), it.t * 64, it.rt * 128);
           bulk_commit();
+          // the store of tile j - 1 has read staging tile s ^ 1: it may be refilled
+          if (j >= 1) {
+            bulk_wait_read<1>();
+            mbar_arrive(bar(SFREE + (s ^ 1)));
+          }
         }
+        __syncwarp();
       }
     }
-    if (leader) bulk_wait_all();
+    if (storer && lane == 0) bulk_wait_all();
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 128 * NB);
   }
 }
 
@@ -469,6 +568,8 @@ permute_mask_tc2_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_co
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *holder;
+  pdl_wait();
+  pdl_trigger();
   const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
   const int row = warp * 32 + lane;
   const int words = cin / 32;
@@ -532,7 +633,8 @@ permute_mask_tc2_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_co
       tmem_ld32(tmem + lane_off + 0, v0);
       tmem_ld32(tmem + lane_off + 32, v1);
       tmem_ld_wait();
-      const uint32_t w0 = nm_word<MGROUP>(v0, n), w1 = nm_word<MGROUP>(v1, n);
+      const uint32_t w0 = MGROUP == 4 ? nm4_keep<32>(v0, n) : nm_word<MGROUP>(v0, n);
+    const uint32_t w1 = MGROUP == 4 ? nm4_keep<32>(v1, n) : nm_word<MGROUP>(v1, n);
       if (grow < cout) {
         const int wi = (col0 + c * 64) / 32;
         *reinterpret_cast<uint2*>(mask + (size_t)grow * words + wi) = make_uint2(w0, w1);
@@ -629,8 +731,8 @@ lcp_status permute_mask2_bc(const CUtensorMap& mW, const CUtensorMap& mPth, cons
   int ry = cdiv(C::CTAS_PER_SM * num_sms(), ntiles);
   if (ry > nrt) ry = nrt;
   if (ry < 1) ry = 1;
-  k<<<dim3(ntiles, ry), 128, C::SMEM, st>>>(mW, mPth, mPtl, mPh, mask, At, Wp, cout, cin, n);
-  return check_launch("permute_mask_tc");
+  return launch_kernel(k, dim3(ntiles, ry), dim3(128), C::SMEM, st, 1, true, "permute_mask_tc", mW, mPth, mPtl, mPh,
+                       mask, At, Wp, cout, cin, n);
 }
 
 template <int BC, int MG>
@@ -640,8 +742,8 @@ lcp_status permute_mask_bc(const CUtensorMap& mW, const CUtensorMap& mPth, const
   auto k = permute_mask_tc_kernel<BC, MG>;
   TC_TRY(set_smem(k, PmCfg<BC>::SMEM, "permute_mask_tc"));
   const dim3 grid(cdiv(cout, 128), cin / BC);
-  k<<<grid, 128, PmCfg<BC>::SMEM, st>>>(mW, mPth, mPtl, mPh, mask, At, Wp, cout, cin, n);
-  return check_launch("permute_mask_tc");
+  return launch_kernel(k, grid, dim3(128), PmCfg<BC>::SMEM, st, 1, true, "permute_mask_tc", mW, mPth, mPtl, mPh, mask,
+                       At, Wp, cout, cin, n);
 }
 
 }  // namespace
@@ -661,14 +763,13 @@ lcp_status launch_permute_mask_tc(const __nv_bfloat16* W, const __nv_bfloat16* i
   if (BC == 64) {
     CUtensorMap mAt;
     TC_TRY(make_map(&mAt, At, cin, cout, 64, 128, "permute_mask At"));
-    constexpr int NSL = 2;
-    using C = PwCfg<NSL>;
-    auto k = (m == 4) ? permute_mask_ws_kernel<4, NSL> : permute_mask_ws_kernel<8, NSL>;
+    using C = PwCfg;
+    auto k = (m == 4) ? permute_mask_ws_kernel<4> : permute_mask_ws_kernel<8>;
     TC_TRY(set_smem(k, C::SMEM, "permute_mask_tc"));
     const int tiles = cdiv(cout, 128) * (cin / 64);
     const int grid = tiles < num_sms() ? tiles : num_sms();
-    k<<<grid, C::THREADS, C::SMEM, st>>>(mW, mPth, mPtl, mPh, mAt, mask, Wp_out, cout, cin, n);
-    return check_launch("permute_mask_tc");
+    return launch_kernel(k, dim3(grid), dim3(C::THREADS), C::SMEM, st, 1, true, "permute_mask_tc", mW, mPth, mPtl,
+                         mPh, mAt, mask, Wp_out, cout, cin, n);
   }
   if (m == 4) {
     if (BC == 128) return permute_mask2_bc<128, 4>(mW, mPth, mPtl, mPh, mask, At, Wp_out, cout, cin, n, st);

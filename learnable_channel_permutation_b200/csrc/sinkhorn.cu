@@ -101,8 +101,11 @@ template <int B>
 __global__ void __launch_bounds__(SkCfg<B>::NT, 1)
 sinkhorn_fwd_kernel(const float* __restrict__ L, float* __restrict__ P, float* __restrict__ ckpt,
                     __nv_bfloat16* __restrict__ pt_hi, __nv_bfloat16* __restrict__ pt_lo,
-                    __nv_bfloat16* __restrict__ p_hi, float tau, int iters) {
+                    __nv_bfloat16* __restrict__ p_hi, unsigned* __restrict__ zero_word, float tau, int iters) {
   using C = SkCfg<B>;
+  pdl_wait();
+  pdl_trigger();
+  if (zero_word && blockIdx.x == 0 && threadIdx.x == 0) *zero_word = 0u;
   constexpr int R = C::R, NT = C::NT, CS = C::CS, TPR = C::TPR, EPR = C::EPR, TPC = C::TPC,
                 EPC = C::EPC, LD = C::LD;
   extern __shared__ __align__(16) float sm[];
@@ -235,6 +238,8 @@ sinkhorn_bwd_kernel(const float* __restrict__ L, const float* __restrict__ ckpt,
                     const float* __restrict__ dP, int splits, int nblocks,
                     float* __restrict__ dL, float tau, int iters) {
   using C = SkCfg<B>;
+  pdl_wait();
+  pdl_trigger();
   constexpr int R = C::R, NT = C::NT, CS = C::CS, TPR = C::TPR, EPR = C::EPR, NW = C::NW, LD = C::LD;
   constexpr int RPW = 32 / TPR;   // rows per warp
   extern __shared__ __align__(16) float sm[];
@@ -349,56 +354,37 @@ template <int B> constexpr size_t bwd_smem() {
   return sizeof(float) * (C::R * C::LD + 2 * B + C::NW * B + B + 2 * B);
 }
 
-template <typename K, typename... Args>
-lcp_status launch_cluster(K kernel, int grid, int threads, size_t smem, int cs, cudaStream_t st,
-                          const char* what, Args... args) {
-  const lcp_status s0 = ensure_smem_limit(reinterpret_cast<const void*>(kernel), (int)smem, what);
-  if (s0 != LCP_OK) return s0;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(threads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = cs;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = cs > 1 ? 1 : 0;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
-  if (e != cudaSuccess) {
-    cudaGetLastError();
-    return fail(LCP_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
-  }
-  return check_launch(what);
-}
-
 template <int B>
 lcp_status fwd_b(const float* L, float* P, float* ckpt, __nv_bfloat16* a, __nv_bfloat16* b,
-                 __nv_bfloat16* c, int nblocks, float tau, int iters, cudaStream_t st) {
+                 __nv_bfloat16* c, unsigned* zero_word, int nblocks, float tau, int iters, cudaStream_t st) {
   using C = SkCfg<B>;
-  return launch_cluster(sinkhorn_fwd_kernel<B>, nblocks * C::CS, C::NT, fwd_smem<B>(), C::CS, st,
-                        "sinkhorn_fwd", L, P, ckpt, a, b, c, tau, iters);
+  const lcp_status s0 = ensure_smem_limit(reinterpret_cast<const void*>(sinkhorn_fwd_kernel<B>), (int)fwd_smem<B>(),
+                                          "sinkhorn_fwd");
+  if (s0 != LCP_OK) return s0;
+  return launch_kernel(sinkhorn_fwd_kernel<B>, dim3(nblocks * C::CS), dim3(C::NT), fwd_smem<B>(), st, C::CS, true,
+                       "sinkhorn_fwd", L, P, ckpt, a, b, c, zero_word, tau, iters);
 }
 template <int B>
 lcp_status bwd_b(const float* L, const float* ckpt, const float* dP, int splits, float* dL,
                  int nblocks, float tau, int iters, cudaStream_t st) {
   using C = SkCfg<B>;
-  return launch_cluster(sinkhorn_bwd_kernel<B>, nblocks * C::CS, C::NT, bwd_smem<B>(), C::CS, st,
-                        "sinkhorn_bwd", L, ckpt, dP, splits, nblocks, dL, tau, iters);
+  const lcp_status s0 = ensure_smem_limit(reinterpret_cast<const void*>(sinkhorn_bwd_kernel<B>), (int)bwd_smem<B>(),
+                                          "sinkhorn_bwd");
+  if (s0 != LCP_OK) return s0;
+  return launch_kernel(sinkhorn_bwd_kernel<B>, dim3(nblocks * C::CS), dim3(C::NT), bwd_smem<B>(), st, C::CS, true,
+                       "sinkhorn_bwd", L, ckpt, dP, splits, nblocks, dL, tau, iters);
 }
 
 }  // namespace
 
 lcp_status launch_sinkhorn_fwd(const float* L, float* P, float* ckpt, __nv_bfloat16* img_pt_hi,
-                               __nv_bfloat16* img_pt_lo, __nv_bfloat16* img_p_hi, int nblocks,
-                               int B, float tau, int iters, cudaStream_t st) {
+                               __nv_bfloat16* img_pt_lo, __nv_bfloat16* img_p_hi, unsigned* zero_word,
+                               int nblocks, int B, float tau, int iters, cudaStream_t st) {
   switch (B) {
-    case 32: return fwd_b<32>(L, P, ckpt, img_pt_hi, img_pt_lo, img_p_hi, nblocks, tau, iters, st);
-    case 64: return fwd_b<64>(L, P, ckpt, img_pt_hi, img_pt_lo, img_p_hi, nblocks, tau, iters, st);
-    case 128: return fwd_b<128>(L, P, ckpt, img_pt_hi, img_pt_lo, img_p_hi, nblocks, tau, iters, st);
-    case 256: return fwd_b<256>(L, P, ckpt, img_pt_hi, img_pt_lo, img_p_hi, nblocks, tau, iters, st);
+    case 32: return fwd_b<32>(L, P, ckpt, img_pt_hi, img_pt_lo, img_p_hi, zero_word, nblocks, tau, iters, st);
+    case 64: return fwd_b<64>(L, P, ckpt, img_pt_hi, img_pt_lo, img_p_hi, zero_word, nblocks, tau, iters, st);
+    case 128: return fwd_b<128>(L, P, ckpt, img_pt_hi, img_pt_lo, img_p_hi, zero_word, nblocks, tau, iters, st);
+    case 256: return fwd_b<256>(L, P, ckpt, img_pt_hi, img_pt_lo, img_p_hi, zero_word, nblocks, tau, iters, st);
   }
   return fail(LCP_ERR_SHAPE, "sinkhorn_fwd: unsupported block size %d", B);
 }

@@ -318,6 +318,7 @@ __device__ __forceinline__ uint32_t nm_word(const uint32_t (&v)[32], int n) {
   return nm_bits<M, 32>(v, n);
 }
 
+
 // ------------------------------------------------------------------ host --
 
 using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
