@@ -75,32 +75,44 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 
 // ---- N:4 keep bits --------------------------------------------------------
 // Bit j of the result keeps element j of NV consecutive values (NV / 4 groups
-// of M = 4 consecutive columns), bit-sliced.  For each
-// element three words record whether it beats each of the other three members
-// of its group (j beats k when |v_j| > |v_k|, or the two are equal and j < k);
-// on the 31-bit magnitudes u the test is the sign of a difference:
-// u_j >= u_k exactly when u_k - u_j - 1 < 0, and u_j > u_k when u_k - u_j < 0.
-// An element is kept when it beats at least 4 - n of the others: all three
-// (n = 1, bitwise AND), two of three (n = 2, bitwise majority) or one (n = 3,
-// OR); n = 4 keeps every element.
-__device__ __forceinline__ uint32_t sign_to(uint32_t d, int pos) { return (d >> 31) << pos; }
+// of M = 4 consecutive columns): the same bits as the pairwise count
+// (nm_bits), computed bit-sliced.  For a pair a < b of a group, bit 4g of
+// T_ab says that element b beats element a (|v_b| > |v_a|; equal magnitudes
+// go to the lower index); it is the sign of the single-precision difference
+// |v_a| - |v_b|, which is exact in sign (equal magnitudes give +0, distinct
+// ones a nonzero difference; no flush to zero in this build).  Element j is
+// kept when it beats at least 4 - n of the other three: all of them (n = 1,
+// bitwise AND), two (n = 2, bitwise majority) or one (n = 3, OR); n = 4 keeps
+// everything.  Six subtractions and bit moves per group, a few word-wide
+// logic operations per 32 values.
+__device__ __forceinline__ uint32_t sign_at(float d, int pos) {
+  return (__float_as_uint(d) >> 31) << pos;
+}
 template <int NV>
 __device__ __forceinline__ uint32_t nm4_keep(const uint32_t (&v)[NV], int n) {
-  uint32_t X = 0, Y = 0, Z = 0;   // element j's 1st, 2nd and 3rd opponent, in index order
+  uint32_t T01 = 0, T02 = 0, T03 = 0, T12 = 0, T13 = 0, T23 = 0;
 #pragma unroll
   for (int g = 0; g < NV / 4; ++g) {
-    const uint32_t u0 = v[4 * g] & 0x7fffffffu, u1 = v[4 * g + 1] & 0x7fffffffu;
-    const uint32_t u2 = v[4 * g + 2] & 0x7fffffffu, u3 = v[4 * g + 3] & 0x7fffffffu;
-    const int b = 4 * g;
-    X |= sign_to(u1 - u0 - 1, b) | sign_to(u0 - u1, b + 1) | sign_to(u0 - u2, b + 2) | sign_to(u0 - u3, b + 3);
-    Y |= sign_to(u2 - u0 - 1, b) | sign_to(u2 - u1 - 1, b + 1) | sign_to(u1 - u2, b + 2) | sign_to(u1 - u3, b + 3);
-    Z |= sign_to(u3 - u0 - 1, b) | sign_to(u3 - u1 - 1, b + 1) | sign_to(u3 - u2 - 1, b + 2) |
-         sign_to(u2 - u3, b + 3);
+    const float a0 = fabsf(__uint_as_float(v[4 * g])), a1 = fabsf(__uint_as_float(v[4 * g + 1]));
+    const float a2 = fabsf(__uint_as_float(v[4 * g + 2])), a3 = fabsf(__uint_as_float(v[4 * g + 3]));
+    const int p = 4 * g;
+    T01 |= sign_at(a0 - a1, p);
+    T02 |= sign_at(a0 - a2, p);
+    T03 |= sign_at(a0 - a3, p);
+    T12 |= sign_at(a1 - a2, p);
+    T13 |= sign_at(a1 - a3, p);
+    T23 |= sign_at(a2 - a3, p);
   }
-  const uint32_t all3 = X & Y & Z, two = (X & Y) | (X & Z) | (Y & Z), one = X | Y | Z;
-  if (n >= 4) return 0xffffffffu;   // nothing pruned
+  if (n >= 4) return NV == 32 ? 0xffffffffu : (1u << NV) - 1u;   // nothing pruned
   if (n <= 0) return 0u;
-  return n == 1 ? all3 : (n == 2 ? two : one);
+  constexpr uint32_t lo = NV == 32 ? 0x11111111u : 0x1111u;   // bit 0 of every group
+  // what element j beats: 0 -> ~T01 ~T02 ~T03, 1 -> T01 ~T12 ~T13, 2 -> T02 T12 ~T23, 3 -> T03 T13 T23
+  auto f = [n](uint32_t x, uint32_t y, uint32_t z) {
+    return n == 1 ? (x & y & z) : (n == 2 ? ((x & y) | (x & z) | (y & z)) : (x | y | z));
+  };
+  const uint32_t k0 = f(~T01, ~T02, ~T03) & lo, k1 = f(T01, ~T12, ~T13) & lo;
+  const uint32_t k2 = f(T02, T12, ~T23) & lo, k3 = f(T03, T13, T23) & lo;
+  return k0 | (k1 << 1) | (k2 << 2) | (k3 << 3);
 }
 
 // ---- launchers (host side; each returns LCP_OK or LCP_ERR_CUDA) ----------

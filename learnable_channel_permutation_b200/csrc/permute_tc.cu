@@ -199,9 +199,10 @@ permute_mask_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
 //   warp 1: MMA issuer: W' = W (P_hi + P_lo) of tile k + 2 into TMEM buffer
 //           (k + 2) % NB, then, once A = M.W' of tile k is in shared memory,
 //           At = A P_hi of tile k into buffer k % NB
-//   warps 2-9: mask warps (two per TMEM lane quadrant, 32 columns each): W'
-//           of tile k -> the N:M keep bits (stored to the mask) and A
-//   warps 10-13: copy-out warps (one per quadrant, 64 columns each): At of
+//   warps 2..: MASK_WARPS mask warps (MASK_WARPS / 4 per TMEM lane quadrant,
+//           MCOLS columns each): W' of tile k -> the N:M keep bits (stored to
+//           the mask) and A
+//   last 4 warps: copy-out warps (one per quadrant, 64 columns each): At of
 //           tile k -> swizzled staging tile -> TMA store
 // The two epilogue roles run side by side (the mask is ALU work, the copy-out
 // memory traffic) and meet only through mbarriers; the mask warps never wait
@@ -217,6 +218,7 @@ struct PwCfg {
   static constexpr int NBAR = 2 * STAGES + 4 * NB + NA + 4 * 2 + 1;
   static constexpr int SMEM = STAGES * W_BYTES + 2 * SLOT + (NA + 2) * A_BYTES + NBAR * 8 + 16 + 1024;
   static constexpr int MASK_WARPS = 8, COPY_WARPS = 4;
+  static constexpr int MCOLS = 64 / (MASK_WARPS / 4);   // columns per mask thread
   static constexpr int MASK0 = 2, COPY0 = MASK0 + MASK_WARPS;   // first warp of each role
   static constexpr int THREADS = 32 * (COPY0 + COPY_WARPS);
   static_assert(SMEM <= 232448, "shared memory budget");
@@ -410,7 +412,8 @@ permute_mask_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
     // completion the MMA warp saw before it could issue W' of tile k
     // (k >= NA: the W' product of tile k follows At of tile k - 2 in issue
     // order, and WF of tile k arrives only after every earlier product)
-    const int e = warp - C::MASK0, q = warp & 3, h = e >> 2;   // h: 32-column half of the tile
+    constexpr int NV = C::MCOLS;
+    const int e = warp - C::MASK0, q = warp & 3, h = e >> 2;   // h: NV-column slice of the tile
     const int row = q * 32 + lane;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     TileIter it(first, nrt);
@@ -418,29 +421,35 @@ permute_mask_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
       const int b = k % NB;
       if (!wait_all(WF + b, (uint32_t)(k / NB) & 1u, 67)) break;
       tc_fence_after();
-      uint32_t v[32];
-      tmem_ld32(tmem + lane_off + b * 128 + h * 32, v);
+      uint32_t v[NV];
+      tmem_ld_cols<NV>(tmem + lane_off + b * 128 + h * NV, v);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(TMW + b));
       const int grow = it.rt * 128 + row;
       if (Wp_out && grow < cout) {
-        float4* o = reinterpret_cast<float4*>(Wp_out + (size_t)grow * cin + it.t * 64 + h * 32);
+        float4* o = reinterpret_cast<float4*>(Wp_out + (size_t)grow * cin + it.t * 64 + h * NV);
 #pragma unroll
-        for (int qq = 0; qq < 8; ++qq)
+        for (int qq = 0; qq < NV / 4; ++qq)
           o[qq] = make_float4(__uint_as_float(v[4 * qq]), __uint_as_float(v[4 * qq + 1]),
                               __uint_as_float(v[4 * qq + 2]), __uint_as_float(v[4 * qq + 3]));
       }
       // keep bits; v becomes A = M.W'
-      const uint32_t w = MGROUP == 4 ? nm4_keep<32>(v, n) : nm_bits<MGROUP, 32>(v, n);
+      const uint32_t w = MGROUP == 4 ? nm4_keep<NV>(v, n) : nm_bits<MGROUP, NV>(v, n);
 #pragma unroll
-      for (int x = 0; x < 32; ++x) v[x] = ((w >> x) & 1u) ? v[x] : 0u;
-      if (grow < cout) mask[(size_t)grow * words + 2 * it.t + h] = w;
+      for (int x = 0; x < NV; ++x) v[x] = ((w >> x) & 1u) ? v[x] : 0u;
+      if (grow < cout) {
+        if constexpr (NV == 32) {
+          mask[(size_t)grow * words + 2 * it.t + h] = w;
+        } else {
+          reinterpret_cast<uint16_t*>(mask)[((size_t)grow * words + 2 * it.t) * 2 + h] = (uint16_t)w;
+        }
+      }
       uint8_t* sa = sA + (k % NA) * C::A_BYTES;
 #pragma unroll
-      for (int c8 = 0; c8 < 4; ++c8)
-        st_sw128(sa, row, h * 4 + c8,
+      for (int c8 = 0; c8 < NV / 8; ++c8)
+        st_sw128(sa, row, h * (NV / 8) + c8,
                  make_uint4(pack_bf16x2(__uint_as_float(v[8 * c8 + 0]), __uint_as_float(v[8 * c8 + 1])),
                             pack_bf16x2(__uint_as_float(v[8 * c8 + 2]), __uint_as_float(v[8 * c8 + 3])),
                             pack_bf16x2(__uint_as_float(v[8 * c8 + 4]), __uint_as_float(v[8 * c8 + 5])),
@@ -463,29 +472,27 @@ permute_mask_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
       const uint32_t us = (uint32_t)(j >> 1) & 1u;
       if (!wait_all(ATF + b, (uint32_t)(j / NB) & 1u, 68)) break;
       tc_fence_after();
-      uint32_t u0[32], u1[32];
-      tmem_ld32(tmem + lane_off + b * 128 + 64, u0);
-      tmem_ld32(tmem + lane_off + b * 128 + 96, u1);
-      tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(TMA + b));
+      // the staging tile is free once the store of tile j - 2 has read it
       if (!wait_all(SFREE + s, us ^ 1u, 70)) break;
       uint8_t* so = sO + s * C::A_BYTES;
 #pragma unroll
-      for (int c8 = 0; c8 < 4; ++c8)
-        st_sw128(so, row, c8,
-                 make_uint4(pack_bf16x2(__uint_as_float(u0[8 * c8 + 0]), __uint_as_float(u0[8 * c8 + 1])),
-                            pack_bf16x2(__uint_as_float(u0[8 * c8 + 2]), __uint_as_float(u0[8 * c8 + 3])),
-                            pack_bf16x2(__uint_as_float(u0[8 * c8 + 4]), __uint_as_float(u0[8 * c8 + 5])),
-                            pack_bf16x2(__uint_as_float(u0[8 * c8 + 6]), __uint_as_float(u0[8 * c8 + 7]))));
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t u[32];
+        tmem_ld32(tmem + lane_off + b * 128 + 64 + 32 * hh, u);
+        tmem_ld_wait();
+        if (hh == 1) {   // both halves read: the TMEM buffer may take At of tile j + NB
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(TMA + b));
+        }
 #pragma unroll
-      for (int c8 = 0; c8 < 4; ++c8)
-        st_sw128(so, row, 4 + c8,
-                 make_uint4(pack_bf16x2(__uint_as_float(u1[8 * c8 + 0]), __uint_as_float(u1[8 * c8 + 1])),
-                            pack_bf16x2(__uint_as_float(u1[8 * c8 + 2]), __uint_as_float(u1[8 * c8 + 3])),
-                            pack_bf16x2(__uint_as_float(u1[8 * c8 + 4]), __uint_as_float(u1[8 * c8 + 5])),
-                            pack_bf16x2(__uint_as_float(u1[8 * c8 + 6]), __uint_as_float(u1[8 * c8 + 7]))));
+        for (int c8 = 0; c8 < 4; ++c8)
+          st_sw128(so, row, 4 * hh + c8,
+                   make_uint4(pack_bf16x2(__uint_as_float(u[8 * c8 + 0]), __uint_as_float(u[8 * c8 + 1])),
+                              pack_bf16x2(__uint_as_float(u[8 * c8 + 2]), __uint_as_float(u[8 * c8 + 3])),
+                              pack_bf16x2(__uint_as_float(u[8 * c8 + 4]), __uint_as_float(u[8 * c8 + 5])),
+                              pack_bf16x2(__uint_as_float(u[8 * c8 + 6]), __uint_as_float(u[8 * c8 + 7]))));
+      }
       fence_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(SFULL + s));
