@@ -123,12 +123,13 @@ sinkhorn_fwd_kernel(const float* __restrict__ L, float* __restrict__ P, float* _
   const int r = tid / TPR, c = tid % TPR;     // row slice: row r, columns c + TPR*e
   const int j = tid / TPC, g = tid % TPC;     // column slice: column j, rows g + TPC*e
 
-  // Z_0 = L / tau.  Division kept exact (not a reciprocal multiply) on load.
+  // Z_0 = L / tau (as L times the correctly rounded 1 / tau: within an ulp)
+  const float inv_tau = 1.0f / tau;
   for (int q = tid; q < R * (B / 4); q += NT) {
     const float4 v = reinterpret_cast<const float4*>(L + base + (size_t)row0 * B)[q];
     const int rr = q / (B / 4), jj = (q % (B / 4)) * 4;
     float* d = tile + rr * LD + jj;
-    d[0] = v.x / tau; d[1] = v.y / tau; d[2] = v.z / tau; d[3] = v.w / tau;
+    d[0] = v.x * inv_tau; d[1] = v.y * inv_tau; d[2] = v.z * inv_tau; d[3] = v.w * inv_tau;
   }
   for (int jj = tid; jj < B; jj += NT) cv[jj] = 0.f;
   __syncthreads();
@@ -260,12 +261,13 @@ sinkhorn_bwd_kernel(const float* __restrict__ L, const float* __restrict__ ckpt,
   const int r = tid / TPR, c = tid % TPR;
 
   float zr[EPR], dz[EPR];
-  // Z_0 = L / tau
+  // Z_0 = L / tau, formed as in the forward kernel
+  const float inv_tau = 1.0f / tau;
   for (int q = tid; q < R * (B / 4); q += NT) {
     const float4 v = reinterpret_cast<const float4*>(L + base + (size_t)row0 * B)[q];
     const int rr = q / (B / 4), jj = (q % (B / 4)) * 4;
     float* d = tile + rr * LD + jj;
-    d[0] = v.x / tau; d[1] = v.y / tau; d[2] = v.z / tau; d[3] = v.w / tau;
+    d[0] = v.x * inv_tau; d[1] = v.y * inv_tau; d[2] = v.z * inv_tau; d[3] = v.w * inv_tau;
   }
   __syncthreads();
 #pragma unroll
@@ -335,7 +337,7 @@ sinkhorn_bwd_kernel(const float* __restrict__ L, const float* __restrict__ ckpt,
   // dL = dZ_0 / tau, staged for coalesced stores
   __syncthreads();
 #pragma unroll
-  for (int e = 0; e < EPR; ++e) tile[r * LD + c + TPR * e] = dz[e] / tau;
+  for (int e = 0; e < EPR; ++e) tile[r * LD + c + TPR * e] = dz[e] * inv_tau;
   __syncthreads();
   for (int q = tid; q < R * B; q += NT) {
     const int rr = q / B, jj = q % B;
