@@ -213,6 +213,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--eager", action="store_true", help="time eager launches instead of CUDA-graph replays")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the secondary measurements (cached dense output, standalone mask, "
+                         "Sinkhorn scaling run, one-core oracle)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
@@ -411,12 +414,114 @@ def main():
                        "pdl": os.environ.get("LCP_PDL", "1") != "0"},
             "roofline": roof, "stages": per_stage, "clocks": clocks, "e2e": e2e, "eager": eager,
             "gpu_launches": step.launches * K}
+    if world == 1 and not args.no_extras and not args.simt:
+        line["extras"] = extras(args, b, synth, wl, li, layer, step, flush, pk, dev)
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)
+        if not args.no_extras:
+            one = cpu_baseline_one_core(wl)
+            if one:
+                line["cpu_baseline_one_core"] = one
     print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
     return 0
+
+
+def extras(args, b, synth, wl, li, layer, step, flush, pk, dev):
+    """Secondary measurements of the same build, rank 0 at N = 1 only.
+
+    - cached_dense: the step with LCP_FLAG_CACHED_DENSE (Y_d read from layer.Yd,
+      written once by an uncached step), same timing protocol as the headline;
+    - nm_mask: the standalone mask kernel on a bf16 W' of the layer's shape,
+      against the measured HBM copy bandwidth (bytes: 2 read + 1/8 written per element);
+    - sinkhorn_scaling: Sinkhorn forward then reverse over the logits of every
+      projection of a 40-layer 13B-shaped model (4 x 5120^2, 2 x 13824 x 5120,
+      5120 x 13824 per layer; 27 840 blocks of 64 x 64, 456 MB of float32 L) in one
+      launch each, against the HBM copy bandwidth.
+    """
+    import torch
+    out = {}
+    K = max(5, min(args.steps, 20))
+
+    def timed(fn, reps, flush_between=True):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0 = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
+        e1 = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
+        for k in range(reps):
+            if flush_between:
+                flush.zero_()
+            e0[k].record()
+            fn()
+            e1[k].record()
+        torch.cuda.synchronize()
+        return sum(e0[k].elapsed_time(e1[k]) for k in range(reps)) / reps
+
+    # cached dense output
+    layer["Yd"] = torch.empty(li.spec.tokens, li.spec.cout, dtype=torch.float32, device=dev)
+    fill = b.Step([layer], wl.block, wl.n, wl.m, wl.iters, wl.tau, workspace=step.ws)
+    fill.run()
+    cached = b.Step([layer], wl.block, wl.n, wl.m, wl.iters, wl.tau, flags=b.FLAG_CACHED_DENSE, workspace=step.ws)
+    g = b.capture(cached)
+    ms = timed(g.replay, K)
+    del g
+    layer.pop("Yd")
+    flop = 2 * 2 * li.spec.tokens * li.spec.cout * li.spec.cin - 2 * li.spec.tokens * li.spec.cout * li.spec.cin
+    out["cached_dense"] = {"value": 1e3 / ms, "unit": UNIT, "ms_per_step": ms, "steps": K,
+                           "note": "LCP_FLAG_CACHED_DENSE: Y_d = X W^T read from layer.Yd (computed once), "
+                                   "so the step runs one calibration GEMM problem instead of two; "
+                                   "not the headline", "algorithmic_flop": 2 * flop}
+
+    # standalone N:M mask on a bf16 W' of the layer's shape
+    Wp = torch.randn(li.spec.cout, li.spec.cin, device=dev).to(torch.bfloat16)
+    bits = torch.empty(li.spec.cout, li.spec.cin // 32, dtype=torch.int32, device=dev)
+    ms = timed(lambda: b.nm_mask(Wp, bits, wl.n, wl.m), K)
+    by = li.spec.cout * li.spec.cin * 2 + li.spec.cout * li.spec.cin // 8
+    out["nm_mask"] = {"ms": ms, "GB/s": by / (ms / 1e3) / 1e9, "frac": by / (ms / 1e3) / 1e9 / pk["hbm_gbs"],
+                      "bytes": by, "shape": [li.spec.cout, li.spec.cin], "nm": f"{wl.n}:{wl.m}"}
+    del Wp, bits
+
+    # Sinkhorn scaling run: every projection of a 40-layer 13B-shaped model
+    nblk = 40 * (6 * 5120 + 13824) // 64
+    Bk = 64
+    gen = torch.Generator(device=dev).manual_seed(7)
+    Lb = torch.randn(nblk, Bk, Bk, device=dev, generator=gen) * 1e-3
+    Pb = torch.empty_like(Lb)
+    ck = torch.empty(nblk, wl.iters, 2, Bk, device=dev)
+    dP = torch.randn(nblk, Bk, Bk, device=dev, generator=gen)
+    dLb = torch.empty_like(Lb)
+    ms_f = timed(lambda: b.sinkhorn_fwd(Lb, Pb, ck, wl.tau, wl.iters), 5, flush_between=False)
+    ms_b = timed(lambda: b.sinkhorn_bwd(Lb, ck, dP, dLb, wl.tau, wl.iters), 5, flush_between=False)
+    bf = nblk * Bk * Bk * 8 + nblk * wl.iters * 2 * Bk * 4
+    bb = nblk * Bk * Bk * 12 + nblk * wl.iters * 2 * Bk * 4
+    out["sinkhorn_scaling"] = {
+        "blocks": nblk, "B": Bk, "iters": wl.iters, "L_MB": nblk * Bk * Bk * 4 / 1e6,
+        "fwd": {"ms": ms_f, "GB/s": bf / (ms_f / 1e3) / 1e9, "frac": bf / (ms_f / 1e3) / 1e9 / pk["hbm_gbs"]},
+        "bwd": {"ms": ms_b, "GB/s": bb / (ms_b / 1e3) / 1e9, "frac": bb / (ms_b / 1e3) / 1e9 / pk["hbm_gbs"]},
+        "note": "inputs larger than L2 (456 MB of logits per launch)"}
+    del Lb, Pb, ck, dP, dLb
+    torch.cuda.empty_cache()
+    return out
+
+
+def cpu_baseline_one_core(wl):
+    """The oracle on one BLAS thread: one whole step of the same layer."""
+    from oracle import lcp_oracle as O
+    from learnable_channel_permutation_b200 import synth
+    try:
+        from threadpoolctl import threadpool_limits
+    except Exception:
+        return None
+    li = synth.make_inputs(wl)[0]
+    with threadpool_limits(limits=1):
+        t0 = time.perf_counter()
+        O.step(li.W, li.X, li.L, wl.tau, wl.iters, wl.n, wl.m)
+        el = time.perf_counter() - t0
+    return {"value": 1.0 / el, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"1 whole fwd+bwd step of the {wl.name} layer (float64 numpy oracle, one BLAS thread), "
+                      f"{el:.1f} s"}
 
 
 def traffic_for(kernel, simt):

@@ -45,7 +45,7 @@
 extern "C" {
 #endif
 
-#define LCP_ABI_VERSION 1
+#define LCP_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define LCP_API __attribute__((visibility("default")))
@@ -71,6 +71,11 @@ typedef enum { LCP_F32 = 0, LCP_BF16 = 1 } lcp_dtype;
 #define LCP_FLAG_SIMT         0x2u  /* run every contraction on the CUDA-core (SIMT) kernels
                                        instead of the tensor-core kernels (bf16 only; the
                                        f32 dtype always uses SIMT kernels)              */
+#define LCP_FLAG_CACHED_DENSE 0x4u  /* read the dense output Y_d = X W^T from layer.Yd
+                                       instead of computing it: the dense output depends
+                                       on neither L nor P, so a loop over one calibration
+                                       batch computes it once (the library's extension of
+                                       the objective; the pages evaluate it per step)  */
 
 typedef struct {
   int block;        /* B, the permutation block size                                */
@@ -91,6 +96,10 @@ typedef struct {
   uint32_t* mask;   /* out [C_out, C_in/32] mask bits (optional, NULL = not returned) */
   float* Wp;        /* out [C_out, C_in] W' (only with LCP_FLAG_WRITE_WPRIME)         */
   int cout, cin, tokens;
+  float* Yd;        /* [T, C_out] float32 dense output X W^T, optional: with
+                       LCP_FLAG_CACHED_DENSE an input (required; it must hold X W^T for
+                       this W and X, e.g. written by an earlier step), otherwise, when
+                       non-NULL, an output the step fills                                */
 } lcp_layer;
 
 /* Bytes of workspace lcp_step needs for these layers (the layers run one after

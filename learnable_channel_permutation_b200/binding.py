@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "csrc", "lib
 F32, BF16 = 0, 1
 FLAG_WRITE_WPRIME = 0x1
 FLAG_SIMT = 0x2
+FLAG_CACHED_DENSE = 0x4
 TIMED_EVENTS = 8
 STAGES = ("sinkhorn_fwd", "permute_mask", "calib_gemm", "loss", "bwd_gemm", "block_bwd", "sinkhorn_bwd")
 
@@ -28,7 +29,7 @@ _c_void_p, _c_int, _c_float = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
 class LcpLayer(ctypes.Structure):
     _fields_ = [("W", _c_void_p), ("X", _c_void_p), ("L", _c_void_p), ("P", _c_void_p),
                 ("dL", _c_void_p), ("loss", _c_void_p), ("mask", _c_void_p), ("Wp", _c_void_p),
-                ("cout", _c_int), ("cin", _c_int), ("tokens", _c_int)]
+                ("cout", _c_int), ("cin", _c_int), ("tokens", _c_int), ("Yd", _c_void_p)]
 
 
 class LcpHparams(ctypes.Structure):
@@ -129,7 +130,8 @@ def make_layer(d: Dict[str, torch.Tensor], wdtype) -> LcpLayer:
     return LcpLayer(_ptr(W, wdtype, "W"), _ptr(X, wdtype, "X"), _ptr(Lg, torch.float32, "L"),
                     _ptr(d["P"], torch.float32, "P"), _ptr(d["dL"], torch.float32, "dL"),
                     _ptr(d["loss"], torch.float32, "loss"), _ptr(d.get("mask"), torch.int32, "mask"),
-                    _ptr(d.get("Wp"), torch.float32, "Wp"), cout, cin, tokens)
+                    _ptr(d.get("Wp"), torch.float32, "Wp"), cout, cin, tokens,
+                    _ptr(d.get("Yd"), torch.float32, "Yd"))
 
 
 class Step:

@@ -120,7 +120,7 @@ lcp_status check_hparams(const lcp_hparams* hp) {
     return fail(LCP_ERR_ARG, "iters = %d is not in [1, 1000]", hp->iters);
   if (!(hp->tau > 0.f) || !std::isfinite(hp->tau))
     return fail(LCP_ERR_ARG, "tau must be positive and finite");
-  if (hp->flags & ~(LCP_FLAG_WRITE_WPRIME | LCP_FLAG_SIMT))
+  if (hp->flags & ~(LCP_FLAG_WRITE_WPRIME | LCP_FLAG_SIMT | LCP_FLAG_CACHED_DENSE))
     return fail(LCP_ERR_ARG, "unknown flags 0x%x", hp->flags);
   return LCP_OK;
 }
@@ -134,6 +134,8 @@ lcp_status check_layer(const lcp_layer& l, const lcp_hparams& hp, int idx) {
     return fail(LCP_ERR_NULL, "layer %d: W, X, L, P, dL and loss are required", idx);
   if ((hp.flags & LCP_FLAG_WRITE_WPRIME) && !l.Wp)
     return fail(LCP_ERR_NULL, "layer %d: LCP_FLAG_WRITE_WPRIME needs layer.Wp", idx);
+  if ((hp.flags & LCP_FLAG_CACHED_DENSE) && !l.Yd)
+    return fail(LCP_ERR_NULL, "layer %d: LCP_FLAG_CACHED_DENSE needs layer.Yd", idx);
   if (l.cout < 8 || l.cout % 8 || l.cout > kMaxDim)
     return fail(LCP_ERR_SHAPE, "layer %d: C_out = %d must be a positive multiple of 8", idx, l.cout);
   if (l.cin < hp.block || l.cin % hp.block || l.cin % 32 || l.cin > kMaxDim)
@@ -145,7 +147,7 @@ lcp_status check_layer(const lcp_layer& l, const lcp_hparams& hp, int idx) {
     return fail(LCP_ERR_SHAPE,
                 "layer %d: C_in = %d must be a multiple of 64 on the tensor-core path "
                 "(LCP_FLAG_SIMT accepts multiples of 32)", idx, l.cin);
-  const void* ptrs[] = {l.W, l.X, l.L, l.P, l.dL, l.mask, l.Wp};
+  const void* ptrs[] = {l.W, l.X, l.L, l.P, l.dL, l.mask, l.Wp, l.Yd};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return fail(LCP_ERR_ARG, "layer %d: every pointer must be 16-byte aligned", idx);
   return LCP_OK;
@@ -184,7 +186,7 @@ Plan make_plan(const lcp_layer& l, const lcp_hparams& hp) {
   p.wp = take(simt_bwd ? oc * ic * 4 : 0);
   p.amask = take(simt_bwd ? oc * ic * 4 : 0);
   p.at = take(oc * ic * es);
-  p.yd = take(T * oc * 4);
+  p.yd = take(l.Yd ? 0 : T * oc * 4);   // the caller's Yd replaces the workspace copy
   p.ys = take(T * oc * 4);
   p.stats = take(T * 16);
   p.counter = take(256);
@@ -241,7 +243,8 @@ lcp_status layer_simt(const lcp_layer& l, const lcp_hparams& hp, const Plan& p, 
   float* Wp = (hp.flags & LCP_FLAG_WRITE_WPRIME) ? l.Wp : at<float>(ws, p.wp);
   float* Am = at<float>(ws, p.amask);
   void* At = at<void>(ws, p.at);
-  float* Yd = at<float>(ws, p.yd);
+  float* Yd = l.Yd ? l.Yd : at<float>(ws, p.yd);
+  const bool cached = (hp.flags & LCP_FLAG_CACHED_DENSE) != 0;
   float* Ys = at<float>(ws, p.ys);
   float* stats = at<float>(ws, p.stats);
   void* G = at<void>(ws, p.g);
@@ -264,8 +267,9 @@ lcp_status layer_simt(const lcp_layer& l, const lcp_hparams& hp, const Plan& p, 
                            LCP_F32, LCP_F32, dt, st));
   LCP_TRY(record(ev, 2, st));
   // Yd = X W^T, Ys = X At^T   ([T, C_out])
-  LCP_TRY(launch_simt_gemm({l.tokens, l.cout, l.cin, 1, l.X, 0, ic, 1, l.W, 0, 1, ic, Yd, 0, oc, 1, 1.f, 0.f},
-                           dt, dt, LCP_F32, st));
+  if (!cached)
+    LCP_TRY(launch_simt_gemm({l.tokens, l.cout, l.cin, 1, l.X, 0, ic, 1, l.W, 0, 1, ic, Yd, 0, oc, 1, 1.f, 0.f},
+                             dt, dt, LCP_F32, st));
   LCP_TRY(launch_simt_gemm({l.tokens, l.cout, l.cin, 1, l.X, 0, ic, 1, At, 0, 1, ic, Ys, 0, oc, 1, 1.f, 0.f},
                            dt, dt, LCP_F32, st));
   LCP_TRY(record(ev, 3, st));
@@ -296,7 +300,7 @@ constexpr int kTcLaunchesSimtBwd = 11;   // B = 256: block backward on CUDA core
 
 int launches_per_layer(const lcp_layer& l, const lcp_hparams& hp) {
   const int loss = loss_launches(l.cout);
-  if (!use_tc(hp)) return kSimtLaunches + loss;
+  if (!use_tc(hp)) return kSimtLaunches - ((hp.flags & LCP_FLAG_CACHED_DENSE) ? 1 : 0) + loss;
   return (block_bwd_tc_supported(hp.block) ? kTcLaunches : kTcLaunchesSimtBwd) + loss;
 }
 
@@ -311,7 +315,8 @@ lcp_status layer_tc(const lcp_layer& l, const lcp_hparams& hp, const Plan& p, vo
   uint32_t* mask = l.mask ? l.mask : at<uint32_t>(ws, p.mask);
   float* Wp = (hp.flags & LCP_FLAG_WRITE_WPRIME) ? l.Wp : nullptr;
   auto* At = at<__nv_bfloat16>(ws, p.at);
-  float* Yd = at<float>(ws, p.yd);
+  float* Yd = l.Yd ? l.Yd : at<float>(ws, p.yd);
+  const bool cached = (hp.flags & LCP_FLAG_CACHED_DENSE) != 0;
   float* Ys = at<float>(ws, p.ys);
   float* stats = at<float>(ws, p.stats);
   auto* G = at<__nv_bfloat16>(ws, p.g);
@@ -326,7 +331,10 @@ lcp_status layer_tc(const lcp_layer& l, const lcp_hparams& hp, const Plan& p, vo
   LCP_TRY(record(ev, 1, st));
   LCP_TRY(launch_permute_mask_tc(W, pt_hi, pt_lo, p_hi, mask, At, Wp, l.cout, l.cin, B, hp.n, hp.m, st));
   LCP_TRY(record(ev, 2, st));
-  LCP_TRY(launch_calib_gemm_tc(X, W, At, Yd, Ys, l.tokens, l.cout, l.cin, st));
+  if (cached)   // Y_s = X At^T alone (one problem)
+    LCP_TRY(launch_calib_gemm_tc(X, At, nullptr, Ys, nullptr, l.tokens, l.cout, l.cin, st));
+  else
+    LCP_TRY(launch_calib_gemm_tc(X, W, At, Yd, Ys, l.tokens, l.cout, l.cin, st));
   LCP_TRY(record(ev, 3, st));
   LCP_TRY(launch_loss(Yd, Ys, stats, G, LCP_BF16, l.loss, at<unsigned>(ws, p.counter), l.cout, l.tokens, st));
   LCP_TRY(record(ev, 4, st));

@@ -74,6 +74,8 @@ def test_workspace_size_for_valid_layers():
     (lambda l, h: setattr(l, "tokens", 0), 2),
     (lambda l, h: setattr(l, "X", 0x10000008), 7),  # misaligned
     (lambda l, h: setattr(h, "flags", b.FLAG_WRITE_WPRIME), 1),  # needs layer.Wp
+    (lambda l, h: setattr(h, "flags", b.FLAG_CACHED_DENSE), 1),  # needs layer.Yd
+    (lambda l, h: (setattr(h, "flags", b.FLAG_CACHED_DENSE), setattr(l, "Yd", 0x10000004)), 7),  # misaligned
 ])
 def test_host_validation_codes(mut, code):
     l = _layer()
@@ -112,3 +114,13 @@ def test_launch_count_reported():
     c = ctypes.c_int(0)
     assert b.lib().lcp_step_launches(arr, 2, ctypes.byref(hp), ctypes.byref(c)) == 0
     assert c.value > 0 and c.value % 2 == 0
+
+
+def test_workspace_shrinks_when_the_caller_holds_yd():
+    """A caller-provided Y_d replaces the workspace copy (T x C_out float32)."""
+    hp = b.hparams(64, 2, 4, 5, 0.5, b.BF16)
+    st, n = _ws([_layer(cout=256, T=512)], hp)
+    l = _layer(cout=256, T=512)
+    l.Yd = 0x70000000
+    st2, n2 = _ws([l], hp)
+    assert st == 0 and st2 == 0 and n - n2 >= 512 * 256 * 4
