@@ -19,9 +19,15 @@ Sources (the web pages the method is taken from):
   N largest |w|, zero the rest) and section 2.2 (Sinkhorn in the log domain,
   row normalisation first, then column normalisation, then exp).
 
+* [PermLLM] "Method", subsection 2 (hardening and gradient approximation):
+  in the forward pass the soft P_hat is hardened to the permutation
+  P = argmax over permutation matrices of Tr(P^T P_hat) (the Hungarian
+  algorithm), and the backward pass takes dP/dP_hat = 1 (straight-through).
+
 Readings where the pages are silent or garbled (each is restated where used):
 
-1. The forward pass uses the soft P (no Hungarian hardening).
+1. The default forward pass uses the soft P; ``step_hard`` is the hardened
+   variant (per block, since P_B is block-diagonal the trace splits by block).
 2. The mask score is |W'| with W' = W P_B.
 3. The mask is a constant in the backward pass (straight-through).
 4. One iteration = a row normalisation followed by a column normalisation.
@@ -200,6 +206,43 @@ def cosine_loss_grad(Yd: np.ndarray, Ys: np.ndarray) -> np.ndarray:
 
 
 # ---------------------------------------------------------------------------
+# Hardening  ([PermLLM] Method 2)
+# ---------------------------------------------------------------------------
+
+def harden(P: np.ndarray) -> np.ndarray:
+    """Per block, the permutation maximising Tr(P_b^T P_hat_b) = sum_i P_hat_b[i, pi(i)].
+
+    Returns pi as an int array [nb, B] (row i of block b goes to column pi[b, i]).
+    The maximisation is a linear assignment problem; scipy's solver is the step
+    used here (the pins check it against enumeration of all permutations).
+    When several permutations reach the maximum any of them is a correct result.
+    """
+    from scipy.optimize import linear_sum_assignment
+    P = np.asarray(P, np.float64)
+    nb, B, _ = P.shape
+    perm = np.empty((nb, B), np.int64)
+    for b in range(nb):
+        rows, cols = linear_sum_assignment(P[b], maximize=True)
+        perm[b, rows] = cols
+    return perm
+
+
+def perm_matrix(perm: np.ndarray) -> np.ndarray:
+    """The 0/1 matrices of per-block permutations pi: P[b, i, pi[b, i]] = 1."""
+    nb, B = perm.shape
+    P = np.zeros((nb, B, B))
+    for b in range(nb):
+        P[b, np.arange(B), perm[b]] = 1.0
+    return P
+
+
+def assignment_value(P: np.ndarray, perm: np.ndarray) -> np.ndarray:
+    """Per block, sum_i P[b, i, pi[b, i]] (the objective the hardening maximises)."""
+    nb, B = perm.shape
+    return np.array([np.sum(np.asarray(P[b], np.float64)[np.arange(B), perm[b]]) for b in range(nb)])
+
+
+# ---------------------------------------------------------------------------
 # One forward + backward step of one layer
 # ---------------------------------------------------------------------------
 
@@ -263,6 +306,28 @@ def step(W: np.ndarray, X_tokens: np.ndarray, logits: np.ndarray, tau: float, n_
     """Forward and backward of one layer; returns the forward dict plus G, dP, dL."""
     fw = forward(W, X_tokens, logits, tau, n_iters, n, m, mask=mask)
     fw.update(backward(fw, tau))
+    return fw
+
+
+def step_hard(W: np.ndarray, X_tokens: np.ndarray, logits: np.ndarray, tau: float, n_iters: int,
+              n: int, m: int, perm: Optional[np.ndarray] = None,
+              mask: Optional[np.ndarray] = None) -> Dict[str, object]:
+    """Forward with the hardened permutation, backward straight through it.
+
+    P_hat = Sinkhorn(L / tau); P = harden(P_hat) (or the given ``perm``, to
+    compare with another implementation's choice among tied maxima); the
+    forward pass uses P; the reverse pass computes dP for P exactly as in
+    ``backward`` and hands it to the Sinkhorn reverse pass as dP_hat
+    (dP/dP_hat = 1).
+    """
+    P_soft, trace = sinkhorn(logits, tau, n_iters)
+    if perm is None:
+        perm = harden(P_soft)
+    P_hard = perm_matrix(np.asarray(perm))
+    fw = forward(W, X_tokens, logits, tau, n_iters, n, m, mask=mask, P=P_hard)
+    fw.update(backward(fw, tau))
+    fw["dL"] = sinkhorn_backward(trace, P_soft, fw["dP"], tau)
+    fw["P_soft"], fw["perm"], fw["trace"] = P_soft, np.asarray(perm), trace
     return fw
 
 

@@ -416,3 +416,83 @@ def test_token_shards_sum_to_the_full_gradient():
     b = O.step(W, X[12:], L, 0.5, 5, 2, 4)
     assert abs((12 * a["loss"] + 18 * b["loss"]) / 30 - full["loss"]) < 1e-14
     assert np.allclose((12 * a["dL"] + 18 * b["dL"]) / 30, full["dL"], rtol=1e-10, atol=1e-16)
+
+
+# --------------------------------------------------------------- hardening ---
+
+def _all_perm_values(Pb):
+    B = Pb.shape[0]
+    return {pi: float(sum(Pb[i, pi[i]] for i in range(B))) for pi in itertools.permutations(range(B))}
+
+
+@pytest.mark.parametrize("B", [2, 3, 5, 7])
+def test_harden_attains_the_brute_force_maximum(B):
+    """Tr(P^T P_hat) at the hardened P equals the maximum over all B! permutations."""
+    rng = np.random.default_rng(100 + B)
+    L = rng.normal(0, 1.0, (4, B, B))
+    P, _ = O.sinkhorn(L, 0.7, 5)
+    perm = O.harden(P)
+    vals = O.assignment_value(P, perm)
+    for b in range(4):
+        allv = _all_perm_values(P[b])
+        assert np.isclose(vals[b], max(allv.values()), rtol=0, atol=1e-12)
+        assert sorted(perm[b]) == list(range(B))
+
+
+def test_harden_recovers_a_dominant_permutation():
+    """P_hat = 0.7 Pi + 0.3 / B (doubly stochastic) hardens to Pi itself."""
+    rng = np.random.default_rng(5)
+    B = 16
+    pis = np.stack([rng.permutation(B) for _ in range(3)])
+    P = 0.7 * O.perm_matrix(pis) + 0.3 / B
+    assert np.array_equal(O.harden(P), pis)
+
+
+def test_harden_ties_give_a_valid_permutation_with_the_maximum():
+    """Uniform P_hat: every permutation is optimal; the result is a permutation of value 1."""
+    P = np.full((2, 8, 8), 1.0 / 8)
+    perm = O.harden(P)
+    for b in range(2):
+        assert sorted(perm[b]) == list(range(8))
+    assert np.allclose(O.assignment_value(P, perm), 1.0)
+
+
+def test_step_hard_forward_equals_the_soft_path_at_the_hard_matrix():
+    """The hardened forward is the plain forward evaluated at P = perm_matrix(pi)."""
+    rng = np.random.default_rng(8)
+    W = rng.normal(0, 0.02, (16, 32))
+    X = rng.normal(0, 1, (24, 32))
+    L = rng.normal(0, 0.3, (2, 16, 16))
+    fw = O.step_hard(W, X, L, 0.5, 5, 2, 4)
+    ref = O.forward(W, X, L, 0.5, 5, 2, 4, P=O.perm_matrix(fw["perm"]))
+    assert fw["loss"] == ref["loss"]
+    assert np.array_equal(fw["mask"], ref["mask"])
+    # a hard permutation makes W' an exact column gather
+    Wp = np.concatenate([W[:, b * 16:(b + 1) * 16][:, np.argsort(fw["perm"][b])] for b in range(2)], axis=1)
+    assert np.array_equal(fw["Wp"], Wp)
+
+
+def test_step_hard_straight_through_gradient():
+    """dL is the Sinkhorn reverse pass of the hard-P gradient (dP_hat = dP), and it
+    differs from the soft-path dL (the estimator is not the true derivative)."""
+    rng = np.random.default_rng(9)
+    W = rng.normal(0, 0.02, (16, 32))
+    X = rng.normal(0, 1, (24, 32))
+    L = rng.normal(0, 0.3, (2, 16, 16))
+    fw = O.step_hard(W, X, L, 0.5, 5, 2, 4)
+    P_soft, trace = O.sinkhorn(L, 0.5, 5)
+    assert np.array_equal(P_soft, fw["P_soft"])
+    dP = fw["dP"]
+    assert np.allclose(fw["dL"], O.sinkhorn_backward(trace, P_soft, dP, 0.5), rtol=0, atol=0)
+    # dP of the hard path by finite differences in P at the hard matrix (mask held)
+    P_hard = O.perm_matrix(fw["perm"])
+    eps = 1e-6
+    for (b, i, j) in [(0, 1, 2), (1, 5, 7), (0, 15, 0)]:
+        Pp, Pm = P_hard.copy(), P_hard.copy()
+        Pp[b, i, j] += eps
+        Pm[b, i, j] -= eps
+        lp = O.forward(W, X, L, 0.5, 5, 2, 4, P=Pp, mask=fw["mask"])["loss"]
+        lm = O.forward(W, X, L, 0.5, 5, 2, 4, P=Pm, mask=fw["mask"])["loss"]
+        assert np.isclose((lp - lm) / (2 * eps), dP[b, i, j], rtol=1e-5, atol=1e-9)
+    soft = O.step(W, X, L, 0.5, 5, 2, 4)
+    assert not np.allclose(soft["dL"], fw["dL"])
