@@ -433,6 +433,7 @@ def extras(args, b, synth, wl, li, layer, step, flush, pk, dev):
 
     - cached_dense: the step with LCP_FLAG_CACHED_DENSE (Y_d read from layer.Yd,
       written once by an uncached step), same timing protocol as the headline;
+    - hard_step: the step with LCP_FLAG_HARD, and the hardening kernel alone;
     - nm_mask: the standalone mask kernel on a bf16 W' of the layer's shape,
       against the measured HBM copy bandwidth (bytes: 2 read + 1/8 written per element);
     - sinkhorn_scaling: Sinkhorn forward then reverse over the logits of every
@@ -473,6 +474,21 @@ def extras(args, b, synth, wl, li, layer, step, flush, pk, dev):
                            "note": "LCP_FLAG_CACHED_DENSE: Y_d = X W^T read from layer.Yd (computed once), "
                                    "so the step runs one calibration GEMM problem instead of two; "
                                    "not the headline", "algorithmic_flop": 2 * flop}
+
+    # hardened step (LCP_FLAG_HARD: per-block assignment, straight-through backward)
+    nb = li.spec.cin // wl.block
+    layer["perm"] = torch.empty(nb, wl.block, dtype=torch.int32, device=dev)
+    hard = b.Step([layer], wl.block, wl.n, wl.m, wl.iters, wl.tau, flags=b.FLAG_HARD)
+    g = b.capture(hard)
+    ms = timed(g.replay, K)
+    del g
+    ms_h = timed(lambda: b.harden(layer["P"], layer["perm"]), K)
+    layer.pop("perm")
+    out["hard_step"] = {"value": 1e3 / ms, "unit": UNIT, "ms_per_step": ms, "steps": K,
+                        "harden_kernel_ms": ms_h, "blocks": nb,
+                        "note": "LCP_FLAG_HARD: the forward pass uses the per-block maximum-weight "
+                                "assignment of the Sinkhorn output (one warp per block), the backward "
+                                "pass is straight-through; not the headline"}
 
     # standalone N:M mask on a bf16 W' of the layer's shape
     Wp = torch.randn(li.spec.cout, li.spec.cin, device=dev).to(torch.bfloat16)

@@ -71,6 +71,11 @@ typedef enum { LCP_F32 = 0, LCP_BF16 = 1 } lcp_dtype;
 #define LCP_FLAG_SIMT         0x2u  /* run every contraction on the CUDA-core (SIMT) kernels
                                        instead of the tensor-core kernels (bf16 only; the
                                        f32 dtype always uses SIMT kernels)              */
+#define LCP_FLAG_HARD         0x8u  /* harden P before use ("Method" 2): every block of the
+                                       Sinkhorn output is replaced by the permutation
+                                       maximising Tr(P^T P_hat) (lcp_harden); the backward
+                                       pass is straight-through, dP_hat = dP.  layer.P
+                                       still returns the soft P_hat                    */
 #define LCP_FLAG_CACHED_DENSE 0x4u  /* read the dense output Y_d = X W^T from layer.Yd
                                        instead of computing it: the dense output depends
                                        on neither L nor P, so a loop over one calibration
@@ -100,6 +105,8 @@ typedef struct {
                        LCP_FLAG_CACHED_DENSE an input (required; it must hold X W^T for
                        this W and X, e.g. written by an earlier step), otherwise, when
                        non-NULL, an output the step fills                                */
+  int32_t* perm;    /* out [C_in/B, B] optional: with LCP_FLAG_HARD, perm[b][i] = the
+                       column of block b that row i is sent to                          */
 } lcp_layer;
 
 /* Bytes of workspace lcp_step needs for these layers (the layers run one after
@@ -144,6 +151,16 @@ LCP_API lcp_status lcp_sinkhorn_fwd(const float* L, float* P, float* ckpt, int n
 LCP_API lcp_status lcp_sinkhorn_bwd(const float* L, const float* ckpt, const float* dP, int dP_splits,
                             float* dL, int nblocks, int B, float tau, int iters,
                             cudaStream_t stream);
+
+/* Hardening ("Method" 2: P = argmax over permutations of Tr(P^T P_hat), the
+ * Hungarian algorithm): for each of `nblocks` B x B blocks of P_hat (float32,
+ * [nblocks, B, B]) the permutation maximising sum_i P_hat[i, perm[i]], solved
+ * exactly (shortest augmenting paths; float32 potentials).  perm: int32
+ * [nblocks, B] (required); P_hard: float32 [nblocks, B, B] 0/1 matrices
+ * (optional, NULL = not written).  B in {32, 64, 128, 256}.  When several
+ * permutations attain the maximum, the result is one of them (deterministic). */
+LCP_API lcp_status lcp_harden(const float* P_hat, int32_t* perm, float* P_hard, int nblocks, int B,
+                              cudaStream_t stream);
 
 /* W' = W * blockdiag(P) ("Method", 3: W_hat_B = W P_B).  W [cout, cin] in
  * `dtype`, P [cin/B, B, B], Wp [cout, cin] float32. */

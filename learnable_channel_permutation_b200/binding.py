@@ -20,6 +20,7 @@ F32, BF16 = 0, 1
 FLAG_WRITE_WPRIME = 0x1
 FLAG_SIMT = 0x2
 FLAG_CACHED_DENSE = 0x4
+FLAG_HARD = 0x8
 TIMED_EVENTS = 8
 STAGES = ("sinkhorn_fwd", "permute_mask", "calib_gemm", "loss", "bwd_gemm", "block_bwd", "sinkhorn_bwd")
 
@@ -29,7 +30,7 @@ _c_void_p, _c_int, _c_float = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
 class LcpLayer(ctypes.Structure):
     _fields_ = [("W", _c_void_p), ("X", _c_void_p), ("L", _c_void_p), ("P", _c_void_p),
                 ("dL", _c_void_p), ("loss", _c_void_p), ("mask", _c_void_p), ("Wp", _c_void_p),
-                ("cout", _c_int), ("cin", _c_int), ("tokens", _c_int), ("Yd", _c_void_p)]
+                ("cout", _c_int), ("cin", _c_int), ("tokens", _c_int), ("Yd", _c_void_p), ("perm", _c_void_p)]
 
 
 class LcpHparams(ctypes.Structure):
@@ -77,6 +78,7 @@ def lib() -> ctypes.CDLL:
                             _c_void_p], _c_int),
         "lcp_grad_gemm": ([_c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_void_p], _c_int),
         "lcp_device_error": ([P(_c_int), _c_int], _c_int),
+        "lcp_harden": ([_c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_void_p], _c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -131,7 +133,7 @@ def make_layer(d: Dict[str, torch.Tensor], wdtype) -> LcpLayer:
                     _ptr(d["P"], torch.float32, "P"), _ptr(d["dL"], torch.float32, "dL"),
                     _ptr(d["loss"], torch.float32, "loss"), _ptr(d.get("mask"), torch.int32, "mask"),
                     _ptr(d.get("Wp"), torch.float32, "Wp"), cout, cin, tokens,
-                    _ptr(d.get("Yd"), torch.float32, "Yd"))
+                    _ptr(d.get("Yd"), torch.float32, "Yd"), _ptr(d.get("perm"), torch.int32, "perm"))
 
 
 class Step:
@@ -232,6 +234,12 @@ def permute_weight(W: torch.Tensor, P: torch.Tensor, Wp: torch.Tensor) -> None:
     cout, cin = W.shape
     check(lib().lcp_permute_weight(_ptr(W, None, "W"), _ptr(P, torch.float32, "P"), _ptr(Wp, torch.float32, "Wp"),
                                    cout, cin, P.shape[1], _dt(W), _stream(None)))
+
+
+def harden(P: torch.Tensor, perm: torch.Tensor, P_hard: Optional[torch.Tensor] = None) -> None:
+    nb, B, _ = P.shape
+    check(lib().lcp_harden(_ptr(P, torch.float32, "P"), _ptr(perm, torch.int32, "perm"),
+                           _ptr(P_hard, torch.float32, "P_hard"), nb, B, _stream(None)))
 
 
 def nm_mask(Wp: torch.Tensor, bits: torch.Tensor, n: int, m: int) -> None:

@@ -120,7 +120,7 @@ lcp_status check_hparams(const lcp_hparams* hp) {
     return fail(LCP_ERR_ARG, "iters = %d is not in [1, 1000]", hp->iters);
   if (!(hp->tau > 0.f) || !std::isfinite(hp->tau))
     return fail(LCP_ERR_ARG, "tau must be positive and finite");
-  if (hp->flags & ~(LCP_FLAG_WRITE_WPRIME | LCP_FLAG_SIMT | LCP_FLAG_CACHED_DENSE))
+  if (hp->flags & ~(LCP_FLAG_WRITE_WPRIME | LCP_FLAG_SIMT | LCP_FLAG_CACHED_DENSE | LCP_FLAG_HARD))
     return fail(LCP_ERR_ARG, "unknown flags 0x%x", hp->flags);
   return LCP_OK;
 }
@@ -147,7 +147,7 @@ lcp_status check_layer(const lcp_layer& l, const lcp_hparams& hp, int idx) {
     return fail(LCP_ERR_SHAPE,
                 "layer %d: C_in = %d must be a multiple of 64 on the tensor-core path "
                 "(LCP_FLAG_SIMT accepts multiples of 32)", idx, l.cin);
-  const void* ptrs[] = {l.W, l.X, l.L, l.P, l.dL, l.mask, l.Wp, l.Yd};
+  const void* ptrs[] = {l.W, l.X, l.L, l.P, l.dL, l.mask, l.Wp, l.Yd, l.perm};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return fail(LCP_ERR_ARG, "layer %d: every pointer must be 16-byte aligned", idx);
   return LCP_OK;
@@ -157,7 +157,7 @@ lcp_status check_layer(const lcp_layer& l, const lcp_hparams& hp, int idx) {
 size_t esize(lcp_dtype d) { return d == LCP_F32 ? 4 : 2; }
 
 struct Plan {
-  size_t ckpt, img0, img1, img2, mask, wp, amask, at, yd, ys, stats, counter, g, dat, da, dp;
+  size_t ckpt, img0, img1, img2, mask, wp, amask, at, yd, ys, stats, counter, g, dat, da, dp, perm, phard;
   size_t total;
   int splits;
 };
@@ -194,6 +194,9 @@ Plan make_plan(const lcp_layer& l, const lcp_hparams& hp) {
   p.dat = take(oc * ic * (tc ? 2 : 4));
   p.da = take(simt_bwd ? oc * ic * 4 : 0);
   p.dp = take((size_t)p.splits * nb * B * B * 4);
+  const bool hard = (hp.flags & LCP_FLAG_HARD) != 0;
+  p.perm = take(hard && !l.perm ? nb * B * 4 : 0);
+  p.phard = take(hard && simt_bwd ? nb * B * B * 4 : 0);   // the CUDA-core products read P_hard as float32
   p.total = off;
   return p;
 }
@@ -256,14 +259,21 @@ lcp_status layer_simt(const lcp_layer& l, const lcp_hparams& hp, const Plan& p, 
   LCP_TRY(record(ev, 0, st));
   LCP_TRY(launch_sinkhorn_fwd(l.L, l.P, ckpt, nullptr, nullptr, nullptr, at<unsigned>(ws, p.counter), nb, B, hp.tau,
                               hp.iters, st));
+  // the permutation every product below uses: P_hat, or its hardening (straight-through)
+  const float* Pu = l.P;
+  if (hp.flags & LCP_FLAG_HARD) {
+    float* Ph = at<float>(ws, p.phard);
+    LCP_TRY(launch_harden(l.P, l.perm ? l.perm : at<int>(ws, p.perm), Ph, nullptr, nullptr, nullptr, nb, B, st));
+    Pu = Ph;
+  }
   LCP_TRY(record(ev, 1, st));
   // W'_b = W_b P_b
-  LCP_TRY(launch_simt_gemm({l.cout, B, B, nb, l.W, B, ic, 1, l.P, BB, B, 1, Wp, B, ic, 1, 1.f, 0.f},
+  LCP_TRY(launch_simt_gemm({l.cout, B, B, nb, l.W, B, ic, 1, Pu, BB, B, 1, Wp, B, ic, 1, 1.f, 0.f},
                            dt, LCP_F32, LCP_F32, st));
   LCP_TRY(launch_nm_mask(Wp, mask, l.cout, l.cin, hp.n, hp.m, LCP_F32, st));
   LCP_TRY(launch_apply_mask(Wp, mask, Am, l.cout, l.cin, st));
   // At_b = A_b P_b^T
-  LCP_TRY(launch_simt_gemm({l.cout, B, B, nb, Am, B, ic, 1, l.P, BB, 1, B, At, B, ic, 1, 1.f, 0.f},
+  LCP_TRY(launch_simt_gemm({l.cout, B, B, nb, Am, B, ic, 1, Pu, BB, 1, B, At, B, ic, 1, 1.f, 0.f},
                            LCP_F32, LCP_F32, dt, st));
   LCP_TRY(record(ev, 2, st));
   // Yd = X W^T, Ys = X At^T   ([T, C_out])
@@ -280,7 +290,7 @@ lcp_status layer_simt(const lcp_layer& l, const lcp_hparams& hp, const Plan& p, 
                            dt, dt, LCP_F32, st));
   LCP_TRY(record(ev, 5, st));
   // dA_b = dAt_b P_b ; dW' = M . dA ; dP_b = dAt_b^T A_b + W_b^T dW'_b
-  LCP_TRY(launch_simt_gemm({l.cout, B, B, nb, dAt, B, ic, 1, l.P, BB, B, 1, dA, B, ic, 1, 1.f, 0.f},
+  LCP_TRY(launch_simt_gemm({l.cout, B, B, nb, dAt, B, ic, 1, Pu, BB, B, 1, dA, B, ic, 1, 1.f, 0.f},
                            LCP_F32, LCP_F32, LCP_F32, st));
   LCP_TRY(launch_apply_mask(dA, mask, dA, l.cout, l.cin, st));
   LCP_TRY(launch_simt_gemm({B, B, l.cout, nb, dAt, B, 1, ic, Am, B, ic, 1, dP, BB, B, 1, 1.f, 0.f},
@@ -299,7 +309,7 @@ constexpr int kTcLaunches = 6;
 constexpr int kTcLaunchesSimtBwd = 11;   // B = 256: block backward on CUDA cores (6 launches)
 
 int launches_per_layer(const lcp_layer& l, const lcp_hparams& hp) {
-  const int loss = loss_launches(l.cout);
+  const int loss = loss_launches(l.cout) + ((hp.flags & LCP_FLAG_HARD) ? 1 : 0);
   if (!use_tc(hp)) return kSimtLaunches - ((hp.flags & LCP_FLAG_CACHED_DENSE) ? 1 : 0) + loss;
   return (block_bwd_tc_supported(hp.block) ? kTcLaunches : kTcLaunchesSimtBwd) + loss;
 }
@@ -328,6 +338,16 @@ lcp_status layer_tc(const lcp_layer& l, const lcp_hparams& hp, const Plan& p, vo
   LCP_TRY(record(ev, 0, st));
   LCP_TRY(launch_sinkhorn_fwd(l.L, l.P, ckpt, pt_hi, pt_lo, p_hi, at<unsigned>(ws, p.counter), nb, B, hp.tau,
                               hp.iters, st));
+  // with hardening the operand images (and, for the CUDA-core block backward,
+  // the float32 matrix) are those of the hard permutation; the Sinkhorn reverse
+  // pass still runs on the soft P_hat (straight-through)
+  const float* Pu = l.P;
+  if (hp.flags & LCP_FLAG_HARD) {
+    float* Ph = p.phard ? at<float>(ws, p.phard) : nullptr;
+    if (!block_bwd_tc_supported(B)) Pu = Ph;
+    LCP_TRY(launch_harden(l.P, l.perm ? l.perm : at<int>(ws, p.perm), block_bwd_tc_supported(B) ? nullptr : Ph,
+                          pt_hi, pt_lo, p_hi, nb, B, st));
+  }
   LCP_TRY(record(ev, 1, st));
   LCP_TRY(launch_permute_mask_tc(W, pt_hi, pt_lo, p_hi, mask, At, Wp, l.cout, l.cin, B, hp.n, hp.m, st));
   LCP_TRY(record(ev, 2, st));
@@ -349,10 +369,10 @@ lcp_status layer_tc(const lcp_layer& l, const lcp_hparams& hp, const Plan& p, vo
     float* Wp32 = at<float>(ws, p.wp);
     float* Am = at<float>(ws, p.amask);
     float* dA = at<float>(ws, p.da);
-    LCP_TRY(launch_simt_gemm({l.cout, B, B, nb, W, B, ic, 1, l.P, BB, B, 1, Wp32, B, ic, 1, 1.f, 0.f},
+    LCP_TRY(launch_simt_gemm({l.cout, B, B, nb, W, B, ic, 1, Pu, BB, B, 1, Wp32, B, ic, 1, 1.f, 0.f},
                              LCP_BF16, LCP_F32, LCP_F32, st));
     LCP_TRY(launch_apply_mask(Wp32, mask, Am, l.cout, l.cin, st));
-    LCP_TRY(launch_simt_gemm({l.cout, B, B, nb, dAt, B, ic, 1, l.P, BB, B, 1, dA, B, ic, 1, 1.f, 0.f},
+    LCP_TRY(launch_simt_gemm({l.cout, B, B, nb, dAt, B, ic, 1, Pu, BB, B, 1, dA, B, ic, 1, 1.f, 0.f},
                              LCP_BF16, LCP_F32, LCP_F32, st));
     LCP_TRY(launch_apply_mask(dA, mask, dA, l.cout, l.cin, st));
     LCP_TRY(launch_simt_gemm({B, B, l.cout, nb, dAt, B, 1, ic, Am, B, ic, 1, dP, BB, B, 1, 1.f, 0.f},
@@ -492,6 +512,19 @@ lcp_status lcp_permute_weight(const void* W, const float* P, float* Wp, int cout
                           dtype, LCP_F32, LCP_F32, stream);
 }
 
+lcp_status lcp_harden(const float* P_hat, int32_t* perm, float* P_hard, int nblocks, int B, cudaStream_t stream) {
+  if (!P_hat || !perm) return fail(LCP_ERR_NULL, "P_hat and perm are required");
+  if (B != 32 && B != 64 && B != 128 && B != 256)
+    return fail(LCP_ERR_SHAPE, "block size %d is not one of 32, 64, 128, 256", B);
+  if (nblocks < 0 || nblocks > kMaxDim) return fail(LCP_ERR_SHAPE, "nblocks = %d", nblocks);
+  if (!aligned16(P_hat) || (P_hard && !aligned16(P_hard)))
+    return fail(LCP_ERR_ARG, "P_hat and P_hard must be 16-byte aligned");
+  if (nblocks == 0) return LCP_OK;
+  LCP_TRY(check_arch());
+  cudaGetLastError();
+  return launch_harden(P_hat, perm, P_hard, nullptr, nullptr, nullptr, nblocks, B, stream);
+}
+
 lcp_status nm_mask(const void* Wp, uint32_t* mask_bits, int rows, int cols, int n, int m,
                    lcp_dtype dtype, cudaStream_t stream) {
   if (!Wp || !mask_bits) return fail(LCP_ERR_NULL, "Wp and mask_bits are required");
@@ -566,7 +599,7 @@ lcp_status lcp_loss_bwd(const float* Yd, const float* Ys, const float* stats, vo
 extern "C" lcp_status lcp_device_error(int* site, int reset) {
   using namespace lcp;
   if (!site) return fail(LCP_ERR_NULL, "site is NULL");
-  lcp_status (*const readers[])(int*, int) = {tc_error_gemm, tc_error_permute, tc_error_block_bwd};
+  lcp_status (*const readers[])(int*, int) = {tc_error_gemm, tc_error_permute, tc_error_block_bwd, harden_error};
   int first = 0;
   for (auto rd : readers) {
     int v = 0;

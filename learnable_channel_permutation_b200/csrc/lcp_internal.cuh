@@ -181,6 +181,13 @@ lcp_status launch_block_bwd_tc(const __nv_bfloat16* W, const __nv_bfloat16* dAt,
 int block_bwd_tc_splits(int cout, int cin, int B);
 bool block_bwd_tc_supported(int B);   // B <= 128 (TMEM/smem budget of the fused kernel)
 
+// Hardening (per-block maximum-weight assignment).  Writes perm [nblocks, B],
+// optionally the 0/1 matrices P_hard and the bf16 operand images of P_hard in
+// the Sinkhorn kernel's tile layout (all three image pointers or none).
+lcp_status launch_harden(const float* P, int* perm, float* P_hard, __nv_bfloat16* img_pt_hi,
+                         __nv_bfloat16* img_pt_lo, __nv_bfloat16* img_p_hi, int nblocks, int B, cudaStream_t st);
+lcp_status harden_error(int* site, int reset);
+
 // Device error words of the tensor-core translation units: the first wait
 // site that timed out since the last reset, 0 if none (cleared when `reset`).
 lcp_status tc_error_gemm(int* site, int reset);
