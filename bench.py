@@ -434,6 +434,7 @@ def extras(args, b, synth, wl, li, layer, step, flush, pk, dev):
     - cached_dense: the step with LCP_FLAG_CACHED_DENSE (Y_d read from layer.Yd,
       written once by an uncached step), same timing protocol as the headline;
     - hard_step: the step with LCP_FLAG_HARD, and the hardening kernel alone;
+    - train: steps of lcp_train (step + AdamW on L, temperature schedule);
     - nm_mask: the standalone mask kernel on a bf16 W' of the layer's shape,
       against the measured HBM copy bandwidth (bytes: 2 read + 1/8 written per element);
     - sinkhorn_scaling: Sinkhorn forward then reverse over the logits of every
@@ -489,6 +490,15 @@ def extras(args, b, synth, wl, li, layer, step, flush, pk, dev):
                         "note": "LCP_FLAG_HARD: the forward pass uses the per-block maximum-weight "
                                 "assignment of the Sinkhorn output (one warp per block), the backward "
                                 "pass is straight-through; not the headline"}
+
+    # training steps: lcp_step at the scheduled temperature + AdamW on L (lcp_train)
+    tr_step = b.Step([layer], wl.block, wl.n, wl.m, wl.iters, wl.tau, workspace=step.ws)
+    total = 10
+    trainer = b.Trainer(tr_step, b.adamw_params(lr=5e-3), total)
+    ms_tr = timed(lambda: trainer.run(0, total), 3) / total
+    out["train"] = {"value": 1e3 / ms_tr, "unit": UNIT, "ms_per_step": ms_tr, "steps_per_call": total,
+                    "note": "lcp_train: ten steps per call (eager launches), temperature 1 -> 0.1, AdamW "
+                            "lr 5e-3 on the logits after every step; L2 flushed before each call only"}
 
     # standalone N:M mask on a bf16 W' of the layer's shape
     Wp = torch.randn(li.spec.cout, li.spec.cin, device=dev).to(torch.bfloat16)

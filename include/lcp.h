@@ -152,6 +152,41 @@ LCP_API lcp_status lcp_sinkhorn_bwd(const float* L, const float* ckpt, const flo
                             float* dL, int nblocks, int B, float tau, int iters,
                             cudaStream_t stream);
 
+/* AdamW on the logits (summary page, "Implementation details": AdamW, learning
+ * rate 1e-3 or 5e-3; the pages fix no betas, epsilon or decay: the usual
+ * defaults are 0.9, 0.999, 1e-8, 0.01).  Decoupled weight decay, bias-corrected
+ * moments, t = the 1-based step count:
+ *   m = b1 m + (1 - b1) g;  v = b2 v + (1 - b2) g^2
+ *   L = L (1 - lr wd) - lr / (1 - b1^t) * m / (sqrt(v / (1 - b2^t)) + eps)     */
+typedef struct {
+  double lr, beta1, beta2, eps, weight_decay;   /* host values; 1 - beta is formed in double */
+} lcp_adamw_params;
+
+/* Per-layer AdamW state: first and second moments, float32 [C_in/B, B, B]
+ * each, zero before the first step, owned by the caller. */
+typedef struct {
+  float* m;
+  float* v;
+} lcp_adamw_state;
+
+/* One AdamW update of n float32 parameters in place (g = dL; n a multiple of 4;
+ * every pointer 16-byte aligned).  t >= 1. */
+LCP_API lcp_status lcp_adamw(float* L, const float* dL, float* m, float* v, long long n,
+                             const lcp_adamw_params* opt, int t, cudaStream_t stream);
+
+/* The training loop of one or more layers ("Implementation details": AdamW,
+ * temperature decreasing linearly from 1 to 0.1): steps s = first, ...,
+ * first + count - 1 of a run of `total` steps, each one lcp_step at
+ * tau_s = tau_start + (tau_end - tau_start) * s / (total - 1) (tau_start when
+ * total = 1) followed by the AdamW update of every layer's L in place (layer.L
+ * is written: the const in lcp_layer does not hold for this call) with
+ * t = s + 1.  hp->tau is ignored.  Enqueues everything on `stream` (capturable
+ * in a CUDA graph); after the call, dL and loss hold step first + count - 1. */
+LCP_API lcp_status lcp_train(const lcp_layer* layers, int nlayers, const lcp_hparams* hp,
+                             const lcp_adamw_params* opt, const lcp_adamw_state* state, int first,
+                             int count, int total, float tau_start, float tau_end, void* ws,
+                             size_t ws_bytes, cudaStream_t stream);
+
 /* Hardening ("Method" 2: P = argmax over permutations of Tr(P^T P_hat), the
  * Hungarian algorithm): for each of `nblocks` B x B blocks of P_hat (float32,
  * [nblocks, B, B]) the permutation maximising sum_i P_hat[i, perm[i]], solved

@@ -38,6 +38,15 @@ class LcpHparams(ctypes.Structure):
                 ("dtype", _c_int), ("flags", ctypes.c_uint)]
 
 
+class LcpAdamwParams(ctypes.Structure):
+    _fields_ = [("lr", ctypes.c_double), ("beta1", ctypes.c_double), ("beta2", ctypes.c_double),
+                ("eps", ctypes.c_double), ("weight_decay", ctypes.c_double)]
+
+
+class LcpAdamwState(ctypes.Structure):
+    _fields_ = [("m", _c_void_p), ("v", _c_void_p)]
+
+
 class LcpError(RuntimeError):
     def __init__(self, status: int, msg: str):
         super().__init__(msg)
@@ -79,6 +88,10 @@ def lib() -> ctypes.CDLL:
         "lcp_grad_gemm": ([_c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_void_p], _c_int),
         "lcp_device_error": ([P(_c_int), _c_int], _c_int),
         "lcp_harden": ([_c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_void_p], _c_int),
+        "lcp_adamw": ([_c_void_p, _c_void_p, _c_void_p, _c_void_p, ctypes.c_longlong, P(LcpAdamwParams), _c_int,
+                       _c_void_p], _c_int),
+        "lcp_train": ([P(LcpLayer), _c_int, P(LcpHparams), P(LcpAdamwParams), P(LcpAdamwState), _c_int, _c_int,
+                       _c_int, _c_float, _c_float, _c_void_p, ctypes.c_size_t, _c_void_p], _c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -174,6 +187,36 @@ class Step:
         arr = (_c_void_p * TIMED_EVENTS)(*[e.cuda_event for e in events])
         check(lib().lcp_step_timed(self.arr, self.n, ctypes.byref(self.hp), self.ws.data_ptr(), self.ws.numel(),
                                    _stream(stream), arr, TIMED_EVENTS))
+
+
+def adamw_params(lr: float = 1e-3, beta1: float = 0.9, beta2: float = 0.999, eps: float = 1e-8,
+                 weight_decay: float = 0.01) -> LcpAdamwParams:
+    return LcpAdamwParams(lr, beta1, beta2, eps, weight_decay)
+
+
+def adamw(L: torch.Tensor, dL: torch.Tensor, m: torch.Tensor, v: torch.Tensor, opt: LcpAdamwParams, t: int) -> None:
+    check(lib().lcp_adamw(_ptr(L, torch.float32, "L"), _ptr(dL, torch.float32, "dL"), _ptr(m, torch.float32, "m"),
+                          _ptr(v, torch.float32, "v"), L.numel(), ctypes.byref(opt), t, _stream(None)))
+
+
+class Trainer:
+    """AdamW training of the logits of prepared layers (lcp_train): ``run(first,
+    count)`` enqueues steps first .. first + count - 1 of a ``total``-step run
+    with the temperature going linearly from ``tau_start`` to ``tau_end``."""
+
+    def __init__(self, step: "Step", opt: LcpAdamwParams, total: int, tau_start: float = 1.0,
+                 tau_end: float = 0.1):
+        self.step, self.opt, self.total = step, opt, total
+        self.tau_start, self.tau_end = tau_start, tau_end
+        self.moments = [(torch.zeros_like(d["L"]), torch.zeros_like(d["L"])) for d in step.layers]
+        self.state = (LcpAdamwState * len(self.moments))(*[LcpAdamwState(m.data_ptr(), v.data_ptr())
+                                                           for m, v in self.moments])
+
+    def run(self, first: int, count: int, stream: Optional[torch.cuda.Stream] = None) -> None:
+        s = self.step
+        check(lib().lcp_train(s.arr, s.n, ctypes.byref(s.hp), ctypes.byref(self.opt), self.state, first, count,
+                              self.total, self.tau_start, self.tau_end, s.ws.data_ptr(), s.ws.numel(),
+                              _stream(stream)))
 
 
 def capture(step: "Step", events: Optional[List[torch.cuda.Event]] = None) -> "torch.cuda.CUDAGraph":

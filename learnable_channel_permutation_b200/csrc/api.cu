@@ -466,6 +466,53 @@ lcp_status lcp_step_timed(const lcp_layer* layers, int nlayers, const lcp_hparam
   return step_impl(layers, nlayers, hp, ws, ws_bytes, stream, events, n_events);
 }
 
+lcp_status lcp_adamw(float* L, const float* dL, float* m, float* v, long long n, const lcp_adamw_params* opt,
+                     int t, cudaStream_t stream) {
+  if (!L || !dL || !m || !v || !opt) return fail(LCP_ERR_NULL, "L, dL, m, v and opt are required");
+  if (n < 0 || n % 4) return fail(LCP_ERR_SHAPE, "n = %lld must be a non-negative multiple of 4", n);
+  if (t < 1) return fail(LCP_ERR_ARG, "t = %d must be >= 1", t);
+  if (!(opt->lr >= 0.0) || !(opt->beta1 >= 0.0 && opt->beta1 < 1.0) || !(opt->beta2 >= 0.0 && opt->beta2 < 1.0) ||
+      !(opt->eps > 0.0) || !(opt->weight_decay >= 0.0) || !std::isfinite(opt->lr))
+    return fail(LCP_ERR_ARG, "AdamW parameters out of range");
+  if (!aligned16(L) || !aligned16(dL) || !aligned16(m) || !aligned16(v))
+    return fail(LCP_ERR_ARG, "every pointer must be 16-byte aligned");
+  if (n == 0) return LCP_OK;
+  LCP_TRY(check_arch());
+  cudaGetLastError();
+  return launch_adamw(L, dL, m, v, n, opt->lr, opt->beta1, opt->beta2, opt->eps, opt->weight_decay, t, stream);
+}
+
+lcp_status lcp_train(const lcp_layer* layers, int nlayers, const lcp_hparams* hp, const lcp_adamw_params* opt,
+                     const lcp_adamw_state* state, int first, int count, int total, float tau_start, float tau_end,
+                     void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (!hp || !opt) return fail(LCP_ERR_NULL, "hp and opt are required");
+  if (nlayers > 0 && !state) return fail(LCP_ERR_NULL, "state is required");
+  if (!(opt->lr >= 0.0) || !(opt->beta1 >= 0.0 && opt->beta1 < 1.0) || !(opt->beta2 >= 0.0 && opt->beta2 < 1.0) ||
+      !(opt->eps > 0.0) || !(opt->weight_decay >= 0.0) || !std::isfinite(opt->lr))
+    return fail(LCP_ERR_ARG, "AdamW parameters out of range");
+  if (total < 1 || first < 0 || count < 0 || first + count > total)
+    return fail(LCP_ERR_ARG, "steps [%d, %d) outside a run of %d", first, first + count, total);
+  if (!(tau_start > 0.f) || !(tau_end > 0.f) || !std::isfinite(tau_start) || !std::isfinite(tau_end))
+    return fail(LCP_ERR_ARG, "temperatures must be positive and finite");
+  for (int i = 0; i < nlayers; ++i) {
+    if (!state[i].m || !state[i].v) return fail(LCP_ERR_NULL, "layer %d: AdamW moments are required", i);
+    if (!aligned16(state[i].m) || !aligned16(state[i].v))
+      return fail(LCP_ERR_ARG, "layer %d: AdamW moments must be 16-byte aligned", i);
+  }
+  lcp_hparams h = *hp;
+  for (int s = first; s < first + count; ++s) {
+    const double frac = total > 1 ? (double)s / (double)(total - 1) : 0.0;
+    h.tau = (float)((double)tau_start + ((double)tau_end - (double)tau_start) * frac);
+    LCP_TRY(step_impl(layers, nlayers, &h, ws, ws_bytes, stream, nullptr, 0));
+    for (int i = 0; i < nlayers; ++i) {
+      const long long n = (long long)layers[i].cin * h.block;
+      LCP_TRY(launch_adamw(const_cast<float*>(layers[i].L), layers[i].dL, state[i].m, state[i].v, n, opt->lr,
+                           opt->beta1, opt->beta2, opt->eps, opt->weight_decay, s + 1, stream));
+    }
+  }
+  return LCP_OK;
+}
+
 lcp_status lcp_sinkhorn_fwd(const float* L, float* P, float* ckpt, int nblocks, int B, float tau,
                             int iters, cudaStream_t stream) {
   if (!L || !P) return fail(LCP_ERR_NULL, "L and P are required");

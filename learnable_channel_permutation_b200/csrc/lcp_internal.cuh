@@ -188,6 +188,10 @@ lcp_status launch_harden(const float* P, int* perm, float* P_hard, __nv_bfloat16
                          __nv_bfloat16* img_pt_lo, __nv_bfloat16* img_p_hi, int nblocks, int B, cudaStream_t st);
 lcp_status harden_error(int* site, int reset);
 
+// AdamW over n float32 values (n a multiple of 4), t the 1-based step.
+lcp_status launch_adamw(float* L, const float* dL, float* m, float* v, long long n, double lr, double beta1,
+                        double beta2, double eps, double weight_decay, int t, cudaStream_t st);
+
 // Device error words of the tensor-core translation units: the first wait
 // site that timed out since the last reset, 0 if none (cleared when `reset`).
 lcp_status tc_error_gemm(int* site, int reset);

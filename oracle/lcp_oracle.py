@@ -24,6 +24,10 @@ Sources (the web pages the method is taken from):
   P = argmax over permutation matrices of Tr(P^T P_hat) (the Hungarian
   algorithm), and the backward pass takes dP/dP_hat = 1 (straight-through).
 
+* [PermLLM] "Implementation details": the logits are trained with AdamW
+  (learning rate 1e-3 or 5e-3), 5 Sinkhorn iterations, the temperature
+  decreasing linearly from 1 to 0.1, block size 64.
+
 Readings where the pages are silent or garbled (each is restated where used):
 
 1. The default forward pass uses the soft P; ``step_hard`` is the hardened
@@ -36,6 +40,10 @@ Readings where the pages are silent or garbled (each is restated where used):
 7. Groups are M consecutive input channels of W' (permuted order).
 8. Cosine denominator max(|y_d| |y_s|, 1e-8).
 9. The loss is the mean over the T tokens (columns of Y).
+10. AdamW is Loshchilov and Hutter's (decoupled weight decay, bias-corrected
+    moments) with the usual defaults beta = (0.9, 0.999), eps = 1e-8, decay
+    0.01 (the pages give only the learning rate); the linear temperature
+    schedule puts 1 at the first step and 0.1 at the last.
 
 Notation follows the pages: W is C_out x C_in, X is the C_in x T matrix of
 calibration activations (the callers store it token-major, [T, C_in]; this
@@ -333,3 +341,43 @@ def step_hard(W: np.ndarray, X_tokens: np.ndarray, logits: np.ndarray, tau: floa
 
 def loss_of_logits(W, X_tokens, logits, tau, n_iters, n, m, mask=None) -> float:
     return forward(W, X_tokens, logits, tau, n_iters, n, m, mask=mask)["loss"]
+
+
+# ---------------------------------------------------------------------------
+# Training loop  ([PermLLM] "Implementation details")
+# ---------------------------------------------------------------------------
+
+def adamw_update(L, g, m, v, t, lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01):
+    """One AdamW step (decoupled decay, bias-corrected moments); returns new (L, m, v)."""
+    L, g, m, v = (np.asarray(a, np.float64) for a in (L, g, m, v))
+    m = beta1 * m + (1.0 - beta1) * g
+    v = beta2 * v + (1.0 - beta2) * g * g
+    m_hat = m / (1.0 - beta1 ** t)
+    v_hat = v / (1.0 - beta2 ** t)
+    L = L * (1.0 - lr * weight_decay) - lr * m_hat / (np.sqrt(v_hat) + eps)
+    return L, m, v
+
+
+def tau_schedule(s: int, total: int, tau_start: float = 1.0, tau_end: float = 0.1) -> float:
+    """Temperature of step s of a total-step run, linear from tau_start to tau_end."""
+    if total <= 1:
+        return float(tau_start)
+    return float(tau_start + (tau_end - tau_start) * s / (total - 1))
+
+
+def train(W, X_tokens, logits, n_iters, n, m, total, steps=None, lr=1e-3, tau_start=1.0, tau_end=0.1,
+          hard=False, **adam):
+    """``steps`` (default all) training steps: forward + backward at tau_s, then
+    AdamW on L.  Returns the logits after the last step, the per-step losses and
+    the last step's dL."""
+    L = np.asarray(logits, np.float64).copy()
+    mom = np.zeros_like(L)
+    vel = np.zeros_like(L)
+    losses, dL = [], None
+    for s in range(total if steps is None else steps):
+        tau = tau_schedule(s, total, tau_start, tau_end)
+        fw = (step_hard if hard else step)(W, X_tokens, L, tau, n_iters, n, m)
+        losses.append(fw["loss"])
+        dL = fw["dL"]
+        L, mom, vel = adamw_update(L, dL, mom, vel, s + 1, lr=lr, **adam)
+    return L, losses, dL

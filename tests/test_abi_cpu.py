@@ -124,3 +124,26 @@ def test_workspace_shrinks_when_the_caller_holds_yd():
     l.Yd = 0x70000000
     st2, n2 = _ws([l], hp)
     assert st == 0 and st2 == 0 and n - n2 >= 512 * 256 * 4
+
+
+def test_adamw_and_train_validation():
+    """Argument checks of lcp_adamw and lcp_train (host side, no launch)."""
+    L = b.lib()
+    opt = b.adamw_params()
+    a = 0x10000000
+    assert L.lcp_adamw(None, a, a, a, 64, ctypes.byref(opt), 1, None) == 1
+    assert L.lcp_adamw(a, a, a, a, 62, ctypes.byref(opt), 1, None) == 2      # not a multiple of 4
+    assert L.lcp_adamw(a, a, a, a, 64, ctypes.byref(opt), 0, None) == 7      # t < 1
+    bad = b.adamw_params(beta2=1.0)
+    assert L.lcp_adamw(a, a, a, a, 64, ctypes.byref(bad), 1, None) == 7
+    assert L.lcp_adamw(a, a, a, a, 0, ctypes.byref(opt), 1, None) == 0       # empty: no-op
+    hp = b.hparams(64, 2, 4, 5, 0.5, b.BF16)
+    arr = (b.LcpLayer * 1)(_layer())
+    st = (b.LcpAdamwState * 1)(b.LcpAdamwState(a, a))
+    call = lambda first, count, total, t0=1.0, t1=0.1, state=st: L.lcp_train(
+        arr, 1, ctypes.byref(hp), ctypes.byref(opt), state, first, count, total, t0, t1, a, 1 << 30, None)
+    assert call(0, 5, 4) == 7            # beyond the run
+    assert call(0, 1, 0) == 7            # empty run
+    assert call(0, 1, 4, t1=0.0) == 7    # temperature must be positive
+    assert call(0, 1, 4, state=None) == 1
+    assert L.lcp_train(arr, 1, ctypes.byref(hp), None, st, 0, 1, 4, 1.0, 0.1, a, 1 << 30, None) == 1

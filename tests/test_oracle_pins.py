@@ -496,3 +496,71 @@ def test_step_hard_straight_through_gradient():
         assert np.isclose((lp - lm) / (2 * eps), dP[b, i, j], rtol=1e-5, atol=1e-9)
     soft = O.step(W, X, L, 0.5, 5, 2, 4)
     assert not np.allclose(soft["dL"], fw["dL"])
+
+
+# --------------------------------------------------------- training loop ---
+
+def test_adamw_first_step_closed_form():
+    """t = 1 from zero moments: m_hat = g and v_hat = g^2, so the step is
+    L (1 - lr wd) - lr g / (|g| + eps)."""
+    rng = np.random.default_rng(30)
+    L = rng.normal(size=50)
+    g = rng.normal(size=50)
+    out, m, v = O.adamw_update(L, g, np.zeros(50), np.zeros(50), 1, lr=5e-3, weight_decay=0.01)
+    assert np.allclose(out, L * (1 - 5e-5) - 5e-3 * g / (np.abs(g) + 1e-8), rtol=1e-14, atol=0)
+    assert np.allclose(m, 0.1 * g) and np.allclose(v, 0.001 * g * g)
+
+
+def test_adamw_constant_gradient_and_pure_decay():
+    """A constant gradient keeps m_hat = g, v_hat = g^2 at every t (bias correction
+    exact): k steps move L by k lr g / (|g| + eps) without decay; a zero gradient
+    only decays, L (1 - lr wd)^k."""
+    g = np.array([0.3, -2.0, 1e-3])
+    L = np.array([1.0, -1.0, 0.5])
+    m = v = np.zeros(3)
+    x = L.copy()
+    for t in range(1, 8):
+        x, m, v = O.adamw_update(x, g, m, v, t, lr=1e-3, weight_decay=0.0)
+    assert np.allclose(x, L - 7 * 1e-3 * g / (np.abs(g) + 1e-8), rtol=1e-12, atol=1e-15)
+    x, m, v = L.copy(), np.zeros(3), np.zeros(3)
+    for t in range(1, 6):
+        x, m, v = O.adamw_update(x, np.zeros(3), m, v, t, lr=1e-2, weight_decay=0.1)
+    assert np.allclose(x, L * (1 - 1e-3) ** 5, rtol=1e-14, atol=0)
+
+
+def test_adamw_matches_torch_adamw():
+    """Five steps on random gradients agree with torch.optim.AdamW (float64, CPU)."""
+    import torch
+    rng = np.random.default_rng(31)
+    L0 = rng.normal(size=(3, 4, 4))
+    grads = [rng.normal(size=(3, 4, 4)) for _ in range(5)]
+    p = torch.nn.Parameter(torch.from_numpy(L0.copy()))
+    opt = torch.optim.AdamW([p], lr=5e-3, betas=(0.9, 0.999), eps=1e-8, weight_decay=0.01)
+    x, m, v = L0.copy(), np.zeros_like(L0), np.zeros_like(L0)
+    for t, gr in enumerate(grads, start=1):
+        p.grad = torch.from_numpy(gr.copy())
+        opt.step()
+        x, m, v = O.adamw_update(x, gr, m, v, t, lr=5e-3)
+    assert np.allclose(x, p.detach().numpy(), rtol=1e-12, atol=1e-14)
+
+
+def test_tau_schedule_endpoints_and_linearity():
+    assert O.tau_schedule(0, 11) == 1.0
+    assert np.isclose(O.tau_schedule(10, 11), 0.1)
+    assert np.allclose(np.diff([O.tau_schedule(s, 11) for s in range(11)]), -0.09)
+    assert O.tau_schedule(0, 1) == 1.0
+
+
+def test_train_loop_lowers_the_loss_and_uses_the_schedule():
+    """Twenty steps on a toy layer with outlier channels lower the loss, and the
+    first step is the plain step at tau = 1."""
+    rng = np.random.default_rng(32)
+    W = rng.normal(0, 0.02, (32, 64))
+    W[:, [3, 40]] *= 10
+    X = rng.normal(0, 1, (96, 64))
+    X[:, [3, 40]] *= 5
+    L0 = rng.normal(0, 1e-3, (2, 32, 32))
+    L, losses, _ = O.train(W, X, L0, 5, 2, 4, total=20, lr=5e-3)
+    assert losses[0] == O.step(W, X, L0, 1.0, 5, 2, 4)["loss"]
+    assert losses[-1] < losses[0]
+    assert not np.allclose(L, L0)
