@@ -40,6 +40,11 @@ Readings where the pages are silent or garbled (each is restated where used):
 7. Groups are M consecutive input channels of W' (permuted order).
 8. Cosine denominator max(|y_d| |y_s|, 1e-8).
 9. The loss is the mean over the T tokens (columns of Y).
+11. Importance scores (the pages name Wanda and RIA as the pruning metrics S
+    of "integration with existing pruning methods" without defining them):
+    the published definitions, Wanda S_ij = |W_ij| ||X_j||_2 and RIA
+    S_ij = (|W_ij| / sum_k |W_kj| + |W_ij| / sum_k |W_ik|) ||X_j||_2^0.5,
+    with X_j the j-th input channel over the calibration tokens.
 10. AdamW is Loshchilov and Hutter's (decoupled weight decay, bias-corrected
     moments) with the usual defaults beta = (0.9, 0.999), eps = 1e-8, decay
     0.01 (the pages give only the learning rate); the linear temperature
@@ -254,15 +259,33 @@ def assignment_value(P: np.ndarray, perm: np.ndarray) -> np.ndarray:
 # One forward + backward step of one layer
 # ---------------------------------------------------------------------------
 
+def importance(W: np.ndarray, X_tokens: np.ndarray, kind: str) -> np.ndarray:
+    """Pruning metric S ([PermLLM] integration with pruning methods; reading 11):
+    "magnitude" |W|, "wanda" |W_ij| ||X_j||, "ria" (|W_ij| / col sum + |W_ij| / row sum) ||X_j||^0.5."""
+    A = np.abs(np.asarray(W, np.float64))
+    xn = np.sqrt(np.sum(np.asarray(X_tokens, np.float64) ** 2, axis=0))      # ||X_j|| over the tokens
+    if kind == "magnitude":
+        return A
+    if kind == "wanda":
+        return A * xn[None, :]
+    if kind == "ria":
+        col = A.sum(axis=0, keepdims=True)       # sum over output rows of column j
+        row = A.sum(axis=1, keepdims=True)       # sum over input columns of row i
+        return (A / col + A / row) * np.sqrt(xn)[None, :]
+    raise ValueError(kind)
+
+
 def forward(W: np.ndarray, X_tokens: np.ndarray, logits: np.ndarray, tau: float, n_iters: int,
             n: int, m: int, mask: Optional[np.ndarray] = None, Wp: Optional[np.ndarray] = None,
-            P: Optional[np.ndarray] = None) -> Dict[str, object]:
+            P: Optional[np.ndarray] = None, score: Optional[np.ndarray] = None) -> Dict[str, object]:
     """Forward pass in the pages' order.
 
     ``X_tokens`` is [T, C_in]; internally X = X_tokens^T (C_in x T).
     ``mask`` / ``Wp`` / ``P`` inject a given mask, permuted weight or soft
     permutation in place of the computed one (used to compare with another
-    implementation on identical intermediate values).
+    implementation on identical intermediate values).  ``score`` is an
+    importance matrix S [C_out, C_in]: the mask is then taken from
+    S_hat = S P_B instead of |W'| ([PermLLM] integration with pruning methods).
     """
     W = np.asarray(W, np.float64)
     Xc = np.asarray(X_tokens, np.float64).T
@@ -272,7 +295,11 @@ def forward(W: np.ndarray, X_tokens: np.ndarray, logits: np.ndarray, tau: float,
     else:
         P = np.asarray(P, np.float64)
     Wp_used = permute_weight(W, P) if Wp is None else np.asarray(Wp)
-    M = nm_mask(Wp_used, n, m) if mask is None else np.asarray(mask, bool)
+    Shat = None if score is None else permute_weight(np.asarray(score, np.float64), P)
+    if mask is not None:
+        M = np.asarray(mask, bool)
+    else:
+        M = nm_mask(Wp_used if Shat is None else Shat, n, m)
     Wp64 = np.asarray(Wp_used, np.float64)
     A = np.where(M, Wp64, 0.0)
     Xp = permute_inputs(P, Xc)
@@ -280,7 +307,7 @@ def forward(W: np.ndarray, X_tokens: np.ndarray, logits: np.ndarray, tau: float,
     Yd = W @ Xc
     loss, cos = cosine_loss(Yd, Ys)
     return dict(P=P, trace=trace, Wp=Wp64, mask=M, A=A, Xc=Xc, Xp=Xp, Yd=Yd, Ys=Ys,
-                loss=loss, cos=cos, W=W)
+                loss=loss, cos=cos, W=W, Shat=Shat)
 
 
 def backward(fw: Dict[str, object], tau: float) -> Dict[str, np.ndarray]:
@@ -310,16 +337,16 @@ def backward(fw: Dict[str, object], tau: float) -> Dict[str, np.ndarray]:
 
 
 def step(W: np.ndarray, X_tokens: np.ndarray, logits: np.ndarray, tau: float, n_iters: int,
-         n: int, m: int, mask: Optional[np.ndarray] = None) -> Dict[str, object]:
+         n: int, m: int, mask: Optional[np.ndarray] = None, score: Optional[np.ndarray] = None) -> Dict[str, object]:
     """Forward and backward of one layer; returns the forward dict plus G, dP, dL."""
-    fw = forward(W, X_tokens, logits, tau, n_iters, n, m, mask=mask)
+    fw = forward(W, X_tokens, logits, tau, n_iters, n, m, mask=mask, score=score)
     fw.update(backward(fw, tau))
     return fw
 
 
 def step_hard(W: np.ndarray, X_tokens: np.ndarray, logits: np.ndarray, tau: float, n_iters: int,
               n: int, m: int, perm: Optional[np.ndarray] = None,
-              mask: Optional[np.ndarray] = None) -> Dict[str, object]:
+              mask: Optional[np.ndarray] = None, score: Optional[np.ndarray] = None) -> Dict[str, object]:
     """Forward with the hardened permutation, backward straight through it.
 
     P_hat = Sinkhorn(L / tau); P = harden(P_hat) (or the given ``perm``, to
@@ -332,7 +359,7 @@ def step_hard(W: np.ndarray, X_tokens: np.ndarray, logits: np.ndarray, tau: floa
     if perm is None:
         perm = harden(P_soft)
     P_hard = perm_matrix(np.asarray(perm))
-    fw = forward(W, X_tokens, logits, tau, n_iters, n, m, mask=mask, P=P_hard)
+    fw = forward(W, X_tokens, logits, tau, n_iters, n, m, mask=mask, P=P_hard, score=score)
     fw.update(backward(fw, tau))
     fw["dL"] = sinkhorn_backward(trace, P_soft, fw["dP"], tau)
     fw["P_soft"], fw["perm"], fw["trace"] = P_soft, np.asarray(perm), trace

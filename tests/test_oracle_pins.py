@@ -564,3 +564,58 @@ def test_train_loop_lowers_the_loss_and_uses_the_schedule():
     assert losses[0] == O.step(W, X, L0, 1.0, 5, 2, 4)["loss"]
     assert losses[-1] < losses[0]
     assert not np.allclose(L, L0)
+
+
+# ------------------------------------------------------ importance scores ---
+
+def test_importance_scores_by_explicit_loops():
+    rng = np.random.default_rng(50)
+    W = rng.normal(size=(5, 8))
+    X = rng.normal(size=(7, 8))
+    S_w = O.importance(W, X, "wanda")
+    S_r = O.importance(W, X, "ria")
+    for i in range(5):
+        for j in range(8):
+            xn = math.sqrt(sum(X[t, j] ** 2 for t in range(7)))
+            col = sum(abs(W[k, j]) for k in range(5))
+            row = sum(abs(W[i, k]) for k in range(8))
+            assert math.isclose(S_w[i, j], abs(W[i, j]) * xn, rel_tol=1e-12)
+            assert math.isclose(S_r[i, j], (abs(W[i, j]) / col + abs(W[i, j]) / row) * math.sqrt(xn), rel_tol=1e-12)
+
+
+def test_score_mask_maximises_each_group_sum():
+    """The mask keeps, in every group of M, the N-subset with the largest sum of S_hat
+    (argmax over masks of sum (M . S_hat) for each group), checked by enumeration."""
+    rng = np.random.default_rng(51)
+    W = rng.normal(size=(6, 16))
+    X = rng.normal(size=(9, 16))
+    L = rng.normal(0, 0.5, (2, 8, 8))
+    S = O.importance(W, X, "wanda")
+    fw = O.forward(W, X, L, 0.7, 5, 2, 4, score=S)
+    Sh = fw["Shat"]
+    for i in range(6):
+        for g in range(4):
+            vals = Sh[i, 4 * g:4 * g + 4]
+            best = max(sum(vals[list(c)]) for c in itertools.combinations(range(4), 2))
+            assert np.isclose(vals[fw["mask"][i, 4 * g:4 * g + 4]].sum(), best)
+
+
+def test_magnitude_score_with_a_hard_permutation_is_the_plain_mask():
+    """S = |W| and P a permutation: S_hat = |W P| = |W'|, so the masks agree (the
+    two scores differ only for soft P)."""
+    rng = np.random.default_rng(52)
+    W = rng.normal(size=(12, 32))
+    X = rng.normal(size=(10, 32))
+    pis = np.stack([rng.permutation(16) for _ in range(2)])
+    P = O.perm_matrix(pis)
+    S = O.importance(W, X, "magnitude")
+    a = O.forward(W, X, None, 1.0, 5, 2, 4, P=P, score=S)["mask"]
+    b_ = O.forward(W, X, None, 1.0, 5, 2, 4, P=P)["mask"]
+    assert np.array_equal(a, b_)
+
+
+def test_wanda_with_equal_channel_norms_is_magnitude():
+    rng = np.random.default_rng(53)
+    W = rng.normal(size=(8, 16))
+    X = np.ones((4, 16)) * np.array([1, -1, 1, -1])[:, None]     # every ||X_j|| = 2
+    assert np.allclose(O.importance(W, X, "wanda"), 2 * np.abs(W))
