@@ -434,6 +434,7 @@ def extras(args, b, synth, wl, li, layer, step, flush, pk, dev):
     - cached_dense: the step with LCP_FLAG_CACHED_DENSE (Y_d read from layer.Yd,
       written once by an uncached step), same timing protocol as the headline;
     - hard_step: the step with LCP_FLAG_HARD, and the hardening kernel alone;
+    - score_step: the step with LCP_FLAG_SCORE and Wanda scores;
     - train: steps of lcp_train (step + AdamW on L, temperature schedule);
     - nm_mask: the standalone mask kernel on a bf16 W' of the layer's shape,
       against the measured HBM copy bandwidth (bytes: 2 read + 1/8 written per element);
@@ -490,6 +491,17 @@ def extras(args, b, synth, wl, li, layer, step, flush, pk, dev):
                         "note": "LCP_FLAG_HARD: the forward pass uses the per-block maximum-weight "
                                 "assignment of the Sinkhorn output (one warp per block), the backward "
                                 "pass is straight-through; not the headline"}
+
+    # mask from Wanda scores (LCP_FLAG_SCORE): S computed once, S_hat = S P_B ranked each step
+    layer["S"] = b.score(layer["W"], layer["X"], b.SCORE_WANDA)
+    sc = b.Step([layer], wl.block, wl.n, wl.m, wl.iters, wl.tau, flags=b.FLAG_SCORE, workspace=step.ws)
+    g = b.capture(sc)
+    ms = timed(g.replay, K)
+    del g
+    layer.pop("S")
+    out["score_step"] = {"value": 1e3 / ms, "unit": UNIT, "ms_per_step": ms, "steps": K, "score": "wanda",
+                         "note": "LCP_FLAG_SCORE: the mask ranks S_hat = S P_B (one permute pass over S for "
+                                 "the mask, one over W with that mask); not the headline"}
 
     # training steps: lcp_step at the scheduled temperature + AdamW on L (lcp_train)
     tr_step = b.Step([layer], wl.block, wl.n, wl.m, wl.iters, wl.tau, workspace=step.ws)

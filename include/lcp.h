@@ -76,6 +76,11 @@ typedef enum { LCP_F32 = 0, LCP_BF16 = 1 } lcp_dtype;
                                        maximising Tr(P^T P_hat) (lcp_harden); the backward
                                        pass is straight-through, dP_hat = dP.  layer.P
                                        still returns the soft P_hat                    */
+#define LCP_FLAG_SCORE        0x10u /* take the N:M mask from S_hat = S P_B, S = layer.S an
+                                       importance matrix ("integration with pruning
+                                       methods"; see lcp_score), instead of |W'|.  With
+                                       LCP_FLAG_WRITE_WPRIME, layer.Wp receives S_hat (the
+                                       matrix the mask ranks).  Tensor-core path: B <= 64 */
 #define LCP_FLAG_CACHED_DENSE 0x4u  /* read the dense output Y_d = X W^T from layer.Yd
                                        instead of computing it: the dense output depends
                                        on neither L nor P, so a loop over one calibration
@@ -107,6 +112,7 @@ typedef struct {
                        non-NULL, an output the step fills                                */
   int32_t* perm;    /* out [C_in/B, B] optional: with LCP_FLAG_HARD, perm[b][i] = the
                        column of block b that row i is sent to                          */
+  const void* S;    /* in  [C_out, C_in] dtype importance scores (with LCP_FLAG_SCORE)  */
 } lcp_layer;
 
 /* Bytes of workspace lcp_step needs for these layers (the layers run one after
@@ -186,6 +192,21 @@ LCP_API lcp_status lcp_train(const lcp_layer* layers, int nlayers, const lcp_hpa
                              const lcp_adamw_params* opt, const lcp_adamw_state* state, int first,
                              int count, int total, float tau_start, float tau_end, void* ws,
                              size_t ws_bytes, cudaStream_t stream);
+
+/* Importance scores of W for the mask ("integration with existing pruning
+ * methods"; the pages name Wanda and RIA without defining them, so their
+ * published definitions are used), with ||X_j|| the 2-norm of input channel j
+ * over the T tokens:
+ *   LCP_SCORE_MAGNITUDE  S_ij = |W_ij|
+ *   LCP_SCORE_WANDA      S_ij = |W_ij| ||X_j||
+ *   LCP_SCORE_RIA        S_ij = (|W_ij| / sum_k |W_kj| + |W_ij| / sum_k |W_ik|) ||X_j||^(1/2)
+ * W [C_out, C_in], X [T, C_in] and S [C_out, C_in] in `dtype` (S rounded to it);
+ * stats: float32 scratch of 2 C_in + C_out values owned by the caller. */
+#define LCP_SCORE_MAGNITUDE 0
+#define LCP_SCORE_WANDA     1
+#define LCP_SCORE_RIA       2
+LCP_API lcp_status lcp_score(const void* W, const void* X, void* S, float* stats, int cout, int cin, int tokens,
+                             int kind, lcp_dtype dtype, cudaStream_t stream);
 
 /* Hardening ("Method" 2: P = argmax over permutations of Tr(P^T P_hat), the
  * Hungarian algorithm): for each of `nblocks` B x B blocks of P_hat (float32,

@@ -21,6 +21,8 @@ FLAG_WRITE_WPRIME = 0x1
 FLAG_SIMT = 0x2
 FLAG_CACHED_DENSE = 0x4
 FLAG_HARD = 0x8
+FLAG_SCORE = 0x10
+SCORE_MAGNITUDE, SCORE_WANDA, SCORE_RIA = 0, 1, 2
 TIMED_EVENTS = 8
 STAGES = ("sinkhorn_fwd", "permute_mask", "calib_gemm", "loss", "bwd_gemm", "block_bwd", "sinkhorn_bwd")
 
@@ -30,7 +32,8 @@ _c_void_p, _c_int, _c_float = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
 class LcpLayer(ctypes.Structure):
     _fields_ = [("W", _c_void_p), ("X", _c_void_p), ("L", _c_void_p), ("P", _c_void_p),
                 ("dL", _c_void_p), ("loss", _c_void_p), ("mask", _c_void_p), ("Wp", _c_void_p),
-                ("cout", _c_int), ("cin", _c_int), ("tokens", _c_int), ("Yd", _c_void_p), ("perm", _c_void_p)]
+                ("cout", _c_int), ("cin", _c_int), ("tokens", _c_int), ("Yd", _c_void_p), ("perm", _c_void_p),
+                ("S", _c_void_p)]
 
 
 class LcpHparams(ctypes.Structure):
@@ -88,6 +91,8 @@ def lib() -> ctypes.CDLL:
         "lcp_grad_gemm": ([_c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_void_p], _c_int),
         "lcp_device_error": ([P(_c_int), _c_int], _c_int),
         "lcp_harden": ([_c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_void_p], _c_int),
+        "lcp_score": ([_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_int, _c_int,
+                       _c_void_p], _c_int),
         "lcp_adamw": ([_c_void_p, _c_void_p, _c_void_p, _c_void_p, ctypes.c_longlong, P(LcpAdamwParams), _c_int,
                        _c_void_p], _c_int),
         "lcp_train": ([P(LcpLayer), _c_int, P(LcpHparams), P(LcpAdamwParams), P(LcpAdamwState), _c_int, _c_int,
@@ -146,7 +151,8 @@ def make_layer(d: Dict[str, torch.Tensor], wdtype) -> LcpLayer:
                     _ptr(d["P"], torch.float32, "P"), _ptr(d["dL"], torch.float32, "dL"),
                     _ptr(d["loss"], torch.float32, "loss"), _ptr(d.get("mask"), torch.int32, "mask"),
                     _ptr(d.get("Wp"), torch.float32, "Wp"), cout, cin, tokens,
-                    _ptr(d.get("Yd"), torch.float32, "Yd"), _ptr(d.get("perm"), torch.int32, "perm"))
+                    _ptr(d.get("Yd"), torch.float32, "Yd"), _ptr(d.get("perm"), torch.int32, "perm"),
+                    _ptr(d.get("S"), wdtype, "S"))
 
 
 class Step:
@@ -277,6 +283,16 @@ def permute_weight(W: torch.Tensor, P: torch.Tensor, Wp: torch.Tensor) -> None:
     cout, cin = W.shape
     check(lib().lcp_permute_weight(_ptr(W, None, "W"), _ptr(P, torch.float32, "P"), _ptr(Wp, torch.float32, "Wp"),
                                    cout, cin, P.shape[1], _dt(W), _stream(None)))
+
+
+def score(W: torch.Tensor, X: torch.Tensor, kind: int) -> torch.Tensor:
+    """Importance scores S of W (LCP_SCORE_*), in W's dtype."""
+    cout, cin = W.shape
+    S = torch.empty_like(W)
+    stats = torch.empty(2 * cin + cout, dtype=torch.float32, device=W.device)
+    check(lib().lcp_score(_ptr(W, None, "W"), _ptr(X, W.dtype, "X"), _ptr(S, W.dtype, "S"),
+                          _ptr(stats, torch.float32, "stats"), cout, cin, X.shape[0], kind, _dt(W), _stream(None)))
+    return S
 
 
 def harden(P: torch.Tensor, perm: torch.Tensor, P_hard: Optional[torch.Tensor] = None) -> None:

@@ -120,7 +120,7 @@ lcp_status check_hparams(const lcp_hparams* hp) {
     return fail(LCP_ERR_ARG, "iters = %d is not in [1, 1000]", hp->iters);
   if (!(hp->tau > 0.f) || !std::isfinite(hp->tau))
     return fail(LCP_ERR_ARG, "tau must be positive and finite");
-  if (hp->flags & ~(LCP_FLAG_WRITE_WPRIME | LCP_FLAG_SIMT | LCP_FLAG_CACHED_DENSE | LCP_FLAG_HARD))
+  if (hp->flags & ~(LCP_FLAG_WRITE_WPRIME | LCP_FLAG_SIMT | LCP_FLAG_CACHED_DENSE | LCP_FLAG_HARD | LCP_FLAG_SCORE))
     return fail(LCP_ERR_ARG, "unknown flags 0x%x", hp->flags);
   return LCP_OK;
 }
@@ -136,6 +136,11 @@ lcp_status check_layer(const lcp_layer& l, const lcp_hparams& hp, int idx) {
     return fail(LCP_ERR_NULL, "layer %d: LCP_FLAG_WRITE_WPRIME needs layer.Wp", idx);
   if ((hp.flags & LCP_FLAG_CACHED_DENSE) && !l.Yd)
     return fail(LCP_ERR_NULL, "layer %d: LCP_FLAG_CACHED_DENSE needs layer.Yd", idx);
+  if ((hp.flags & LCP_FLAG_SCORE) && !l.S)
+    return fail(LCP_ERR_NULL, "layer %d: LCP_FLAG_SCORE needs layer.S", idx);
+  if ((hp.flags & LCP_FLAG_SCORE) && use_tc(hp) && hp.block > 64)
+    return fail(LCP_ERR_ARG, "layer %d: LCP_FLAG_SCORE on the tensor-core path takes B <= 64 "
+                "(B = %d: add LCP_FLAG_SIMT)", idx, hp.block);
   if (l.cout < 8 || l.cout % 8 || l.cout > kMaxDim)
     return fail(LCP_ERR_SHAPE, "layer %d: C_out = %d must be a positive multiple of 8", idx, l.cout);
   if (l.cin < hp.block || l.cin % hp.block || l.cin % 32 || l.cin > kMaxDim)
@@ -147,7 +152,7 @@ lcp_status check_layer(const lcp_layer& l, const lcp_hparams& hp, int idx) {
     return fail(LCP_ERR_SHAPE,
                 "layer %d: C_in = %d must be a multiple of 64 on the tensor-core path "
                 "(LCP_FLAG_SIMT accepts multiples of 32)", idx, l.cin);
-  const void* ptrs[] = {l.W, l.X, l.L, l.P, l.dL, l.mask, l.Wp, l.Yd, l.perm};
+  const void* ptrs[] = {l.W, l.X, l.L, l.P, l.dL, l.mask, l.Wp, l.Yd, l.perm, l.S};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return fail(LCP_ERR_ARG, "layer %d: every pointer must be 16-byte aligned", idx);
   return LCP_OK;
@@ -157,7 +162,7 @@ lcp_status check_layer(const lcp_layer& l, const lcp_hparams& hp, int idx) {
 size_t esize(lcp_dtype d) { return d == LCP_F32 ? 4 : 2; }
 
 struct Plan {
-  size_t ckpt, img0, img1, img2, mask, wp, amask, at, yd, ys, stats, counter, g, dat, da, dp, perm, phard;
+  size_t ckpt, img0, img1, img2, mask, wp, amask, at, yd, ys, stats, counter, g, dat, da, dp, perm, phard, shat;
   size_t total;
   int splits;
 };
@@ -197,6 +202,7 @@ Plan make_plan(const lcp_layer& l, const lcp_hparams& hp) {
   const bool hard = (hp.flags & LCP_FLAG_HARD) != 0;
   p.perm = take(hard && !l.perm ? nb * B * 4 : 0);
   p.phard = take(hard && simt_bwd ? nb * B * B * 4 : 0);   // the CUDA-core products read P_hard as float32
+  p.shat = take((hp.flags & LCP_FLAG_SCORE) && !tc ? oc * ic * 4 : 0);   // S_hat of the CUDA-core path
   p.total = off;
   return p;
 }
@@ -243,7 +249,10 @@ lcp_status layer_simt(const lcp_layer& l, const lcp_hparams& hp, const Plan& p, 
   const lcp_dtype dt = hp.dtype;
   float* ckpt = at<float>(ws, p.ckpt);
   uint32_t* mask = l.mask ? l.mask : at<uint32_t>(ws, p.mask);
-  float* Wp = (hp.flags & LCP_FLAG_WRITE_WPRIME) ? l.Wp : at<float>(ws, p.wp);
+  const bool score = (hp.flags & LCP_FLAG_SCORE) != 0, write_wp = (hp.flags & LCP_FLAG_WRITE_WPRIME) != 0;
+  // W' (float32); with scores the ranked S_hat goes to layer.Wp when requested
+  float* Wp = (write_wp && !score) ? l.Wp : at<float>(ws, p.wp);
+  float* Shat = score ? (write_wp ? l.Wp : at<float>(ws, p.shat)) : nullptr;
   float* Am = at<float>(ws, p.amask);
   void* At = at<void>(ws, p.at);
   float* Yd = l.Yd ? l.Yd : at<float>(ws, p.yd);
@@ -270,7 +279,13 @@ lcp_status layer_simt(const lcp_layer& l, const lcp_hparams& hp, const Plan& p, 
   // W'_b = W_b P_b
   LCP_TRY(launch_simt_gemm({l.cout, B, B, nb, l.W, B, ic, 1, Pu, BB, B, 1, Wp, B, ic, 1, 1.f, 0.f},
                            dt, LCP_F32, LCP_F32, st));
-  LCP_TRY(launch_nm_mask(Wp, mask, l.cout, l.cin, hp.n, hp.m, LCP_F32, st));
+  if (score) {   // S_hat_b = S_b P_b, ranked in place of |W'|
+    LCP_TRY(launch_simt_gemm({l.cout, B, B, nb, l.S, B, ic, 1, Pu, BB, B, 1, Shat, B, ic, 1, 1.f, 0.f},
+                             dt, LCP_F32, LCP_F32, st));
+    LCP_TRY(launch_nm_mask(Shat, mask, l.cout, l.cin, hp.n, hp.m, LCP_F32, st));
+  } else {
+    LCP_TRY(launch_nm_mask(Wp, mask, l.cout, l.cin, hp.n, hp.m, LCP_F32, st));
+  }
   LCP_TRY(launch_apply_mask(Wp, mask, Am, l.cout, l.cin, st));
   // At_b = A_b P_b^T
   LCP_TRY(launch_simt_gemm({l.cout, B, B, nb, Am, B, ic, 1, Pu, BB, 1, B, At, B, ic, 1, 1.f, 0.f},
@@ -309,7 +324,8 @@ constexpr int kTcLaunches = 6;
 constexpr int kTcLaunchesSimtBwd = 11;   // B = 256: block backward on CUDA cores (6 launches)
 
 int launches_per_layer(const lcp_layer& l, const lcp_hparams& hp) {
-  const int loss = loss_launches(l.cout) + ((hp.flags & LCP_FLAG_HARD) ? 1 : 0);
+  const int loss = loss_launches(l.cout) + ((hp.flags & LCP_FLAG_HARD) ? 1 : 0) +
+                   ((hp.flags & LCP_FLAG_SCORE) ? 1 : 0);   // hardening; the score GEMM or score-mask pass
   if (!use_tc(hp)) return kSimtLaunches - ((hp.flags & LCP_FLAG_CACHED_DENSE) ? 1 : 0) + loss;
   return (block_bwd_tc_supported(hp.block) ? kTcLaunches : kTcLaunchesSimtBwd) + loss;
 }
@@ -349,7 +365,15 @@ lcp_status layer_tc(const lcp_layer& l, const lcp_hparams& hp, const Plan& p, vo
                           pt_hi, pt_lo, p_hi, nb, B, st));
   }
   LCP_TRY(record(ev, 1, st));
-  LCP_TRY(launch_permute_mask_tc(W, pt_hi, pt_lo, p_hi, mask, At, Wp, l.cout, l.cin, B, hp.n, hp.m, st));
+  if (hp.flags & LCP_FLAG_SCORE) {
+    // mask from S_hat = S P_B (exported to layer.Wp when requested), then A and At from W'
+    LCP_TRY(launch_score_mask_tc(static_cast<const __nv_bfloat16*>(l.S), pt_hi, pt_lo, p_hi, mask, Wp, l.cout, l.cin,
+                                 B, hp.n, hp.m, st));
+    LCP_TRY(launch_permute_mask_tc(W, pt_hi, pt_lo, p_hi, mask, At, nullptr, l.cout, l.cin, B, hp.n, hp.m, true,
+                                   st));
+  } else {
+    LCP_TRY(launch_permute_mask_tc(W, pt_hi, pt_lo, p_hi, mask, At, Wp, l.cout, l.cin, B, hp.n, hp.m, false, st));
+  }
   LCP_TRY(record(ev, 2, st));
   if (cached)   // Y_s = X At^T alone (one problem)
     LCP_TRY(launch_calib_gemm_tc(X, At, nullptr, Ys, nullptr, l.tokens, l.cout, l.cin, st));
@@ -557,6 +581,20 @@ lcp_status lcp_permute_weight(const void* W, const float* P, float* Wp, int cout
   const long long ic = cin, BB = (long long)B * B;
   return launch_simt_gemm({cout, B, B, cin / B, W, B, ic, 1, P, BB, B, 1, Wp, B, ic, 1, 1.f, 0.f},
                           dtype, LCP_F32, LCP_F32, stream);
+}
+
+lcp_status lcp_score(const void* W, const void* X, void* S, float* stats, int cout, int cin, int tokens, int kind,
+                     lcp_dtype dtype, cudaStream_t stream) {
+  if (!W || !X || !S || !stats) return fail(LCP_ERR_NULL, "W, X, S and stats are required");
+  if (dtype != LCP_F32 && dtype != LCP_BF16) return fail(LCP_ERR_DTYPE, "unknown dtype %d", (int)dtype);
+  if (kind != LCP_SCORE_MAGNITUDE && kind != LCP_SCORE_WANDA && kind != LCP_SCORE_RIA)
+    return fail(LCP_ERR_ARG, "unknown score kind %d", kind);
+  if (cout < 0 || cin < 0 || tokens < 1 || cout > kMaxDim || cin > kMaxDim || tokens > kMaxDim)
+    return fail(LCP_ERR_SHAPE, "C_out = %d, C_in = %d, T = %d", cout, cin, tokens);
+  if (cout == 0 || cin == 0) return LCP_OK;
+  LCP_TRY(check_arch());
+  cudaGetLastError();
+  return launch_score(W, X, S, stats, cout, cin, tokens, kind, dtype, stream);
 }
 
 lcp_status lcp_harden(const float* P_hat, int32_t* perm, float* P_hard, int nblocks, int B, cudaStream_t stream) {

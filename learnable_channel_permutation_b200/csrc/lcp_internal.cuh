@@ -164,10 +164,16 @@ lcp_status launch_loss_fused(const float* Yd, const float* Ys, float* stats, voi
                              float* loss, unsigned* counter, int cout, int tokens, cudaStream_t st);
 
 // Tensor-core (tcgen05) kernels, bf16 operands, float32 accumulation.
+// given_mask (B <= 64): the mask is read from `mask` instead of computed.
 lcp_status launch_permute_mask_tc(const __nv_bfloat16* W, const __nv_bfloat16* img_pt_hi,
                                   const __nv_bfloat16* img_pt_lo, const __nv_bfloat16* img_p_hi,
                                   uint32_t* mask, __nv_bfloat16* At, float* Wp_out, int cout,
-                                  int cin, int B, int n, int m, cudaStream_t st);
+                                  int cin, int B, int n, int m, bool given_mask, cudaStream_t st);
+// B <= 64: the N:M mask of S_hat = S P_B (an importance score permuted like W)
+// into `mask`; Shat_out (optional) receives S_hat as float32.
+lcp_status launch_score_mask_tc(const __nv_bfloat16* S, const __nv_bfloat16* img_pt_hi,
+                                const __nv_bfloat16* img_pt_lo, const __nv_bfloat16* img_p_hi, uint32_t* mask,
+                                float* Shat_out, int cout, int cin, int B, int n, int m, cudaStream_t st);
 lcp_status launch_calib_gemm_tc(const __nv_bfloat16* X, const __nv_bfloat16* W,
                                 const __nv_bfloat16* At, float* Yd, float* Ys, int tokens,
                                 int cout, int cin, cudaStream_t st);
@@ -187,6 +193,10 @@ bool block_bwd_tc_supported(int B);   // B <= 128 (TMEM/smem budget of the fused
 lcp_status launch_harden(const float* P, int* perm, float* P_hard, __nv_bfloat16* img_pt_hi,
                          __nv_bfloat16* img_pt_lo, __nv_bfloat16* img_p_hi, int nblocks, int B, cudaStream_t st);
 lcp_status harden_error(int* site, int reset);
+
+// Importance scores (LCP_SCORE_*) of W into S; stats: 2 cin + cout floats.
+lcp_status launch_score(const void* W, const void* X, void* S, float* stats, int cout, int cin, int tokens, int kind,
+                        lcp_dtype dt, cudaStream_t st);
 
 // AdamW over n float32 values (n a multiple of 4), t the 1-based step.
 lcp_status launch_adamw(float* L, const float* dL, float* m, float* v, long long n, double lr, double beta1,

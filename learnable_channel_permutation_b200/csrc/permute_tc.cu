@@ -233,7 +233,11 @@ struct TileIter {
   }
 };
 
-template <int MGROUP>
+// MODE: kFull (W' -> mask, A, At), kMaskOnly (the ranked matrix -> mask only:
+// no A, no At) or kGivenMask (W' -> A and At with the mask read from `mask`).
+constexpr int kFull = 0, kMaskOnly = 1, kGivenMask = 2;
+
+template <int MGROUP, int MODE>
 __global__ void __launch_bounds__(PwCfg::THREADS, 1)
 permute_mask_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmPth,
                        const __grid_constant__ CUtensorMap tmPtl, const __grid_constant__ CUtensorMap tmPh,
@@ -384,10 +388,18 @@ permute_mask_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
         i1.next();
         return true;
       };
-      // W' runs two tiles ahead of At, so the mask warps find W' ready
       bool ok = true;
-      for (int k = 0; k < 2 && k < nloc && ok; ++k) ok = mma1(k);
-      for (int k = 0; k < nloc && ok; ++k, i2.next()) {
+      if constexpr (MODE == kMaskOnly) {
+        for (int k = 0; k < nloc && ok; ++k) {
+          const int jt = i1.t - t_first;
+          const bool last_of_t = k + 1 == nloc || i1.rt == nrt - 1;
+          ok = mma1(k);
+          if (ok && last_of_t) mma_commit(bar(PFREE + (jt & 1)));   // slot reusable
+        }
+      }
+      // W' runs two tiles ahead of At, so the mask warps find W' ready
+      for (int k = 0; k < 2 && k < nloc && ok && MODE != kMaskOnly; ++k) ok = mma1(k);
+      for (int k = 0; k < nloc && ok && MODE != kMaskOnly; ++k, i2.next()) {
         const int b = k % NB, jt = i2.t - t_first;
         const uint32_t ub = (uint32_t)(k / NB) & 1u;
         if (k + 2 < nloc && !mma1(k + 2)) break;
@@ -435,17 +447,24 @@ permute_mask_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
           o[qq] = make_float4(__uint_as_float(v[4 * qq]), __uint_as_float(v[4 * qq + 1]),
                               __uint_as_float(v[4 * qq + 2]), __uint_as_float(v[4 * qq + 3]));
       }
-      // keep bits; v becomes A = M.W'
-      const uint32_t w = MGROUP == 4 ? nm4_keep<NV>(v, n) : nm_bits<MGROUP, NV>(v, n);
-#pragma unroll
-      for (int x = 0; x < NV; ++x) v[x] = ((w >> x) & 1u) ? v[x] : 0u;
-      if (grow < cout) {
-        if constexpr (NV == 32) {
-          mask[(size_t)grow * words + 2 * it.t + h] = w;
-        } else {
-          reinterpret_cast<uint16_t*>(mask)[((size_t)grow * words + 2 * it.t) * 2 + h] = (uint16_t)w;
+      // keep bits (computed, or given); v becomes A = M.W'
+      uint32_t w;
+      if constexpr (MODE == kGivenMask) {
+        static_assert(NV == 32, "one mask word per thread");
+        w = grow < cout ? mask[(size_t)grow * words + 2 * it.t + h] : 0u;
+      } else {
+        w = MGROUP == 4 ? nm4_keep<NV>(v, n) : nm_bits<MGROUP, NV>(v, n);
+        if (grow < cout) {
+          if constexpr (NV == 32) {
+            mask[(size_t)grow * words + 2 * it.t + h] = w;
+          } else {
+            reinterpret_cast<uint16_t*>(mask)[((size_t)grow * words + 2 * it.t) * 2 + h] = (uint16_t)w;
+          }
         }
       }
+      if constexpr (MODE == kMaskOnly) continue;
+#pragma unroll
+      for (int x = 0; x < NV; ++x) v[x] = ((w >> x) & 1u) ? v[x] : 0u;
       uint8_t* sa = sA + (k % NA) * C::A_BYTES;
 #pragma unroll
       for (int c8 = 0; c8 < NV / 8; ++c8)
@@ -467,7 +486,7 @@ permute_mask_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     const bool storer = warp == C::COPY0;
     TileIter it(first, nrt);
-    for (int j = 0; j < nloc; ++j, it.next()) {
+    for (int j = 0; j < nloc && MODE != kMaskOnly; ++j, it.next()) {
       const int b = j % NB, s = j & 1;
       const uint32_t us = (uint32_t)(j >> 1) & 1u;
       if (!wait_all(ATF + b, (uint32_t)(j / NB) & 1u, 68)) break;
@@ -757,10 +776,29 @@ lcp_status permute_mask_bc(const CUtensorMap& mW, const CUtensorMap& mPth, const
 
 lcp_status tc_error_permute(int* site, int reset) { return read_tc_error(site, reset); }
 
+lcp_status launch_score_mask_tc(const __nv_bfloat16* S, const __nv_bfloat16* img_pt_hi,
+                                const __nv_bfloat16* img_pt_lo, const __nv_bfloat16* img_p_hi, uint32_t* mask,
+                                float* Shat_out, int cout, int cin, int B, int n, int m, cudaStream_t st) {
+  if (B > 64) return fail(LCP_ERR_SHAPE, "score_mask_tc: B = %d (the tensor-core score path takes B <= 64)", B);
+  CUtensorMap mS, mPth, mPtl, mPh;
+  TC_TRY(make_map(&mS, S, cin, cout, 64, 128, "score_mask S"));
+  TC_TRY(make_map(&mPth, img_pt_hi, 64, cin, 64, 64, "score_mask Pt_hi"));
+  TC_TRY(make_map(&mPtl, img_pt_lo, 64, cin, 64, 64, "score_mask Pt_lo"));
+  TC_TRY(make_map(&mPh, img_p_hi, 64, cin, 64, 64, "score_mask P_hi"));
+  using C = PwCfg;
+  auto k = (m == 4) ? permute_mask_ws_kernel<4, kMaskOnly> : permute_mask_ws_kernel<8, kMaskOnly>;
+  TC_TRY(set_smem(k, C::SMEM, "score_mask_tc"));
+  const int tiles = cdiv(cout, 128) * (cin / 64);
+  const int grid = tiles < num_sms() ? tiles : num_sms();
+  // no At in this mode: the At map is never used (the S map stands in)
+  return launch_kernel(k, dim3(grid), dim3(C::THREADS), C::SMEM, st, 1, true, "score_mask_tc", mS, mPth, mPtl, mPh,
+                       mS, mask, Shat_out, cout, cin, n);
+}
+
 lcp_status launch_permute_mask_tc(const __nv_bfloat16* W, const __nv_bfloat16* img_pt_hi,
                                   const __nv_bfloat16* img_pt_lo, const __nv_bfloat16* img_p_hi, uint32_t* mask,
                                   __nv_bfloat16* At, float* Wp_out, int cout, int cin, int B, int n, int m,
-                                  cudaStream_t st) {
+                                  bool given_mask, cudaStream_t st) {
   const int BC = B < 64 ? 64 : B;
   CUtensorMap mW, mPth, mPtl, mPh;
   TC_TRY(make_map(&mW, W, cin, cout, 64, 128, "permute_mask W"));
@@ -771,13 +809,15 @@ lcp_status launch_permute_mask_tc(const __nv_bfloat16* W, const __nv_bfloat16* i
     CUtensorMap mAt;
     TC_TRY(make_map(&mAt, At, cin, cout, 64, 128, "permute_mask At"));
     using C = PwCfg;
-    auto k = (m == 4) ? permute_mask_ws_kernel<4> : permute_mask_ws_kernel<8>;
+    auto k = (m == 4) ? (given_mask ? permute_mask_ws_kernel<4, kGivenMask> : permute_mask_ws_kernel<4, kFull>)
+                      : (given_mask ? permute_mask_ws_kernel<8, kGivenMask> : permute_mask_ws_kernel<8, kFull>);
     TC_TRY(set_smem(k, C::SMEM, "permute_mask_tc"));
     const int tiles = cdiv(cout, 128) * (cin / 64);
     const int grid = tiles < num_sms() ? tiles : num_sms();
     return launch_kernel(k, dim3(grid), dim3(C::THREADS), C::SMEM, st, 1, true, "permute_mask_tc", mW, mPth, mPtl,
                          mPh, mAt, mask, Wp_out, cout, cin, n);
   }
+  if (given_mask) return fail(LCP_ERR_SHAPE, "permute_mask_tc: a given mask needs B <= 64 (B = %d)", B);
   if (m == 4) {
     if (BC == 128) return permute_mask2_bc<128, 4>(mW, mPth, mPtl, mPh, mask, At, Wp_out, cout, cin, n, st);
     return permute_mask_bc<256, 4>(mW, mPth, mPtl, mPh, mask, At, Wp_out, cout, cin, n, st);

@@ -76,6 +76,9 @@ def test_workspace_size_for_valid_layers():
     (lambda l, h: setattr(h, "flags", b.FLAG_WRITE_WPRIME), 1),  # needs layer.Wp
     (lambda l, h: setattr(h, "flags", b.FLAG_CACHED_DENSE), 1),  # needs layer.Yd
     (lambda l, h: (setattr(h, "flags", b.FLAG_CACHED_DENSE), setattr(l, "Yd", 0x10000004)), 7),  # misaligned
+    (lambda l, h: setattr(h, "flags", b.FLAG_SCORE), 1),          # needs layer.S
+    (lambda l, h: (setattr(h, "flags", b.FLAG_SCORE), setattr(l, "S", 0x30000000), setattr(h, "block", 128),
+                   setattr(l, "cin", 256)), 7),                     # tensor-core score path: B <= 64
 ])
 def test_host_validation_codes(mut, code):
     l = _layer()
