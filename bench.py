@@ -436,6 +436,8 @@ def extras(args, b, synth, wl, li, layer, step, flush, pk, dev):
     - hard_step: the step with LCP_FLAG_HARD, and the hardening kernel alone;
     - score_step: the step with LCP_FLAG_SCORE and Wanda scores;
     - train: steps of lcp_train (step + AdamW on L, temperature schedule);
+    - cublas_same_products: the two dense products of the step through torch.mm
+      on the same shapes (context for the calib_gemm and bwd_gemm stages);
     - nm_mask: the standalone mask kernel on a bf16 W' of the layer's shape,
       against the measured HBM copy bandwidth (bytes: 2 read + 1/8 written per element);
     - sinkhorn_scaling: Sinkhorn forward then reverse over the logits of every
@@ -511,6 +513,28 @@ def extras(args, b, synth, wl, li, layer, step, flush, pk, dev):
     out["train"] = {"value": 1e3 / ms_tr, "unit": UNIT, "ms_per_step": ms_tr, "steps_per_call": total,
                     "note": "lcp_train: ten steps per call (eager launches), temperature 1 -> 0.1, AdamW "
                             "lr 5e-3 on the logits after every step; L2 flushed before each call only"}
+
+    # the step's two dense products through cuBLAS (torch.mm), same shapes and L2 flush, for
+    # context beside the calib_gemm / bwd_gemm stages: Y_d = X W^T and Y_s = X At^T
+    # (float32 outputs where torch.mm takes out_dtype, else bf16), and dAt = G^T X
+    T_, co, ci = li.spec.tokens, li.spec.cout, li.spec.cin
+    Xb = layer["X"] if layer["X"].dtype == torch.bfloat16 else layer["X"].to(torch.bfloat16)
+    Wb = layer["W"] if layer["W"].dtype == torch.bfloat16 else layer["W"].to(torch.bfloat16)
+    Gb = torch.randn(T_, co, device=dev).to(torch.bfloat16)
+    try:
+        torch.mm(Xb[:8], Wb[:8].t(), out_dtype=torch.float32)
+        f32_out = True
+    except Exception:
+        f32_out = False
+    kw = {"out_dtype": torch.float32} if f32_out else {}
+    ms_c = timed(lambda: (torch.mm(Xb, Wb.t(), **kw), torch.mm(Xb, Wb.t(), **kw)), K)
+    ms_g = timed(lambda: torch.mm(Gb.t(), Xb), K)
+    fl = 2.0 * T_ * co * ci
+    out["cublas_same_products"] = {
+        "calib_ms": ms_c, "calib_TFLOP/s": 2 * fl / (ms_c / 1e3) / 1e12, "calib_out": "f32" if f32_out else "bf16",
+        "bwd_ms": ms_g, "bwd_TFLOP/s": fl / (ms_g / 1e3) / 1e12,
+        "note": "library GEMMs on the same shapes for context; the step itself runs only this build's kernels"}
+    del Gb
 
     # standalone N:M mask on a bf16 W' of the layer's shape
     Wp = torch.randn(li.spec.cout, li.spec.cin, device=dev).to(torch.bfloat16)

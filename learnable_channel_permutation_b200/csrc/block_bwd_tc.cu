@@ -9,14 +9,16 @@ namespace {
 
 // ---------------------------------------- block backward, warp-specialised ---
 // BC = 64 (B = 32 or 64).  One CTA per (channel tile, row segment).  Warp 0
-// streams the (dAt, W) tiles of each 128-row chunk into a 3-stage ring; warp 1
-// issues W' = W (P_hi + P_lo) and dA = dAt P_hi into one of two TMEM buffers,
-// then, once the epilogue has written A = M.W' and dW' = M.dA, the stacked
-// dP product; warps 2-9 (two per TMEM lane quadrant, 32 columns each) turn
-// W', dA and the mask into the bf16 operands.  The dP accumulator stays in
-// TMEM for the whole segment and is written once at the end.
+// streams the (dAt, W) tiles of each 128-row chunk into a 4-stage ring; warp 1
+// issues [W P_hi | W P_lo] (one N = 128 product: the two P images are adjacent
+// in shared memory) and dA = dAt P_hi into one of two TMEM buffers, then, once
+// the epilogue has written A = M.W' and dW' = M.dA, the stacked dP product;
+// warps 2-9 (two per TMEM lane quadrant, 32 columns each) form W' = W P_hi +
+// W P_lo and turn W', dA and the mask into the bf16 operands.  The dP
+// accumulator stays in TMEM for the whole segment and is written once at the
+// end.  TMEM columns: buffer a at 192 a (W P_hi, W P_lo, dA: 64 each), dP at 384.
 template <int NSL> struct BwCfg {
-  static constexpr int STAGES = 3;
+  static constexpr int STAGES = 4;
   static constexpr int T_BYTES = 16384;                  // 128 rows x 64 bf16
   static constexpr int STAGE = 2 * T_BYTES;              // dAt | W (adjacent: stacked A operand)
   static constexpr int IMG_BYTES = 8192;
@@ -42,11 +44,13 @@ block_bwd_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_consta
   uint8_t* sPtl = sPth + C::IMG_BYTES;
   uint8_t* sAB = sPtl + C::IMG_BYTES;      // buffer a at + a * 2 * T_BYTES: A | dW' (adjacent)
   uint64_t* bars = reinterpret_cast<uint64_t*>(sAB + 2 * 2 * C::T_BYTES);
-  // bars: full[3] empty[3] wd[2] abf[2] abe[2] dpf drain img
-  uint32_t* holder = reinterpret_cast<uint32_t*>(bars + 16);
+  // bars: full[S] empty[S] wd[2] abf[2] abe[2] dpf drain img
+  constexpr int S = C::STAGES;
+  uint32_t* holder = reinterpret_cast<uint32_t*>(bars + 2 * S + 10);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(holder + 1);
   auto bar = [&](int i) { return smem_u32(bars + i); };
-  const int FULL = 0, EMPTY = 3, WD = 6, ABF = 8, ABE = 10, DPF = 12, DRAIN = 13, IMG = 14;
+  const int FULL = 0, EMPTY = S, WD = 2 * S, ABF = 2 * S + 2, ABE = 2 * S + 4, DPF = 2 * S + 6, DRAIN = 2 * S + 7,
+            IMG = 2 * S + 8;
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int t = blockIdx.x, sidx = blockIdx.y, col0 = t * 64;
@@ -55,7 +59,7 @@ block_bwd_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_consta
   const int nchunk = cdiv(rend - rbeg, 128);
   const int words = cin / 32;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 3; ++i) { mbar_init(bar(FULL + i), 1); mbar_init(bar(EMPTY + i), 1); }
+    for (int i = 0; i < S; ++i) { mbar_init(bar(FULL + i), 1); mbar_init(bar(EMPTY + i), 1); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(WD + i), 1);
       mbar_init(bar(ABF + i), C::EPI_WARPS);
@@ -74,7 +78,7 @@ block_bwd_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_consta
   const uint32_t tmem = *holder;
   pdl_wait();
   pdl_trigger();
-  const uint32_t tDP = tmem + 256;
+  const uint32_t tDP = tmem + 384;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -106,9 +110,10 @@ block_bwd_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_consta
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc_n = idesc_bf16(128, 64, false, false);
+      constexpr uint32_t idesc_w = idesc_bf16(128, 128, false, false);
       constexpr uint32_t idesc_dp = idesc_bf16(128, 128, true, true);
       bool ok = nchunk == 0 || mbar_wait(bar(IMG), 0, abort_flag, 74);
-      // W' = W (P_hi + P_lo) and dA = dAt P_hi of chunk c into TMEM buffer c & 1
+      // [W P_hi | W P_lo] and dA = dAt P_hi of chunk c into TMEM buffer c & 1
       auto mma1 = [&](int c) -> bool {
         const int st = c % C::STAGES, a = c & 1;
         const uint32_t use = (uint32_t)(c / C::STAGES) & 1u, ua = (uint32_t)(c >> 1) & 1u;
@@ -117,14 +122,12 @@ block_bwd_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_consta
         if (c >= 2 && !mbar_wait(bar(ABF + a), ua ^ 1u, abort_flag, 76)) return false;
         tc_fence_after();
         const uint32_t sg = smem_u32(sStage + st * C::STAGE);
-        const uint32_t tW = tmem + a * 128, tDA = tmem + a * 128 + 64;
+        const uint32_t tW = tmem + a * 192, tDA = tmem + a * 192 + 128;
 #pragma unroll
         for (int k16 = 0; k16 < 4; ++k16) {
-          const uint64_t wdesc = sdesc(sg + C::T_BYTES + k16 * 32, 16, 1024);
-          mma_bf16(tW, wdesc, sdesc(smem_u32(sPth) + k16 * 32, 16, 1024), idesc_n, k16 != 0);
-          mma_bf16(tW, wdesc, sdesc(smem_u32(sPtl) + k16 * 32, 16, 1024), idesc_n, true);
-          mma_bf16(tDA, sdesc(sg + k16 * 32, 16, 1024), sdesc(smem_u32(sPth) + k16 * 32, 16, 1024), idesc_n,
-                   k16 != 0);
+          const uint64_t pdesc = sdesc(smem_u32(sPth) + k16 * 32, 16, 1024);   // rows 64..127: P_lo image
+          mma_bf16(tW, sdesc(sg + C::T_BYTES + k16 * 32, 16, 1024), pdesc, idesc_w, k16 != 0);
+          mma_bf16(tDA, sdesc(sg + k16 * 32, 16, 1024), pdesc, idesc_n, k16 != 0);
         }
         mma_commit(bar(WD + a));
         return true;
@@ -172,9 +175,10 @@ block_bwd_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_consta
       ok = named_and(1, C::EPI, mbar_wait(bar(WD + a), ua, abort_flag, 79));
       if (!ok) break;
       tc_fence_after();
-      uint32_t wv[NV], dv[NV];
-      tmem_ld_cols<NV>(tmem + lane_off + a * 128 + h * NV, wv);
-      tmem_ld_cols<NV>(tmem + lane_off + a * 128 + 64 + h * NV, dv);
+      uint32_t wv[NV], wl[NV], dv[NV];
+      tmem_ld_cols<NV>(tmem + lane_off + a * 192 + h * NV, wv);
+      tmem_ld_cols<NV>(tmem + lane_off + a * 192 + 64 + h * NV, wl);
+      tmem_ld_cols<NV>(tmem + lane_off + a * 192 + 128 + h * NV, dv);
       tmem_ld_wait();
       // buffer a was last read by the dP product of chunk c - 2
       ok = named_and(1, C::EPI, c < 2 || mbar_wait(bar(ABE + a), ua ^ 1u, abort_flag, 80));
@@ -187,7 +191,7 @@ block_bwd_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_consta
 #pragma unroll
         for (int x = 0; x < 8; ++x) {
           const bool keep = (bits >> (8 * c8 + x)) & 1u;
-          fa[x] = keep ? __uint_as_float(wv[8 * c8 + x]) : 0.f;
+          fa[x] = keep ? __uint_as_float(wv[8 * c8 + x]) + __uint_as_float(wl[8 * c8 + x]) : 0.f;
           fd[x] = keep ? __uint_as_float(dv[8 * c8 + x]) : 0.f;
         }
         const int chunk = h * (NV / 8) + c8;

@@ -17,10 +17,41 @@ constexpr int GM_THREADS = 192;   // warp 0: TMA producer, warp 1: MMA issuer, w
 // (rank 0) issues M = 256, N = 256 MMAs that read both CTAs' operands, and each
 // CTA holds its 128 x 256 half of the accumulator in its own tensor memory.
 // Per SM this halves the B bytes per MMA cycle (32 KB of operands per 64-deep
-// k-block instead of 48 KB), and six stages fit in shared memory.
-constexpr int G2_BM = 256, G2_BN = 256, G2_BK = 64, G2_STAGES = 6;
+// k-block instead of 48 KB), and seven stages fit in shared memory.
+//
+// Tiles go to pairs round-robin.  When the last round would leave more than half
+// of the pairs idle, its tiles are split into two 256 x 128 halves (N = 128
+// MMAs, 64 B rows per CTA), so the pairs that still work finish in about half a
+// tile's time instead of a whole one.
+constexpr int G2_BM = 256, G2_BN = 256, G2_BK = 64, G2_STAGES = 7;
 constexpr int G2_HALF = 128 * G2_BK * 2;               // one 128-row operand half: 16 KB
 constexpr int G2_SMEM = G2_STAGES * 2 * G2_HALF + 1024 + 256;
+
+// Work items of the round-robin schedule: whole tiles [0, split_base), then the
+// remaining tiles as two halves each.
+struct PairSched {
+  int items, split_base;
+  __device__ PairSched(int total, int npairs) {
+    const int rem = total % npairs;
+    if (rem != 0 && 2 * rem <= npairs) {
+      split_base = total - rem;
+      items = split_base + 2 * rem;
+    } else {
+      split_base = total;
+      items = total;
+    }
+  }
+  // tile of item it; half -1 for the whole tile, else the 128-column half
+  __device__ void at(int it, int& tile, int& half) const {
+    if (it < split_base) {
+      tile = it;
+      half = -1;
+    } else {
+      tile = split_base + ((it - split_base) >> 1);
+      half = (it - split_base) & 1;
+    }
+  }
+};
 
 template <bool A_MN, bool B_MN, bool OUT_BF16>
 __global__ void __launch_bounds__(GM_THREADS, 1)
@@ -67,24 +98,30 @@ gemm_pair_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
   const int mtiles = cdiv(M, G2_BM), ntiles = cdiv(N, G2_BN);
   const int total = mtiles * ntiles * nprob;
   const int nk = cdiv(K, G2_BK);
+  const PairSched sched(total, npairs);
 
   if (warp == 0) {
     if (lane == 0) {
       int stage = 0;
       uint32_t ph = 0;
       uint32_t issued = 0, issued_par = 0;
-      for (int tile = pair; tile < total; tile += npairs) {
+      for (int it = pair; it < sched.items; it += npairs) {
+        int tile, half;
+        sched.at(it, tile, half);
         const int mt = tile % mtiles, rest = tile / mtiles;
         const int nt = rest % ntiles, prob = rest / ntiles;
         const CUtensorMap* mb = prob ? &tmB1 : &tmB0;
-        const int a_row = mt * G2_BM + (int)rank * 128, b_row = nt * G2_BN + (int)rank * 128;
+        // each CTA stages half of the tile's B rows: 128 of a whole tile, 64 of a half
+        const int a_row = mt * G2_BM + (int)rank * 128;
+        const int b_row = nt * G2_BN + (half < 0 ? (int)rank * 128 : half * 128 + (int)rank * 64);
+        const uint32_t bytes = half < 0 ? 2 * G2_HALF : G2_HALF + G2_HALF / 2;
         bool ok = true;
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(empty(stage), ph ^ 1u, abort_flag, 91)) { ok = false; break; }
           issued |= 1u << stage;
           issued_par = (issued_par & ~(1u << stage)) | (ph << stage);
           const uint32_t fbar = mapa(full(stage), 0);
-          mbar_expect_tx_cluster(fbar, 2 * G2_HALF);
+          mbar_expect_tx_cluster(fbar, bytes);
           const uint32_t a_dst = smem_u32(sA + stage * G2_HALF);
           const uint32_t b_dst = smem_u32(sB + stage * G2_HALF);
           if (!A_MN) {
@@ -93,11 +130,13 @@ gemm_pair_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             tma_load_2d_pair(a_dst, &tmA, fbar, a_row, kb * G2_BK);
             tma_load_2d_pair(a_dst + 8192, &tmA, fbar, a_row + 64, kb * G2_BK);
           }
+          // B in boxes of 64 rows (K-major) or 64 columns (MN-major), 8 KB each
           if (!B_MN) {
             tma_load_2d_pair(b_dst, mb, fbar, kb * G2_BK, b_row);
+            if (half < 0) tma_load_2d_pair(b_dst + 8192, mb, fbar, kb * G2_BK, b_row + 64);
           } else {
             tma_load_2d_pair(b_dst, mb, fbar, b_row, kb * G2_BK);
-            tma_load_2d_pair(b_dst + 8192, mb, fbar, b_row + 64, kb * G2_BK);
+            if (half < 0) tma_load_2d_pair(b_dst + 8192, mb, fbar, b_row + 64, kb * G2_BK);
           }
           if (++stage == G2_STAGES) { stage = 0; ph ^= 1u; }
         }
@@ -116,10 +155,14 @@ gemm_pair_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0 && rank == 0) {
-      constexpr uint32_t idesc = idesc_bf16(G2_BM, G2_BN, A_MN, B_MN);
+      constexpr uint32_t idesc_full = idesc_bf16(G2_BM, G2_BN, A_MN, B_MN);
+      constexpr uint32_t idesc_half = idesc_bf16(G2_BM, G2_BN / 2, A_MN, B_MN);
       int stage = 0, lt = 0;
       uint32_t ph = 0;
-      for (int tile = pair; tile < total; tile += npairs, ++lt) {
+      for (int it = pair; it < sched.items; it += npairs, ++lt) {
+        int tile, half;
+        sched.at(it, tile, half);
+        const uint32_t idesc = half < 0 ? idesc_full : idesc_half;
         const int acc = lt & 1;
         const uint32_t aph = (uint32_t)(lt >> 1) & 1u;
         if (!mbar_wait(tempty(acc), aph ^ 1u, abort_flag, 94)) break;
@@ -151,7 +194,9 @@ gemm_pair_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     const int q = warp & 3;
     const uint32_t tempty_leader0 = mapa(tempty(0), 0), tempty_leader1 = mapa(tempty(1), 0);
     int lt = 0;
-    for (int tile = pair; tile < total; tile += npairs, ++lt) {
+    for (int it = pair; it < sched.items; it += npairs, ++lt) {
+      int tile, half;
+      sched.at(it, tile, half);
       const int acc = lt & 1;
       const uint32_t aph = (uint32_t)(lt >> 1) & 1u;
       if (!warp_all(mbar_wait(tfull(acc), aph, abort_flag, 97))) break;
@@ -159,13 +204,15 @@ gemm_pair_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       const int mt = tile % mtiles, rest = tile / mtiles;
       const int nt = rest % ntiles, prob = rest / ntiles;
       const int row = mt * G2_BM + (int)rank * 128 + q * 32 + lane;
+      const int chunks = half < 0 ? G2_BN / 32 : G2_BN / 64;
+      const int col_base = nt * G2_BN + (half < 0 ? 0 : half * (G2_BN / 2));
       void* Dp = prob ? D1 : D0;
 #pragma unroll 1
-      for (int c = 0; c < G2_BN / 32; ++c) {
+      for (int c = 0; c < chunks; ++c) {
         uint32_t r[32];
         tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * G2_BN + c * 32), r);
         tmem_ld_wait();
-        const int col0 = nt * G2_BN + c * 32;
+        const int col0 = col_base + c * 32;
         if (row < M && col0 < N) {
           if constexpr (OUT_BF16) {
             __nv_bfloat16* out = static_cast<__nv_bfloat16*>(Dp) + (size_t)row * ldd + col0;
@@ -215,7 +262,8 @@ lcp_status launch_pair(K kernel, int tiles, const CUtensorMap& a, const CUtensor
                        const char* what) {
   TC_TRY(set_smem(kernel, G2_SMEM, what));
   const int max_pairs = num_sms() / 2;
-  const int pairs = tiles < max_pairs ? tiles : max_pairs;
+  // few tiles: twice as many pairs, each taking one half tile
+  const int pairs = 2 * tiles <= max_pairs ? 2 * tiles : (tiles < max_pairs ? tiles : max_pairs);
   return launch_kernel(kernel, dim3(2 * pairs), dim3(GM_THREADS), G2_SMEM, st, 2, true, what, a, b0, b1, d0, d1, M, N,
                        Kd, ldd, nprob);
 }
@@ -226,12 +274,12 @@ lcp_status tc_error_gemm(int* site, int reset) { return read_tc_error(site, rese
 
 lcp_status launch_calib_gemm_tc(const __nv_bfloat16* X, const __nv_bfloat16* W, const __nv_bfloat16* At,
                                 float* Yd, float* Ys, int tokens, int cout, int cin, cudaStream_t st) {
-  // operand halves of 128 rows: each CTA of a pair stages its own half
+  // A in boxes of 128 rows, B in boxes of 64 rows: each CTA of a pair stages its own half
   CUtensorMap mA, mB0, mB1;
   const int nprob = Ys ? 2 : 1;
   TC_TRY(make_map(&mA, X, cin, tokens, 64, 128, "calib_gemm X"));
-  TC_TRY(make_map(&mB0, W, cin, cout, 64, 128, "calib_gemm W"));
-  TC_TRY(make_map(&mB1, Ys ? (const void*)At : (const void*)W, cin, cout, 64, 128, "calib_gemm At"));
+  TC_TRY(make_map(&mB0, W, cin, cout, 64, 64, "calib_gemm W"));
+  TC_TRY(make_map(&mB1, Ys ? (const void*)At : (const void*)W, cin, cout, 64, 64, "calib_gemm At"));
   const int tiles = cdiv(tokens, G2_BM) * cdiv(cout, G2_BN) * nprob;
   return launch_pair(gemm_pair_tc_kernel<false, false, false>, tiles, mA, mB0, mB1, Yd, Ys, tokens, cout, cin,
                      cout, nprob, st, "calib_gemm");
