@@ -24,6 +24,10 @@ Sources (the web pages the method is taken from):
   P = argmax over permutation matrices of Tr(P^T P_hat) (the Hungarian
   algorithm), and the backward pass takes dP/dP_hat = 1 (straight-through).
 
+* [PermLLM] "Effect on inference acceleration": the deployed layer applies
+  the channel permutation to its input at run time (a custom CUDA kernel,
+  compared there with PyTorch) and multiplies by the 2:4 sparse weight.
+
 * [PermLLM] "Implementation details": the logits are trained with AdamW
   (learning rate 1e-3 or 5e-3), 5 Sinkhorn iterations, the temperature
   decreasing linearly from 1 to 0.1, block size 64.
@@ -45,6 +49,13 @@ Readings where the pages are silent or garbled (each is restated where used):
     the published definitions, Wanda S_ij = |W_ij| ||X_j||_2 and RIA
     S_ij = (|W_ij| / sum_k |W_kj| + |W_ij| / sum_k |W_ik|) ||X_j||_2^0.5,
     with X_j the j-th input channel over the calibration tokens.
+12. Inference format (the pages give none): the deployed weight is
+    A = M (.) (W P_B) for the hard P_B, in permuted column order, kept as the
+    two kept entries of every group of four columns (in column order) and
+    their positions 0..3 in the group; the positions are packed as 4-bit
+    fields (first position in the low two bits) of 32-bit words, eight
+    groups a word, group g at bits 4 (g % 8) of word g // 8.  The input side
+    is x_pi = P_B^T x, i.e. x_pi[bB + pi_b(i)] = x[bB + i].
 10. AdamW is Loshchilov and Hutter's (decoupled weight decay, bias-corrected
     moments) with the usual defaults beta = (0.9, 0.999), eps = 1e-8, decay
     0.01 (the pages give only the learning rate); the linear temperature
@@ -408,3 +419,86 @@ def train(W, X_tokens, logits, n_iters, n, m, total, steps=None, lr=1e-3, tau_st
         dL = fw["dL"]
         L, mom, vel = adamw_update(L, dL, mom, vel, s + 1, lr=lr, **adam)
     return L, losses, dL
+
+
+# ---------------------------------------------------------------------------
+# Inference side  ([PermLLM] "Effect on inference acceleration")
+# ---------------------------------------------------------------------------
+# The deployed layer computes y = A x_pi with A = M (.) (W P_B) (hard P_B, 2:4
+# mask) and x_pi = P_B^T x.  The functions below restate that product on the
+# compressed form of A (reading 12): gather the inputs, then for every kept
+# entry multiply by the input at its position.
+
+def gather_channels(X_tokens: np.ndarray, perm: np.ndarray) -> np.ndarray:
+    """x_pi = P_B^T x for every token: X_pi[t, bB + perm[b, i]] = X[t, bB + i].
+
+    ``perm`` [nb, B] is the hardening's permutation (row i of block b goes to
+    column perm[b, i]), so the source channel i of block b lands in slot perm[b, i].
+    """
+    X = np.asarray(X_tokens)
+    perm = np.asarray(perm)
+    nb, B = perm.shape
+    out = np.empty_like(X)
+    for b in range(nb):
+        out[:, b * B + perm[b]] = X[:, b * B:(b + 1) * B]
+    return out
+
+
+def pack_24(A: np.ndarray, mask: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
+    """Compressed 2:4 form of A under ``mask`` (exactly two kept of every four
+    consecutive columns): values[:, 2g + k] is the k-th kept entry of group g in
+    column order and idx[:, 2g + k] its position 0..3 in the group."""
+    A = np.asarray(A)
+    M = np.asarray(mask, bool)
+    rows, cols = A.shape
+    if cols % 4:
+        raise ValueError("columns must be a multiple of 4")
+    G = M.reshape(rows, cols // 4, 4)
+    if not np.all(G.sum(axis=2) == 2):
+        raise ValueError("every group of four must keep exactly two entries")
+    # positions of the kept entries, ascending: a stable sort puts kept (key 0) first
+    pos = np.argsort(np.where(G, 0, 1), axis=2, kind="stable")[:, :, :2]
+    vals = np.take_along_axis(A.reshape(rows, cols // 4, 4), pos, axis=2)
+    return vals.reshape(rows, cols // 2), pos.reshape(rows, cols // 2).astype(np.int64)
+
+
+def meta_words(idx: np.ndarray) -> np.ndarray:
+    """Positions -> 32-bit metadata words (reading 12): group g's field at bits
+    4 (g % 8) of word g // 8, first position in the low two bits."""
+    idx = np.asarray(idx, np.uint64)
+    rows, half = idx.shape
+    if half % 16:
+        raise ValueError("columns must be a multiple of 32")
+    field = idx[:, 0::2] | (idx[:, 1::2] << np.uint64(2))          # [rows, groups]
+    field = field.reshape(rows, half // 16, 8)
+    shifts = (np.uint64(4) * np.arange(8, dtype=np.uint64))
+    return (field << shifts).sum(axis=2).astype(np.uint32)
+
+
+def unpack_24(vals: np.ndarray, idx: np.ndarray) -> np.ndarray:
+    """The dense matrix of a compressed form (zeros where nothing is kept)."""
+    vals = np.asarray(vals, np.float64)
+    rows, half = vals.shape
+    cols = 4 * (np.arange(half) // 2)[None, :] + np.asarray(idx)
+    A = np.zeros((rows, 2 * half))
+    A[np.arange(rows)[:, None], cols] = vals
+    return A
+
+
+def sparse24_mm(vals: np.ndarray, idx: np.ndarray, X_tokens: np.ndarray,
+                perm: Optional[np.ndarray] = None) -> np.ndarray:
+    """Y[t, o] = sum over the kept entries k of row o of vals[o, k] * x_pi[t, slot(o, k)],
+    slot(o, k) = 4 (k // 2) + idx[o, k]; x_pi = gather_channels(X, perm) (``perm``
+    None: X is already in permuted order).  Returns Y as [T, rows]."""
+    Xp = np.asarray(X_tokens, np.float64)
+    if perm is not None:
+        Xp = gather_channels(Xp, perm)
+    vals = np.asarray(vals, np.float64)
+    rows, half = vals.shape
+    slot = 4 * (np.arange(half) // 2)[None, :] + np.asarray(idx)
+    Y = np.empty((Xp.shape[0], rows))
+    for r0 in range(0, rows, 128):
+        r1 = min(rows, r0 + 128)
+        Y[:, r0:r1] = np.einsum("ok,tok->to", vals[r0:r1], Xp[:, slot[r0:r1]])
+    return Y
+

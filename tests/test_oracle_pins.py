@@ -619,3 +619,83 @@ def test_wanda_with_equal_channel_norms_is_magnitude():
     W = rng.normal(size=(8, 16))
     X = np.ones((4, 16)) * np.array([1, -1, 1, -1])[:, None]     # every ||X_j|| = 2
     assert np.allclose(O.importance(W, X, "wanda"), 2 * np.abs(W))
+
+
+# --------------------------------------------------------- inference side ---
+
+def test_pack_24_worked_example():
+    """One row by hand: groups (1, -5, 3, 2) and (0.5, 4, -4, 1) keep (-5, 3) at
+    positions 1, 2 and (4, -4) at 1, 2 (|4| = |-4|: both are the two largest);
+    every field is 1 | 2 << 2 = 9.  With x = 1..8: -5*2 + 3*3 + 4*6 - 4*7 = -5."""
+    W = np.array([[1.0, -5.0, 3.0, 2.0, 0.5, 4.0, -4.0, 1.0]])
+    M = O.nm_mask(W, 2, 4)
+    vals, idx = O.pack_24(W, M)
+    assert vals.tolist() == [[-5.0, 3.0, 4.0, -4.0]]
+    assert idx.tolist() == [[1, 2, 1, 2]]
+    assert int(O.meta_words(np.tile(idx, (1, 8)))[0, 0]) == 0x99999999
+    Y = O.sparse24_mm(vals, idx, np.arange(1.0, 9.0)[None, :])
+    assert Y.tolist() == [[-5.0]]
+
+
+def test_meta_words_field_by_field():
+    rng = np.random.default_rng(60)
+    first = rng.integers(0, 3, (3, 16))
+    second = first + 1 + rng.integers(0, 3 - first)      # first < second <= 3
+    idx = np.stack([first, second], axis=2).reshape(3, 32)
+    words = O.meta_words(idx)
+    for r in range(3):
+        for g in range(16):
+            field = (int(words[r, g // 8]) >> (4 * (g % 8))) & 0xF
+            assert field & 3 == first[r, g] and field >> 2 == second[r, g]
+
+
+def test_pack_24_round_trip_and_positions():
+    rng = np.random.default_rng(61)
+    A = rng.normal(size=(6, 64))
+    M = O.nm_mask(rng.normal(size=(6, 64)), 2, 4)
+    vals, idx = O.pack_24(A, M)
+    assert np.array_equal(O.unpack_24(vals, idx), np.where(M, A, 0.0))
+    assert np.all(idx[:, 0::2] < idx[:, 1::2])
+    with pytest.raises(ValueError):
+        O.pack_24(A, O.nm_mask(A, 1, 4))
+
+
+def test_gather_is_the_block_permutation_of_the_inputs():
+    """x_pi = P_B^T x: as token rows, X_pi = X P_B with P_B from perm_matrix."""
+    rng = np.random.default_rng(62)
+    pis = np.stack([rng.permutation(8) for _ in range(3)])
+    X = rng.normal(size=(5, 24))
+    assert np.array_equal(O.gather_channels(X, pis), X @ O.block_diag(O.perm_matrix(pis)))
+    ident = np.tile(np.arange(8), (3, 1))
+    assert np.array_equal(O.gather_channels(X, ident), X)
+
+
+def test_sparse24_mm_is_the_hardened_sparse_output():
+    """The deployed product on the compressed weight equals the training
+    forward's sparse output Y_s = A P_B^T X for the same hard permutation and
+    mask (a different route: dense block-diagonal matrices)."""
+    rng = np.random.default_rng(63)
+    W = rng.normal(size=(10, 32))
+    X = rng.normal(size=(7, 32))
+    pis = np.stack([rng.permutation(16) for _ in range(2)])
+    fw = O.forward(W, X, None, 1.0, 5, 2, 4, P=O.perm_matrix(pis))
+    vals, idx = O.pack_24(fw["A"], fw["mask"])
+    Y = O.sparse24_mm(vals, idx, X, pis)
+    assert np.allclose(Y.T, fw["Ys"], rtol=1e-12, atol=1e-12)
+
+
+def test_sparse24_mm_by_explicit_loops():
+    rng = np.random.default_rng(64)
+    vals = rng.normal(size=(3, 8))
+    idx = np.array([[0, 3, 1, 2, 0, 1, 2, 3]] * 3)
+    X = rng.normal(size=(2, 16))
+    pis = np.array([rng.permutation(8), rng.permutation(8)])
+    Y = O.sparse24_mm(vals, idx, X, pis)
+    src = {}                     # slot -> source channel
+    for b in range(2):
+        for i in range(8):
+            src[8 * b + pis[b, i]] = 8 * b + i
+    for t in range(2):
+        for o in range(3):
+            ref = sum(vals[o, k] * X[t, src[4 * (k // 2) + idx[o, k]]] for k in range(8))
+            assert math.isclose(Y[t, o], ref, rel_tol=1e-12, abs_tol=1e-12)
