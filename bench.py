@@ -536,6 +536,10 @@ def extras(args, b, synth, wl, li, layer, step, flush, pk, dev):
         "note": "library GEMMs on the same shapes for context; the step itself runs only this build's kernels"}
     del Gb
 
+    # inference side: the layer deployed as a 2:4 compressed weight (the hard
+    # permutation and mask of one LCP_FLAG_HARD step), decode-sized token counts
+    out["inference_24"] = inference_24(b, layer, wl, li, dev, pk, timed, K)
+
     # standalone N:M mask on a bf16 W' of the layer's shape
     Wp = torch.randn(li.spec.cout, li.spec.cin, device=dev).to(torch.bfloat16)
     bits = torch.empty(li.spec.cout, li.spec.cin // 32, dtype=torch.int32, device=dev)
@@ -566,6 +570,88 @@ def extras(args, b, synth, wl, li, layer, step, flush, pk, dev):
     del Lb, Pb, ck, dP, dLb
     torch.cuda.empty_cache()
     return out
+
+
+def inference_24(b, layer, wl, li, dev, pk, timed, K):
+    """The deployed layer: lcp_sparse24_mm (gather fused) against the dense
+    bf16 product through cuBLAS (torch.mm) at decode-sized T, and the
+    standalone gather against PyTorch's column indexing at T = 2048.
+
+    These calls take microseconds, less than the host's cost of issuing them,
+    so each is timed inside a CUDA graph of R repetitions of (L2 flush, call)
+    minus a graph of R flushes alone."""
+    import torch
+    cout, cin, B = li.spec.cout, li.spec.cin, wl.block
+    nb = cin // B
+    layer["perm"] = torch.empty(nb, B, dtype=torch.int32, device=dev)
+    hard = b.Step([layer], B, wl.n, wl.m, wl.iters, wl.tau, flags=b.FLAG_HARD)
+    hard.run()
+    perm = layer.pop("perm")
+    W = layer["W"] if layer["W"].dtype == torch.bfloat16 else layer["W"].to(torch.bfloat16)
+    vals, meta = b.pack24(W, perm, layer["mask"], B)
+    torch.cuda.synchronize()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    R = max(5, min(K, 20))
+
+    def graph_us(fn):
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            for _ in range(2):
+                flush.zero_()
+                if fn is not None:
+                    fn()
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(R):
+                flush.zero_()
+                if fn is not None:
+                    fn()
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(5):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        del g
+        return e0.elapsed_time(e1) / 5 / R * 1e3
+
+    t_flush = graph_us(None)
+    res = {"shape": [cout, cin], "B": B, "per_T": {}, "timing": f"CUDA graph of {R} x (L2 flush, call) "
+                                                                 f"minus {R} flushes alone"}
+    gen = torch.Generator(device=dev).manual_seed(11)
+    for T in (1, 4, 8, 16):
+        X = torch.randn(T, cin, device=dev, generator=gen).to(torch.bfloat16)
+        Y = torch.empty(T, cout, dtype=torch.float32, device=dev)
+        us_s = graph_us(lambda: b.sparse24_mm(vals, meta, X, perm, B, Y)) - t_flush
+        us_d = graph_us(lambda: torch.mm(X, W.t())) - t_flush
+        by = cout * cin // 2 * 2 + cout * cin // 8 + T * cin * 2 + T * cout * 4
+        res["per_T"][str(T)] = {"sparse_us": us_s, "dense_cublas_us": us_d, "speedup": us_d / us_s,
+                                "sparse_GB/s": by / us_s / 1e3, "sparse_frac_hbm": by / us_s / 1e3 / pk["hbm_gbs"],
+                                "bytes": by}
+    # the run-time permutation alone on a prefill-sized activation
+    T = li.spec.tokens
+    X = torch.randn(T, cin, device=dev, generator=gen).to(torch.bfloat16)
+    Xp = torch.empty_like(X)
+    src = torch.empty(cin, dtype=torch.long, device=dev)
+    pl = perm.long()
+    base = (torch.arange(nb, device=dev) * B)[:, None]
+    src[(base + pl).reshape(-1)] = (base + torch.arange(B, device=dev)[None, :]).reshape(-1)
+    us_g = graph_us(lambda: b.gather(X, perm, Xp)) - t_flush
+    us_t = graph_us(lambda: X[:, src]) - t_flush
+    assert torch.equal(X[:, src], b.gather(X, perm))
+    byg = 2 * T * cin * 2
+    res["gather"] = {"T": T, "us": us_g, "torch_index_us": us_t, "speedup_vs_torch": us_t / us_g,
+                     "GB/s": byg / us_g / 1e3, "frac_hbm": byg / us_g / 1e3 / pk["hbm_gbs"]}
+    res["note"] = ("permutation and mask from one LCP_FLAG_HARD step of the layer; bytes of the sparse "
+                   "product = kept values + 4-bit position fields + X + Y")
+    del flush
+    return res
 
 
 def cpu_baseline_one_core(wl):

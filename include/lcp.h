@@ -45,7 +45,7 @@
 extern "C" {
 #endif
 
-#define LCP_ABI_VERSION 2
+#define LCP_ABI_VERSION 3
 
 #if defined(__GNUC__)
 #define LCP_API __attribute__((visibility("default")))
@@ -257,6 +257,45 @@ LCP_API lcp_status lcp_calib_gemm(const void* X, const void* W, const void* At, 
  * accumulation over the T tokens). */
 LCP_API lcp_status lcp_grad_gemm(const void* G, const void* X, void* dAt, int tokens, int cout,
                                  int cin, cudaStream_t stream);
+
+/* ---- Inference side ("Effect on inference acceleration": the deployed layer
+ * permutes its input channels at run time and multiplies by the 2:4 sparse
+ * weight).  The deployed weight is A = M.(W P_B) for a hard block permutation
+ * P_B and a 2:4 mask M, in permuted column order, kept compressed:
+ *   values [C_out, C_in/2] in `dtype`: the two kept entries of every group of
+ *          four columns, in column order;
+ *   meta   [C_out, C_in/32] uint32: group g's 4-bit field at bits 4 (g % 8) of
+ *          word g / 8, first kept position (0..3) in the low two bits, second
+ *          (larger) in the high two.
+ * perm [C_in/B, B] int32 is the hardening's permutation (lcp_harden: row i of
+ * block b goes to column perm[b][i]); the input side is x_pi = P_B^T x, i.e.
+ * x_pi[bB + perm[b][i]] = x[bB + i].  A perm entry outside [0, B) is skipped
+ * and recorded in lcp_device_error (302); a perm that is not a permutation of
+ * its block gives unspecified (in-bounds) results. */
+
+/* Compressed weight from W [C_out, C_in] (original column order, `dtype`), perm
+ * (NULL: identity, B then only needs to divide C_in; 0 is accepted) and the
+ * mask bits of M [C_out, C_in/32] in permuted order (as lcp_step writes them
+ * for LCP_FLAG_HARD).  A group without exactly two kept bits is written as
+ * positions (0, 1) with zero values and recorded in lcp_device_error (301); a
+ * repeated perm entry is recorded as 303.  C_in % 32 == 0, C_in % B == 0,
+ * B in {32, 64, 128, 256}. */
+LCP_API lcp_status lcp_pack24(const void* W, const int32_t* perm, const uint32_t* mask, void* values,
+                              uint32_t* meta, int cout, int cin, int B, lcp_dtype dtype, cudaStream_t stream);
+
+/* The input gather (the pages' run-time channel permutation): Xp = x_pi for
+ * every token, X and Xp [T, C_in] in `dtype`, out of place. */
+LCP_API lcp_status lcp_gather(const void* X, const int32_t* perm, void* Xp, int tokens, int cin, int B,
+                              lcp_dtype dtype, cudaStream_t stream);
+
+/* The deployed product Y = x_pi A^T for every token: X [T, C_in] in `dtype`
+ * (original channel order when perm is given, already permuted when perm is
+ * NULL), values / meta as above, Y [T, C_out] float32 (float32 accumulation).
+ * Built for decode-sized T (tiles of up to 16 tokens; larger T runs tile by
+ * tile, re-streaming the weight); C_in up to 102400 (bf16) / 51200 (float32). */
+LCP_API lcp_status lcp_sparse24_mm(const void* values, const uint32_t* meta, const void* X, const int32_t* perm,
+                                   float* Y, int cout, int cin, int tokens, int B, lcp_dtype dtype,
+                                   cudaStream_t stream);
 
 /* Diagnostic (synchronous: reads a device word).  Every wait inside the
  * tensor-core kernels is bounded; a wait that expires records its site here

@@ -97,6 +97,11 @@ def lib() -> ctypes.CDLL:
                        _c_void_p], _c_int),
         "lcp_train": ([P(LcpLayer), _c_int, P(LcpHparams), P(LcpAdamwParams), P(LcpAdamwState), _c_int, _c_int,
                        _c_int, _c_float, _c_float, _c_void_p, ctypes.c_size_t, _c_void_p], _c_int),
+        "lcp_pack24": ([_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_int,
+                        _c_void_p], _c_int),
+        "lcp_gather": ([_c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_int, _c_void_p], _c_int),
+        "lcp_sparse24_mm": ([_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_int,
+                             _c_int, _c_void_p], _c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -305,6 +310,39 @@ def nm_mask(Wp: torch.Tensor, bits: torch.Tensor, n: int, m: int) -> None:
     rows, cols = Wp.shape
     check(lib().nm_mask(_ptr(Wp, None, "Wp"), _ptr(bits, torch.int32, "bits"), rows, cols, n, m, _dt(Wp),
                         _stream(None)))
+
+
+def pack24(W: torch.Tensor, perm: Optional[torch.Tensor], mask_bits: torch.Tensor, block: int):
+    """Compressed 2:4 weight (values [C_out, C_in/2] in W's dtype, meta [C_out, C_in/32]
+    int32 words) of A = M.(W P_B) for the hard permutation perm [C_in/B, B]."""
+    cout, cin = W.shape
+    vals = torch.empty(cout, cin // 2, dtype=W.dtype, device=W.device)
+    meta = torch.empty(cout, cin // 32, dtype=torch.int32, device=W.device)
+    check(lib().lcp_pack24(_ptr(W, None, "W"), _ptr(perm, torch.int32, "perm"), _ptr(mask_bits, torch.int32, "mask"),
+                           _ptr(vals, W.dtype, "values"), _ptr(meta, torch.int32, "meta"), cout, cin, block, _dt(W),
+                           _stream(None)))
+    return vals, meta
+
+
+def gather(X: torch.Tensor, perm: torch.Tensor, Xp: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """x_pi = P_B^T x for every token row of X [T, C_in]."""
+    T, cin = X.shape
+    Xp = torch.empty_like(X) if Xp is None else Xp
+    check(lib().lcp_gather(_ptr(X, None, "X"), _ptr(perm, torch.int32, "perm"), _ptr(Xp, X.dtype, "Xp"), T, cin,
+                           perm.shape[1], _dt(X), _stream(None)))
+    return Xp
+
+
+def sparse24_mm(vals: torch.Tensor, meta: torch.Tensor, X: torch.Tensor, perm: Optional[torch.Tensor],
+                block: int, Y: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Y [T, C_out] float32 = x_pi A^T from the compressed weight (perm None: X already permuted)."""
+    T, cin = X.shape
+    cout = vals.shape[0]
+    Y = torch.empty(T, cout, dtype=torch.float32, device=X.device) if Y is None else Y
+    check(lib().lcp_sparse24_mm(_ptr(vals, X.dtype, "values"), _ptr(meta, torch.int32, "meta"), _ptr(X, None, "X"),
+                                _ptr(perm, torch.int32, "perm"), _ptr(Y, torch.float32, "Y"), cout, cin, T, block,
+                                _dt(X), _stream(None)))
+    return Y
 
 
 def calib_gemm(X: torch.Tensor, W: torch.Tensor, At: Optional[torch.Tensor], Yd: torch.Tensor,

@@ -610,6 +610,60 @@ lcp_status lcp_harden(const float* P_hat, int32_t* perm, float* P_hard, int nblo
   return launch_harden(P_hat, perm, P_hard, nullptr, nullptr, nullptr, nblocks, B, stream);
 }
 
+static lcp_status check_infer_shape(int cout, int cin, int B, bool need_block) {
+  if (cout < 1 || cout > kMaxDim) return fail(LCP_ERR_SHAPE, "C_out = %d", cout);
+  if (cin < 32 || cin % 32 || cin > kMaxDim) return fail(LCP_ERR_SHAPE, "C_in = %d must be a positive multiple of 32", cin);
+  if (need_block) {
+    if (B != 32 && B != 64 && B != 128 && B != 256)
+      return fail(LCP_ERR_SHAPE, "block size %d is not one of 32, 64, 128, 256", B);
+    if (cin % B) return fail(LCP_ERR_SHAPE, "C_in = %d is not a multiple of B = %d", cin, B);
+  }
+  return LCP_OK;
+}
+
+lcp_status lcp_pack24(const void* W, const int32_t* perm, const uint32_t* mask, void* values, uint32_t* meta,
+                      int cout, int cin, int B, lcp_dtype dtype, cudaStream_t stream) {
+  if (!W || !mask || !values || !meta) return fail(LCP_ERR_NULL, "W, mask, values and meta are required");
+  if (dtype != LCP_F32 && dtype != LCP_BF16) return fail(LCP_ERR_DTYPE, "unknown dtype %d", (int)dtype);
+  if (!perm && B == 0) B = 32;                       // no permutation: any block width of the columns
+  LCP_TRY(check_infer_shape(cout, cin, B, true));
+  if (!aligned16(W) || !aligned16(mask) || !aligned16(values) || !aligned16(meta) || (perm && !aligned16(perm)))
+    return fail(LCP_ERR_ARG, "pointers must be 16-byte aligned");
+  LCP_TRY(check_arch());
+  cudaGetLastError();
+  return launch_pack24(W, perm, mask, values, meta, cout, cin, B, dtype, stream);
+}
+
+lcp_status lcp_gather(const void* X, const int32_t* perm, void* Xp, int tokens, int cin, int B, lcp_dtype dtype,
+                      cudaStream_t stream) {
+  if (!X || !perm || !Xp) return fail(LCP_ERR_NULL, "X, perm and Xp are required");
+  if (dtype != LCP_F32 && dtype != LCP_BF16) return fail(LCP_ERR_DTYPE, "unknown dtype %d", (int)dtype);
+  LCP_TRY(check_infer_shape(1, cin, B, true));
+  if (tokens < 0 || tokens > kMaxDim) return fail(LCP_ERR_SHAPE, "T = %d", tokens);
+  if (X == Xp) return fail(LCP_ERR_ARG, "the gather is out of place: X and Xp must differ");
+  if (!aligned16(X) || !aligned16(Xp) || !aligned16(perm)) return fail(LCP_ERR_ARG, "pointers must be 16-byte aligned");
+  if (tokens == 0) return LCP_OK;
+  LCP_TRY(check_arch());
+  cudaGetLastError();
+  return launch_gather(X, perm, Xp, tokens, cin, B, dtype, stream);
+}
+
+lcp_status lcp_sparse24_mm(const void* values, const uint32_t* meta, const void* X, const int32_t* perm, float* Y,
+                           int cout, int cin, int tokens, int B, lcp_dtype dtype, cudaStream_t stream) {
+  if (!values || !meta || !X || !Y) return fail(LCP_ERR_NULL, "values, meta, X and Y are required");
+  if (dtype != LCP_F32 && dtype != LCP_BF16) return fail(LCP_ERR_DTYPE, "unknown dtype %d", (int)dtype);
+  LCP_TRY(check_infer_shape(cout, cin, B, perm != nullptr));
+  if (tokens < 0 || tokens > kMaxDim) return fail(LCP_ERR_SHAPE, "T = %d", tokens);
+  if (sparse24_tile_tokens(cin, tokens < 1 ? 1 : tokens, dtype == LCP_F32 ? 4 : 2) == 0)
+    return fail(LCP_ERR_SHAPE, "C_in = %d: one token's inputs do not fit in shared memory", cin);
+  if (!aligned16(values) || !aligned16(meta) || !aligned16(X) || (perm && !aligned16(perm)) || !aligned16(Y))
+    return fail(LCP_ERR_ARG, "pointers must be 16-byte aligned");
+  if (tokens == 0) return LCP_OK;
+  LCP_TRY(check_arch());
+  cudaGetLastError();
+  return launch_sparse24_mm(values, meta, X, perm, Y, cout, cin, tokens, B, dtype, stream);
+}
+
 lcp_status nm_mask(const void* Wp, uint32_t* mask_bits, int rows, int cols, int n, int m,
                    lcp_dtype dtype, cudaStream_t stream) {
   if (!Wp || !mask_bits) return fail(LCP_ERR_NULL, "Wp and mask_bits are required");
@@ -684,7 +738,8 @@ lcp_status lcp_loss_bwd(const float* Yd, const float* Ys, const float* stats, vo
 extern "C" lcp_status lcp_device_error(int* site, int reset) {
   using namespace lcp;
   if (!site) return fail(LCP_ERR_NULL, "site is NULL");
-  lcp_status (*const readers[])(int*, int) = {tc_error_gemm, tc_error_permute, tc_error_block_bwd, harden_error};
+  lcp_status (*const readers[])(int*, int) = {tc_error_gemm, tc_error_permute, tc_error_block_bwd, harden_error,
+                                               infer_error};
   int first = 0;
   for (auto rd : readers) {
     int v = 0;

@@ -202,6 +202,18 @@ lcp_status launch_score(const void* W, const void* X, void* S, float* stats, int
 lcp_status launch_adamw(float* L, const float* dL, float* m, float* v, long long n, double lr, double beta1,
                         double beta2, double eps, double weight_decay, int t, cudaStream_t st);
 
+// Inference side: the 2:4 compressed weight (values [cout, cin/2], meta
+// [cout, cin/32]) from W, the hard permutation and the mask bits; the input
+// gather x_pi = P_B^T x; the product Y = x_pi A^T ([tokens, cout] float32).
+lcp_status launch_pack24(const void* W, const int32_t* perm, const uint32_t* mask, void* vals, uint32_t* meta,
+                         int cout, int cin, int B, lcp_dtype dt, cudaStream_t st);
+lcp_status launch_gather(const void* X, const int32_t* perm, void* Xp, int tokens, int cin, int B, lcp_dtype dt,
+                         cudaStream_t st);
+lcp_status launch_sparse24_mm(const void* vals, const uint32_t* meta, const void* X, const int32_t* perm, float* Y,
+                              int cout, int cin, int tokens, int B, lcp_dtype dt, cudaStream_t st);
+int sparse24_tile_tokens(int cin, int tokens, int esize);   // 0: C_in too wide for one token
+lcp_status infer_error(int* site, int reset);
+
 // Device error words of the tensor-core translation units: the first wait
 // site that timed out since the last reset, 0 if none (cleared when `reset`).
 lcp_status tc_error_gemm(int* site, int reset);

@@ -111,6 +111,27 @@ def test_standalone_entry_points_validate_before_launch():
     assert L.lcp_sinkhorn_bwd(0x1000, 0x2000, 0x3000, 0, 0x4000, 1, 64, 1.0, 5, None) == 7
 
 
+def test_inference_entry_points_validate_before_launch():
+    L = b.lib()
+    # pack: W, mask, values, meta required; C_in a multiple of 32 and of B; B in {32, 64, 128, 256}
+    assert L.lcp_pack24(None, 0x1000, 0x2000, 0x3000, 0x4000, 8, 128, 64, 1, None) == 1
+    assert L.lcp_pack24(0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 8, 100, 64, 1, None) == 2
+    assert L.lcp_pack24(0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 8, 128, 48, 1, None) == 2
+    assert L.lcp_pack24(0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 8, 96, 64, 1, None) == 2
+    assert L.lcp_pack24(0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 8, 128, 64, 9, None) == 3
+    assert L.lcp_pack24(0x1008, 0x2000, 0x3000, 0x4000, 0x5000, 8, 128, 64, 1, None) == 7
+    # gather: perm required, out of place, empty token count is a no-op
+    assert L.lcp_gather(0x1000, None, 0x2000, 4, 128, 64, 1, None) == 1
+    assert L.lcp_gather(0x1000, 0x3000, 0x1000, 4, 128, 64, 1, None) == 7
+    assert L.lcp_gather(0x1000, 0x3000, 0x2000, 4, 128, 40, 1, None) == 2
+    assert L.lcp_gather(0x1000, 0x3000, 0x2000, 0, 128, 64, 1, None) == 0
+    # product: perm optional (B then unchecked), C_in too wide for one token's inputs
+    assert L.lcp_sparse24_mm(0x1000, None, 0x2000, None, 0x3000, 8, 128, 4, 64, 1, None) == 1
+    assert L.lcp_sparse24_mm(0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 8, 128, 4, 40, 1, None) == 2
+    assert L.lcp_sparse24_mm(0x1000, 0x2000, 0x3000, None, 0x5000, 8, 1 << 20, 1, 64, 1, None) == 2
+    assert L.lcp_sparse24_mm(0x1000, 0x2000, 0x3000, None, 0x5000, 8, 128, 0, 0, 1, None) == 0
+
+
 def test_launch_count_reported():
     hp = b.hparams(64, 2, 4, 5, 0.5, b.F32)
     arr = (b.LcpLayer * 2)(_layer(), _layer())
