@@ -739,7 +739,7 @@ extern "C" lcp_status lcp_device_error(int* site, int reset) {
   using namespace lcp;
   if (!site) return fail(LCP_ERR_NULL, "site is NULL");
   lcp_status (*const readers[])(int*, int) = {tc_error_gemm, tc_error_permute, tc_error_block_bwd, harden_error,
-                                               infer_error};
+                                               infer_error, tc_error_infer};
   int first = 0;
   for (auto rd : readers) {
     int v = 0;

@@ -16,13 +16,13 @@
 // Kernels:
 //   pack24_kernel    A from W, perm and the mask bits -> values, meta (offline);
 //   gather_kernel    x_pi for every token (the standalone permutation);
-//   sp24_mm_kernel   Y = x_pi A^T for a tile of up to 16 tokens, with the
-//                    gather fused into the staging of the inputs.  Decode-sized
-//                    token counts make this a stream over the compressed
-//                    weight (HBM-bound: 2 B per kept bf16 value + 1/8 B of
-//                    metadata per weight column), so it runs on the CUDA cores:
+//   sp24_mm_kernel   Y = x_pi A^T for a tile of up to 16 tokens on the CUDA
+//                    cores, the gather fused into the staging of the inputs:
 //                    one warp per output row, 16-byte value loads, the inputs
-//                    of the tile resident in shared memory.
+//                    of the tile resident in shared memory.  Used for float32,
+//                    for fewer than 8 tokens and for bf16 shapes the
+//                    tensor-core variant (infer24_tc.cu: C_in a multiple of 256)
+//                    does not take.
 
 #include "lcp_internal.cuh"
 
@@ -165,7 +165,8 @@ template <typename T, int TT> struct Sp24Cfg {
   static constexpr int PAD = U < 4 ? 4 : (U > 16 ? 16 : U);
   static constexpr int CHUNK = 16 * U + PAD;
   static constexpr int WARPS = TT >= 16 ? 8 : 16;   // 16 tokens: registers for 255 a thread
-  static constexpr int KP = 4;                     // chunks per lane per batch
+  // chunks per lane per batch
+  static constexpr int KP = 4;
   static constexpr int VU = (int)sizeof(T) / 2;    // 16-byte loads per chunk of values
 };
 
@@ -436,6 +437,11 @@ lcp_status launch_gather(const void* X, const int32_t* perm, void* Xp, int token
 lcp_status launch_sparse24_mm(const void* vals, const uint32_t* meta, const void* X, const int32_t* perm, float* Y,
                               int cout, int cin, int tokens, int B, lcp_dtype dt, cudaStream_t st) {
   const int bshift = perm ? log2_block(B) : 0;
+  // a handful of tokens: the CUDA-core kernel (its per-row stream has the shorter
+  // dependency chain); from 8 tokens on the tensor-core kernel
+  if (dt == LCP_BF16 && tokens >= 8 && sparse24_tc_splits(cout, cin) > 0)
+    return launch_sparse24_tc(static_cast<const __nv_bfloat16*>(vals), meta, static_cast<const __nv_bfloat16*>(X),
+                              perm, Y, cout, cin, tokens, bshift, st);
   if (dt == LCP_F32) return sp24_dispatch<float>(vals, meta, X, perm, Y, cout, cin, tokens, bshift, st);
   return sp24_dispatch<__nv_bfloat16>(vals, meta, X, perm, Y, cout, cin, tokens, bshift, st);
 }

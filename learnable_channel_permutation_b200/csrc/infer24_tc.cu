@@ -1,0 +1,279 @@
+// Deployed 2:4 product on the tensor cores (PermLLM summary, "Effect on
+// inference acceleration"): Y = x_pi A^T for up to 16 tokens, A kept in the
+// compressed form of infer24.cu (values [C_out, C_in/2], 4-bit position fields
+// [C_out, C_in/32]).
+//
+// The weight stays compressed in HBM (0.5625 of the dense bytes) and is
+// expanded to dense bf16 operand tiles in shared memory on the way to the MMA:
+//   - the CTA owns 128 output rows and a K range of C_in / S channels; the S
+//     CTAs of a row tile form a cluster;
+//   - TMA brings the compressed values (128 rows x 64 values, 128-byte
+//     swizzle) and the position words (128 rows x 4 words) of each 128-channel
+//     stage into a 4-stage ring;
+//   - 512 threads (four per row, 32 channels each) place every kept value at
+//     its position in two dense 128 x 64 K-major tiles (128-byte swizzle), zeros
+//     elsewhere;
+//   - one thread issues M = 128, N = 16 MMAs (the tokens, zero-padded to 16)
+//     against the inputs x_pi, staged once per launch in the same tile format
+//     with the gather applied;
+//   - the S partial accumulators are summed in rank order through distributed
+//     shared memory by the cluster's rank 0, which writes Y (deterministic, no
+//     workspace).
+
+#include "tc_common.cuh"
+
+namespace lcp {
+namespace {
+
+struct StCfg {
+  static constexpr int THREADS = 512;
+  static constexpr int STG = 4;                     // ring stages of 128 channels
+  static constexpr int V_BYTES = 128 * 128;         // 128 rows x 64 bf16 values
+  static constexpr int M_BYTES = 128 * 16;          // 128 rows x 4 position words
+  static constexpr int A_BYTES = 2 * 128 * 128;     // two dense 128 x 64 bf16 tiles
+  static constexpr int RED_BYTES = 16 * 128 * 4;    // 16 tokens x 128 rows float32
+  static constexpr int MAX_KR = 2048;               // channels per CTA (input image 64 KB)
+  static int smem(int kr) { return 2 * A_BYTES + STG * V_BYTES + (kr / 64) * 2048 + STG * M_BYTES + RED_BYTES + 256 + 1024; }
+};
+
+__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+__global__ void __launch_bounds__(StCfg::THREADS, 1)
+sp24_tc_kernel(const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmM,
+               const __nv_bfloat16* __restrict__ X, const int32_t* __restrict__ perm, float* __restrict__ Y,
+               int cout, int cin, int tokens, int bshift, int kr) {
+  using C = StCfg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sA = smem;                                   // 2 buffers x 32 KB
+  uint8_t* sV = sA + 2 * C::A_BYTES;                    // STG x 16 KB
+  uint8_t* sX = sV + C::STG * C::V_BYTES;               // kr / 64 blocks x 2 KB
+  uint8_t* sM = sX + (kr / 64) * 2048;                  // STG x 2 KB
+  float* sRed = reinterpret_cast<float*>(sM + C::STG * C::M_BYTES);   // [16][128]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sRed + 16 * 128);
+  uint32_t* holder = reinterpret_cast<uint32_t*>(bars + C::STG + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(holder + 1);
+  auto full = [&](int q) { return smem_u32(bars + q); };
+  auto done = [&](int b) { return smem_u32(bars + C::STG + b); };
+
+  const int tid = threadIdx.x, warp = tid / 32;
+  const int S = (int)gridDim.x;                         // cluster = the S splits of a row tile
+  const uint32_t rank = S > 1 ? cluster_rank() : 0u;
+  const int row0 = blockIdx.y * 128, k0 = (int)rank * kr;
+  const int nst = kr / 128;
+  if (tid == 0) {
+    for (int q = 0; q < C::STG; ++q) mbar_init(full(q), 1);
+    for (int b = 0; b < 2; ++b) mbar_init(done(b), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) tmem_alloc(smem_u32(holder), 32);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *holder;
+
+  // the weight does not come from the previous kernel: its first stages load at once
+  int last_issued[C::STG];                              // per ring slot, the last stage loaded into it
+#pragma unroll
+  for (int q = 0; q < C::STG; ++q) last_issued[q] = -1;
+  auto issue = [&](int j) {
+    const int q = j % C::STG;
+    mbar_expect_tx(full(q), C::V_BYTES + C::M_BYTES);
+    tma_load_2d(smem_u32(sV + q * C::V_BYTES), &tmV, full(q), (k0 + 128 * j) / 2, row0);
+    tma_load_2d(smem_u32(sM + q * C::M_BYTES), &tmM, full(q), (k0 + 128 * j) / 32, row0);
+    last_issued[q] = j;
+  };
+  if (tid == 0)
+    for (int j = 0; j < C::STG && j < nst; ++j) issue(j);
+  pdl_wait();
+  pdl_trigger();
+
+  // inputs x_pi of this K range, tokens zero-padded to 16: source channel i goes
+  // to slot s = (i & ~(B-1)) | perm[i]; element (t, s) of block (s - k0) / 64 at
+  // row t, 16-byte chunk ((s - k0) % 64) / 8 (swizzled), position (s - k0) % 8
+  {
+    const int Bm = perm ? (1 << bshift) - 1 : 0x7fffffff;
+    constexpr int KS = C::MAX_KR / C::THREADS;
+    __nv_bfloat16 e[KS][16];
+    int slot[KS];
+#pragma unroll
+    for (int m = 0; m < KS; ++m) {
+      const int il = tid + m * C::THREADS;
+      const int i = k0 + il;
+      const bool in = il < kr;
+      slot[m] = in ? (perm ? __ldg(perm + i) : (i & Bm)) : 0;
+#pragma unroll
+      for (int t = 0; t < 16; ++t)
+        e[m][t] = (in && t < tokens) ? X[(size_t)t * cin + i] : __float2bfloat16_rn(0.f);
+    }
+#pragma unroll
+    for (int m = 0; m < KS; ++m) {
+      const int il = tid + m * C::THREADS;
+      if (il >= kr) continue;
+      const int i = k0 + il;
+      if (slot[m] < 0 || slot[m] > Bm) {
+        atomicCAS(&g_tc_error, 0, 302);   // out-of-range permutation entry: skipped
+        continue;
+      }
+      const int loc = ((i & ~Bm) | slot[m]) - k0;
+      uint8_t* blk = sX + (loc >> 6) * 2048;
+      const int ch = (loc & 63) >> 3, pos = loc & 7;
+#pragma unroll
+      for (int t = 0; t < 16; ++t)
+        *reinterpret_cast<__nv_bfloat16*>(blk + t * 128 + ((ch ^ (t & 7)) << 4) + pos * 2) = e[m][t];
+    }
+  }
+  fence_async_smem();
+  __syncthreads();
+
+  // main loop: expand stage j into dense tile buffer j & 1, then the MMAs
+  constexpr uint32_t idesc = idesc_bf16(128, 16, false, false);
+  const int r = tid & 127, qt = tid >> 7;               // row of the tile, quarter of the stage
+  bool ok = true;
+  for (int j = 0; j < nst; ++j) {
+    const int q = j % C::STG, b = j & 1;
+    ok = ok && mbar_wait(full(q), (uint32_t)(j / C::STG) & 1u, abort_flag, 311);
+    if (j >= 2) ok = ok && mbar_wait(done(b), (uint32_t)((j - 2) >> 1) & 1u, abort_flag, 312);
+    if (ok) {
+      // this thread: channels 32 qt .. 32 qt + 31 of the stage = value chunks 2 qt, 2 qt + 1
+      const uint8_t* vrow = sV + q * C::V_BYTES + r * 128;
+      const uint4 v0 = *reinterpret_cast<const uint4*>(vrow + (((2 * qt) ^ (r & 7)) << 4));
+      const uint4 v1 = *reinterpret_cast<const uint4*>(vrow + (((2 * qt + 1) ^ (r & 7)) << 4));
+      const uint32_t f = *reinterpret_cast<const uint32_t*>(sM + q * C::M_BYTES + r * 16 + qt * 4);
+      const uint32_t vw[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};   // value pair of group g
+      uint8_t* tile = sA + b * C::A_BYTES + (qt >> 1) * (C::A_BYTES / 2);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {                     // dense chunk: groups 2c, 2c + 1 (8 channels)
+        uint32_t w[4];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int g = 2 * c + h;
+          const uint32_t fld = (f >> (4 * g)) & 0xFu;
+          const uint32_t p0 = fld & 3u, p1 = fld >> 2;
+          // the two kept values at their positions p of the group: word p / 2, half p % 2
+          const uint32_t a = (vw[g] & 0xFFFFu) << (16 * (p0 & 1u)), bv = (vw[g] >> 16) << (16 * (p1 & 1u));
+          w[2 * h] = (p0 < 2 ? a : 0u) | (p1 < 2 ? bv : 0u);
+          w[2 * h + 1] = (p0 >= 2 ? a : 0u) | (p1 >= 2 ? bv : 0u);
+        }
+        st_sw128(tile, r, (qt & 1) * 4 + c, make_uint4(w[0], w[1], w[2], w[3]));
+      }
+    }
+    fence_async_smem();
+    __syncthreads();
+    if (tid == 0 && ok) {
+      tc_fence_after();
+#pragma unroll
+      for (int tt = 0; tt < 2; ++tt) {
+        const uint32_t a0 = smem_u32(sA + b * C::A_BYTES + tt * (C::A_BYTES / 2));
+        const uint32_t b0 = smem_u32(sX + (2 * j + tt) * 2048);
+#pragma unroll
+        for (int k16 = 0; k16 < 4; ++k16)
+          mma_bf16(tmem, sdesc(a0 + k16 * 32, 16, 1024), sdesc(b0 + k16 * 32, 16, 1024), idesc,
+                   (j | tt | k16) != 0);
+      }
+      mma_commit(done(b));
+      if (j + C::STG < nst) issue(j + C::STG);   // stage q has been read by every thread
+    }
+  }
+  // every product has landed once the last stage's commit arrives
+  if (ok && nst > 0) ok = mbar_wait(done((nst - 1) & 1), (uint32_t)((nst - 1) >> 1) & 1u, abort_flag, 313);
+  if (warp < 4) {
+    tc_fence_after();
+    uint32_t acc[16];
+    tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16), acc);
+    tmem_ld_wait();
+#pragma unroll
+    for (int t = 0; t < 16; ++t) sRed[t * 128 + r] = (ok && nst > 0) ? __uint_as_float(acc[t]) : 0.f;
+  }
+  // drain: copies this CTA started and nobody consumed (only after an abort)
+  if (tid == 0 && !ok)
+    for (int q = 0; q < C::STG; ++q)
+      if (last_issued[q] >= 0) mbar_wait_drain(full(q), (uint32_t)(last_issued[q] / C::STG) & 1u, 314);
+  tc_fence_before();
+  if (S == 1) {
+    __syncthreads();
+    for (int idx = tid; idx < 16 * 128; idx += C::THREADS) {
+      const int t = idx >> 7, rr = idx & 127;
+      if (t < tokens && row0 + rr < cout) Y[(size_t)t * cout + row0 + rr] = sRed[idx];
+    }
+  } else {
+    cluster_sync_all();                                 // partials visible cluster-wide
+    if (rank == 0) {
+      const uint32_t red = smem_u32(sRed);
+      for (int idx = tid; idx < 16 * 128; idx += C::THREADS) {
+        const int t = idx >> 7, rr = idx & 127;
+        if (t >= tokens || row0 + rr >= cout) continue;
+        float v = 0.f;
+        for (int q = 0; q < S; ++q) v += ld_cluster_f32(mapa(red + idx * 4, (uint32_t)q));
+        Y[(size_t)t * cout + row0 + rr] = v;
+      }
+    }
+    cluster_sync_all();                                 // peers keep their partials until read
+  }
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 32);
+  }
+}
+
+// 2-D uint32 tensor map, no swizzle
+lcp_status make_map_u32(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t bx, uint32_t by,
+                        const char* what) {
+  EncodeFn fn = encode_fn();
+  if (!fn) return fail(LCP_ERR_CUDA, "%s: cuTensorMapEncodeTiled is unavailable from the driver", what);
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {inner * 4};
+  const cuuint32_t box[2] = {bx, by};
+  const cuuint32_t es[2] = {1, 1};
+  const CUresult res = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(base), dims, strides, box, es,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (res != CUDA_SUCCESS) return fail(LCP_ERR_CUDA, "%s: cuTensorMapEncodeTiled failed (%d)", what, (int)res);
+  return LCP_OK;
+}
+
+}  // namespace
+
+lcp_status tc_error_infer(int* site, int reset) { return read_tc_error(site, reset); }
+
+// Splits of C_in for the tensor-core product (0: the shape is not supported):
+// S in {1, 2, 4} with C_in / S a multiple of 256 and at most 2048, as many as
+// keep the grid (S x row tiles) within one wave of the SMs.
+int sparse24_tc_splits(int cout, int cin) {
+  if (cin % 256) return 0;
+  const int tiles = cdiv(cout, 128);
+  int best = 0;
+  for (int s = 1; s <= 4; s *= 2) {
+    if (cin % (256 * s) || cin / s > StCfg::MAX_KR) continue;
+    if (best == 0) best = s;                            // the fewest splits that fit
+    else if (tiles * s <= num_sms()) best = s;          // more, while one wave holds them
+  }
+  return best;
+}
+
+lcp_status launch_sparse24_tc(const __nv_bfloat16* vals, const uint32_t* meta, const __nv_bfloat16* X,
+                              const int32_t* perm, float* Y, int cout, int cin, int tokens, int bshift,
+                              cudaStream_t st) {
+  const int S = sparse24_tc_splits(cout, cin);
+  if (S == 0) return fail(LCP_ERR_SHAPE, "sparse24 tensor-core path: C_in = %d is not supported", cin);
+  const int kr = cin / S;
+  CUtensorMap mV, mM;
+  TC_TRY(make_map(&mV, vals, (uint64_t)cin / 2, (uint64_t)cout, 64, 128, "sparse24 values"));
+  TC_TRY(make_map_u32(&mM, meta, (uint64_t)cin / 32, (uint64_t)cout, 4, 128, "sparse24 positions"));
+  const int smem = StCfg::smem(kr);
+  TC_TRY(set_smem(sp24_tc_kernel, smem, "sparse24_tc"));
+  const dim3 grid((unsigned)S, (unsigned)cdiv(cout, 128));
+  for (int t0 = 0; t0 < tokens; t0 += 16) {
+    const int tt = tokens - t0 < 16 ? tokens - t0 : 16;
+    TC_TRY(launch_kernel(sp24_tc_kernel, grid, dim3(StCfg::THREADS), smem, st, S, true, "sparse24_tc", mV, mM,
+                         X + (size_t)t0 * cin, perm, Y + (size_t)t0 * cout, cout, cin, tt, bshift, kr));
+  }
+  return LCP_OK;
+}
+
+}  // namespace lcp

@@ -212,6 +212,12 @@ lcp_status launch_gather(const void* X, const int32_t* perm, void* Xp, int token
 lcp_status launch_sparse24_mm(const void* vals, const uint32_t* meta, const void* X, const int32_t* perm, float* Y,
                               int cout, int cin, int tokens, int B, lcp_dtype dt, cudaStream_t st);
 int sparse24_tile_tokens(int cin, int tokens, int esize);   // 0: C_in too wide for one token
+// the same product on the tensor cores (bf16; C_in splits from sparse24_tc_splits, 0 = unsupported)
+int sparse24_tc_splits(int cout, int cin);
+lcp_status launch_sparse24_tc(const __nv_bfloat16* vals, const uint32_t* meta, const __nv_bfloat16* X,
+                              const int32_t* perm, float* Y, int cout, int cin, int tokens, int bshift,
+                              cudaStream_t st);
+lcp_status tc_error_infer(int* site, int reset);
 lcp_status infer_error(int* site, int reset);
 
 // Device error words of the tensor-core translation units: the first wait

@@ -117,20 +117,37 @@ def test_sparse24_mm_matches_the_oracle(gpu_lib, dtype, T, fused):
     assert b.device_error() == 0
 
 
-@pytest.mark.parametrize("B", [32, 256])
-def test_sparse24_mm_block_sizes_and_wide_rows(gpu_lib, B):
+@pytest.mark.parametrize("T", [1, 5, 16])
+def test_sparse24_mm_cuda_core_path(gpu_lib, T):
+    """bf16 with C_in not a multiple of 256 takes the CUDA-core kernel at every
+    token count (the other cases cover it below 8 tokens and the tensor-core
+    kernel from 8 on)."""
+    cout, cin, B = 72, 1120, 32
+    W, perm, Wp, M = _case(cout, cin, B, "bf16", seed=40 + T)
+    vals, meta, pd = _pack_gpu(W, perm, M, B, "bf16")
+    rng = np.random.default_rng(41 + T)
+    X = torch.from_numpy(rng.normal(size=(T, cin))).to(torch.bfloat16)
+    Y = b.sparse24_mm(vals, meta, X.cuda(), pd, B)
+    torch.cuda.synchronize()
+    rv, ri = O.pack_24(Wp, M)
+    _check_product(Y.cpu().numpy().astype(np.float64), rv, ri, X.float().numpy().astype(np.float64), perm)
+    assert b.device_error() == 0
+
+
+@pytest.mark.parametrize("B,T", [(32, 4), (256, 4), (32, 12), (256, 12)])
+def test_sparse24_mm_block_sizes_and_wide_rows(gpu_lib, B, T):
     cout, cin = 48, 8192
     W, perm, Wp, M = _case(cout, cin, B, "bf16", seed=B)
     vals, meta, pd = _pack_gpu(W, perm, M, B, "bf16")
     rng = np.random.default_rng(B + 1)
-    X = torch.from_numpy(rng.normal(size=(4, cin))).to(torch.bfloat16)
+    X = torch.from_numpy(rng.normal(size=(T, cin))).to(torch.bfloat16)
     Y = b.sparse24_mm(vals, meta, X.cuda(), pd, B)
     torch.cuda.synchronize()
     rv, ri = O.pack_24(Wp, M)
     _check_product(Y.cpu().numpy().astype(np.float64), rv, ri, X.float().numpy().astype(np.float64), perm)
 
 
-@pytest.mark.parametrize("T", [1, 16])
+@pytest.mark.parametrize("T", [1, 8, 16, 40])
 def test_sparse24_mm_full_size_q_proj(gpu_lib, T):
     """The 4096 x 4096 layer of the calibration workload (outlier channels,
     bf16), decode-sized token counts, every output against the oracle."""
