@@ -10,15 +10,14 @@
 //   - TMA brings the compressed values (128 rows x 64 values, 128-byte
 //     swizzle) and the position words (128 rows x 4 words) of each 128-channel
 //     stage into a 4-stage ring;
-//   - 512 threads (four per row, 32 channels each) place every kept value at
-//     its position in two dense 128 x 64 K-major tiles (128-byte swizzle), zeros
-//     elsewhere;
-//   - one thread issues M = 128, N = 16 MMAs (the tokens, zero-padded to 16)
+//   - 16 expander warps (four threads per row, 2 x 16 channels each) place every
+//     kept value at its position in two dense 128 x 64 K-major tiles (128-byte
+//     swizzle), zeros elsewhere, into one of two operand buffers;
+//   - an MMA warp issues M = 128, N = 16 MMAs (the tokens, zero-padded to 16)
 //     against the inputs x_pi, staged once per launch in the same tile format
 //     with the gather applied;
 //   - the S partial accumulators are summed in rank order through distributed
-//     shared memory by the cluster's rank 0, which writes Y (deterministic, no
-//     workspace).
+//     shared memory, each rank writing 1/S of Y (deterministic, no workspace).
 
 #include "tc_common.cuh"
 
@@ -26,14 +25,21 @@ namespace lcp {
 namespace {
 
 struct StCfg {
-  static constexpr int THREADS = 512;
+  static constexpr int EXP_WARPS = 16;              // expanders (four threads per row of the tile)
+  static constexpr int PROD_WARP = EXP_WARPS, MMA_WARP = EXP_WARPS + 1;
+  static constexpr int THREADS = 32 * (EXP_WARPS + 2);
+  static constexpr int EXP_THREADS = 32 * EXP_WARPS;
   static constexpr int STG = 4;                     // ring stages of 128 channels
+  static constexpr int NA = 2;                      // dense operand buffers
   static constexpr int V_BYTES = 128 * 128;         // 128 rows x 64 bf16 values
   static constexpr int M_BYTES = 128 * 16;          // 128 rows x 4 position words
   static constexpr int A_BYTES = 2 * 128 * 128;     // two dense 128 x 64 bf16 tiles
   static constexpr int RED_BYTES = 16 * 128 * 4;    // 16 tokens x 128 rows float32
   static constexpr int MAX_KR = 2048;               // channels per CTA (input image 64 KB)
-  static int smem(int kr) { return 2 * A_BYTES + STG * V_BYTES + (kr / 64) * 2048 + STG * M_BYTES + RED_BYTES + 256 + 1024; }
+  static constexpr int NBAR = 2 * STG + 2 * NA + 1;
+  static int smem(int kr) {
+    return NA * A_BYTES + STG * V_BYTES + (kr / 64) * 2048 + STG * M_BYTES + RED_BYTES + 256 + 1024;
+  }
 };
 
 __device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
@@ -42,6 +48,14 @@ __device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
   return v;
 }
 
+// Roles (18 warps): warp 16 loads the ring (TMA), warp 17 issues the MMAs,
+// warps 0-15 stage the inputs, then expand each stage into a dense operand
+// buffer; they meet only through mbarriers:
+//   full[q]  (TMA bytes)        ring slot q holds stage j       -> expanders
+//   empty[q] (16 warp arrivals) every expander has read slot q  -> producer
+//   aready[b] (16 warp arrivals) dense buffer b holds stage j   -> MMA warp
+//   adone[b] (MMA commit)       the products reading b are done -> expanders
+//   fin      (MMA commit)       every product has landed        -> epilogue
 __global__ void __launch_bounds__(StCfg::THREADS, 1)
 sp24_tc_kernel(const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmM,
                const __nv_bfloat16* __restrict__ X, const int32_t* __restrict__ perm, float* __restrict__ Y,
@@ -49,152 +63,206 @@ sp24_tc_kernel(const __grid_constant__ CUtensorMap tmV, const __grid_constant__ 
   using C = StCfg;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
-  uint8_t* sA = smem;                                   // 2 buffers x 32 KB
-  uint8_t* sV = sA + 2 * C::A_BYTES;                    // STG x 16 KB
+  uint8_t* sA = smem;                                   // NA buffers x 32 KB
+  uint8_t* sV = sA + C::NA * C::A_BYTES;                // STG x 16 KB
   uint8_t* sX = sV + C::STG * C::V_BYTES;               // kr / 64 blocks x 2 KB
   uint8_t* sM = sX + (kr / 64) * 2048;                  // STG x 2 KB
   float* sRed = reinterpret_cast<float*>(sM + C::STG * C::M_BYTES);   // [16][128]
   uint64_t* bars = reinterpret_cast<uint64_t*>(sRed + 16 * 128);
-  uint32_t* holder = reinterpret_cast<uint32_t*>(bars + C::STG + 2);
+  uint32_t* holder = reinterpret_cast<uint32_t*>(bars + C::NBAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(holder + 1);
   auto full = [&](int q) { return smem_u32(bars + q); };
-  auto done = [&](int b) { return smem_u32(bars + C::STG + b); };
+  auto empty = [&](int q) { return smem_u32(bars + C::STG + q); };
+  auto aready = [&](int b) { return smem_u32(bars + 2 * C::STG + b); };
+  auto adone = [&](int b) { return smem_u32(bars + 2 * C::STG + C::NA + b); };
+  const uint32_t fin = smem_u32(bars + 2 * C::STG + 2 * C::NA);
 
-  const int tid = threadIdx.x, warp = tid / 32;
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const int S = (int)gridDim.x;                         // cluster = the S splits of a row tile
   const uint32_t rank = S > 1 ? cluster_rank() : 0u;
   const int row0 = blockIdx.y * 128, k0 = (int)rank * kr;
   const int nst = kr / 128;
   if (tid == 0) {
-    for (int q = 0; q < C::STG; ++q) mbar_init(full(q), 1);
-    for (int b = 0; b < 2; ++b) mbar_init(done(b), 1);
+    for (int q = 0; q < C::STG; ++q) {
+      mbar_init(full(q), 1);
+      mbar_init(empty(q), C::EXP_WARPS);
+    }
+    for (int b = 0; b < C::NA; ++b) {
+      mbar_init(aready(b), C::EXP_WARPS);
+      mbar_init(adone(b), 1);
+    }
+    mbar_init(fin, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0) tmem_alloc(smem_u32(holder), 32);
+  if (warp == C::MMA_WARP) tmem_alloc(smem_u32(holder), 32);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *holder;
-
-  // the weight does not come from the previous kernel: its first stages load at once
-  int last_issued[C::STG];                              // per ring slot, the last stage loaded into it
-#pragma unroll
-  for (int q = 0; q < C::STG; ++q) last_issued[q] = -1;
-  auto issue = [&](int j) {
-    const int q = j % C::STG;
-    mbar_expect_tx(full(q), C::V_BYTES + C::M_BYTES);
-    tma_load_2d(smem_u32(sV + q * C::V_BYTES), &tmV, full(q), (k0 + 128 * j) / 2, row0);
-    tma_load_2d(smem_u32(sM + q * C::M_BYTES), &tmM, full(q), (k0 + 128 * j) / 32, row0);
-    last_issued[q] = j;
-  };
-  if (tid == 0)
-    for (int j = 0; j < C::STG && j < nst; ++j) issue(j);
-  pdl_wait();
-  pdl_trigger();
-
-  // inputs x_pi of this K range, tokens zero-padded to 16: source channel i goes
-  // to slot s = (i & ~(B-1)) | perm[i]; element (t, s) of block (s - k0) / 64 at
-  // row t, 16-byte chunk ((s - k0) % 64) / 8 (swizzled), position (s - k0) % 8
-  {
-    const int Bm = perm ? (1 << bshift) - 1 : 0x7fffffff;
-    constexpr int KS = C::MAX_KR / C::THREADS;
-    __nv_bfloat16 e[KS][16];
-    int slot[KS];
-#pragma unroll
-    for (int m = 0; m < KS; ++m) {
-      const int il = tid + m * C::THREADS;
-      const int i = k0 + il;
-      const bool in = il < kr;
-      slot[m] = in ? (perm ? __ldg(perm + i) : (i & Bm)) : 0;
-#pragma unroll
-      for (int t = 0; t < 16; ++t)
-        e[m][t] = (in && t < tokens) ? X[(size_t)t * cin + i] : __float2bfloat16_rn(0.f);
-    }
-#pragma unroll
-    for (int m = 0; m < KS; ++m) {
-      const int il = tid + m * C::THREADS;
-      if (il >= kr) continue;
-      const int i = k0 + il;
-      if (slot[m] < 0 || slot[m] > Bm) {
-        atomicCAS(&g_tc_error, 0, 302);   // out-of-range permutation entry: skipped
-        continue;
-      }
-      const int loc = ((i & ~Bm) | slot[m]) - k0;
-      uint8_t* blk = sX + (loc >> 6) * 2048;
-      const int ch = (loc & 63) >> 3, pos = loc & 7;
-#pragma unroll
-      for (int t = 0; t < 16; ++t)
-        *reinterpret_cast<__nv_bfloat16*>(blk + t * 128 + ((ch ^ (t & 7)) << 4) + pos * 2) = e[m][t];
-    }
-  }
-  fence_async_smem();
-  __syncthreads();
-
-  // main loop: expand stage j into dense tile buffer j & 1, then the MMAs
-  constexpr uint32_t idesc = idesc_bf16(128, 16, false, false);
-  const int r = tid & 127, qt = tid >> 7;               // row of the tile, quarter of the stage
   bool ok = true;
-  for (int j = 0; j < nst; ++j) {
-    const int q = j % C::STG, b = j & 1;
-    ok = ok && mbar_wait(full(q), (uint32_t)(j / C::STG) & 1u, abort_flag, 311);
-    if (j >= 2) ok = ok && mbar_wait(done(b), (uint32_t)((j - 2) >> 1) & 1u, abort_flag, 312);
-    if (ok) {
-      // this thread: channels 32 qt .. 32 qt + 31 of the stage = value chunks 2 qt, 2 qt + 1
-      const uint8_t* vrow = sV + q * C::V_BYTES + r * 128;
-      const uint4 v0 = *reinterpret_cast<const uint4*>(vrow + (((2 * qt) ^ (r & 7)) << 4));
-      const uint4 v1 = *reinterpret_cast<const uint4*>(vrow + (((2 * qt + 1) ^ (r & 7)) << 4));
-      const uint32_t f = *reinterpret_cast<const uint32_t*>(sM + q * C::M_BYTES + r * 16 + qt * 4);
-      const uint32_t vw[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};   // value pair of group g
-      uint8_t* tile = sA + b * C::A_BYTES + (qt >> 1) * (C::A_BYTES / 2);
+
+  if (warp == C::PROD_WARP) {
+    // the weight does not come from the previous kernel: the ring fills at once
+    if (lane == 0) {
+      int last_issued[C::STG];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {                     // dense chunk: groups 2c, 2c + 1 (8 channels)
-        uint32_t w[4];
+      for (int q = 0; q < C::STG; ++q) last_issued[q] = -1;
+      for (int j = 0; j < nst; ++j) {
+        const int q = j % C::STG;
+        if (j >= C::STG && !mbar_wait(empty(q), (uint32_t)((j - C::STG) / C::STG) & 1u, abort_flag, 311)) break;
+        mbar_expect_tx(full(q), C::V_BYTES + C::M_BYTES);
+        tma_load_2d(smem_u32(sV + q * C::V_BYTES), &tmV, full(q), (k0 + 128 * j) / 2, row0);
+        tma_load_2d(smem_u32(sM + q * C::M_BYTES), &tmM, full(q), (k0 + 128 * j) / 32, row0);
+        last_issued[q] = j;
+      }
+      // every copy started here lands before the CTA moves on
+      for (int q = 0; q < C::STG; ++q)
+        if (last_issued[q] >= 0) mbar_wait_drain(full(q), (uint32_t)(last_issued[q] / C::STG) & 1u, 314);
+    }
+    __syncwarp();
+    pdl_wait();
+    pdl_trigger();
+  } else if (warp == C::MMA_WARP) {
+    pdl_wait();
+    pdl_trigger();
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(128, 16, false, false);
+      int j = 0;
+      for (; j < nst; ++j) {
+        const int b = j % C::NA;
+        if (!mbar_wait(aready(b), (uint32_t)(j / C::NA) & 1u, abort_flag, 312)) break;
+        tc_fence_after();
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int g = 2 * c + h;
-          const uint32_t fld = (f >> (4 * g)) & 0xFu;
-          const uint32_t p0 = fld & 3u, p1 = fld >> 2;
-          // the two kept values at their positions p of the group: word p / 2, half p % 2
-          const uint32_t a = (vw[g] & 0xFFFFu) << (16 * (p0 & 1u)), bv = (vw[g] >> 16) << (16 * (p1 & 1u));
-          w[2 * h] = (p0 < 2 ? a : 0u) | (p1 < 2 ? bv : 0u);
-          w[2 * h + 1] = (p0 >= 2 ? a : 0u) | (p1 >= 2 ? bv : 0u);
+        for (int tt = 0; tt < 2; ++tt) {
+          const uint32_t a0 = smem_u32(sA + b * C::A_BYTES + tt * (C::A_BYTES / 2));
+          const uint32_t b0 = smem_u32(sX + (2 * j + tt) * 2048);
+#pragma unroll
+          for (int k16 = 0; k16 < 4; ++k16)
+            mma_bf16(tmem, sdesc(a0 + k16 * 32, 16, 1024), sdesc(b0 + k16 * 32, 16, 1024), idesc,
+                     (j | tt | k16) != 0);
         }
-        st_sw128(tile, r, (qt & 1) * 4 + c, make_uint4(w[0], w[1], w[2], w[3]));
+        mma_commit(adone(b));
+      }
+      mma_commit(fin);                                  // arrives once every issued product is done
+    }
+    __syncwarp();
+  } else {
+    // inputs x_pi of this K range, tokens zero-padded to 16: source channel i goes
+    // to slot s = (i & ~(B-1)) | perm[i]; element (t, s) of block (s - k0) / 64 at
+    // row t, 16-byte chunk ((s - k0) % 64) / 8 (swizzled), position (s - k0) % 8.
+    // Thread = (run c of 8 source channels, token group): the run's slots (two
+    // 16-byte loads) and x of tokens g, g + G, ... (one 16-byte load each), every
+    // load issued before the stores.
+    {
+      const int Bm = perm ? (1 << bshift) - 1 : 0x7fffffff;
+      const int runs = kr / 8;                          // 32 .. 256
+      const int G = C::EXP_THREADS / runs;              // token groups: 16 .. 2
+      constexpr int TPT = 16 * C::MAX_KR / 8 / C::EXP_THREADS;   // tokens per thread at most (8)
+      const int c = tid % runs, g = tid / runs;
+      const int i0 = k0 + c * 8;
+      int4 pv[2] = {make_int4(0, 0, 0, 0), make_int4(0, 0, 0, 0)};
+      if (perm) {                                       // the permutation is no kernel's output
+        pv[0] = __ldg(reinterpret_cast<const int4*>(perm + i0));
+        pv[1] = __ldg(reinterpret_cast<const int4*>(perm + i0) + 1);
+      }
+      pdl_wait();
+      pdl_trigger();
+      uint4 xv[TPT];
+#pragma unroll
+      for (int m = 0; m < TPT; ++m) {
+        const int t = g + m * G;
+        xv[m] = make_uint4(0u, 0u, 0u, 0u);
+        if (t < 16 && t < tokens) xv[m] = __ldg(reinterpret_cast<const uint4*>(X + (size_t)t * cin + i0));
+      }
+      const int* pk = reinterpret_cast<const int*>(&pv[0]);
+      int loc[8];
+#pragma unroll
+      for (int v = 0; v < 8; ++v) {
+        const int i = i0 + v;
+        const int p = perm ? pk[v] : (i & Bm);
+        if (p < 0 || p > Bm) {
+          atomicCAS(&g_tc_error, 0, 302);   // out-of-range permutation entry: skipped
+          loc[v] = -1;
+        } else {
+          loc[v] = ((i & ~Bm) | p) - k0;
+        }
+      }
+#pragma unroll
+      for (int m = 0; m < TPT; ++m) {
+        const int t = g + m * G;
+        if (t >= 16) continue;
+        const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&xv[m]);
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+          if (loc[v] < 0) continue;
+          const int ch = (loc[v] & 63) >> 3, pos = loc[v] & 7;
+          *reinterpret_cast<__nv_bfloat16*>(sX + (loc[v] >> 6) * 2048 + t * 128 + ((ch ^ (t & 7)) << 4) + pos * 2) =
+              e[v];
+        }
       }
     }
     fence_async_smem();
-    __syncthreads();
-    if (tid == 0 && ok) {
-      tc_fence_after();
+
+    // expand stage j into dense buffer j % NA: thread = (row r, eighths e and e + 4
+    // of the 128 channels: value chunk e, 16 channels = dense chunks 2e, 2e + 1)
+    const int r = tid & 127;
+    for (int j = 0; j < nst; ++j) {
+      const int q = j % C::STG, b = j % C::NA;
+      ok = ok && warp_all(mbar_wait(full(q), (uint32_t)(j / C::STG) & 1u, abort_flag, 315));
+      if (j >= C::NA)
+        ok = ok && warp_all(mbar_wait(adone(b), (uint32_t)((j - C::NA) / C::NA) & 1u, abort_flag, 316));
+      if (!ok) break;
+      constexpr int EPT = 1024 / C::EXP_THREADS;        // eighths per thread
+      uint4 v[EPT];
+      uint32_t fh[EPT];
 #pragma unroll
-      for (int tt = 0; tt < 2; ++tt) {
-        const uint32_t a0 = smem_u32(sA + b * C::A_BYTES + tt * (C::A_BYTES / 2));
-        const uint32_t b0 = smem_u32(sX + (2 * j + tt) * 2048);
-#pragma unroll
-        for (int k16 = 0; k16 < 4; ++k16)
-          mma_bf16(tmem, sdesc(a0 + k16 * 32, 16, 1024), sdesc(b0 + k16 * 32, 16, 1024), idesc,
-                   (j | tt | k16) != 0);
+      for (int k = 0; k < EPT; ++k) {
+        const int e8 = (tid >> 7) + k * (C::EXP_THREADS / 128);
+        v[k] = *reinterpret_cast<const uint4*>(sV + q * C::V_BYTES + r * 128 + ((e8 ^ (r & 7)) << 4));
+        fh[k] = *reinterpret_cast<const uint16_t*>(sM + q * C::M_BYTES + r * 16 + e8 * 2);
       }
-      mma_commit(done(b));
-      if (j + C::STG < nst) issue(j + C::STG);   // stage q has been read by every thread
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty(q));             // this warp is done with ring slot q
+#pragma unroll
+      for (int k = 0; k < EPT; ++k) {
+        const int e8 = (tid >> 7) + k * (C::EXP_THREADS / 128);
+        const uint32_t f = fh[k];
+        const uint32_t vw[4] = {v[k].x, v[k].y, v[k].z, v[k].w};   // value pair of group g
+        uint8_t* tile = sA + b * C::A_BYTES + (e8 >> 2) * (C::A_BYTES / 2);
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {                     // dense chunk: groups 2c, 2c + 1 (8 channels)
+          uint32_t w[4];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int g = 2 * c + h;
+            const uint32_t fld = (f >> (4 * g)) & 0xFu;
+            const uint32_t p0 = fld & 3u, p1 = fld >> 2;
+            // the two kept values at their positions p of the group: word p / 2, half p % 2
+            const uint32_t a = (vw[g] & 0xFFFFu) << (16 * (p0 & 1u)), bv = (vw[g] >> 16) << (16 * (p1 & 1u));
+            w[2 * h] = (p0 < 2 ? a : 0u) | (p1 < 2 ? bv : 0u);
+            w[2 * h + 1] = (p0 >= 2 ? a : 0u) | (p1 >= 2 ? bv : 0u);
+          }
+          st_sw128(tile, r, (e8 & 3) * 2 + c, make_uint4(w[0], w[1], w[2], w[3]));
+        }
+      }
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(aready(b));
+    }
+    // epilogue: four warps, one per TMEM lane quadrant (warp w reads lanes 32 (w % 4) ..)
+    if (warp < 4) {
+      const bool got = ok && nst > 0 && warp_all(mbar_wait(fin, 0, abort_flag, 313));
+      tc_fence_after();
+      uint32_t acc[16];
+      tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16), acc);
+      tmem_ld_wait();
+#pragma unroll
+      for (int t = 0; t < 16; ++t) sRed[t * 128 + warp * 32 + lane] = got ? __uint_as_float(acc[t]) : 0.f;
     }
   }
-  // every product has landed once the last stage's commit arrives
-  if (ok && nst > 0) ok = mbar_wait(done((nst - 1) & 1), (uint32_t)((nst - 1) >> 1) & 1u, abort_flag, 313);
-  if (warp < 4) {
-    tc_fence_after();
-    uint32_t acc[16];
-    tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16), acc);
-    tmem_ld_wait();
-#pragma unroll
-    for (int t = 0; t < 16; ++t) sRed[t * 128 + r] = (ok && nst > 0) ? __uint_as_float(acc[t]) : 0.f;
-  }
-  // drain: copies this CTA started and nobody consumed (only after an abort)
-  if (tid == 0 && !ok)
-    for (int q = 0; q < C::STG; ++q)
-      if (last_issued[q] >= 0) mbar_wait_drain(full(q), (uint32_t)(last_issued[q] / C::STG) & 1u, 314);
   tc_fence_before();
+  // the S partials are summed in rank order; rank q writes the outputs [q, q + 1) * 2048 / S
   if (S == 1) {
     __syncthreads();
     for (int idx = tid; idx < 16 * 128; idx += C::THREADS) {
@@ -203,19 +271,18 @@ sp24_tc_kernel(const __grid_constant__ CUtensorMap tmV, const __grid_constant__ 
     }
   } else {
     cluster_sync_all();                                 // partials visible cluster-wide
-    if (rank == 0) {
-      const uint32_t red = smem_u32(sRed);
-      for (int idx = tid; idx < 16 * 128; idx += C::THREADS) {
-        const int t = idx >> 7, rr = idx & 127;
-        if (t >= tokens || row0 + rr >= cout) continue;
-        float v = 0.f;
-        for (int q = 0; q < S; ++q) v += ld_cluster_f32(mapa(red + idx * 4, (uint32_t)q));
-        Y[(size_t)t * cout + row0 + rr] = v;
-      }
+    const uint32_t red = smem_u32(sRed);
+    const int per = 16 * 128 / S, base = (int)rank * per;
+    for (int idx = base + tid; idx < base + per; idx += C::THREADS) {
+      const int t = idx >> 7, rr = idx & 127;
+      if (t >= tokens || row0 + rr >= cout) continue;
+      float v = 0.f;
+      for (int q = 0; q < S; ++q) v += ld_cluster_f32(mapa(red + idx * 4, (uint32_t)q));
+      Y[(size_t)t * cout + row0 + rr] = v;
     }
     cluster_sync_all();                                 // peers keep their partials until read
   }
-  if (warp == 0) {
+  if (warp == C::MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem, 32);
   }
