@@ -292,7 +292,8 @@ LCP_API lcp_status lcp_gather(const void* X, const int32_t* perm, void* Xp, int 
  * (original channel order when perm is given, already permuted when perm is
  * NULL), values / meta as above, Y [T, C_out] float32 (float32 accumulation).
  * Built for decode-sized T (tiles of up to 16 tokens; larger T runs tile by
- * tile, re-streaming the weight); C_in up to 102400 (bf16) / 51200 (float32). */
+ * tile, re-streaming the weight).  One token's inputs must fit in 200 KB of
+ * shared memory: C_in <= 91008 (bf16) / 48160 (float32), else LCP_ERR_SHAPE. */
 LCP_API lcp_status lcp_sparse24_mm(const void* values, const uint32_t* meta, const void* X, const int32_t* perm,
                                    float* Y, int cout, int cin, int tokens, int B, lcp_dtype dtype,
                                    cudaStream_t stream);

@@ -21,8 +21,8 @@
 //                    one warp per output row, 16-byte value loads, the inputs
 //                    of the tile resident in shared memory.  Used for float32,
 //                    for fewer than 8 tokens and for bf16 shapes the
-//                    tensor-core variant (infer24_tc.cu: C_in a multiple of 256)
-//                    does not take.
+//                    tensor-core variant (infer24_tc.cu: C_in a multiple of 256,
+//                    at most 8192) does not take.
 
 #include "lcp_internal.cuh"
 

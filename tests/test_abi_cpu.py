@@ -130,6 +130,11 @@ def test_inference_entry_points_validate_before_launch():
     assert L.lcp_sparse24_mm(0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 8, 128, 4, 40, 1, None) == 2
     assert L.lcp_sparse24_mm(0x1000, 0x2000, 0x3000, None, 0x5000, 8, 1 << 20, 1, 64, 1, None) == 2
     assert L.lcp_sparse24_mm(0x1000, 0x2000, 0x3000, None, 0x5000, 8, 128, 0, 0, 1, None) == 0
+    # the widest rows whose one-token input image fits the 200 KB tile (bf16, float32)
+    assert L.lcp_sparse24_mm(0x1000, 0x2000, 0x3000, None, 0x5000, 8, 91008 + 32, 1, 0, 1, None) == 2
+    assert L.lcp_sparse24_mm(0x1000, 0x2000, 0x3000, None, 0x5000, 8, 91008, 1, 0, 1, None) != 2
+    assert L.lcp_sparse24_mm(0x1000, 0x2000, 0x3000, None, 0x5000, 8, 48160 + 32, 1, 0, 0, None) == 2
+    assert L.lcp_sparse24_mm(0x1000, 0x2000, 0x3000, None, 0x5000, 8, 48160, 1, 0, 0, None) != 2
 
 
 def test_launch_count_reported():
