@@ -304,6 +304,13 @@ LCP_API lcp_status lcp_sparse24_mm(const void* values, const uint32_t* meta, con
  * reset != 0 the word is cleared after reading. */
 LCP_API lcp_status lcp_device_error(int* site, int reset);
 
+/* Self-test (synchronous; allocates and frees 4 bytes of device memory).  One
+ * thread waits on a barrier phase that nothing completes, with the time limit
+ * every wait of the tensor-core kernels uses (2 s); the wait must give up,
+ * record its site and return.  On success *site is 901 and the CUDA context
+ * stays usable.  Not for use while other work of the library is in flight. */
+LCP_API lcp_status lcp_selftest_bounded_wait(int* site);
+
 /* Allocation-free variant of lcp_loss_fwd (the paper has no counterpart; this
  * is a library convenience).  Same loss, same arguments minus the scratch
  * buffer: the per-token scratch lives in a static __device__ array of

@@ -97,6 +97,7 @@ def lib() -> ctypes.CDLL:
                        _c_void_p], _c_int),
         "lcp_train": ([P(LcpLayer), _c_int, P(LcpHparams), P(LcpAdamwParams), P(LcpAdamwState), _c_int, _c_int,
                        _c_int, _c_float, _c_float, _c_void_p, ctypes.c_size_t, _c_void_p], _c_int),
+        "lcp_selftest_bounded_wait": ([P(_c_int)], _c_int),
         "lcp_pack24": ([_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_int,
                         _c_void_p], _c_int),
         "lcp_gather": ([_c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_int, _c_void_p], _c_int),
@@ -361,6 +362,13 @@ def grad_gemm(G: torch.Tensor, X: torch.Tensor, dAt: torch.Tensor) -> None:
     bf = torch.bfloat16
     check(lib().lcp_grad_gemm(_ptr(G, bf, "G"), _ptr(X, bf, "X"), _ptr(dAt, bf, "dAt"), T, cout, cin,
                               _stream(None)))
+
+
+def selftest_bounded_wait() -> int:
+    """Runs the bounded-wait self-test (about 2 s) and returns the recorded site (901)."""
+    v = _c_int(0)
+    check(lib().lcp_selftest_bounded_wait(ctypes.byref(v)))
+    return v.value
 
 
 def device_error(reset: bool = True) -> int:
