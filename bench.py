@@ -455,7 +455,8 @@ def extras(args, b, synth, wl, li, layer, step, flush, pk, dev):
     - cublas_same_products: the two dense products of the step through torch.mm
       on the same shapes (context for the calib_gemm and bwd_gemm stages);
     - nm_mask: the standalone mask kernel on a bf16 W' of the layer's shape,
-      against the measured HBM copy bandwidth (bytes: 2 read + 1/8 written per element);
+      against the measured HBM copy bandwidth (bytes: 2 read + 1/8 written per element),
+      and on a 16384 x 16384 W' (nm_mask_large: its steady state);
     - sinkhorn_scaling: Sinkhorn forward then reverse over the logits of every
       projection of a 40-layer 13B-shaped model (4 x 5120^2, 2 x 13824 x 5120,
       5120 x 13824 per layer; 27 840 blocks of 64 x 64, 456 MB of float32 L) in one
@@ -563,6 +564,16 @@ def extras(args, b, synth, wl, li, layer, step, flush, pk, dev):
     by = li.spec.cout * li.spec.cin * 2 + li.spec.cout * li.spec.cin // 8
     out["nm_mask"] = {"ms": ms, "GB/s": by / (ms / 1e3) / 1e9, "frac": by / (ms / 1e3) / 1e9 / pk["hbm_gbs"],
                       "bytes": by, "shape": [li.spec.cout, li.spec.cin], "nm": f"{wl.n}:{wl.m}"}
+    del Wp, bits
+    # the same kernel on a 16384 x 16384 bf16 W' (512 MiB read): its steady-state bandwidth
+    big = (16384, 16384)
+    Wp = torch.empty(big, device=dev, dtype=torch.bfloat16).normal_()
+    bits = torch.empty(big[0], big[1] // 32, dtype=torch.int32, device=dev)
+    ms = timed(lambda: b.nm_mask(Wp, bits, wl.n, wl.m), K, flush_between=False)
+    by = big[0] * big[1] * 2 + big[0] * big[1] // 8
+    out["nm_mask_large"] = {"ms": ms, "GB/s": by / (ms / 1e3) / 1e9, "frac": by / (ms / 1e3) / 1e9 / pk["hbm_gbs"],
+                            "bytes": by, "shape": list(big), "nm": f"{wl.n}:{wl.m}",
+                            "note": "input larger than L2; no flush needed"}
     del Wp, bits
 
     # Sinkhorn scaling run: every projection of a 40-layer 13B-shaped model
