@@ -231,10 +231,12 @@ sinkhorn_fwd_kernel(const float* __restrict__ L, float* __restrict__ P, float* _
   cluster_barrier<CS>();
 }
 
-// Reverse.  dZ lives in registers in the row layout.
+// Reverse.  dZ lives in registers in the row layout.  For B = 64 the kernel is
+// held to 64 registers a thread so that two CTAs share an SM when many blocks
+// are in flight (a whole model's logits in one launch).
 // Shared memory (floats): tile[R*(B+1)] ck[B] ck1[B] part[NW*B] cs[B] xs[2B]
 template <int B>
-__global__ void __launch_bounds__(SkCfg<B>::NT, 1)
+__global__ void __launch_bounds__(SkCfg<B>::NT, B == 64 ? 2 : 1)
 sinkhorn_bwd_kernel(const float* __restrict__ L, const float* __restrict__ ckpt,
                     const float* __restrict__ dP, int splits, int nblocks,
                     float* __restrict__ dL, float tau, int iters) {
