@@ -4,7 +4,6 @@ import numpy as np
 import torch
 
 from learnable_channel_permutation_b200 import binding as b
-from learnable_channel_permutation_b200 import synth
 from oracle import lcp_oracle as O
 
 # Tolerances (normwise relative error ||gpu - oracle|| / ||oracle||).

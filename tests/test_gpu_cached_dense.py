@@ -1,13 +1,11 @@
 """LCP_FLAG_CACHED_DENSE: a step that reads Y_d = X W^T from layer.Yd gives the
 same P, loss, dL and mask as the step that computes it, and the Y_d a step
 writes matches the float64 oracle's dense output."""
-import numpy as np
 import pytest
 import torch
 
 from learnable_channel_permutation_b200 import binding as b
 from learnable_channel_permutation_b200 import synth
-from oracle import lcp_oracle as O
 
 import gpu_helpers as H
 

@@ -11,9 +11,7 @@ then compared with the full float64 oracle (loss and mask-conditioned dL).
 """
 import numpy as np
 import pytest
-import torch
 
-from learnable_channel_permutation_b200 import binding as b
 from learnable_channel_permutation_b200 import synth
 from oracle import lcp_oracle as O
 

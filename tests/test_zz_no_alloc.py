@@ -8,7 +8,6 @@ allocator).  Its scratch is a static device array shared by every call, so the
 second call here uses different shapes to show that the first call's contents
 do not leak into its result.  This file is collected last on purpose.
 """
-import ctypes
 
 import numpy as np
 import pytest
