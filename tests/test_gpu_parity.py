@@ -141,9 +141,9 @@ def _step_case(wl, flags=0, tol_loss=None, tol_dl=None, cos=None, L_override=Non
     f32 = wl.dtype == "f32"
     errs = []
     for li, g in zip(inputs, out):
+        td, tc = H.dl_bounds(li.spec, wl.dtype)
         errs.append(H.check_layer(li, wl, g, tol_loss or (H.TOL_LOSS_F32 if f32 else H.TOL_LOSS_BF16),
-                                  tol_dl or (H.TOL_DL_F32 if f32 else H.TOL_DL_BF16),
-                                  cos if cos is not None else (None if f32 else H.COS_DL_BF16)))
+                                  tol_dl or td, cos if cos is not None else tc))
     return errs
 
 

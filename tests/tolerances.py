@@ -1,0 +1,42 @@
+"""Tolerances of the GPU-vs-oracle comparisons (normwise relative error
+||gpu - oracle|| / ||oracle|| unless stated), shared by the GPU parity tests and
+the CPU test of the bf16 rounding model that derives the bf16 dL bounds.
+
+The pages fix no precision for dL on the bf16 path, so its bounds are derived
+from the arithmetic: tests/bf16_rounding_model.py restates where the
+tensor-core path rounds to bf16 and predicts the dL error against the float64
+oracle (it reproduces the GPU's measured error on the 7B down projection at
+T = 256 to four digits: 1.6403e-2 modelled, 1.6399e-2 measured).  Each bound is
+about twice the worst modelled layer of its input class, and
+tests/test_rounding_model.py checks the model against half of each bound.
+"""
+
+TOL_P = 1e-5            # P is float32 on every path
+TOL_LOSS_F32 = 1e-5
+TOL_LOSS_BF16 = 2e-2
+TOL_DL_F32 = 1e-3       # mask-conditioned: the oracle is given the GPU's mask
+
+# bf16 path, layers with zero-mean inputs (every layer but a ReLU-like down
+# projection): the model's worst full-size layer is 3.5e-3 (4096^2, B = 256,
+# 20 iterations, tau = 0.1), its worst at 256 tokens 2.8e-3 (7B gate/up).
+TOL_DL_BF16 = 3e-2
+COS_DL_BF16 = 0.9995
+
+# bf16 path, ReLU-like (half-normal) inputs: the 7B down projection models at
+# 1.64e-2 with 256 tokens and 4.31e-2 (cosine 0.99907) with its full 2048.  Near
+# the initialisation P is within ~1e-3 of uniform, and a nonzero-mean input gives
+# dP a large row- and column-constant part, which the Sinkhorn reverse pass
+# projects out; the bf16 rounding of At (alone 3.9e-2) and of P in the small
+# products (2.4e-2) is amplified accordingly.
+TOL_DL_BF16_RELU = 9e-2
+COS_DL_BF16_RELU = 0.998
+
+
+def dl_bounds(spec, dtype="bf16"):
+    """(normwise bound, cosine bound) of the mask-conditioned dL comparison for
+    a layer of the given synth.LayerSpec."""
+    if dtype == "f32":
+        return TOL_DL_F32, None
+    if spec.x_kind == "halfnormal":
+        return TOL_DL_BF16_RELU, COS_DL_BF16_RELU
+    return TOL_DL_BF16, COS_DL_BF16
