@@ -278,6 +278,32 @@ def test_cosine_loss_gradient_by_finite_differences():
     assert np.max(np.abs(np.sum(G * Ys, axis=0))) < 1e-14
 
 
+def test_cosine_loss_gradient_in_the_clamped_region_by_finite_differences():
+    """Reading: the cosine denominator is max(|y_d| |y_s|, 1e-8).  Where the clamp
+    binds (here a token whose sparse output is exactly zero) the token's loss is
+    1 - <y_d, y_s> / 1e-8, linear in y_s, so its gradient is -y_d / (1e-8 T).
+    Both points of every central difference stay inside the clamp region
+    (|y_d| h < 1e-8), where the difference is exact for a linear function."""
+    rng = np.random.default_rng(22)
+    Yd, Ys = rng.standard_normal((2, 6, 3))
+    Ys[:, 1] = 0.0                      # token 1: zero-norm sparse output, the clamp binds
+    G = O.cosine_loss_grad(Yd, Ys)
+    T = Ys.shape[1]
+    h = 1e-2 * O.COS_EPS / np.linalg.norm(Yd[:, 1])
+    num = np.zeros(Ys.shape[0])
+    for k in range(Ys.shape[0]):
+        e = np.zeros_like(Ys)
+        e[k, 1] = h
+        num[k] = (O.cosine_loss(Yd, Ys + e)[0] - O.cosine_loss(Yd, Ys - e)[0]) / (2 * h)
+    assert np.allclose(G[:, 1], num, rtol=1e-6, atol=0)
+    assert np.allclose(G[:, 1], -Yd[:, 1] / (O.COS_EPS * T), rtol=1e-15, atol=0)
+    # the token's loss is 1 there (cosine 0 at y_s = 0), and the other tokens are unaffected
+    _, cos = O.cosine_loss(Yd, Ys)
+    assert cos[1] == 0.0
+    G_ref = O.cosine_loss_grad(Yd[:, [0, 2]], Ys[:, [0, 2]]) * 2 / 3
+    assert np.allclose(G[:, [0, 2]], G_ref, rtol=1e-14, atol=0)
+
+
 # -------------------------------------------------------- brute force over 8! --
 
 def _hard_loss_independent(W, X_tokens, sigma, n, m):
