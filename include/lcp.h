@@ -21,6 +21,9 @@
  *    is enqueued and a status other than LCP_OK is returned; lcp_last_error()
  *    then holds a message for the calling thread.
  *  - A launch failure is reported as LCP_ERR_CUDA (message kept likewise).
+ *    A CUDA error that earlier work left pending (cudaPeekAtLastError) is
+ *    also reported as LCP_ERR_CUDA, before anything is enqueued, and is left
+ *    pending for its owner (the library never clears another caller's error).
  *  - Matrices are row-major and densely packed:
  *      W  [C_out, C_in]    X  [T, C_in]      (dtype of the call: f32 or bf16)
  *      L, P, dL  [C_in/B, B, B] float32; P_b[i][j] moves source channel bB+i
@@ -314,15 +317,17 @@ LCP_API lcp_status lcp_selftest_bounded_wait(int* site);
 /* Allocation-free variant of lcp_loss_fwd (the paper has no counterpart; this
  * is a library convenience).  Same loss, same arguments minus the scratch
  * buffer: the per-token scratch lives in a static __device__ array of
- * LCP_STATIC_MAX_TOKENS * 4 floats that every GPU loading the library holds
- * until exit.  For callers that cannot allocate device memory: code running
- * while a stream is captured into a CUDA graph or inside a stream-ordered
- * pipeline (cudaMalloc may synchronise the device), and embedders whose device
- * memory belongs to another allocator or is reserved up front.
+ * LCP_STATIC_MAX_TOKENS * 4 floats (1 MiB) that every GPU loading the library
+ * holds until exit.  For callers that cannot allocate device memory: embedders
+ * whose device memory belongs to another allocator or is reserved up front
+ * under a fixed budget, and latency-critical pipelines in which cudaMalloc's
+ * implicit device synchronisation would stall work on other streams.
  * - tokens > LCP_STATIC_MAX_TOKENS is rejected with LCP_ERR_SHAPE.
  * - The first call on a device looks up the array's device address
- *   (cudaGetSymbolAddress) with that device current; make it before any
- *   stream capture begins.
+ *   (cudaGetSymbolAddress) with that device current and caches it with the
+ *   ID of the current CUDA context; make that first call before any stream
+ *   capture begins.  After cudaDeviceReset (any change of context) the next
+ *   call repeats the lookup.
  * - All calls share the array (each call overwrites all of it that it reads,
  *   so nothing must be cleared); calls that overlap on the GPU race on it.
  * - Allocates and frees nothing, calls no allocating routine. */

@@ -68,6 +68,14 @@ lcp_status check_launch(const char* what) {
   return LCP_OK;
 }
 
+lcp_status check_pending() {
+  const cudaError_t e = cudaPeekAtLastError();
+  if (e != cudaSuccess)
+    return fail(LCP_ERR_CUDA, "a CUDA error from earlier work is pending (%s); nothing was enqueued and the "
+                "error is left for its owner", cudaGetErrorString(e));
+  return LCP_OK;
+}
+
 namespace {
 
 #define LCP_TRY(expr)                     \
@@ -424,7 +432,7 @@ lcp_status step_impl(const lcp_layer* layers, int nlayers, const lcp_hparams* hp
   if (ws_bytes < need)
     return fail(LCP_ERR_WORKSPACE, "workspace has %zu bytes, %zu needed", ws_bytes, need);
   LCP_TRY(check_arch());
-  cudaGetLastError();  // a stale error from elsewhere must not be blamed on us
+  LCP_TRY(check_pending());
   for (int i = 0; i < nlayers; ++i) {
     const Plan p = make_plan(layers[i], *hp);
     cudaEvent_t* e = (i == 0 && nev) ? ev : nullptr;
@@ -502,7 +510,7 @@ lcp_status lcp_adamw(float* L, const float* dL, float* m, float* v, long long n,
     return fail(LCP_ERR_ARG, "every pointer must be 16-byte aligned");
   if (n == 0) return LCP_OK;
   LCP_TRY(check_arch());
-  cudaGetLastError();
+  LCP_TRY(check_pending());
   return launch_adamw(L, dL, m, v, n, opt->lr, opt->beta1, opt->beta2, opt->eps, opt->weight_decay, t, stream);
 }
 
@@ -547,7 +555,7 @@ lcp_status lcp_sinkhorn_fwd(const float* L, float* P, float* ckpt, int nblocks, 
   if (!(tau > 0.f) || !std::isfinite(tau)) return fail(LCP_ERR_ARG, "tau must be positive and finite");
   if (nblocks == 0) return LCP_OK;
   LCP_TRY(check_arch());
-  cudaGetLastError();
+  LCP_TRY(check_pending());
   return launch_sinkhorn_fwd(L, P, ckpt, nullptr, nullptr, nullptr, nullptr, nblocks, B, tau, iters, stream);
 }
 
@@ -563,7 +571,7 @@ lcp_status lcp_sinkhorn_bwd(const float* L, const float* ckpt, const float* dP, 
   if (!(tau > 0.f) || !std::isfinite(tau)) return fail(LCP_ERR_ARG, "tau must be positive and finite");
   if (nblocks == 0) return LCP_OK;
   LCP_TRY(check_arch());
-  cudaGetLastError();
+  LCP_TRY(check_pending());
   return launch_sinkhorn_bwd(L, ckpt, dP, dP_splits, dL, nblocks, B, tau, iters, stream);
 }
 
@@ -577,7 +585,7 @@ lcp_status lcp_permute_weight(const void* W, const float* P, float* Wp, int cout
     return fail(LCP_ERR_SHAPE, "C_out = %d, C_in = %d (C_in must be a multiple of B)", cout, cin);
   if (cout == 0 || cin == 0) return LCP_OK;
   LCP_TRY(check_arch());
-  cudaGetLastError();
+  LCP_TRY(check_pending());
   const long long ic = cin, BB = (long long)B * B;
   return launch_simt_gemm({cout, B, B, cin / B, W, B, ic, 1, P, BB, B, 1, Wp, B, ic, 1, 1.f, 0.f},
                           dtype, LCP_F32, LCP_F32, stream);
@@ -593,7 +601,7 @@ lcp_status lcp_score(const void* W, const void* X, void* S, float* stats, int co
     return fail(LCP_ERR_SHAPE, "C_out = %d, C_in = %d, T = %d", cout, cin, tokens);
   if (cout == 0 || cin == 0) return LCP_OK;
   LCP_TRY(check_arch());
-  cudaGetLastError();
+  LCP_TRY(check_pending());
   return launch_score(W, X, S, stats, cout, cin, tokens, kind, dtype, stream);
 }
 
@@ -606,7 +614,7 @@ lcp_status lcp_harden(const float* P_hat, int32_t* perm, float* P_hard, int nblo
     return fail(LCP_ERR_ARG, "P_hat and P_hard must be 16-byte aligned");
   if (nblocks == 0) return LCP_OK;
   LCP_TRY(check_arch());
-  cudaGetLastError();
+  LCP_TRY(check_pending());
   return launch_harden(P_hat, perm, P_hard, nullptr, nullptr, nullptr, nblocks, B, stream);
 }
 
@@ -630,7 +638,7 @@ lcp_status lcp_pack24(const void* W, const int32_t* perm, const uint32_t* mask, 
   if (!aligned16(W) || !aligned16(mask) || !aligned16(values) || !aligned16(meta) || (perm && !aligned16(perm)))
     return fail(LCP_ERR_ARG, "pointers must be 16-byte aligned");
   LCP_TRY(check_arch());
-  cudaGetLastError();
+  LCP_TRY(check_pending());
   return launch_pack24(W, perm, mask, values, meta, cout, cin, B, dtype, stream);
 }
 
@@ -644,7 +652,7 @@ lcp_status lcp_gather(const void* X, const int32_t* perm, void* Xp, int tokens, 
   if (!aligned16(X) || !aligned16(Xp) || !aligned16(perm)) return fail(LCP_ERR_ARG, "pointers must be 16-byte aligned");
   if (tokens == 0) return LCP_OK;
   LCP_TRY(check_arch());
-  cudaGetLastError();
+  LCP_TRY(check_pending());
   return launch_gather(X, perm, Xp, tokens, cin, B, dtype, stream);
 }
 
@@ -660,7 +668,7 @@ lcp_status lcp_sparse24_mm(const void* values, const uint32_t* meta, const void*
     return fail(LCP_ERR_ARG, "pointers must be 16-byte aligned");
   if (tokens == 0) return LCP_OK;
   LCP_TRY(check_arch());
-  cudaGetLastError();
+  LCP_TRY(check_pending());
   return launch_sparse24_mm(values, meta, X, perm, Y, cout, cin, tokens, B, dtype, stream);
 }
 
@@ -675,7 +683,7 @@ lcp_status nm_mask(const void* Wp, uint32_t* mask_bits, int rows, int cols, int 
   if (!aligned16(Wp) || !aligned16(mask_bits)) return fail(LCP_ERR_ARG, "pointers must be 16-byte aligned");
   if (rows == 0 || cols == 0) return LCP_OK;
   LCP_TRY(check_arch());
-  cudaGetLastError();
+  LCP_TRY(check_pending());
   return launch_nm_mask(Wp, mask_bits, rows, cols, n, m, dtype, stream);
 }
 
@@ -690,7 +698,7 @@ lcp_status lcp_calib_gemm(const void* X, const void* W, const void* At, float* Y
   for (const void* q : ptrs)
     if (q && !aligned16(q)) return fail(LCP_ERR_ARG, "pointers must be 16-byte aligned");
   LCP_TRY(check_arch());
-  cudaGetLastError();
+  LCP_TRY(check_pending());
   return launch_calib_gemm_tc(static_cast<const __nv_bfloat16*>(X), static_cast<const __nv_bfloat16*>(W),
                               static_cast<const __nv_bfloat16*>(At), Yd, Ys, tokens, cout, cin, stream);
 }
@@ -703,7 +711,7 @@ lcp_status lcp_grad_gemm(const void* G, const void* X, void* dAt, int tokens, in
   if (tokens < 1 || tokens > kMaxDim) return fail(LCP_ERR_SHAPE, "T = %d must be >= 1", tokens);
   if (!aligned16(G) || !aligned16(X) || !aligned16(dAt)) return fail(LCP_ERR_ARG, "pointers must be 16-byte aligned");
   LCP_TRY(check_arch());
-  cudaGetLastError();
+  LCP_TRY(check_pending());
   return launch_bwd_gemm_tc(static_cast<const __nv_bfloat16*>(G), static_cast<const __nv_bfloat16*>(X),
                             static_cast<__nv_bfloat16*>(dAt), tokens, cout, cin, stream);
 }
@@ -715,7 +723,7 @@ lcp_status lcp_loss_fwd(const float* Yd, const float* Ys, float* loss, float* st
   if (tokens < 1 || tokens > kMaxDim) return fail(LCP_ERR_SHAPE, "T = %d must be >= 1", tokens);
   if (!aligned16(Yd) || !aligned16(Ys) || !aligned16(stats)) return fail(LCP_ERR_ARG, "pointers must be 16-byte aligned");
   LCP_TRY(check_arch());
-  cudaGetLastError();
+  LCP_TRY(check_pending());
   LCP_TRY(launch_loss_token(Yd, Ys, stats, nullptr, LCP_F32, cout, tokens, stream));
   return launch_loss_reduce(stats, loss, tokens, stream);
 }
@@ -729,7 +737,7 @@ lcp_status lcp_loss_bwd(const float* Yd, const float* Ys, const float* stats, vo
   if (!aligned16(Yd) || !aligned16(Ys) || !aligned16(stats) || !aligned16(G))
     return fail(LCP_ERR_ARG, "pointers must be 16-byte aligned");
   LCP_TRY(check_arch());
-  cudaGetLastError();
+  LCP_TRY(check_pending());
   return launch_loss_grad(Yd, Ys, stats, G, dtype, cout, tokens, stream);
 }
 

@@ -14,6 +14,10 @@ void set_error(const char* fmt, ...);
 lcp_status fail(lcp_status s, const char* fmt, ...);
 // Checks cudaGetLastError() after a launch; returns LCP_ERR_CUDA with `what`.
 lcp_status check_launch(const char* what);
+// Before the first launch of an entry point: an error another caller left
+// pending (cudaPeekAtLastError) is reported as LCP_ERR_CUDA and NOT cleared,
+// so that neither is it blamed on this call's launches nor lost to its owner.
+lcp_status check_pending();
 
 // Raises `func`'s dynamic shared-memory limit to `bytes` on the current device
 // unless an earlier call already did (the attribute persists for the process).

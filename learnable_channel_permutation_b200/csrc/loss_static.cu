@@ -3,18 +3,21 @@
 //
 // lcp_loss_fwd needs a caller-provided scratch buffer of 4 floats per token
 // (the per-token dot product, squared norms and cosine).  Some callers cannot
-// provide one: code that must not call cudaMalloc because it runs while a
-// stream is being captured into a CUDA graph or inside a stream-ordered
-// pipeline that cudaMalloc's implicit device synchronisation would stall, and
-// embedders whose device memory is owned by another allocator or reserved up
-// front under a fixed budget.  This entry point keeps that scratch in a
-// file-scope __device__ array instead: every GPU that loads the library holds
+// provide one: embedders whose device memory is owned by another allocator or
+// reserved up front under a fixed budget, and latency-critical pipelines that
+// must not call cudaMalloc because its implicit device synchronisation would
+// stall work running on other streams.  This entry point keeps that scratch in
+// a file-scope __device__ array instead: every GPU that loads the library holds
 // LCP_STATIC_MAX_TOKENS * 16 bytes of it until the process exits.
 //
 // Host code cannot use the array's name as a device address (in host code it
-// names a host-side shadow).  The device address is obtained once per device
-// with cudaGetSymbolAddress, with that device current, on the first call made
-// on that device; make that first call before any stream capture begins.
+// names a host-side shadow).  The device address is obtained with
+// cudaGetSymbolAddress, with the device current, by the first call made on a
+// device, and cached together with the unique ID of the CUDA context it
+// belongs to; a call that finds another context current (after
+// cudaDeviceReset, for example) repeats the lookup instead of launching with a
+// stale address.  Make the first call on a device before any stream capture
+// begins.
 //
 // Every call shares the one array.  The token kernel writes all 4 * tokens
 // floats before the reduction reads them, so nothing has to start at zero and
@@ -22,6 +25,7 @@
 // kernels overlap on the GPU (different streams, no ordering between them)
 // race on the array and must not be issued.
 
+#include <cuda.h>
 #include <mutex>
 
 #include "lcp_internal.cuh"
@@ -34,6 +38,37 @@ namespace {
 constexpr int kMaxDevices = 64;
 std::mutex g_static_mu;
 float* g_static_ptr[kMaxDevices] = {};
+unsigned long long g_static_ctx[kMaxDevices] = {};   // context ID the cached address belongs to
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+template <typename F> F driver_fn(const char* name) {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q{};
+  if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess || q != cudaDriverEntryPointSuccess) {
+    cudaGetLastError();   // our own lookup's error
+    return nullptr;
+  }
+  return reinterpret_cast<F>(p);
+}
+
+// Unique ID of the calling thread's current CUDA context, 0 when there is none
+// yet or the driver cannot tell.
+unsigned long long current_ctx_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    get_current = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+    get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+  });
+  if (!get_current || !get_id) return 0;
+  CUcontext c = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&c) != CUDA_SUCCESS || !c || get_id(c, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
 
 lcp_status static_scratch(float** out) {
   int dev = 0;
@@ -44,15 +79,17 @@ lcp_status static_scratch(float** out) {
   }
   if (dev < 0 || dev >= kMaxDevices) return fail(LCP_ERR_ARG, "device ordinal %d is out of range", dev);
   std::lock_guard<std::mutex> lk(g_static_mu);
-  if (!g_static_ptr[dev]) {
+  const unsigned long long ctx = current_ctx_id();
+  if (!g_static_ptr[dev] || ctx == 0 || ctx != g_static_ctx[dev]) {
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_lcp_static_loss_stats);
+    e = cudaGetSymbolAddress(&p, g_lcp_static_loss_stats);   // set-up: also makes the context current
     if (e != cudaSuccess || !p) {
       cudaGetLastError();
       return fail(LCP_ERR_CUDA, "cudaGetSymbolAddress of the static loss scratch on device %d: %s", dev,
                   cudaGetErrorString(e));
     }
     g_static_ptr[dev] = static_cast<float*>(p);
+    g_static_ctx[dev] = current_ctx_id();
   }
   *out = g_static_ptr[dev];
   return LCP_OK;
@@ -84,10 +121,11 @@ extern "C" lcp_status lcp_loss_fwd_static(const float* Yd, const float* Ys, floa
   }
   if (major != 10 || minor != 0)
     return fail(LCP_ERR_ARCH, "device %d is sm_%d%d, this library is built for sm_100a", dev, major, minor);
+  const lcp_status s0 = check_pending();
+  if (s0 != LCP_OK) return s0;
   float* stats = nullptr;
   const lcp_status s = static_scratch(&stats);
   if (s != LCP_OK) return s;
-  cudaGetLastError();
   const lcp_status s1 = launch_loss_token(Yd, Ys, stats, nullptr, LCP_F32, cout, tokens, stream);
   if (s1 != LCP_OK) return s1;
   return launch_loss_reduce(stats, loss, tokens, stream);
