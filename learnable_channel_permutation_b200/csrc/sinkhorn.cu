@@ -1,4 +1,4 @@
-// Block-wise log-domain Sinkhorn normalisation, forward and reverse.
+// Block-wise Sinkhorn normalisation, forward and reverse.
 //
 // PermLLM ("Learnable Channel Permutation for N:M Sparse LLMs"), Method 1:
 // S_0(X) = exp(X), S_i(X) = T_c(T_r(S_{i-1}(X))), P = S_L(W_P / tau), applied
@@ -6,23 +6,38 @@
 // gives the log-domain form: subtract each row's log-sum-exp, then each
 // column's, `iters` times, then exponentiate.
 //
-// Every log-domain iterate has the form Z = Z_0 - R_i - C_j, so a row step
-// only has to compute R_i = LSE_j(Z_0[i,j] - C_j) and a column step
-// C_j = LSE_i(Z_0[i,j] - R_i).  Z_0 = L / tau never changes, so each thread
-// keeps its share of Z_0 in registers twice: a row slice (TPR adjacent lanes
-// per row, interleaved columns) for the row steps and a column slice (TPC
-// adjacent lanes per column, interleaved rows) for the column steps.  A step
-// is then register arithmetic, a read of the other side's normaliser vector
-// from shared memory and two or three shuffles; the (R, C) pair of every
-// iteration is the checkpoint the reverse pass replays.
+// Every iterate has the form Z = Z_0 - R_i - C_j, so a row step only has to
+// compute R_i = LSE_j(Z_0[i,j] - C_j) and a column step C_j = LSE_i(Z_0[i,j] -
+// R_i); (R, C) after every step is the checkpoint the reverse pass replays.
+// Two arithmetics compute these, chosen per block from the range of Z_0 = L/tau:
+//
+//  * linear (max Z_0 - min Z_0 <= 64, every block of a run near its
+//    initialisation): with K = exp(Z_0 - max Z_0) formed once per element
+//    (entries in [e^-64, 1]), exp(Z) = a_i K_ij b_j with a = e^{max - R},
+//    b = e^{-C}; a row step is a_i = 1 / sum_j K_ij b_j and a column step
+//    b_j = 1 / sum_i a_i K_ij -- multiply-adds and one reciprocal per row or
+//    column instead of two exponentials per element.  The checkpoint stores
+//    R_i = max + log(sum_j K_ij b_j) and C_j = log(sum_i a_i K_ij), the same
+//    normalisers as the log domain.  The scalings stay within e^{+-70}, inside
+//    the float32 range.
+//  * log domain (wider ranges, e.g. sharply peaked logits, where K would
+//    underflow): the log-sum-exp steps themselves.
+//
+// Z_0 never changes, so each thread keeps its share of Z_0 (or K) in registers
+// twice: a row slice (TPR adjacent lanes per row, interleaved columns) for the
+// row steps and a column slice (TPC adjacent lanes per column, interleaved
+// rows) for the column steps.  A step is then register arithmetic, a read of
+// the other side's vector from shared memory and two or three shuffles.
 //
 // One CTA owns one block for B <= 128.  For B = 256 a cluster of 4 CTAs
 // splits the rows; column reductions combine the per-CTA partials through
 // distributed shared memory in a fixed rank order, so every CTA gets
-// bit-identical results.  Every reduction runs in a fixed order.  Exponentials
-// and logarithms use the hardware approximations (__expf, __logf): about 1e-6
+// bit-identical results (the range that picks the arithmetic is combined the
+// same way).  Every reduction runs in a fixed order.  Exponentials and
+// logarithms use the hardware approximations (__expf, __logf): about 1e-6
 // relative error, well inside the 1e-5 tolerance on P.
 
+#include <algorithm>
 #include <cooperative_groups.h>
 #include <math_constants.h>
 
@@ -58,6 +73,12 @@ template <int CS> __device__ __forceinline__ void cluster_barrier() {
 template <int CS> __device__ __forceinline__ const float* peer(float* p, int r) {
   if constexpr (CS > 1) return cg::this_cluster().map_shared_rank(p, r);
   else return p;
+}
+
+// two floats -> packed bf16x2 (round to nearest even), low half first
+__device__ __forceinline__ uint32_t pack_bf16x2_rn(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
 }
 
 // reductions over `W` adjacent lanes (W a power of two)
@@ -96,30 +117,85 @@ __device__ __forceinline__ void load_slab(float* tile, const float* __restrict__
   }
 }
 
-// Forward.  Shared memory (floats): tile[R*(B+1)] rv[R] cv[B] xm[2B] xs[2B]
+// Widest range of Z_0 = L / tau over a block for which the linear arithmetic
+// is used: K = exp(Z_0 - max Z_0) then lies in [e^-64, 1].
+constexpr float kLinearRange = 64.f;
+
+// Largest and smallest value over the CTA (and over the cluster for CS > 1),
+// bit-identical on every thread of every CTA of the cluster.  red: 66 floats
+// of shared memory, not reused afterwards.  Ends with a CTA (cluster) barrier.
+template <int NT, int CS>
+__device__ __forceinline__ void block_range(float mx, float mn, float* red, float& gmx, float& gmn) {
+  constexpr int NW = NT / 32;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  mx = group_max<32>(mx);
+  mn = -group_max<32>(-mn);
+  if (lane == 0) {
+    red[warp] = mx;
+    red[32 + warp] = mn;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    float a = lane < NW ? red[lane] : -CUDART_INF_F;
+    float b = lane < NW ? -red[32 + lane] : -CUDART_INF_F;
+    a = group_max<32>(a);
+    b = group_max<32>(b);
+    if (lane == 0) {
+      red[64] = a;
+      red[65] = -b;
+    }
+  }
+  if constexpr (CS == 1) {
+    __syncthreads();
+    gmx = red[64];
+    gmn = red[65];
+  } else {
+    cluster_barrier<CS>();
+    float a = -CUDART_INF_F, b = CUDART_INF_F;
+#pragma unroll
+    for (int q = 0; q < CS; ++q) {
+      const float* pr = peer<CS>(red, q);
+      a = fmaxf(a, pr[64]);
+      b = fminf(b, pr[65]);
+    }
+    gmx = a;
+    gmn = b;
+  }
+}
+
+// Forward.  Shared memory (floats): tile[R*(B+1)] rv[R] cv[B] xm[2B] xs[2B] red[66]
 template <int B>
 __global__ void __launch_bounds__(SkCfg<B>::NT, 1)
-sinkhorn_fwd_kernel(const float* __restrict__ L, float* __restrict__ P, float* __restrict__ ckpt,
-                    __nv_bfloat16* __restrict__ pt_hi, __nv_bfloat16* __restrict__ pt_lo,
-                    __nv_bfloat16* __restrict__ p_hi, unsigned* __restrict__ zero_word, float tau, int iters) {
+sinkhorn_fwd_kernel(const __grid_constant__ SkFwdBatch batch, float tau, int iters) {
   using C = SkCfg<B>;
   pdl_wait();
   pdl_trigger();
-  if (zero_word && blockIdx.x == 0 && threadIdx.x == 0) *zero_word = 0u;
+  // this CTA's layer and block within it (the layers' blocks follow each other in the grid)
+  int blk = blockIdx.x / C::CS, li = 0;
+  while (li + 1 < batch.n && blk >= batch.layer[li].blocks) blk -= batch.layer[li++].blocks;
+  const SkFwdLayer& ly = batch.layer[li];
+  const float* __restrict__ L = ly.L;
+  float* __restrict__ P = ly.P;
+  float* __restrict__ ckpt = ly.ckpt;
+  __nv_bfloat16* __restrict__ pt_hi = ly.pt_hi;
+  __nv_bfloat16* __restrict__ pt_lo = ly.pt_lo;
+  __nv_bfloat16* __restrict__ p_hi = ly.p_hi;
+  if (ly.zero_word && blk == 0 && blockIdx.x % C::CS == 0 && threadIdx.x == 0) *ly.zero_word = 0u;
   constexpr int R = C::R, NT = C::NT, CS = C::CS, TPR = C::TPR, EPR = C::EPR, TPC = C::TPC,
                 EPC = C::EPC, LD = C::LD;
   extern __shared__ __align__(16) float sm[];
   float* tile = sm;
-  float* rv = tile + R * LD;
-  float* cv = rv + R;
-  float* xm = cv + B;   // this CTA's column partials, double-buffered by iteration parity
+  float* rv = tile + R * LD;   // per row of this CTA: a_i (linear) or R_i (log domain)
+  float* cv = rv + R;          // per column: b_j (linear) or C_j (log domain)
+  float* xm = cv + B;          // this CTA's column partials, double-buffered by iteration parity
   float* xs = xm + 2 * B;
+  float* red = xs + 2 * B;
 
   const int rank = cta_rank<CS>();
-  const int blk = blockIdx.x / CS;
   const int row0 = rank * R;
   const int tid = threadIdx.x;
   const size_t base = (size_t)blk * B * B;
+  const size_t ck0 = (size_t)blk * iters * 2 * B;
   const int r = tid / TPR, c = tid % TPR;     // row slice: row r, columns c + TPR*e
   const int j = tid / TPC, g = tid % TPC;     // column slice: column j, rows g + TPC*e
 
@@ -131,130 +207,224 @@ sinkhorn_fwd_kernel(const float* __restrict__ L, float* __restrict__ P, float* _
     float* d = tile + rr * LD + jj;
     d[0] = v.x * inv_tau; d[1] = v.y * inv_tau; d[2] = v.z * inv_tau; d[3] = v.w * inv_tau;
   }
-  for (int jj = tid; jj < B; jj += NT) cv[jj] = 0.f;
   __syncthreads();
   float zr[EPR], zc[EPC];
 #pragma unroll
   for (int e = 0; e < EPR; ++e) zr[e] = tile[r * LD + c + TPR * e];
 #pragma unroll
   for (int e = 0; e < EPC; ++e) zc[e] = tile[(g + TPC * e) * LD + j];
-
-  float myR = 0.f;
-  for (int k = 0; k < iters; ++k) {
-    // T_r: R_i = LSE_j(z_ij - C_j)
-    {
-      float x[EPR];
+  float lmx = zr[0], lmn = zr[0];
 #pragma unroll
-      for (int e = 0; e < EPR; ++e) x[e] = zr[e] - cv[c + TPR * e];
-      float m, s;
-      lse_parts<EPR, TPR>(x, m, s);
-      myR = m + __logf(s);
-      if (c == 0) {
-        rv[r] = myR;
-        if (ckpt) ckpt[((size_t)blk * iters + k) * 2 * B + row0 + r] = myR;
-      }
-    }
-    __syncthreads();
-    // T_c: C_j = LSE_i(z_ij - R_i) over all B rows of the block
-    {
-      float x[EPC];
-#pragma unroll
-      for (int e = 0; e < EPC; ++e) x[e] = zc[e] - rv[g + TPC * e];
-      float m, s;
-      lse_parts<EPC, TPC>(x, m, s);
-      if constexpr (CS == 1) {
-        if (g == 0) {
-          const float v = m + __logf(s);
-          cv[j] = v;
-          if (ckpt) ckpt[(((size_t)blk * iters + k) * 2 + 1) * B + j] = v;
-        }
-        __syncthreads();
-      } else {
-        float* bm = xm + (k & 1) * B;
-        float* bs = xs + (k & 1) * B;
-        if (g == 0) { bm[j] = m; bs[j] = s; }
-        cluster_barrier<CS>();
-        if (g == 0) {
-          float M = -CUDART_INF_F;
-#pragma unroll
-          for (int q = 0; q < CS; ++q) M = fmaxf(M, peer<CS>(bm, q)[j]);
-          float S = 0.f;
-#pragma unroll
-          for (int q = 0; q < CS; ++q) S += peer<CS>(bs, q)[j] * __expf(peer<CS>(bm, q)[j] - M);
-          const float v = M + __logf(S);
-          cv[j] = v;
-          if (ckpt && rank == 0) ckpt[(((size_t)blk * iters + k) * 2 + 1) * B + j] = v;
-        }
-        __syncthreads();
-      }
-    }
+  for (int e = 1; e < EPR; ++e) {
+    lmx = fmaxf(lmx, zr[e]);
+    lmn = fminf(lmn, zr[e]);
   }
+  float zmax, zmin;
+  block_range<NT, CS>(lmx, lmn, red, zmax, zmin);
+  const bool linear = (zmax - zmin) <= kLinearRange;
 
-  // P = exp(Z_0 - R - C), staged through the tile for coalesced stores
+  float myR = 0.f;   // this thread's row: a_i (linear) or R_i (log domain)
+  if (linear) {
 #pragma unroll
-  for (int e = 0; e < EPR; ++e) tile[r * LD + c + TPR * e] = __expf(zr[e] - myR - cv[c + TPR * e]);
+    for (int e = 0; e < EPR; ++e) zr[e] = __expf(zr[e] - zmax);
+#pragma unroll
+    for (int e = 0; e < EPC; ++e) zc[e] = __expf(zc[e] - zmax);
+    for (int jj = tid; jj < B; jj += NT) cv[jj] = 1.f;
+    __syncthreads();
+    for (int k = 0; k < iters; ++k) {
+      // T_r: a_i = 1 / sum_j K_ij b_j   (R_i = max Z_0 + log of that sum)
+      {
+        float s = 0.f;
+#pragma unroll
+        for (int e = 0; e < EPR; ++e) s = fmaf(zr[e], cv[c + TPR * e], s);
+        s = group_sum<TPR>(s);
+        myR = __frcp_rn(s);
+        if (c == 0) {
+          rv[r] = myR;
+          if (ckpt) ckpt[ck0 + (size_t)k * 2 * B + row0 + r] = zmax + __logf(s);
+        }
+      }
+      __syncthreads();
+      // T_c: b_j = 1 / sum_i a_i K_ij over all B rows   (C_j = log of that sum)
+      {
+        float s = 0.f;
+#pragma unroll
+        for (int e = 0; e < EPC; ++e) s = fmaf(zc[e], rv[g + TPC * e], s);
+        s = group_sum<TPC>(s);
+        if constexpr (CS == 1) {
+          if (g == 0) {
+            cv[j] = __frcp_rn(s);
+            if (ckpt) ckpt[ck0 + ((size_t)k * 2 + 1) * B + j] = __logf(s);
+          }
+        } else {
+          float* bs = xs + (k & 1) * B;
+          if (g == 0) bs[j] = s;
+          cluster_barrier<CS>();
+          if (g == 0) {
+            float S = 0.f;
+#pragma unroll
+            for (int q = 0; q < CS; ++q) S += peer<CS>(bs, q)[j];
+            cv[j] = __frcp_rn(S);
+            if (ckpt && rank == 0) ckpt[ck0 + ((size_t)k * 2 + 1) * B + j] = __logf(S);
+          }
+        }
+        __syncthreads();
+      }
+    }
+    // P = a_i K_ij b_j, staged through the tile for coalesced stores
+#pragma unroll
+    for (int e = 0; e < EPR; ++e) tile[r * LD + c + TPR * e] = myR * zr[e] * cv[c + TPR * e];
+  } else {
+    for (int jj = tid; jj < B; jj += NT) cv[jj] = 0.f;
+    __syncthreads();
+    for (int k = 0; k < iters; ++k) {
+      // T_r: R_i = LSE_j(z_ij - C_j)
+      {
+        float x[EPR];
+#pragma unroll
+        for (int e = 0; e < EPR; ++e) x[e] = zr[e] - cv[c + TPR * e];
+        float m, s;
+        lse_parts<EPR, TPR>(x, m, s);
+        myR = m + __logf(s);
+        if (c == 0) {
+          rv[r] = myR;
+          if (ckpt) ckpt[ck0 + (size_t)k * 2 * B + row0 + r] = myR;
+        }
+      }
+      __syncthreads();
+      // T_c: C_j = LSE_i(z_ij - R_i) over all B rows of the block
+      {
+        float x[EPC];
+#pragma unroll
+        for (int e = 0; e < EPC; ++e) x[e] = zc[e] - rv[g + TPC * e];
+        float m, s;
+        lse_parts<EPC, TPC>(x, m, s);
+        if constexpr (CS == 1) {
+          if (g == 0) {
+            const float v = m + __logf(s);
+            cv[j] = v;
+            if (ckpt) ckpt[ck0 + ((size_t)k * 2 + 1) * B + j] = v;
+          }
+          __syncthreads();
+        } else {
+          float* bm = xm + (k & 1) * B;
+          float* bs = xs + (k & 1) * B;
+          if (g == 0) { bm[j] = m; bs[j] = s; }
+          cluster_barrier<CS>();
+          if (g == 0) {
+            float M = -CUDART_INF_F;
+#pragma unroll
+            for (int q = 0; q < CS; ++q) M = fmaxf(M, peer<CS>(bm, q)[j]);
+            float S = 0.f;
+#pragma unroll
+            for (int q = 0; q < CS; ++q) S += peer<CS>(bs, q)[j] * __expf(peer<CS>(bm, q)[j] - M);
+            const float v = M + __logf(S);
+            cv[j] = v;
+            if (ckpt && rank == 0) ckpt[ck0 + ((size_t)k * 2 + 1) * B + j] = v;
+          }
+          __syncthreads();
+        }
+      }
+    }
+    // P = exp(Z_0 - R - C), staged through the tile for coalesced stores
+#pragma unroll
+    for (int e = 0; e < EPR; ++e) tile[r * LD + c + TPR * e] = __expf(zr[e] - myR - cv[c + TPR * e]);
+  }
   __syncthreads();
-  for (int q = tid; q < R * B; q += NT) {
-    const int rr = q / B, jj = q % B;
-    P[base + (size_t)(row0 + rr) * B + jj] = tile[rr * LD + jj];
+  // P, four consecutive columns a thread (16-byte stores)
+  for (int q = tid; q < R * (B / 4); q += NT) {
+    const int rr = q / (B / 4), jj = (q % (B / 4)) * 4;
+    const float* src = tile + rr * LD + jj;
+    reinterpret_cast<float4*>(P + base + (size_t)(row0 + rr) * B)[jj / 4] = make_float4(src[0], src[1], src[2], src[3]);
   }
   if (pt_hi) {
     // Operand images for the tensor-core kernels, in tiles of BC = max(B, 64)
     // columns: tile t holds the BC x BC block-diagonal slice of P_B covering
     // channels [t*BC, (t+1)*BC) (for B = 32 two blocks share one tile and the
-    // off-diagonal quadrants are written as zeros).
+    // off-diagonal quadrants are written as zeros).  Eight consecutive bf16 a
+    // thread (16-byte stores).
     constexpr int BC = B < 64 ? 64 : B;
     const int gcol0 = blk * B;
     const size_t tb = (size_t)(gcol0 / BC) * BC * BC;
     const int q0 = gcol0 % BC;
-    const __nv_bfloat16 zero = __float2bfloat16_rn(0.f);
-    // transposed images: consecutive threads take consecutive source rows i
-    for (int q = tid; q < R * B; q += NT) {
-      const int jj = q / R, rr = q % R, i = row0 + rr;
-      const float p = tile[rr * LD + jj];
-      const __nv_bfloat16 hi = __float2bfloat16_rn(p);
-      pt_hi[tb + (size_t)(q0 + jj) * BC + q0 + i] = hi;
-      pt_lo[tb + (size_t)(q0 + jj) * BC + q0 + i] = __float2bfloat16_rn(p - __bfloat162float(hi));
+    const int zc0 = (q0 == 0) ? B : 0;   // the zero quadrant's columns (B < BC)
+    const uint4 zero4 = make_uint4(0u, 0u, 0u, 0u);
+    // transposed images: image row q0 + jj, source rows i = row0 + 8 g .. + 7
+    for (int q = tid; q < B * (R / 8); q += NT) {
+      const int jj = q / (R / 8), g8 = (q % (R / 8)) * 8;
+      float hv[8], lv[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const float p = tile[(g8 + u) * LD + jj];
+        const __nv_bfloat16 hi = __float2bfloat16_rn(p);
+        hv[u] = __bfloat162float(hi);
+        lv[u] = p - hv[u];
+      }
+      const size_t at = tb + (size_t)(q0 + jj) * BC + q0 + row0 + g8;
+      *reinterpret_cast<uint4*>(pt_hi + at) = make_uint4(pack_bf16x2_rn(hv[0], hv[1]), pack_bf16x2_rn(hv[2], hv[3]),
+                                                         pack_bf16x2_rn(hv[4], hv[5]), pack_bf16x2_rn(hv[6], hv[7]));
+      *reinterpret_cast<uint4*>(pt_lo + at) = make_uint4(pack_bf16x2_rn(lv[0], lv[1]), pack_bf16x2_rn(lv[2], lv[3]),
+                                                         pack_bf16x2_rn(lv[4], lv[5]), pack_bf16x2_rn(lv[6], lv[7]));
       if constexpr (B < BC) {
-        const int zc0 = (q0 == 0) ? B : 0;
-        pt_hi[tb + (size_t)(q0 + jj) * BC + zc0 + i] = zero;
-        pt_lo[tb + (size_t)(q0 + jj) * BC + zc0 + i] = zero;
+        const size_t az = tb + (size_t)(q0 + jj) * BC + zc0 + row0 + g8;
+        *reinterpret_cast<uint4*>(pt_hi + az) = zero4;
+        *reinterpret_cast<uint4*>(pt_lo + az) = zero4;
       }
     }
-    for (int q = tid; q < R * B; q += NT) {
-      const int rr = q / B, jj = q % B, i = row0 + rr;
-      p_hi[tb + (size_t)(q0 + i) * BC + q0 + jj] = __float2bfloat16_rn(tile[rr * LD + jj]);
-      if constexpr (B < BC) p_hi[tb + (size_t)(q0 + i) * BC + ((q0 == 0) ? B : 0) + jj] = zero;
+    // P_hi: image row q0 + i, columns q0 + 8 g .. + 7
+    for (int q = tid; q < R * (B / 8); q += NT) {
+      const int rr = q / (B / 8), g8 = (q % (B / 8)) * 8;
+      const float* src = tile + rr * LD + g8;
+      const size_t at = tb + (size_t)(q0 + row0 + rr) * BC;
+      *reinterpret_cast<uint4*>(p_hi + at + q0 + g8) =
+          make_uint4(pack_bf16x2_rn(src[0], src[1]), pack_bf16x2_rn(src[2], src[3]), pack_bf16x2_rn(src[4], src[5]),
+                     pack_bf16x2_rn(src[6], src[7]));
+      if constexpr (B < BC) *reinterpret_cast<uint4*>(p_hi + at + zc0 + g8) = zero4;
     }
   }
   // keep peers' shared memory alive until every CTA of the cluster is done reading it
   cluster_barrier<CS>();
 }
 
-// Reverse.  dZ lives in registers in the row layout.  For B = 64 the kernel is
-// held to 64 registers a thread so that two CTAs share an SM when many blocks
-// are in flight (a whole model's logits in one launch).
-// Shared memory (floats): tile[R*(B+1)] ck[B] ck1[B] part[NW*B] cs[B] xs[2B]
-template <int B>
+// Reverse.  dZ lives in registers in the row layout.  The iterate after each
+// normalisation is rebuilt from the checkpoint: exp(Z) = a_i K_ij b_j with
+// a_i = e^{max - R_i}, b_j = e^{-C_j} in the linear arithmetic, exp(Z_0 - R_i -
+// C_j) per element in the log domain; the forward kernel's choice is
+// recomputed from the same Z_0.  STAGED: the block's whole checkpoint
+// (iters x 2 x B floats, already turned into a and b in the linear
+// arithmetic) is staged in shared memory once, so an iteration has no global
+// load and two barriers; otherwise each iteration fetches its two vectors.
+// For B = 64 the kernel is held to 64 registers a thread so that two CTAs
+// share an SM when many blocks are in flight (a whole model's logits in one
+// launch).
+// Shared memory (floats): tile[R*(B+1)] ck[B] ck1[B] part[NW*B] cs[B] xs[2B] red[66]
+//                         (+ stage[iters*2*B] when STAGED)
+template <int B, bool STAGED>
 __global__ void __launch_bounds__(SkCfg<B>::NT, B == 64 ? 2 : 1)
-sinkhorn_bwd_kernel(const float* __restrict__ L, const float* __restrict__ ckpt,
-                    const float* __restrict__ dP, int splits, int nblocks,
-                    float* __restrict__ dL, float tau, int iters) {
+sinkhorn_bwd_kernel(const __grid_constant__ SkBwdBatch batch, float tau, int iters) {
   using C = SkCfg<B>;
   pdl_wait();
   pdl_trigger();
+  int blk = blockIdx.x / C::CS, li = 0;
+  while (li + 1 < batch.n && blk >= batch.layer[li].blocks) blk -= batch.layer[li++].blocks;
+  const SkBwdLayer& ly = batch.layer[li];
+  const float* __restrict__ L = ly.L;
+  const float* __restrict__ ckpt = ly.ckpt;
+  const float* __restrict__ dP = ly.dP;
+  float* __restrict__ dL = ly.dL;
+  const int splits = ly.splits, nblocks = ly.blocks;
   constexpr int R = C::R, NT = C::NT, CS = C::CS, TPR = C::TPR, EPR = C::EPR, NW = C::NW, LD = C::LD;
-  constexpr int RPW = 32 / TPR;   // rows per warp
   extern __shared__ __align__(16) float sm[];
   float* tile = sm;
-  float* ck = tile + R * LD;   // C^(k+1)
-  float* ck1 = ck + B;         // C^(k)
+  float* ck = tile + R * LD;   // C^(k+1) (log domain) or b^(k+1) = e^{-C^(k+1)} (linear)
+  float* ck1 = ck + B;         // C^(k) or b^(k)
   float* part = ck1 + B;       // per-warp column partial sums
   float* cs = part + NW * B;   // column sums of dZ
   float* xs = cs + B;          // this CTA's column sums for the cluster, double-buffered
+  float* red = xs + 2 * B;
+  float* stage = red + 66;     // STAGED: [iters][2][B] in the arithmetic's form
 
   const int rank = cta_rank<CS>();
-  const int blk = blockIdx.x / CS;
   const int row0 = rank * R;
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const size_t base = (size_t)blk * B * B;
@@ -274,7 +444,19 @@ sinkhorn_bwd_kernel(const float* __restrict__ L, const float* __restrict__ ckpt,
   __syncthreads();
 #pragma unroll
   for (int e = 0; e < EPR; ++e) zr[e] = tile[r * LD + c + TPR * e];
-  __syncthreads();
+  float lmx = zr[0], lmn = zr[0];
+#pragma unroll
+  for (int e = 1; e < EPR; ++e) {
+    lmx = fmaxf(lmx, zr[e]);
+    lmn = fminf(lmn, zr[e]);
+  }
+  float zmax, zmin;
+  block_range<NT, CS>(lmx, lmn, red, zmax, zmin);   // ends with a barrier: the tile is free again
+  const bool linear = (zmax - zmin) <= kLinearRange;
+  if (linear) {
+#pragma unroll
+    for (int e = 0; e < EPR; ++e) zr[e] = __expf(zr[e] - zmax);   // K
+  }
   // dP summed over the splits in index order
   for (int q = tid; q < R * (B / 4); q += NT) {
     float4 a = reinterpret_cast<const float4*>(dP + base + (size_t)row0 * B)[q];
@@ -286,20 +468,65 @@ sinkhorn_bwd_kernel(const float* __restrict__ L, const float* __restrict__ ckpt,
     float* d = tile + rr * LD + jj;
     d[0] = a.x; d[1] = a.y; d[2] = a.z; d[3] = a.w;
   }
-  for (int jj = tid; jj < B; jj += NT) ck[jj] = ckb[(size_t)(iters - 1) * 2 * B + B + jj];
+  if constexpr (STAGED) {
+    // every (R, C) pair in the form the loop uses: a_i = e^{max - R_i} and
+    // b_j = e^{-C_j} (linear), R and C as they are (log domain)
+    for (int q = tid; q < iters * 2 * B; q += NT) {
+      const float v = ckb[q];
+      const bool is_row = (q / B) % 2 == 0;
+      stage[q] = linear ? __expf(is_row ? zmax - v : -v) : v;
+    }
+    for (int jj = tid; jj < B; jj += NT) ck1[jj] = linear ? 1.f : 0.f;   // b^(0) = 1, C^(0) = 0
+  } else {
+    for (int jj = tid; jj < B; jj += NT) {
+      const float v = ckb[(size_t)(iters - 1) * 2 * B + B + jj];
+      ck[jj] = linear ? __expf(-v) : v;
+    }
+  }
   __syncthreads();
-  float myR = ckb[(size_t)(iters - 1) * 2 * B + row0 + r];
-  // dZ = dP (.) P with P = exp(z - R^(K) - C^(K))
+  // the vectors after iteration k + 1 (k = iters - 1 ... 0): row values of this thread's row,
+  // column values, and the column values after iteration k
+  auto rowv = [&](int k) -> float {
+    if constexpr (STAGED) return stage[(size_t)k * 2 * B + row0 + r];
+    else {
+      const float v = ckb[(size_t)k * 2 * B + row0 + r];
+      return linear ? __expf(zmax - v) : v;
+    }
+  };
+  auto colv = [&](int k) -> const float* {
+    if constexpr (STAGED) return stage + (size_t)k * 2 * B + B;
+    else return ck;
+  };
+  auto colv1 = [&](int k) -> const float* {
+    if constexpr (STAGED) return k > 0 ? stage + (size_t)(k - 1) * 2 * B + B : ck1;
+    else return ck1;
+  };
+  // dZ = dP (.) P with P the final iterate
+  {
+    const float rv = rowv(iters - 1);
+    const float* cvp = colv(iters - 1);
+    if (linear) {
 #pragma unroll
-  for (int e = 0; e < EPR; ++e) dz[e] = tile[r * LD + c + TPR * e] * __expf(zr[e] - myR - ck[c + TPR * e]);
+      for (int e = 0; e < EPR; ++e) dz[e] = tile[r * LD + c + TPR * e] * (rv * zr[e] * cvp[c + TPR * e]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < EPR; ++e) dz[e] = tile[r * LD + c + TPR * e] * __expf(zr[e] - rv - cvp[c + TPR * e]);
+    }
+  }
 
   for (int k = iters - 1; k >= 0; --k) {
-    __syncthreads();   // previous iteration done with ck, ck1, part, cs
-    for (int jj = tid; jj < B; jj += NT) {
-      ck[jj] = ckb[(size_t)k * 2 * B + B + jj];
-      ck1[jj] = (k > 0) ? ckb[(size_t)(k - 1) * 2 * B + B + jj] : 0.f;
+    if constexpr (!STAGED) {
+      __syncthreads();   // previous iteration done with ck, ck1, part, cs
+      for (int jj = tid; jj < B; jj += NT) {
+        const float v = ckb[(size_t)k * 2 * B + B + jj];
+        const float v1 = (k > 0) ? ckb[(size_t)(k - 1) * 2 * B + B + jj] : 0.f;
+        ck[jj] = linear ? __expf(-v) : v;
+        ck1[jj] = linear ? __expf(-v1) : v1;
+      }
     }
-    myR = ckb[(size_t)k * 2 * B + row0 + r];
+    const float rv = rowv(k);
+    const float* cvp = colv(k);
+    const float* cvp1 = colv1(k);
     // column sums of dZ: over the rows of this warp (lanes with equal c), then over warps
 #pragma unroll
     for (int e = 0; e < EPR; ++e) {
@@ -325,16 +552,29 @@ sinkhorn_bwd_kernel(const float* __restrict__ L, const float* __restrict__ ckpt,
       }
     }
     __syncthreads();
-    // column step: dZ -= exp(Z') colsum, Z' = z - R^(k+1) - C^(k+1)
+    if (linear) {
+      // column step: dZ -= exp(Z') colsum with exp(Z') = a_i K_ij b_j^(k+1)
 #pragma unroll
-    for (int e = 0; e < EPR; ++e) dz[e] -= __expf(zr[e] - myR - ck[c + TPR * e]) * cs[c + TPR * e];
-    // row step: dZ -= exp(Z') rowsum, Z' = z - R^(k+1) - C^(k)
-    float rs = 0.f;
+      for (int e = 0; e < EPR; ++e) dz[e] -= (rv * zr[e] * cvp[c + TPR * e]) * cs[c + TPR * e];
+      // row step: dZ -= exp(Z') rowsum with exp(Z') = a_i K_ij b_j^(k)
+      float rs = 0.f;
 #pragma unroll
-    for (int e = 0; e < EPR; ++e) rs += dz[e];
-    rs = group_sum<TPR>(rs);
+      for (int e = 0; e < EPR; ++e) rs += dz[e];
+      rs = group_sum<TPR>(rs);
 #pragma unroll
-    for (int e = 0; e < EPR; ++e) dz[e] -= __expf(zr[e] - myR - ck1[c + TPR * e]) * rs;
+      for (int e = 0; e < EPR; ++e) dz[e] -= (rv * zr[e] * cvp1[c + TPR * e]) * rs;
+    } else {
+      // column step: dZ -= exp(Z') colsum, Z' = z - R^(k+1) - C^(k+1)
+#pragma unroll
+      for (int e = 0; e < EPR; ++e) dz[e] -= __expf(zr[e] - rv - cvp[c + TPR * e]) * cs[c + TPR * e];
+      // row step: dZ -= exp(Z') rowsum, Z' = z - R^(k+1) - C^(k)
+      float rs = 0.f;
+#pragma unroll
+      for (int e = 0; e < EPR; ++e) rs += dz[e];
+      rs = group_sum<TPR>(rs);
+#pragma unroll
+      for (int e = 0; e < EPR; ++e) dz[e] -= __expf(zr[e] - rv - cvp1[c + TPR * e]) * rs;
+    }
   }
   // dL = dZ_0 / tau, staged for coalesced stores
   __syncthreads();
@@ -346,63 +586,129 @@ sinkhorn_bwd_kernel(const float* __restrict__ L, const float* __restrict__ ckpt,
     dL[base + (size_t)(row0 + rr) * B + jj] = tile[rr * LD + jj];
   }
   cluster_barrier<CS>();
-  (void)RPW;
+}
+
+// out = sum over s of parts[s] (n floats each, summed in index order), float4-wide.
+__global__ void __launch_bounds__(256) sum_splits_kernel(const float4* __restrict__ parts, int splits, size_t n4,
+                                                         float4* __restrict__ out) {
+  pdl_wait();
+  pdl_trigger();
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n4; i += (size_t)gridDim.x * blockDim.x) {
+    float4 a = parts[i];
+    for (int s = 1; s < splits; ++s) {
+      const float4 b = parts[(size_t)s * n4 + i];
+      a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+    }
+    out[i] = a;
+  }
 }
 
 template <int B> constexpr size_t fwd_smem() {
   using C = SkCfg<B>;
-  return sizeof(float) * (C::R * C::LD + C::R + B + 4 * B);
+  return sizeof(float) * (C::R * C::LD + C::R + B + 4 * B + 66);
 }
 template <int B> constexpr size_t bwd_smem() {
   using C = SkCfg<B>;
-  return sizeof(float) * (C::R * C::LD + 2 * B + C::NW * B + B + 2 * B);
+  return sizeof(float) * (C::R * C::LD + 2 * B + C::NW * B + B + 2 * B + 66);
 }
 
+// the reverse kernel stages the checkpoint in shared memory up to this many bytes
+constexpr size_t kStageBytes = 64 * 1024;
+
 template <int B>
-lcp_status fwd_b(const float* L, float* P, float* ckpt, __nv_bfloat16* a, __nv_bfloat16* b,
-                 __nv_bfloat16* c, unsigned* zero_word, int nblocks, float tau, int iters, cudaStream_t st) {
+lcp_status fwd_b(const SkFwdBatch& batch, int blocks, float tau, int iters, cudaStream_t st) {
   using C = SkCfg<B>;
   const lcp_status s0 = ensure_smem_limit(reinterpret_cast<const void*>(sinkhorn_fwd_kernel<B>), (int)fwd_smem<B>(),
                                           "sinkhorn_fwd");
   if (s0 != LCP_OK) return s0;
-  return launch_kernel(sinkhorn_fwd_kernel<B>, dim3(nblocks * C::CS), dim3(C::NT), fwd_smem<B>(), st, C::CS, true,
-                       "sinkhorn_fwd", L, P, ckpt, a, b, c, zero_word, tau, iters);
+  return launch_kernel(sinkhorn_fwd_kernel<B>, dim3(blocks * C::CS), dim3(C::NT), fwd_smem<B>(), st, C::CS, true,
+                       "sinkhorn_fwd", batch, tau, iters);
 }
+
 template <int B>
-lcp_status bwd_b(const float* L, const float* ckpt, const float* dP, int splits, float* dL,
-                 int nblocks, float tau, int iters, cudaStream_t st) {
+lcp_status bwd_b(const SkBwdBatch& batch, int blocks, float tau, int iters, cudaStream_t st) {
   using C = SkCfg<B>;
-  const lcp_status s0 = ensure_smem_limit(reinterpret_cast<const void*>(sinkhorn_bwd_kernel<B>), (int)bwd_smem<B>(),
-                                          "sinkhorn_bwd");
+  const size_t stage = (size_t)iters * 2 * B * sizeof(float);
+  if (stage <= kStageBytes) {
+    const size_t bytes = bwd_smem<B>() + stage;
+    const lcp_status s0 = ensure_smem_limit(reinterpret_cast<const void*>(sinkhorn_bwd_kernel<B, true>), (int)bytes,
+                                            "sinkhorn_bwd");
+    if (s0 != LCP_OK) return s0;
+    return launch_kernel(sinkhorn_bwd_kernel<B, true>, dim3(blocks * C::CS), dim3(C::NT), bytes, st, C::CS, true,
+                         "sinkhorn_bwd", batch, tau, iters);
+  }
+  const lcp_status s0 = ensure_smem_limit(reinterpret_cast<const void*>(sinkhorn_bwd_kernel<B, false>),
+                                          (int)bwd_smem<B>(), "sinkhorn_bwd");
   if (s0 != LCP_OK) return s0;
-  return launch_kernel(sinkhorn_bwd_kernel<B>, dim3(nblocks * C::CS), dim3(C::NT), bwd_smem<B>(), st, C::CS, true,
-                       "sinkhorn_bwd", L, ckpt, dP, splits, nblocks, dL, tau, iters);
+  return launch_kernel(sinkhorn_bwd_kernel<B, false>, dim3(blocks * C::CS), dim3(C::NT), bwd_smem<B>(), st, C::CS,
+                       true, "sinkhorn_bwd", batch, tau, iters);
+}
+
+// Launches `kernel_b` over `layers` in batches of up to kSkMaxLayers layers.
+template <typename Layer, typename Batch, typename F>
+lcp_status in_batches(const Layer* layers, int n, F launch) {
+  for (int first = 0; first < n; first += kSkMaxLayers) {
+    Batch b{};
+    b.n = std::min(kSkMaxLayers, n - first);
+    int blocks = 0;
+    for (int i = 0; i < b.n; ++i) {
+      b.layer[i] = layers[first + i];
+      blocks += b.layer[i].blocks;
+    }
+    if (blocks == 0) continue;
+    const lcp_status s = launch(b, blocks);
+    if (s != LCP_OK) return s;
+  }
+  return LCP_OK;
 }
 
 }  // namespace
 
+lcp_status launch_sinkhorn_fwd_batch(const SkFwdLayer* layers, int n, int B, float tau, int iters,
+                                     cudaStream_t st) {
+  return in_batches<SkFwdLayer, SkFwdBatch>(layers, n, [&](const SkFwdBatch& b, int blocks) -> lcp_status {
+    switch (B) {
+      case 32: return fwd_b<32>(b, blocks, tau, iters, st);
+      case 64: return fwd_b<64>(b, blocks, tau, iters, st);
+      case 128: return fwd_b<128>(b, blocks, tau, iters, st);
+      case 256: return fwd_b<256>(b, blocks, tau, iters, st);
+    }
+    return fail(LCP_ERR_SHAPE, "sinkhorn_fwd: unsupported block size %d", B);
+  });
+}
+
 lcp_status launch_sinkhorn_fwd(const float* L, float* P, float* ckpt, __nv_bfloat16* img_pt_hi,
                                __nv_bfloat16* img_pt_lo, __nv_bfloat16* img_p_hi, unsigned* zero_word,
                                int nblocks, int B, float tau, int iters, cudaStream_t st) {
-  switch (B) {
-    case 32: return fwd_b<32>(L, P, ckpt, img_pt_hi, img_pt_lo, img_p_hi, zero_word, nblocks, tau, iters, st);
-    case 64: return fwd_b<64>(L, P, ckpt, img_pt_hi, img_pt_lo, img_p_hi, zero_word, nblocks, tau, iters, st);
-    case 128: return fwd_b<128>(L, P, ckpt, img_pt_hi, img_pt_lo, img_p_hi, zero_word, nblocks, tau, iters, st);
-    case 256: return fwd_b<256>(L, P, ckpt, img_pt_hi, img_pt_lo, img_p_hi, zero_word, nblocks, tau, iters, st);
-  }
-  return fail(LCP_ERR_SHAPE, "sinkhorn_fwd: unsupported block size %d", B);
+  const SkFwdLayer one{L, P, ckpt, img_pt_hi, img_pt_lo, img_p_hi, zero_word, nblocks};
+  return launch_sinkhorn_fwd_batch(&one, 1, B, tau, iters, st);
+}
+
+lcp_status launch_sum_splits(const float* parts, int splits, size_t n, float* out, cudaStream_t st) {
+  const size_t n4 = n / 4;
+  const int grid = (int)std::min<size_t>((n4 + 255) / 256, 148 * 8);
+  return launch_kernel(sum_splits_kernel, dim3(grid > 0 ? grid : 1), dim3(256), 0, st, 1, true, "sum_splits",
+                       reinterpret_cast<const float4*>(parts), splits, n4, reinterpret_cast<float4*>(out));
+}
+
+lcp_status launch_sinkhorn_bwd_batch(const SkBwdLayer* layers, int n, int B, float tau, int iters,
+                                     cudaStream_t st) {
+  return in_batches<SkBwdLayer, SkBwdBatch>(layers, n, [&](const SkBwdBatch& b, int blocks) -> lcp_status {
+    switch (B) {
+      case 32: return bwd_b<32>(b, blocks, tau, iters, st);
+      case 64: return bwd_b<64>(b, blocks, tau, iters, st);
+      case 128: return bwd_b<128>(b, blocks, tau, iters, st);
+      case 256: return bwd_b<256>(b, blocks, tau, iters, st);
+    }
+    return fail(LCP_ERR_SHAPE, "sinkhorn_bwd: unsupported block size %d", B);
+  });
 }
 
 lcp_status launch_sinkhorn_bwd(const float* L, const float* ckpt, const float* dP, int splits,
                                float* dL, int nblocks, int B, float tau, int iters,
                                cudaStream_t st) {
-  switch (B) {
-    case 32: return bwd_b<32>(L, ckpt, dP, splits, dL, nblocks, tau, iters, st);
-    case 64: return bwd_b<64>(L, ckpt, dP, splits, dL, nblocks, tau, iters, st);
-    case 128: return bwd_b<128>(L, ckpt, dP, splits, dL, nblocks, tau, iters, st);
-    case 256: return bwd_b<256>(L, ckpt, dP, splits, dL, nblocks, tau, iters, st);
-  }
-  return fail(LCP_ERR_SHAPE, "sinkhorn_bwd: unsupported block size %d", B);
+  const SkBwdLayer one{L, ckpt, dP, dL, splits, nblocks};
+  return launch_sinkhorn_bwd_batch(&one, 1, B, tau, iters, st);
 }
 
 }  // namespace lcp
