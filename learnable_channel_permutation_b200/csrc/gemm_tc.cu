@@ -2,6 +2,13 @@
 // the calibration outputs Y_d = X W^T and Y_s = X At^T (PermLLM summary,
 // "optimization objective": the dense and sparse outputs), and the weight
 // gradient dAt = G^T X of the reverse pass.
+//
+// The calibration products can also run with the cosine-loss reduction in the
+// epilogue (LOSS mode): both outputs of the same 256 tokens x 128 channels come
+// out of one MMA, and the epilogue writes, instead of the two float32 outputs,
+// per-token partial sums <y_d, y_s>, |y_d|^2, |y_s|^2 over each 64-channel
+// slot and the pair D = Y_d - Y_s, Y_s in bf16 -- all the loss and its
+// gradient G need (see loss.cu, loss_pair_kernel).
 
 #include "tc_common.cuh"
 
@@ -53,11 +60,20 @@ struct PairSched {
   }
 };
 
-template <bool A_MN, bool B_MN, bool OUT_BF16>
+// LOSS mode (calibration products only): item = 256 tokens x 128 channels of
+// both problems.  CTA 0 of the pair stages the channels' rows of B0 = W, CTA 1
+// the same rows of B1 = At, so the N = 256 MMA leaves accumulator columns
+// [0, 128) = Y_d and [128, 256) = Y_s (a half item: 64 channels, N = 128,
+// columns [0, 64) and [64, 128)).  D0 receives D = Y_d - Y_s and D1 Y_s, both
+// bf16 [M, N] with row stride ldd; part[row * nslots + s] the float4
+// (<y_d, y_s>, |y_d|^2, |y_s|^2, 0) of channels [64 s, 64 s + 64).
+template <bool A_MN, bool B_MN, bool OUT_BF16, bool LOSS>
 __global__ void __launch_bounds__(GM_THREADS, 1)
 gemm_pair_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                     const __grid_constant__ CUtensorMap tmB1, void* __restrict__ D0, void* __restrict__ D1,
-                    int M, int N, int K, int ldd, int nprob) {
+                    float4* __restrict__ part, int nslots, int M, int N, int K, int ldd, int nprob) {
+  static_assert(!LOSS || (!A_MN && !B_MN && !OUT_BF16), "the loss epilogue belongs to the calibration products");
+  constexpr int BNT = LOSS ? 128 : G2_BN;   // output channels per item (of each problem in LOSS mode)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sA = smem;
@@ -95,7 +111,7 @@ gemm_pair_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
   pdl_wait();           // operands come from the previous kernel
   pdl_trigger();
 
-  const int mtiles = cdiv(M, G2_BM), ntiles = cdiv(N, G2_BN);
+  const int mtiles = cdiv(M, G2_BM), ntiles = cdiv(N, BNT);
   const int total = mtiles * ntiles * nprob;
   const int nk = cdiv(K, G2_BK);
   const PairSched sched(total, npairs);
@@ -110,10 +126,12 @@ gemm_pair_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         sched.at(it, tile, half);
         const int mt = tile % mtiles, rest = tile / mtiles;
         const int nt = rest % ntiles, prob = rest / ntiles;
-        const CUtensorMap* mb = prob ? &tmB1 : &tmB0;
+        const CUtensorMap* mb = (LOSS ? rank : prob) ? &tmB1 : &tmB0;
         // each CTA stages half of the tile's B rows: 128 of a whole tile, 64 of a half
+        // (LOSS: CTA r stages all the item's channels of problem r)
         const int a_row = mt * G2_BM + (int)rank * 128;
-        const int b_row = nt * G2_BN + (half < 0 ? (int)rank * 128 : half * 128 + (int)rank * 64);
+        const int b_row = LOSS ? nt * BNT + (half < 0 ? 0 : half * 64)
+                               : nt * G2_BN + (half < 0 ? (int)rank * 128 : half * 128 + (int)rank * 64);
         const uint32_t bytes = half < 0 ? 2 * G2_HALF : G2_HALF + G2_HALF / 2;
         bool ok = true;
         for (int kb = 0; kb < nk; ++kb) {
@@ -203,6 +221,64 @@ gemm_pair_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       tc_fence_after();
       const int mt = tile % mtiles, rest = tile / mtiles;
       const int nt = rest % ntiles, prob = rest / ntiles;
+      if constexpr (LOSS) {
+        const int row = mt * G2_BM + (int)rank * 128 + q * 32 + lane;
+        const int ncol = half < 0 ? 128 : 64;             // channels of each problem in this item
+        const int col_base = nt * BNT + (half < 0 ? 0 : half * 64);
+        const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * G2_BN);
+#pragma unroll 1
+        for (int s64 = 0; s64 < ncol / 64; ++s64) {
+          float dot = 0.f, nd = 0.f, ns = 0.f;
+#pragma unroll 1
+          for (int h = 0; h < 2; ++h) {
+            const int cc = s64 * 64 + h * 32;
+            uint32_t rd[32], rs[32];
+            tmem_ld32(tbase + (uint32_t)cc, rd);
+            tmem_ld32(tbase + (uint32_t)(ncol + cc), rs);
+            tmem_ld_wait();
+#pragma unroll
+            for (int v = 0; v < 32; ++v) {
+              const float yd = __uint_as_float(rd[v]), ys = __uint_as_float(rs[v]);
+              dot = fmaf(yd, ys, dot);
+              nd = fmaf(yd, yd, nd);
+              ns = fmaf(ys, ys, ns);
+            }
+            const int col0 = col_base + cc;
+            if (row < M && col0 < N) {
+              __nv_bfloat16* od = static_cast<__nv_bfloat16*>(D0) + (size_t)row * ldd + col0;
+              __nv_bfloat16* os = static_cast<__nv_bfloat16*>(D1) + (size_t)row * ldd + col0;
+#pragma unroll
+              for (int v = 0; v < 4; ++v) {
+                if (col0 + 8 * v < N) {
+                  float fd[8], fs[8];
+#pragma unroll
+                  for (int u = 0; u < 8; ++u) {
+                    fs[u] = __uint_as_float(rs[8 * v + u]);
+                    fd[u] = __uint_as_float(rd[8 * v + u]) - fs[u];
+                  }
+                  uint4 ud, us;
+                  ud.x = pack_bf16x2(fd[0], fd[1]);
+                  ud.y = pack_bf16x2(fd[2], fd[3]);
+                  ud.z = pack_bf16x2(fd[4], fd[5]);
+                  ud.w = pack_bf16x2(fd[6], fd[7]);
+                  us.x = pack_bf16x2(fs[0], fs[1]);
+                  us.y = pack_bf16x2(fs[2], fs[3]);
+                  us.z = pack_bf16x2(fs[4], fs[5]);
+                  us.w = pack_bf16x2(fs[6], fs[7]);
+                  reinterpret_cast<uint4*>(od)[v] = ud;
+                  reinterpret_cast<uint4*>(os)[v] = us;
+                }
+              }
+            }
+          }
+          const int slot = (col_base + s64 * 64) / 64;
+          if (row < M && slot < nslots) part[(size_t)row * nslots + slot] = make_float4(dot, nd, ns, 0.f);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
+        continue;
+      }
       const int row = mt * G2_BM + (int)rank * 128 + q * 32 + lane;
       const int chunks = half < 0 ? G2_BN / 32 : G2_BN / 64;
       const int col_base = nt * G2_BN + (half < 0 ? 0 : half * (G2_BN / 2));
@@ -258,14 +334,14 @@ gemm_pair_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 
 template <typename K>
 lcp_status launch_pair(K kernel, int tiles, const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
-                       void* d0, void* d1, int M, int N, int Kd, int ldd, int nprob, cudaStream_t st,
-                       const char* what) {
+                       void* d0, void* d1, float4* part, int nslots, int M, int N, int Kd, int ldd, int nprob,
+                       cudaStream_t st, const char* what) {
   TC_TRY(set_smem(kernel, G2_SMEM, what));
   const int max_pairs = num_sms() / 2;
   // few tiles: twice as many pairs, each taking one half tile
   const int pairs = 2 * tiles <= max_pairs ? 2 * tiles : (tiles < max_pairs ? tiles : max_pairs);
-  return launch_kernel(kernel, dim3(2 * pairs), dim3(GM_THREADS), G2_SMEM, st, 2, true, what, a, b0, b1, d0, d1, M, N,
-                       Kd, ldd, nprob);
+  return launch_kernel(kernel, dim3(2 * pairs), dim3(GM_THREADS), G2_SMEM, st, 2, true, what, a, b0, b1, d0, d1, part,
+                       nslots, M, N, Kd, ldd, nprob);
 }
 
 }  // namespace
@@ -281,8 +357,24 @@ lcp_status launch_calib_gemm_tc(const __nv_bfloat16* X, const __nv_bfloat16* W, 
   TC_TRY(make_map(&mB0, W, cin, cout, 64, 64, "calib_gemm W"));
   TC_TRY(make_map(&mB1, Ys ? (const void*)At : (const void*)W, cin, cout, 64, 64, "calib_gemm At"));
   const int tiles = cdiv(tokens, G2_BM) * cdiv(cout, G2_BN) * nprob;
-  return launch_pair(gemm_pair_tc_kernel<false, false, false>, tiles, mA, mB0, mB1, Yd, Ys, tokens, cout, cin,
-                     cout, nprob, st, "calib_gemm");
+  return launch_pair(gemm_pair_tc_kernel<false, false, false, false>, tiles, mA, mB0, mB1, Yd, Ys, nullptr, 0, tokens,
+                     cout, cin, cout, nprob, st, "calib_gemm");
+}
+
+int calib_loss_slots(int cout) { return cdiv(cout, 64); }
+
+lcp_status launch_calib_loss_tc(const __nv_bfloat16* X, const __nv_bfloat16* W, const __nv_bfloat16* At,
+                                __nv_bfloat16* D, __nv_bfloat16* Ys, float* partials, int tokens, int cout, int cin,
+                                cudaStream_t st) {
+  // A in boxes of 128 rows; B in boxes of 64 rows, CTA 0 of a pair from W, CTA 1 from At
+  CUtensorMap mA, mB0, mB1;
+  TC_TRY(make_map(&mA, X, cin, tokens, 64, 128, "calib_loss X"));
+  TC_TRY(make_map(&mB0, W, cin, cout, 64, 64, "calib_loss W"));
+  TC_TRY(make_map(&mB1, At, cin, cout, 64, 64, "calib_loss At"));
+  const int tiles = cdiv(tokens, G2_BM) * cdiv(cout, 128);
+  return launch_pair(gemm_pair_tc_kernel<false, false, false, true>, tiles, mA, mB0, mB1, D, Ys,
+                     reinterpret_cast<float4*>(partials), calib_loss_slots(cout), tokens, cout, cin, cout, 1, st,
+                     "calib_loss");
 }
 
 lcp_status launch_bwd_gemm_tc(const __nv_bfloat16* G, const __nv_bfloat16* X, __nv_bfloat16* dAt, int tokens,
@@ -291,8 +383,8 @@ lcp_status launch_bwd_gemm_tc(const __nv_bfloat16* G, const __nv_bfloat16* X, __
   TC_TRY(make_map(&mA, G, cout, tokens, 64, 64, "grad_gemm G"));
   TC_TRY(make_map(&mB, X, cin, tokens, 64, 64, "grad_gemm X"));
   const int tiles = cdiv(cout, G2_BM) * cdiv(cin, G2_BN);
-  return launch_pair(gemm_pair_tc_kernel<true, true, true>, tiles, mA, mB, mB, dAt, nullptr, cout, cin, tokens, cin,
-                     1, st, "grad_gemm");
+  return launch_pair(gemm_pair_tc_kernel<true, true, true, false>, tiles, mA, mB, mB, dAt, nullptr, nullptr, 0, cout,
+                     cin, tokens, cin, 1, st, "grad_gemm");
 }
 
 }  // namespace lcp

@@ -121,7 +121,7 @@ template <typename TG, int NTH, int QPT, bool PREFETCH>
 __global__ void __launch_bounds__(NTH, PREFETCH ? 2 : 1)
 loss_fused_kernel(const float* __restrict__ Yd, const float* __restrict__ Ys, float* __restrict__ stats,
                   TG* __restrict__ G, float* __restrict__ loss, unsigned* __restrict__ counter, int cout,
-                  int tokens, float inv_T) {
+                  int tokens, int norm, float inv_T) {
   pdl_wait();
   pdl_trigger();
   constexpr int NWARP = NTH / 32;
@@ -209,13 +209,126 @@ loss_fused_kernel(const float* __restrict__ Yd, const float* __restrict__ Ys, fl
   if (threadIdx.x == 0) {
     double tot = 0.0;
     for (int w = 0; w < NWARP; ++w) tot += redd[w];
-    *loss = (float)(tot / tokens);
+    *loss = (float)(tot / norm);
+    *counter = 0u;
+  }
+}
+
+// The loss and its gradient from the calibration GEMM's loss epilogue
+// (gemm_tc.cu, LOSS mode): per token t, the float4 partial sums
+// (<y_d, y_s>, |y_d|^2, |y_s|^2, 0) of its nslots 64-channel slots, and the
+// pair D = Y_d - Y_s, Y_s in bf16.  One warp per token, warps persistent over
+// the tokens, no barrier between them: the warp issues its first row loads,
+// sums the slot partials (lane-strided, then a butterfly: a fixed order) into
+// c_t, and streams the rows in steps of NS 16-byte chunks a lane, the next
+// step's loads in flight, writing G_t = ca y_d + cb y_s with y_d = D + Y_s,
+// y_s = Y_s and the coefficients of token_grad in bf16, and stats[t] as
+// loss_token_kernel writes it.  The CTA that finishes last (counter zero at
+// launch) sums the cosines in index order into the loss and re-zeroes the
+// counter: deterministic.
+constexpr int kPairThreads = 256;
+
+template <int NS>
+__global__ void __launch_bounds__(kPairThreads)
+loss_pair_kernel(const __nv_bfloat16* __restrict__ D, const __nv_bfloat16* __restrict__ Ys,
+                 const float4* __restrict__ part, int nslots, float* __restrict__ stats,
+                 __nv_bfloat16* __restrict__ G, float* __restrict__ loss, unsigned* __restrict__ counter, int cout,
+                 int tokens, int norm, float inv_T) {
+  constexpr int NWARP = kPairThreads / 32, STEP = 32 * NS;   // chunks of one step
+  pdl_wait();
+  pdl_trigger();
+  __shared__ double redd[NWARP];
+  __shared__ int is_last;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int gw = blockIdx.x * NWARP + warp, nw = gridDim.x * NWARP;
+  const int oct = cout / 8;   // 16-byte chunks of 8 bf16 per row
+  for (int t = gw; t < tokens; t += nw) {
+    const uint4* d8 = reinterpret_cast<const uint4*>(D + (size_t)t * cout);
+    const uint4* y8 = reinterpret_cast<const uint4*>(Ys + (size_t)t * cout);
+    uint4* g8 = reinterpret_cast<uint4*>(G + (size_t)t * cout);
+    uint4 d[NS], y[NS], dn[NS], yn[NS];
+    auto load = [&](int q0, uint4 (&dd)[NS], uint4 (&yy)[NS]) {
+#pragma unroll
+      for (int u = 0; u < NS; ++u) {
+        const int q = q0 + lane + 32 * u;
+        if (q < oct) {
+          dd[u] = __ldcs(d8 + q);
+          yy[u] = __ldcs(y8 + q);
+        }
+      }
+    };
+    load(0, dn, yn);
+    float dot = 0.f, nd2 = 0.f, ns2 = 0.f;
+    for (int k = lane; k < nslots; k += 32) {
+      const float4 p = __ldcs(part + (size_t)t * nslots + k);
+      dot += p.x;
+      nd2 += p.y;
+      ns2 += p.z;
+    }
+    dot = warp_sum(dot);
+    nd2 = warp_sum(nd2);
+    ns2 = warp_sum(ns2);
+    const float den = sqrtf(nd2) * sqrtf(ns2);
+    const float c = dot / fmaxf(den, kCosEps);
+    if (lane == 0) {
+      float4 sv;
+      sv.x = dot; sv.y = nd2; sv.z = ns2; sv.w = c;
+      reinterpret_cast<float4*>(stats)[t] = sv;
+    }
+    const bool ok = den > kCosEps;
+    const float ca = ok ? -inv_T / den : -inv_T / kCosEps;   // coefficient of y_d
+    const float cb = ok ? inv_T * c / ns2 : 0.f;             // coefficient of y_s
+    for (int q0 = 0; q0 < oct; q0 += STEP) {
+#pragma unroll
+      for (int u = 0; u < NS; ++u) { d[u] = dn[u]; y[u] = yn[u]; }
+      if (q0 + STEP < oct) load(q0 + STEP, dn, yn);   // the next step's chunks, in flight meanwhile
+#pragma unroll
+      for (int u = 0; u < NS; ++u) {
+        const int q = q0 + lane + 32 * u;
+        if (q < oct) {
+          const uint32_t dw[4] = {d[u].x, d[u].y, d[u].z, d[u].w};
+          const uint32_t yw[4] = {y[u].x, y[u].y, y[u].z, y[u].w};
+          uint32_t gwd[4];
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const float2 df = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&dw[v]));
+            const float2 yf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&yw[v]));
+            const __nv_bfloat162 gv =
+                __floats2bfloat162_rn(ca * (df.x + yf.x) + cb * yf.x, ca * (df.y + yf.y) + cb * yf.y);
+            gwd[v] = *reinterpret_cast<const uint32_t*>(&gv);
+          }
+          g8[q] = make_uint4(gwd[0], gwd[1], gwd[2], gwd[3]);
+        }
+      }
+    }
+  }
+  // last CTA: the loss (as in loss_fused_kernel).  Every lane 0 wrote its
+  // warp's statistics; the barrier and thread 0's fence order them before the
+  // CTA's vote.
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    is_last = (atomicAdd(counter, 1u) == gridDim.x - 1u);
+  }
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  double sum = 0.0;
+  for (int u = threadIdx.x; u < tokens; u += kPairThreads) sum += 1.0 - (double)__ldcg(stats + 4 * (size_t)u + 3);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if (lane == 0) redd[warp] = sum;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double tot = 0.0;
+    for (int w = 0; w < NWARP; ++w) tot += redd[w];
+    *loss = (float)(tot / norm);
     *counter = 0u;
   }
 }
 
 __global__ void __launch_bounds__(1024)
-loss_reduce_kernel(const float* __restrict__ stats, float* __restrict__ loss, int tokens) {
+loss_reduce_kernel(const float* __restrict__ stats, float* __restrict__ loss, int tokens, int norm) {
   pdl_wait();
   pdl_trigger();
   __shared__ double red[32];
@@ -228,15 +341,15 @@ loss_reduce_kernel(const float* __restrict__ stats, float* __restrict__ loss, in
   if (threadIdx.x == 0) {
     double tot = 0.0;
     for (int w = 0; w < 32; ++w) tot += red[w];
-    *loss = (float)(tot / tokens);
+    *loss = (float)(tot / norm);
   }
 }
 
 }  // namespace
 
 lcp_status launch_loss_token(const float* Yd, const float* Ys, float* stats, void* G,
-                             lcp_dtype gdt, int cout, int tokens, cudaStream_t st) {
-  const float inv_T = 1.0f / (float)tokens;
+                             lcp_dtype gdt, int cout, int tokens, int norm, cudaStream_t st) {
+  const float inv_T = 1.0f / (float)norm;
   const dim3 grid(tokens), block(NT);
   if (!G)
     return launch_kernel(loss_token_kernel<float, false>, grid, block, 0, st, 1, true, "loss_token", Yd, Ys, stats,
@@ -249,8 +362,8 @@ lcp_status launch_loss_token(const float* Yd, const float* Ys, float* stats, voi
 }
 
 lcp_status launch_loss_grad(const float* Yd, const float* Ys, const float* stats, void* G,
-                            lcp_dtype gdt, int cout, int tokens, cudaStream_t st) {
-  const float inv_T = 1.0f / (float)tokens;
+                            lcp_dtype gdt, int cout, int tokens, int norm, cudaStream_t st) {
+  const float inv_T = 1.0f / (float)norm;
   const dim3 grid(tokens), block(NT);
   if (gdt == LCP_F32)
     return launch_kernel(loss_grad_kernel<float>, grid, block, 0, st, 1, true, "loss_grad", Yd, Ys, stats,
@@ -262,8 +375,8 @@ lcp_status launch_loss_grad(const float* Yd, const float* Ys, const float* stats
 bool loss_fused_supported(int cout) { return cout <= 8 * 4 * 512; }
 
 lcp_status launch_loss_fused(const float* Yd, const float* Ys, float* stats, void* G, lcp_dtype gdt,
-                             float* loss, unsigned* counter, int cout, int tokens, cudaStream_t st) {
-  const float inv_T = 1.0f / (float)tokens;
+                             float* loss, unsigned* counter, int cout, int tokens, int norm, cudaStream_t st) {
+  const float inv_T = 1.0f / (float)norm;
   const int quads = cout / 4;
   int sms = 148, dev = 0;
   cudaGetDevice(&dev);
@@ -271,7 +384,7 @@ lcp_status launch_loss_fused(const float* Yd, const float* Ys, float* stats, voi
   const dim3 grid(tokens < 2 * sms ? tokens : 2 * sms);
 #define LCP_LOSS_FUSED(TG, NTH, QPT)                                                                             \
   return launch_kernel(loss_fused_kernel<TG, NTH, QPT, (QPT <= 4)>, grid, dim3(NTH), 0, st, 1, true, "loss_fused", \
-                       Yd, Ys, stats, static_cast<TG*>(G), loss, counter, cout, tokens, inv_T)
+                       Yd, Ys, stats, static_cast<TG*>(G), loss, counter, cout, tokens, norm, inv_T)
   if (gdt == LCP_F32) {
     if (quads <= 4 * 256) LCP_LOSS_FUSED(float, 256, 4);
     if (quads <= 8 * 256) LCP_LOSS_FUSED(float, 256, 8);
@@ -283,8 +396,31 @@ lcp_status launch_loss_fused(const float* Yd, const float* Ys, float* stats, voi
 #undef LCP_LOSS_FUSED
 }
 
-lcp_status launch_loss_reduce(const float* stats, float* loss, int tokens, cudaStream_t st) {
-  return launch_kernel(loss_reduce_kernel, dim3(1), dim3(1024), 0, st, 1, true, "loss_reduce", stats, loss, tokens);
+bool loss_pair_supported(int cout) { return cout <= 16384; }
+
+lcp_status launch_loss_pair(const __nv_bfloat16* D, const __nv_bfloat16* Ys, const float* partials, int nslots,
+                            float* stats, __nv_bfloat16* G, float* loss, unsigned* counter, int cout, int tokens,
+                            int norm, cudaStream_t st) {
+  constexpr int NS = 4;
+  int sms = 148, dev = 0, per_sm = 1;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, loss_pair_kernel<NS>, kPairThreads, 0) != cudaSuccess ||
+      per_sm < 1) {
+    cudaGetLastError();   // this query's own error
+    per_sm = 1;
+  }
+  const int warps = (kPairThreads / 32);
+  const int need = (tokens + warps - 1) / warps;   // CTAs for one token a warp
+  const int resident = per_sm * sms;
+  return launch_kernel(loss_pair_kernel<NS>, dim3(need < resident ? need : resident), dim3(kPairThreads), 0, st, 1,
+                       true, "loss_pair", D, Ys, reinterpret_cast<const float4*>(partials), nslots, stats, G, loss,
+                       counter, cout, tokens, norm, 1.0f / (float)norm);
+}
+
+lcp_status launch_loss_reduce(const float* stats, float* loss, int tokens, int norm, cudaStream_t st) {
+  return launch_kernel(loss_reduce_kernel, dim3(1), dim3(1024), 0, st, 1, true, "loss_reduce", stats, loss, tokens,
+                       norm);
 }
 
 }  // namespace lcp

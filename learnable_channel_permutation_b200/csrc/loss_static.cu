@@ -126,7 +126,7 @@ extern "C" lcp_status lcp_loss_fwd_static(const float* Yd, const float* Ys, floa
   float* stats = nullptr;
   const lcp_status s = static_scratch(&stats);
   if (s != LCP_OK) return s;
-  const lcp_status s1 = launch_loss_token(Yd, Ys, stats, nullptr, LCP_F32, cout, tokens, stream);
+  const lcp_status s1 = launch_loss_token(Yd, Ys, stats, nullptr, LCP_F32, cout, tokens, tokens, stream);
   if (s1 != LCP_OK) return s1;
-  return launch_loss_reduce(stats, loss, tokens, stream);
+  return launch_loss_reduce(stats, loss, tokens, tokens, stream);
 }
