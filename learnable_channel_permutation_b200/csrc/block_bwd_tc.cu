@@ -482,9 +482,191 @@ lcp_status block_bwd_bc(const CUtensorMap& mW, const CUtensorMap& mD, const CUte
                        dP, cout, cin, rows);
 }
 
+// ------------------------------------------ block backward, B = 256 ---
+// The 256 x 256 dP_b does not fit one SM's tensor memory next to W' and dA,
+// so four CTAs share a block, CTA (qr, qc) owning the dP quadrant of rows
+// (input channels i) [128 qr, 128 qr + 128) and columns (permuted slots j)
+// [128 qc, 128 qc + 128).  Per 128-row chunk o of the CTA's row segment:
+//   W'[:, qc] = W_chunk P_hi[:, qc],  dA[:, qc] = dAt_chunk P_hi[:, qc]
+//                    (M = 128, N = 128, K = 256: all of the block's columns)
+//   A = M.W', dW' = M.dA -> bf16 operand tiles
+//   dP[qr, qc] += dAt_chunk[:, qr]^T A + W_chunk[:, qr]^T dW'   (K = 128 rows)
+// Shared memory: the chunk's W and dAt tiles over the block's 256 columns (four
+// 16 KB column quarters each) and the 128 rows of the transposed P_hi image
+// this CTA's columns need (64 KB): 192 KB.  Once the first two products have
+// read the tiles, the two column quarters of W and of dAt outside the row half
+// qr are free and receive the A and dW' operand tiles, which the dP product
+// reads (MN-major) next to the qr quarters of dAt and W.
+// W' uses P_hi alone here (the forward pass forms W' from P_hi + P_lo, which
+// decides the mask; the mask bits are read from the forward): the two P
+// images would not fit beside the tiles.  TMEM: W' 128 | dA 128 | dP 128.
+constexpr int Q_T_BYTES = 16384;                  // 128 rows x 64 bf16: one column quarter
+constexpr int Q_SMEM = 12 * Q_T_BYTES + 1024 + 128;
+
+__global__ void __launch_bounds__(128)
+block_bwd_q_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmDAt,
+                   const __grid_constant__ CUtensorMap tmPth, const uint32_t* __restrict__ mask,
+                   float* __restrict__ dP, int cout, int cin, int rows_per_split) {
+  constexpr int B = 256;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sW = smem;                       // 4 quarters
+  uint8_t* sDAt = sW + 4 * Q_T_BYTES;       // 4 quarters
+  uint8_t* sPth = sDAt + 4 * Q_T_BYTES;     // 4 K-quarters of the 128 image rows j
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sPth + 4 * Q_T_BYTES);
+  uint32_t* holder = reinterpret_cast<uint32_t*>(bars + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(holder + 1);
+  const uint32_t bar_load = smem_u32(bars + 0), bar_mma1 = smem_u32(bars + 1), bar_mma2 = smem_u32(bars + 2);
+  const uint32_t bar_drain = smem_u32(bars + 3);
+
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const int t = blockIdx.x >> 2, qr = (blockIdx.x >> 1) & 1, qc = blockIdx.x & 1;
+  const int s = blockIdx.y, col0 = t * B;
+  const int rbeg = s * rows_per_split;
+  const int rend = min(cout, rbeg + rows_per_split);
+  const int nchunk = cdiv(rend - rbeg, 128);
+  // the quarters of the row half qr (read by the dP product) and the free ones (operand tiles)
+  uint8_t* wq = sW + 2 * qr * Q_T_BYTES;
+  uint8_t* dq = sDAt + 2 * qr * Q_T_BYTES;
+  uint8_t* sAb = sW + 2 * (1 - qr) * Q_T_BYTES;     // A = M.W'  [o][j], two 64-column regions
+  uint8_t* sdWb = sDAt + 2 * (1 - qr) * Q_T_BYTES;  // dW' = M.dA
+  if (tid == 0) {
+    mbar_init(bar_load, 1);
+    mbar_init(bar_mma1, 1);
+    mbar_init(bar_mma2, 1);
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) tmem_alloc(smem_u32(holder), 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *holder;
+  pdl_wait();
+  pdl_trigger();
+  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  const int row = warp * 32 + lane;
+  const int words = cin / 32;
+  int pending_load = -1;
+  constexpr uint32_t idesc_n = idesc_bf16(128, 128, false, false);
+  constexpr uint32_t idesc_dp = idesc_bf16(128, 128, true, true);
+  const uint32_t tW = tmem, tDA = tmem + 128, tDP = tmem + 256;
+
+  bool ok = true;
+  for (int ch = 0; ch < nchunk && ok; ++ch) {
+    const int r0 = rbeg + ch * 128;
+    if (tid == 0) {
+      // the previous chunk's dP product has read every tile this load overwrites
+      bool go = (ch == 0) || mbar_wait(bar_mma2, (uint32_t)(ch - 1) & 1u, abort_flag, 41);
+      if (go) {
+        pending_load = ch & 1;
+        mbar_expect_tx(bar_load, 8 * Q_T_BYTES + (ch == 0 ? 4 * Q_T_BYTES : 0));
+        for (int kc = 0; kc < 4; ++kc) {
+          tma_load_2d(smem_u32(sW + kc * Q_T_BYTES), &tmW, bar_load, col0 + kc * 64, r0);
+          tma_load_2d(smem_u32(sDAt + kc * Q_T_BYTES), &tmDAt, bar_load, col0 + kc * 64, r0);
+        }
+        if (ch == 0)
+          for (int kc = 0; kc < 4; ++kc)
+            tma_load_2d(smem_u32(sPth + kc * Q_T_BYTES), &tmPth, bar_load, kc * 64, col0 + qc * 128);
+        go = mbar_wait(bar_load, (uint32_t)ch & 1u, abort_flag, 42);
+        if (go) pending_load = -1;
+      }
+      if (!go) *abort_flag = 1;
+      if (go) {
+        tc_fence_after();
+        for (int kc = 0; kc < 4; ++kc)
+#pragma unroll
+          for (int k16 = 0; k16 < 4; ++k16) {
+            const uint64_t pd = sdesc(smem_u32(sPth + kc * Q_T_BYTES) + k16 * 32, 16, 1024);
+            mma_bf16(tW, sdesc(smem_u32(sW + kc * Q_T_BYTES) + k16 * 32, 16, 1024), pd, idesc_n, (kc | k16) != 0);
+            mma_bf16(tDA, sdesc(smem_u32(sDAt + kc * Q_T_BYTES) + k16 * 32, 16, 1024), pd, idesc_n,
+                     (kc | k16) != 0);
+          }
+        mma_commit(bar_mma1);
+      }
+    }
+    ok = __syncthreads_and(mbar_wait(bar_mma1, (uint32_t)ch & 1u, abort_flag, 43));
+    if (!ok) break;
+    tc_fence_after();
+    const int grow = r0 + row;
+    const bool valid = grow < rend;
+#pragma unroll 1
+    for (int cc = 0; cc < 4; ++cc) {
+      uint32_t wv[32], dv[32];
+      tmem_ld32(tW + lane_off + cc * 32, wv);
+      tmem_ld32(tDA + lane_off + cc * 32, dv);
+      tmem_ld_wait();
+      const uint32_t bits = valid ? __ldg(mask + (size_t)grow * words + (col0 + qc * 128) / 32 + cc) : 0u;
+      uint8_t* rA = sAb + (cc / 2) * Q_T_BYTES;
+      uint8_t* rD = sdWb + (cc / 2) * Q_T_BYTES;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float fa[8], fd[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const bool keep = (bits >> (8 * q + e)) & 1u;
+          fa[e] = keep ? __uint_as_float(wv[8 * q + e]) : 0.f;
+          fd[e] = keep ? __uint_as_float(dv[8 * q + e]) : 0.f;
+        }
+        const int chunk16 = (cc & 1) * 4 + q;
+        st_sw128(rA, row, chunk16, make_uint4(pack_bf16x2(fa[0], fa[1]), pack_bf16x2(fa[2], fa[3]),
+                                              pack_bf16x2(fa[4], fa[5]), pack_bf16x2(fa[6], fa[7])));
+        st_sw128(rD, row, chunk16, make_uint4(pack_bf16x2(fd[0], fd[1]), pack_bf16x2(fd[2], fd[3]),
+                                              pack_bf16x2(fd[4], fd[5]), pack_bf16x2(fd[6], fd[7])));
+      }
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      // dP[qr, qc] += dAt[:, qr]^T A + W[:, qr]^T dW', contracted over the chunk's 128 rows
+#pragma unroll
+      for (int k16 = 0; k16 < 8; ++k16)
+        mma_bf16(tDP, sdesc(smem_u32(dq) + k16 * 2048, Q_T_BYTES, 1024),
+                 sdesc(smem_u32(sAb) + k16 * 2048, Q_T_BYTES, 1024), idesc_dp, (ch | k16) != 0);
+#pragma unroll
+      for (int k16 = 0; k16 < 8; ++k16)
+        mma_bf16(tDP, sdesc(smem_u32(wq) + k16 * 2048, Q_T_BYTES, 1024),
+                 sdesc(smem_u32(sdWb) + k16 * 2048, Q_T_BYTES, 1024), idesc_dp, true);
+      mma_commit(bar_mma2);
+    }
+  }
+  if (ok && nchunk > 0) ok = __syncthreads_and(mbar_wait(bar_mma2, (uint32_t)(nchunk - 1) & 1u, abort_flag, 44));
+  const int nb = cin / B;
+  if (ok) {
+    tc_fence_after();
+    // thread `row` holds dP row i = 128 qr + row of the quadrant, columns 128 qc + (0..127)
+    float* o = dP + (size_t)s * nb * B * B + ((size_t)t * B + qr * 128 + row) * B + qc * 128;
+#pragma unroll 1
+    for (int cc = 0; cc < 4; ++cc) {
+      uint32_t r[32];
+      tmem_ld32(tDP + lane_off + cc * 32, r);
+      tmem_ld_wait();
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        reinterpret_cast<float4*>(o + cc * 32)[e] = make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]),
+                                                                __uint_as_float(r[4 * e + 2]),
+                                                                __uint_as_float(r[4 * e + 3]));
+    }
+  }
+  if (tid == 0) {
+    if (pending_load >= 0) mbar_wait_drain(bar_load, (uint32_t)pending_load, 45);
+    mma_commit(bar_drain);
+    mbar_wait_drain(bar_drain, 0, 46);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 int bb_rows_per_split(int cout, int cin, int B) {
   const int BC = B < 64 ? 64 : B;
-  const int tiles = cin / BC;
+  const int tiles = (cin / BC) * (B == 256 ? 4 : 1);   // CTAs of one row segment (B = 256: quadrants)
   const int chunks = cdiv(cout, 128);
   // one CTA per SM: as many row segments per channel tile as fill the SMs once
   int S = 148 / tiles;
@@ -498,7 +680,7 @@ int bb_rows_per_split(int cout, int cin, int B) {
 
 lcp_status tc_error_block_bwd(int* site, int reset) { return read_tc_error(site, reset); }
 
-bool block_bwd_tc_supported(int B) { return B <= 128; }
+bool block_bwd_tc_supported(int B) { return B == 32 || B == 64 || B == 128 || B == 256; }
 
 int block_bwd_tc_splits(int cout, int cin, int B) {
   if (!block_bwd_tc_supported(B)) return 1;
@@ -515,6 +697,13 @@ lcp_status launch_block_bwd_tc(const __nv_bfloat16* W, const __nv_bfloat16* dAt,
   CUtensorMap mW, mD, mPth, mPtl;
   TC_TRY(make_map(&mW, W, cin, cout, 64, 128, "block_bwd W"));
   TC_TRY(make_map(&mD, dAt, cin, cout, 64, 128, "block_bwd dAt"));
+  if (B == 256) {
+    // the 128 transposed-image rows of one quadrant's columns, in 64-column K quarters
+    TC_TRY(make_map(&mPth, img_pt_hi, BC, cin, 64, 128, "block_bwd Pt_hi"));
+    TC_TRY(set_smem(block_bwd_q_kernel, Q_SMEM, "block_bwd_q"));
+    return launch_kernel(block_bwd_q_kernel, dim3((cin / 256) * 4, splits), dim3(128), Q_SMEM, st, 1, true,
+                         "block_bwd_q", mW, mD, mPth, mask, dP_partials, cout, cin, rows);
+  }
   TC_TRY(make_map(&mPth, img_pt_hi, BC, cin, 64, BC, "block_bwd Pt_hi"));
   TC_TRY(make_map(&mPtl, img_pt_lo, BC, cin, 64, BC, "block_bwd Pt_lo"));
   if (B <= 64) {

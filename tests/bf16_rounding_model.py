@@ -16,7 +16,8 @@ stores or feeds a value in that precision:
   them with the exact per-token statistics;
 * dAt = G^T X is stored in bf16;
 * the block backward multiplies bf16 operands: dA = dAt P_hi, dW' = M (.) dA
-  rounded to bf16, A = M (.) W' in bf16, dP_b = dAt_b^T A_b + W_b^T dW'_b;
+  rounded to bf16, A = M (.) W' in bf16, dP_b = dAt_b^T A_b + W_b^T dW'_b
+  (for B = 256 its W' is W P_hi alone: the kernel has no room for P_lo);
 * the Sinkhorn passes are float32 (modelled exactly).
 
 The model returns the mask it took (from its own float32 W'), so the oracle
@@ -74,10 +75,11 @@ def modelled_step(W, X_tokens, L, tau, iters, n, m, g_from_pair=False):
     dAt = bf(G.T @ X)                                         # [C_out, C_in]
     dWp = bf(np.where(mask, block_right(dAt, P_hi), 0.0))
     nb, B, _ = P.shape
+    Ab = bf(np.where(mask, f32(block_right(W, P_hi)), 0.0)) if B == 256 else A
     dP = np.empty_like(P)
     for b in range(nb):
         s = slice(b * B, (b + 1) * B)
-        dP[b] = dAt[:, s].T @ A[:, s] + W[:, s].T @ dWp[:, s]
+        dP[b] = dAt[:, s].T @ Ab[:, s] + W[:, s].T @ dWp[:, s]
     dL = O.sinkhorn_backward(trace, P, dP, tau)
     return dict(loss=loss, dL=dL, mask=mask, P=P)
 

@@ -4,7 +4,7 @@ the dL error against the float64 oracle, and each bound must sit at least a
 factor of two above the modelled layers of its input class.
 
 * zero-mean inputs: the 7B gate projection with 256 tokens (the full-size
-  layers of the other configurations model lower still, 2.3e-3 to 3.5e-3);
+  layers of the other configurations model at 1.5e-3 to 5.3e-3);
 * ReLU-like inputs: the 7B down projection at its full 2048 tokens, the worst
   layer of every configuration.
 
