@@ -48,7 +48,7 @@
 extern "C" {
 #endif
 
-#define LCP_ABI_VERSION 3
+#define LCP_ABI_VERSION 4
 
 #if defined(__GNUC__)
 #define LCP_API __attribute__((visibility("default")))
@@ -134,11 +134,32 @@ LCP_API lcp_status lcp_step(const lcp_layer* layers, int nlayers, const lcp_hpar
 /* As lcp_step, and records events[k] (caller-created cudaEvent_t) on `stream`
  * at the stage boundaries of the FIRST layer: 0 before the Sinkhorn forward,
  * then after each stage (Sinkhorn fwd, permute+mask, calibration GEMM, loss,
- * backward GEMM, block backward, Sinkhorn bwd).  n_events must be 0 or
- * LCP_TIMED_EVENTS.  Used to time each kernel inside a real step. */
+ * backward GEMM, block backward, Sinkhorn bwd).  n_events must be 0,
+ * LCP_TIMED_EVENTS, or LCP_TIMED_EVENTS * nlayers: then layer i records
+ * events[LCP_TIMED_EVENTS * i + k] the same way.  Used to time each kernel
+ * inside a real step. */
 #define LCP_TIMED_EVENTS 8
 LCP_API lcp_status lcp_step_timed(const lcp_layer* layers, int nlayers, const lcp_hparams* hp, void* ws,
                           size_t ws_bytes, cudaStream_t stream, cudaEvent_t* events, int n_events);
+
+/* One token shard of a token-parallel step (the loss is a mean over tokens, so
+ * the calibration batch of T tokens can be split across GPUs: "Implementation
+ * details" trains 7B on 4 GPUs and 13B on 8).  As lcp_step on this call's
+ * layers, whose X hold this shard's layer.tokens tokens, except that
+ *  - the mean over tokens is taken over `total_tokens` (the whole batch):
+ *    layer.loss receives (1/total_tokens) * sum over the shard of (1 - c_t),
+ *    and every gradient is scaled the same way, so the shards' losses and
+ *    gradients add up to the whole batch's;
+ *  - the step stops before the Sinkhorn reverse pass: dP[i] (float32
+ *    [C_in/B, B, B], caller-owned) receives d loss / d P of layer i for the
+ *    shard and ckpt[i] (float32 [C_in/B, iters, 2, B]) the Sinkhorn
+ *    checkpoint of lcp_sinkhorn_fwd; layer.dL is not written.
+ * Summing dP[i] and the losses over the shards (an all-reduce) and calling
+ * lcp_sinkhorn_bwd(L, ckpt, dP_sum, 1, dL, ...) gives the whole batch's dL.
+ * Every layer.tokens <= total_tokens; dP and ckpt 16-byte aligned. */
+LCP_API lcp_status lcp_step_shard(const lcp_layer* layers, int nlayers, const lcp_hparams* hp, int total_tokens,
+                                  float* const* dP, float* const* ckpt, void* ws, size_t ws_bytes,
+                                  cudaStream_t stream);
 
 /* Number of kernel launches lcp_step enqueues for these layers. */
 LCP_API lcp_status lcp_step_launches(const lcp_layer* layers, int nlayers, const lcp_hparams* hp,
@@ -254,6 +275,31 @@ LCP_API lcp_status lcp_loss_bwd(const float* Yd, const float* Ys, const float* s
  * accumulation).  C_out and C_in multiples of 8, T >= 1. */
 LCP_API lcp_status lcp_calib_gemm(const void* X, const void* W, const void* At, float* Yd, float* Ys,
                                   int tokens, int cout, int cin, cudaStream_t stream);
+
+/* The calibration outputs with the cosine-loss reduction in the GEMM's epilogue
+ * ("optimization objective": the loss needs, per token, <y, y~>, |y|^2 and
+ * |y~|^2, and its gradient G a combination of y and y~): y_d = X W^T and
+ * y_s = X At^T come out of one tensor-core pass (float32 accumulation), and
+ * instead of the two float32 outputs the call writes
+ *   partials [T, ceil(C_out / 64), 4] float32: for token t and 64-channel
+ *            slot s, (sum y_d y_s, sum y_d^2, sum y_s^2, 0) over channels
+ *            [64 s, 64 s + 64) (a fixed summation order);
+ *   D = Y_d - Y_s and Ys = Y_s, bf16 [T, C_out] (the difference is formed
+ *            in float32 before rounding).
+ * X [T, C_in], W and At [C_out, C_in] bf16.  C_out and C_in multiples of 8,
+ * T >= 1.  lcp_step uses it for bf16 layers without layer.Yd. */
+LCP_API lcp_status lcp_calib_gemm_loss(const void* X, const void* W, const void* At, void* D, void* Ys,
+                                       float* partials, int tokens, int cout, int cin, cudaStream_t stream);
+
+/* The token-averaged cosine loss and G = d loss / d Ys (bf16 [T, C_out]) from
+ * lcp_calib_gemm_loss's outputs: the slot partials of each token, summed in a
+ * fixed order, give c_t = <y_d,y_s> / max(|y_d||y_s|, 1e-8) and the loss
+ * (1/T) sum_t (1 - c_t); G_t = -(1/T)(y_d / (|y_d||y_s|) - c_t y_s / |y_s|^2)
+ * with y_d = D + Ys and y_s = Ys.  stats [T, 4] receives what lcp_loss_fwd
+ * writes there.  counter: one uint32 of device memory, zero before the call
+ * and left zero by it (not shared by calls that may overlap).  C_out <= 16384. */
+LCP_API lcp_status lcp_loss_pair(const void* D, const void* Ys, const float* partials, float* loss, float* stats,
+                                 void* G, unsigned* counter, int cout, int tokens, cudaStream_t stream);
 
 /* Weight gradient of the sparse output on the tensor cores: dAt = G^T X with
  * G [T, C_out] and X [T, C_in] bf16 and dAt [C_out, C_in] bf16 (float32

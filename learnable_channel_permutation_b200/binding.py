@@ -78,6 +78,8 @@ def lib() -> ctypes.CDLL:
         "lcp_step": ([P(LcpLayer), _c_int, P(LcpHparams), _c_void_p, ctypes.c_size_t, _c_void_p], _c_int),
         "lcp_step_timed": ([P(LcpLayer), _c_int, P(LcpHparams), _c_void_p, ctypes.c_size_t, _c_void_p,
                             P(_c_void_p), _c_int], _c_int),
+        "lcp_step_shard": ([P(LcpLayer), _c_int, P(LcpHparams), _c_int, P(_c_void_p), P(_c_void_p), _c_void_p,
+                            ctypes.c_size_t, _c_void_p], _c_int),
         "lcp_sinkhorn_fwd": ([_c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_float, _c_int, _c_void_p], _c_int),
         "lcp_sinkhorn_bwd": ([_c_void_p, _c_void_p, _c_void_p, _c_int, _c_void_p, _c_int, _c_int, _c_float,
                               _c_int, _c_void_p], _c_int),
@@ -89,6 +91,10 @@ def lib() -> ctypes.CDLL:
         "lcp_calib_gemm": ([_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_int,
                             _c_void_p], _c_int),
         "lcp_grad_gemm": ([_c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_void_p], _c_int),
+        "lcp_calib_gemm_loss": ([_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_int, _c_int,
+                                 _c_int, _c_void_p], _c_int),
+        "lcp_loss_pair": ([_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_int,
+                           _c_int, _c_void_p], _c_int),
         "lcp_device_error": ([P(_c_int), _c_int], _c_int),
         "lcp_harden": ([_c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_void_p], _c_int),
         "lcp_score": ([_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_int, _c_int,
@@ -191,14 +197,29 @@ class Step:
                              _stream(stream)))
 
     def run_timed(self, events: List[torch.cuda.Event], stream: Optional[torch.cuda.Stream] = None) -> None:
-        if len(events) != TIMED_EVENTS:
-            raise ValueError(f"need {TIMED_EVENTS} events")
+        """Stage events of the first layer (TIMED_EVENTS events) or of every
+        layer (TIMED_EVENTS per layer, layer by layer)."""
+        if len(events) not in (TIMED_EVENTS, TIMED_EVENTS * self.n):
+            raise ValueError(f"need {TIMED_EVENTS} or {TIMED_EVENTS} x {self.n} events")
         for e in events:
             if e.cuda_event == 0:
                 raise ValueError("events must be created (record once) before use")
-        arr = (_c_void_p * TIMED_EVENTS)(*[e.cuda_event for e in events])
+        arr = (_c_void_p * len(events))(*[e.cuda_event for e in events])
         check(lib().lcp_step_timed(self.arr, self.n, ctypes.byref(self.hp), self.ws.data_ptr(), self.ws.numel(),
-                                   _stream(stream), arr, TIMED_EVENTS))
+                                   _stream(stream), arr, len(events)))
+
+
+def step_shard(step: "Step", total_tokens: int, dP: Sequence[torch.Tensor], ckpt: Sequence[torch.Tensor],
+               stream: Optional[torch.cuda.Stream] = None) -> None:
+    """lcp_step_shard on a prepared Step whose layers hold one token shard:
+    dP[i] and ckpt[i] receive layer i's shard gradient d loss / d P and its
+    Sinkhorn checkpoint; the losses are normalised by ``total_tokens``."""
+    if len(dP) != step.n or len(ckpt) != step.n:
+        raise ValueError("one dP and one ckpt tensor per layer")
+    dps = (_c_void_p * step.n)(*[_ptr(t, torch.float32, "dP") for t in dP])
+    cks = (_c_void_p * step.n)(*[_ptr(t, torch.float32, "ckpt") for t in ckpt])
+    check(lib().lcp_step_shard(step.arr, step.n, ctypes.byref(step.hp), int(total_tokens), dps, cks,
+                               step.ws.data_ptr(), step.ws.numel(), _stream(stream)))
 
 
 def adamw_params(lr: float = 1e-3, beta1: float = 0.9, beta2: float = 0.999, eps: float = 1e-8,
@@ -354,6 +375,29 @@ def calib_gemm(X: torch.Tensor, W: torch.Tensor, At: Optional[torch.Tensor], Yd:
     check(lib().lcp_calib_gemm(_ptr(X, bf, "X"), _ptr(W, bf, "W"), _ptr(At, bf, "At"),
                                _ptr(Yd, torch.float32, "Yd"), _ptr(Ys, torch.float32, "Ys"), T, cout, cin,
                                _stream(None)))
+
+
+def calib_gemm_loss(X: torch.Tensor, W: torch.Tensor, At: torch.Tensor, D: torch.Tensor, Ys: torch.Tensor,
+                    partials: torch.Tensor) -> None:
+    """lcp_calib_gemm_loss: D = Y_d - Y_s and Y_s (bf16 [T, C_out]) and the
+    per-token slot partials (float32 [T, ceil(C_out/64), 4])."""
+    T, cin = X.shape
+    cout = W.shape[0]
+    bf = torch.bfloat16
+    check(lib().lcp_calib_gemm_loss(_ptr(X, bf, "X"), _ptr(W, bf, "W"), _ptr(At, bf, "At"), _ptr(D, bf, "D"),
+                                    _ptr(Ys, bf, "Ys"), _ptr(partials, torch.float32, "partials"), T, cout, cin,
+                                    _stream(None)))
+
+
+def loss_pair(D: torch.Tensor, Ys: torch.Tensor, partials: torch.Tensor, loss: torch.Tensor, stats: torch.Tensor,
+              G: torch.Tensor, counter: torch.Tensor) -> None:
+    """lcp_loss_pair: the loss and G (bf16) from lcp_calib_gemm_loss's outputs;
+    ``counter`` is one int32 of device memory, zero before the call."""
+    T, cout = D.shape
+    bf = torch.bfloat16
+    check(lib().lcp_loss_pair(_ptr(D, bf, "D"), _ptr(Ys, bf, "Ys"), _ptr(partials, torch.float32, "partials"),
+                              _ptr(loss, torch.float32, "loss"), _ptr(stats, torch.float32, "stats"), _ptr(G, bf, "G"),
+                              _ptr(counter, torch.int32, "counter"), cout, T, _stream(None)))
 
 
 def grad_gemm(G: torch.Tensor, X: torch.Tensor, dAt: torch.Tensor) -> None:

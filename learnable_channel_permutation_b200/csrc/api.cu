@@ -13,6 +13,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "lcp_internal.cuh"
 
@@ -169,50 +170,80 @@ lcp_status check_layer(const lcp_layer& l, const lcp_hparams& hp, int idx) {
 
 size_t esize(lcp_dtype d) { return d == LCP_F32 ? 4 : 2; }
 
+// Workspace layout.  Each layer has a persistent region that lives for the
+// whole call (its Sinkhorn checkpoint, the bf16 operand images of P, its dP
+// partials and the loss counter: the Sinkhorn kernels run once over every
+// layer, before and after the other stages), laid out layer after layer; one
+// shared region after them holds everything else and is reused layer by layer.
 struct Plan {
-  size_t ckpt, img0, img1, img2, mask, wp, amask, at, yd, ys, stats, counter, g, dat, da, dp, perm, phard, shat;
-  size_t total;
+  size_t ckpt, img0, img1, img2, counter, dp;                                          // persistent
+  size_t mask, wp, amask, at, yd, ys, stats, g, dat, da, perm, phard, shat;            // shared
+  size_t persist, shared;   // bytes of this layer's persistent and shared parts
   int splits;
 };
 
-Plan make_plan(const lcp_layer& l, const lcp_hparams& hp) {
+Plan make_plan(const lcp_layer& l, const lcp_hparams& hp, size_t pbase, size_t sbase) {
   const bool tc = use_tc(hp);
   const size_t B = hp.block, nb = l.cin / hp.block;
   const size_t oc = l.cout, ic = l.cin, T = l.tokens;
   const size_t es = esize(hp.dtype);
   Plan p{};
-  size_t off = 0;
+  size_t po = pbase, so = sbase;
+  auto takep = [&](size_t bytes) {
+    const size_t at = po;
+    po += (bytes + 1023) & ~(size_t)1023;
+    return at;
+  };
   auto take = [&](size_t bytes) {
-    const size_t at = off;
-    off += (bytes + 1023) & ~(size_t)1023;
+    const size_t at = so;
+    so += (bytes + 1023) & ~(size_t)1023;
     return at;
   };
   p.splits = tc ? block_bwd_tc_splits(l.cout, l.cin, hp.block) : 1;
-  p.ckpt = take(nb * hp.iters * 2 * B * 4);
+  p.ckpt = takep(nb * hp.iters * 2 * B * 4);
   const size_t BC = B < 64 ? 64 : B;   // tile width of the operand images
-  p.img0 = take(tc ? ic * BC * 2 : 0);
-  p.img1 = take(tc ? ic * BC * 2 : 0);
-  p.img2 = take(tc ? ic * BC * 2 : 0);
+  p.img0 = takep(tc ? ic * BC * 2 : 0);
+  p.img1 = takep(tc ? ic * BC * 2 : 0);
+  p.img2 = takep(tc ? ic * BC * 2 : 0);
+  p.counter = takep(256);
+  p.dp = takep((size_t)p.splits * nb * B * B * 4);
   p.mask = take(oc * ic / 8);
-  // the CUDA-core block backward (f32, LCP_FLAG_SIMT, or B = 256) works on float32 W', A, dA
-  const bool simt_bwd = !tc || !block_bwd_tc_supported(hp.block);
+  // the CUDA-core block backward (f32 or LCP_FLAG_SIMT) works on float32 W', A, dA
+  const bool simt_bwd = !tc;
   p.wp = take(simt_bwd ? oc * ic * 4 : 0);
   p.amask = take(simt_bwd ? oc * ic * 4 : 0);
   p.at = take(oc * ic * es);
   p.yd = take(l.Yd ? 0 : T * oc * 4);   // the caller's Yd replaces the workspace copy
   p.ys = take(T * oc * 4);
   p.stats = take(T * 16);
-  p.counter = take(256);
   p.g = take(T * oc * es);
   p.dat = take(oc * ic * (tc ? 2 : 4));
   p.da = take(simt_bwd ? oc * ic * 4 : 0);
-  p.dp = take((size_t)p.splits * nb * B * B * 4);
   const bool hard = (hp.flags & LCP_FLAG_HARD) != 0;
   p.perm = take(hard && !l.perm ? nb * B * 4 : 0);
   p.phard = take(hard && simt_bwd ? nb * B * B * 4 : 0);   // the CUDA-core products read P_hard as float32
   p.shat = take((hp.flags & LCP_FLAG_SCORE) && !tc ? oc * ic * 4 : 0);   // S_hat of the CUDA-core path
-  p.total = off;
+  p.persist = po - pbase;
+  p.shared = so - sbase;
   return p;
+}
+
+// Every layer's plan; *total receives the workspace bytes the call needs.
+std::vector<Plan> layout(const lcp_layer* layers, int nlayers, const lcp_hparams& hp, size_t* total) {
+  std::vector<Plan> plans((size_t)nlayers);
+  size_t persist = 0, shared = 0;
+  for (int i = 0; i < nlayers; ++i) {
+    const Plan q = make_plan(layers[i], hp, 0, 0);
+    persist += q.persist;
+    shared = std::max(shared, q.shared);
+  }
+  size_t pb = 0;
+  for (int i = 0; i < nlayers; ++i) {
+    plans[i] = make_plan(layers[i], hp, pb, persist);
+    pb += plans[i].persist;
+  }
+  *total = persist + shared;
+  return plans;
 }
 
 lcp_status validate_all(const lcp_layer* layers, int nlayers, const lcp_hparams* hp) {
@@ -230,12 +261,20 @@ template <typename T> T* at(void* ws, size_t off) {
 // Loss stage of a step: the fused one-launch kernel when a token row fits its
 // registers, else per-token statistics + gradient and a separate reduction.
 lcp_status launch_loss(const float* Yd, const float* Ys, float* stats, void* G, lcp_dtype gdt, float* loss,
-                       unsigned* counter, int cout, int tokens, cudaStream_t st) {
-  if (loss_fused_supported(cout)) return launch_loss_fused(Yd, Ys, stats, G, gdt, loss, counter, cout, tokens, st);
-  LCP_TRY(launch_loss_token(Yd, Ys, stats, G, gdt, cout, tokens, st));
-  return launch_loss_reduce(stats, loss, tokens, st);
+                       unsigned* counter, int cout, int tokens, int norm, cudaStream_t st) {
+  if (loss_fused_supported(cout))
+    return launch_loss_fused(Yd, Ys, stats, G, gdt, loss, counter, cout, tokens, norm, st);
+  LCP_TRY(launch_loss_token(Yd, Ys, stats, G, gdt, cout, tokens, norm, st));
+  return launch_loss_reduce(stats, loss, tokens, norm, st);
 }
 int loss_launches(int cout) { return loss_fused_supported(cout) ? 1 : 2; }
+
+// The tensor-core step takes the loss from the calibration GEMM's epilogue
+// unless the caller wants the float32 dense output (layer.Yd, as input or
+// output) or C_out is wider than the pair kernel takes.
+bool fused_loss(const lcp_layer& l, const lcp_hparams& hp) {
+  return use_tc(hp) && !l.Yd && !(hp.flags & LCP_FLAG_CACHED_DENSE) && loss_pair_supported(l.cout);
+}
 
 // Stage events.  Under stream capture they become event-record nodes of the
 // graph (external records), so a replayed graph still times every stage.
@@ -251,11 +290,21 @@ lcp_status record(cudaEvent_t* ev, int k, cudaStream_t st) {
 }
 
 // ---- one layer, CUDA-core path (float32, or bf16 with LCP_FLAG_SIMT) -------
+// Options of a layer's step beyond lcp_step's: the token count the loss mean is
+// taken over (norm), and, for one shard of a token-parallel step, caller-owned
+// buffers for the Sinkhorn checkpoint and for dP, in which case the step stops
+// before the Sinkhorn reverse pass.
+struct LayerOpts {
+  int norm;
+  float* ckpt;
+  float* dP;
+};
+
 lcp_status layer_simt(const lcp_layer& l, const lcp_hparams& hp, const Plan& p, void* ws,
-                      cudaStream_t st, cudaEvent_t* ev) {
+                      cudaStream_t st, cudaEvent_t* ev, const LayerOpts& o) {
   const int B = hp.block, nb = l.cin / B;
   const lcp_dtype dt = hp.dtype;
-  float* ckpt = at<float>(ws, p.ckpt);
+  float* ckpt = o.ckpt ? o.ckpt : at<float>(ws, p.ckpt);
   uint32_t* mask = l.mask ? l.mask : at<uint32_t>(ws, p.mask);
   const bool score = (hp.flags & LCP_FLAG_SCORE) != 0, write_wp = (hp.flags & LCP_FLAG_WRITE_WPRIME) != 0;
   // W' (float32); with scores the ranked S_hat goes to layer.Wp when requested
@@ -270,7 +319,7 @@ lcp_status layer_simt(const lcp_layer& l, const lcp_hparams& hp, const Plan& p, 
   void* G = at<void>(ws, p.g);
   float* dAt = at<float>(ws, p.dat);
   float* dA = at<float>(ws, p.da);
-  float* dP = at<float>(ws, p.dp);
+  float* dP = o.dP ? o.dP : at<float>(ws, p.dp);
   const long long ic = l.cin, oc = l.cout, BB = (long long)B * B;
 
   LCP_TRY(record(ev, 0, st));
@@ -306,7 +355,7 @@ lcp_status layer_simt(const lcp_layer& l, const lcp_hparams& hp, const Plan& p, 
   LCP_TRY(launch_simt_gemm({l.tokens, l.cout, l.cin, 1, l.X, 0, ic, 1, At, 0, 1, ic, Ys, 0, oc, 1, 1.f, 0.f},
                            dt, dt, LCP_F32, st));
   LCP_TRY(record(ev, 3, st));
-  LCP_TRY(launch_loss(Yd, Ys, stats, G, dt, l.loss, at<unsigned>(ws, p.counter), l.cout, l.tokens, st));
+  LCP_TRY(launch_loss(Yd, Ys, stats, G, dt, l.loss, at<unsigned>(ws, p.counter), l.cout, l.tokens, o.norm, st));
   LCP_TRY(record(ev, 4, st));
   // dAt = G^T X   ([C_out, C_in], K = T)
   LCP_TRY(launch_simt_gemm({l.cout, l.cin, l.tokens, 1, G, 0, 1, oc, l.X, 0, ic, 1, dAt, 0, ic, 1, 1.f, 0.f},
@@ -321,7 +370,7 @@ lcp_status layer_simt(const lcp_layer& l, const lcp_hparams& hp, const Plan& p, 
   LCP_TRY(launch_simt_gemm({B, B, l.cout, nb, l.W, B, 1, ic, dA, B, ic, 1, dP, BB, B, 1, 1.f, 1.f},
                            dt, LCP_F32, LCP_F32, st));
   LCP_TRY(record(ev, 6, st));
-  LCP_TRY(launch_sinkhorn_bwd(l.L, ckpt, dP, 1, l.dL, nb, B, hp.tau, hp.iters, st));
+  if (!o.dP) LCP_TRY(launch_sinkhorn_bwd(l.L, ckpt, dP, 1, l.dL, nb, B, hp.tau, hp.iters, st));
   LCP_TRY(record(ev, 7, st));
   return LCP_OK;
 }
@@ -329,20 +378,25 @@ lcp_status layer_simt(const lcp_layer& l, const lcp_hparams& hp, const Plan& p, 
 // kernel launches per layer, not counting the loss stage (1 or 2 launches)
 constexpr int kSimtLaunches = 13;
 constexpr int kTcLaunches = 6;
-constexpr int kTcLaunchesSimtBwd = 11;   // B = 256: block backward on CUDA cores (6 launches)
 
 int launches_per_layer(const lcp_layer& l, const lcp_hparams& hp) {
-  const int loss = loss_launches(l.cout) + ((hp.flags & LCP_FLAG_HARD) ? 1 : 0) +
+  const int loss = (fused_loss(l, hp) ? 1 : loss_launches(l.cout)) + ((hp.flags & LCP_FLAG_HARD) ? 1 : 0) +
                    ((hp.flags & LCP_FLAG_SCORE) ? 1 : 0);   // hardening; the score GEMM or score-mask pass
   if (!use_tc(hp)) return kSimtLaunches - ((hp.flags & LCP_FLAG_CACHED_DENSE) ? 1 : 0) + loss;
-  return (block_bwd_tc_supported(hp.block) ? kTcLaunches : kTcLaunchesSimtBwd) + loss;
+  return kTcLaunches - 2 + loss;   // the two Sinkhorn launches are shared by all layers
 }
 
-// ---- one layer, tensor-core path (bf16 operands, float32 accumulation) -----
-lcp_status layer_tc(const lcp_layer& l, const lcp_hparams& hp, const Plan& p, void* ws,
-                    cudaStream_t st, cudaEvent_t* ev) {
+// ---- the tensor-core path (bf16 operands, float32 accumulation) -----------
+// The Sinkhorn forward pass runs once over every layer's blocks, then each
+// layer's middle stages run in turn, then the Sinkhorn reverse pass runs once
+// over every layer (with stage events, layer 0's Sinkhorn forward stage holds
+// the batched launch and the last layer's Sinkhorn reverse stage the other).
+
+// the middle of one layer: hardening, permute + mask, calibration products +
+// loss, gradient product, block backward (and, for a token shard, its dP out)
+lcp_status layer_tc_middle(const lcp_layer& l, const lcp_hparams& hp, const Plan& p, void* ws,
+                           cudaStream_t st, cudaEvent_t* ev, bool first, const LayerOpts& o) {
   const int B = hp.block, nb = l.cin / B;
-  float* ckpt = at<float>(ws, p.ckpt);
   auto* pt_hi = at<__nv_bfloat16>(ws, p.img0);
   auto* pt_lo = at<__nv_bfloat16>(ws, p.img1);
   auto* p_hi = at<__nv_bfloat16>(ws, p.img2);
@@ -359,19 +413,11 @@ lcp_status layer_tc(const lcp_layer& l, const lcp_hparams& hp, const Plan& p, vo
   const auto* W = static_cast<const __nv_bfloat16*>(l.W);
   const auto* X = static_cast<const __nv_bfloat16*>(l.X);
 
-  LCP_TRY(record(ev, 0, st));
-  LCP_TRY(launch_sinkhorn_fwd(l.L, l.P, ckpt, pt_hi, pt_lo, p_hi, at<unsigned>(ws, p.counter), nb, B, hp.tau,
-                              hp.iters, st));
-  // with hardening the operand images (and, for the CUDA-core block backward,
-  // the float32 matrix) are those of the hard permutation; the Sinkhorn reverse
-  // pass still runs on the soft P_hat (straight-through)
-  const float* Pu = l.P;
-  if (hp.flags & LCP_FLAG_HARD) {
-    float* Ph = p.phard ? at<float>(ws, p.phard) : nullptr;
-    if (!block_bwd_tc_supported(B)) Pu = Ph;
-    LCP_TRY(launch_harden(l.P, l.perm ? l.perm : at<int>(ws, p.perm), block_bwd_tc_supported(B) ? nullptr : Ph,
-                          pt_hi, pt_lo, p_hi, nb, B, st));
-  }
+  if (!first) LCP_TRY(record(ev, 0, st));
+  // with hardening the operand images are those of the hard permutation; the
+  // Sinkhorn reverse pass still runs on the soft P_hat (straight-through)
+  if (hp.flags & LCP_FLAG_HARD)
+    LCP_TRY(launch_harden(l.P, l.perm ? l.perm : at<int>(ws, p.perm), nullptr, pt_hi, pt_lo, p_hi, nb, B, st));
   LCP_TRY(record(ev, 1, st));
   if (hp.flags & LCP_FLAG_SCORE) {
     // mask from S_hat = S P_B (exported to layer.Wp when requested), then A and At from W'
@@ -383,62 +429,106 @@ lcp_status layer_tc(const lcp_layer& l, const lcp_hparams& hp, const Plan& p, vo
     LCP_TRY(launch_permute_mask_tc(W, pt_hi, pt_lo, p_hi, mask, At, Wp, l.cout, l.cin, B, hp.n, hp.m, false, st));
   }
   LCP_TRY(record(ev, 2, st));
-  if (cached)   // Y_s = X At^T alone (one problem)
-    LCP_TRY(launch_calib_gemm_tc(X, At, nullptr, Ys, nullptr, l.tokens, l.cout, l.cin, st));
-  else
-    LCP_TRY(launch_calib_gemm_tc(X, W, At, Yd, Ys, l.tokens, l.cout, l.cin, st));
-  LCP_TRY(record(ev, 3, st));
-  LCP_TRY(launch_loss(Yd, Ys, stats, G, LCP_BF16, l.loss, at<unsigned>(ws, p.counter), l.cout, l.tokens, st));
+  if (fused_loss(l, hp)) {
+    // the loss reduction in the calibration GEMM's epilogue: it leaves D = Y_d - Y_s
+    // and Y_s in bf16 (in the Y_d slot) and per-token slot partials (in the Y_s slot)
+    auto* Dq = at<__nv_bfloat16>(ws, p.yd);
+    auto* Ysq = Dq + (size_t)l.tokens * l.cout;
+    float* part = at<float>(ws, p.ys);
+    LCP_TRY(launch_calib_loss_tc(X, W, At, Dq, Ysq, part, l.tokens, l.cout, l.cin, st));
+    LCP_TRY(record(ev, 3, st));
+    LCP_TRY(launch_loss_pair(Dq, Ysq, part, calib_loss_slots(l.cout), stats, G, l.loss, at<unsigned>(ws, p.counter),
+                             l.cout, l.tokens, o.norm, st));
+  } else {
+    if (cached)   // Y_s = X At^T alone (one problem)
+      LCP_TRY(launch_calib_gemm_tc(X, At, nullptr, Ys, nullptr, l.tokens, l.cout, l.cin, st));
+    else
+      LCP_TRY(launch_calib_gemm_tc(X, W, At, Yd, Ys, l.tokens, l.cout, l.cin, st));
+    LCP_TRY(record(ev, 3, st));
+    LCP_TRY(launch_loss(Yd, Ys, stats, G, LCP_BF16, l.loss, at<unsigned>(ws, p.counter), l.cout, l.tokens, o.norm,
+                        st));
+  }
   LCP_TRY(record(ev, 4, st));
   LCP_TRY(launch_bwd_gemm_tc(G, X, dAt, l.tokens, l.cout, l.cin, st));
   LCP_TRY(record(ev, 5, st));
-  if (block_bwd_tc_supported(B)) {
-    LCP_TRY(launch_block_bwd_tc(W, dAt, mask, pt_hi, pt_lo, dP, p.splits, l.cout, l.cin, B, st));
-  } else {
-    // B = 256: the fused kernel does not fit one SM's tensor memory; use the
-    // CUDA-core products on float32 W', A = M.W' and dA.
-    const long long ic = l.cin, BB = (long long)B * B;
-    float* Wp32 = at<float>(ws, p.wp);
-    float* Am = at<float>(ws, p.amask);
-    float* dA = at<float>(ws, p.da);
-    LCP_TRY(launch_simt_gemm({l.cout, B, B, nb, W, B, ic, 1, Pu, BB, B, 1, Wp32, B, ic, 1, 1.f, 0.f},
-                             LCP_BF16, LCP_F32, LCP_F32, st));
-    LCP_TRY(launch_apply_mask(Wp32, mask, Am, l.cout, l.cin, st));
-    LCP_TRY(launch_simt_gemm({l.cout, B, B, nb, dAt, B, ic, 1, Pu, BB, B, 1, dA, B, ic, 1, 1.f, 0.f},
-                             LCP_BF16, LCP_F32, LCP_F32, st));
-    LCP_TRY(launch_apply_mask(dA, mask, dA, l.cout, l.cin, st));
-    LCP_TRY(launch_simt_gemm({B, B, l.cout, nb, dAt, B, 1, ic, Am, B, ic, 1, dP, BB, B, 1, 1.f, 0.f},
-                             LCP_BF16, LCP_F32, LCP_F32, st));
-    LCP_TRY(launch_simt_gemm({B, B, l.cout, nb, W, B, 1, ic, dA, B, ic, 1, dP, BB, B, 1, 1.f, 1.f},
-                             LCP_BF16, LCP_F32, LCP_F32, st));
-  }
+  LCP_TRY(launch_block_bwd_tc(W, dAt, mask, pt_hi, pt_lo, dP, p.splits, l.cout, l.cin, B, st));
   LCP_TRY(record(ev, 6, st));
-  LCP_TRY(launch_sinkhorn_bwd(l.L, ckpt, dP, p.splits, l.dL, nb, B, hp.tau, hp.iters, st));
-  LCP_TRY(record(ev, 7, st));
+  if (o.dP) LCP_TRY(launch_sum_splits(dP, p.splits, (size_t)nb * B * B, o.dP, st));
   return LCP_OK;
 }
 
+lcp_status step_tc(const lcp_layer* layers, int n, const lcp_hparams& hp, const std::vector<Plan>& plans,
+                   void* ws, cudaStream_t st, cudaEvent_t* (*evl)(void*, int), void* evctx,
+                   const std::vector<LayerOpts>& opts) {
+  const int B = hp.block;
+  const bool shard = opts[0].dP != nullptr;
+  std::vector<SkFwdLayer> fl((size_t)n);
+  for (int i = 0; i < n; ++i) {
+    const lcp_layer& l = layers[i];
+    const Plan& p = plans[i];
+    fl[i] = SkFwdLayer{l.L, l.P, opts[i].ckpt ? opts[i].ckpt : at<float>(ws, p.ckpt), at<__nv_bfloat16>(ws, p.img0),
+                       at<__nv_bfloat16>(ws, p.img1), at<__nv_bfloat16>(ws, p.img2), at<unsigned>(ws, p.counter),
+                       l.cin / B};
+  }
+  LCP_TRY(record(evl(evctx, 0), 0, st));
+  LCP_TRY(launch_sinkhorn_fwd_batch(fl.data(), n, B, hp.tau, hp.iters, st));
+  for (int i = 0; i < n; ++i) {
+    cudaEvent_t* e = evl(evctx, i);
+    LCP_TRY(layer_tc_middle(layers[i], hp, plans[i], ws, st, e, i == 0, opts[i]));
+    if (i + 1 < n || shard) LCP_TRY(record(e, 7, st));
+  }
+  if (shard) return LCP_OK;
+  std::vector<SkBwdLayer> bl((size_t)n);
+  for (int i = 0; i < n; ++i) {
+    const lcp_layer& l = layers[i];
+    const Plan& p = plans[i];
+    bl[i] = SkBwdLayer{l.L, fl[i].ckpt, at<float>(ws, p.dp), l.dL, p.splits, l.cin / B};
+  }
+  LCP_TRY(launch_sinkhorn_bwd_batch(bl.data(), n, B, hp.tau, hp.iters, st));
+  return record(evl(evctx, n - 1), 7, st);
+}
+
+// total_tokens > 0, dP and ckpt: one token shard of a token-parallel step (see lcp_step_shard)
 lcp_status step_impl(const lcp_layer* layers, int nlayers, const lcp_hparams* hp, void* ws,
-                     size_t ws_bytes, cudaStream_t st, cudaEvent_t* ev, int nev) {
+                     size_t ws_bytes, cudaStream_t st, cudaEvent_t* ev, int nev, int total_tokens = 0,
+                     float* const* dP = nullptr, float* const* ckpt = nullptr) {
   LCP_TRY(validate_all(layers, nlayers, hp));
-  if (nev != 0 && nev != LCP_TIMED_EVENTS)
-    return fail(LCP_ERR_ARG, "n_events must be 0 or %d", LCP_TIMED_EVENTS);
+  if (total_tokens > 0) {
+    if (!dP || !ckpt) return fail(LCP_ERR_NULL, "dP and ckpt are required");
+    for (int i = 0; i < nlayers; ++i) {
+      if (layers[i].tokens > total_tokens)
+        return fail(LCP_ERR_SHAPE, "layer %d: its %d tokens exceed total_tokens = %d", i, layers[i].tokens,
+                    total_tokens);
+      if (!dP[i] || !ckpt[i]) return fail(LCP_ERR_NULL, "layer %d: dP and ckpt are required", i);
+      if (!aligned16(dP[i]) || !aligned16(ckpt[i]))
+        return fail(LCP_ERR_ARG, "layer %d: dP and ckpt must be 16-byte aligned", i);
+    }
+  }
+  if (nev != 0 && nev != LCP_TIMED_EVENTS && !(nlayers > 0 && nev == LCP_TIMED_EVENTS * nlayers))
+    return fail(LCP_ERR_ARG, "n_events must be 0, %d or %d x nlayers", LCP_TIMED_EVENTS, LCP_TIMED_EVENTS);
   if (nev && !ev) return fail(LCP_ERR_NULL, "events is NULL");
   if (nlayers == 0) return LCP_OK;
   size_t need = 0;
-  for (int i = 0; i < nlayers; ++i) need = std::max(need, make_plan(layers[i], *hp).total);
+  const std::vector<Plan> plans = layout(layers, nlayers, *hp, &need);
   if (!ws) return fail(LCP_ERR_NULL, "workspace is NULL");
   if (((uintptr_t)ws & 255u) != 0) return fail(LCP_ERR_WORKSPACE, "workspace must be 256-byte aligned");
   if (ws_bytes < need)
     return fail(LCP_ERR_WORKSPACE, "workspace has %zu bytes, %zu needed", ws_bytes, need);
   LCP_TRY(check_arch());
   LCP_TRY(check_pending());
-  for (int i = 0; i < nlayers; ++i) {
-    const Plan p = make_plan(layers[i], *hp);
-    cudaEvent_t* e = (i == 0 && nev) ? ev : nullptr;
-    if (use_tc(*hp)) LCP_TRY(layer_tc(layers[i], *hp, p, ws, st, e));
-    else LCP_TRY(layer_simt(layers[i], *hp, p, ws, st, e));
-  }
+  struct EvCtx { cudaEvent_t* ev; int nev, nlayers; } ectx{ev, nev, nlayers};
+  auto evl = [](void* c, int i) -> cudaEvent_t* {
+    const EvCtx& x = *static_cast<const EvCtx*>(c);
+    if (!x.nev) return nullptr;
+    if (x.nev == LCP_TIMED_EVENTS * x.nlayers) return x.ev + (size_t)LCP_TIMED_EVENTS * i;
+    return i == 0 ? x.ev : nullptr;
+  };
+  std::vector<LayerOpts> opts((size_t)nlayers);
+  for (int i = 0; i < nlayers; ++i)
+    opts[i] = LayerOpts{total_tokens > 0 ? total_tokens : layers[i].tokens, total_tokens > 0 ? ckpt[i] : nullptr,
+                        total_tokens > 0 ? dP[i] : nullptr};
+  if (use_tc(*hp)) return step_tc(layers, nlayers, *hp, plans, ws, st, evl, &ectx, opts);
+  for (int i = 0; i < nlayers; ++i) LCP_TRY(layer_simt(layers[i], *hp, plans[i], ws, st, evl(&ectx, i), opts[i]));
   return LCP_OK;
 }
 
@@ -472,7 +562,7 @@ lcp_status lcp_workspace_size(const lcp_layer* layers, int nlayers, const lcp_hp
   if (!bytes) return fail(LCP_ERR_NULL, "bytes is NULL");
   LCP_TRY(validate_all(layers, nlayers, hp));
   size_t need = 0;
-  for (int i = 0; i < nlayers; ++i) need = std::max(need, make_plan(layers[i], *hp).total);
+  layout(layers, nlayers, *hp, &need);
   *bytes = need;
   return LCP_OK;
 }
@@ -483,6 +573,7 @@ lcp_status lcp_step_launches(const lcp_layer* layers, int nlayers, const lcp_hpa
   LCP_TRY(validate_all(layers, nlayers, hp));
   int n = 0;
   for (int i = 0; i < nlayers; ++i) n += launches_per_layer(layers[i], *hp);
+  if (use_tc(*hp) && nlayers > 0) n += 2 * ((nlayers + kSkMaxLayers - 1) / kSkMaxLayers);   // batched Sinkhorn
   *launches = n;
   return LCP_OK;
 }
@@ -496,6 +587,12 @@ lcp_status lcp_step_timed(const lcp_layer* layers, int nlayers, const lcp_hparam
                           size_t ws_bytes, cudaStream_t stream, cudaEvent_t* events,
                           int n_events) {
   return step_impl(layers, nlayers, hp, ws, ws_bytes, stream, events, n_events);
+}
+
+lcp_status lcp_step_shard(const lcp_layer* layers, int nlayers, const lcp_hparams* hp, int total_tokens,
+                          float* const* dP, float* const* ckpt, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (total_tokens < 1 || total_tokens > kMaxDim) return fail(LCP_ERR_SHAPE, "total_tokens = %d", total_tokens);
+  return step_impl(layers, nlayers, hp, ws, ws_bytes, stream, nullptr, 0, total_tokens, dP, ckpt);
 }
 
 lcp_status lcp_adamw(float* L, const float* dL, float* m, float* v, long long n, const lcp_adamw_params* opt,
@@ -703,6 +800,38 @@ lcp_status lcp_calib_gemm(const void* X, const void* W, const void* At, float* Y
                               static_cast<const __nv_bfloat16*>(At), Yd, Ys, tokens, cout, cin, stream);
 }
 
+lcp_status lcp_calib_gemm_loss(const void* X, const void* W, const void* At, void* D, void* Ys, float* partials,
+                               int tokens, int cout, int cin, cudaStream_t stream) {
+  if (!X || !W || !At || !D || !Ys || !partials) return fail(LCP_ERR_NULL, "X, W, At, D, Ys and partials are required");
+  if (cout < 8 || cout % 8 || cout > kMaxDim) return fail(LCP_ERR_SHAPE, "C_out = %d must be a positive multiple of 8", cout);
+  if (cin < 8 || cin % 8 || cin > kMaxDim) return fail(LCP_ERR_SHAPE, "C_in = %d must be a positive multiple of 8", cin);
+  if (tokens < 1 || tokens > kMaxDim) return fail(LCP_ERR_SHAPE, "T = %d must be >= 1", tokens);
+  const void* ptrs[] = {X, W, At, D, Ys, partials};
+  for (const void* q : ptrs)
+    if (!aligned16(q)) return fail(LCP_ERR_ARG, "pointers must be 16-byte aligned");
+  LCP_TRY(check_arch());
+  LCP_TRY(check_pending());
+  return launch_calib_loss_tc(static_cast<const __nv_bfloat16*>(X), static_cast<const __nv_bfloat16*>(W),
+                              static_cast<const __nv_bfloat16*>(At), static_cast<__nv_bfloat16*>(D),
+                              static_cast<__nv_bfloat16*>(Ys), partials, tokens, cout, cin, stream);
+}
+
+lcp_status lcp_loss_pair(const void* D, const void* Ys, const float* partials, float* loss, float* stats, void* G,
+                         unsigned* counter, int cout, int tokens, cudaStream_t stream) {
+  if (!D || !Ys || !partials || !loss || !stats || !G || !counter)
+    return fail(LCP_ERR_NULL, "D, Ys, partials, loss, stats, G and counter are required");
+  if (cout < 8 || cout % 8 || !loss_pair_supported(cout))
+    return fail(LCP_ERR_SHAPE, "C_out = %d must be a positive multiple of 8, at most 16384", cout);
+  if (tokens < 1 || tokens > kMaxDim) return fail(LCP_ERR_SHAPE, "T = %d must be >= 1", tokens);
+  if (!aligned16(D) || !aligned16(Ys) || !aligned16(partials) || !aligned16(stats) || !aligned16(G))
+    return fail(LCP_ERR_ARG, "D, Ys, partials, stats and G must be 16-byte aligned");
+  LCP_TRY(check_arch());
+  LCP_TRY(check_pending());
+  return launch_loss_pair(static_cast<const __nv_bfloat16*>(D), static_cast<const __nv_bfloat16*>(Ys), partials,
+                          calib_loss_slots(cout), stats, static_cast<__nv_bfloat16*>(G), loss, counter, cout, tokens,
+                          tokens, stream);
+}
+
 lcp_status lcp_grad_gemm(const void* G, const void* X, void* dAt, int tokens, int cout, int cin,
                          cudaStream_t stream) {
   if (!G || !X || !dAt) return fail(LCP_ERR_NULL, "G, X and dAt are required");
@@ -724,8 +853,8 @@ lcp_status lcp_loss_fwd(const float* Yd, const float* Ys, float* loss, float* st
   if (!aligned16(Yd) || !aligned16(Ys) || !aligned16(stats)) return fail(LCP_ERR_ARG, "pointers must be 16-byte aligned");
   LCP_TRY(check_arch());
   LCP_TRY(check_pending());
-  LCP_TRY(launch_loss_token(Yd, Ys, stats, nullptr, LCP_F32, cout, tokens, stream));
-  return launch_loss_reduce(stats, loss, tokens, stream);
+  LCP_TRY(launch_loss_token(Yd, Ys, stats, nullptr, LCP_F32, cout, tokens, tokens, stream));
+  return launch_loss_reduce(stats, loss, tokens, tokens, stream);
 }
 
 lcp_status lcp_loss_bwd(const float* Yd, const float* Ys, const float* stats, void* G, int cout,
@@ -738,7 +867,7 @@ lcp_status lcp_loss_bwd(const float* Yd, const float* Ys, const float* stats, vo
     return fail(LCP_ERR_ARG, "pointers must be 16-byte aligned");
   LCP_TRY(check_arch());
   LCP_TRY(check_pending());
-  return launch_loss_grad(Yd, Ys, stats, G, dtype, cout, tokens, stream);
+  return launch_loss_grad(Yd, Ys, stats, G, dtype, cout, tokens, tokens, stream);
 }
 
 }  // extern "C"

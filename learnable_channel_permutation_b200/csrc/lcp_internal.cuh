@@ -129,12 +129,48 @@ __device__ __forceinline__ uint32_t nm4_keep(const uint32_t (&v)[NV], int n) {
 //   img_p_hi [t][i][j] = bf16(P[i][j])          (high part)
 // zero_word (optional) is set to 0 by the first CTA: the counter of the
 // layer's fused loss kernel, which runs later on the same stream.
+// One launch over the blocks of several layers (same B, tau, iters): the
+// layers' blocks follow each other in the grid, in layer order; more than
+// kSkMaxLayers layers take several launches.
+constexpr int kSkMaxLayers = 16;
+struct SkFwdLayer {
+  const float* L;
+  float* P;
+  float* ckpt;
+  __nv_bfloat16* pt_hi;
+  __nv_bfloat16* pt_lo;
+  __nv_bfloat16* p_hi;
+  unsigned* zero_word;
+  int blocks;
+};
+struct SkFwdBatch {
+  SkFwdLayer layer[kSkMaxLayers];
+  int n;
+};
+struct SkBwdLayer {
+  const float* L;
+  const float* ckpt;
+  const float* dP;   // [splits, blocks, B, B]
+  float* dL;
+  int splits;
+  int blocks;
+};
+struct SkBwdBatch {
+  SkBwdLayer layer[kSkMaxLayers];
+  int n;
+};
+lcp_status launch_sinkhorn_fwd_batch(const SkFwdLayer* layers, int n, int B, float tau, int iters, cudaStream_t st);
+lcp_status launch_sinkhorn_bwd_batch(const SkBwdLayer* layers, int n, int B, float tau, int iters, cudaStream_t st);
 lcp_status launch_sinkhorn_fwd(const float* L, float* P, float* ckpt, __nv_bfloat16* img_pt_hi,
                                __nv_bfloat16* img_pt_lo, __nv_bfloat16* img_p_hi, unsigned* zero_word,
                                int nblocks, int B, float tau, int iters, cudaStream_t st);
 lcp_status launch_sinkhorn_bwd(const float* L, const float* ckpt, const float* dP, int splits,
                                float* dL, int nblocks, int B, float tau, int iters,
                                cudaStream_t st);
+
+// out[i] = sum over s < splits of parts[s * n + i] (float32, n a multiple of 4,
+// summed in index order): the block backward's dP partials for a caller.
+lcp_status launch_sum_splits(const float* parts, int splits, size_t n, float* out, cudaStream_t st);
 
 // N:M mask of a [rows, cols] matrix (float or bf16) into packed bits.
 lcp_status launch_nm_mask(const void* Wp, uint32_t* bits, int rows, int cols, int n, int m,
@@ -156,16 +192,28 @@ lcp_status launch_simt_gemm(const SimtGemm& g, lcp_dtype ta, lcp_dtype tb, lcp_d
                             cudaStream_t st);
 
 // Loss.  stats[t] = {<yd,ys>, |yd|^2, |ys|^2, cos}.  G (optional) in dtype.
+// `norm` is the token count the mean is taken over: `tokens` for a whole
+// batch, the global count for one shard of it (the shards' losses and
+// gradients then add up to the whole batch's).
 lcp_status launch_loss_token(const float* Yd, const float* Ys, float* stats, void* G,
-                             lcp_dtype gdt, int cout, int tokens, cudaStream_t st);
+                             lcp_dtype gdt, int cout, int tokens, int norm, cudaStream_t st);
 lcp_status launch_loss_grad(const float* Yd, const float* Ys, const float* stats, void* G,
-                            lcp_dtype gdt, int cout, int tokens, cudaStream_t st);
-lcp_status launch_loss_reduce(const float* stats, float* loss, int tokens, cudaStream_t st);
+                            lcp_dtype gdt, int cout, int tokens, int norm, cudaStream_t st);
+lcp_status launch_loss_reduce(const float* stats, float* loss, int tokens, int norm, cudaStream_t st);
 // One launch: stats, G and the loss.  cout <= 16384.  `counter` must be zero
 // at launch (an earlier kernel of the step clears it); the kernel leaves it zero.
 bool loss_fused_supported(int cout);
 lcp_status launch_loss_fused(const float* Yd, const float* Ys, float* stats, void* G, lcp_dtype gdt,
-                             float* loss, unsigned* counter, int cout, int tokens, cudaStream_t st);
+                             float* loss, unsigned* counter, int cout, int tokens, int norm, cudaStream_t st);
+
+// Loss and G (bf16) from the calibration GEMM's loss epilogue: the pair
+// D = Y_d - Y_s, Y_s (bf16 [tokens, cout]) and the per-token partials of the
+// nslots 64-channel slots (float4 [tokens, nslots]).  cout <= 16384 (see
+// loss_pair_supported).  `counter` as for launch_loss_fused.
+bool loss_pair_supported(int cout);
+lcp_status launch_loss_pair(const __nv_bfloat16* D, const __nv_bfloat16* Ys, const float* partials, int nslots,
+                            float* stats, __nv_bfloat16* G, float* loss, unsigned* counter, int cout, int tokens,
+                            int norm, cudaStream_t st);
 
 // Tensor-core (tcgen05) kernels, bf16 operands, float32 accumulation.
 // given_mask (B <= 64): the mask is read from `mask` instead of computed.
@@ -181,6 +229,13 @@ lcp_status launch_score_mask_tc(const __nv_bfloat16* S, const __nv_bfloat16* img
 lcp_status launch_calib_gemm_tc(const __nv_bfloat16* X, const __nv_bfloat16* W,
                                 const __nv_bfloat16* At, float* Yd, float* Ys, int tokens,
                                 int cout, int cin, cudaStream_t st);
+// The calibration products with the loss reduction in the epilogue: D = Y_d -
+// Y_s and Ys (bf16 [tokens, cout]) and the slot partials (float4 [tokens,
+// calib_loss_slots(cout)]) -- see gemm_tc.cu.
+int calib_loss_slots(int cout);
+lcp_status launch_calib_loss_tc(const __nv_bfloat16* X, const __nv_bfloat16* W, const __nv_bfloat16* At,
+                                __nv_bfloat16* D, __nv_bfloat16* Ys, float* partials, int tokens, int cout, int cin,
+                                cudaStream_t st);
 lcp_status launch_bwd_gemm_tc(const __nv_bfloat16* G, const __nv_bfloat16* X,
                               __nv_bfloat16* dAt, int tokens, int cout, int cin,
                               cudaStream_t st);
@@ -189,7 +244,7 @@ lcp_status launch_block_bwd_tc(const __nv_bfloat16* W, const __nv_bfloat16* dAt,
                                const __nv_bfloat16* img_pt_lo, float* dP_partials, int splits,
                                int cout, int cin, int B, cudaStream_t st);
 int block_bwd_tc_splits(int cout, int cin, int B);
-bool block_bwd_tc_supported(int B);   // B <= 128 (TMEM/smem budget of the fused kernel)
+bool block_bwd_tc_supported(int B);   // every B (B = 256: four CTAs per block, one dP quadrant each)
 
 // Hardening (per-block maximum-weight assignment).  Writes perm [nblocks, B],
 // optionally the 0/1 matrices P_hard and the bf16 operand images of P_hard in
