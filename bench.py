@@ -59,21 +59,26 @@ def workload(name):
     raise SystemExit(f"unknown workload {name}")
 
 
-def stage_work(wl, li, splits=1):
+def stage_work(wl, li, splits=1, fused_loss=True):
     """Algorithmic work of each stage for one layer: (kind, amount).
 
     kind "flop" for the tensor-core contractions, "byte" for the HBM-bound
     stages (compulsory bytes: every input read once, every output written once).
+    With the loss reduction in the calibration GEMM's epilogue (the bf16
+    tensor-core path) the loss stage reads D and Y_s in bf16 and the slot
+    partials; otherwise Y_d and Y_s in float32.
     """
     co, ci, T = li.spec.cout, li.spec.cin, li.spec.tokens
     B, it = wl.block, wl.iters
     nb = ci // B
     e = 2 if wl.dtype == "bf16" else 4
+    loss_bytes = (T * co * (2 + 2 + e) + T * ((co + 63) // 64) * 16 + T * 16 if fused_loss
+                  else T * co * (4 + 4 + e) + T * 16)
     return {
         "sinkhorn_fwd": ("byte", nb * B * B * (4 + 4 + 3 * 2) + nb * it * 2 * B * 4),
         "permute_mask": ("byte", co * ci * (e + e) + co * ci // 8 + 3 * nb * B * B * 2),
         "calib_gemm": ("flop", 2 * 2 * T * co * ci),
-        "loss": ("byte", T * co * (4 + 4 + e) + T * 16),
+        "loss": ("byte", loss_bytes),
         "bwd_gemm": ("flop", 2 * T * co * ci),
         "block_bwd": ("byte", co * ci * (e + e) + co * ci // 8 + splits * nb * B * B * 4),
         "sinkhorn_bwd": ("byte", nb * B * B * (4 + 4 * splits + 4) + nb * it * 2 * B * 4),
@@ -389,7 +394,7 @@ def main():
         return 0
 
     pk, pk_src = peaks()
-    work = stage_work(wl, li)
+    work = stage_work(wl, li, fused_loss=wl.dtype == "bf16" and not args.simt)
     dom = max(stage_ms, key=lambda s: stage_ms[s])
     kind, amount = work[dom]
     dur_s = stage_ms[dom] / 1e3
@@ -550,6 +555,9 @@ def extras(args, b, synth, wl, li, layer, step, flush, pk, dev):
         "note": "library GEMMs on the same shapes for context; the step itself runs only this build's kernels"}
     del Gb
 
+    # the other workload configurations (7B MLP, 13B block, the 4096^2 sweep)
+    out["configs"] = config_runs(b, synth, pk, dev, flush, K)
+
     # inference side: the layer deployed as a 2:4 compressed weight (the hard
     # permutation and mask of one LCP_FLAG_HARD step), decode-sized token counts
     out["inference_24"] = inference_24(b, layer, wl, li, dev, pk, timed, K)
@@ -593,6 +601,112 @@ def extras(args, b, synth, wl, li, layer, step, flush, pk, dev):
         "note": "inputs larger than L2 (456 MB of logits per launch)"}
     del Lb, Pb, ck, dP, dLb
     torch.cuda.empty_cache()
+    return out
+
+
+def config_runs(b, synth, pk, dev, flush, K):
+    """The other workload configurations, each step one lcp_step call over all
+    of its layers, timed like the headline (CUDA-graph replays, L2 flushed
+    before each, inputs already on the device):
+
+    - mlp_7b: gate/up 11008 x 4096 (sharing X) and down 4096 x 11008 with a
+      ReLU-like input, T = 2048;
+    - block_13b: the seven projections of a 13B layer (q/k/v/o 5120^2, gate/up
+      13824 x 5120, down 5120 x 13824), T = 4096;
+    - sweep_4096: the 32 points B x iters x tau x N:M on W 4096 x 4096, T = 2048.
+
+    mlp_7b and block_13b also report the stage times summed over their layers
+    (stage events of every layer, a separate graph) and the calibration GEMM's
+    fraction of the bf16 peak."""
+    import torch
+
+    def timed(fn, reps):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0 = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
+        e1 = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
+        for k in range(reps):
+            flush.zero_()
+            e0[k].record()
+            fn()
+            e1[k].record()
+        torch.cuda.synchronize()
+        return sum(e0[k].elapsed_time(e1[k]) for k in range(reps)) / reps
+
+    def device_layers(inputs):
+        xs, layers = {}, []
+        for li in inputs:
+            X = xs.get(li.spec.x_key)
+            if X is None:
+                X = xs[li.spec.x_key] = torch.from_numpy(li.X).to(dev).to(torch.bfloat16)
+            layers.append(b.alloc_outputs(torch.from_numpy(li.W).to(dev).to(torch.bfloat16), X,
+                                          torch.from_numpy(li.L).to(dev)))
+        return layers
+
+    def flops(inputs, wl):
+        calib = sum(4.0 * li.spec.tokens * li.spec.cout * li.spec.cin for li in inputs)
+        step = sum(6.0 * li.spec.tokens * li.spec.cout * li.spec.cin
+                   + 10.0 * li.spec.cout * li.spec.cin * wl.block for li in inputs)
+        return calib, step
+
+    out = {}
+    for wl in (synth.mlp_7b(), synth.block_13b()):
+        inputs = synth.make_inputs(wl)
+        layers = device_layers(inputs)
+        st = b.Step(layers, wl.block, wl.n, wl.m, wl.iters, wl.tau)
+        g = b.capture(st)
+        ms = timed(g.replay, K)
+        del g
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(b.TIMED_EVENTS * len(layers))]
+        for e in ev:
+            e.record()
+        g = b.capture(st, ev)
+        for _ in range(3):
+            g.replay()
+        reps = max(3, K // 2)
+        stages = {name: 0.0 for name in b.STAGES}
+        for _ in range(reps):
+            flush.zero_()
+            g.replay()
+            torch.cuda.synchronize()
+            for i in range(len(layers)):
+                for k, name in enumerate(b.STAGES):
+                    stages[name] += ev[b.TIMED_EVENTS * i + k].elapsed_time(ev[b.TIMED_EVENTS * i + k + 1]) / reps
+        del g
+        calib, total = flops(inputs, wl)
+        tf = calib / (stages["calib_gemm"] / 1e3) / 1e12
+        out[wl.name] = {
+            "value": 1e3 / ms, "unit": "steps/s", "ms_per_step": ms, "steps": K, "layers": len(layers),
+            "shapes": [[li.spec.cout, li.spec.cin, li.spec.tokens] for li in inputs],
+            "launches": st.launches, "step_TFLOP/s": total / (ms / 1e3) / 1e12,
+            "step_frac_bf16": total / (ms / 1e3) / 1e12 / pk["bf16_tflops"],
+            "stages_ms_summed_over_layers": stages,
+            "roofline_calib_gemm": {"bound": "tensor", "achieved": tf, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                                    "frac": tf / pk["bf16_tflops"]},
+            "note": "one lcp_step call over every layer per step; stage events of every layer in a second graph"}
+        del st, layers, inputs
+        torch.cuda.empty_cache()
+
+    points = {}
+    for B in (32, 64, 128, 256):
+        inputs = synth.make_inputs(synth.sweep_4096(B, 5, 1.0, 2, 4))
+        layers = device_layers(inputs)
+        calib, total = flops(inputs, synth.sweep_4096(B, 5, 1.0, 2, 4))
+        for it in (5, 20):
+            for tau in (1.0, 0.1):
+                for (n, m) in ((2, 4), (4, 8)):
+                    st = b.Step(layers, B, n, m, it, tau)
+                    g = b.capture(st)
+                    ms = timed(g.replay, max(5, K // 2))
+                    del g, st
+                    points[f"B{B}_it{it}_tau{tau:g}_{n}of{m}"] = {
+                        "steps/s": 1e3 / ms, "ms": ms, "step_TFLOP/s": total / (ms / 1e3) / 1e12}
+        del layers, inputs
+        torch.cuda.empty_cache()
+    out["sweep_4096"] = {"points": points, "shape": [4096, 4096, 2048],
+                         "note": "B=256 runs the block backward on CUDA cores (its 256 x 256 dP accumulator "
+                                 "does not fit the fused kernel's tensor memory)"}
     return out
 
 
