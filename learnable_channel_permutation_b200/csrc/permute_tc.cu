@@ -429,16 +429,32 @@ permute_mask_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
     const int row = q * 32 + lane;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     TileIter it(first, nrt);
-    for (int k = 0; k < nloc; ++k, it.next()) {
-      const int b = k % NB;
-      if (!wait_all(WF + b, (uint32_t)(k / NB) & 1u, 67)) break;
+    // W' of tile k + 1 is loaded from TMEM while tile k is processed (tcgen05.wait::ld
+    // waits for every outstanding load of the thread, so the next load is issued
+    // only after the current one has been waited for)
+    uint32_t vn[NV];
+    bool have_next = nloc > 0 && wait_all(WF + 0, 0u, 67);
+    if (have_next) {
       tc_fence_after();
-      uint32_t v[NV];
-      tmem_ld_cols<NV>(tmem + lane_off + b * 128 + h * NV, v);
+      tmem_ld_cols<NV>(tmem + lane_off + h * NV, vn);
+    }
+    for (int k = 0; k < nloc && have_next; ++k, it.next()) {
+      const int b = k % NB;
       tmem_ld_wait();
+      uint32_t v[NV];
+#pragma unroll
+      for (int x = 0; x < NV; ++x) v[x] = vn[x];
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(TMW + b));
+      have_next = false;
+      if (k + 1 < nloc) {
+        const int bn = (k + 1) % NB;
+        if (!wait_all(WF + bn, (uint32_t)((k + 1) / NB) & 1u, 67)) break;
+        tc_fence_after();
+        tmem_ld_cols<NV>(tmem + lane_off + bn * 128 + h * NV, vn);
+        have_next = true;
+      }
       const int grow = it.rt * 128 + row;
       if (Wp_out && grow < cout) {
         float4* o = reinterpret_cast<float4*>(Wp_out + (size_t)grow * cin + it.t * 64 + h * NV);
@@ -476,7 +492,9 @@ permute_mask_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
       fence_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(AF + k % NA));
+      if (k + 1 == nloc) break;
     }
+    tmem_ld_wait();   // no TMEM load of this thread is left outstanding
   } else {
     // copy-out warps: At of tile j -> staging tile j & 1 (refilled once the
     // store of tile j - 2 has read it: SFREE) -> TMA store by the first copy
@@ -494,24 +512,23 @@ permute_mask_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
       // the staging tile is free once the store of tile j - 2 has read it
       if (!wait_all(SFREE + s, us ^ 1u, 70)) break;
       uint8_t* so = sO + s * C::A_BYTES;
+      // both 32-column halves in one round trip; then the TMEM buffer may take At of tile j + NB
+      uint32_t u[2][32];
+      tmem_ld32(tmem + lane_off + b * 128 + 64, u[0]);
+      tmem_ld32(tmem + lane_off + b * 128 + 96, u[1]);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(TMA + b));
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        uint32_t u[32];
-        tmem_ld32(tmem + lane_off + b * 128 + 64 + 32 * hh, u);
-        tmem_ld_wait();
-        if (hh == 1) {   // both halves read: the TMEM buffer may take At of tile j + NB
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar(TMA + b));
-        }
+      for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
         for (int c8 = 0; c8 < 4; ++c8)
           st_sw128(so, row, 4 * hh + c8,
-                   make_uint4(pack_bf16x2(__uint_as_float(u[8 * c8 + 0]), __uint_as_float(u[8 * c8 + 1])),
-                              pack_bf16x2(__uint_as_float(u[8 * c8 + 2]), __uint_as_float(u[8 * c8 + 3])),
-                              pack_bf16x2(__uint_as_float(u[8 * c8 + 4]), __uint_as_float(u[8 * c8 + 5])),
-                              pack_bf16x2(__uint_as_float(u[8 * c8 + 6]), __uint_as_float(u[8 * c8 + 7]))));
-      }
+                   make_uint4(pack_bf16x2(__uint_as_float(u[hh][8 * c8 + 0]), __uint_as_float(u[hh][8 * c8 + 1])),
+                              pack_bf16x2(__uint_as_float(u[hh][8 * c8 + 2]), __uint_as_float(u[hh][8 * c8 + 3])),
+                              pack_bf16x2(__uint_as_float(u[hh][8 * c8 + 4]), __uint_as_float(u[hh][8 * c8 + 5])),
+                              pack_bf16x2(__uint_as_float(u[hh][8 * c8 + 6]), __uint_as_float(u[hh][8 * c8 + 7]))));
       fence_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(SFULL + s));

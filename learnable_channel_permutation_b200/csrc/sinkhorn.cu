@@ -23,14 +23,19 @@
 //  * log domain (wider ranges, e.g. sharply peaked logits, where K would
 //    underflow): the log-sum-exp steps themselves.
 //
+// The kernels are persistent: a CTA (cluster) walks blocks g, g + grid, ... of
+// every layer of the launch, the next block's inputs loaded into registers
+// while the current one runs (B <= 128), so a launch over a whole model's
+// logits keeps its loads in flight.
+//
 // Z_0 never changes, so each thread keeps its share of Z_0 (or K) in registers
 // twice: a row slice (TPR adjacent lanes per row, interleaved columns) for the
 // row steps and a column slice (TPC adjacent lanes per column, interleaved
 // rows) for the column steps.  A step is then register arithmetic, a read of
 // the other side's vector from shared memory and two or three shuffles.
 //
-// One CTA owns one block for B <= 128.  For B = 256 a cluster of 4 CTAs
-// splits the rows; column reductions combine the per-CTA partials through
+// A CTA owns one block at a time for B <= 64; for B = 128 a cluster of 2 CTAs
+// and for B = 256 a cluster of 4 splits the rows; column reductions combine the per-CTA partials through
 // distributed shared memory in a fixed rank order, so every CTA gets
 // bit-identical results (the range that picks the arithmetic is combined the
 // same way).  Every reduction runs in a fixed order.  Exponentials and
@@ -48,8 +53,13 @@ namespace cg = cooperative_groups;
 namespace lcp {
 namespace {
 
+// CTAs (a cluster) per B = 128 block (tuning: 1 or 2)
+#ifndef LCP_SINKHORN_B128_CTAS
+#define LCP_SINKHORN_B128_CTAS 2
+#endif
+
 template <int B> struct SkCfg {
-  static constexpr int CS = (B == 256) ? 4 : 1;                   // CTAs per block
+  static constexpr int CS = (B == 256) ? 4 : (B == 128 ? LCP_SINKHORN_B128_CTAS : 1);  // CTAs per block
   static constexpr int NT = (B == 32) ? 256 : (B == 64 ? 512 : 1024);
   static constexpr int R = B / CS;                                 // rows per CTA
   static constexpr int TPR = NT / R;                               // lanes per row
@@ -165,24 +175,15 @@ __device__ __forceinline__ void block_range(float mx, float mn, float* red, floa
 
 // Forward.  Shared memory (floats): tile[R*(B+1)] rv[R] cv[B] xm[2B] xs[2B] red[66]
 template <int B>
-__global__ void __launch_bounds__(SkCfg<B>::NT, 1)
+__global__ void __launch_bounds__(SkCfg<B>::NT, 1024 / SkCfg<B>::NT)
 sinkhorn_fwd_kernel(const __grid_constant__ SkFwdBatch batch, float tau, int iters) {
   using C = SkCfg<B>;
   pdl_wait();
   pdl_trigger();
-  // this CTA's layer and block within it (the layers' blocks follow each other in the grid)
-  int blk = blockIdx.x / C::CS, li = 0;
-  while (li + 1 < batch.n && blk >= batch.layer[li].blocks) blk -= batch.layer[li++].blocks;
-  const SkFwdLayer& ly = batch.layer[li];
-  const float* __restrict__ L = ly.L;
-  float* __restrict__ P = ly.P;
-  float* __restrict__ ckpt = ly.ckpt;
-  __nv_bfloat16* __restrict__ pt_hi = ly.pt_hi;
-  __nv_bfloat16* __restrict__ pt_lo = ly.pt_lo;
-  __nv_bfloat16* __restrict__ p_hi = ly.p_hi;
-  if (ly.zero_word && blk == 0 && blockIdx.x % C::CS == 0 && threadIdx.x == 0) *ly.zero_word = 0u;
   constexpr int R = C::R, NT = C::NT, CS = C::CS, TPR = C::TPR, EPR = C::EPR, TPC = C::TPC,
                 EPC = C::EPC, LD = C::LD;
+  constexpr int NPRE = R * (B / 4) / NT;   // float4 of L a thread stages per block
+  static_assert(NPRE * NT == R * (B / 4), "the L slab must split evenly over the threads");
   extern __shared__ __align__(16) float sm[];
   float* tile = sm;
   float* rv = tile + R * LD;   // per row of this CTA: a_i (linear) or R_i (log domain)
@@ -194,19 +195,54 @@ sinkhorn_fwd_kernel(const __grid_constant__ SkFwdBatch batch, float tau, int ite
   const int rank = cta_rank<CS>();
   const int row0 = rank * R;
   const int tid = threadIdx.x;
-  const size_t base = (size_t)blk * B * B;
-  const size_t ck0 = (size_t)blk * iters * 2 * B;
   const int r = tid / TPR, c = tid % TPR;     // row slice: row r, columns c + TPR*e
   const int j = tid / TPC, g = tid % TPC;     // column slice: column j, rows g + TPC*e
+  const float inv_tau = 1.0f / tau;
+  // The CTA (cluster) walks the blocks g = blockIdx.x / CS, + gridDim.x / CS, ...
+  // of every layer; the next block's slab of L is loaded into registers while
+  // the current one iterates.
+  int total = 0;
+  for (int i = 0; i < batch.n; ++i) total += batch.layer[i].blocks;
+  const int gstride = gridDim.x / CS;
+  auto locate = [&](int gb, int& li, int& blk) {
+    blk = gb;
+    li = 0;
+    while (li + 1 < batch.n && blk >= batch.layer[li].blocks) blk -= batch.layer[li++].blocks;
+  };
+  float4 pre[NPRE];
+  auto prefetch = [&](int gb) {
+    int li, blk;
+    locate(gb, li, blk);
+    const float4* src = reinterpret_cast<const float4*>(batch.layer[li].L + (size_t)blk * B * B + (size_t)row0 * B);
+#pragma unroll
+    for (int k = 0; k < NPRE; ++k) pre[k] = src[tid + k * NT];
+  };
+  // the look-ahead needs NPRE more registers a thread: not for the 1024-thread B = 256 CTAs
+  constexpr bool AHEAD = NPRE <= 2;
+  if (AHEAD && blockIdx.x / CS < total) prefetch(blockIdx.x / CS);
+  for (int gb = blockIdx.x / CS; gb < total; gb += gstride) {
+  if constexpr (!AHEAD) prefetch(gb);
+  int li, blk;
+  locate(gb, li, blk);
+  const SkFwdLayer& ly = batch.layer[li];
+  float* __restrict__ P = ly.P;
+  float* __restrict__ ckpt = ly.ckpt;
+  __nv_bfloat16* __restrict__ pt_hi = ly.pt_hi;
+  __nv_bfloat16* __restrict__ pt_lo = ly.pt_lo;
+  __nv_bfloat16* __restrict__ p_hi = ly.p_hi;
+  if (ly.zero_word && blk == 0 && rank == 0 && tid == 0) *ly.zero_word = 0u;
+  const size_t base = (size_t)blk * B * B;
+  const size_t ck0 = (size_t)blk * iters * 2 * B;
 
   // Z_0 = L / tau (as L times the correctly rounded 1 / tau: within an ulp)
-  const float inv_tau = 1.0f / tau;
-  for (int q = tid; q < R * (B / 4); q += NT) {
-    const float4 v = reinterpret_cast<const float4*>(L + base + (size_t)row0 * B)[q];
+#pragma unroll
+  for (int k = 0; k < NPRE; ++k) {
+    const int q = tid + k * NT;
     const int rr = q / (B / 4), jj = (q % (B / 4)) * 4;
     float* d = tile + rr * LD + jj;
-    d[0] = v.x * inv_tau; d[1] = v.y * inv_tau; d[2] = v.z * inv_tau; d[3] = v.w * inv_tau;
+    d[0] = pre[k].x * inv_tau; d[1] = pre[k].y * inv_tau; d[2] = pre[k].z * inv_tau; d[3] = pre[k].w * inv_tau;
   }
+  if (AHEAD && gb + gstride < total) prefetch(gb + gstride);   // in flight while this block iterates
   __syncthreads();
   float zr[EPR], zc[EPC];
 #pragma unroll
@@ -382,8 +418,11 @@ sinkhorn_fwd_kernel(const __grid_constant__ SkFwdBatch batch, float tau, int ite
       if constexpr (B < BC) *reinterpret_cast<uint4*>(p_hi + at + zc0 + g8) = zero4;
     }
   }
-  // keep peers' shared memory alive until every CTA of the cluster is done reading it
-  cluster_barrier<CS>();
+  // every thread (and every CTA of the cluster) is done with this block's shared
+  // memory before the next block overwrites it
+  if constexpr (CS > 1) cluster_barrier<CS>();
+  else __syncthreads();
+  }
 }
 
 // Reverse.  dZ lives in registers in the row layout.  The iterate after each
@@ -400,20 +439,14 @@ sinkhorn_fwd_kernel(const __grid_constant__ SkFwdBatch batch, float tau, int ite
 // Shared memory (floats): tile[R*(B+1)] ck[B] ck1[B] part[NW*B] cs[B] xs[2B] red[66]
 //                         (+ stage[iters*2*B] when STAGED)
 template <int B, bool STAGED>
-__global__ void __launch_bounds__(SkCfg<B>::NT, B == 64 ? 2 : 1)
+__global__ void __launch_bounds__(SkCfg<B>::NT, 1024 / SkCfg<B>::NT)
 sinkhorn_bwd_kernel(const __grid_constant__ SkBwdBatch batch, float tau, int iters) {
   using C = SkCfg<B>;
   pdl_wait();
   pdl_trigger();
-  int blk = blockIdx.x / C::CS, li = 0;
-  while (li + 1 < batch.n && blk >= batch.layer[li].blocks) blk -= batch.layer[li++].blocks;
-  const SkBwdLayer& ly = batch.layer[li];
-  const float* __restrict__ L = ly.L;
-  const float* __restrict__ ckpt = ly.ckpt;
-  const float* __restrict__ dP = ly.dP;
-  float* __restrict__ dL = ly.dL;
-  const int splits = ly.splits, nblocks = ly.blocks;
   constexpr int R = C::R, NT = C::NT, CS = C::CS, TPR = C::TPR, EPR = C::EPR, NW = C::NW, LD = C::LD;
+  constexpr int NPRE = R * (B / 4) / NT;   // float4 of L and of dP a thread stages per block
+  static_assert(NPRE * NT == R * (B / 4), "the slab must split evenly over the threads");
   extern __shared__ __align__(16) float sm[];
   float* tile = sm;
   float* ck = tile + R * LD;   // C^(k+1) (log domain) or b^(k+1) = e^{-C^(k+1)} (linear)
@@ -427,19 +460,58 @@ sinkhorn_bwd_kernel(const __grid_constant__ SkBwdBatch batch, float tau, int ite
   const int rank = cta_rank<CS>();
   const int row0 = rank * R;
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-  const size_t base = (size_t)blk * B * B;
-  const size_t split_stride = (size_t)nblocks * B * B;
-  const float* ckb = ckpt + (size_t)blk * iters * 2 * B;
   const int r = tid / TPR, c = tid % TPR;
+  const float inv_tau = 1.0f / tau;
+  // persistent over the blocks of every layer, as the forward kernel: the next
+  // block's slabs of L and of dP (its splits summed in index order) are loaded
+  // into registers while the current one runs
+  int total = 0;
+  for (int i = 0; i < batch.n; ++i) total += batch.layer[i].blocks;
+  const int gstride = gridDim.x / CS;
+  auto locate = [&](int gb, int& li, int& blk) {
+    blk = gb;
+    li = 0;
+    while (li + 1 < batch.n && blk >= batch.layer[li].blocks) blk -= batch.layer[li++].blocks;
+  };
+  float4 preL[NPRE], preD[NPRE];
+  auto prefetch = [&](int gb) {
+    int li, blk;
+    locate(gb, li, blk);
+    const SkBwdLayer& y = batch.layer[li];
+    const size_t off = (size_t)blk * B * B + (size_t)row0 * B;
+    const size_t sstride = (size_t)y.blocks * B * B;
+#pragma unroll
+    for (int k = 0; k < NPRE; ++k) {
+      const int q = tid + k * NT;
+      preL[k] = reinterpret_cast<const float4*>(y.L + off)[q];
+      float4 a = reinterpret_cast<const float4*>(y.dP + off)[q];
+      for (int sp = 1; sp < y.splits; ++sp) {
+        const float4 b = reinterpret_cast<const float4*>(y.dP + (size_t)sp * sstride + off)[q];
+        a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+      }
+      preD[k] = a;
+    }
+  };
+  constexpr bool AHEAD = NPRE <= 2;   // as in the forward kernel
+  if (AHEAD && blockIdx.x / CS < total) prefetch(blockIdx.x / CS);
+  for (int gb = blockIdx.x / CS; gb < total; gb += gstride) {
+  if constexpr (!AHEAD) prefetch(gb);
+  int li, blk;
+  locate(gb, li, blk);
+  const SkBwdLayer& ly = batch.layer[li];
+  const float* __restrict__ ckpt = ly.ckpt;
+  float* __restrict__ dL = ly.dL;
+  const size_t base = (size_t)blk * B * B;
+  const float* ckb = ckpt + (size_t)blk * iters * 2 * B;
 
   float zr[EPR], dz[EPR];
   // Z_0 = L / tau, formed as in the forward kernel
-  const float inv_tau = 1.0f / tau;
-  for (int q = tid; q < R * (B / 4); q += NT) {
-    const float4 v = reinterpret_cast<const float4*>(L + base + (size_t)row0 * B)[q];
+#pragma unroll
+  for (int k = 0; k < NPRE; ++k) {
+    const int q = tid + k * NT;
     const int rr = q / (B / 4), jj = (q % (B / 4)) * 4;
     float* d = tile + rr * LD + jj;
-    d[0] = v.x * inv_tau; d[1] = v.y * inv_tau; d[2] = v.z * inv_tau; d[3] = v.w * inv_tau;
+    d[0] = preL[k].x * inv_tau; d[1] = preL[k].y * inv_tau; d[2] = preL[k].z * inv_tau; d[3] = preL[k].w * inv_tau;
   }
   __syncthreads();
 #pragma unroll
@@ -457,17 +529,15 @@ sinkhorn_bwd_kernel(const __grid_constant__ SkBwdBatch batch, float tau, int ite
 #pragma unroll
     for (int e = 0; e < EPR; ++e) zr[e] = __expf(zr[e] - zmax);   // K
   }
-  // dP summed over the splits in index order
-  for (int q = tid; q < R * (B / 4); q += NT) {
-    float4 a = reinterpret_cast<const float4*>(dP + base + (size_t)row0 * B)[q];
-    for (int s = 1; s < splits; ++s) {
-      const float4 b = reinterpret_cast<const float4*>(dP + (size_t)s * split_stride + base + (size_t)row0 * B)[q];
-      a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
-    }
+  // dP (splits summed)
+#pragma unroll
+  for (int k = 0; k < NPRE; ++k) {
+    const int q = tid + k * NT;
     const int rr = q / (B / 4), jj = (q % (B / 4)) * 4;
     float* d = tile + rr * LD + jj;
-    d[0] = a.x; d[1] = a.y; d[2] = a.z; d[3] = a.w;
+    d[0] = preD[k].x; d[1] = preD[k].y; d[2] = preD[k].z; d[3] = preD[k].w;
   }
+  if (AHEAD && gb + gstride < total) prefetch(gb + gstride);   // in flight while this block runs
   if constexpr (STAGED) {
     // every (R, C) pair in the form the loop uses: a_i = e^{max - R_i} and
     // b_j = e^{-C_j} (linear), R and C as they are (log domain)
@@ -581,11 +651,16 @@ sinkhorn_bwd_kernel(const __grid_constant__ SkBwdBatch batch, float tau, int ite
 #pragma unroll
   for (int e = 0; e < EPR; ++e) tile[r * LD + c + TPR * e] = dz[e] * inv_tau;
   __syncthreads();
-  for (int q = tid; q < R * B; q += NT) {
-    const int rr = q / B, jj = q % B;
-    dL[base + (size_t)(row0 + rr) * B + jj] = tile[rr * LD + jj];
+  for (int q = tid; q < R * (B / 4); q += NT) {
+    const int rr = q / (B / 4), jj = (q % (B / 4)) * 4;
+    const float* src = tile + rr * LD + jj;
+    reinterpret_cast<float4*>(dL + base + (size_t)(row0 + rr) * B)[jj / 4] = make_float4(src[0], src[1], src[2], src[3]);
   }
-  cluster_barrier<CS>();
+  // every thread (and every CTA of the cluster) is done with this block's shared
+  // memory before the next block overwrites it
+  if constexpr (CS > 1) cluster_barrier<CS>();
+  else __syncthreads();
+  }
 }
 
 // out = sum over s of parts[s] (n floats each, summed in index order), float4-wide.
@@ -615,13 +690,29 @@ template <int B> constexpr size_t bwd_smem() {
 // the reverse kernel stages the checkpoint in shared memory up to this many bytes
 constexpr size_t kStageBytes = 64 * 1024;
 
+// Grid of a persistent Sinkhorn launch: one CTA (cluster) per block, at most
+// as many as are resident at once (the kernels walk the remaining blocks).
+template <typename K>
+int grid_blocks(K kernel, int nt, size_t smem, int cs, int blocks) {
+  int per_sm = 1, sms = 148, dev = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, nt, smem) != cudaSuccess || per_sm < 1) {
+    cudaGetLastError();   // this query's own error
+    per_sm = 1;
+  }
+  const int resident = std::max(1, per_sm * sms / cs);
+  return std::min(blocks, resident);
+}
+
 template <int B>
 lcp_status fwd_b(const SkFwdBatch& batch, int blocks, float tau, int iters, cudaStream_t st) {
   using C = SkCfg<B>;
   const lcp_status s0 = ensure_smem_limit(reinterpret_cast<const void*>(sinkhorn_fwd_kernel<B>), (int)fwd_smem<B>(),
                                           "sinkhorn_fwd");
   if (s0 != LCP_OK) return s0;
-  return launch_kernel(sinkhorn_fwd_kernel<B>, dim3(blocks * C::CS), dim3(C::NT), fwd_smem<B>(), st, C::CS, true,
+  const int g = grid_blocks(sinkhorn_fwd_kernel<B>, C::NT, fwd_smem<B>(), C::CS, blocks);
+  return launch_kernel(sinkhorn_fwd_kernel<B>, dim3(g * C::CS), dim3(C::NT), fwd_smem<B>(), st, C::CS, true,
                        "sinkhorn_fwd", batch, tau, iters);
 }
 
@@ -634,13 +725,15 @@ lcp_status bwd_b(const SkBwdBatch& batch, int blocks, float tau, int iters, cuda
     const lcp_status s0 = ensure_smem_limit(reinterpret_cast<const void*>(sinkhorn_bwd_kernel<B, true>), (int)bytes,
                                             "sinkhorn_bwd");
     if (s0 != LCP_OK) return s0;
-    return launch_kernel(sinkhorn_bwd_kernel<B, true>, dim3(blocks * C::CS), dim3(C::NT), bytes, st, C::CS, true,
+    const int g = grid_blocks(sinkhorn_bwd_kernel<B, true>, C::NT, bytes, C::CS, blocks);
+    return launch_kernel(sinkhorn_bwd_kernel<B, true>, dim3(g * C::CS), dim3(C::NT), bytes, st, C::CS, true,
                          "sinkhorn_bwd", batch, tau, iters);
   }
   const lcp_status s0 = ensure_smem_limit(reinterpret_cast<const void*>(sinkhorn_bwd_kernel<B, false>),
                                           (int)bwd_smem<B>(), "sinkhorn_bwd");
   if (s0 != LCP_OK) return s0;
-  return launch_kernel(sinkhorn_bwd_kernel<B, false>, dim3(blocks * C::CS), dim3(C::NT), bwd_smem<B>(), st, C::CS,
+  const int g = grid_blocks(sinkhorn_bwd_kernel<B, false>, C::NT, bwd_smem<B>(), C::CS, blocks);
+  return launch_kernel(sinkhorn_bwd_kernel<B, false>, dim3(g * C::CS), dim3(C::NT), bwd_smem<B>(), st, C::CS,
                        true, "sinkhorn_bwd", batch, tau, iters);
 }
 
