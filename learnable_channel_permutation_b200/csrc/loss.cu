@@ -240,7 +240,8 @@ loss_pair_kernel(const __nv_bfloat16* __restrict__ D, const __nv_bfloat16* __res
   __shared__ double redd[NWARP];
   __shared__ int is_last;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int gw = blockIdx.x * NWARP + warp, nw = gridDim.x * NWARP;
+  // token t goes to CTA t % gridDim.x: every SM gets the same number of tokens to within one
+  const int gw = warp * gridDim.x + blockIdx.x, nw = gridDim.x * NWARP;
   const int oct = cout / 8;   // 16-byte chunks of 8 bf16 per row
   for (int t = gw; t < tokens; t += nw) {
     const uint4* d8 = reinterpret_cast<const uint4*>(D + (size_t)t * cout);
@@ -398,10 +399,15 @@ lcp_status launch_loss_fused(const float* Yd, const float* Ys, float* stats, voi
 
 bool loss_pair_supported(int cout) { return cout <= 16384; }
 
+// 16-byte chunks a lane streams per step of loss_pair_kernel (tuning)
+#ifndef LCP_LOSS_PAIR_NS
+#define LCP_LOSS_PAIR_NS 4
+#endif
+
 lcp_status launch_loss_pair(const __nv_bfloat16* D, const __nv_bfloat16* Ys, const float* partials, int nslots,
                             float* stats, __nv_bfloat16* G, float* loss, unsigned* counter, int cout, int tokens,
                             int norm, cudaStream_t st) {
-  constexpr int NS = 4;
+  constexpr int NS = LCP_LOSS_PAIR_NS;
   int sms = 148, dev = 0, per_sm = 1;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -410,10 +416,9 @@ lcp_status launch_loss_pair(const __nv_bfloat16* D, const __nv_bfloat16* Ys, con
     cudaGetLastError();   // this query's own error
     per_sm = 1;
   }
-  const int warps = (kPairThreads / 32);
-  const int need = (tokens + warps - 1) / warps;   // CTAs for one token a warp
+  // every resident CTA (at most one a token), the tokens interleaved over them
   const int resident = per_sm * sms;
-  return launch_kernel(loss_pair_kernel<NS>, dim3(need < resident ? need : resident), dim3(kPairThreads), 0, st, 1,
+  return launch_kernel(loss_pair_kernel<NS>, dim3(tokens < resident ? tokens : resident), dim3(kPairThreads), 0, st, 1,
                        true, "loss_pair", D, Ys, reinterpret_cast<const float4*>(partials), nslots, stats, G, loss,
                        counter, cout, tokens, norm, 1.0f / (float)norm);
 }
