@@ -11,12 +11,16 @@ namespace {
 // BC = 64 (B = 32 or 64).  One CTA per (channel tile, row segment).  Warp 0
 // streams the (dAt, W) tiles of each 128-row chunk into a 4-stage ring; warp 1
 // issues [W P_hi | W P_lo] (one N = 128 product: the two P images are adjacent
-// in shared memory) and dA = dAt P_hi into one of two TMEM buffers, then, once
-// the epilogue has written A = M.W' and dW' = M.dA, the stacked dP product;
-// warps 2-9 (two per TMEM lane quadrant, 32 columns each) form W' = W P_hi +
-// W P_lo and turn W', dA and the mask into the bf16 operands.  The dP
-// accumulator stays in TMEM for the whole segment and is written once at the
-// end.  TMEM columns: buffer a at 192 a (W P_hi, W P_lo, dA: 64 each), dP at 384.
+// in shared memory) and dA = dAt P_hi into one of two TMEM buffers; warp 2,
+// once the epilogue has written A = M.W' and dW' = M.dA, issues the stacked dP
+// product; warps 3-10 (two per TMEM lane quadrant, 32 columns each) form
+// W' = W P_hi + W P_lo and turn W', dA and the mask into the bf16 operands.
+// The two issuers sit on different SM sub-partitions: issuing a tcgen05.mma
+// costs one thread about 60 cycles on an idle SM and more next to busy
+// epilogue warps, and these products (16 a chunk) take about 70 cycles each
+// on the tensor core, so one issuer would set the pace.  The dP accumulator
+// stays in TMEM for the whole segment and is written once at the end.  TMEM
+// columns: buffer a at 192 a (W P_hi, W P_lo, dA: 64 each), dP at 384.
 template <int NSL> struct BwCfg {
   static constexpr int STAGES = 4;
   static constexpr int T_BYTES = 16384;                  // 128 rows x 64 bf16
@@ -25,7 +29,8 @@ template <int NSL> struct BwCfg {
   static constexpr int SMEM = STAGES * STAGE + 2 * IMG_BYTES + 2 * (2 * T_BYTES) + 1024 + 256;
   static constexpr int EPI_WARPS = 4 * NSL;              // NSL column slices per TMEM lane quadrant
   static constexpr int COLS = 64 / NSL;
-  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+  static constexpr int CTRL_WARPS = 3;                   // producer, two MMA issuers
+  static constexpr int THREADS = 32 * (CTRL_WARPS + EPI_WARPS);
   static constexpr int EPI = 32 * EPI_WARPS;
 };
 
@@ -44,13 +49,13 @@ block_bwd_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_consta
   uint8_t* sPtl = sPth + C::IMG_BYTES;
   uint8_t* sAB = sPtl + C::IMG_BYTES;      // buffer a at + a * 2 * T_BYTES: A | dW' (adjacent)
   uint64_t* bars = reinterpret_cast<uint64_t*>(sAB + 2 * 2 * C::T_BYTES);
-  // bars: full[S] empty[S] wd[2] abf[2] abe[2] dpf drain img
+  // bars: full[S] empty[S] wd[2] abf[2] abe[2] dpf drain img drain2
   constexpr int S = C::STAGES;
-  uint32_t* holder = reinterpret_cast<uint32_t*>(bars + 2 * S + 10);
+  uint32_t* holder = reinterpret_cast<uint32_t*>(bars + 2 * S + 11);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(holder + 1);
   auto bar = [&](int i) { return smem_u32(bars + i); };
   const int FULL = 0, EMPTY = S, WD = 2 * S, ABF = 2 * S + 2, ABE = 2 * S + 4, DPF = 2 * S + 6, DRAIN = 2 * S + 7,
-            IMG = 2 * S + 8;
+            IMG = 2 * S + 8, DRAIN2 = 2 * S + 9;
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int t = blockIdx.x, sidx = blockIdx.y, col0 = t * 64;
@@ -67,6 +72,7 @@ block_bwd_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_consta
     }
     mbar_init(bar(DPF), 1);
     mbar_init(bar(DRAIN), 1);
+    mbar_init(bar(DRAIN2), 1);
     mbar_init(bar(IMG), 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -111,7 +117,6 @@ block_bwd_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_consta
     if (lane == 0) {
       constexpr uint32_t idesc_n = idesc_bf16(128, 64, false, false);
       constexpr uint32_t idesc_w = idesc_bf16(128, 128, false, false);
-      constexpr uint32_t idesc_dp = idesc_bf16(128, 128, true, true);
       bool ok = nchunk == 0 || mbar_wait(bar(IMG), 0, abort_flag, 74);
       // [W P_hi | W P_lo] and dA = dAt P_hi of chunk c into TMEM buffer c & 1
       auto mma1 = [&](int c) -> bool {
@@ -132,11 +137,21 @@ block_bwd_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_consta
         mma_commit(bar(WD + a));
         return true;
       };
-      if (ok && nchunk > 0) ok = mma1(0);
-      for (int c = 0; c < nchunk && ok; ++c) {
+      for (int c = 0; c < nchunk && ok; ++c) ok = mma1(c);
+      mma_commit(bar(DRAIN));
+      mbar_wait_drain(bar(DRAIN), 0, 78);
+    }
+    __syncwarp();
+  } else if (warp == 2) {
+    // dP issuer: the stage of chunk c (dAt | W) and buffer a (A | dW') once the epilogue has
+    // written the latter; its completion also frees the stage (the W' / dA products of the
+    // chunk completed before the epilogue could start)
+    if (lane == 0) {
+      constexpr uint32_t idesc_dp = idesc_bf16(128, 128, true, true);
+      for (int c = 0; c < nchunk; ++c) {
         const int st = c % C::STAGES, a = c & 1;
-        const uint32_t ua = (uint32_t)(c >> 1) & 1u;
-        if (c + 1 < nchunk && !mma1(c + 1)) break;
+        const uint32_t use = (uint32_t)(c / C::STAGES) & 1u, ua = (uint32_t)(c >> 1) & 1u;
+        if (!mbar_wait(bar(FULL + st), use, abort_flag, 82)) break;
         if (!mbar_wait(bar(ABF + a), ua, abort_flag, 77)) break;
         tc_fence_after();
         const uint32_t sg = smem_u32(sStage + st * C::STAGE);
@@ -150,12 +165,12 @@ block_bwd_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_consta
         mma_commit(bar(EMPTY + st));
       }
       mma_commit(bar(DPF));
-      mma_commit(bar(DRAIN));
-      mbar_wait_drain(bar(DRAIN), 0, 78);
+      mma_commit(bar(DRAIN2));
+      mbar_wait_drain(bar(DRAIN2), 0, 83);
     }
     __syncwarp();
   } else {
-    const int e = warp - 2, q = warp & 3, h = e >> 2;   // h: column slice of NV columns
+    const int e = warp - C::CTRL_WARPS, q = warp & 3, h = e >> 2;   // h: column slice of NV columns
     const int row = q * 32 + lane;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     bool ok = true;

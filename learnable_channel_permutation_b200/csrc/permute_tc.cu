@@ -195,33 +195,44 @@ permute_mask_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
 // channel tile stay resident in one of two shared-memory slots.  The ring then
 // carries W tiles only and a stage is free as soon as W' of its tile is
 // formed, so the loads run STAGES tiles ahead of the tensor core.
+// Per tile k two products:
+//   W'_k = W_k [P_hi | P_lo]   one N = 128 product (the two transposed images sit
+//                              side by side in shared memory): TMEM columns
+//                              [0, 64) W P_hi, [64, 128) W P_lo, summed in float32
+//   At_k = A_k P_hi^T          N = 64, once A = M.W'_k is in shared memory
+// Issuing a tcgen05.mma takes one thread about 60 cycles on an idle SM and
+// several times that when the other warps of its SM sub-partition are busy
+// with ALU work, while these small-N products take about 70 cycles each on the
+// tensor core.  So the MMAs are shared by three issuing threads on three
+// sub-partitions, each owning its products' commits:
 //   warp 0: TMA producer (W ring; the images of each channel tile once)
-//   warp 1: MMA issuer: W' = W (P_hi + P_lo) of tile k + 2 into TMEM buffer
-//           (k + 2) % NB, then, once A = M.W' of tile k is in shared memory,
-//           At = A P_hi of tile k into buffer k % NB
-//   warps 2..: MASK_WARPS mask warps (MASK_WARPS / 4 per TMEM lane quadrant,
-//           MCOLS columns each): W' of tile k -> the N:M keep bits (stored to
-//           the mask) and A
-//   last 4 warps: copy-out warps (one per quadrant, 64 columns each): At of
+//   warp 1: W' of every tile into TMEM buffer k % 3
+//   warps 2, 3: At of the even / odd tiles into TMEM buffer k % 2
+//   warps 4..11: 8 mask warps (two per TMEM lane quadrant, 32 columns each):
+//           W' of tile k -> the N:M keep bits (stored to the mask) and A
+//   warps 12..15: copy-out warps (one per quadrant, 64 columns each): At of
 //           tile k -> swizzled staging tile -> TMA store
-// The two epilogue roles run side by side (the mask is ALU work, the copy-out
-// memory traffic) and meet only through mbarriers; the mask warps never wait
-// for the tensor core in steady state.
+// Sixteen warps, four per sub-partition, leave each thread 128 registers.
+// The P-image slot of a channel tile is free once every issuer that had a
+// tile in it has committed; the producer arrives for the At issuer that had
+// none, so each phase of that barrier counts all three.
 struct PwCfg {
   static constexpr int STAGES = 5;
-  static constexpr int NB = 4;                          // TMEM (W', At) buffers of 128 columns
-  static constexpr int NA = 3;                          // A buffers
+  static constexpr int NW = 3;                          // W' TMEM buffers (128 columns: hi | lo)
+  static constexpr int NAT = 2;                         // At TMEM buffers (64 columns)
+  static constexpr int NA = 3;                          // A buffers in shared memory
   static constexpr int W_BYTES = 16384;                 // 128 rows x 64 bf16
   static constexpr int IMG_BYTES = 8192;                // 64 x 64 bf16
   static constexpr int SLOT = 3 * IMG_BYTES;            // Pt_hi | Pt_lo | P_hi
   static constexpr int A_BYTES = 16384;
-  static constexpr int NBAR = 2 * STAGES + 4 * NB + NA + 4 * 2 + 1;
-  static constexpr int SMEM = STAGES * W_BYTES + 2 * SLOT + (NA + 2) * A_BYTES + NBAR * 8 + 16 + 1024;
-  static constexpr int MASK_WARPS = 8, COPY_WARPS = 4;
+  static constexpr int ISSUERS = 3, MASK_WARPS = 8, COPY_WARPS = 4;
   static constexpr int MCOLS = 64 / (MASK_WARPS / 4);   // columns per mask thread
-  static constexpr int MASK0 = 2, COPY0 = MASK0 + MASK_WARPS;   // first warp of each role
+  static constexpr int MASK0 = 1 + ISSUERS, COPY0 = MASK0 + MASK_WARPS;   // first warp of each role
   static constexpr int THREADS = 32 * (COPY0 + COPY_WARPS);
+  static constexpr int NBAR = 2 * STAGES + 2 * NW + 2 * NAT + 2 * NA + 8 + ISSUERS;
+  static constexpr int SMEM = STAGES * W_BYTES + 2 * SLOT + (NA + 2) * A_BYTES + NBAR * 8 + 16 + 1024;
   static_assert(SMEM <= 232448, "shared memory budget");
+  static_assert(NW * 128 + NAT * 64 <= 512, "tensor memory budget");
 };
 
 // position in the flat t-major tile list, advanced one tile at a time
@@ -254,11 +265,12 @@ permute_mask_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
   uint32_t* holder = reinterpret_cast<uint32_t*>(bars + C::NBAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(holder + 1);
   auto bar = [&](int i) { return smem_u32(bars + i); };
-  constexpr int NB = C::NB, NA = C::NA;
-  constexpr int FULL = 0, EMPTY = C::STAGES, WF = 2 * C::STAGES, ATF = WF + NB, TMW = ATF + NB, TMA = TMW + NB,
-                AF = TMA + NB, PREADY = AF + NA, PFREE = PREADY + 2, SFULL = PFREE + 2, SFREE = SFULL + 2,
+  constexpr int S = C::STAGES, NW = C::NW, NAT = C::NAT, NA = C::NA;
+  constexpr int FULL = 0, EMPTY = S, WF = 2 * S, TMW = WF + NW, ATF = TMW + NW, TMA = ATF + NAT, AF = TMA + NAT,
+                AE = AF + NA, PREADY = AE + NA, PFREE = PREADY + 2, SFULL = PFREE + 2, SFREE = SFULL + 2,
                 DRAIN = SFREE + 2;
-  static_assert(DRAIN + 1 == C::NBAR, "barrier count");
+  static_assert(DRAIN + C::ISSUERS == C::NBAR, "barrier count");
+  constexpr bool HAS_AT = MODE != kMaskOnly;
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int nrt = cdiv(cout, 128), ntc = cin / 64;
@@ -269,26 +281,23 @@ permute_mask_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
   const int t_first = first / nrt;
   const int nt = nloc > 0 ? (last - 1) / nrt - t_first + 1 : 0;   // channel tiles met by the run
   const int words = cin / 32;
+  auto jt_of = [&](int k) { return (first + k) / nrt - t_first; };   // run-local channel tile of tile k
   if (threadIdx.x == 0) {
-    for (int i = 0; i < C::STAGES; ++i) { mbar_init(bar(FULL + i), 1); mbar_init(bar(EMPTY + i), 1); }
-    for (int i = 0; i < NB; ++i) {
-      mbar_init(bar(WF + i), 1);
-      mbar_init(bar(ATF + i), 1);
-      mbar_init(bar(TMW + i), C::MASK_WARPS);
-      mbar_init(bar(TMA + i), C::COPY_WARPS);
-    }
-    for (int i = 0; i < NA; ++i) mbar_init(bar(AF + i), C::MASK_WARPS);
+    for (int i = 0; i < S; ++i) { mbar_init(bar(FULL + i), 1); mbar_init(bar(EMPTY + i), 1); }
+    for (int i = 0; i < NW; ++i) { mbar_init(bar(WF + i), 1); mbar_init(bar(TMW + i), C::MASK_WARPS); }
+    for (int i = 0; i < NAT; ++i) { mbar_init(bar(ATF + i), 1); mbar_init(bar(TMA + i), C::COPY_WARPS); }
+    for (int i = 0; i < NA; ++i) { mbar_init(bar(AF + i), C::MASK_WARPS); mbar_init(bar(AE + i), 1); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(PREADY + i), 1);
-      mbar_init(bar(PFREE + i), 1);
+      mbar_init(bar(PFREE + i), HAS_AT ? 3 : 1);   // the issuers that read the P images
       mbar_init(bar(SFULL + i), C::COPY_WARPS);
       mbar_init(bar(SFREE + i), 1);
     }
-    mbar_init(bar(DRAIN), 1);
+    for (int i = 0; i < C::ISSUERS; ++i) mbar_init(bar(DRAIN + i), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 1) tmem_alloc(smem_u32(holder), 128 * NB);
+  if (warp == 1) tmem_alloc(smem_u32(holder), 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -308,6 +317,12 @@ permute_mask_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
       uint32_t img_issued = 0;        // per slot: images in flight
       int img_next = 0;               // next channel tile (run-local) whose images to load
       bool ok = true;
+      // At issuers (even / odd tiles) without a tile in channel tile jt; the W' issuer has them all
+      auto absent = [&](int jt) -> int {
+        const int k0 = max(0, (t_first + jt) * nrt - first);
+        const int k1 = min(nloc - 1, (t_first + jt + 1) * nrt - 1 - first);
+        return HAS_AT && k1 == k0 ? 1 : 0;
+      };
       // images of run-local channel tiles up to jt, each into slot jt & 1 once
       // the products of channel tile jt - 2 that read the slot have completed
       auto images_upto = [&](int jt) -> bool {
@@ -321,12 +336,14 @@ permute_mask_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
           tma_load_2d(d + C::IMG_BYTES, &tmPtl, bar(PREADY + s), 0, t * 64);
           tma_load_2d(d + 2 * C::IMG_BYTES, &tmPh, bar(PREADY + s), 0, t * 64);
           img_issued |= 1u << s;
+          // this phase of the slot's free barrier: one arrival for each issuer with no tile here
+          for (int a = absent(img_next); a > 0; --a) mbar_arrive(bar(PFREE + s));
         }
         return true;
       };
       // first ring fill: W tiles at once, the P images (written by the
       // Sinkhorn kernel) once the previous kernel has completed
-      const int pre = nloc < C::STAGES ? nloc : C::STAGES;
+      const int pre = nloc < S ? nloc : S;
       TileIter it(first, nrt);
       for (int k = 0; k < pre; ++k, it.next()) {
         mbar_expect_tx(bar(FULL + k), C::W_BYTES);
@@ -340,8 +357,8 @@ permute_mask_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
         ok = images_upto(jt_pre > 1 ? jt_pre : (nt > 1 ? 1 : 0));
       }
       for (int k = pre; k < nloc && ok; ++k, it.next()) {
-        const int st = k % C::STAGES;
-        const uint32_t use = (uint32_t)(k / C::STAGES) & 1u;
+        const int st = k % S;
+        const uint32_t use = (uint32_t)(k / S) & 1u;
         if (!mbar_wait(bar(EMPTY + st), use ^ 1u, abort_flag, 61)) break;
         if (!images_upto(it.t - t_first)) break;
         mbar_expect_tx(bar(FULL + st), C::W_BYTES);
@@ -350,7 +367,7 @@ permute_mask_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
         par = (par & ~(1u << st)) | (use << st);
       }
       // drain: every copy this thread started has landed before the CTA exits
-      for (int st = 0; st < C::STAGES; ++st)
+      for (int st = 0; st < S; ++st)
         if (issued & (1u << st)) mbar_wait_drain(bar(FULL + st), (par >> st) & 1u, 62);
       for (int s = 0; s < 2; ++s)
         if (img_issued & (1u << s)) {
@@ -359,100 +376,87 @@ permute_mask_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
         }
     }
     __syncwarp();
-  } else if (warp == 1) {
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16(128, 64, false, false);
-      TileIter i1(first, nrt), i2(first, nrt);   // tiles of the W' and the At products
-      // W' = W (P_hi + P_lo) of local tile k into the W' half of TMEM buffer
-      // k % NB; the ring stage is free once these products complete
-      auto mma1 = [&](int k) -> bool {
-        const int st = k % C::STAGES, b = k % NB, jt = i1.t - t_first;
-        const uint32_t use = (uint32_t)(k / C::STAGES) & 1u, ub = (uint32_t)(k / NB) & 1u;
-        if ((k == 0 || i1.rt == 0) &&
-            !mbar_wait(bar(PREADY + (jt & 1)), (uint32_t)(jt >> 1) & 1u, abort_flag, 58))
-          return false;                                                        // images of this channel tile
-        if (!mbar_wait(bar(FULL + st), use, abort_flag, 63)) return false;
-        if (!mbar_wait(bar(TMW + b), ub ^ 1u, abort_flag, 64)) return false;   // W' of tile k - NB read
-        tc_fence_after();
-        const uint32_t sw = smem_u32(sStage + st * C::W_BYTES);
+  } else if (warp < C::MASK0) {
+    // issuers: warp 1 issues W' of every tile, warp 2 + p At of the tiles k = p (mod 2)
+    const int role = warp == 1 ? 0 : 1;
+    const int k_first = warp == 1 ? 0 : warp - 2, k_step = warp == 1 ? 1 : 2;
+    if (lane == 0 && (role == 0 || HAS_AT)) {
+      int cur_jt = -1;
+      for (int k = k_first; k < nloc; k += k_step) {
+        const int jt = jt_of(k);
+        // the products of this thread that read the previous channel tile's images are issued
+        if (jt != cur_jt) {
+          if (cur_jt >= 0) mma_commit(bar(PFREE + (cur_jt & 1)));
+          cur_jt = jt;
+        }
+        if (!mbar_wait(bar(PREADY + (jt & 1)), (uint32_t)(jt >> 1) & 1u, abort_flag, 58)) break;
         const uint32_t sp = smem_u32(sSlot + (jt & 1) * C::SLOT);
-        const uint32_t dW = tmem + b * 128;
+        if (role == 0) {
+          const int st = k % S, b = k % NW;
+          if (!mbar_wait(bar(FULL + st), (uint32_t)(k / S) & 1u, abort_flag, 63)) break;
+          if (!mbar_wait(bar(TMW + b), ((uint32_t)(k / NW) & 1u) ^ 1u, abort_flag, 64)) break;   // W' of k - NW read
+          tc_fence_after();
+          constexpr uint32_t idesc = idesc_bf16(128, 128, false, false);
+          const uint32_t sw = smem_u32(sStage + st * C::W_BYTES);
 #pragma unroll
-        for (int k16 = 0; k16 < 4; ++k16) {
-          const uint64_t ad = sdesc(sw + k16 * 32, 16, 1024);
-          mma_bf16(dW, ad, sdesc(sp + k16 * 32, 16, 1024), idesc, k16 != 0);
-          mma_bf16(dW, ad, sdesc(sp + C::IMG_BYTES + k16 * 32, 16, 1024), idesc, true);
-        }
-        mma_commit(bar(WF + b));
-        mma_commit(bar(EMPTY + st));
-        i1.next();
-        return true;
-      };
-      bool ok = true;
-      if constexpr (MODE == kMaskOnly) {
-        for (int k = 0; k < nloc && ok; ++k) {
-          const int jt = i1.t - t_first;
-          const bool last_of_t = k + 1 == nloc || i1.rt == nrt - 1;
-          ok = mma1(k);
-          if (ok && last_of_t) mma_commit(bar(PFREE + (jt & 1)));   // slot reusable
+          for (int k16 = 0; k16 < 4; ++k16)
+            mma_bf16(tmem + b * 128, sdesc(sw + k16 * 32, 16, 1024), sdesc(sp + k16 * 32, 16, 1024), idesc, k16 != 0);
+          mma_commit(bar(WF + b));
+          mma_commit(bar(EMPTY + st));
+        } else {
+          const int a = k % NAT, c = k % NA;
+          if (!mbar_wait(bar(AF + c), (uint32_t)(k / NA) & 1u, abort_flag, 65)) break;            // A of tile k
+          if (!mbar_wait(bar(TMA + a), ((uint32_t)(k / NAT) & 1u) ^ 1u, abort_flag, 69)) break;  // At of k - NAT read
+          tc_fence_after();
+          constexpr uint32_t idesc = idesc_bf16(128, 64, false, false);
+          const uint32_t sa = smem_u32(sA + c * C::A_BYTES);
+          const uint32_t sph = sp + 2 * C::IMG_BYTES;
+#pragma unroll
+          for (int k16 = 0; k16 < 4; ++k16)
+            mma_bf16(tmem + NW * 128 + a * 64, sdesc(sa + k16 * 32, 16, 1024), sdesc(sph + k16 * 32, 16, 1024), idesc,
+                     k16 != 0);
+          mma_commit(bar(ATF + a));
+          mma_commit(bar(AE + c));   // A buffer c reusable
         }
       }
-      // W' runs two tiles ahead of At, so the mask warps find W' ready
-      for (int k = 0; k < 2 && k < nloc && ok && MODE != kMaskOnly; ++k) ok = mma1(k);
-      for (int k = 0; k < nloc && ok && MODE != kMaskOnly; ++k, i2.next()) {
-        const int b = k % NB, jt = i2.t - t_first;
-        const uint32_t ub = (uint32_t)(k / NB) & 1u;
-        if (k + 2 < nloc && !mma1(k + 2)) break;
-        if (!mbar_wait(bar(AF + k % NA), (uint32_t)(k / NA) & 1u, abort_flag, 65)) break;   // A of tile k
-        if (!mbar_wait(bar(TMA + b), ub ^ 1u, abort_flag, 69)) break;   // At of tile k - NB read
-        tc_fence_after();
-        const uint32_t sa = smem_u32(sA + (k % NA) * C::A_BYTES);
-        const uint32_t sph = smem_u32(sSlot + (jt & 1) * C::SLOT + 2 * C::IMG_BYTES);
-        const uint32_t dAt = tmem + b * 128 + 64;
-#pragma unroll
-        for (int k16 = 0; k16 < 4; ++k16)
-          mma_bf16(dAt, sdesc(sa + k16 * 32, 16, 1024), sdesc(sph + k16 * 32, 16, 1024), idesc, k16 != 0);
-        mma_commit(bar(ATF + b));
-        if (k + 1 == nloc || i2.rt == nrt - 1) mma_commit(bar(PFREE + (jt & 1)));   // slot reusable
-      }
-      mma_commit(bar(DRAIN));
-      mbar_wait_drain(bar(DRAIN), 0, 66);
+      if (cur_jt >= 0) mma_commit(bar(PFREE + (cur_jt & 1)));
+      mma_commit(bar(DRAIN + warp - 1));
+      mbar_wait_drain(bar(DRAIN + warp - 1), 0, 66);
     }
     __syncwarp();
   } else if (warp < C::COPY0) {
-    // mask warps: A buffer k % NA was last read by At of tile k - NA, whose
-    // completion the MMA warp saw before it could issue W' of tile k
-    // (k >= NA: the W' product of tile k follows At of tile k - 2 in issue
-    // order, and WF of tile k arrives only after every earlier product)
     constexpr int NV = C::MCOLS;
     const int e = warp - C::MASK0, q = warp & 3, h = e >> 2;   // h: NV-column slice of the tile
     const int row = q * 32 + lane;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     TileIter it(first, nrt);
-    // W' of tile k + 1 is loaded from TMEM while tile k is processed (tcgen05.wait::ld
-    // waits for every outstanding load of the thread, so the next load is issued
-    // only after the current one has been waited for)
-    uint32_t vn[NV];
+    // W' of tile k + 1 (its hi and lo parts) is loaded from TMEM while tile k
+    // is processed (tcgen05.wait::ld waits for every outstanding load of the
+    // thread, so the next load is issued only after the current one has been
+    // waited for)
+    uint32_t hn[NV], ln[NV];
     bool have_next = nloc > 0 && wait_all(WF + 0, 0u, 67);
     if (have_next) {
       tc_fence_after();
-      tmem_ld_cols<NV>(tmem + lane_off + h * NV, vn);
+      tmem_ld_cols<NV>(tmem + lane_off + h * NV, hn);
+      tmem_ld_cols<NV>(tmem + lane_off + 64 + h * NV, ln);
     }
     for (int k = 0; k < nloc && have_next; ++k, it.next()) {
-      const int b = k % NB;
+      const int b = k % NW;
       tmem_ld_wait();
       uint32_t v[NV];
 #pragma unroll
-      for (int x = 0; x < NV; ++x) v[x] = vn[x];
+      for (int x = 0; x < NV; ++x) v[x] = __float_as_uint(__uint_as_float(hn[x]) + __uint_as_float(ln[x]));
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(TMW + b));
       have_next = false;
       if (k + 1 < nloc) {
-        const int bn = (k + 1) % NB;
-        if (!wait_all(WF + bn, (uint32_t)((k + 1) / NB) & 1u, 67)) break;
+        const int bn = (k + 1) % NW;
+        if (!wait_all(WF + bn, (uint32_t)((k + 1) / NW) & 1u, 67)) break;
         tc_fence_after();
-        tmem_ld_cols<NV>(tmem + lane_off + bn * 128 + h * NV, vn);
+        tmem_ld_cols<NV>(tmem + lane_off + bn * 128 + h * NV, hn);
+        tmem_ld_cols<NV>(tmem + lane_off + bn * 128 + 64 + h * NV, ln);
         have_next = true;
       }
       const int grow = it.rt * 128 + row;
@@ -463,24 +467,25 @@ permute_mask_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
           o[qq] = make_float4(__uint_as_float(v[4 * qq]), __uint_as_float(v[4 * qq + 1]),
                               __uint_as_float(v[4 * qq + 2]), __uint_as_float(v[4 * qq + 3]));
       }
-      // keep bits (computed, or given); v becomes A = M.W'
+      // keep bits (computed, or given) of this thread's NV columns: a mask word (NV = 32) or
+      // one 16-bit half of one (NV = 16)
+      const size_t wi = (size_t)grow * words + 2 * it.t;
       uint32_t w;
       if constexpr (MODE == kGivenMask) {
-        static_assert(NV == 32, "one mask word per thread");
-        w = grow < cout ? mask[(size_t)grow * words + 2 * it.t + h] : 0u;
+        if constexpr (NV == 32) w = grow < cout ? mask[wi + h] : 0u;
+        else w = grow < cout ? (uint32_t)reinterpret_cast<const uint16_t*>(mask)[wi * 2 + h] : 0u;
       } else {
         w = MGROUP == 4 ? nm4_keep<NV>(v, n) : nm_bits<MGROUP, NV>(v, n);
         if (grow < cout) {
-          if constexpr (NV == 32) {
-            mask[(size_t)grow * words + 2 * it.t + h] = w;
-          } else {
-            reinterpret_cast<uint16_t*>(mask)[((size_t)grow * words + 2 * it.t) * 2 + h] = (uint16_t)w;
-          }
+          if constexpr (NV == 32) mask[wi + h] = w;
+          else reinterpret_cast<uint16_t*>(mask)[wi * 2 + h] = (uint16_t)w;
         }
       }
       if constexpr (MODE == kMaskOnly) continue;
 #pragma unroll
       for (int x = 0; x < NV; ++x) v[x] = ((w >> x) & 1u) ? v[x] : 0u;
+      // A buffer k % NA was last read by At of tile k - NA
+      if (!wait_all(AE + k % NA, ((uint32_t)(k / NA) & 1u) ^ 1u, 57)) break;
       uint8_t* sa = sA + (k % NA) * C::A_BYTES;
 #pragma unroll
       for (int c8 = 0; c8 < NV / 8; ++c8)
@@ -492,7 +497,6 @@ permute_mask_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
       fence_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(AF + k % NA));
-      if (k + 1 == nloc) break;
     }
     tmem_ld_wait();   // no TMEM load of this thread is left outstanding
   } else {
@@ -504,31 +508,33 @@ permute_mask_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     const bool storer = warp == C::COPY0;
     TileIter it(first, nrt);
-    for (int j = 0; j < nloc && MODE != kMaskOnly; ++j, it.next()) {
-      const int b = j % NB, s = j & 1;
+    for (int j = 0; j < nloc && HAS_AT; ++j, it.next()) {
+      const int a = j % NAT, s = j & 1;
       const uint32_t us = (uint32_t)(j >> 1) & 1u;
-      if (!wait_all(ATF + b, (uint32_t)(j / NB) & 1u, 68)) break;
+      if (!wait_all(ATF + a, (uint32_t)(j / NAT) & 1u, 68)) break;
       tc_fence_after();
       // the staging tile is free once the store of tile j - 2 has read it
       if (!wait_all(SFREE + s, us ^ 1u, 70)) break;
       uint8_t* so = sO + s * C::A_BYTES;
-      // both 32-column halves in one round trip; then the TMEM buffer may take At of tile j + NB
-      uint32_t u[2][32];
-      tmem_ld32(tmem + lane_off + b * 128 + 64, u[0]);
-      tmem_ld32(tmem + lane_off + b * 128 + 96, u[1]);
-      tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(TMA + b));
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh)
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t u[32];
+        tmem_ld32(tmem + lane_off + NW * 128 + a * 64 + hh * 32, u);
+        tmem_ld_wait();
+        if (hh == 1) {
+          // the TMEM buffer may take At of tile j + NAT
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(TMA + a));
+        }
 #pragma unroll
         for (int c8 = 0; c8 < 4; ++c8)
           st_sw128(so, row, 4 * hh + c8,
-                   make_uint4(pack_bf16x2(__uint_as_float(u[hh][8 * c8 + 0]), __uint_as_float(u[hh][8 * c8 + 1])),
-                              pack_bf16x2(__uint_as_float(u[hh][8 * c8 + 2]), __uint_as_float(u[hh][8 * c8 + 3])),
-                              pack_bf16x2(__uint_as_float(u[hh][8 * c8 + 4]), __uint_as_float(u[hh][8 * c8 + 5])),
-                              pack_bf16x2(__uint_as_float(u[hh][8 * c8 + 6]), __uint_as_float(u[hh][8 * c8 + 7]))));
+                   make_uint4(pack_bf16x2(__uint_as_float(u[8 * c8 + 0]), __uint_as_float(u[8 * c8 + 1])),
+                              pack_bf16x2(__uint_as_float(u[8 * c8 + 2]), __uint_as_float(u[8 * c8 + 3])),
+                              pack_bf16x2(__uint_as_float(u[8 * c8 + 4]), __uint_as_float(u[8 * c8 + 5])),
+                              pack_bf16x2(__uint_as_float(u[8 * c8 + 6]), __uint_as_float(u[8 * c8 + 7]))));
+      }
       fence_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(SFULL + s));
@@ -552,7 +558,7 @@ permute_mask_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 128 * NB);
+    tmem_dealloc(tmem, 512);
   }
 }
 
