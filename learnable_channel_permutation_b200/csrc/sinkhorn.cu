@@ -43,6 +43,7 @@
 // relative error, well inside the 1e-5 tolerance on P.
 
 #include <algorithm>
+#include <type_traits>
 #include <cooperative_groups.h>
 #include <math_constants.h>
 
@@ -52,6 +53,18 @@ namespace cg = cooperative_groups;
 
 namespace lcp {
 namespace {
+
+// B = 64 launches with at least this many blocks in all run the forward pass
+// one warp a block (sinkhorn_fwd_warp_kernel) and the reverse pass two warps a
+// block (sinkhorn_bwd_pair_kernel); smaller ones one 512-thread CTA a block.
+// The forward threshold is higher: below it the warp kernel's log-domain
+// fallback is slower than the CTA kernel's.
+#ifndef LCP_SINKHORN_WARP_MIN_BLOCKS
+#define LCP_SINKHORN_WARP_MIN_BLOCKS 1024
+#endif
+#ifndef LCP_SINKHORN_PAIR_MIN_BLOCKS
+#define LCP_SINKHORN_PAIR_MIN_BLOCKS 256
+#endif
 
 // CTAs (a cluster) per B = 128 block (tuning: 1 or 2)
 #ifndef LCP_SINKHORN_B128_CTAS
@@ -692,6 +705,454 @@ constexpr size_t kStageBytes = 64 * 1024;
 
 // Grid of a persistent Sinkhorn launch: one CTA (cluster) per block, at most
 // as many as are resident at once (the kernels walk the remaining blocks).
+// ------------------------------------------- forward, one warp per block ---
+// B = 64, for launches with many blocks (a whole model's logits): the
+// 512-thread kernel above keeps two blocks in flight per SM, and a block's
+// iteration is a chain of barriers and short reductions, so at that size it
+// runs far below the memory bandwidth.  Here one warp owns a block: lane l
+// holds columns 2l and 2l + 1 of all 64 rows of Z_0 (or K) in registers, a
+// column sum is the lane's own loop, a row sum a reduce-scatter across the
+// warp after which lane l holds the sums of rows 2l and 2l + 1, and the row
+// scalings reach every lane through 256 bytes of shared memory.  No barrier
+// beyond the warp's own, and about a dozen blocks in flight per SM.  The
+// arithmetic (linear or log domain, chosen by the same range test), the
+// checkpoint and the outputs are those of sinkhorn_fwd_kernel; only the
+// order of the sums differs.
+constexpr int kSkWarpWarps = 4;   // warps (blocks in flight) per CTA
+
+// One step of a reduce-scatter across the warp: of v[0, 2N) every lane keeps
+// the half selected by `up` and adds the partner lane's copy of it (the
+// partner keeps the other half).
+template <int N>
+__device__ __forceinline__ void rs_step(float (&v)[32], bool up, int o) {
+#pragma unroll
+  for (int q = 0; q < N; ++q) {
+    const float send = up ? v[q] : v[q + N];
+    const float keep = up ? v[q + N] : v[q];
+    v[q] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+  }
+}
+// Row sums of a 64-row block: part(i) is this lane's partial sum of row i;
+// returns the full sums of rows 2 lane and 2 lane + 1 (fixed order).  The
+// first step pairs rows q and q + 32 as their partials are formed, so only 32
+// partials are ever live.
+template <typename F>
+__device__ __forceinline__ float2 row_sums(F part, int lane) {
+  float v[32];
+  const bool up = lane & 16;
+#pragma unroll
+  for (int q = 0; q < 32; ++q) {
+    const float lo = part(q), hi = part(q + 32);
+    v[q] = (up ? hi : lo) + __shfl_xor_sync(0xffffffffu, up ? lo : hi, 16);
+  }
+  rs_step<16>(v, lane & 8, 8);
+  rs_step<8>(v, lane & 4, 4);
+  rs_step<4>(v, lane & 2, 2);
+  rs_step<2>(v, lane & 1, 1);
+  return make_float2(v[0], v[1]);
+}
+// (max, sum of exponentials) pairs of a log-sum-exp, combined
+__device__ __forceinline__ void lse_add(float& m, float& s, float m2, float s2) {
+  const float M = fmaxf(m, m2);
+  s = s * __expf(m - M) + s2 * __expf(m2 - M);
+  m = M;
+}
+template <int N>
+__device__ __forceinline__ void rs_step_lse(float (&m)[32], float (&s)[32], bool up, int o) {
+#pragma unroll
+  for (int q = 0; q < N; ++q) {
+    const float sm = up ? m[q] : m[q + N], ss = up ? s[q] : s[q + N];
+    m[q] = up ? m[q + N] : m[q];
+    s[q] = up ? s[q + N] : s[q];
+    lse_add(m[q], s[q], __shfl_xor_sync(0xffffffffu, sm, o), __shfl_xor_sync(0xffffffffu, ss, o));
+  }
+}
+
+__global__ void __launch_bounds__(32 * kSkWarpWarps)
+sinkhorn_fwd_warp_kernel(const __grid_constant__ SkFwdBatch batch, float tau, int iters) {
+  constexpr int B = 64;
+  pdl_wait();
+  pdl_trigger();
+  __shared__ __align__(16) float rowv[kSkWarpWarps][B];   // a_i (linear) or R_i (log domain)
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  float* rv = rowv[warp];
+  const float inv_tau = 1.0f / tau;
+  int total = 0;
+  for (int i = 0; i < batch.n; ++i) total += batch.layer[i].blocks;
+  const int nw = gridDim.x * kSkWarpWarps;
+  for (int gb = blockIdx.x * kSkWarpWarps + warp; gb < total; gb += nw) {
+    int li = 0, blk = gb;
+    while (li + 1 < batch.n && blk >= batch.layer[li].blocks) blk -= batch.layer[li++].blocks;
+    const SkFwdLayer& ly = batch.layer[li];
+    if (ly.zero_word && blk == 0 && lane == 0) *ly.zero_word = 0u;
+    const size_t base = (size_t)blk * B * B;
+    const size_t ck0 = (size_t)blk * iters * 2 * B;
+    float* __restrict__ ckpt = ly.ckpt;
+    // Z_0, columns 2 lane and 2 lane + 1 (as L times the correctly rounded 1 / tau)
+    float z0[B], z1[B];
+    const float2* src = reinterpret_cast<const float2*>(ly.L + base) + lane;
+#pragma unroll
+    for (int i = 0; i < B; ++i) {
+      const float2 x = __ldcs(src + i * (B / 2));
+      z0[i] = x.x * inv_tau;
+      z1[i] = x.y * inv_tau;
+    }
+    float mx = z0[0], mn = z0[0];
+#pragma unroll
+    for (int i = 0; i < B; ++i) {
+      mx = fmaxf(mx, fmaxf(z0[i], z1[i]));
+      mn = fminf(mn, fminf(z0[i], z1[i]));
+    }
+    const float zmax = group_max<32>(mx), zmin = -group_max<32>(-mn);
+    float b0, b1;   // the lane's columns: b_j (linear) or C_j (log domain)
+    if (zmax - zmin <= kLinearRange) {
+#pragma unroll
+      for (int i = 0; i < B; ++i) {
+        z0[i] = __expf(z0[i] - zmax);
+        z1[i] = __expf(z1[i] - zmax);
+      }
+      b0 = b1 = 1.f;
+      for (int k = 0; k < iters; ++k) {
+        // T_r: a_i = 1 / sum_j K_ij b_j   (R_i = max Z_0 + log of that sum)
+        const float2 rs = row_sums([&](int i) { return fmaf(z0[i], b0, z1[i] * b1); }, lane);
+        __syncwarp();   // every lane has read the previous row scalings
+        reinterpret_cast<float2*>(rv)[lane] = make_float2(__frcp_rn(rs.x), __frcp_rn(rs.y));
+        if (ckpt)
+          reinterpret_cast<float2*>(ckpt + ck0 + (size_t)k * 2 * B)[lane] =
+              make_float2(zmax + __logf(rs.x), zmax + __logf(rs.y));
+        __syncwarp();
+        // T_c: b_j = 1 / sum_i a_i K_ij   (C_j = log of that sum); rows i = r (mod 4)
+        // accumulate separately, then pairwise: four short chains instead of one long one
+        float c0, c1;
+        {
+          float p0[4] = {0.f, 0.f, 0.f, 0.f}, p1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int i = 0; i < B; i += 4) {
+            const float4 a = reinterpret_cast<const float4*>(rv)[i / 4];
+            p0[0] = fmaf(a.x, z0[i], p0[0]); p1[0] = fmaf(a.x, z1[i], p1[0]);
+            p0[1] = fmaf(a.y, z0[i + 1], p0[1]); p1[1] = fmaf(a.y, z1[i + 1], p1[1]);
+            p0[2] = fmaf(a.z, z0[i + 2], p0[2]); p1[2] = fmaf(a.z, z1[i + 2], p1[2]);
+            p0[3] = fmaf(a.w, z0[i + 3], p0[3]); p1[3] = fmaf(a.w, z1[i + 3], p1[3]);
+          }
+          c0 = (p0[0] + p0[1]) + (p0[2] + p0[3]);
+          c1 = (p1[0] + p1[1]) + (p1[2] + p1[3]);
+        }
+        b0 = __frcp_rn(c0);
+        b1 = __frcp_rn(c1);
+        if (ckpt)
+          reinterpret_cast<float2*>(ckpt + ck0 + ((size_t)k * 2 + 1) * B)[lane] = make_float2(__logf(c0), __logf(c1));
+      }
+      // P = a_i K_ij b_j (a_i of the last row step, in shared memory)
+#pragma unroll
+      for (int i = 0; i < B; ++i) {
+        const float a = rv[i];
+        z0[i] = a * z0[i] * b0;
+        z1[i] = a * z1[i] * b1;
+      }
+    } else {
+      // log domain (rare: sharply peaked logits).  Z_0 is read again from L (just loaded, so
+      // cache-resident) instead of being kept, which leaves the registers to the reductions.
+      auto zat = [&](int i, int e) {
+        const float2 x = __ldg(src + i * (B / 2));
+        return (e ? x.y : x.x) * inv_tau;
+      };
+      b0 = b1 = 0.f;
+      for (int k = 0; k < iters; ++k) {
+        // T_r: R_i = LSE_j(z_ij - C_j); the first step pairs rows q and q + 32
+        float m[32], s[32];
+        {
+          const bool up = lane & 16;
+#pragma unroll
+          for (int q = 0; q < 32; ++q) {
+            float mq[2], sq[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const float x0 = zat(q + 32 * h, 0) - b0, x1 = zat(q + 32 * h, 1) - b1;
+              mq[h] = fmaxf(x0, x1);
+              sq[h] = __expf(x0 - mq[h]) + __expf(x1 - mq[h]);
+            }
+            m[q] = up ? mq[1] : mq[0];
+            s[q] = up ? sq[1] : sq[0];
+            lse_add(m[q], s[q], __shfl_xor_sync(0xffffffffu, up ? mq[0] : mq[1], 16),
+                    __shfl_xor_sync(0xffffffffu, up ? sq[0] : sq[1], 16));
+          }
+        }
+        rs_step_lse<16>(m, s, lane & 8, 8);
+        rs_step_lse<8>(m, s, lane & 4, 4);
+        rs_step_lse<4>(m, s, lane & 2, 2);
+        rs_step_lse<2>(m, s, lane & 1, 1);
+        const float R0 = m[0] + __logf(s[0]), R1 = m[1] + __logf(s[1]);
+        __syncwarp();
+        reinterpret_cast<float2*>(rv)[lane] = make_float2(R0, R1);
+        if (ckpt) reinterpret_cast<float2*>(ckpt + ck0 + (size_t)k * 2 * B)[lane] = make_float2(R0, R1);
+        __syncwarp();
+        // T_c: C_j = LSE_i(z_ij - R_i)
+        float m0 = -CUDART_INF_F, m1 = -CUDART_INF_F;
+        for (int i = 0; i < B; ++i) {
+          const float r = rv[i];
+          m0 = fmaxf(m0, zat(i, 0) - r);
+          m1 = fmaxf(m1, zat(i, 1) - r);
+        }
+        float s0 = 0.f, s1 = 0.f;
+        for (int i = 0; i < B; ++i) {
+          const float r = rv[i];
+          s0 += __expf(zat(i, 0) - r - m0);
+          s1 += __expf(zat(i, 1) - r - m1);
+        }
+        b0 = m0 + __logf(s0);
+        b1 = m1 + __logf(s1);
+        if (ckpt) reinterpret_cast<float2*>(ckpt + ck0 + ((size_t)k * 2 + 1) * B)[lane] = make_float2(b0, b1);
+      }
+      // P = exp(Z_0 - R - C)
+#pragma unroll
+      for (int i = 0; i < B; ++i) {
+        const float r = rv[i];
+        z0[i] = __expf(zat(i, 0) - r - b0);
+        z1[i] = __expf(zat(i, 1) - r - b1);
+      }
+    }
+    __syncwarp();   // every lane has read the row vector before the next block rewrites it
+    // P, row i: 256 contiguous bytes a warp store
+    float2* dst = reinterpret_cast<float2*>(ly.P + base) + lane;
+#pragma unroll
+    for (int i = 0; i < B; ++i) dst[i * (B / 2)] = make_float2(z0[i], z1[i]);
+    if (ly.pt_hi) {
+      // operand images (one 64 x 64 tile per block): Pt[j][i] = P[i][j] as
+      // bf16 high and low parts -- rows 2 lane and 2 lane + 1 are this lane's
+      // columns -- and P_hi[i][j] = bf16(P[i][j])
+      __nv_bfloat16* pth = ly.pt_hi + base;
+      __nv_bfloat16* ptl = ly.pt_lo + base;
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float* col = e ? z1 : z0;
+        uint4* oh = reinterpret_cast<uint4*>(pth + (size_t)(2 * lane + e) * B);
+        uint4* ol = reinterpret_cast<uint4*>(ptl + (size_t)(2 * lane + e) * B);
+#pragma unroll
+        for (int g8 = 0; g8 < B / 8; ++g8) {
+          float hv[8], lv[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const float p = col[8 * g8 + u];
+            hv[u] = __bfloat162float(__float2bfloat16_rn(p));
+            lv[u] = p - hv[u];
+          }
+          oh[g8] = make_uint4(pack_bf16x2_rn(hv[0], hv[1]), pack_bf16x2_rn(hv[2], hv[3]),
+                              pack_bf16x2_rn(hv[4], hv[5]), pack_bf16x2_rn(hv[6], hv[7]));
+          ol[g8] = make_uint4(pack_bf16x2_rn(lv[0], lv[1]), pack_bf16x2_rn(lv[2], lv[3]),
+                              pack_bf16x2_rn(lv[4], lv[5]), pack_bf16x2_rn(lv[6], lv[7]));
+        }
+      }
+      uint32_t* ph = reinterpret_cast<uint32_t*>(ly.p_hi + base) + lane;
+#pragma unroll
+      for (int i = 0; i < B; ++i) ph[i * (B / 2)] = pack_bf16x2_rn(z0[i], z1[i]);
+    }
+  }
+}
+
+// ------------------------------------- reverse, two warps per block ---
+// B = 64, for launches with many blocks: a pair of warps owns a block, warp h
+// of the pair rows [32 h, 32 h + 32), lane l columns 2l and 2l + 1, so that
+// both K = exp(Z_0 - max) (or Z_0) and dZ sit in registers (64 values each a
+// lane).  A column sum is the lane's own loop plus the partner warp's
+// partial, exchanged through shared memory with one 64-thread named barrier
+// per column step; a row sum is a reduce-scatter over the warp (lane l ends
+// with row 32 h + l), broadcast through 128 bytes of shared memory.  The
+// block's checkpoint is staged once in the form the loop uses (a_i =
+// e^{max - R_i}, b_j = e^{-C_j}, or R and C).  The steps are those of
+// sinkhorn_bwd_kernel.
+constexpr int kSkPairSlots = 2;   // blocks in flight per CTA (two warps each)
+// shared memory of one slot (floats): checkpoint [iters][2][64], column partials [2 buffers][2 warps][64],
+// row sums [2 warps][32], range [2 warps][2]
+__host__ __device__ constexpr size_t skp_floats(int iters) { return (size_t)iters * 2 * 64 + 256 + 64 + 4; }
+
+__device__ __forceinline__ void pair_sync(int slot) {
+  asm volatile("bar.sync %0, 64;" ::"r"(1 + slot) : "memory");
+}
+
+// Sum over the warp of v[0, 32) per index -> lane l holds the sum of index l.
+__device__ __forceinline__ float rows32_sum(float (&v)[32], int lane) {
+  rs_step<16>(v, lane & 16, 16);
+  rs_step<8>(v, lane & 8, 8);
+  rs_step<4>(v, lane & 4, 4);
+  rs_step<2>(v, lane & 2, 2);
+  rs_step<1>(v, lane & 1, 1);
+  return v[0];
+}
+
+template <bool LIN>
+__device__ __forceinline__ void skp_steps(float (&d0)[32], float (&d1)[32], const float (&k0)[32],
+                                          const float (&k1)[32], const float* stage, float* colp, float* rsum,
+                                          int iters, int h, int lane, int slot) {
+  constexpr int B = 64;
+  for (int k = iters - 1; k >= 0; --k) {
+    const float* av = stage + (size_t)k * 2 * B + 32 * h;   // this warp's rows
+    const float2 bk = reinterpret_cast<const float2*>(stage + ((size_t)k * 2 + 1) * B)[lane];
+    const float2 bk1 = k > 0 ? reinterpret_cast<const float2*>(stage + ((size_t)k * 2 - 1) * B)[lane]
+                             : make_float2(LIN ? 1.f : 0.f, LIN ? 1.f : 0.f);
+    // column sums of dZ: this warp's rows (rows i = r (mod 4) separately, then pairwise),
+    // then both warps' partials in a fixed order
+    float c0, c1;
+    {
+      float p0[4] = {0.f, 0.f, 0.f, 0.f}, p1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        p0[i & 3] += d0[i];
+        p1[i & 3] += d1[i];
+      }
+      c0 = (p0[0] + p0[1]) + (p0[2] + p0[3]);
+      c1 = (p1[0] + p1[1]) + (p1[2] + p1[3]);
+    }
+    float* cp = colp + (k & 1) * 128;   // double-buffered by iteration
+    reinterpret_cast<float2*>(cp + 64 * h)[lane] = make_float2(c0, c1);
+    pair_sync(slot);
+    const float2 p0 = reinterpret_cast<const float2*>(cp)[lane], p1 = reinterpret_cast<const float2*>(cp + 64)[lane];
+    c0 = p0.x + p1.x;
+    c1 = p0.y + p1.y;
+    // column step: dZ -= exp(Z') colsum, Z' the iterate after the column step k;
+    // linear: exp(Z') colsum = (a_i K_ij) (b_j colsum_j)
+    const float g0 = bk.x * c0, g1 = bk.y * c1;
+#pragma unroll
+    for (int i = 0; i < 32; i += 4) {
+      const float4 r4 = *reinterpret_cast<const float4*>(av + i);
+      const float rr[4] = {r4.x, r4.y, r4.z, r4.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if constexpr (LIN) {
+          d0[i + u] = fmaf(-(rr[u] * k0[i + u]), g0, d0[i + u]);
+          d1[i + u] = fmaf(-(rr[u] * k1[i + u]), g1, d1[i + u]);
+        } else {
+          d0[i + u] -= __expf(k0[i + u] - rr[u] - bk.x) * c0;
+          d1[i + u] -= __expf(k1[i + u] - rr[u] - bk.y) * c1;
+        }
+      }
+    }
+    // row step: dZ -= exp(Z'') rowsum, Z'' the iterate after the row step k;
+    // linear: exp(Z'') rowsum = (K_ij b_j) (a_i rowsum_i), the row factor formed by the row's lane
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = d0[i] + d1[i];
+    const float rs = rows32_sum(v, lane);
+    __syncwarp();   // every lane has read the previous row factors
+    rsum[lane] = LIN ? av[lane] * rs : rs;
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < 32; i += 4) {
+      const float4 f4 = *reinterpret_cast<const float4*>(rsum + i);
+      const float ff[4] = {f4.x, f4.y, f4.z, f4.w};
+      float rr[4];
+      if constexpr (!LIN) {
+        const float4 r4 = *reinterpret_cast<const float4*>(av + i);
+        rr[0] = r4.x; rr[1] = r4.y; rr[2] = r4.z; rr[3] = r4.w;
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if constexpr (LIN) {
+          d0[i + u] = fmaf(-(k0[i + u] * bk1.x), ff[u], d0[i + u]);
+          d1[i + u] = fmaf(-(k1[i + u] * bk1.y), ff[u], d1[i + u]);
+        } else {
+          d0[i + u] -= __expf(k0[i + u] - rr[u] - bk1.x) * ff[u];
+          d1[i + u] -= __expf(k1[i + u] - rr[u] - bk1.y) * ff[u];
+        }
+      }
+    }
+  }
+}
+
+__global__ void __launch_bounds__(64 * kSkPairSlots, 3)
+sinkhorn_bwd_pair_kernel(const __grid_constant__ SkBwdBatch batch, float tau, int iters) {
+  constexpr int B = 64;
+  pdl_wait();
+  pdl_trigger();
+  extern __shared__ __align__(16) float skp_smem[];
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int slot = warp >> 1, h = warp & 1;
+  float* stage = skp_smem + (size_t)slot * skp_floats(iters);
+  float* colp = stage + (size_t)iters * 2 * B;
+  float* rsum = colp + 256 + 32 * h;
+  float* rng = colp + 256 + 64;
+  const float inv_tau = 1.0f / tau;
+  int total = 0;
+  for (int i = 0; i < batch.n; ++i) total += batch.layer[i].blocks;
+  const int ns = gridDim.x * kSkPairSlots;
+  for (int gb = blockIdx.x * kSkPairSlots + slot; gb < total; gb += ns) {
+    int li = 0, blk = gb;
+    while (li + 1 < batch.n && blk >= batch.layer[li].blocks) blk -= batch.layer[li++].blocks;
+    const SkBwdLayer& ly = batch.layer[li];
+    const size_t base = (size_t)blk * B * B + (size_t)32 * h * B;   // this warp's first row
+    const float* ckb = ly.ckpt + (size_t)blk * iters * 2 * B;
+    // Z_0 (as in the forward kernel) and its range over the block
+    float k0[32], k1[32];
+    const float2* lsrc = reinterpret_cast<const float2*>(ly.L + base) + lane;
+    float mx = -CUDART_INF_F, mn = CUDART_INF_F;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const float2 x = __ldcs(lsrc + i * (B / 2));
+      k0[i] = x.x * inv_tau;
+      k1[i] = x.y * inv_tau;
+      mx = fmaxf(mx, fmaxf(k0[i], k1[i]));
+      mn = fminf(mn, fminf(k0[i], k1[i]));
+    }
+    mx = group_max<32>(mx);
+    mn = -group_max<32>(-mn);
+    if (lane == 0) {
+      rng[2 * h] = mx;
+      rng[2 * h + 1] = mn;
+    }
+    // dP of this warp's rows, splits summed in index order
+    float d0[32], d1[32];
+    {
+      const size_t sstride = (size_t)ly.blocks * B * B;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        float2 a = __ldcs(reinterpret_cast<const float2*>(ly.dP + base) + lane + i * (B / 2));
+        for (int sp = 1; sp < ly.splits; ++sp) {
+          const float2 bb = __ldcs(reinterpret_cast<const float2*>(ly.dP + (size_t)sp * sstride + base) + lane + i * (B / 2));
+          a.x += bb.x;
+          a.y += bb.y;
+        }
+        d0[i] = a.x;
+        d1[i] = a.y;
+      }
+    }
+    pair_sync(slot);   // both ranges written; the previous block's use of the slot is over
+    const float zmax = fmaxf(rng[0], rng[2]), zmin = fminf(rng[1], rng[3]);
+    const bool linear = zmax - zmin <= kLinearRange;
+    if (linear) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        k0[i] = __expf(k0[i] - zmax);
+        k1[i] = __expf(k1[i] - zmax);
+      }
+    }
+    // the checkpoint, warp h its vectors q = h, h + 2, ... (lane l entries 2l and 2l + 1)
+    for (int q = h; q < iters * 2; q += 2) {
+      const float2 v = reinterpret_cast<const float2*>(ckb + (size_t)q * B)[lane];
+      const bool is_row = (q & 1) == 0;
+      reinterpret_cast<float2*>(stage + (size_t)q * B)[lane] =
+          linear ? (is_row ? make_float2(__expf(zmax - v.x), __expf(zmax - v.y)) : make_float2(__expf(-v.x), __expf(-v.y)))
+                 : v;
+    }
+    pair_sync(slot);
+    // dZ = dP (.) P, P the final iterate
+    {
+      const float2 bL = reinterpret_cast<const float2*>(stage + ((size_t)(iters - 1) * 2 + 1) * B)[lane];
+      const float* aL = stage + (size_t)(iters - 1) * 2 * B + 32 * h;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float ri = aL[i];
+        d0[i] *= linear ? ri * k0[i] * bL.x : __expf(k0[i] - ri - bL.x);
+        d1[i] *= linear ? ri * k1[i] * bL.y : __expf(k1[i] - ri - bL.y);
+      }
+    }
+    if (linear) skp_steps<true>(d0, d1, k0, k1, stage, colp, rsum, iters, h, lane, slot);
+    else skp_steps<false>(d0, d1, k0, k1, stage, colp, rsum, iters, h, lane, slot);
+    // dL = dZ_0 / tau, row i: 256 contiguous bytes a warp store
+    float2* dst = reinterpret_cast<float2*>(ly.dL + base) + lane;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) dst[i * (B / 2)] = make_float2(d0[i] * inv_tau, d1[i] * inv_tau);
+  }
+}
+
 template <typename K>
 int grid_blocks(K kernel, int nt, size_t smem, int cs, int blocks) {
   int per_sm = 1, sms = 148, dev = 0;
@@ -708,6 +1169,13 @@ int grid_blocks(K kernel, int nt, size_t smem, int cs, int blocks) {
 template <int B>
 lcp_status fwd_b(const SkFwdBatch& batch, int blocks, float tau, int iters, cudaStream_t st) {
   using C = SkCfg<B>;
+  if (B == 64 && blocks >= LCP_SINKHORN_WARP_MIN_BLOCKS) {
+    // one warp a block: enough blocks to keep every SM's warps busy
+    const int g = grid_blocks(sinkhorn_fwd_warp_kernel, 32 * kSkWarpWarps, 0, 1,
+                              (blocks + kSkWarpWarps - 1) / kSkWarpWarps);
+    return launch_kernel(sinkhorn_fwd_warp_kernel, dim3(g), dim3(32 * kSkWarpWarps), 0, st, 1, true, "sinkhorn_fwd",
+                         batch, tau, iters);
+  }
   const lcp_status s0 = ensure_smem_limit(reinterpret_cast<const void*>(sinkhorn_fwd_kernel<B>), (int)fwd_smem<B>(),
                                           "sinkhorn_fwd");
   if (s0 != LCP_OK) return s0;
@@ -719,6 +1187,17 @@ lcp_status fwd_b(const SkFwdBatch& batch, int blocks, float tau, int iters, cuda
 template <int B>
 lcp_status bwd_b(const SkBwdBatch& batch, int blocks, float tau, int iters, cudaStream_t st) {
   using C = SkCfg<B>;
+  const size_t pbytes = kSkPairSlots * skp_floats(iters) * sizeof(float);
+  if (B == 64 && blocks >= LCP_SINKHORN_PAIR_MIN_BLOCKS && pbytes <= 96 * 1024) {
+    // two warps a block, everything in registers
+    const lcp_status s0 =
+        ensure_smem_limit(reinterpret_cast<const void*>(sinkhorn_bwd_pair_kernel), (int)pbytes, "sinkhorn_bwd");
+    if (s0 != LCP_OK) return s0;
+    const int g = grid_blocks(sinkhorn_bwd_pair_kernel, 64 * kSkPairSlots, pbytes, 1,
+                              (blocks + kSkPairSlots - 1) / kSkPairSlots);
+    return launch_kernel(sinkhorn_bwd_pair_kernel, dim3(g), dim3(64 * kSkPairSlots), pbytes, st, 1, true,
+                         "sinkhorn_bwd", batch, tau, iters);
+  }
   const size_t stage = (size_t)iters * 2 * B * sizeof(float);
   if (stage <= kStageBytes) {
     const size_t bytes = bwd_smem<B>() + stage;
