@@ -218,6 +218,13 @@ def main():
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the secondary measurements (cached dense output, standalone mask, "
                          "Sinkhorn scaling run, one-core oracle)")
+    ap.add_argument("--only-extra", default=None,
+                    choices=["cached_dense", "hard_step", "score_step", "train", "cublas_same_products", "configs",
+                             "inference_24", "nm_mask", "sinkhorn_scaling"],
+                    help="run this one secondary measurement only")
+    ap.add_argument("--scaling-blocks", type=int, default=40 * (6 * 5120 + 13824) // 64,
+                    help="64 x 64 blocks of the Sinkhorn scaling run (default: every projection of a "
+                         "40-layer 13B-shaped model, 27 840 blocks)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
@@ -468,6 +475,9 @@ def extras(args, b, synth, wl, li, layer, step, flush, pk, dev):
     out = {}
     K = max(5, min(args.steps, 20))
 
+    def want(name):
+        return args.only_extra is None or args.only_extra == name
+
     def timed(fn, reps, flush_between=True):
         for _ in range(3):
             fn()
@@ -483,124 +493,133 @@ def extras(args, b, synth, wl, li, layer, step, flush, pk, dev):
         torch.cuda.synchronize()
         return sum(e0[k].elapsed_time(e1[k]) for k in range(reps)) / reps
 
-    # cached dense output
-    layer["Yd"] = torch.empty(li.spec.tokens, li.spec.cout, dtype=torch.float32, device=dev)
-    fill = b.Step([layer], wl.block, wl.n, wl.m, wl.iters, wl.tau, workspace=step.ws)
-    fill.run()
-    cached = b.Step([layer], wl.block, wl.n, wl.m, wl.iters, wl.tau, flags=b.FLAG_CACHED_DENSE, workspace=step.ws)
-    g = b.capture(cached)
-    ms = timed(g.replay, K)
-    del g
-    layer.pop("Yd")
-    flop = 2 * 2 * li.spec.tokens * li.spec.cout * li.spec.cin - 2 * li.spec.tokens * li.spec.cout * li.spec.cin
-    out["cached_dense"] = {"value": 1e3 / ms, "unit": UNIT, "ms_per_step": ms, "steps": K,
-                           "note": "LCP_FLAG_CACHED_DENSE: Y_d = X W^T read from layer.Yd (computed once), "
-                                   "so the step runs one calibration GEMM problem instead of two; "
-                                   "not the headline", "algorithmic_flop": 2 * flop}
+    if want("cached_dense"):
+        # cached dense output
+        layer["Yd"] = torch.empty(li.spec.tokens, li.spec.cout, dtype=torch.float32, device=dev)
+        fill = b.Step([layer], wl.block, wl.n, wl.m, wl.iters, wl.tau, workspace=step.ws)
+        fill.run()
+        cached = b.Step([layer], wl.block, wl.n, wl.m, wl.iters, wl.tau, flags=b.FLAG_CACHED_DENSE, workspace=step.ws)
+        g = b.capture(cached)
+        ms = timed(g.replay, K)
+        del g
+        layer.pop("Yd")
+        flop = 2 * 2 * li.spec.tokens * li.spec.cout * li.spec.cin - 2 * li.spec.tokens * li.spec.cout * li.spec.cin
+        out["cached_dense"] = {"value": 1e3 / ms, "unit": UNIT, "ms_per_step": ms, "steps": K,
+                               "note": "LCP_FLAG_CACHED_DENSE: Y_d = X W^T read from layer.Yd (computed once), "
+                                       "so the step runs one calibration GEMM problem instead of two; "
+                                       "not the headline", "algorithmic_flop": 2 * flop}
 
-    # hardened step (LCP_FLAG_HARD: per-block assignment, straight-through backward)
-    nb = li.spec.cin // wl.block
-    layer["perm"] = torch.empty(nb, wl.block, dtype=torch.int32, device=dev)
-    hard = b.Step([layer], wl.block, wl.n, wl.m, wl.iters, wl.tau, flags=b.FLAG_HARD)
-    g = b.capture(hard)
-    ms = timed(g.replay, K)
-    del g
-    ms_h = timed(lambda: b.harden(layer["P"], layer["perm"]), K)
-    layer.pop("perm")
-    out["hard_step"] = {"value": 1e3 / ms, "unit": UNIT, "ms_per_step": ms, "steps": K,
-                        "harden_kernel_ms": ms_h, "blocks": nb,
-                        "note": "LCP_FLAG_HARD: the forward pass uses the per-block maximum-weight "
-                                "assignment of the Sinkhorn output (one warp per block), the backward "
-                                "pass is straight-through; not the headline"}
+    if want("hard_step"):
+        # hardened step (LCP_FLAG_HARD: per-block assignment, straight-through backward)
+        nb = li.spec.cin // wl.block
+        layer["perm"] = torch.empty(nb, wl.block, dtype=torch.int32, device=dev)
+        hard = b.Step([layer], wl.block, wl.n, wl.m, wl.iters, wl.tau, flags=b.FLAG_HARD)
+        g = b.capture(hard)
+        ms = timed(g.replay, K)
+        del g
+        ms_h = timed(lambda: b.harden(layer["P"], layer["perm"]), K)
+        layer.pop("perm")
+        out["hard_step"] = {"value": 1e3 / ms, "unit": UNIT, "ms_per_step": ms, "steps": K,
+                            "harden_kernel_ms": ms_h, "blocks": nb,
+                            "note": "LCP_FLAG_HARD: the forward pass uses the per-block maximum-weight "
+                                    "assignment of the Sinkhorn output (one warp per block), the backward "
+                                    "pass is straight-through; not the headline"}
 
-    # mask from Wanda scores (LCP_FLAG_SCORE): S computed once, S_hat = S P_B ranked each step
-    layer["S"] = b.score(layer["W"], layer["X"], b.SCORE_WANDA)
-    sc = b.Step([layer], wl.block, wl.n, wl.m, wl.iters, wl.tau, flags=b.FLAG_SCORE, workspace=step.ws)
-    g = b.capture(sc)
-    ms = timed(g.replay, K)
-    del g
-    layer.pop("S")
-    out["score_step"] = {"value": 1e3 / ms, "unit": UNIT, "ms_per_step": ms, "steps": K, "score": "wanda",
-                         "note": "LCP_FLAG_SCORE: the mask ranks S_hat = S P_B (one permute pass over S for "
-                                 "the mask, one over W with that mask); not the headline"}
+    if want("score_step"):
+        # mask from Wanda scores (LCP_FLAG_SCORE): S computed once, S_hat = S P_B ranked each step
+        layer["S"] = b.score(layer["W"], layer["X"], b.SCORE_WANDA)
+        sc = b.Step([layer], wl.block, wl.n, wl.m, wl.iters, wl.tau, flags=b.FLAG_SCORE, workspace=step.ws)
+        g = b.capture(sc)
+        ms = timed(g.replay, K)
+        del g
+        layer.pop("S")
+        out["score_step"] = {"value": 1e3 / ms, "unit": UNIT, "ms_per_step": ms, "steps": K, "score": "wanda",
+                             "note": "LCP_FLAG_SCORE: the mask ranks S_hat = S P_B (one permute pass over S for "
+                                     "the mask, one over W with that mask); not the headline"}
 
-    # training steps: lcp_step at the scheduled temperature + AdamW on L (lcp_train)
-    tr_step = b.Step([layer], wl.block, wl.n, wl.m, wl.iters, wl.tau, workspace=step.ws)
-    total = 10
-    trainer = b.Trainer(tr_step, b.adamw_params(lr=5e-3), total)
-    ms_tr = timed(lambda: trainer.run(0, total), 3) / total
-    out["train"] = {"value": 1e3 / ms_tr, "unit": UNIT, "ms_per_step": ms_tr, "steps_per_call": total,
-                    "note": "lcp_train: ten steps per call (eager launches), temperature 1 -> 0.1, AdamW "
-                            "lr 5e-3 on the logits after every step; L2 flushed before each call only"}
+    if want("train"):
+        # training steps: lcp_step at the scheduled temperature + AdamW on L (lcp_train)
+        tr_step = b.Step([layer], wl.block, wl.n, wl.m, wl.iters, wl.tau, workspace=step.ws)
+        total = 10
+        trainer = b.Trainer(tr_step, b.adamw_params(lr=5e-3), total)
+        ms_tr = timed(lambda: trainer.run(0, total), 3) / total
+        out["train"] = {"value": 1e3 / ms_tr, "unit": UNIT, "ms_per_step": ms_tr, "steps_per_call": total,
+                        "note": "lcp_train: ten steps per call (eager launches), temperature 1 -> 0.1, AdamW "
+                                "lr 5e-3 on the logits after every step; L2 flushed before each call only"}
 
-    # the step's two dense products through cuBLAS (torch.mm), same shapes and L2 flush, for
-    # context beside the calib_gemm / bwd_gemm stages: Y_d = X W^T and Y_s = X At^T
-    # (float32 outputs where torch.mm takes out_dtype, else bf16), and dAt = G^T X
-    T_, co, ci = li.spec.tokens, li.spec.cout, li.spec.cin
-    Xb = layer["X"] if layer["X"].dtype == torch.bfloat16 else layer["X"].to(torch.bfloat16)
-    Wb = layer["W"] if layer["W"].dtype == torch.bfloat16 else layer["W"].to(torch.bfloat16)
-    Gb = torch.randn(T_, co, device=dev).to(torch.bfloat16)
-    try:
-        torch.mm(Xb[:8], Wb[:8].t(), out_dtype=torch.float32)
-        f32_out = True
-    except Exception:
-        f32_out = False
-    kw = {"out_dtype": torch.float32} if f32_out else {}
-    ms_c = timed(lambda: (torch.mm(Xb, Wb.t(), **kw), torch.mm(Xb, Wb.t(), **kw)), K)
-    ms_g = timed(lambda: torch.mm(Gb.t(), Xb), K)
-    fl = 2.0 * T_ * co * ci
-    out["cublas_same_products"] = {
-        "calib_ms": ms_c, "calib_TFLOP/s": 2 * fl / (ms_c / 1e3) / 1e12, "calib_out": "f32" if f32_out else "bf16",
-        "bwd_ms": ms_g, "bwd_TFLOP/s": fl / (ms_g / 1e3) / 1e12,
-        "note": "library GEMMs on the same shapes for context; the step itself runs only this build's kernels"}
-    del Gb
+    if want("cublas_same_products"):
+        # the step's two dense products through cuBLAS (torch.mm), same shapes and L2 flush, for
+        # context beside the calib_gemm / bwd_gemm stages: Y_d = X W^T and Y_s = X At^T
+        # (float32 outputs where torch.mm takes out_dtype, else bf16), and dAt = G^T X
+        T_, co, ci = li.spec.tokens, li.spec.cout, li.spec.cin
+        Xb = layer["X"] if layer["X"].dtype == torch.bfloat16 else layer["X"].to(torch.bfloat16)
+        Wb = layer["W"] if layer["W"].dtype == torch.bfloat16 else layer["W"].to(torch.bfloat16)
+        Gb = torch.randn(T_, co, device=dev).to(torch.bfloat16)
+        try:
+            torch.mm(Xb[:8], Wb[:8].t(), out_dtype=torch.float32)
+            f32_out = True
+        except Exception:
+            f32_out = False
+        kw = {"out_dtype": torch.float32} if f32_out else {}
+        ms_c = timed(lambda: (torch.mm(Xb, Wb.t(), **kw), torch.mm(Xb, Wb.t(), **kw)), K)
+        ms_g = timed(lambda: torch.mm(Gb.t(), Xb), K)
+        fl = 2.0 * T_ * co * ci
+        out["cublas_same_products"] = {
+            "calib_ms": ms_c, "calib_TFLOP/s": 2 * fl / (ms_c / 1e3) / 1e12, "calib_out": "f32" if f32_out else "bf16",
+            "bwd_ms": ms_g, "bwd_TFLOP/s": fl / (ms_g / 1e3) / 1e12,
+            "note": "library GEMMs on the same shapes for context; the step itself runs only this build's kernels"}
+        del Gb
 
-    # the other workload configurations (7B MLP, 13B block, the 4096^2 sweep)
-    out["configs"] = config_runs(b, synth, pk, dev, flush, K)
+    if want("configs"):
+        # the other workload configurations (7B MLP, 13B block, the 4096^2 sweep)
+        out["configs"] = config_runs(b, synth, pk, dev, flush, K)
 
-    # inference side: the layer deployed as a 2:4 compressed weight (the hard
-    # permutation and mask of one LCP_FLAG_HARD step), decode-sized token counts
-    out["inference_24"] = inference_24(b, layer, wl, li, dev, pk, timed, K)
+    if want("inference_24"):
+        # inference side: the layer deployed as a 2:4 compressed weight (the hard
+        # permutation and mask of one LCP_FLAG_HARD step), decode-sized token counts
+        out["inference_24"] = inference_24(b, layer, wl, li, dev, pk, timed, K)
 
-    # standalone N:M mask on a bf16 W' of the layer's shape
-    Wp = torch.randn(li.spec.cout, li.spec.cin, device=dev).to(torch.bfloat16)
-    bits = torch.empty(li.spec.cout, li.spec.cin // 32, dtype=torch.int32, device=dev)
-    ms = timed(lambda: b.nm_mask(Wp, bits, wl.n, wl.m), K)
-    by = li.spec.cout * li.spec.cin * 2 + li.spec.cout * li.spec.cin // 8
-    out["nm_mask"] = {"ms": ms, "GB/s": by / (ms / 1e3) / 1e9, "frac": by / (ms / 1e3) / 1e9 / pk["hbm_gbs"],
-                      "bytes": by, "shape": [li.spec.cout, li.spec.cin], "nm": f"{wl.n}:{wl.m}"}
-    del Wp, bits
-    # the same kernel on a 16384 x 16384 bf16 W' (512 MiB read): its steady-state bandwidth
-    big = (16384, 16384)
-    Wp = torch.empty(big, device=dev, dtype=torch.bfloat16).normal_()
-    bits = torch.empty(big[0], big[1] // 32, dtype=torch.int32, device=dev)
-    ms = timed(lambda: b.nm_mask(Wp, bits, wl.n, wl.m), K, flush_between=False)
-    by = big[0] * big[1] * 2 + big[0] * big[1] // 8
-    out["nm_mask_large"] = {"ms": ms, "GB/s": by / (ms / 1e3) / 1e9, "frac": by / (ms / 1e3) / 1e9 / pk["hbm_gbs"],
-                            "bytes": by, "shape": list(big), "nm": f"{wl.n}:{wl.m}",
-                            "note": "input larger than L2; no flush needed"}
-    del Wp, bits
+    if want("nm_mask"):
+        # standalone N:M mask on a bf16 W' of the layer's shape
+        Wp = torch.randn(li.spec.cout, li.spec.cin, device=dev).to(torch.bfloat16)
+        bits = torch.empty(li.spec.cout, li.spec.cin // 32, dtype=torch.int32, device=dev)
+        ms = timed(lambda: b.nm_mask(Wp, bits, wl.n, wl.m), K)
+        by = li.spec.cout * li.spec.cin * 2 + li.spec.cout * li.spec.cin // 8
+        out["nm_mask"] = {"ms": ms, "GB/s": by / (ms / 1e3) / 1e9, "frac": by / (ms / 1e3) / 1e9 / pk["hbm_gbs"],
+                          "bytes": by, "shape": [li.spec.cout, li.spec.cin], "nm": f"{wl.n}:{wl.m}"}
+        del Wp, bits
+        # the same kernel on a 16384 x 16384 bf16 W' (512 MiB read): its steady-state bandwidth
+        big = (16384, 16384)
+        Wp = torch.empty(big, device=dev, dtype=torch.bfloat16).normal_()
+        bits = torch.empty(big[0], big[1] // 32, dtype=torch.int32, device=dev)
+        ms = timed(lambda: b.nm_mask(Wp, bits, wl.n, wl.m), K, flush_between=False)
+        by = big[0] * big[1] * 2 + big[0] * big[1] // 8
+        out["nm_mask_large"] = {"ms": ms, "GB/s": by / (ms / 1e3) / 1e9, "frac": by / (ms / 1e3) / 1e9 / pk["hbm_gbs"],
+                                "bytes": by, "shape": list(big), "nm": f"{wl.n}:{wl.m}",
+                                "note": "input larger than L2; no flush needed"}
+        del Wp, bits
 
-    # Sinkhorn scaling run: every projection of a 40-layer 13B-shaped model
-    nblk = 40 * (6 * 5120 + 13824) // 64
-    Bk = 64
-    gen = torch.Generator(device=dev).manual_seed(7)
-    Lb = torch.randn(nblk, Bk, Bk, device=dev, generator=gen) * 1e-3
-    Pb = torch.empty_like(Lb)
-    ck = torch.empty(nblk, wl.iters, 2, Bk, device=dev)
-    dP = torch.randn(nblk, Bk, Bk, device=dev, generator=gen)
-    dLb = torch.empty_like(Lb)
-    ms_f = timed(lambda: b.sinkhorn_fwd(Lb, Pb, ck, wl.tau, wl.iters), 5, flush_between=False)
-    ms_b = timed(lambda: b.sinkhorn_bwd(Lb, ck, dP, dLb, wl.tau, wl.iters), 5, flush_between=False)
-    bf = nblk * Bk * Bk * 8 + nblk * wl.iters * 2 * Bk * 4
-    bb = nblk * Bk * Bk * 12 + nblk * wl.iters * 2 * Bk * 4
-    out["sinkhorn_scaling"] = {
-        "blocks": nblk, "B": Bk, "iters": wl.iters, "L_MB": nblk * Bk * Bk * 4 / 1e6,
-        "fwd": {"ms": ms_f, "GB/s": bf / (ms_f / 1e3) / 1e9, "frac": bf / (ms_f / 1e3) / 1e9 / pk["hbm_gbs"]},
-        "bwd": {"ms": ms_b, "GB/s": bb / (ms_b / 1e3) / 1e9, "frac": bb / (ms_b / 1e3) / 1e9 / pk["hbm_gbs"]},
-        "note": "inputs larger than L2 (456 MB of logits per launch)"}
-    del Lb, Pb, ck, dP, dLb
-    torch.cuda.empty_cache()
+    if want("sinkhorn_scaling"):
+        # Sinkhorn scaling run: every projection of a 40-layer 13B-shaped model
+        nblk = args.scaling_blocks
+        Bk = 64
+        gen = torch.Generator(device=dev).manual_seed(7)
+        Lb = torch.randn(nblk, Bk, Bk, device=dev, generator=gen) * 1e-3
+        Pb = torch.empty_like(Lb)
+        ck = torch.empty(nblk, wl.iters, 2, Bk, device=dev)
+        dP = torch.randn(nblk, Bk, Bk, device=dev, generator=gen)
+        dLb = torch.empty_like(Lb)
+        ms_f = timed(lambda: b.sinkhorn_fwd(Lb, Pb, ck, wl.tau, wl.iters), 5, flush_between=False)
+        ms_b = timed(lambda: b.sinkhorn_bwd(Lb, ck, dP, dLb, wl.tau, wl.iters), 5, flush_between=False)
+        bf = nblk * Bk * Bk * 8 + nblk * wl.iters * 2 * Bk * 4
+        bb = nblk * Bk * Bk * 12 + nblk * wl.iters * 2 * Bk * 4
+        out["sinkhorn_scaling"] = {
+            "blocks": nblk, "B": Bk, "iters": wl.iters, "L_MB": nblk * Bk * Bk * 4 / 1e6,
+            "fwd": {"ms": ms_f, "GB/s": bf / (ms_f / 1e3) / 1e9, "frac": bf / (ms_f / 1e3) / 1e9 / pk["hbm_gbs"]},
+            "bwd": {"ms": ms_b, "GB/s": bb / (ms_b / 1e3) / 1e9, "frac": bb / (ms_b / 1e3) / 1e9 / pk["hbm_gbs"]},
+            "note": f"inputs larger than L2 ({nblk * Bk * Bk * 4 / 1e6:.0f} MB of logits per launch)"}
+        del Lb, Pb, ck, dP, dLb
+        torch.cuda.empty_cache()
     return out
 
 
