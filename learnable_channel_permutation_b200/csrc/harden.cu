@@ -8,19 +8,24 @@
 //
 // Solver: the Hungarian method in its shortest-augmenting-path form, exact up
 // to float32 rounding of the potentials.  Costs c[i][j] = -P_hat[i][j].  Start
-// from u = 0, v[j] = min_i c[i][j] (feasible), and match every column to the
-// row of its minimum when no lower-numbered column claims that row (tight
-// edges).  Then each still-free row grows a shortest-path tree over reduced
-// costs c[i][j] - u[i] - v[j] one column at a time until it reaches a free
-// column, updating the potentials by each step's minimum so that the matched
-// edges stay tight, and flips the matching along the path.
+// from v[j] = min_i c[i][j] (feasible), and match every column to the row of
+// its minimum when no lower-numbered column claims that row (tight edges).
+// Then each still-free row i0 runs a Dijkstra search over reduced costs with
+// the potentials held fixed: tentative distances d[j] = c[i0][j] - v[j]; the
+// nearest unscanned column is scanned, and if it is matched to row i, every
+// unscanned column relaxes to d[j*] - u_i + c[i][j] - v[j], where the row
+// potential u_i = c[i][j*] - v[j*] is implicit (matched edges are tight).
+// Once a free column is reached at distance D, each scanned column's
+// potential moves by d[j] - D and the matching flips along the path.
 //
 // One warp per block.  Lane l owns columns l, l + 32, ...: their potential v,
-// tentative distance and "in tree" flag live in registers; the row potentials
-// u, the column -> row matching and the tree's predecessor links sit in shared
-// memory, next to the block's costs (B <= 128; B = 256 reads its cost rows
-// from global memory).  A tree step is one scan of the owned columns and one
-// warp-wide argmin (ties: lowest column), so the result is deterministic.
+// matched row, tentative distance, predecessor row and scanned flag live in
+// registers; the row -> column matching sits in shared memory next to the
+// block's costs (B <= 128; for B = 256 the first 216 of its 256 rows, the rest
+// read from global memory).  A
+// search step is one scan of the owned columns, one warp-wide argmin (ties:
+// lowest column) and two shuffles from the scanned column's owner, so the
+// result is deterministic.
 
 #include <math_constants.h>
 
@@ -37,9 +42,11 @@ constexpr int kRoot = -2;   // the virtual column the tree of the current row gr
 template <int B> struct HdCfg {
   static constexpr int CPL = B / 32;                        // columns per lane
   static constexpr bool SMEM_COST = B <= 128;
+  // B = 256: the first CROWS cost rows in shared memory, the rest read from global memory
+  static constexpr int CROWS = SMEM_COST ? B : 216;
   static constexpr int WARPS = B <= 64 ? 4 : 1;             // blocks per CTA
-  static constexpr int COST_FLOATS = SMEM_COST ? B * B : 0;
-  static constexpr int PER_WARP = COST_FLOATS + 3 * B;      // costs, u, match, way (4-byte words)
+  static constexpr int COST_FLOATS = CROWS * B;
+  static constexpr int PER_WARP = COST_FLOATS + 3 * B;      // costs, row -> column, match, claims (4-byte words)
   static constexpr size_t SMEM = (size_t)WARPS * PER_WARP * 4;
 };
 
@@ -74,21 +81,21 @@ harden_kernel(const float* __restrict__ P, int* __restrict__ perm, float* __rest
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int blk = blockIdx.x * C::WARPS + warp;
   if (blk >= nblocks) return;
-  float* cost = hd_smem + (size_t)warp * C::PER_WARP;       // c[i][j] = -P[i][j] (B <= 128)
-  float* u = cost + C::COST_FLOATS;                          // row potentials
+  float* cost = hd_smem + (size_t)warp * C::PER_WARP;       // c[i][j] = -P[i][j], rows [0, CROWS)
+  float* u = cost + C::COST_FLOATS;                          // later the row -> column matching
   int* match = reinterpret_cast<int*>(u + B);                // column -> row, kFree if none
-  int* way = match + B;                                      // predecessor column in the tree
+  int* way = match + B;                                      // row -> lowest claiming column
   const float* Pb = P + (size_t)blk * B * B;
 
-  if constexpr (C::SMEM_COST) {
-    for (int q = lane; q < B * B / 4; q += 32) {
+  {
+    for (int q = lane; q < C::CROWS * B / 4; q += 32) {
       const float4 x = reinterpret_cast<const float4*>(Pb)[q];
       cost[4 * q + 0] = -x.x; cost[4 * q + 1] = -x.y; cost[4 * q + 2] = -x.z; cost[4 * q + 3] = -x.w;
     }
   }
   auto c_at = [&](int i, int j) -> float {
     if constexpr (C::SMEM_COST) return cost[i * B + j];
-    else return -__ldg(Pb + (size_t)i * B + j);
+    else return i < C::CROWS ? cost[i * B + j] : -__ldg(Pb + (size_t)i * B + j);
   };
   for (int i = lane; i < B; i += 32) { u[i] = 0.f; match[i] = kFree; way[i] = kRoot; }
   __syncwarp();
@@ -121,76 +128,100 @@ harden_kernel(const float* __restrict__ P, int* __restrict__ perm, float* __rest
     if (way[claim[s]] == j) match[j] = claim[s];
   }
   __syncwarp();
-  // rows left free, as a bitmask over 32-row words, in increasing order
+  // match[] -> registers: x[s] the row of column lane + 32 s; y[] (in the u slot) row -> column
+  int* y = reinterpret_cast<int*>(u);
+  for (int i = lane; i < B; i += 32) y[i] = kFree;
+  __syncwarp();
+  int x[CPL];
+#pragma unroll
+  for (int s = 0; s < CPL; ++s) {
+    x[s] = match[lane + 32 * s];
+    if (x[s] != kFree) y[x[s]] = lane + 32 * s;
+  }
+  __syncwarp();
+  // each free row in increasing order: shortest augmenting path over reduced costs with the
+  // potentials held fixed during the search (the row potentials stay implicit: a matched edge
+  // is tight, u_i = c[i][col(i)] - v[col(i)]), then one update of the scanned columns'
+  // potentials and a flip of the path
   bool ok = true;
   for (int i0 = 0; i0 < B && ok; ++i0) {
-    // is row i0 matched?  (some column holds it)
-    bool held = false;
+    if (y[i0] != kFree) continue;
+    float d[CPL];
+    int pred[CPL];
+    bool sc[CPL];
 #pragma unroll
-    for (int s = 0; s < CPL; ++s) held |= match[lane + 32 * s] == i0;
-    if (__any_sync(0xffffffffu, held)) continue;
-
-    // shortest augmenting path from row i0
-    float minv[CPL];
-    bool used[CPL];
-#pragma unroll
-    for (int s = 0; s < CPL; ++s) { minv[s] = CUDART_INF_F; used[s] = false; }
-    int j0 = kRoot;
-    float u_root = 0.f;     // potential increment of row i0 accumulated in registers
-    int steps = 0;
-    for (;;) {
-      const int r = (j0 == kRoot) ? i0 : match[j0];
-      const float ur = (r == i0) ? u[i0] + u_root : u[r];
+    for (int s = 0; s < CPL; ++s) {
+      d[s] = c_at(i0, lane + 32 * s) - v[s];
+      pred[s] = i0;
+      sc[s] = false;
+    }
+    int jend = -1;
+    float D = 0.f;
+    for (int steps = 0; steps < B; ++steps) {   // at most B columns get scanned
       float best = CUDART_INF_F;
       int bj = B;
 #pragma unroll
       for (int s = 0; s < CPL; ++s) {
         const int j = lane + 32 * s;
-        if (!used[s]) {
-          const float cur = c_at(r, j) - ur - v[s];
-          if (cur < minv[s]) { minv[s] = cur; way[j] = j0; }
-          if (minv[s] < best || (minv[s] == best && j < bj)) { best = minv[s]; bj = j; }
-        }
+        if (!sc[s] && (d[s] < best || (d[s] == best && j < bj))) { best = d[s]; bj = j; }
       }
       warp_argmin(best, bj);
-      const float delta = best;
-      // potentials: rows in the tree up, columns in the tree down, distances down
+      D = best;
+      const int ol = bj & 31, os = bj >> 5;   // owner lane and slot of column bj
+      int xo = x[0];
+      float vo = v[0];
 #pragma unroll
-      for (int s = 0; s < CPL; ++s) {
-        const int j = lane + 32 * s;
-        if (used[s]) {
-          u[match[j]] += delta;
-          v[s] -= delta;
-        } else {
-          minv[s] -= delta;
-        }
-      }
-      u_root += delta;
-      __syncwarp();
-      j0 = bj;
+      for (int s = 1; s < CPL; ++s)
+        if (os == s) { xo = x[s]; vo = v[s]; }
+      const int xi = __shfl_sync(0xffffffffu, xo, ol);
+      const float vj = __shfl_sync(0xffffffffu, vo, ol);
 #pragma unroll
       for (int s = 0; s < CPL; ++s)
-        if (j0 == lane + 32 * s) used[s] = true;
-      if (match[j0] == kFree) break;
-      if (++steps > B) { ok = false; break; }   // cannot happen: a free column is always reachable
-    }
-    if (lane == 0) {
-      u[i0] += u_root;
-      // flip the matching along the tree path back to the root
-      int j = j0;
-      while (ok) {
-        const int jp = way[j];
-        match[j] = (jp == kRoot) ? i0 : match[jp];
-        if (jp == kRoot) break;
-        j = jp;
+        if (s == os && lane == ol) sc[s] = true;
+      if (xi == kFree) { jend = bj; break; }
+      // through column bj to its row xi: distance of that row, less its implicit potential
+      const float h = D - (c_at(xi, bj) - vj);
+#pragma unroll
+      for (int s = 0; s < CPL; ++s) {
+        if (!sc[s]) {
+          const float nd = h + (c_at(xi, lane + 32 * s) - v[s]);
+          if (nd < d[s]) { d[s] = nd; pred[s] = xi; }
+        }
       }
     }
-    __syncwarp();
+    if (jend < 0) { ok = false; break; }   // cannot happen: a free column is always reachable
+    // potentials: every scanned column moves by its distance short of D (the path becomes tight)
+#pragma unroll
+    for (int s = 0; s < CPL; ++s)
+      if (sc[s]) v[s] += d[s] - D;
+    // flip the path from column jend back to row i0
+    int j = jend;
+    for (int guard = 0; guard <= B; ++guard) {
+      const int ol = j & 31, os = j >> 5;
+      int po = pred[0];
+#pragma unroll
+      for (int s = 1; s < CPL; ++s)
+        if (os == s) po = pred[s];
+      const int i = __shfl_sync(0xffffffffu, po, ol);   // the row before column j on the path
+      const int jn = y[i];                                // its column so far (free for i0)
+      __syncwarp();
+#pragma unroll
+      for (int s = 0; s < CPL; ++s)
+        if (s == os && lane == ol) x[s] = i;
+      if (lane == 0) y[i] = j;
+      __syncwarp();
+      if (i == i0) break;
+      if (guard == B) ok = false;                         // cannot happen: the path ends at i0
+      j = jn;
+    }
   }
   if (!__all_sync(0xffffffffu, ok)) {
     if (lane == 0) atomicCAS(&g_harden_error, 0, 201);
     return;
   }
+#pragma unroll
+  for (int s = 0; s < CPL; ++s) match[lane + 32 * s] = x[s];
+  __syncwarp();
 
   // outputs: pi(i) = the column matched to row i, and the hard matrix
   int* pb = perm + (size_t)blk * B;
