@@ -20,9 +20,9 @@
 //                    cores, the gather fused into the staging of the inputs:
 //                    one warp per output row, 16-byte value loads, the inputs
 //                    of the tile resident in shared memory.  Used for float32,
-//                    for fewer than 8 tokens and for bf16 shapes the
-//                    tensor-core variant (infer24_tc.cu: C_in a multiple of 256,
-//                    at most 8192) does not take.
+//                    for one token and for bf16 shapes the tensor-core variant
+//                    (infer24_tc.cu: C_in a multiple of 256, at most 8192) does
+//                    not take.
 
 #include "lcp_internal.cuh"
 
@@ -437,9 +437,10 @@ lcp_status launch_gather(const void* X, const int32_t* perm, void* Xp, int token
 lcp_status launch_sparse24_mm(const void* vals, const uint32_t* meta, const void* X, const int32_t* perm, float* Y,
                               int cout, int cin, int tokens, int B, lcp_dtype dt, cudaStream_t st) {
   const int bshift = perm ? log2_block(B) : 0;
-  // a handful of tokens: the CUDA-core kernel (its per-row stream has the shorter
-  // dependency chain); from 8 tokens on the tensor-core kernel
-  if (dt == LCP_BF16 && tokens >= 8 && sparse24_tc_splits(cout, cin) > 0)
+  // one token: the CUDA-core kernel (its per-row stream has the shorter dependency
+  // chain); from 2 tokens on the sparse tensor-core kernel (its time hardly depends on
+  // the token count up to 16)
+  if (dt == LCP_BF16 && tokens >= 2 && sparse24_tc_splits(cout, cin) > 0)
     return launch_sparse24_tc(static_cast<const __nv_bfloat16*>(vals), meta, static_cast<const __nv_bfloat16*>(X),
                               perm, Y, cout, cin, tokens, bshift, st);
   if (dt == LCP_F32) return sp24_dispatch<float>(vals, meta, X, perm, Y, cout, cin, tokens, bshift, st);

@@ -3,19 +3,24 @@
 // compressed form of infer24.cu (values [C_out, C_in/2], 4-bit position fields
 // [C_out, C_in/32]).
 //
-// The weight stays compressed in HBM (0.5625 of the dense bytes) and is
-// expanded to dense bf16 operand tiles in shared memory on the way to the MMA:
+// The weight stays compressed in HBM (0.5625 of the dense bytes) and goes to
+// the tensor cores compressed: tcgen05.mma.sp (kind::f16, M = 128, N = 16, 32
+// channels a product) takes the two kept values of every group of four as its
+// A operand and their positions as metadata in tensor memory.
 //   - the CTA owns 128 output rows and a K range of C_in / S channels; the S
 //     CTAs of a row tile form a cluster;
 //   - TMA brings the compressed values (128 rows x 64 values, 128-byte
-//     swizzle) and the position words (128 rows x 4 words) of each 128-channel
-//     stage into a 4-stage ring;
-//   - 16 expander warps (four threads per row, 2 x 16 channels each) place every
-//     kept value at its position in two dense 128 x 64 K-major tiles (128-byte
-//     swizzle), zeros elsewhere, into one of two operand buffers;
-//   - an MMA warp issues M = 128, N = 16 MMAs (the tokens, zero-padded to 16)
-//     against the inputs x_pi, staged once per launch in the same tile format
-//     with the gather applied;
+//     swizzle: the A operand of four products as it lands) and the position
+//     words (128 rows x 4 words) of each 128-channel stage into a 4-stage ring;
+//   - four metadata warps (one per TMEM lane quadrant) write each stage's
+//     position words into four TMEM columns (eight-column aligned) in the
+//     layout the sparse product reads: per 16-row group b and j < 8, lane 16 b + j holds the 16-bit
+//     position fields of channels 0-15 of rows 16 b + j (low half) and
+//     16 b + 8 + j (high half), lane 16 b + 8 + j those of channels 16-31
+//     (found with a probe on a B200: one sparse product on known inputs);
+//   - an MMA warp issues the four products of a stage against the inputs
+//     x_pi (the tokens zero-padded to 16), staged once per launch as K-major
+//     tiles with the gather applied;
 //   - the S partial accumulators are summed in rank order through distributed
 //     shared memory, each rank writing 1/S of Y (deterministic, no workspace).
 
@@ -25,22 +30,38 @@ namespace lcp {
 namespace {
 
 struct StCfg {
-  static constexpr int EXP_WARPS = 16;              // expanders (four threads per row of the tile)
+  static constexpr int EXP_WARPS = 16;              // stage the inputs; warps 0-3 then write the metadata
   static constexpr int PROD_WARP = EXP_WARPS, MMA_WARP = EXP_WARPS + 1;
   static constexpr int THREADS = 32 * (EXP_WARPS + 2);
   static constexpr int EXP_THREADS = 32 * EXP_WARPS;
   static constexpr int STG = 4;                     // ring stages of 128 channels
-  static constexpr int NA = 2;                      // dense operand buffers
+  static constexpr int NM = 2;                      // metadata buffers in TMEM (4 columns each)
   static constexpr int V_BYTES = 128 * 128;         // 128 rows x 64 bf16 values
   static constexpr int M_BYTES = 128 * 16;          // 128 rows x 4 position words
-  static constexpr int A_BYTES = 2 * 128 * 128;     // two dense 128 x 64 bf16 tiles
   static constexpr int RED_BYTES = 16 * 128 * 4;    // 16 tokens x 128 rows float32
   static constexpr int MAX_KR = 2048;               // channels per CTA (input image 64 KB)
-  static constexpr int NBAR = 2 * STG + 2 * NA + 1;
-  static int smem(int kr) {
-    return NA * A_BYTES + STG * V_BYTES + (kr / 64) * 2048 + STG * M_BYTES + RED_BYTES + 256 + 1024;
-  }
+  // metadata of product k of buffer m at column TMEM_META + 8 (4 m + k): eight-column
+  // aligned, the placement the probe used (the accumulator: columns 0-15)
+  static constexpr int TMEM_META = 64, TMEM_COLS = 128;
+  static constexpr int NBAR = 2 * STG + 2 * NM + 1;
+  static int smem(int kr) { return STG * V_BYTES + (kr / 64) * 2048 + STG * M_BYTES + RED_BYTES + 256 + 1024; }
 };
+
+// tcgen05.mma.sp, kind::f16: D (+)= A B^T with A the 2:4-compressed M x 16 stored values of
+// 32 channels and their positions at TMEM address `meta`
+__device__ __forceinline__ void mma_bf16_sp(uint32_t d, uint64_t a, uint64_t b, uint32_t meta, uint32_t idesc,
+                                            bool accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "tcgen05.mma.sp.cta_group::1.kind::f16 [%0], %1, %2, [%3], %4, p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(meta), "r"(idesc), "r"(accumulate ? 1u : 0u)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st1(uint32_t taddr, uint32_t v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(v) : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 __device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
   float v;
@@ -48,14 +69,14 @@ __device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
   return v;
 }
 
-// Roles (18 warps): warp 16 loads the ring (TMA), warp 17 issues the MMAs,
-// warps 0-15 stage the inputs, then expand each stage into a dense operand
-// buffer; they meet only through mbarriers:
-//   full[q]  (TMA bytes)        ring slot q holds stage j       -> expanders
-//   empty[q] (16 warp arrivals) every expander has read slot q  -> producer
-//   aready[b] (16 warp arrivals) dense buffer b holds stage j   -> MMA warp
-//   adone[b] (MMA commit)       the products reading b are done -> expanders
-//   fin      (MMA commit)       every product has landed        -> epilogue
+// Roles (18 warps): warp 16 loads the ring (TMA), warp 17 issues the products,
+// warps 0-15 stage the inputs, then warps 0-3 write each stage's metadata into
+// TMEM; they meet only through mbarriers:
+//   full[q]   (TMA bytes)          ring slot q holds stage j        -> metadata warps, MMA warp
+//   empty[q]  (MMA commit)         the products reading slot q done -> producer
+//   mready[m] (4 warp arrivals)    TMEM metadata buffer m holds j   -> MMA warp
+//   mfree[m]  (MMA commit)         the products reading m are done  -> metadata warps
+//   fin       (MMA commit)         every product has landed         -> epilogue
 __global__ void __launch_bounds__(StCfg::THREADS, 1)
 sp24_tc_kernel(const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmM,
                const __nv_bfloat16* __restrict__ X, const int32_t* __restrict__ perm, float* __restrict__ Y,
@@ -63,8 +84,7 @@ sp24_tc_kernel(const __grid_constant__ CUtensorMap tmV, const __grid_constant__ 
   using C = StCfg;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
-  uint8_t* sA = smem;                                   // NA buffers x 32 KB
-  uint8_t* sV = sA + C::NA * C::A_BYTES;                // STG x 16 KB
+  uint8_t* sV = smem;                                   // STG x 16 KB
   uint8_t* sX = sV + C::STG * C::V_BYTES;               // kr / 64 blocks x 2 KB
   uint8_t* sM = sX + (kr / 64) * 2048;                  // STG x 2 KB
   float* sRed = reinterpret_cast<float*>(sM + C::STG * C::M_BYTES);   // [16][128]
@@ -73,9 +93,9 @@ sp24_tc_kernel(const __grid_constant__ CUtensorMap tmV, const __grid_constant__ 
   volatile int* abort_flag = reinterpret_cast<volatile int*>(holder + 1);
   auto full = [&](int q) { return smem_u32(bars + q); };
   auto empty = [&](int q) { return smem_u32(bars + C::STG + q); };
-  auto aready = [&](int b) { return smem_u32(bars + 2 * C::STG + b); };
-  auto adone = [&](int b) { return smem_u32(bars + 2 * C::STG + C::NA + b); };
-  const uint32_t fin = smem_u32(bars + 2 * C::STG + 2 * C::NA);
+  auto mready = [&](int m) { return smem_u32(bars + 2 * C::STG + m); };
+  auto mfree = [&](int m) { return smem_u32(bars + 2 * C::STG + C::NM + m); };
+  const uint32_t fin = smem_u32(bars + 2 * C::STG + 2 * C::NM);
 
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const int S = (int)gridDim.x;                         // cluster = the S splits of a row tile
@@ -85,17 +105,17 @@ sp24_tc_kernel(const __grid_constant__ CUtensorMap tmV, const __grid_constant__ 
   if (tid == 0) {
     for (int q = 0; q < C::STG; ++q) {
       mbar_init(full(q), 1);
-      mbar_init(empty(q), C::EXP_WARPS);
+      mbar_init(empty(q), 1);
     }
-    for (int b = 0; b < C::NA; ++b) {
-      mbar_init(aready(b), C::EXP_WARPS);
-      mbar_init(adone(b), 1);
+    for (int m = 0; m < C::NM; ++m) {
+      mbar_init(mready(m), 4);
+      mbar_init(mfree(m), 1);
     }
     mbar_init(fin, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == C::MMA_WARP) tmem_alloc(smem_u32(holder), 32);
+  if (warp == C::MMA_WARP) tmem_alloc(smem_u32(holder), C::TMEM_COLS);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -127,22 +147,24 @@ sp24_tc_kernel(const __grid_constant__ CUtensorMap tmV, const __grid_constant__ 
     pdl_wait();
     pdl_trigger();
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16(128, 16, false, false);
+      constexpr uint32_t idesc = idesc_bf16(128, 16, false, false) | (1u << 2);   // sparse A
       int j = 0;
       for (; j < nst; ++j) {
-        const int b = j % C::NA;
-        if (!mbar_wait(aready(b), (uint32_t)(j / C::NA) & 1u, abort_flag, 312)) break;
+        const int q = j % C::STG, m = j % C::NM;
+        if (!mbar_wait(full(q), (uint32_t)(j / C::STG) & 1u, abort_flag, 312)) break;
+        if (!mbar_wait(mready(m), (uint32_t)(j / C::NM) & 1u, abort_flag, 317)) break;
         tc_fence_after();
+        const uint32_t a0 = smem_u32(sV + q * C::V_BYTES);
 #pragma unroll
-        for (int tt = 0; tt < 2; ++tt) {
-          const uint32_t a0 = smem_u32(sA + b * C::A_BYTES + tt * (C::A_BYTES / 2));
-          const uint32_t b0 = smem_u32(sX + (2 * j + tt) * 2048);
-#pragma unroll
-          for (int k16 = 0; k16 < 4; ++k16)
-            mma_bf16(tmem, sdesc(a0 + k16 * 32, 16, 1024), sdesc(b0 + k16 * 32, 16, 1024), idesc,
-                     (j | tt | k16) != 0);
+        for (int k = 0; k < 4; ++k) {
+          // 32 channels: stored values k * 16 .. + 15 of the 64 a row; inputs of block
+          // (128 j + 32 k) / 64, half k % 2 of its 128-byte rows
+          const uint32_t b0 = smem_u32(sX + (2 * j + k / 2) * 2048) + (k & 1) * 64;
+          mma_bf16_sp(tmem, sdesc(a0 + k * 32, 16, 1024), sdesc(b0, 16, 1024),
+                      tmem + C::TMEM_META + 8 * (m * 4 + k), idesc, (j | k) != 0);
         }
-        mma_commit(adone(b));
+        mma_commit(empty(q));
+        mma_commit(mfree(m));
       }
       mma_commit(fin);                                  // arrives once every issued product is done
     }
@@ -203,55 +225,40 @@ sp24_tc_kernel(const __grid_constant__ CUtensorMap tmV, const __grid_constant__ 
       }
     }
     fence_async_smem();
+    // the inputs are in shared memory before the first product reads them: every
+    // metadata warp arrives on mready only after this point, and the staging warps
+    // 4-15 join the metadata warps at a named barrier
+    asm volatile("bar.sync 1, %0;" ::"r"(C::EXP_THREADS) : "memory");
 
-    // expand stage j into dense buffer j % NA: thread = (row r, eighths e and e + 4
-    // of the 128 channels: value chunk e, 16 channels = dense chunks 2e, 2e + 1)
-    const int r = tid & 127;
-    for (int j = 0; j < nst; ++j) {
-      const int q = j % C::STG, b = j % C::NA;
-      ok = ok && warp_all(mbar_wait(full(q), (uint32_t)(j / C::STG) & 1u, abort_flag, 315));
-      if (j >= C::NA)
-        ok = ok && warp_all(mbar_wait(adone(b), (uint32_t)((j - C::NA) / C::NA) & 1u, abort_flag, 316));
-      if (!ok) break;
-      constexpr int EPT = 1024 / C::EXP_THREADS;        // eighths per thread
-      uint4 v[EPT];
-      uint32_t fh[EPT];
-#pragma unroll
-      for (int k = 0; k < EPT; ++k) {
-        const int e8 = (tid >> 7) + k * (C::EXP_THREADS / 128);
-        v[k] = *reinterpret_cast<const uint4*>(sV + q * C::V_BYTES + r * 128 + ((e8 ^ (r & 7)) << 4));
-        fh[k] = *reinterpret_cast<const uint16_t*>(sM + q * C::M_BYTES + r * 16 + e8 * 2);
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(empty(q));             // this warp is done with ring slot q
-#pragma unroll
-      for (int k = 0; k < EPT; ++k) {
-        const int e8 = (tid >> 7) + k * (C::EXP_THREADS / 128);
-        const uint32_t f = fh[k];
-        const uint32_t vw[4] = {v[k].x, v[k].y, v[k].z, v[k].w};   // value pair of group g
-        uint8_t* tile = sA + b * C::A_BYTES + (e8 >> 2) * (C::A_BYTES / 2);
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {                     // dense chunk: groups 2c, 2c + 1 (8 channels)
-          uint32_t w[4];
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int g = 2 * c + h;
-            const uint32_t fld = (f >> (4 * g)) & 0xFu;
-            const uint32_t p0 = fld & 3u, p1 = fld >> 2;
-            // the two kept values at their positions p of the group: word p / 2, half p % 2
-            const uint32_t a = (vw[g] & 0xFFFFu) << (16 * (p0 & 1u)), bv = (vw[g] >> 16) << (16 * (p1 & 1u));
-            w[2 * h] = (p0 < 2 ? a : 0u) | (p1 < 2 ? bv : 0u);
-            w[2 * h + 1] = (p0 >= 2 ? a : 0u) | (p1 >= 2 ? bv : 0u);
-          }
-          st_sw128(tile, r, (e8 & 3) * 2 + c, make_uint4(w[0], w[1], w[2], w[3]));
-        }
-      }
-      fence_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(aready(b));
-    }
-    // epilogue: four warps, one per TMEM lane quadrant (warp w reads lanes 32 (w % 4) ..)
     if (warp < 4) {
+      // metadata of stage j -> TMEM columns TMEM_META + 8 (4 (j % NM) + k), lanes of this
+      // warp's quadrant: lane L = 32 warp + lane, rows r0 = 16 (L / 16) + L % 8 and r0 + 8
+      const int L = warp * 32 + lane;
+      const int r0 = (L & ~15) + (L & 7), r1 = r0 + 8;
+      const bool hi = (L & 8) != 0;                     // channels 16-31 of each 32
+      const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16) + C::TMEM_META;
+      for (int j = 0; j < nst; ++j) {
+        const int q = j % C::STG, m = j % C::NM;
+        ok = ok && warp_all(mbar_wait(full(q), (uint32_t)(j / C::STG) & 1u, abort_flag, 315));
+        if (j >= C::NM)
+          ok = ok && warp_all(mbar_wait(mfree(m), (uint32_t)((j - C::NM) / C::NM) & 1u, abort_flag, 316));
+        if (!ok) break;
+        tc_fence_after();
+        const uint4 w0 = *reinterpret_cast<const uint4*>(sM + q * C::M_BYTES + r0 * 16);
+        const uint4 w1 = *reinterpret_cast<const uint4*>(sM + q * C::M_BYTES + r1 * 16);
+        auto pick = [&](uint32_t a, uint32_t b) {
+          return hi ? ((a >> 16) | (b & 0xFFFF0000u)) : ((a & 0xFFFFu) | (b << 16));
+        };
+        tmem_st1(taddr + 8 * (m * 4 + 0), pick(w0.x, w1.x));
+        tmem_st1(taddr + 8 * (m * 4 + 1), pick(w0.y, w1.y));
+        tmem_st1(taddr + 8 * (m * 4 + 2), pick(w0.z, w1.z));
+        tmem_st1(taddr + 8 * (m * 4 + 3), pick(w0.w, w1.w));
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(mready(m));
+      }
+      // epilogue: one warp per TMEM lane quadrant (warp w reads lanes 32 w ..)
       const bool got = ok && nst > 0 && warp_all(mbar_wait(fin, 0, abort_flag, 313));
       tc_fence_after();
       uint32_t acc[16];
@@ -284,7 +291,7 @@ sp24_tc_kernel(const __grid_constant__ CUtensorMap tmV, const __grid_constant__ 
   }
   if (warp == C::MMA_WARP) {
     tc_fence_after();
-    tmem_dealloc(tmem, 32);
+    tmem_dealloc(tmem, C::TMEM_COLS);
   }
 }
 

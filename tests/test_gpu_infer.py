@@ -120,8 +120,8 @@ def test_sparse24_mm_matches_the_oracle(gpu_lib, dtype, T, fused):
 @pytest.mark.parametrize("T", [1, 5, 16])
 def test_sparse24_mm_cuda_core_path(gpu_lib, T):
     """bf16 with C_in not a multiple of 256 takes the CUDA-core kernel at every
-    token count (the other cases cover it below 8 tokens and the tensor-core
-    kernel from 8 on)."""
+    token count (the other cases cover it at one token and the sparse
+    tensor-core kernel from 2 tokens on)."""
     cout, cin, B = 72, 1120, 32
     W, perm, Wp, M = _case(cout, cin, B, "bf16", seed=40 + T)
     vals, meta, pd = _pack_gpu(W, perm, M, B, "bf16")
