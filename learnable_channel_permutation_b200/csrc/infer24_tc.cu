@@ -318,11 +318,16 @@ lcp_status tc_error_infer(int* site, int reset) { return read_tc_error(site, res
 // Splits of C_in for the tensor-core product (0: the shape is not supported):
 // S in {1, 2, 4} with C_in / S a multiple of 256 and at most 2048, as many as
 // keep the grid (S x row tiles) within one wave of the SMs.
+// most C_in splits of a row tile (tuning: 1, 2 or 4)
+#ifndef LCP_SP24_MAX_SPLITS
+#define LCP_SP24_MAX_SPLITS 4
+#endif
+
 int sparse24_tc_splits(int cout, int cin) {
   if (cin % 256) return 0;
   const int tiles = cdiv(cout, 128);
   int best = 0;
-  for (int s = 1; s <= 4; s *= 2) {
+  for (int s = 1; s <= LCP_SP24_MAX_SPLITS; s *= 2) {
     if (cin % (256 * s) || cin / s > StCfg::MAX_KR) continue;
     if (best == 0) best = s;                            // the fewest splits that fit
     else if (tiles * s <= num_sms()) best = s;          // more, while one wave holds them
