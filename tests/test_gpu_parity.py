@@ -41,6 +41,35 @@ def test_sinkhorn_fwd_matches_oracle(B, iters, tau, scale):
     assert np.max(np.abs(P.cpu().numpy().sum(axis=1) - 1)) < 1e-5
 
 
+def test_sinkhorn_model_scale_kernels_match_oracle():
+    """B = 64 launches of at least 1024 blocks run the forward pass one warp a block and the
+    reverse pass two warps a block: 1100 blocks, every fifth one peaked enough (range of Z_0
+    above 64) for the log-domain fallback, the rest in the linear domain; reverse with two
+    dP partials."""
+    nb, B, iters, tau, splits = 1100, 64, 5, 0.1, 2
+    rng = np.random.default_rng(64064)
+    scale = np.where(np.arange(nb) % 5 == 0, 1.5, 0.01)[:, None, None]
+    L = (rng.standard_normal((nb, B, B)) * scale).astype(np.float32)
+    dP = rng.standard_normal((splits, nb, B, B)).astype(np.float32)
+    Ld = torch.from_numpy(L).cuda()
+    P = torch.empty_like(Ld)
+    ck = torch.empty(nb, iters, 2, B, device="cuda")
+    dL = torch.empty_like(Ld)
+    b.sinkhorn_fwd(Ld, P, ck, tau, iters)
+    b.sinkhorn_bwd(Ld, ck, torch.from_numpy(dP).cuda(), dL, tau, iters)
+    torch.cuda.synchronize()
+    Pref, tr = O.sinkhorn(L, tau, iters)
+    ref = O.sinkhorn_backward(tr, Pref, dP.astype(np.float64).sum(axis=0), tau)
+    Pg, dLg = P.cpu().numpy(), dL.cpu().numpy()
+    z = L / tau
+    peaked = (z.max(axis=(1, 2)) - z.min(axis=(1, 2))) > 64
+    assert 0 < peaked.sum() < nb                      # both arithmetics are exercised
+    for sel in (peaked, ~peaked):
+        assert H.relerr(Pg[sel], Pref[sel]) <= H.TOL_P
+        assert H.relerr(dLg[sel], ref[sel]) <= 1e-5
+    assert np.max(np.abs(Pg.sum(axis=1) - 1)) < 1e-5
+
+
 @pytest.mark.parametrize("B", [32, 64, 128, 256])
 @pytest.mark.parametrize("splits", [1, 3])
 def test_sinkhorn_bwd_matches_oracle(B, splits):
