@@ -562,226 +562,316 @@ permute_mask_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
   }
 }
 
-// ----------------------------------------- permute + mask, row-streamed ---
-// For BC <= 128 the P images of the CTA's channel tile stay resident and the
-// CTA walks the row tiles rt = blockIdx.y, blockIdx.y + gridDim.y, ...; the W
-// tile of the next-but-one row tile streams in (two buffers) while the current
-// one is processed, so that HBM reads stay in flight across the whole launch.
-template <int BC> struct Pm2Cfg {
-  static constexpr int NCH = BC / 64;
-  static constexpr int W_BYTES = BC * 256;        // 128 rows x BC
-  static constexpr int PT_BYTES = BC * BC * 2;    // every chunk of one transposed image
-  static constexpr int PH_BYTES = BC * BC * 2;
-  static constexpr int A_BYTES = 16384;
-  static constexpr uint32_t TMEM_COLS = (64 + BC <= 128) ? 128u : 256u;
-  static constexpr int SMEM = 2 * W_BYTES + 2 * PT_BYTES + PH_BYTES + A_BYTES + 1024 + 128;
-  static constexpr int CTAS_PER_SM = BC == 64 ? 3 : 1;
+// ------------------------------- permute + mask, warp-specialised, B = 128 ---
+// The B <= 64 kernel's scheme for 128-channel blocks.  Tile k = (channel tile t
+// of 128 channels, row tile rt); each of its two 64-column chunks c needs all
+// 128 input channels of the block:
+//   W'_{k,c} = W_k [P_hi | P_lo]_{rows of chunk c}   N = 128 (the two transposed
+//              images of the chunk stacked), K = 128 (two 64-channel W halves)
+//   At_k     = A_k P_hi^T                              N = 128, K = 128
+// Shared memory: a 2-stage ring of W tiles (128 rows x 128 channels, 32 KB),
+// one slot with the channel tile's images (Pt_hi / Pt_lo pairs per chunk and
+// K half, 4 x 16 KB, and P_hi, 2 x 16 KB) reloaded when the run moves to the
+// next channel tile, and two A buffers (32 KB): 224 KB.  TMEM: two W' chunk
+// buffers (hi | lo, 128 columns) and two At buffers (128 columns).  The copy-out
+// warps write At straight from registers (16-byte stores).  Roles as in the
+// B <= 64 kernel: warp 0 TMA producer; warp 1 issues W' of every chunk, warps
+// 2 and 3 At of the even / odd tiles; warps 4..11 mask warps (two per TMEM lane
+// quadrant, 32 columns of the chunk each); warps 12..15 copy-out.
+struct Pw128Cfg {
+  static constexpr int STAGES = 2;
+  static constexpr int W_BYTES = 32768;                 // 128 rows x 128 bf16 (two 16 KB halves)
+  static constexpr int SLOT = 6 * 16384;                // Pt pairs [c][kc] (hi 8 KB | lo 8 KB), then P_hi [kj]
+  static constexpr int A_BYTES = 32768;                 // two 16 KB K halves
+  static constexpr int ISSUERS = 3, MASK_WARPS = 8, COPY_WARPS = 4;
+  static constexpr int MASK0 = 1 + ISSUERS, COPY0 = MASK0 + MASK_WARPS;
+  static constexpr int THREADS = 32 * (COPY0 + COPY_WARPS);
+  static constexpr int NBAR = 2 * STAGES + 2 + 2 * 2 + 2 * 2 + 2 * 2 + ISSUERS;
+  static constexpr int SMEM = STAGES * W_BYTES + SLOT + 2 * A_BYTES + NBAR * 8 + 16 + 1024;
+  static_assert(SMEM <= 232448, "shared memory budget");
 };
 
-template <int BC, int MGROUP>
-__global__ void __launch_bounds__(128)
-permute_mask_tc2_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmPth,
-                        const __grid_constant__ CUtensorMap tmPtl, const __grid_constant__ CUtensorMap tmPh,
-                        uint32_t* __restrict__ mask, __nv_bfloat16* __restrict__ At,
-                        float* __restrict__ Wp_out, int cout, int cin, int n) {
-  using C = Pm2Cfg<BC>;
-  constexpr int NCH = C::NCH;
+template <int MGROUP>
+__global__ void __launch_bounds__(Pw128Cfg::THREADS, 1)
+permute_mask_ws128_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmPth,
+                          const __grid_constant__ CUtensorMap tmPtl, const __grid_constant__ CUtensorMap tmPh,
+                          uint32_t* __restrict__ mask, __nv_bfloat16* __restrict__ At, float* __restrict__ Wp_out,
+                          int cout, int cin, int n) {
+  using C = Pw128Cfg;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
-  uint8_t* sW0 = smem;
-  uint8_t* sPth = sW0 + 2 * C::W_BYTES;
-  uint8_t* sPtl = sPth + C::PT_BYTES;
-  uint8_t* sPh = sPtl + C::PT_BYTES;
-  uint8_t* sA = sPh + C::PH_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sA + C::A_BYTES);
-  uint32_t* holder = reinterpret_cast<uint32_t*>(bars + 5);
+  uint8_t* sStage = smem;
+  uint8_t* sSlot = sStage + C::STAGES * C::W_BYTES;
+  uint8_t* sA = sSlot + C::SLOT;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sA + 2 * C::A_BYTES);
+  uint32_t* holder = reinterpret_cast<uint32_t*>(bars + C::NBAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(holder + 1);
-  const uint32_t bar_full0 = smem_u32(bars + 0);          // +8 for buffer 1
-  const uint32_t bar_mma1 = smem_u32(bars + 2), bar_mma2 = smem_u32(bars + 3), bar_drain = smem_u32(bars + 4);
+  auto bar = [&](int i) { return smem_u32(bars + i); };
+  constexpr int S = C::STAGES;
+  constexpr int FULL = 0, EMPTY = S, PREADY = 2 * S, PFREE = PREADY + 1, WF = PFREE + 1, TMW = WF + 2,
+                ATF = TMW + 2, TMA = ATF + 2, AF = TMA + 2, AE = AF + 2, DRAIN = AE + 2;
+  static_assert(DRAIN + C::ISSUERS == C::NBAR, "barrier count");
+  constexpr uint32_t TM_AT = 256;   // At buffers at columns 256 + 128 b
 
-  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-  const int t = blockIdx.x, col0 = t * BC;
-  const int nrt = cdiv(cout, 128), first = blockIdx.y, step = gridDim.y;
-  const int nloc = first < nrt ? cdiv(nrt - first, step) : 0;
-  if (tid == 0) {
-    mbar_init(bar_full0, 1);
-    mbar_init(bar_full0 + 8, 1);
-    mbar_init(bar_mma1, 1);
-    mbar_init(bar_mma2, 1);
-    mbar_init(bar_drain, 1);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int nrt = cdiv(cout, 128), ntc = cin / 128;
+  const int total = nrt * ntc;
+  const int first = (int)((long long)blockIdx.x * total / gridDim.x);
+  const int last = (int)((long long)(blockIdx.x + 1) * total / gridDim.x);
+  const int nloc = last - first;
+  const int t_first = first / nrt;
+  const int nt = nloc > 0 ? (last - 1) / nrt - t_first + 1 : 0;
+  const int words = cin / 32;
+  auto jt_of = [&](int k) { return (first + k) / nrt - t_first; };
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) { mbar_init(bar(FULL + i), 1); mbar_init(bar(EMPTY + i), 1); }
+    mbar_init(bar(PREADY), 1);
+    mbar_init(bar(PFREE), 3);   // the W' issuer and both At issuers
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(WF + i), 1);
+      mbar_init(bar(TMW + i), C::MASK_WARPS);
+      mbar_init(bar(ATF + i), 1);
+      mbar_init(bar(TMA + i), C::COPY_WARPS);
+      mbar_init(bar(AF + i), C::MASK_WARPS);
+      mbar_init(bar(AE + i), 1);
+    }
+    for (int i = 0; i < C::ISSUERS; ++i) mbar_init(bar(DRAIN + i), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0) tmem_alloc(smem_u32(holder), C::TMEM_COLS);
+  if (warp == 1) tmem_alloc(smem_u32(holder), 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *holder;
-  pdl_wait();
-  pdl_trigger();
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-  const int row = warp * 32 + lane;
-  const int words = cin / 32;
-  constexpr uint32_t idesc1 = idesc_bf16(128, 64, false, false);
-  constexpr uint32_t idesc2 = idesc_bf16(128, BC, false, false);
-
-  auto load_w = [&](int k, int b) {   // thread 0: W rows of local tile k into buffer b
-    const int r0 = (first + k * step) * 128;
-    for (int kc = 0; kc < NCH; ++kc)
-      tma_load_2d(smem_u32(sW0 + b * C::W_BYTES + kc * 16384), &tmW, bar_full0 + 8 * b, col0 + kc * 64, r0);
-  };
-  int issued = 0;   // thread 0: local tiles whose W load has been issued
-  if (tid == 0 && nloc > 0) {
-    mbar_expect_tx(bar_full0, C::W_BYTES + 2 * C::PT_BYTES + C::PH_BYTES);
-    for (int c = 0; c < NCH; ++c) {
-      for (int kc = 0; kc < NCH; ++kc) {
-        tma_load_2d(smem_u32(sPth + (c * NCH + kc) * 8192), &tmPth, bar_full0, kc * 64, col0 + c * 64);
-        tma_load_2d(smem_u32(sPtl + (c * NCH + kc) * 8192), &tmPtl, bar_full0, kc * 64, col0 + c * 64);
-      }
-      tma_load_2d(smem_u32(sPh + c * BC * 128), &tmPh, bar_full0, c * 64, col0);
-    }
-    load_w(0, 0);
-    issued = 1;
-    if (nloc > 1) {
-      mbar_expect_tx(bar_full0 + 8, C::W_BYTES);
-      load_w(1, 1);
-      issued = 2;
-    }
+  if (warp != 0) {
+    pdl_wait();
+    pdl_trigger();
   }
+  auto wait_all = [&](int b, uint32_t parity, int site) {
+    return __all_sync(0xffffffffu, mbar_wait(bar(b), parity, abort_flag, site));
+  };
 
-  bool ok = true;
-  uint32_t n1 = 0, n2 = 0;   // completed phases of bar_mma1 / bar_mma2
-  int consumed = 0;          // thread 0: local tiles whose W load was seen complete
-  for (int k = 0; k < nloc && ok; ++k) {
-    const int b = k & 1;
-    const int grow = (first + k * step) * 128 + row;
-    const uint8_t* sW = sW0 + b * C::W_BYTES;
-    if (tid == 0) {
-      if (mbar_wait(bar_full0 + 8 * b, (uint32_t)(k >> 1) & 1u, abort_flag, 41)) consumed = k + 1;
-      else *abort_flag = 1;
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t issued = 0, par = 0;
+      int img_next = 0;
+      bool img_issued = false;
+      bool ok = true;
+      auto absent = [&](int jt) -> int {   // At issuers with no tile in channel tile jt
+        const int k0 = max(0, (t_first + jt) * nrt - first);
+        const int k1 = min(nloc - 1, (t_first + jt + 1) * nrt - 1 - first);
+        return k1 == k0 ? 1 : 0;
+      };
+      // images of channel tile jt into the slot once every product of jt - 1 has completed
+      auto images_upto = [&](int jt) -> bool {
+        for (; img_next <= jt && img_next < nt; ++img_next) {
+          if (!mbar_wait(bar(PFREE), ((uint32_t)img_next & 1u) ^ 1u, abort_flag, 160)) return false;
+          const int t = t_first + img_next;
+          const uint32_t d = smem_u32(sSlot);
+          mbar_expect_tx(bar(PREADY), C::SLOT);
+          for (int c = 0; c < 2; ++c)
+            for (int kc = 0; kc < 2; ++kc) {
+              const uint32_t pair = d + (c * 2 + kc) * 16384;
+              tma_load_2d(pair, &tmPth, bar(PREADY), kc * 64, t * 128 + c * 64);
+              tma_load_2d(pair + 8192, &tmPtl, bar(PREADY), kc * 64, t * 128 + c * 64);
+            }
+          for (int kj = 0; kj < 2; ++kj) tma_load_2d(d + (4 + kj) * 16384, &tmPh, bar(PREADY), kj * 64, t * 128);
+          img_issued = true;
+          for (int a = absent(img_next); a > 0; --a) mbar_arrive(bar(PFREE));
+        }
+        return true;
+      };
+      auto load_w = [&](int k, int st) {
+        const int idx = first + k, t = idx / nrt, rt = idx % nrt;
+        mbar_expect_tx(bar(FULL + st), C::W_BYTES);
+        for (int kc = 0; kc < 2; ++kc)
+          tma_load_2d(smem_u32(sStage + st * C::W_BYTES + kc * 16384), &tmW, bar(FULL + st), t * 128 + kc * 64,
+                      rt * 128);
+      };
+      const int pre = nloc < S ? nloc : S;
+      for (int k = 0; k < pre; ++k) {
+        load_w(k, k);
+        issued |= 1u << k;
+      }
+      pdl_wait();
+      pdl_trigger();
+      if (nloc > 0) ok = images_upto(0);
+      for (int k = pre; k < nloc && ok; ++k) {
+        const int st = k % S;
+        const uint32_t use = (uint32_t)(k / S) & 1u;
+        if (!mbar_wait(bar(EMPTY + st), use ^ 1u, abort_flag, 161)) break;
+        if (!images_upto(jt_of(k))) break;
+        load_w(k, st);
+        issued |= 1u << st;
+        par = (par & ~(1u << st)) | (use << st);
+      }
+      for (int st = 0; st < S; ++st)
+        if (issued & (1u << st)) mbar_wait_drain(bar(FULL + st), (par >> st) & 1u, 162);
+      if (img_issued) mbar_wait_drain(bar(PREADY), (uint32_t)(img_next - 1) & 1u, 163);
     }
-    for (int c = 0; c < NCH; ++c) {
-      if (tid == 0 && !*abort_flag) {
-        tc_fence_after();
-#pragma unroll 1
-        for (int pass = 0; pass < 2; ++pass) {
-          const uint8_t* sB = (pass ? sPtl : sPth) + c * NCH * 8192;
-          for (int kc = 0; kc < NCH; ++kc)
+    __syncwarp();
+  } else if (warp < C::MASK0) {
+    const int role = warp == 1 ? 0 : 1;
+    const int k_first = warp == 1 ? 0 : warp - 2, k_step = warp == 1 ? 1 : 2;
+    if (lane == 0) {
+      int cur_jt = -1;
+      const uint32_t slot = smem_u32(sSlot);
+      for (int k = k_first; k < nloc; k += k_step) {
+        const int jt = jt_of(k);
+        if (jt != cur_jt) {
+          if (cur_jt >= 0) mma_commit(bar(PFREE));
+          cur_jt = jt;
+        }
+        if (!mbar_wait(bar(PREADY), (uint32_t)jt & 1u, abort_flag, 158)) break;
+        bool ok = true;
+        if (role == 0) {
+          const int st = k % S;
+          if (!mbar_wait(bar(FULL + st), (uint32_t)(k / S) & 1u, abort_flag, 163)) break;
+          constexpr uint32_t idesc = idesc_bf16(128, 128, false, false);
+          const uint32_t sw = smem_u32(sStage + st * C::W_BYTES);
+          for (int c = 0; c < 2 && ok; ++c) {
+            const int q = 2 * k + c, b = q & 1;
+            if (!mbar_wait(bar(TMW + b), ((uint32_t)(q >> 1) & 1u) ^ 1u, abort_flag, 164)) { ok = false; break; }
+            tc_fence_after();
+#pragma unroll
+            for (int kc = 0; kc < 2; ++kc)
+#pragma unroll
+              for (int k16 = 0; k16 < 4; ++k16)
+                mma_bf16(tmem + b * 128, sdesc(sw + kc * 16384 + k16 * 32, 16, 1024),
+                         sdesc(slot + (c * 2 + kc) * 16384 + k16 * 32, 16, 1024), idesc, (kc | k16) != 0);
+            mma_commit(bar(WF + b));
+          }
+          if (!ok) break;
+          mma_commit(bar(EMPTY + st));
+        } else {
+          const int a = k & 1;
+          if (!mbar_wait(bar(AF + a), (uint32_t)(k >> 1) & 1u, abort_flag, 165)) break;
+          if (!mbar_wait(bar(TMA + a), ((uint32_t)(k >> 1) & 1u) ^ 1u, abort_flag, 169)) break;
+          tc_fence_after();
+          constexpr uint32_t idesc = idesc_bf16(128, 128, false, false);
+          const uint32_t sa = smem_u32(sA + a * C::A_BYTES);
+#pragma unroll
+          for (int kj = 0; kj < 2; ++kj)
 #pragma unroll
             for (int k16 = 0; k16 < 4; ++k16)
-              mma_bf16(tmem, sdesc(smem_u32(sW + kc * 16384) + k16 * 32, 16, 1024),
-                       sdesc(smem_u32(sB + kc * 8192) + k16 * 32, 16, 1024), idesc1, (pass | kc | k16) != 0);
+              mma_bf16(tmem + TM_AT + a * 128, sdesc(sa + kj * 16384 + k16 * 32, 16, 1024),
+                       sdesc(slot + (4 + kj) * 16384 + k16 * 32, 16, 1024), idesc, (kj | k16) != 0);
+          mma_commit(bar(ATF + a));
+          mma_commit(bar(AE + a));
         }
-        mma_commit(bar_mma1);
       }
-      ok = __syncthreads_and(mbar_wait(bar_mma1, n1 & 1u, abort_flag, 42));
-      ++n1;
-      if (!ok) break;
+      if (cur_jt >= 0) mma_commit(bar(PFREE));
+      mma_commit(bar(DRAIN + warp - 1));
+      mbar_wait_drain(bar(DRAIN + warp - 1), 0, 166);
+    }
+    __syncwarp();
+  } else if (warp < C::COPY0) {
+    // mask warps: chunk q = 2 k + c of tile k.  W' of chunk q + 1 is waited for and loaded
+    // only once chunk q is finished (its A half written, the A buffer released after chunk 1):
+    // with one image slot, W' of the first chunk of the next channel tile waits for the images,
+    // the images for every At product of this channel tile, and those for this tile's A.
+    constexpr int NV = 32;
+    const int e = warp - C::MASK0, qd = warp & 3, h = e >> 2;
+    const int row = qd * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
+    const int nq = 2 * nloc;
+    uint32_t hi[NV], lo[NV];
+    bool have = nq > 0 && wait_all(WF + 0, 0u, 167);
+    if (have) {
       tc_fence_after();
-      uint32_t v0[32], v1[32];
-      tmem_ld32(tmem + lane_off + 0, v0);
-      tmem_ld32(tmem + lane_off + 32, v1);
+      tmem_ld32(tmem + lane_off + h * NV, hi);
+      tmem_ld32(tmem + lane_off + 64 + h * NV, lo);
+    }
+    for (int q = 0; q < nq && have; ++q) {
+      const int k = q >> 1, c = q & 1, b = q & 1;
       tmem_ld_wait();
-      const uint32_t w0 = MGROUP == 4 ? nm4_keep<32>(v0, n) : nm_word<MGROUP>(v0, n);
-    const uint32_t w1 = MGROUP == 4 ? nm4_keep<32>(v1, n) : nm_word<MGROUP>(v1, n);
-      if (grow < cout) {
-        const int wi = (col0 + c * 64) / 32;
-        *reinterpret_cast<uint2*>(mask + (size_t)grow * words + wi) = make_uint2(w0, w1);
-        if (Wp_out) {
-          float4* o = reinterpret_cast<float4*>(Wp_out + (size_t)grow * cin + col0 + c * 64);
+      uint32_t v[NV];
 #pragma unroll
-          for (int q = 0; q < 8; ++q)
-            o[q] = make_float4(__uint_as_float(v0[4 * q]), __uint_as_float(v0[4 * q + 1]),
-                               __uint_as_float(v0[4 * q + 2]), __uint_as_float(v0[4 * q + 3]));
+      for (int x = 0; x < NV; ++x) v[x] = __float_as_uint(__uint_as_float(hi[x]) + __uint_as_float(lo[x]));
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(TMW + b));
+      const int idx = first + k, t = idx / nrt, rt = idx % nrt;
+      const int grow = rt * 128 + row;
+      const int col = t * 128 + c * 64 + h * NV;
+      if (Wp_out && grow < cout) {
+        float4* o = reinterpret_cast<float4*>(Wp_out + (size_t)grow * cin + col);
 #pragma unroll
-          for (int q = 0; q < 8; ++q)
-            o[8 + q] = make_float4(__uint_as_float(v1[4 * q]), __uint_as_float(v1[4 * q + 1]),
-                                   __uint_as_float(v1[4 * q + 2]), __uint_as_float(v1[4 * q + 3]));
+        for (int qq = 0; qq < NV / 4; ++qq)
+          o[qq] = make_float4(__uint_as_float(v[4 * qq]), __uint_as_float(v[4 * qq + 1]),
+                              __uint_as_float(v[4 * qq + 2]), __uint_as_float(v[4 * qq + 3]));
+      }
+      const uint32_t w = MGROUP == 4 ? nm4_keep<NV>(v, n) : nm_bits<MGROUP, NV>(v, n);
+      if (grow < cout) mask[(size_t)grow * words + col / 32] = w;
+#pragma unroll
+      for (int x = 0; x < NV; ++x) v[x] = ((w >> x) & 1u) ? v[x] : 0u;
+      // A buffer k & 1 was last read by At of tile k - 2
+      if (c == 0 && !wait_all(AE + (k & 1), ((uint32_t)(k >> 1) & 1u) ^ 1u, 157)) break;
+      uint8_t* sa = sA + (k & 1) * C::A_BYTES + c * 16384;
+#pragma unroll
+      for (int c8 = 0; c8 < NV / 8; ++c8)
+        st_sw128(sa, row, h * (NV / 8) + c8,
+                 make_uint4(pack_bf16x2(__uint_as_float(v[8 * c8 + 0]), __uint_as_float(v[8 * c8 + 1])),
+                            pack_bf16x2(__uint_as_float(v[8 * c8 + 2]), __uint_as_float(v[8 * c8 + 3])),
+                            pack_bf16x2(__uint_as_float(v[8 * c8 + 4]), __uint_as_float(v[8 * c8 + 5])),
+                            pack_bf16x2(__uint_as_float(v[8 * c8 + 6]), __uint_as_float(v[8 * c8 + 7]))));
+      if (c == 1) {
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(AF + (k & 1)));
+      }
+      have = false;
+      if (q + 1 < nq) {
+        const int bn = (q + 1) & 1;
+        if (!wait_all(WF + bn, (uint32_t)((q + 1) >> 1) & 1u, 167)) break;
+        tc_fence_after();
+        tmem_ld32(tmem + lane_off + bn * 128 + h * NV, hi);
+        tmem_ld32(tmem + lane_off + bn * 128 + 64 + h * NV, lo);
+        have = true;
+      }
+    }
+    tmem_ld_wait();
+  } else {
+    // copy-out warps: At of tile k (128 columns) -> 16-byte stores of the row
+    const int qd = warp & 3;
+    const int row = qd * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
+    for (int k = 0; k < nloc; ++k) {
+      const int a = k & 1;
+      if (!wait_all(ATF + a, (uint32_t)(k >> 1) & 1u, 168)) break;
+      tc_fence_after();
+      const int idx = first + k, t = idx / nrt, rt = idx % nrt;
+      const int grow = rt * 128 + row;
+      uint4* o = reinterpret_cast<uint4*>(At + (size_t)grow * cin + t * 128);
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t u[32];
+        tmem_ld32(tmem + lane_off + TM_AT + a * 128 + cc * 32, u);
+        tmem_ld_wait();
+        if (cc == 3) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(TMA + a));   // the buffer may take At of tile k + 2
+        }
+        if (grow < cout) {
+#pragma unroll
+          for (int c8 = 0; c8 < 4; ++c8)
+            o[cc * 4 + c8] =
+                make_uint4(pack_bf16x2(__uint_as_float(u[8 * c8 + 0]), __uint_as_float(u[8 * c8 + 1])),
+                           pack_bf16x2(__uint_as_float(u[8 * c8 + 2]), __uint_as_float(u[8 * c8 + 3])),
+                           pack_bf16x2(__uint_as_float(u[8 * c8 + 4]), __uint_as_float(u[8 * c8 + 5])),
+                           pack_bf16x2(__uint_as_float(u[8 * c8 + 6]), __uint_as_float(u[8 * c8 + 7])));
         }
       }
-#pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
-        const uint32_t* v = ch < 4 ? v0 : v1;
-        const uint32_t w = ch < 4 ? w0 : w1;
-        const int b0 = (ch & 3) * 8;
-        float f[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) f[e] = ((w >> (b0 + e)) & 1u) ? __uint_as_float(v[b0 + e]) : 0.f;
-        st_sw128(sA, row, ch, make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
-                                         pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7])));
-      }
-      fence_async_smem();
-      tc_fence_before();
-      __syncthreads();
-      if (tid == 0) {
-        tc_fence_after();
-#pragma unroll
-        for (int k16 = 0; k16 < 4; ++k16)
-          mma_bf16(tmem + 64, sdesc(smem_u32(sA) + k16 * 32, 16, 1024),
-                   sdesc(smem_u32(sPh + c * BC * 128) + k16 * 32, 16, 1024), idesc2, (c | k16) != 0);
-        mma_commit(bar_mma2);
-      }
     }
-    if (!ok) break;
-    n2 += NCH;
-    // the W buffer of this tile is free once its MMAs are done: stream tile k + 2 into it
-    if (tid == 0 && k + 2 < nloc) {
-      if (mbar_wait(bar_mma2, (n2 - 1) & 1u, abort_flag, 43)) {
-        mbar_expect_tx(bar_full0 + 8 * b, C::W_BYTES);
-        load_w(k + 2, b);
-        issued = k + 3;
-      } else {
-        *abort_flag = 1;
-      }
-    }
-    ok = __syncthreads_and(mbar_wait(bar_mma2, (n2 - 1) & 1u, abort_flag, 44));
-    if (!ok) break;
-    tc_fence_after();
-#pragma unroll 1
-    for (int cc = 0; cc < BC / 32; ++cc) {
-      uint32_t r[32];
-      tmem_ld32(tmem + lane_off + 64 + cc * 32, r);
-      tmem_ld_wait();
-      if (grow < cout) {
-        uint4* o = reinterpret_cast<uint4*>(At + (size_t)grow * cin + col0 + cc * 32);
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-          o[q] = make_uint4(pack_bf16x2(__uint_as_float(r[8 * q]), __uint_as_float(r[8 * q + 1])),
-                            pack_bf16x2(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3])),
-                            pack_bf16x2(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5])),
-                            pack_bf16x2(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7])));
-      }
-    }
-    tc_fence_before();
-    __syncthreads();   // the next tile's MMAs overwrite the accumulators just read
-  }
-  if (tid == 0) {
-    for (int kk = consumed; kk < issued; ++kk)
-      mbar_wait_drain(bar_full0 + 8 * (kk & 1), (uint32_t)(kk >> 1) & 1u, 45);
-    mma_commit(bar_drain);
-    mbar_wait_drain(bar_drain, 0, 46);
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, C::TMEM_COLS);
+    tmem_dealloc(tmem, 512);
   }
-}
-
-template <int BC, int MG>
-lcp_status permute_mask2_bc(const CUtensorMap& mW, const CUtensorMap& mPth, const CUtensorMap& mPtl,
-                            const CUtensorMap& mPh, uint32_t* mask, __nv_bfloat16* At, float* Wp, int cout,
-                            int cin, int n, cudaStream_t st) {
-  using C = Pm2Cfg<BC>;
-  auto k = permute_mask_tc2_kernel<BC, MG>;
-  TC_TRY(set_smem(k, C::SMEM, "permute_mask_tc"));
-  const int ntiles = cin / BC, nrt = cdiv(cout, 128);
-  int ry = cdiv(C::CTAS_PER_SM * num_sms(), ntiles);
-  if (ry > nrt) ry = nrt;
-  if (ry < 1) ry = 1;
-  return launch_kernel(k, dim3(ntiles, ry), dim3(128), C::SMEM, st, 1, true, "permute_mask_tc", mW, mPth, mPtl, mPh,
-                       mask, At, Wp, cout, cin, n);
 }
 
 template <int BC, int MG>
@@ -841,11 +931,16 @@ lcp_status launch_permute_mask_tc(const __nv_bfloat16* W, const __nv_bfloat16* i
                          mPh, mAt, mask, Wp_out, cout, cin, n);
   }
   if (given_mask) return fail(LCP_ERR_SHAPE, "permute_mask_tc: a given mask needs B <= 64 (B = %d)", B);
-  if (m == 4) {
-    if (BC == 128) return permute_mask2_bc<128, 4>(mW, mPth, mPtl, mPh, mask, At, Wp_out, cout, cin, n, st);
-    return permute_mask_bc<256, 4>(mW, mPth, mPtl, mPh, mask, At, Wp_out, cout, cin, n, st);
+  if (BC == 128) {
+    using C = Pw128Cfg;
+    auto k = (m == 4) ? permute_mask_ws128_kernel<4> : permute_mask_ws128_kernel<8>;
+    TC_TRY(set_smem(k, C::SMEM, "permute_mask_tc"));
+    const int tiles = cdiv(cout, 128) * (cin / 128);
+    const int grid = tiles < num_sms() ? tiles : num_sms();
+    return launch_kernel(k, dim3(grid), dim3(C::THREADS), C::SMEM, st, 1, true, "permute_mask_tc", mW, mPth, mPtl,
+                         mPh, mask, At, Wp_out, cout, cin, n);
   }
-  if (BC == 128) return permute_mask2_bc<128, 8>(mW, mPth, mPtl, mPh, mask, At, Wp_out, cout, cin, n, st);
+  if (m == 4) return permute_mask_bc<256, 4>(mW, mPth, mPtl, mPh, mask, At, Wp_out, cout, cin, n, st);
   return permute_mask_bc<256, 8>(mW, mPth, mPtl, mPh, mask, At, Wp_out, cout, cin, n, st);
 }
 
