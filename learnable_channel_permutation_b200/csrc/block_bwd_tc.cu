@@ -266,6 +266,240 @@ block_bwd_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_consta
   }
 }
 
+// ----------------------------- block backward, warp-specialised, B = 128 ---
+// One CTA per (128-channel block t, row segment), with the B <= 64 kernel's roles: warp 0
+// streams the (dAt, W) tiles of each 128-row chunk (two 64-channel halves each, 64 KB a stage)
+// into a 2-stage ring; warp 1 issues W' = W P_hi and dA = dAt P_hi (M = 128, N = 128, K = 128)
+// into one TMEM buffer once the epilogue has read the previous chunk's; warp 2 issues
+// dP += dAt^T A + W^T dW' (K = 128 rows, MN-major operands) once the epilogue has written A and
+// dW'; warps 3..10 (two per TMEM lane quadrant, 64 columns each) load W' and dA, release the
+// buffer, and write the bf16 operand tiles.  W' is formed from P_hi alone, as for B = 256: the
+// ring, the operand tiles and a second P image would need 256 KB of shared memory.  TMEM: dP at
+// columns 0..127, W' at 128, dA at 256.
+struct Bw128Cfg {
+  static constexpr int STAGES = 2;
+  static constexpr int HALF = 16384;                 // 128 rows x 64 bf16
+  static constexpr int STAGE = 4 * HALF;             // dAt (two channel halves) | W (two channel halves)
+  static constexpr int IMG = 2 * HALF;               // transposed P_hi of the block, two K halves
+  static constexpr int AB = 4 * HALF;                // A (two slot halves) | dW' (two slot halves)
+  static constexpr int CTRL_WARPS = 3, EPI_WARPS = 8;
+  static constexpr int THREADS = 32 * (CTRL_WARPS + EPI_WARPS);
+  static constexpr int NBAR = 2 * STAGES + 8;
+  static constexpr int SMEM = STAGES * STAGE + IMG + AB + NBAR * 8 + 16 + 1024;
+  static_assert(SMEM <= 232448, "shared memory budget");
+};
+
+__global__ void __launch_bounds__(Bw128Cfg::THREADS, 1)
+block_bwd_ws128_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmDAt,
+                       const __grid_constant__ CUtensorMap tmPth, const uint32_t* __restrict__ mask,
+                       float* __restrict__ dP, int cout, int cin, int rows_per_split) {
+  using C = Bw128Cfg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sStage = smem;
+  uint8_t* sPth = sStage + C::STAGES * C::STAGE;
+  uint8_t* sAB = sPth + C::IMG;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sAB + C::AB);
+  uint32_t* holder = reinterpret_cast<uint32_t*>(bars + C::NBAR);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(holder + 1);
+  auto bar = [&](int i) { return smem_u32(bars + i); };
+  constexpr int S = C::STAGES;
+  constexpr int FULL = 0, EMPTY = S, IMG = 2 * S, WD = IMG + 1, TF = WD + 1, ABF = TF + 1, ABE = ABF + 1,
+                DPF = ABE + 1, DRAIN = DPF + 1, DRAIN2 = DRAIN + 1;
+  static_assert(DRAIN2 + 1 == C::NBAR, "barrier count");
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int t = blockIdx.x, sidx = blockIdx.y, col0 = t * 128;
+  const int rbeg = sidx * rows_per_split;
+  const int rend = min(cout, rbeg + rows_per_split);
+  const int nchunk = cdiv(rend - rbeg, 128);
+  const int words = cin / 32;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) { mbar_init(bar(FULL + i), 1); mbar_init(bar(EMPTY + i), 1); }
+    mbar_init(bar(IMG), 1);
+    mbar_init(bar(WD), 1);
+    mbar_init(bar(TF), C::EPI_WARPS);
+    mbar_init(bar(ABF), C::EPI_WARPS);
+    mbar_init(bar(ABE), 1);
+    mbar_init(bar(DPF), 1);
+    mbar_init(bar(DRAIN), 1);
+    mbar_init(bar(DRAIN2), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(smem_u32(holder), 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *holder;
+  pdl_wait();
+  pdl_trigger();
+  const uint32_t tDP = tmem, tW = tmem + 128, tDA = tmem + 256;
+  auto wait_all = [&](int b, uint32_t parity, int site) {
+    return __all_sync(0xffffffffu, mbar_wait(bar(b), parity, abort_flag, site));
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      if (nchunk > 0) {
+        mbar_expect_tx(bar(IMG), C::IMG);
+        for (int kc = 0; kc < 2; ++kc) tma_load_2d(smem_u32(sPth + kc * C::HALF), &tmPth, bar(IMG), kc * 64, col0);
+      }
+      uint32_t issued = 0, par = 0;
+      for (int c = 0; c < nchunk; ++c) {
+        const int st = c % S;
+        const uint32_t use = (uint32_t)(c / S) & 1u;
+        if (!mbar_wait(bar(EMPTY + st), use ^ 1u, abort_flag, 84)) break;
+        uint8_t* sg = sStage + st * C::STAGE;
+        const int r0 = rbeg + c * 128;
+        mbar_expect_tx(bar(FULL + st), C::STAGE);
+        for (int kc = 0; kc < 2; ++kc) {
+          tma_load_2d(smem_u32(sg + kc * C::HALF), &tmDAt, bar(FULL + st), col0 + kc * 64, r0);
+          tma_load_2d(smem_u32(sg + (2 + kc) * C::HALF), &tmW, bar(FULL + st), col0 + kc * 64, r0);
+        }
+        issued |= 1u << st;
+        par = (par & ~(1u << st)) | (use << st);
+      }
+      for (int st = 0; st < S; ++st)
+        if (issued & (1u << st)) mbar_wait_drain(bar(FULL + st), (par >> st) & 1u, 85);
+      if (nchunk > 0) mbar_wait_drain(bar(IMG), 0, 86);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(128, 128, false, false);
+      bool ok = nchunk == 0 || mbar_wait(bar(IMG), 0, abort_flag, 87);
+      for (int c = 0; c < nchunk && ok; ++c) {
+        const int st = c % S;
+        if (!mbar_wait(bar(FULL + st), (uint32_t)(c / S) & 1u, abort_flag, 88)) break;
+        // the epilogue has loaded W' and dA of chunk c - 1
+        if (c >= 1 && !mbar_wait(bar(TF), (uint32_t)(c - 1) & 1u, abort_flag, 89)) break;
+        tc_fence_after();
+        const uint32_t sg = smem_u32(sStage + st * C::STAGE);
+#pragma unroll
+        for (int kc = 0; kc < 2; ++kc)
+#pragma unroll
+          for (int k16 = 0; k16 < 4; ++k16) {
+            const uint64_t pdesc = sdesc(smem_u32(sPth) + kc * C::HALF + k16 * 32, 16, 1024);
+            mma_bf16(tW, sdesc(sg + (2 + kc) * C::HALF + k16 * 32, 16, 1024), pdesc, idesc, (kc | k16) != 0);
+            mma_bf16(tDA, sdesc(sg + kc * C::HALF + k16 * 32, 16, 1024), pdesc, idesc, (kc | k16) != 0);
+          }
+        mma_commit(bar(WD));
+      }
+      mma_commit(bar(DRAIN));
+      mbar_wait_drain(bar(DRAIN), 0, 90);
+    }
+    __syncwarp();
+  } else if (warp == 2) {
+    // dP issuer; its completion also frees the stage (W' and dA of the chunk completed before
+    // the epilogue could start)
+    if (lane == 0) {
+      constexpr uint32_t idesc_dp = idesc_bf16(128, 128, true, true);
+      const uint32_t sab = smem_u32(sAB);
+      for (int c = 0; c < nchunk; ++c) {
+        const int st = c % S;
+        if (!mbar_wait(bar(FULL + st), (uint32_t)(c / S) & 1u, abort_flag, 91)) break;
+        if (!mbar_wait(bar(ABF), (uint32_t)c & 1u, abort_flag, 92)) break;
+        tc_fence_after();
+        const uint32_t sg = smem_u32(sStage + st * C::STAGE);
+        // dAt^T A, then W^T dW' (M = 128 input channels, N = 128 slots, K = 128 rows)
+#pragma unroll
+        for (int k16 = 0; k16 < 8; ++k16)
+          mma_bf16(tDP, sdesc(sg + k16 * 2048, C::HALF, 1024), sdesc(sab + k16 * 2048, C::HALF, 1024), idesc_dp,
+                   (c | k16) != 0);
+#pragma unroll
+        for (int k16 = 0; k16 < 8; ++k16)
+          mma_bf16(tDP, sdesc(sg + 2 * C::HALF + k16 * 2048, C::HALF, 1024),
+                   sdesc(sab + 2 * C::HALF + k16 * 2048, C::HALF, 1024), idesc_dp, true);
+        mma_commit(bar(ABE));
+        mma_commit(bar(EMPTY + st));
+      }
+      mma_commit(bar(DPF));
+      mma_commit(bar(DRAIN2));
+      mbar_wait_drain(bar(DRAIN2), 0, 93);
+    }
+    __syncwarp();
+  } else {
+    const int e = warp - C::CTRL_WARPS, q = warp & 3, h = e >> 2;   // h: 64-column half
+    const int row = q * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    uint8_t* rA = sAB + h * C::HALF;
+    uint8_t* rD = sAB + (2 + h) * C::HALF;
+    // the two mask words of this thread's 64 columns, one chunk ahead
+    auto mask_bits = [&](int c) -> uint2 {
+      const int grow = rbeg + c * 128 + row;
+      if (c >= nchunk || grow >= rend) return make_uint2(0u, 0u);
+      return __ldg(reinterpret_cast<const uint2*>(mask + (size_t)grow * words + col0 / 32 + 2 * h));
+    };
+    // A = M.W' and dW' = M.dA of 32 columns, packed to bf16 pairs at pa / pd [base, base + 16)
+    uint32_t pa[32], pd[32];
+    auto pack32 = [&](const uint32_t (&wv)[32], const uint32_t (&dv)[32], uint32_t bits, int base) {
+#pragma unroll
+      for (int x = 0; x < 16; ++x) {
+        const bool k0 = (bits >> (2 * x)) & 1u, k1 = (bits >> (2 * x + 1)) & 1u;
+        pa[base + x] = pack_bf16x2(k0 ? __uint_as_float(wv[2 * x]) : 0.f, k1 ? __uint_as_float(wv[2 * x + 1]) : 0.f);
+        pd[base + x] = pack_bf16x2(k0 ? __uint_as_float(dv[2 * x]) : 0.f, k1 ? __uint_as_float(dv[2 * x + 1]) : 0.f);
+      }
+    };
+    bool ok = true;
+    uint2 next_bits = mask_bits(0);
+    for (int c = 0; c < nchunk; ++c) {
+      const uint2 bits = next_bits;
+      next_bits = mask_bits(c + 1);
+      ok = wait_all(WD, (uint32_t)c & 1u, 94);
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll
+      for (int g = 0; g < 2; ++g) {
+        uint32_t wv[32], dv[32];
+        tmem_ld32(tW + lane_off + h * 64 + g * 32, wv);
+        tmem_ld32(tDA + lane_off + h * 64 + g * 32, dv);
+        tmem_ld_wait();
+        pack32(wv, dv, g ? bits.y : bits.x, 16 * g);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(TF));
+      // the operand tiles were last read by the dP product of chunk c - 1
+      ok = c < 1 || wait_all(ABE, (uint32_t)(c - 1) & 1u, 95);
+      if (!ok) break;
+#pragma unroll
+      for (int c8 = 0; c8 < 8; ++c8) {
+        st_sw128(rA, row, c8, make_uint4(pa[4 * c8], pa[4 * c8 + 1], pa[4 * c8 + 2], pa[4 * c8 + 3]));
+        st_sw128(rD, row, c8, make_uint4(pd[4 * c8], pd[4 * c8 + 1], pd[4 * c8 + 2], pd[4 * c8 + 3]));
+      }
+      fence_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(ABF));
+    }
+    if (ok) ok = wait_all(DPF, 0, 96);
+    if (ok) {
+      tc_fence_after();
+      // thread `row` holds dP row i = row of block t, columns j = 64 h .. 64 h + 63
+      const int nb = cin / 128;
+      float* o = dP + (size_t)sidx * nb * 128 * 128 + ((size_t)t * 128 + row) * 128 + h * 64;
+#pragma unroll 1
+      for (int cc = 0; cc < 2; ++cc) {
+        uint32_t r[32];
+        tmem_ld32(tDP + lane_off + h * 64 + cc * 32, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int x = 0; x < 8; ++x)
+          reinterpret_cast<float4*>(o + cc * 32)[x] = make_float4(__uint_as_float(r[4 * x]), __uint_as_float(r[4 * x + 1]),
+                                                                  __uint_as_float(r[4 * x + 2]),
+                                                                  __uint_as_float(r[4 * x + 3]));
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 // ------------------------------------------------------- block backward ---
 // One CTA: channel tile t (BC columns) x a segment of C_out rows, in chunks of
 // 128 rows o:
@@ -729,7 +963,10 @@ lcp_status launch_block_bwd_tc(const __nv_bfloat16* W, const __nv_bfloat16* dAt,
     return launch_kernel(k, dim3(cin / 64, splits), dim3(C::THREADS), C::SMEM, st, 1, true, "block_bwd_tc", mW, mD,
                          mPth, mPtl, mask, dP_partials, cout, cin, rows);
   }
-  return block_bwd_bc<128, 128>(mW, mD, mPth, mPtl, mask, dP_partials, splits, rows, cout, cin, st);
+  using C = Bw128Cfg;
+  TC_TRY(set_smem(block_bwd_ws128_kernel, C::SMEM, "block_bwd_tc"));
+  return launch_kernel(block_bwd_ws128_kernel, dim3(cin / 128, splits), dim3(C::THREADS), C::SMEM, st, 1, true,
+                       "block_bwd_tc", mW, mD, mPth, mask, dP_partials, cout, cin, rows);
 }
 
 }  // namespace lcp

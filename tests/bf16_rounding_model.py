@@ -17,7 +17,7 @@ stores or feeds a value in that precision:
 * dAt = G^T X is stored in bf16;
 * the block backward multiplies bf16 operands: dA = dAt P_hi, dW' = M (.) dA
   rounded to bf16, A = M (.) W' in bf16, dP_b = dAt_b^T A_b + W_b^T dW'_b
-  (for B = 256 its W' is W P_hi alone: the kernel has no room for P_lo);
+  (for B = 128 and 256 its W' is W P_hi alone: those kernels have no room for P_lo);
 * the Sinkhorn passes are float32 (modelled exactly).
 
 The model returns the mask it took (from its own float32 W'), so the oracle
@@ -75,7 +75,7 @@ def modelled_step(W, X_tokens, L, tau, iters, n, m, g_from_pair=False):
     dAt = bf(G.T @ X)                                         # [C_out, C_in]
     dWp = bf(np.where(mask, block_right(dAt, P_hi), 0.0))
     nb, B, _ = P.shape
-    Ab = bf(np.where(mask, f32(block_right(W, P_hi)), 0.0)) if B == 256 else A
+    Ab = bf(np.where(mask, f32(block_right(W, P_hi)), 0.0)) if B >= 128 else A
     dP = np.empty_like(P)
     for b in range(nb):
         s = slice(b * B, (b + 1) * B)
