@@ -220,7 +220,7 @@ def main():
                          "Sinkhorn scaling run, one-core oracle)")
     ap.add_argument("--only-extra", default=None,
                     choices=["cached_dense", "hard_step", "score_step", "train", "cublas_same_products", "configs",
-                             "inference_24", "nm_mask", "sinkhorn_scaling"],
+                             "inference_24", "nm_mask", "sinkhorn_scaling", "stream_ref"],
                     help="run this one secondary measurement only")
     ap.add_argument("--scaling-blocks", type=int, default=40 * (6 * 5120 + 13824) // 64,
                     help="64 x 64 blocks of the Sinkhorn scaling run (default: every projection of a "
@@ -469,7 +469,12 @@ def extras(args, b, synth, wl, li, layer, step, flush, pk, dev):
     - sinkhorn_scaling: Sinkhorn forward then reverse over the logits of every
       projection of a 40-layer 13B-shaped model (4 x 5120^2, 2 x 13824 x 5120,
       5120 x 13824 per layer; 27 840 blocks of 64 x 64, 456 MB of float32 L) in one
-      launch each, against the HBM copy bandwidth.
+      launch each, against the HBM copy bandwidth;
+    - stream_ref: a plain device copy (torch) of a bf16 tensor of the layer's
+      weight shape (C_out x C_in read and written: about the bytes the permute
+      and block-backward stages move), L2 flushed before each, and of a ten
+      times larger tensor: what a streaming kernel of that size reaches, the
+      practical ceiling for the memory-bound stages.
     """
     import torch
     out = {}
@@ -598,6 +603,19 @@ def extras(args, b, synth, wl, li, layer, step, flush, pk, dev):
                                 "bytes": by, "shape": list(big), "nm": f"{wl.n}:{wl.m}",
                                 "note": "input larger than L2; no flush needed"}
         del Wp, bits
+
+    if want("stream_ref"):
+        # plain copies of the layer's weight bytes and of ten times as many
+        res = {}
+        for name, rows, fl in (("layer", li.spec.cout, True), ("x10", li.spec.cout * 10, False)):
+            src = torch.empty(rows, li.spec.cin, device=dev, dtype=torch.bfloat16).normal_()
+            dst = torch.empty_like(src)
+            ms = timed(lambda: dst.copy_(src), K, flush_between=fl)
+            by = 2 * src.numel() * 2
+            res[name] = {"ms": ms, "GB/s": by / (ms / 1e3) / 1e9, "frac": by / (ms / 1e3) / 1e9 / pk["hbm_gbs"],
+                         "bytes": by, "shape": [rows, li.spec.cin], "l2": "flushed" if fl else "larger than L2"}
+            del src, dst
+        out["stream_ref"] = res
 
     if want("sinkhorn_scaling"):
         # Sinkhorn scaling run: every projection of a 40-layer 13B-shaped model

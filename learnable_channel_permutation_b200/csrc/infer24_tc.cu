@@ -61,7 +61,6 @@ __device__ __forceinline__ void mma_bf16_sp(uint32_t d, uint64_t a, uint64_t b, 
 __device__ __forceinline__ void tmem_st1(uint32_t taddr, uint32_t v) {
   asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(v) : "memory");
 }
-__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 __device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
   float v;

@@ -196,10 +196,11 @@ permute_mask_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
 // carries W tiles only and a stage is free as soon as W' of its tile is
 // formed, so the loads run STAGES tiles ahead of the tensor core.
 // Per tile k two products:
-//   W'_k = W_k [P_hi | P_lo]   one N = 128 product (the two transposed images sit
-//                              side by side in shared memory): TMEM columns
-//                              [0, 64) W P_hi, [64, 128) W P_lo, summed in float32
-//   At_k = A_k P_hi^T          N = 64, once A = M.W'_k is in shared memory
+//   W'_k = W_k P_hi + W_k P_lo  both N = 64 products accumulate into one TMEM
+//                              buffer (float32), so W' is read with one load
+//   At_k = A_k P_hi^T          N = 64, with A = M.W'_k written by the mask warps
+//                              straight into tensor memory (bf16 pairs, row r in
+//                              lane r) and read from there as the MMA's A operand
 // Issuing a tcgen05.mma takes one thread about 60 cycles on an idle SM and
 // several times that when the other warps of its SM sub-partition are busy
 // with ALU work, while these small-N products take about 70 cycles each on the
@@ -209,18 +210,21 @@ permute_mask_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
 //   warp 1: W' of every tile into TMEM buffer k % 3
 //   warps 2, 3: At of the even / odd tiles into TMEM buffer k % 2
 //   warps 4..11: 8 mask warps (two per TMEM lane quadrant, 32 columns each):
-//           W' of tile k -> the N:M keep bits (stored to the mask) and A
+//           W' of tile k -> the N:M keep bits (stored to the mask) and A (tcgen05.st)
 //   warps 12..15: copy-out warps (one per quadrant, 64 columns each): At of
 //           tile k -> swizzled staging tile -> TMA store
 // Sixteen warps, four per sub-partition, leave each thread 128 registers.
 // The P-image slot of a channel tile is free once every issuer that had a
 // tile in it has committed; the producer arrives for the At issuer that had
 // none, so each phase of that barrier counts all three.
+#ifndef LCP_PERMUTE_STAGES
+#define LCP_PERMUTE_STAGES 5
+#endif
 struct PwCfg {
-  static constexpr int STAGES = 5;
-  static constexpr int NW = 3;                          // W' TMEM buffers (128 columns: hi | lo)
+  static constexpr int STAGES = LCP_PERMUTE_STAGES;
+  static constexpr int NW = 3;                          // W' TMEM buffers (64 columns)
   static constexpr int NAT = 2;                         // At TMEM buffers (64 columns)
-  static constexpr int NA = 3;                          // A buffers in shared memory
+  static constexpr int NA = 3;                          // A TMEM buffers (32 columns of bf16 pairs)
   static constexpr int W_BYTES = 16384;                 // 128 rows x 64 bf16
   static constexpr int IMG_BYTES = 8192;                // 64 x 64 bf16
   static constexpr int SLOT = 3 * IMG_BYTES;            // Pt_hi | Pt_lo | P_hi
@@ -230,9 +234,11 @@ struct PwCfg {
   static constexpr int MASK0 = 1 + ISSUERS, COPY0 = MASK0 + MASK_WARPS;   // first warp of each role
   static constexpr int THREADS = 32 * (COPY0 + COPY_WARPS);
   static constexpr int NBAR = 2 * STAGES + 2 * NW + 2 * NAT + 2 * NA + 8 + ISSUERS;
-  static constexpr int SMEM = STAGES * W_BYTES + 2 * SLOT + (NA + 2) * A_BYTES + NBAR * 8 + 16 + 1024;
+  static constexpr int SMEM = STAGES * W_BYTES + 2 * SLOT + 2 * A_BYTES + NBAR * 8 + 16 + 1024;
+  static constexpr uint32_t TM_AT = NW * 64, TM_A = TM_AT + NAT * 64;   // TMEM column bases
   static_assert(SMEM <= 232448, "shared memory budget");
-  static_assert(NW * 128 + NAT * 64 <= 512, "tensor memory budget");
+  static_assert(TM_A + NA * 32 <= 512, "tensor memory budget");
+  static_assert(MCOLS == 32, "a mask thread stores 16 columns of bf16 pairs");
 };
 
 // position in the flat t-major tile list, advanced one tile at a time
@@ -259,8 +265,7 @@ permute_mask_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sStage = smem;
   uint8_t* sSlot = sStage + C::STAGES * C::W_BYTES;     // 2 slots of P images
-  uint8_t* sA = sSlot + 2 * C::SLOT;                    // NA buffers of A = M.W'
-  uint8_t* sO = sA + C::NA * C::A_BYTES;                // 2 staging tiles for At
+  uint8_t* sO = sSlot + 2 * C::SLOT;                    // 2 staging tiles for At
   uint64_t* bars = reinterpret_cast<uint64_t*>(sO + 2 * C::A_BYTES);
   uint32_t* holder = reinterpret_cast<uint32_t*>(bars + C::NBAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(holder + 1);
@@ -396,11 +401,14 @@ permute_mask_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
           if (!mbar_wait(bar(FULL + st), (uint32_t)(k / S) & 1u, abort_flag, 63)) break;
           if (!mbar_wait(bar(TMW + b), ((uint32_t)(k / NW) & 1u) ^ 1u, abort_flag, 64)) break;   // W' of k - NW read
           tc_fence_after();
-          constexpr uint32_t idesc = idesc_bf16(128, 128, false, false);
+          constexpr uint32_t idesc = idesc_bf16(128, 64, false, false);
           const uint32_t sw = smem_u32(sStage + st * C::W_BYTES);
 #pragma unroll
-          for (int k16 = 0; k16 < 4; ++k16)
-            mma_bf16(tmem + b * 128, sdesc(sw + k16 * 32, 16, 1024), sdesc(sp + k16 * 32, 16, 1024), idesc, k16 != 0);
+          for (int k16 = 0; k16 < 4; ++k16) {
+            const uint64_t wdesc = sdesc(sw + k16 * 32, 16, 1024);
+            mma_bf16(tmem + b * 64, wdesc, sdesc(sp + k16 * 32, 16, 1024), idesc, k16 != 0);
+            mma_bf16(tmem + b * 64, wdesc, sdesc(sp + C::IMG_BYTES + k16 * 32, 16, 1024), idesc, true);
+          }
           mma_commit(bar(WF + b));
           mma_commit(bar(EMPTY + st));
         } else {
@@ -409,12 +417,11 @@ permute_mask_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
           if (!mbar_wait(bar(TMA + a), ((uint32_t)(k / NAT) & 1u) ^ 1u, abort_flag, 69)) break;  // At of k - NAT read
           tc_fence_after();
           constexpr uint32_t idesc = idesc_bf16(128, 64, false, false);
-          const uint32_t sa = smem_u32(sA + c * C::A_BYTES);
           const uint32_t sph = sp + 2 * C::IMG_BYTES;
 #pragma unroll
           for (int k16 = 0; k16 < 4; ++k16)
-            mma_bf16(tmem + NW * 128 + a * 64, sdesc(sa + k16 * 32, 16, 1024), sdesc(sph + k16 * 32, 16, 1024), idesc,
-                     k16 != 0);
+            mma_bf16_ts(tmem + C::TM_AT + a * 64, tmem + C::TM_A + c * 32 + k16 * 8, sdesc(sph + k16 * 32, 16, 1024),
+                        idesc, k16 != 0);
           mma_commit(bar(ATF + a));
           mma_commit(bar(AE + c));   // A buffer c reusable
         }
@@ -430,23 +437,21 @@ permute_mask_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
     const int row = q * 32 + lane;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     TileIter it(first, nrt);
-    // W' of tile k + 1 (its hi and lo parts) is loaded from TMEM while tile k
-    // is processed (tcgen05.wait::ld waits for every outstanding load of the
-    // thread, so the next load is issued only after the current one has been
-    // waited for)
-    uint32_t hn[NV], ln[NV];
+    // W' of tile k + 1 is loaded from TMEM while tile k is processed
+    // (tcgen05.wait::ld waits for every outstanding load of the thread, so the
+    // next load is issued only after the current one has been waited for)
+    uint32_t hn[NV];
     bool have_next = nloc > 0 && wait_all(WF + 0, 0u, 67);
     if (have_next) {
       tc_fence_after();
       tmem_ld_cols<NV>(tmem + lane_off + h * NV, hn);
-      tmem_ld_cols<NV>(tmem + lane_off + 64 + h * NV, ln);
     }
     for (int k = 0; k < nloc && have_next; ++k, it.next()) {
       const int b = k % NW;
       tmem_ld_wait();
       uint32_t v[NV];
 #pragma unroll
-      for (int x = 0; x < NV; ++x) v[x] = __float_as_uint(__uint_as_float(hn[x]) + __uint_as_float(ln[x]));
+      for (int x = 0; x < NV; ++x) v[x] = hn[x];
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(TMW + b));
@@ -455,8 +460,7 @@ permute_mask_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
         const int bn = (k + 1) % NW;
         if (!wait_all(WF + bn, (uint32_t)((k + 1) / NW) & 1u, 67)) break;
         tc_fence_after();
-        tmem_ld_cols<NV>(tmem + lane_off + bn * 128 + h * NV, hn);
-        tmem_ld_cols<NV>(tmem + lane_off + bn * 128 + 64 + h * NV, ln);
+        tmem_ld_cols<NV>(tmem + lane_off + bn * 64 + h * NV, hn);
         have_next = true;
       }
       const int grow = it.rt * 128 + row;
@@ -484,17 +488,14 @@ permute_mask_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
       if constexpr (MODE == kMaskOnly) continue;
 #pragma unroll
       for (int x = 0; x < NV; ++x) v[x] = ((w >> x) & 1u) ? v[x] : 0u;
+      uint32_t pk[NV / 2];
+#pragma unroll
+      for (int x = 0; x < NV / 2; ++x) pk[x] = pack_bf16x2(__uint_as_float(v[2 * x]), __uint_as_float(v[2 * x + 1]));
       // A buffer k % NA was last read by At of tile k - NA
       if (!wait_all(AE + k % NA, ((uint32_t)(k / NA) & 1u) ^ 1u, 57)) break;
-      uint8_t* sa = sA + (k % NA) * C::A_BYTES;
-#pragma unroll
-      for (int c8 = 0; c8 < NV / 8; ++c8)
-        st_sw128(sa, row, h * (NV / 8) + c8,
-                 make_uint4(pack_bf16x2(__uint_as_float(v[8 * c8 + 0]), __uint_as_float(v[8 * c8 + 1])),
-                            pack_bf16x2(__uint_as_float(v[8 * c8 + 2]), __uint_as_float(v[8 * c8 + 3])),
-                            pack_bf16x2(__uint_as_float(v[8 * c8 + 4]), __uint_as_float(v[8 * c8 + 5])),
-                            pack_bf16x2(__uint_as_float(v[8 * c8 + 6]), __uint_as_float(v[8 * c8 + 7]))));
-      fence_async_smem();
+      tmem_st16(tmem + lane_off + C::TM_A + (k % NA) * 32 + h * (NV / 2), pk);
+      tmem_st_wait();
+      tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(AF + k % NA));
     }
@@ -519,7 +520,7 @@ permute_mask_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         uint32_t u[32];
-        tmem_ld32(tmem + lane_off + NW * 128 + a * 64 + hh * 32, u);
+        tmem_ld32(tmem + lane_off + C::TM_AT + a * 64 + hh * 32, u);
         tmem_ld_wait();
         if (hh == 1) {
           // the TMEM buffer may take At of tile j + NAT
