@@ -29,9 +29,9 @@
 // logits keeps its loads in flight.
 //
 // Z_0 never changes, so each thread keeps its share of Z_0 (or K) in registers
-// twice: a row slice (TPR adjacent lanes per row, interleaved columns) for the
-// row steps and a column slice (TPC adjacent lanes per column, interleaved
-// rows) for the column steps.  A step is then register arithmetic, a read of
+// twice: a row slice (TPR adjacent lanes per row) for the row steps and a
+// column slice (TPC adjacent lanes per column, interleaved rows) for the column
+// steps.  A step is then register arithmetic, a read of
 // the other side's vector from shared memory and two or three shuffles.
 //
 // A CTA owns one block at a time for B <= 64; for B = 128 a cluster of 2 CTAs
@@ -81,6 +81,25 @@ template <int B> struct SkCfg {
   static constexpr int EPC = R / TPC;                              // elements per column slice
   static constexpr int NW = NT / 32;
   static constexpr int LD = B + 1;                                 // padded smem tile row
+  static_assert(TPR >= 1 && TPR <= 32 && (32 % TPR) == 0, "row slices must sit inside a warp");
+  static_assert(TPC >= 1 && TPC <= 32 && (32 % TPC) == 0, "column slices must sit inside a warp");
+  static_assert(R * TPR == NT && B * TPC == NT, "bad Sinkhorn configuration");
+};
+
+// The forward kernel's threads: for B <= 64 a 128-thread CTA (one warp per SM sub-partition,
+// 32 elements of a row and 32 of a column a thread: one shuffle per reduction and a four-warp
+// barrier per step, the step's latency being what bounds a block); the clusters of B = 128 and
+// B = 256 keep 1024 threads a CTA.
+template <int B> struct SkFwdCfg {
+  static constexpr int CS = SkCfg<B>::CS;
+  static constexpr int NT = (B <= 64) ? 128 : 1024;
+  static constexpr int R = B / CS;
+  static constexpr int TPR = NT / R;
+  static constexpr int EPR = B / TPR;
+  static constexpr int TPC = NT / B;
+  static constexpr int EPC = R / TPC;
+  static constexpr int NW = NT / 32;
+  static constexpr int MINB = (B <= 64) ? 4 : 1;   // CTAs an SM (register bound 128 / 64)
   static_assert(TPR >= 1 && TPR <= 32 && (32 % TPR) == 0, "row slices must sit inside a warp");
   static_assert(TPC >= 1 && TPC <= 32 && (32 % TPC) == 0, "column slices must sit inside a warp");
   static_assert(R * TPR == NT && B * TPC == NT, "bad Sinkhorn configuration");
@@ -186,17 +205,31 @@ __device__ __forceinline__ void block_range(float mx, float mn, float* red, floa
   }
 }
 
-// Forward.  Shared memory (floats): tile[R*(B+1)] rv[R] cv[B] xm[2B] xs[2B] red[66]
+// Forward.  A thread's row slice is EPR consecutive columns c EPR .. c EPR + EPR - 1 of row r
+// and its column slice EPC consecutive rows g EPC .. g EPC + EPC - 1 of column j, so both
+// vectors are read with 16-byte loads, P and its row-major bf16 image are written from the
+// row slice and the transposed images from the column slice, straight from registers (the same
+// operands in the same order: the same values).  Z_0 is staged with a row pitch of B + 4
+// (16-byte rows).  The range of Z_0 is reduced from the staged registers under the barrier
+// that publishes the tile.
+// Shared memory (floats): tile[R*(B+4)] rv[R] cv[B] xm[2B] xs[2B] red[66]
+template <int B> __host__ __device__ constexpr int fwd_ld() { return B + 4; }
+template <int B> constexpr size_t fwd_smem_base() {
+  using C = SkFwdCfg<B>;
+  return sizeof(float) * (C::R * fwd_ld<B>() + C::R + B + 4 * B + 66);
+}
+
 template <int B>
-__global__ void __launch_bounds__(SkCfg<B>::NT, 1024 / SkCfg<B>::NT)
+__global__ void __launch_bounds__(SkFwdCfg<B>::NT, SkFwdCfg<B>::MINB)
 sinkhorn_fwd_kernel(const __grid_constant__ SkFwdBatch batch, float tau, int iters) {
-  using C = SkCfg<B>;
+  using C = SkFwdCfg<B>;
   pdl_wait();
   pdl_trigger();
   constexpr int R = C::R, NT = C::NT, CS = C::CS, TPR = C::TPR, EPR = C::EPR, TPC = C::TPC,
-                EPC = C::EPC, LD = C::LD;
+                EPC = C::EPC, NW = C::NW, LD = fwd_ld<B>();
   constexpr int NPRE = R * (B / 4) / NT;   // float4 of L a thread stages per block
   static_assert(NPRE * NT == R * (B / 4), "the L slab must split evenly over the threads");
+  static_assert(EPR % 4 == 0 && LD % 4 == 0, "row slices are read and written as float4");
   extern __shared__ __align__(16) float sm[];
   float* tile = sm;
   float* rv = tile + R * LD;   // per row of this CTA: a_i (linear) or R_i (log domain)
@@ -207,9 +240,9 @@ sinkhorn_fwd_kernel(const __grid_constant__ SkFwdBatch batch, float tau, int ite
 
   const int rank = cta_rank<CS>();
   const int row0 = rank * R;
-  const int tid = threadIdx.x;
-  const int r = tid / TPR, c = tid % TPR;     // row slice: row r, columns c + TPR*e
-  const int j = tid / TPC, g = tid % TPC;     // column slice: column j, rows g + TPC*e
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const int r = tid / TPR, c = tid % TPR;     // row slice: row r, columns c EPR + e
+  const int j = tid / TPC, g = tid % TPC;     // column slice: column j, rows g EPC + e
   const float inv_tau = 1.0f / tau;
   // The CTA (cluster) walks the blocks g = blockIdx.x / CS, + gridDim.x / CS, ...
   // of every layer; the next block's slab of L is loaded into registers while
@@ -247,32 +280,64 @@ sinkhorn_fwd_kernel(const __grid_constant__ SkFwdBatch batch, float tau, int ite
   const size_t base = (size_t)blk * B * B;
   const size_t ck0 = (size_t)blk * iters * 2 * B;
 
-  // Z_0 = L / tau (as L times the correctly rounded 1 / tau: within an ulp)
+  // Z_0 = L / tau (as L times the correctly rounded 1 / tau: within an ulp) into the tile, and
+  // the range of this thread's staged values, reduced per warp
+  float lmx = -CUDART_INF_F, lmn = CUDART_INF_F;
 #pragma unroll
   for (int k = 0; k < NPRE; ++k) {
     const int q = tid + k * NT;
     const int rr = q / (B / 4), jj = (q % (B / 4)) * 4;
-    float* d = tile + rr * LD + jj;
-    d[0] = pre[k].x * inv_tau; d[1] = pre[k].y * inv_tau; d[2] = pre[k].z * inv_tau; d[3] = pre[k].w * inv_tau;
+    const float4 z = make_float4(pre[k].x * inv_tau, pre[k].y * inv_tau, pre[k].z * inv_tau, pre[k].w * inv_tau);
+    *reinterpret_cast<float4*>(tile + rr * LD + jj) = z;
+    lmx = fmaxf(lmx, fmaxf(fmaxf(z.x, z.y), fmaxf(z.z, z.w)));
+    lmn = fminf(lmn, fminf(fminf(z.x, z.y), fminf(z.z, z.w)));
   }
   if (AHEAD && gb + gstride < total) prefetch(gb + gstride);   // in flight while this block iterates
+  lmx = group_max<32>(lmx);
+  lmn = -group_max<32>(-lmn);
+  if (lane == 0) {
+    red[warp] = lmx;
+    red[32 + warp] = lmn;
+  }
   __syncthreads();
+  float zmax = red[0], zmin = red[32];
+#pragma unroll
+  for (int w = 1; w < NW; ++w) {
+    zmax = fmaxf(zmax, red[w]);
+    zmin = fminf(zmin, red[32 + w]);
+  }
+  if constexpr (CS > 1) {
+    if (tid == 0) {
+      red[64] = zmax;
+      red[65] = zmin;
+    }
+    cluster_barrier<CS>();
+    float a = -CUDART_INF_F, bmin = CUDART_INF_F;
+#pragma unroll
+    for (int q = 0; q < CS; ++q) {
+      const float* pr = peer<CS>(red, q);
+      a = fmaxf(a, pr[64]);
+      bmin = fminf(bmin, pr[65]);
+    }
+    zmax = a;
+    zmin = bmin;
+  }
   float zr[EPR], zc[EPC];
 #pragma unroll
-  for (int e = 0; e < EPR; ++e) zr[e] = tile[r * LD + c + TPR * e];
-#pragma unroll
-  for (int e = 0; e < EPC; ++e) zc[e] = tile[(g + TPC * e) * LD + j];
-  float lmx = zr[0], lmn = zr[0];
-#pragma unroll
-  for (int e = 1; e < EPR; ++e) {
-    lmx = fmaxf(lmx, zr[e]);
-    lmn = fminf(lmn, zr[e]);
+  for (int e = 0; e < EPR; e += 4) {
+    const float4 v = *reinterpret_cast<const float4*>(tile + r * LD + c * EPR + e);
+    zr[e] = v.x; zr[e + 1] = v.y; zr[e + 2] = v.z; zr[e + 3] = v.w;
   }
-  float zmax, zmin;
-  block_range<NT, CS>(lmx, lmn, red, zmax, zmin);
+#pragma unroll
+  for (int e = 0; e < EPC; ++e) zc[e] = tile[(g * EPC + e) * LD + j];
   const bool linear = (zmax - zmin) <= kLinearRange;
+  // checkpoint value of row r / column j after step k, in the log form the reverse pass reads
+  // (R_i = max + log s and C_j = log s in the linear arithmetic)
+  auto ck_row = [&](int k, float v) { ckpt[ck0 + (size_t)k * 2 * B + row0 + r] = linear ? zmax + __logf(v) : v; };
+  auto ck_col = [&](int k, float v) { ckpt[ck0 + ((size_t)k * 2 + 1) * B + j] = linear ? __logf(v) : v; };
 
   float myR = 0.f;   // this thread's row: a_i (linear) or R_i (log domain)
+  float pv[EPR];     // P of this thread's row slice
   if (linear) {
 #pragma unroll
     for (int e = 0; e < EPR; ++e) zr[e] = __expf(zr[e] - zmax);
@@ -283,27 +348,39 @@ sinkhorn_fwd_kernel(const __grid_constant__ SkFwdBatch batch, float tau, int ite
     for (int k = 0; k < iters; ++k) {
       // T_r: a_i = 1 / sum_j K_ij b_j   (R_i = max Z_0 + log of that sum)
       {
-        float s = 0.f;
+        float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
 #pragma unroll
-        for (int e = 0; e < EPR; ++e) s = fmaf(zr[e], cv[c + TPR * e], s);
-        s = group_sum<TPR>(s);
-        myR = __frcp_rn(s);
+        for (int e = 0; e < EPR; e += 4) {
+          const float4 b4 = *reinterpret_cast<const float4*>(cv + c * EPR + e);
+          s0 = fmaf(zr[e], b4.x, s0);
+          s1 = fmaf(zr[e + 1], b4.y, s1);
+          s2 = fmaf(zr[e + 2], b4.z, s2);
+          s3 = fmaf(zr[e + 3], b4.w, s3);
+        }
+        const float s = group_sum<TPR>((s0 + s1) + (s2 + s3));
+        myR = __fdividef(1.f, s);
         if (c == 0) {
           rv[r] = myR;
-          if (ckpt) ckpt[ck0 + (size_t)k * 2 * B + row0 + r] = zmax + __logf(s);
+          if (ckpt) ck_row(k, s);
         }
       }
       __syncthreads();
       // T_c: b_j = 1 / sum_i a_i K_ij over all B rows   (C_j = log of that sum)
       {
-        float s = 0.f;
+        float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
 #pragma unroll
-        for (int e = 0; e < EPC; ++e) s = fmaf(zc[e], rv[g + TPC * e], s);
-        s = group_sum<TPC>(s);
+        for (int e = 0; e < EPC; e += 4) {
+          const float4 a4 = *reinterpret_cast<const float4*>(rv + g * EPC + e);
+          s0 = fmaf(zc[e], a4.x, s0);
+          s1 = fmaf(zc[e + 1], a4.y, s1);
+          s2 = fmaf(zc[e + 2], a4.z, s2);
+          s3 = fmaf(zc[e + 3], a4.w, s3);
+        }
+        const float s = group_sum<TPC>((s0 + s1) + (s2 + s3));
         if constexpr (CS == 1) {
           if (g == 0) {
-            cv[j] = __frcp_rn(s);
-            if (ckpt) ckpt[ck0 + ((size_t)k * 2 + 1) * B + j] = __logf(s);
+            cv[j] = __fdividef(1.f, s);
+            if (ckpt) ck_col(k, s);
           }
         } else {
           float* bs = xs + (k & 1) * B;
@@ -313,16 +390,22 @@ sinkhorn_fwd_kernel(const __grid_constant__ SkFwdBatch batch, float tau, int ite
             float S = 0.f;
 #pragma unroll
             for (int q = 0; q < CS; ++q) S += peer<CS>(bs, q)[j];
-            cv[j] = __frcp_rn(S);
-            if (ckpt && rank == 0) ckpt[ck0 + ((size_t)k * 2 + 1) * B + j] = __logf(S);
+            cv[j] = __fdividef(1.f, S);
+            if (ckpt && rank == 0) ck_col(k, S);
           }
         }
         __syncthreads();
       }
     }
-    // P = a_i K_ij b_j, staged through the tile for coalesced stores
+    // P = a_i K_ij b_j
 #pragma unroll
-    for (int e = 0; e < EPR; ++e) tile[r * LD + c + TPR * e] = myR * zr[e] * cv[c + TPR * e];
+    for (int e = 0; e < EPR; e += 4) {
+      const float4 b4 = *reinterpret_cast<const float4*>(cv + c * EPR + e);
+      pv[e] = myR * zr[e] * b4.x;
+      pv[e + 1] = myR * zr[e + 1] * b4.y;
+      pv[e + 2] = myR * zr[e + 2] * b4.z;
+      pv[e + 3] = myR * zr[e + 3] * b4.w;
+    }
   } else {
     for (int jj = tid; jj < B; jj += NT) cv[jj] = 0.f;
     __syncthreads();
@@ -331,13 +414,16 @@ sinkhorn_fwd_kernel(const __grid_constant__ SkFwdBatch batch, float tau, int ite
       {
         float x[EPR];
 #pragma unroll
-        for (int e = 0; e < EPR; ++e) x[e] = zr[e] - cv[c + TPR * e];
+        for (int e = 0; e < EPR; e += 4) {
+          const float4 b4 = *reinterpret_cast<const float4*>(cv + c * EPR + e);
+          x[e] = zr[e] - b4.x; x[e + 1] = zr[e + 1] - b4.y; x[e + 2] = zr[e + 2] - b4.z; x[e + 3] = zr[e + 3] - b4.w;
+        }
         float m, s;
         lse_parts<EPR, TPR>(x, m, s);
         myR = m + __logf(s);
         if (c == 0) {
           rv[r] = myR;
-          if (ckpt) ckpt[ck0 + (size_t)k * 2 * B + row0 + r] = myR;
+          if (ckpt) ck_row(k, myR);
         }
       }
       __syncthreads();
@@ -345,14 +431,17 @@ sinkhorn_fwd_kernel(const __grid_constant__ SkFwdBatch batch, float tau, int ite
       {
         float x[EPC];
 #pragma unroll
-        for (int e = 0; e < EPC; ++e) x[e] = zc[e] - rv[g + TPC * e];
+        for (int e = 0; e < EPC; e += 4) {
+          const float4 a4 = *reinterpret_cast<const float4*>(rv + g * EPC + e);
+          x[e] = zc[e] - a4.x; x[e + 1] = zc[e + 1] - a4.y; x[e + 2] = zc[e + 2] - a4.z; x[e + 3] = zc[e + 3] - a4.w;
+        }
         float m, s;
         lse_parts<EPC, TPC>(x, m, s);
         if constexpr (CS == 1) {
           if (g == 0) {
             const float v = m + __logf(s);
             cv[j] = v;
-            if (ckpt) ckpt[ck0 + ((size_t)k * 2 + 1) * B + j] = v;
+            if (ckpt) ck_col(k, v);
           }
           __syncthreads();
         } else {
@@ -369,66 +458,83 @@ sinkhorn_fwd_kernel(const __grid_constant__ SkFwdBatch batch, float tau, int ite
             for (int q = 0; q < CS; ++q) S += peer<CS>(bs, q)[j] * __expf(peer<CS>(bm, q)[j] - M);
             const float v = M + __logf(S);
             cv[j] = v;
-            if (ckpt && rank == 0) ckpt[ck0 + ((size_t)k * 2 + 1) * B + j] = v;
+            if (ckpt && rank == 0) ck_col(k, v);
           }
           __syncthreads();
         }
       }
     }
-    // P = exp(Z_0 - R - C), staged through the tile for coalesced stores
+    // P = exp(Z_0 - R - C)
 #pragma unroll
-    for (int e = 0; e < EPR; ++e) tile[r * LD + c + TPR * e] = __expf(zr[e] - myR - cv[c + TPR * e]);
+    for (int e = 0; e < EPR; e += 4) {
+      const float4 b4 = *reinterpret_cast<const float4*>(cv + c * EPR + e);
+      pv[e] = __expf(zr[e] - myR - b4.x);
+      pv[e + 1] = __expf(zr[e + 1] - myR - b4.y);
+      pv[e + 2] = __expf(zr[e + 2] - myR - b4.z);
+      pv[e + 3] = __expf(zr[e + 3] - myR - b4.w);
+    }
   }
-  __syncthreads();
-  // P, four consecutive columns a thread (16-byte stores)
-  for (int q = tid; q < R * (B / 4); q += NT) {
-    const int rr = q / (B / 4), jj = (q % (B / 4)) * 4;
-    const float* src = tile + rr * LD + jj;
-    reinterpret_cast<float4*>(P + base + (size_t)(row0 + rr) * B)[jj / 4] = make_float4(src[0], src[1], src[2], src[3]);
+  // P and its row-major bf16 image, straight from registers
+  {
+    float* prow = P + base + (size_t)(row0 + r) * B + c * EPR;
+#pragma unroll
+    for (int e = 0; e < EPR; e += 4)
+      *reinterpret_cast<float4*>(prow + e) = make_float4(pv[e], pv[e + 1], pv[e + 2], pv[e + 3]);
   }
   if (pt_hi) {
     // Operand images for the tensor-core kernels, in tiles of BC = max(B, 64)
     // columns: tile t holds the BC x BC block-diagonal slice of P_B covering
     // channels [t*BC, (t+1)*BC) (for B = 32 two blocks share one tile and the
-    // off-diagonal quadrants are written as zeros).  Eight consecutive bf16 a
-    // thread (16-byte stores).
+    // off-diagonal quadrants are written as zeros).
     constexpr int BC = B < 64 ? 64 : B;
     const int gcol0 = blk * B;
     const size_t tb = (size_t)(gcol0 / BC) * BC * BC;
     const int q0 = gcol0 % BC;
     const int zc0 = (q0 == 0) ? B : 0;   // the zero quadrant's columns (B < BC)
     const uint4 zero4 = make_uint4(0u, 0u, 0u, 0u);
-    // transposed images: image row q0 + jj, source rows i = row0 + 8 g .. + 7
-    for (int q = tid; q < B * (R / 8); q += NT) {
-      const int jj = q / (R / 8), g8 = (q % (R / 8)) * 8;
-      float hv[8], lv[8];
+    // P_hi: image row q0 + row0 + r, columns q0 + c EPR .. (from registers)
+    {
+      __nv_bfloat16* prow = p_hi + tb + (size_t)(q0 + row0 + r) * BC;
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const float p = tile[(g8 + u) * LD + jj];
-        const __nv_bfloat16 hi = __float2bfloat16_rn(p);
-        hv[u] = __bfloat162float(hi);
-        lv[u] = p - hv[u];
+      for (int e = 0; e < EPR; e += 8) {
+        if constexpr (EPR % 8 == 0) {
+          *reinterpret_cast<uint4*>(prow + q0 + c * EPR + e) =
+              make_uint4(pack_bf16x2_rn(pv[e], pv[e + 1]), pack_bf16x2_rn(pv[e + 2], pv[e + 3]),
+                         pack_bf16x2_rn(pv[e + 4], pv[e + 5]), pack_bf16x2_rn(pv[e + 6], pv[e + 7]));
+          if constexpr (B < BC) *reinterpret_cast<uint4*>(prow + zc0 + c * EPR + e) = zero4;
+        }
       }
-      const size_t at = tb + (size_t)(q0 + jj) * BC + q0 + row0 + g8;
-      *reinterpret_cast<uint4*>(pt_hi + at) = make_uint4(pack_bf16x2_rn(hv[0], hv[1]), pack_bf16x2_rn(hv[2], hv[3]),
-                                                         pack_bf16x2_rn(hv[4], hv[5]), pack_bf16x2_rn(hv[6], hv[7]));
-      *reinterpret_cast<uint4*>(pt_lo + at) = make_uint4(pack_bf16x2_rn(lv[0], lv[1]), pack_bf16x2_rn(lv[2], lv[3]),
-                                                         pack_bf16x2_rn(lv[4], lv[5]), pack_bf16x2_rn(lv[6], lv[7]));
-      if constexpr (B < BC) {
-        const size_t az = tb + (size_t)(q0 + jj) * BC + zc0 + row0 + g8;
-        *reinterpret_cast<uint4*>(pt_hi + az) = zero4;
-        *reinterpret_cast<uint4*>(pt_lo + az) = zero4;
+      if constexpr (EPR == 4) {
+        *reinterpret_cast<uint2*>(prow + q0 + c * EPR) =
+            make_uint2(pack_bf16x2_rn(pv[0], pv[1]), pack_bf16x2_rn(pv[2], pv[3]));
+        if constexpr (B < BC) *reinterpret_cast<uint2*>(prow + zc0 + c * EPR) = make_uint2(0u, 0u);
       }
     }
-    // P_hi: image row q0 + i, columns q0 + 8 g .. + 7
-    for (int q = tid; q < R * (B / 8); q += NT) {
-      const int rr = q / (B / 8), g8 = (q % (B / 8)) * 8;
-      const float* src = tile + rr * LD + g8;
-      const size_t at = tb + (size_t)(q0 + row0 + rr) * BC;
-      *reinterpret_cast<uint4*>(p_hi + at + q0 + g8) =
-          make_uint4(pack_bf16x2_rn(src[0], src[1]), pack_bf16x2_rn(src[2], src[3]), pack_bf16x2_rn(src[4], src[5]),
-                     pack_bf16x2_rn(src[6], src[7]));
-      if constexpr (B < BC) *reinterpret_cast<uint4*>(p_hi + at + zc0 + g8) = zero4;
+    // transposed images from the column slice: image row q0 + j, columns q0 + row0 + g EPC ..
+    {
+      const size_t at = tb + (size_t)(q0 + j) * BC + q0 + row0 + g * EPC;
+      const float bj = cv[j];
+#pragma unroll
+      for (int e = 0; e < EPC; e += 8) {
+        float hv[8], lv[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float ai = rv[g * EPC + e + u];
+          const float p = linear ? ai * zc[e + u] * bj : __expf(zc[e + u] - ai - bj);
+          const __nv_bfloat16 hi = __float2bfloat16_rn(p);
+          hv[u] = __bfloat162float(hi);
+          lv[u] = p - hv[u];
+        }
+        *reinterpret_cast<uint4*>(pt_hi + at + e) = make_uint4(pack_bf16x2_rn(hv[0], hv[1]), pack_bf16x2_rn(hv[2], hv[3]),
+                                                               pack_bf16x2_rn(hv[4], hv[5]), pack_bf16x2_rn(hv[6], hv[7]));
+        *reinterpret_cast<uint4*>(pt_lo + at + e) = make_uint4(pack_bf16x2_rn(lv[0], lv[1]), pack_bf16x2_rn(lv[2], lv[3]),
+                                                               pack_bf16x2_rn(lv[4], lv[5]), pack_bf16x2_rn(lv[6], lv[7]));
+        if constexpr (B < BC) {
+          const size_t az = tb + (size_t)(q0 + j) * BC + zc0 + row0 + g * EPC + e;
+          *reinterpret_cast<uint4*>(pt_hi + az) = zero4;
+          *reinterpret_cast<uint4*>(pt_lo + az) = zero4;
+        }
+      }
     }
   }
   // every thread (and every CTA of the cluster) is done with this block's shared
@@ -691,10 +797,6 @@ __global__ void __launch_bounds__(256) sum_splits_kernel(const float4* __restric
   }
 }
 
-template <int B> constexpr size_t fwd_smem() {
-  using C = SkCfg<B>;
-  return sizeof(float) * (C::R * C::LD + C::R + B + 4 * B + 66);
-}
 template <int B> constexpr size_t bwd_smem() {
   using C = SkCfg<B>;
   return sizeof(float) * (C::R * C::LD + 2 * B + C::NW * B + B + 2 * B + 66);
@@ -1168,7 +1270,7 @@ int grid_blocks(K kernel, int nt, size_t smem, int cs, int blocks) {
 
 template <int B>
 lcp_status fwd_b(const SkFwdBatch& batch, int blocks, float tau, int iters, cudaStream_t st) {
-  using C = SkCfg<B>;
+  using C = SkFwdCfg<B>;
   if (B == 64 && blocks >= LCP_SINKHORN_WARP_MIN_BLOCKS) {
     // one warp a block: enough blocks to keep every SM's warps busy
     const int g = grid_blocks(sinkhorn_fwd_warp_kernel, 32 * kSkWarpWarps, 0, 1,
@@ -1176,11 +1278,12 @@ lcp_status fwd_b(const SkFwdBatch& batch, int blocks, float tau, int iters, cuda
     return launch_kernel(sinkhorn_fwd_warp_kernel, dim3(g), dim3(32 * kSkWarpWarps), 0, st, 1, true, "sinkhorn_fwd",
                          batch, tau, iters);
   }
-  const lcp_status s0 = ensure_smem_limit(reinterpret_cast<const void*>(sinkhorn_fwd_kernel<B>), (int)fwd_smem<B>(),
-                                          "sinkhorn_fwd");
+  const size_t smem = fwd_smem_base<B>();
+  const lcp_status s0 =
+      ensure_smem_limit(reinterpret_cast<const void*>(sinkhorn_fwd_kernel<B>), (int)smem, "sinkhorn_fwd");
   if (s0 != LCP_OK) return s0;
-  const int g = grid_blocks(sinkhorn_fwd_kernel<B>, C::NT, fwd_smem<B>(), C::CS, blocks);
-  return launch_kernel(sinkhorn_fwd_kernel<B>, dim3(g * C::CS), dim3(C::NT), fwd_smem<B>(), st, C::CS, true,
+  const int g = grid_blocks(sinkhorn_fwd_kernel<B>, C::NT, smem, C::CS, blocks);
+  return launch_kernel(sinkhorn_fwd_kernel<B>, dim3(g * C::CS), dim3(C::NT), smem, st, C::CS, true,
                        "sinkhorn_fwd", batch, tau, iters);
 }
 
