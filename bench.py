@@ -56,6 +56,9 @@ def workload(name):
         return synth.q_proj_4096()
     if name == "toy_256":
         return synth.toy_256()
+    if name in ("sweep_4096_b128", "sweep_4096_b256"):
+        # the sweep's 4096 x 4096 layer (T = 2048) at B = 128 / 256, 5 iterations, tau 1.0, 2:4
+        return synth.sweep_4096(int(name[-3:]), 5, 1.0, 2, 4)
     raise SystemExit(f"unknown workload {name}")
 
 

@@ -552,13 +552,15 @@ sinkhorn_fwd_kernel(const __grid_constant__ SkFwdBatch batch, float tau, int ite
 // (iters x 2 x B floats, already turned into a and b in the linear
 // arithmetic) is staged in shared memory once, so an iteration has no global
 // load and two barriers; otherwise each iteration fetches its two vectors.
-// For B = 64 the kernel is held to 64 registers a thread so that two CTAs
-// share an SM when many blocks are in flight (a whole model's logits in one
-// launch).
+// It runs launches of fewer than LCP_SINKHORN_PAIR_MIN_BLOCKS blocks of 64 (larger ones take
+// the two-warps-a-block kernel) and the cluster sizes, so for B <= 64 it takes one CTA an SM
+// and the registers that leaves; the range of Z_0 is reduced from the staged registers under
+// the barrier that publishes the tile, and the block's checkpoint values are loaded with L and
+// dP.
 // Shared memory (floats): tile[R*(B+1)] ck[B] ck1[B] part[NW*B] cs[B] xs[2B] red[66]
 //                         (+ stage[iters*2*B] when STAGED)
 template <int B, bool STAGED>
-__global__ void __launch_bounds__(SkCfg<B>::NT, 1024 / SkCfg<B>::NT)
+__global__ void __launch_bounds__(SkCfg<B>::NT, B <= 64 ? 1 : 1024 / SkCfg<B>::NT)
 sinkhorn_bwd_kernel(const __grid_constant__ SkBwdBatch batch, float tau, int iters) {
   using C = SkCfg<B>;
   pdl_wait();
@@ -624,25 +626,70 @@ sinkhorn_bwd_kernel(const __grid_constant__ SkBwdBatch batch, float tau, int ite
   const float* ckb = ckpt + (size_t)blk * iters * 2 * B;
 
   float zr[EPR], dz[EPR];
-  // Z_0 = L / tau, formed as in the forward kernel
+  // the block's checkpoint values this thread stages (STAGED), loaded now so that their latency
+  // overlaps the staging of Z_0 and the range reduction
+  constexpr int NCK = (STAGED && CS == 1) ? 2 : 0;   // (the cluster CTAs have no registers to spare)
+  float ckr[NCK > 0 ? NCK : 1];
+  if constexpr (NCK > 0) {
 #pragma unroll
-  for (int k = 0; k < NPRE; ++k) {
-    const int q = tid + k * NT;
-    const int rr = q / (B / 4), jj = (q % (B / 4)) * 4;
-    float* d = tile + rr * LD + jj;
-    d[0] = preL[k].x * inv_tau; d[1] = preL[k].y * inv_tau; d[2] = preL[k].z * inv_tau; d[3] = preL[k].w * inv_tau;
-  }
-  __syncthreads();
-#pragma unroll
-  for (int e = 0; e < EPR; ++e) zr[e] = tile[r * LD + c + TPR * e];
-  float lmx = zr[0], lmn = zr[0];
-#pragma unroll
-  for (int e = 1; e < EPR; ++e) {
-    lmx = fmaxf(lmx, zr[e]);
-    lmn = fminf(lmn, zr[e]);
+    for (int u = 0; u < NCK; ++u) {
+      const int q = tid + u * NT;
+      ckr[u] = q < iters * 2 * B ? ckb[q] : 0.f;
+    }
   }
   float zmax, zmin;
-  block_range<NT, CS>(lmx, lmn, red, zmax, zmin);   // ends with a barrier: the tile is free again
+  if constexpr (CS == 1) {
+    // Z_0 = L / tau, formed as in the forward kernel, and the range of this thread's values
+    // reduced per warp under the barrier that publishes the tile (the same values, so the same
+    // range and arithmetic as the forward kernel)
+    float lmx = -CUDART_INF_F, lmn = CUDART_INF_F;
+#pragma unroll
+    for (int k = 0; k < NPRE; ++k) {
+      const int q = tid + k * NT;
+      const int rr = q / (B / 4), jj = (q % (B / 4)) * 4;
+      const float z0 = preL[k].x * inv_tau, z1 = preL[k].y * inv_tau, z2 = preL[k].z * inv_tau, z3 = preL[k].w * inv_tau;
+      float* d = tile + rr * LD + jj;
+      d[0] = z0; d[1] = z1; d[2] = z2; d[3] = z3;
+      lmx = fmaxf(lmx, fmaxf(fmaxf(z0, z1), fmaxf(z2, z3)));
+      lmn = fminf(lmn, fminf(fminf(z0, z1), fminf(z2, z3)));
+    }
+    lmx = group_max<32>(lmx);
+    lmn = -group_max<32>(-lmn);
+    if (lane == 0) {
+      red[warp] = lmx;
+      red[32 + warp] = lmn;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int e = 0; e < EPR; ++e) zr[e] = tile[r * LD + c + TPR * e];
+    zmax = red[0];
+    zmin = red[32];
+#pragma unroll
+    for (int w = 1; w < NW; ++w) {
+      zmax = fmaxf(zmax, red[w]);
+      zmin = fminf(zmin, red[32 + w]);
+    }
+    __syncthreads();   // every thread has read its row slice: the tile is free again
+  } else {
+    // Z_0 = L / tau, formed as in the forward kernel
+#pragma unroll
+    for (int k = 0; k < NPRE; ++k) {
+      const int q = tid + k * NT;
+      const int rr = q / (B / 4), jj = (q % (B / 4)) * 4;
+      float* d = tile + rr * LD + jj;
+      d[0] = preL[k].x * inv_tau; d[1] = preL[k].y * inv_tau; d[2] = preL[k].z * inv_tau; d[3] = preL[k].w * inv_tau;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int e = 0; e < EPR; ++e) zr[e] = tile[r * LD + c + TPR * e];
+    float lmx = zr[0], lmn = zr[0];
+#pragma unroll
+    for (int e = 1; e < EPR; ++e) {
+      lmx = fmaxf(lmx, zr[e]);
+      lmn = fminf(lmn, zr[e]);
+    }
+    block_range<NT, CS>(lmx, lmn, red, zmax, zmin);   // ends with a barrier: the tile is free again
+  }
   const bool linear = (zmax - zmin) <= kLinearRange;
   if (linear) {
 #pragma unroll
@@ -660,7 +707,15 @@ sinkhorn_bwd_kernel(const __grid_constant__ SkBwdBatch batch, float tau, int ite
   if constexpr (STAGED) {
     // every (R, C) pair in the form the loop uses: a_i = e^{max - R_i} and
     // b_j = e^{-C_j} (linear), R and C as they are (log domain)
-    for (int q = tid; q < iters * 2 * B; q += NT) {
+#pragma unroll
+    for (int u = 0; u < NCK; ++u) {
+      const int q = tid + u * NT;
+      if (q < iters * 2 * B) {
+        const bool is_row = (q / B) % 2 == 0;
+        stage[q] = linear ? __expf(is_row ? zmax - ckr[u] : -ckr[u]) : ckr[u];
+      }
+    }
+    for (int q = tid + NCK * NT; q < iters * 2 * B; q += NT) {
       const float v = ckb[q];
       const bool is_row = (q / B) % 2 == 0;
       stage[q] = linear ? __expf(is_row ? zmax - v : -v) : v;
