@@ -228,16 +228,17 @@ block_bwd_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_consta
       const uint32_t cbase = (row < 64 ? 0u : 64u) + h * NV;
       tmem_ld_cols<NV>(tDP + lane_off + cbase, v);
       tmem_ld_wait();
-      float* scratch = reinterpret_cast<float*>(sAB);   // 64 x 64 floats; every MMA is done
+      // 64 x 64 floats, row pitch 65 (a warp's 32 rows fall in distinct banks); every MMA is done
+      float* scratch = reinterpret_cast<float*>(sAB);
       if (row >= 64) {
 #pragma unroll
-        for (int x = 0; x < NV; ++x) scratch[(row - 64) * 64 + h * NV + x] = __uint_as_float(v[x]);
+        for (int x = 0; x < NV; ++x) scratch[(row - 64) * 65 + h * NV + x] = __uint_as_float(v[x]);
       }
       named_sync(1, C::EPI);
       if (row < 64) {
         const int nb = cin / B;
         float* dPs = dP + (size_t)sidx * nb * B * B;
-        const float* add = scratch + row * 64 + h * NV;
+        const float* add = scratch + row * 65 + h * NV;
         if constexpr (B == 64) {
           float4* o = reinterpret_cast<float4*>(dPs + ((size_t)t * 64 + row) * 64 + h * NV);
 #pragma unroll
