@@ -220,6 +220,9 @@ permute_mask_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
 #ifndef LCP_PERMUTE_STAGES
 #define LCP_PERMUTE_STAGES 5
 #endif
+#ifndef LCP_PERMUTE_MASK_WARPS
+#define LCP_PERMUTE_MASK_WARPS 8   // 8 or 16 (two or four per TMEM lane quadrant)
+#endif
 struct PwCfg {
   static constexpr int STAGES = LCP_PERMUTE_STAGES;
   static constexpr int NW = 3;                          // W' TMEM buffers (64 columns)
@@ -229,7 +232,7 @@ struct PwCfg {
   static constexpr int IMG_BYTES = 8192;                // 64 x 64 bf16
   static constexpr int SLOT = 3 * IMG_BYTES;            // Pt_hi | Pt_lo | P_hi
   static constexpr int A_BYTES = 16384;
-  static constexpr int ISSUERS = 3, MASK_WARPS = 8, COPY_WARPS = 4;
+  static constexpr int ISSUERS = 3, MASK_WARPS = LCP_PERMUTE_MASK_WARPS, COPY_WARPS = 4;
   static constexpr int MCOLS = 64 / (MASK_WARPS / 4);   // columns per mask thread
   static constexpr int MASK0 = 1 + ISSUERS, COPY0 = MASK0 + MASK_WARPS;   // first warp of each role
   static constexpr int THREADS = 32 * (COPY0 + COPY_WARPS);
@@ -238,7 +241,7 @@ struct PwCfg {
   static constexpr uint32_t TM_AT = NW * 64, TM_A = TM_AT + NAT * 64;   // TMEM column bases
   static_assert(SMEM <= 232448, "shared memory budget");
   static_assert(TM_A + NA * 32 <= 512, "tensor memory budget");
-  static_assert(MCOLS == 32, "a mask thread stores 16 columns of bf16 pairs");
+  static_assert(MCOLS == 32 || MCOLS == 16, "a mask thread stores MCOLS / 2 columns of bf16 pairs");
 };
 
 // position in the flat t-major tile list, advanced one tile at a time
@@ -493,7 +496,7 @@ permute_mask_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
       for (int x = 0; x < NV / 2; ++x) pk[x] = pack_bf16x2(__uint_as_float(v[2 * x]), __uint_as_float(v[2 * x + 1]));
       // A buffer k % NA was last read by At of tile k - NA
       if (!wait_all(AE + k % NA, ((uint32_t)(k / NA) & 1u) ^ 1u, 57)) break;
-      tmem_st16(tmem + lane_off + C::TM_A + (k % NA) * 32 + h * (NV / 2), pk);
+      tmem_st_cols<NV / 2>(tmem + lane_off + C::TM_A + (k % NA) * 32 + h * (NV / 2), pk);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
