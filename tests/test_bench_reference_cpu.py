@@ -31,3 +31,19 @@ def test_reference_arm_prints_one_contract_line():
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
     # the arm times what it prints: its K timed steps fit inside the process's wall time
     assert d["ms_per_step"] * d["steps"] / 1e3 <= wall
+
+
+def test_bench_workloads_are_the_named_layers():
+    """--workload names the layer it runs: the q_proj-shaped headline layer and the sweep's
+    4096 x 4096 layer at B = 128 / 256 (5 iterations, tau 1.0, 2:4)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from learnable_channel_permutation_b200 import synth
+    q = bench.workload("q_proj_4096")
+    assert (q.block, q.n, q.m, q.iters, q.tau) == (64, 2, 4, 5, 0.5)
+    assert (q.layers[0].cout, q.layers[0].cin, q.layers[0].tokens) == (4096, 4096, 2048)
+    for B in (128, 256):
+        w = bench.workload(f"sweep_4096_b{B}")
+        ref = synth.sweep_4096(B, 5, 1.0, 2, 4)
+        assert w.name == ref.name and (w.block, w.n, w.m, w.iters, w.tau) == (B, 2, 4, 5, 1.0)
+        assert [(l.cout, l.cin, l.tokens) for l in w.layers] == [(4096, 4096, 2048)]
