@@ -205,7 +205,8 @@ __device__ __forceinline__ void block_range(float mx, float mn, float* red, floa
   }
 }
 
-// Forward.  A thread's row slice is EPR consecutive columns c EPR .. c EPR + EPR - 1 of row r
+// Forward for B <= 64 (one CTA a block; the cluster sizes run sinkhorn_fwd_cluster_kernel).
+// A thread's row slice is EPR consecutive columns c EPR .. c EPR + EPR - 1 of row r
 // and its column slice EPC consecutive rows g EPC .. g EPC + EPC - 1 of column j, so both
 // vectors are read with 16-byte loads, P and its row-major bf16 image are written from the
 // row slice and the transposed images from the column slice, straight from registers (the same
@@ -544,6 +545,261 @@ sinkhorn_fwd_kernel(const __grid_constant__ SkFwdBatch batch, float tau, int ite
   }
 }
 
+// Forward for the cluster sizes (B = 128, 256: 2 / 4 CTAs of 1024 threads a block): row slices
+// interleaved over the TPR lanes of a row, P staged through the tile for coalesced stores and
+// the transposed images (measured faster at these sizes than the B <= 64 kernel's layout).
+// Shared memory (floats): tile[R*(B+1)] rv[R] cv[B] xm[2B] xs[2B] red[66]
+template <int B>
+__global__ void __launch_bounds__(SkCfg<B>::NT, 1024 / SkCfg<B>::NT)
+sinkhorn_fwd_cluster_kernel(const __grid_constant__ SkFwdBatch batch, float tau, int iters) {
+  using C = SkCfg<B>;
+  pdl_wait();
+  pdl_trigger();
+  constexpr int R = C::R, NT = C::NT, CS = C::CS, TPR = C::TPR, EPR = C::EPR, TPC = C::TPC,
+                EPC = C::EPC, LD = C::LD;
+  constexpr int NPRE = R * (B / 4) / NT;   // float4 of L a thread stages per block
+  static_assert(NPRE * NT == R * (B / 4), "the L slab must split evenly over the threads");
+  extern __shared__ __align__(16) float sm[];
+  float* tile = sm;
+  float* rv = tile + R * LD;   // per row of this CTA: a_i (linear) or R_i (log domain)
+  float* cv = rv + R;          // per column: b_j (linear) or C_j (log domain)
+  float* xm = cv + B;          // this CTA's column partials, double-buffered by iteration parity
+  float* xs = xm + 2 * B;
+  float* red = xs + 2 * B;
+
+  const int rank = cta_rank<CS>();
+  const int row0 = rank * R;
+  const int tid = threadIdx.x;
+  const int r = tid / TPR, c = tid % TPR;     // row slice: row r, columns c + TPR*e
+  const int j = tid / TPC, g = tid % TPC;     // column slice: column j, rows g + TPC*e
+  const float inv_tau = 1.0f / tau;
+  // The CTA (cluster) walks the blocks g = blockIdx.x / CS, + gridDim.x / CS, ...
+  // of every layer; the next block's slab of L is loaded into registers while
+  // the current one iterates.
+  int total = 0;
+  for (int i = 0; i < batch.n; ++i) total += batch.layer[i].blocks;
+  const int gstride = gridDim.x / CS;
+  auto locate = [&](int gb, int& li, int& blk) {
+    blk = gb;
+    li = 0;
+    while (li + 1 < batch.n && blk >= batch.layer[li].blocks) blk -= batch.layer[li++].blocks;
+  };
+  float4 pre[NPRE];
+  auto prefetch = [&](int gb) {
+    int li, blk;
+    locate(gb, li, blk);
+    const float4* src = reinterpret_cast<const float4*>(batch.layer[li].L + (size_t)blk * B * B + (size_t)row0 * B);
+#pragma unroll
+    for (int k = 0; k < NPRE; ++k) pre[k] = src[tid + k * NT];
+  };
+  // the look-ahead needs NPRE more registers a thread: not for the 1024-thread B = 256 CTAs
+  constexpr bool AHEAD = NPRE <= 2;
+  if (AHEAD && blockIdx.x / CS < total) prefetch(blockIdx.x / CS);
+  for (int gb = blockIdx.x / CS; gb < total; gb += gstride) {
+  if constexpr (!AHEAD) prefetch(gb);
+  int li, blk;
+  locate(gb, li, blk);
+  const SkFwdLayer& ly = batch.layer[li];
+  float* __restrict__ P = ly.P;
+  float* __restrict__ ckpt = ly.ckpt;
+  __nv_bfloat16* __restrict__ pt_hi = ly.pt_hi;
+  __nv_bfloat16* __restrict__ pt_lo = ly.pt_lo;
+  __nv_bfloat16* __restrict__ p_hi = ly.p_hi;
+  if (ly.zero_word && blk == 0 && rank == 0 && tid == 0) *ly.zero_word = 0u;
+  const size_t base = (size_t)blk * B * B;
+  const size_t ck0 = (size_t)blk * iters * 2 * B;
+
+  // Z_0 = L / tau (as L times the correctly rounded 1 / tau: within an ulp)
+#pragma unroll
+  for (int k = 0; k < NPRE; ++k) {
+    const int q = tid + k * NT;
+    const int rr = q / (B / 4), jj = (q % (B / 4)) * 4;
+    float* d = tile + rr * LD + jj;
+    d[0] = pre[k].x * inv_tau; d[1] = pre[k].y * inv_tau; d[2] = pre[k].z * inv_tau; d[3] = pre[k].w * inv_tau;
+  }
+  if (AHEAD && gb + gstride < total) prefetch(gb + gstride);   // in flight while this block iterates
+  __syncthreads();
+  float zr[EPR], zc[EPC];
+#pragma unroll
+  for (int e = 0; e < EPR; ++e) zr[e] = tile[r * LD + c + TPR * e];
+#pragma unroll
+  for (int e = 0; e < EPC; ++e) zc[e] = tile[(g + TPC * e) * LD + j];
+  float lmx = zr[0], lmn = zr[0];
+#pragma unroll
+  for (int e = 1; e < EPR; ++e) {
+    lmx = fmaxf(lmx, zr[e]);
+    lmn = fminf(lmn, zr[e]);
+  }
+  float zmax, zmin;
+  block_range<NT, CS>(lmx, lmn, red, zmax, zmin);
+  const bool linear = (zmax - zmin) <= kLinearRange;
+
+  float myR = 0.f;   // this thread's row: a_i (linear) or R_i (log domain)
+  if (linear) {
+#pragma unroll
+    for (int e = 0; e < EPR; ++e) zr[e] = __expf(zr[e] - zmax);
+#pragma unroll
+    for (int e = 0; e < EPC; ++e) zc[e] = __expf(zc[e] - zmax);
+    for (int jj = tid; jj < B; jj += NT) cv[jj] = 1.f;
+    __syncthreads();
+    for (int k = 0; k < iters; ++k) {
+      // T_r: a_i = 1 / sum_j K_ij b_j   (R_i = max Z_0 + log of that sum)
+      {
+        float s = 0.f;
+#pragma unroll
+        for (int e = 0; e < EPR; ++e) s = fmaf(zr[e], cv[c + TPR * e], s);
+        s = group_sum<TPR>(s);
+        myR = __frcp_rn(s);
+        if (c == 0) {
+          rv[r] = myR;
+          if (ckpt) ckpt[ck0 + (size_t)k * 2 * B + row0 + r] = zmax + __logf(s);
+        }
+      }
+      __syncthreads();
+      // T_c: b_j = 1 / sum_i a_i K_ij over all B rows   (C_j = log of that sum)
+      {
+        float s = 0.f;
+#pragma unroll
+        for (int e = 0; e < EPC; ++e) s = fmaf(zc[e], rv[g + TPC * e], s);
+        s = group_sum<TPC>(s);
+        if constexpr (CS == 1) {
+          if (g == 0) {
+            cv[j] = __frcp_rn(s);
+            if (ckpt) ckpt[ck0 + ((size_t)k * 2 + 1) * B + j] = __logf(s);
+          }
+        } else {
+          float* bs = xs + (k & 1) * B;
+          if (g == 0) bs[j] = s;
+          cluster_barrier<CS>();
+          if (g == 0) {
+            float S = 0.f;
+#pragma unroll
+            for (int q = 0; q < CS; ++q) S += peer<CS>(bs, q)[j];
+            cv[j] = __frcp_rn(S);
+            if (ckpt && rank == 0) ckpt[ck0 + ((size_t)k * 2 + 1) * B + j] = __logf(S);
+          }
+        }
+        __syncthreads();
+      }
+    }
+    // P = a_i K_ij b_j, staged through the tile for coalesced stores
+#pragma unroll
+    for (int e = 0; e < EPR; ++e) tile[r * LD + c + TPR * e] = myR * zr[e] * cv[c + TPR * e];
+  } else {
+    for (int jj = tid; jj < B; jj += NT) cv[jj] = 0.f;
+    __syncthreads();
+    for (int k = 0; k < iters; ++k) {
+      // T_r: R_i = LSE_j(z_ij - C_j)
+      {
+        float x[EPR];
+#pragma unroll
+        for (int e = 0; e < EPR; ++e) x[e] = zr[e] - cv[c + TPR * e];
+        float m, s;
+        lse_parts<EPR, TPR>(x, m, s);
+        myR = m + __logf(s);
+        if (c == 0) {
+          rv[r] = myR;
+          if (ckpt) ckpt[ck0 + (size_t)k * 2 * B + row0 + r] = myR;
+        }
+      }
+      __syncthreads();
+      // T_c: C_j = LSE_i(z_ij - R_i) over all B rows of the block
+      {
+        float x[EPC];
+#pragma unroll
+        for (int e = 0; e < EPC; ++e) x[e] = zc[e] - rv[g + TPC * e];
+        float m, s;
+        lse_parts<EPC, TPC>(x, m, s);
+        if constexpr (CS == 1) {
+          if (g == 0) {
+            const float v = m + __logf(s);
+            cv[j] = v;
+            if (ckpt) ckpt[ck0 + ((size_t)k * 2 + 1) * B + j] = v;
+          }
+          __syncthreads();
+        } else {
+          float* bm = xm + (k & 1) * B;
+          float* bs = xs + (k & 1) * B;
+          if (g == 0) { bm[j] = m; bs[j] = s; }
+          cluster_barrier<CS>();
+          if (g == 0) {
+            float M = -CUDART_INF_F;
+#pragma unroll
+            for (int q = 0; q < CS; ++q) M = fmaxf(M, peer<CS>(bm, q)[j]);
+            float S = 0.f;
+#pragma unroll
+            for (int q = 0; q < CS; ++q) S += peer<CS>(bs, q)[j] * __expf(peer<CS>(bm, q)[j] - M);
+            const float v = M + __logf(S);
+            cv[j] = v;
+            if (ckpt && rank == 0) ckpt[ck0 + ((size_t)k * 2 + 1) * B + j] = v;
+          }
+          __syncthreads();
+        }
+      }
+    }
+    // P = exp(Z_0 - R - C), staged through the tile for coalesced stores
+#pragma unroll
+    for (int e = 0; e < EPR; ++e) tile[r * LD + c + TPR * e] = __expf(zr[e] - myR - cv[c + TPR * e]);
+  }
+  __syncthreads();
+  // P, four consecutive columns a thread (16-byte stores)
+  for (int q = tid; q < R * (B / 4); q += NT) {
+    const int rr = q / (B / 4), jj = (q % (B / 4)) * 4;
+    const float* src = tile + rr * LD + jj;
+    reinterpret_cast<float4*>(P + base + (size_t)(row0 + rr) * B)[jj / 4] = make_float4(src[0], src[1], src[2], src[3]);
+  }
+  if (pt_hi) {
+    // Operand images for the tensor-core kernels, in tiles of BC = max(B, 64)
+    // columns: tile t holds the BC x BC block-diagonal slice of P_B covering
+    // channels [t*BC, (t+1)*BC) (for B = 32 two blocks share one tile and the
+    // off-diagonal quadrants are written as zeros).  Eight consecutive bf16 a
+    // thread (16-byte stores).
+    constexpr int BC = B < 64 ? 64 : B;
+    const int gcol0 = blk * B;
+    const size_t tb = (size_t)(gcol0 / BC) * BC * BC;
+    const int q0 = gcol0 % BC;
+    const int zc0 = (q0 == 0) ? B : 0;   // the zero quadrant's columns (B < BC)
+    const uint4 zero4 = make_uint4(0u, 0u, 0u, 0u);
+    // transposed images: image row q0 + jj, source rows i = row0 + 8 g .. + 7
+    for (int q = tid; q < B * (R / 8); q += NT) {
+      const int jj = q / (R / 8), g8 = (q % (R / 8)) * 8;
+      float hv[8], lv[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const float p = tile[(g8 + u) * LD + jj];
+        const __nv_bfloat16 hi = __float2bfloat16_rn(p);
+        hv[u] = __bfloat162float(hi);
+        lv[u] = p - hv[u];
+      }
+      const size_t at = tb + (size_t)(q0 + jj) * BC + q0 + row0 + g8;
+      *reinterpret_cast<uint4*>(pt_hi + at) = make_uint4(pack_bf16x2_rn(hv[0], hv[1]), pack_bf16x2_rn(hv[2], hv[3]),
+                                                         pack_bf16x2_rn(hv[4], hv[5]), pack_bf16x2_rn(hv[6], hv[7]));
+      *reinterpret_cast<uint4*>(pt_lo + at) = make_uint4(pack_bf16x2_rn(lv[0], lv[1]), pack_bf16x2_rn(lv[2], lv[3]),
+                                                         pack_bf16x2_rn(lv[4], lv[5]), pack_bf16x2_rn(lv[6], lv[7]));
+      if constexpr (B < BC) {
+        const size_t az = tb + (size_t)(q0 + jj) * BC + zc0 + row0 + g8;
+        *reinterpret_cast<uint4*>(pt_hi + az) = zero4;
+        *reinterpret_cast<uint4*>(pt_lo + az) = zero4;
+      }
+    }
+    // P_hi: image row q0 + i, columns q0 + 8 g .. + 7
+    for (int q = tid; q < R * (B / 8); q += NT) {
+      const int rr = q / (B / 8), g8 = (q % (B / 8)) * 8;
+      const float* src = tile + rr * LD + g8;
+      const size_t at = tb + (size_t)(q0 + row0 + rr) * BC;
+      *reinterpret_cast<uint4*>(p_hi + at + q0 + g8) =
+          make_uint4(pack_bf16x2_rn(src[0], src[1]), pack_bf16x2_rn(src[2], src[3]), pack_bf16x2_rn(src[4], src[5]),
+                     pack_bf16x2_rn(src[6], src[7]));
+      if constexpr (B < BC) *reinterpret_cast<uint4*>(p_hi + at + zc0 + g8) = zero4;
+    }
+  }
+  // every thread (and every CTA of the cluster) is done with this block's shared
+  // memory before the next block overwrites it
+  if constexpr (CS > 1) cluster_barrier<CS>();
+  else __syncthreads();
+  }
+}
+
 // Reverse.  dZ lives in registers in the row layout.  The iterate after each
 // normalisation is rebuilt from the checkpoint: exp(Z) = a_i K_ij b_j with
 // a_i = e^{max - R_i}, b_j = e^{-C_j} in the linear arithmetic, exp(Z_0 - R_i -
@@ -852,6 +1108,10 @@ __global__ void __launch_bounds__(256) sum_splits_kernel(const float4* __restric
   }
 }
 
+template <int B> constexpr size_t fwd_cluster_smem() {
+  using C = SkCfg<B>;
+  return sizeof(float) * (C::R * C::LD + C::R + B + 4 * B + 66);
+}
 template <int B> constexpr size_t bwd_smem() {
   using C = SkCfg<B>;
   return sizeof(float) * (C::R * C::LD + 2 * B + C::NW * B + B + 2 * B + 66);
@@ -1333,13 +1593,23 @@ lcp_status fwd_b(const SkFwdBatch& batch, int blocks, float tau, int iters, cuda
     return launch_kernel(sinkhorn_fwd_warp_kernel, dim3(g), dim3(32 * kSkWarpWarps), 0, st, 1, true, "sinkhorn_fwd",
                          batch, tau, iters);
   }
-  const size_t smem = fwd_smem_base<B>();
-  const lcp_status s0 =
-      ensure_smem_limit(reinterpret_cast<const void*>(sinkhorn_fwd_kernel<B>), (int)smem, "sinkhorn_fwd");
-  if (s0 != LCP_OK) return s0;
-  const int g = grid_blocks(sinkhorn_fwd_kernel<B>, C::NT, smem, C::CS, blocks);
-  return launch_kernel(sinkhorn_fwd_kernel<B>, dim3(g * C::CS), dim3(C::NT), smem, st, C::CS, true,
-                       "sinkhorn_fwd", batch, tau, iters);
+  if constexpr (C::CS > 1) {
+    const size_t smem = fwd_cluster_smem<B>();
+    const lcp_status s0 = ensure_smem_limit(reinterpret_cast<const void*>(sinkhorn_fwd_cluster_kernel<B>),
+                                            (int)smem, "sinkhorn_fwd");
+    if (s0 != LCP_OK) return s0;
+    const int g = grid_blocks(sinkhorn_fwd_cluster_kernel<B>, C::NT, smem, C::CS, blocks);
+    return launch_kernel(sinkhorn_fwd_cluster_kernel<B>, dim3(g * C::CS), dim3(C::NT), smem, st, C::CS, true,
+                         "sinkhorn_fwd", batch, tau, iters);
+  } else {
+    const size_t smem = fwd_smem_base<B>();
+    const lcp_status s0 =
+        ensure_smem_limit(reinterpret_cast<const void*>(sinkhorn_fwd_kernel<B>), (int)smem, "sinkhorn_fwd");
+    if (s0 != LCP_OK) return s0;
+    const int g = grid_blocks(sinkhorn_fwd_kernel<B>, C::NT, smem, C::CS, blocks);
+    return launch_kernel(sinkhorn_fwd_kernel<B>, dim3(g * C::CS), dim3(C::NT), smem, st, C::CS, true,
+                         "sinkhorn_fwd", batch, tau, iters);
+  }
 }
 
 template <int B>
