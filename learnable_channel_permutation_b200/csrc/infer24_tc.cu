@@ -8,7 +8,8 @@
 // channels a product) takes the two kept values of every group of four as its
 // A operand and their positions as metadata in tensor memory.
 //   - the CTA owns 128 output rows and a K range of C_in / S channels; the S
-//     CTAs of a row tile form a cluster;
+//     CTAs of a row tile form a cluster (S <= 4 with 16 staging warps, S <= 8
+//     with 8 and two CTAs an SM);
 //   - TMA brings the compressed values (128 rows x 64 values, 128-byte
 //     swizzle: the A operand of four products as it lands) and the position
 //     words (128 rows x 4 words) of each 128-channel stage into a 4-stage ring;
@@ -29,8 +30,14 @@
 namespace lcp {
 namespace {
 
-struct StCfg {
-  static constexpr int EXP_WARPS = 16;              // stage the inputs; warps 0-3 then write the metadata
+// Two configurations: 16 staging warps (one CTA an SM, up to 2048 channels and 4 splits), and 8
+// (two CTAs an SM, up to 1024 channels and 8 splits: twice the weight streams in flight and half
+// the staging a CTA, measured faster at 4 and 8 tokens on the 4096^2 layer), used whenever it
+// takes the shape.
+template <int EW> struct StCfgT {
+  static constexpr int EXP_WARPS = EW;              // stage the inputs; warps 0-3 then write the metadata
+  static constexpr int CTAS_PER_SM = EW <= 8 ? 2 : 1;
+  static constexpr int MAX_SPLITS = EW <= 8 ? 8 : 4;
   static constexpr int PROD_WARP = EXP_WARPS, MMA_WARP = EXP_WARPS + 1;
   static constexpr int THREADS = 32 * (EXP_WARPS + 2);
   static constexpr int EXP_THREADS = 32 * EXP_WARPS;
@@ -39,7 +46,7 @@ struct StCfg {
   static constexpr int V_BYTES = 128 * 128;         // 128 rows x 64 bf16 values
   static constexpr int M_BYTES = 128 * 16;          // 128 rows x 4 position words
   static constexpr int RED_BYTES = 16 * 128 * 4;    // 16 tokens x 128 rows float32
-  static constexpr int MAX_KR = 2048;               // channels per CTA (input image 64 KB)
+  static constexpr int MAX_KR = 128 * EXP_WARPS;   // channels per CTA (input image up to 64 KB)
   // metadata of product k of buffer m at column TMEM_META + 8 (4 m + k): eight-column
   // aligned, the placement the probe used (the accumulator: columns 0-15)
   static constexpr int TMEM_META = 64, TMEM_COLS = 128;
@@ -68,19 +75,20 @@ __device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
   return v;
 }
 
-// Roles (18 warps): warp 16 loads the ring (TMA), warp 17 issues the products,
-// warps 0-15 stage the inputs, then warps 0-3 write each stage's metadata into
+// Roles (EW + 2 warps): warp EW loads the ring (TMA), warp EW + 1 issues the products,
+// warps 0 .. EW - 1 stage the inputs, then warps 0-3 write each stage's metadata into
 // TMEM; they meet only through mbarriers:
 //   full[q]   (TMA bytes)          ring slot q holds stage j        -> metadata warps, MMA warp
 //   empty[q]  (MMA commit)         the products reading slot q done -> producer
 //   mready[m] (4 warp arrivals)    TMEM metadata buffer m holds j   -> MMA warp
 //   mfree[m]  (MMA commit)         the products reading m are done  -> metadata warps
 //   fin       (MMA commit)         every product has landed         -> epilogue
-__global__ void __launch_bounds__(StCfg::THREADS, 1)
+template <int EW>
+__global__ void __launch_bounds__(StCfgT<EW>::THREADS, StCfgT<EW>::CTAS_PER_SM)
 sp24_tc_kernel(const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmM,
                const __nv_bfloat16* __restrict__ X, const int32_t* __restrict__ perm, float* __restrict__ Y,
                int cout, int cin, int tokens, int bshift, int kr) {
-  using C = StCfg;
+  using C = StCfgT<EW>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sV = smem;                                   // STG x 16 KB
@@ -178,7 +186,7 @@ sp24_tc_kernel(const __grid_constant__ CUtensorMap tmV, const __grid_constant__ 
     {
       const int Bm = perm ? (1 << bshift) - 1 : 0x7fffffff;
       const int runs = kr / 8;                          // 32 .. 256
-      const int G = C::EXP_THREADS / runs;              // token groups: 16 .. 2
+      const int G = C::EXP_THREADS / runs;              // token groups
       constexpr int TPT = 16 * C::MAX_KR / 8 / C::EXP_THREADS;   // tokens per thread at most (8)
       const int c = tid % runs, g = tid / runs;
       const int i0 = k0 + c * 8;
@@ -318,40 +326,52 @@ lcp_status tc_error_infer(int* site, int reset) { return read_tc_error(site, res
 // S in {1, 2, 4} with C_in / S a multiple of 256 and at most 2048, as many as
 // keep the grid (S x row tiles) within one wave of the SMs.
 // most C_in splits of a row tile (tuning: 1, 2 or 4)
-#ifndef LCP_SP24_MAX_SPLITS
-#define LCP_SP24_MAX_SPLITS 4
-#endif
-
-int sparse24_tc_splits(int cout, int cin) {
+// C_in splits S of a row tile for configuration EW: C_in / S a multiple of 256 and at most
+// MAX_KR; the fewest that fit, then more while one wave of the SMs holds the grid.
+template <int EW> int tc_splits(int cout, int cin) {
+  using C = StCfgT<EW>;
   if (cin % 256) return 0;
   const int tiles = cdiv(cout, 128);
   int best = 0;
-  for (int s = 1; s <= LCP_SP24_MAX_SPLITS; s *= 2) {
-    if (cin % (256 * s) || cin / s > StCfg::MAX_KR) continue;
-    if (best == 0) best = s;                            // the fewest splits that fit
-    else if (tiles * s <= num_sms()) best = s;          // more, while one wave holds them
+  for (int s = 1; s <= C::MAX_SPLITS; s *= 2) {
+    if (cin % (256 * s) || cin / s > C::MAX_KR) continue;
+    if (best == 0) best = s;
+    else if (tiles * s <= num_sms() * C::CTAS_PER_SM) best = s;
   }
   return best;
+}
+
+template <int EW>
+lcp_status launch_sp24(const CUtensorMap& mV, const CUtensorMap& mM, const __nv_bfloat16* X, const int32_t* perm,
+                       float* Y, int cout, int cin, int tokens, int bshift, int S, cudaStream_t st) {
+  using C = StCfgT<EW>;
+  const int kr = cin / S;
+  const int smem = C::smem(kr);
+  TC_TRY(set_smem(sp24_tc_kernel<EW>, smem, "sparse24_tc"));
+  const dim3 grid((unsigned)S, (unsigned)cdiv(cout, 128));
+  for (int t0 = 0; t0 < tokens; t0 += 16) {
+    const int tt = tokens - t0 < 16 ? tokens - t0 : 16;
+    TC_TRY(launch_kernel(sp24_tc_kernel<EW>, grid, dim3(C::THREADS), smem, st, S, true, "sparse24_tc", mV, mM,
+                         X + (size_t)t0 * cin, perm, Y + (size_t)t0 * cout, cout, cin, tt, bshift, kr));
+  }
+  return LCP_OK;
+}
+
+int sparse24_tc_splits(int cout, int cin) {
+  const int s8 = tc_splits<8>(cout, cin);
+  return s8 > 0 ? s8 : tc_splits<16>(cout, cin);
 }
 
 lcp_status launch_sparse24_tc(const __nv_bfloat16* vals, const uint32_t* meta, const __nv_bfloat16* X,
                               const int32_t* perm, float* Y, int cout, int cin, int tokens, int bshift,
                               cudaStream_t st) {
-  const int S = sparse24_tc_splits(cout, cin);
-  if (S == 0) return fail(LCP_ERR_SHAPE, "sparse24 tensor-core path: C_in = %d is not supported", cin);
-  const int kr = cin / S;
+  const int s8 = tc_splits<8>(cout, cin), s16 = s8 > 0 ? 0 : tc_splits<16>(cout, cin);
+  if (s8 == 0 && s16 == 0) return fail(LCP_ERR_SHAPE, "sparse24 tensor-core path: C_in = %d is not supported", cin);
   CUtensorMap mV, mM;
   TC_TRY(make_map(&mV, vals, (uint64_t)cin / 2, (uint64_t)cout, 64, 128, "sparse24 values"));
   TC_TRY(make_map_u32(&mM, meta, (uint64_t)cin / 32, (uint64_t)cout, 4, 128, "sparse24 positions"));
-  const int smem = StCfg::smem(kr);
-  TC_TRY(set_smem(sp24_tc_kernel, smem, "sparse24_tc"));
-  const dim3 grid((unsigned)S, (unsigned)cdiv(cout, 128));
-  for (int t0 = 0; t0 < tokens; t0 += 16) {
-    const int tt = tokens - t0 < 16 ? tokens - t0 : 16;
-    TC_TRY(launch_kernel(sp24_tc_kernel, grid, dim3(StCfg::THREADS), smem, st, S, true, "sparse24_tc", mV, mM,
-                         X + (size_t)t0 * cin, perm, Y + (size_t)t0 * cout, cout, cin, tt, bshift, kr));
-  }
-  return LCP_OK;
+  if (s8 > 0) return launch_sp24<8>(mV, mM, X, perm, Y, cout, cin, tokens, bshift, s8, st);
+  return launch_sp24<16>(mV, mM, X, perm, Y, cout, cin, tokens, bshift, s16, st);
 }
 
 }  // namespace lcp
