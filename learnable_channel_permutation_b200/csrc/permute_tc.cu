@@ -16,6 +16,9 @@ namespace {
 // P enters through the tile-format images written by the Sinkhorn kernel:
 // Pt[t][j][i] = P[i][j] (B operand of the first product, rows j of chunk c),
 // Ph[t][i][j] = P[i][j] (B operand of the second product, columns of chunk c).
+// The images of chunk c + 1 load while chunk c is finished: Pt once the first
+// product of chunk c has completed (bar_pt), Ph once its second product has
+// (bar_ph, waited for only before the second product of chunk c + 1).
 
 template <int BC> struct PmCfg {
   static constexpr int NCH = BC / 64;
@@ -42,15 +45,16 @@ permute_mask_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
   uint8_t* sPh = sPtl + C::PT_BYTES;
   uint8_t* sA = sPh + C::PH_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sA + C::A_BYTES);
-  uint32_t* holder = reinterpret_cast<uint32_t*>(bars + 4);
+  uint32_t* holder = reinterpret_cast<uint32_t*>(bars + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(holder + 1);
-  const uint32_t bar_load = smem_u32(bars + 0), bar_mma1 = smem_u32(bars + 1), bar_mma2 = smem_u32(bars + 2);
-  const uint32_t bar_drain = smem_u32(bars + 3);
+  const uint32_t bar_pt = smem_u32(bars + 0), bar_mma1 = smem_u32(bars + 1), bar_mma2 = smem_u32(bars + 2);
+  const uint32_t bar_drain = smem_u32(bars + 3), bar_ph = smem_u32(bars + 4);
 
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const int r0 = blockIdx.x * 128, t = blockIdx.y, col0 = t * BC;
   if (tid == 0) {
-    mbar_init(bar_load, 1);
+    mbar_init(bar_pt, 1);
+    mbar_init(bar_ph, 1);
     mbar_init(bar_mma1, 1);
     mbar_init(bar_mma2, 1);
     mbar_init(bar_drain, 1);
@@ -71,25 +75,31 @@ permute_mask_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
   constexpr uint32_t idesc2 = idesc_bf16(128, BC, false, false);
 
   bool ok = true;
-  int pending_load = -1;   // thread 0: parity of a load not yet seen complete
+  // thread 0: parity of a load not yet seen complete (Pt, Ph), -1 if none
+  int pending_pt = -1, pending_ph = -1;
+  auto load_pt = [&](int c) {   // the transposed images of chunk c (and, for c = 0, the W tile)
+    pending_pt = c & 1;
+    mbar_expect_tx(bar_pt, (c == 0 ? C::W_BYTES : 0) + 2 * C::PT_BYTES);
+    if (c == 0)
+      for (int kc = 0; kc < C::NCH; ++kc) tma_load_2d(smem_u32(sW + kc * 16384), &tmW, bar_pt, col0 + kc * 64, r0);
+    for (int kc = 0; kc < C::NCH; ++kc) {
+      tma_load_2d(smem_u32(sPth + kc * 8192), &tmPth, bar_pt, kc * 64, col0 + c * 64);
+      tma_load_2d(smem_u32(sPtl + kc * 8192), &tmPtl, bar_pt, kc * 64, col0 + c * 64);
+    }
+  };
+  auto load_ph = [&](int c) {   // P_hi columns of chunk c
+    pending_ph = c & 1;
+    mbar_expect_tx(bar_ph, C::PH_BYTES);
+    tma_load_2d(smem_u32(sPh), &tmPh, bar_ph, c * 64, col0);
+  };
+  if (tid == 0) {
+    load_pt(0);
+    load_ph(0);
+  }
   for (int c = 0; c < C::NCH && ok; ++c) {
     if (tid == 0) {
-      bool go = (c == 0) || mbar_wait(bar_mma2, (uint32_t)(c - 1) & 1u, abort_flag, 21);
-      if (go) {
-        pending_load = c & 1;
-        mbar_expect_tx(bar_load, (c == 0 ? C::W_BYTES : 0) + 2 * C::PT_BYTES + C::PH_BYTES);
-        if (c == 0)
-          for (int kc = 0; kc < C::NCH; ++kc)
-            tma_load_2d(smem_u32(sW + kc * 16384), &tmW, bar_load, col0 + kc * 64, r0);
-        for (int kc = 0; kc < C::NCH; ++kc) {
-          tma_load_2d(smem_u32(sPth + kc * 8192), &tmPth, bar_load, kc * 64, col0 + c * 64);
-          tma_load_2d(smem_u32(sPtl + kc * 8192), &tmPtl, bar_load, kc * 64, col0 + c * 64);
-        }
-        tma_load_2d(smem_u32(sPh), &tmPh, bar_load, c * 64, col0);
-        go = mbar_wait(bar_load, (uint32_t)c & 1u, abort_flag, 22);
-        if (go) pending_load = -1;
-      }
-      if (!go) *abort_flag = 1;
+      bool go = mbar_wait(bar_pt, (uint32_t)c & 1u, abort_flag, 22);
+      if (go) pending_pt = -1;
       if (go) {
         tc_fence_after();
 #pragma unroll 1
@@ -103,10 +113,19 @@ permute_mask_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
                        (pass | kc | k16) != 0);
         }
         mma_commit(bar_mma1);
+        // the second product of chunk c - 1 has read the A tile and Ph: the epilogue below may
+        // overwrite the former, and Ph takes chunk c (chunk 0's was loaded up front)
+        if (c > 0) {
+          go = mbar_wait(bar_mma2, (uint32_t)(c - 1) & 1u, abort_flag, 21);
+          if (go) load_ph(c);
+        }
       }
+      if (!go) *abort_flag = 1;
     }
     ok = __syncthreads_and(mbar_wait(bar_mma1, (uint32_t)c & 1u, abort_flag, 23));
     if (!ok) break;
+    // the first product of chunk c has read Pt: the next chunk's transposed images may load
+    if (tid == 0 && c + 1 < C::NCH) load_pt(c + 1);
     tc_fence_after();
     uint32_t v0[32], v1[32];
     tmem_ld32(tmem + lane_off + 0, v0);
@@ -146,12 +165,17 @@ permute_mask_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
     tc_fence_before();
     __syncthreads();
     if (tid == 0) {
-      tc_fence_after();
+      bool go = mbar_wait(bar_ph, (uint32_t)c & 1u, abort_flag, 27);
+      if (go) pending_ph = -1;
+      if (!go) *abort_flag = 1;
+      if (go) {
+        tc_fence_after();
 #pragma unroll
-      for (int k16 = 0; k16 < 4; ++k16)
-        mma_bf16(tmem + 64, sdesc(smem_u32(sA) + k16 * 32, 16, 1024), sdesc(smem_u32(sPh) + k16 * 32, 16, 1024),
-                 idesc2, (c | k16) != 0);
-      mma_commit(bar_mma2);
+        for (int k16 = 0; k16 < 4; ++k16)
+          mma_bf16(tmem + 64, sdesc(smem_u32(sA) + k16 * 32, 16, 1024), sdesc(smem_u32(sPh) + k16 * 32, 16, 1024),
+                   idesc2, (c | k16) != 0);
+        mma_commit(bar_mma2);
+      }
     }
   }
   if (ok) ok = __syncthreads_and(mbar_wait(bar_mma2, (uint32_t)(C::NCH - 1) & 1u, abort_flag, 24));
@@ -175,7 +199,8 @@ permute_mask_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
   }
   if (tid == 0) {
     // no copy or MMA of ours may still be running when the CTA exits
-    if (pending_load >= 0) mbar_wait_drain(bar_load, (uint32_t)pending_load, 25);
+    if (pending_pt >= 0) mbar_wait_drain(bar_pt, (uint32_t)pending_pt, 25);
+    if (pending_ph >= 0) mbar_wait_drain(bar_ph, (uint32_t)pending_ph, 28);
     mma_commit(bar_drain);
     mbar_wait_drain(bar_drain, 0, 26);
   }
