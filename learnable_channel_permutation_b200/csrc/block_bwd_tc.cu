@@ -501,237 +501,6 @@ block_bwd_ws128_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
   }
 }
 
-// ------------------------------------------------------- block backward ---
-// One CTA: channel tile t (BC columns) x a segment of C_out rows, in chunks of
-// 128 rows o:
-//   W'  = W_tile (P_hi + P_lo)          dA = dAt_tile P_hi          (TMEM)
-//   A = M.W', dW' = M.dA  -> bf16 operand tiles in shared memory
-//   dP += dAt_tile^T A + W_tile^T dW'   (contraction over the 128 rows: the
-//         row-major tiles are read as MN-major operands)
-// For BC = 64 the two products share one M = 128 MMA: the A operand stacks the
-// dAt and W tiles (adjacent, LBO = 16 KB) and the B operand stacks A and dW',
-// so the wanted sums are the two diagonal 64 x 64 quadrants of the result.
-// The partial dP of each segment goes to dP[s] (summed by the Sinkhorn reverse).
-
-template <int BC> struct BbCfg {
-  static constexpr int NCH = BC / 64;
-  static constexpr int T_BYTES = BC * 256;   // 128 rows x BC bf16
-  static constexpr int P_BYTES = BC * BC * 2;
-  static constexpr uint32_t TMEM_COLS = (2 * BC + 128 <= 256) ? 256u : 512u;
-  // sDAt | sW | sPth | sPtl | sAb | sdWb
-  static constexpr int SMEM = 4 * T_BYTES + 2 * P_BYTES + 1024 + 128;
-};
-
-template <int BC, int B>
-__global__ void __launch_bounds__(128)
-block_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmDAt,
-                    const __grid_constant__ CUtensorMap tmPth, const __grid_constant__ CUtensorMap tmPtl,
-                    const uint32_t* __restrict__ mask, float* __restrict__ dP, int cout, int cin,
-                    int rows_per_split) {
-  using C = BbCfg<BC>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = align1024(smem_raw);
-  uint8_t* sDAt = smem;
-  uint8_t* sW = sDAt + C::T_BYTES;
-  uint8_t* sPth = sW + C::T_BYTES;
-  uint8_t* sPtl = sPth + C::P_BYTES;
-  uint8_t* sAb = sPtl + C::P_BYTES;
-  uint8_t* sdWb = sAb + C::T_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sdWb + C::T_BYTES);
-  uint32_t* holder = reinterpret_cast<uint32_t*>(bars + 4);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(holder + 1);
-  const uint32_t bar_load = smem_u32(bars + 0), bar_mma1 = smem_u32(bars + 1), bar_mma2 = smem_u32(bars + 2);
-  const uint32_t bar_drain = smem_u32(bars + 3);
-
-  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-  const int t = blockIdx.x, s = blockIdx.y, col0 = t * BC;
-  const int rbeg = s * rows_per_split;
-  const int rend = min(cout, rbeg + rows_per_split);
-  const int nchunk = cdiv(rend - rbeg, 128);
-  if (tid == 0) {
-    mbar_init(bar_load, 1);
-    mbar_init(bar_mma1, 1);
-    mbar_init(bar_mma2, 1);
-    mbar_init(bar_drain, 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == 0) tmem_alloc(smem_u32(holder), C::TMEM_COLS);
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *holder;
-  pdl_wait();
-  pdl_trigger();
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-  const int row = warp * 32 + lane;
-  const int words = cin / 32;
-  int pending_load = -1;
-  constexpr uint32_t idesc_n = idesc_bf16(128, BC, false, false);
-  constexpr uint32_t idesc_dp = idesc_bf16(128, 128, true, true);
-  const uint32_t tW = tmem, tDA = tmem + BC, tDP = tmem + 2 * BC;
-
-  bool ok = true;
-  for (int ch = 0; ch < nchunk && ok; ++ch) {
-    const int r0 = rbeg + ch * 128;
-    if (tid == 0) {
-      bool go = (ch == 0) || mbar_wait(bar_mma2, (uint32_t)(ch - 1) & 1u, abort_flag, 31);
-      if (go) {
-        pending_load = ch & 1;
-        mbar_expect_tx(bar_load, 2 * C::T_BYTES + (ch == 0 ? 2 * C::P_BYTES : 0));
-        for (int kc = 0; kc < C::NCH; ++kc) {
-          tma_load_2d(smem_u32(sW + kc * 16384), &tmW, bar_load, col0 + kc * 64, r0);
-          tma_load_2d(smem_u32(sDAt + kc * 16384), &tmDAt, bar_load, col0 + kc * 64, r0);
-        }
-        if (ch == 0)
-          for (int kc = 0; kc < C::NCH; ++kc) {
-            tma_load_2d(smem_u32(sPth + kc * BC * 128), &tmPth, bar_load, kc * 64, col0);
-            tma_load_2d(smem_u32(sPtl + kc * BC * 128), &tmPtl, bar_load, kc * 64, col0);
-          }
-        go = mbar_wait(bar_load, (uint32_t)ch & 1u, abort_flag, 32);
-        if (go) pending_load = -1;
-      }
-      if (!go) *abort_flag = 1;
-      if (go) {
-        tc_fence_after();
-        for (int kc = 0; kc < C::NCH; ++kc)
-#pragma unroll
-          for (int k16 = 0; k16 < 4; ++k16) {
-            const uint64_t a = sdesc(smem_u32(sW + kc * 16384) + k16 * 32, 16, 1024);
-            mma_bf16(tW, a, sdesc(smem_u32(sPth + kc * BC * 128) + k16 * 32, 16, 1024), idesc_n,
-                     (kc | k16) != 0);
-            mma_bf16(tW, a, sdesc(smem_u32(sPtl + kc * BC * 128) + k16 * 32, 16, 1024), idesc_n, true);
-            mma_bf16(tDA, sdesc(smem_u32(sDAt + kc * 16384) + k16 * 32, 16, 1024),
-                     sdesc(smem_u32(sPth + kc * BC * 128) + k16 * 32, 16, 1024), idesc_n, (kc | k16) != 0);
-          }
-        mma_commit(bar_mma1);
-      }
-    }
-    ok = __syncthreads_and(mbar_wait(bar_mma1, (uint32_t)ch & 1u, abort_flag, 33));
-    if (!ok) break;
-    tc_fence_after();
-    const int grow = r0 + row;
-    const bool valid = grow < rend;
-#pragma unroll 1
-    for (int cc = 0; cc < BC / 32; ++cc) {
-      uint32_t wv[32], dv[32];
-      tmem_ld32(tW + lane_off + cc * 32, wv);
-      tmem_ld32(tDA + lane_off + cc * 32, dv);
-      tmem_ld_wait();
-      const uint32_t bits = valid ? __ldg(mask + (size_t)grow * words + col0 / 32 + cc) : 0u;
-      uint8_t* rA = sAb + (cc / 2) * 16384;
-      uint8_t* rD = sdWb + (cc / 2) * 16384;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        float fa[8], fd[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const bool keep = (bits >> (8 * q + e)) & 1u;
-          fa[e] = keep ? __uint_as_float(wv[8 * q + e]) : 0.f;
-          fd[e] = keep ? __uint_as_float(dv[8 * q + e]) : 0.f;
-        }
-        const int chunk16 = (cc & 1) * 4 + q;
-        st_sw128(rA, row, chunk16, make_uint4(pack_bf16x2(fa[0], fa[1]), pack_bf16x2(fa[2], fa[3]),
-                                              pack_bf16x2(fa[4], fa[5]), pack_bf16x2(fa[6], fa[7])));
-        st_sw128(rD, row, chunk16, make_uint4(pack_bf16x2(fd[0], fd[1]), pack_bf16x2(fd[2], fd[3]),
-                                              pack_bf16x2(fd[4], fd[5]), pack_bf16x2(fd[6], fd[7])));
-      }
-    }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0) {
-      tc_fence_after();
-      if constexpr (BC == 64) {
-        // stacked: A = [dAt | W] (M = 128), B = [A | dW'] (N = 128), LBO = 16 KB
-#pragma unroll
-        for (int k16 = 0; k16 < 8; ++k16)
-          mma_bf16(tDP, sdesc(smem_u32(sDAt) + k16 * 2048, 16384, 1024),
-                   sdesc(smem_u32(sAb) + k16 * 2048, 16384, 1024), idesc_dp, (ch | k16) != 0);
-      } else {
-#pragma unroll
-        for (int k16 = 0; k16 < 8; ++k16)
-          mma_bf16(tDP, sdesc(smem_u32(sDAt) + k16 * 2048, 16384, 1024),
-                   sdesc(smem_u32(sAb) + k16 * 2048, 16384, 1024), idesc_dp, (ch | k16) != 0);
-#pragma unroll
-        for (int k16 = 0; k16 < 8; ++k16)
-          mma_bf16(tDP, sdesc(smem_u32(sW) + k16 * 2048, 16384, 1024),
-                   sdesc(smem_u32(sdWb) + k16 * 2048, 16384, 1024), idesc_dp, true);
-      }
-      mma_commit(bar_mma2);
-    }
-  }
-  if (ok && nchunk > 0) ok = __syncthreads_and(mbar_wait(bar_mma2, (uint32_t)(nchunk - 1) & 1u, abort_flag, 34));
-  const int nb = cin / B;
-  float* dPs = dP + (size_t)s * nb * B * B;
-  if (ok) {
-    tc_fence_after();
-    if constexpr (BC == 64) {
-      // rows 0..63: dAt^T A in columns 0..63; rows 64..127: W^T dW' in columns 64..127
-      float* scratch = reinterpret_cast<float*>(sAb);   // 64 x 64 floats (free: last MMA done)
-      uint32_t r0v[32], r1v[32];
-      const uint32_t cbase = (row < 64) ? 0u : 64u;
-      tmem_ld32(tDP + lane_off + cbase, r0v);
-      tmem_ld32(tDP + lane_off + cbase + 32, r1v);
-      tmem_ld_wait();
-      if (row >= 64) {
-        float* dst = scratch + (row - 64) * 64;
-#pragma unroll
-        for (int e = 0; e < 32; ++e) { dst[e] = __uint_as_float(r0v[e]); dst[32 + e] = __uint_as_float(r1v[e]); }
-      }
-      __syncthreads();
-      if (row < 64) {
-        const float* add = scratch + row * 64;
-        float v[64];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) { v[e] = __uint_as_float(r0v[e]) + add[e]; v[32 + e] = __uint_as_float(r1v[e]) + add[32 + e]; }
-        if constexpr (B == 64) {
-          float* o = dPs + ((size_t)t * 64 + row) * 64;
-#pragma unroll
-          for (int e = 0; e < 64; ++e) o[e] = v[e];
-        } else {
-          const int qb = row / 32;            // which 32-block of the tile
-          float* o = dPs + ((size_t)(2 * t + qb) * 32 + (row - 32 * qb)) * 32;
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = v[32 * qb + e];
-        }
-      }
-    } else {
-      float* o = dPs + ((size_t)t * BC + row) * BC;
-#pragma unroll 1
-      for (int cc = 0; cc < BC / 32; ++cc) {
-        uint32_t r[32];
-        tmem_ld32(tDP + lane_off + cc * 32, r);
-        tmem_ld_wait();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) o[cc * 32 + e] = __uint_as_float(r[e]);
-      }
-    }
-  }
-  if (tid == 0) {
-    if (pending_load >= 0) mbar_wait_drain(bar_load, (uint32_t)pending_load, 35);
-    mma_commit(bar_drain);
-    mbar_wait_drain(bar_drain, 0, 36);
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 0) {
-    tc_fence_after();
-    tmem_dealloc(tmem, C::TMEM_COLS);
-  }
-}
-
-template <int BC, int B>
-lcp_status block_bwd_bc(const CUtensorMap& mW, const CUtensorMap& mD, const CUtensorMap& mPth,
-                        const CUtensorMap& mPtl, const uint32_t* mask, float* dP, int splits, int rows,
-                        int cout, int cin, cudaStream_t st) {
-  auto k = block_bwd_tc_kernel<BC, B>;
-  TC_TRY(set_smem(k, BbCfg<BC>::SMEM, "block_bwd_tc"));
-  const dim3 grid(cin / BC, splits);
-  return launch_kernel(k, grid, dim3(128), BbCfg<BC>::SMEM, st, 1, true, "block_bwd_tc", mW, mD, mPth, mPtl, mask,
-                       dP, cout, cin, rows);
-}
-
 // ------------------------------------------ block backward, B = 256 ---
 // The 256 x 256 dP_b does not fit one SM's tensor memory next to W' and dA,
 // so four CTAs share a block, CTA (qr, qc) owning the dP quadrant of rows
@@ -764,10 +533,12 @@ block_bwd_q_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
   uint8_t* sDAt = sW + 4 * Q_T_BYTES;       // 4 quarters
   uint8_t* sPth = sDAt + 4 * Q_T_BYTES;     // 4 K-quarters of the 128 image rows j
   uint64_t* bars = reinterpret_cast<uint64_t*>(sPth + 4 * Q_T_BYTES);
-  uint32_t* holder = reinterpret_cast<uint32_t*>(bars + 4);
+  uint32_t* holder = reinterpret_cast<uint32_t*>(bars + 7);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(holder + 1);
-  const uint32_t bar_load = smem_u32(bars + 0), bar_mma1 = smem_u32(bars + 1), bar_mma2 = smem_u32(bars + 2);
-  const uint32_t bar_drain = smem_u32(bars + 3);
+  // bar_q[kc]: column quarter kc of the chunk's W and dAt (and, with the first chunk, of the
+  // image) has landed, so the first products run on each quarter as it arrives
+  const uint32_t bar_q0 = smem_u32(bars + 3), bar_mma1 = smem_u32(bars + 0), bar_mma2 = smem_u32(bars + 1);
+  const uint32_t bar_drain = smem_u32(bars + 2);
 
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const int t = blockIdx.x >> 2, qr = (blockIdx.x >> 1) & 1, qc = blockIdx.x & 1;
@@ -781,7 +552,7 @@ block_bwd_q_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
   uint8_t* sAb = sW + 2 * (1 - qr) * Q_T_BYTES;     // A = M.W'  [o][j], two 64-column regions
   uint8_t* sdWb = sDAt + 2 * (1 - qr) * Q_T_BYTES;  // dW' = M.dA
   if (tid == 0) {
-    mbar_init(bar_load, 1);
+    for (int kc = 0; kc < 4; ++kc) mbar_init(bar_q0 + 8 * kc, 1);
     mbar_init(bar_mma1, 1);
     mbar_init(bar_mma2, 1);
     mbar_init(bar_drain, 1);
@@ -798,7 +569,8 @@ block_bwd_q_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
   const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
   const int row = warp * 32 + lane;
   const int words = cin / 32;
-  int pending_load = -1;
+  uint32_t pending = 0;   // thread 0: quarters with a load not yet seen complete (parity pending_par)
+  uint32_t pending_par = 0;
   constexpr uint32_t idesc_n = idesc_bf16(128, 128, false, false);
   constexpr uint32_t idesc_dp = idesc_bf16(128, 128, true, true);
   const uint32_t tW = tmem, tDA = tmem + 128, tDP = tmem + 256;
@@ -810,22 +582,20 @@ block_bwd_q_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
       // the previous chunk's dP product has read every tile this load overwrites
       bool go = (ch == 0) || mbar_wait(bar_mma2, (uint32_t)(ch - 1) & 1u, abort_flag, 41);
       if (go) {
-        pending_load = ch & 1;
-        mbar_expect_tx(bar_load, 8 * Q_T_BYTES + (ch == 0 ? 4 * Q_T_BYTES : 0));
+        pending = 0xFu;
+        pending_par = (uint32_t)ch & 1u;
         for (int kc = 0; kc < 4; ++kc) {
-          tma_load_2d(smem_u32(sW + kc * Q_T_BYTES), &tmW, bar_load, col0 + kc * 64, r0);
-          tma_load_2d(smem_u32(sDAt + kc * Q_T_BYTES), &tmDAt, bar_load, col0 + kc * 64, r0);
+          const uint32_t bq = bar_q0 + 8 * kc;
+          mbar_expect_tx(bq, 2 * Q_T_BYTES + (ch == 0 ? Q_T_BYTES : 0));
+          tma_load_2d(smem_u32(sW + kc * Q_T_BYTES), &tmW, bq, col0 + kc * 64, r0);
+          tma_load_2d(smem_u32(sDAt + kc * Q_T_BYTES), &tmDAt, bq, col0 + kc * 64, r0);
+          if (ch == 0) tma_load_2d(smem_u32(sPth + kc * Q_T_BYTES), &tmPth, bq, kc * 64, col0 + qc * 128);
         }
-        if (ch == 0)
-          for (int kc = 0; kc < 4; ++kc)
-            tma_load_2d(smem_u32(sPth + kc * Q_T_BYTES), &tmPth, bar_load, kc * 64, col0 + qc * 128);
-        go = mbar_wait(bar_load, (uint32_t)ch & 1u, abort_flag, 42);
-        if (go) pending_load = -1;
-      }
-      if (!go) *abort_flag = 1;
-      if (go) {
-        tc_fence_after();
-        for (int kc = 0; kc < 4; ++kc)
+        for (int kc = 0; kc < 4 && go; ++kc) {
+          go = mbar_wait(bar_q0 + 8 * kc, (uint32_t)ch & 1u, abort_flag, 42);
+          if (!go) break;
+          pending &= ~(1u << kc);
+          tc_fence_after();
 #pragma unroll
           for (int k16 = 0; k16 < 4; ++k16) {
             const uint64_t pd = sdesc(smem_u32(sPth + kc * Q_T_BYTES) + k16 * 32, 16, 1024);
@@ -833,8 +603,10 @@ block_bwd_q_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
             mma_bf16(tDA, sdesc(smem_u32(sDAt + kc * Q_T_BYTES) + k16 * 32, 16, 1024), pd, idesc_n,
                      (kc | k16) != 0);
           }
-        mma_commit(bar_mma1);
+        }
+        if (go) mma_commit(bar_mma1);
       }
+      if (!go) *abort_flag = 1;
     }
     ok = __syncthreads_and(mbar_wait(bar_mma1, (uint32_t)ch & 1u, abort_flag, 43));
     if (!ok) break;
@@ -902,7 +674,8 @@ block_bwd_q_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
     }
   }
   if (tid == 0) {
-    if (pending_load >= 0) mbar_wait_drain(bar_load, (uint32_t)pending_load, 45);
+    for (int kc = 0; kc < 4; ++kc)
+      if (pending & (1u << kc)) mbar_wait_drain(bar_q0 + 8 * kc, pending_par, 45);
     mma_commit(bar_drain);
     mbar_wait_drain(bar_drain, 0, 46);
   }
