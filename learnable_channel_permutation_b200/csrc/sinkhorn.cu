@@ -66,13 +66,16 @@ namespace {
 #define LCP_SINKHORN_PAIR_MIN_BLOCKS 256
 #endif
 
-// CTAs (a cluster) per B = 128 block (tuning: 1 or 2)
+// CTAs (a cluster) per B = 128 block (tuning: 1 or 2) and per B = 256 block (4 or 8)
 #ifndef LCP_SINKHORN_B128_CTAS
 #define LCP_SINKHORN_B128_CTAS 2
 #endif
+#ifndef LCP_SINKHORN_B256_CTAS
+#define LCP_SINKHORN_B256_CTAS 4
+#endif
 
 template <int B> struct SkCfg {
-  static constexpr int CS = (B == 256) ? 4 : (B == 128 ? LCP_SINKHORN_B128_CTAS : 1);  // CTAs per block
+  static constexpr int CS = (B == 256) ? LCP_SINKHORN_B256_CTAS : (B == 128 ? LCP_SINKHORN_B128_CTAS : 1);  // CTAs per block
   static constexpr int NT = (B == 32) ? 256 : (B == 64 ? 512 : 1024);
   static constexpr int R = B / CS;                                 // rows per CTA
   static constexpr int TPR = NT / R;                               // lanes per row
