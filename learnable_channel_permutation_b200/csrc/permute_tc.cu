@@ -28,10 +28,13 @@ template <int BC> struct PmCfg {
   static constexpr int A_BYTES = 16384;      // 128 rows x 64 bf16
   static constexpr uint32_t TMEM_COLS = (64 + BC <= 128) ? 128u : ((64 + BC <= 256) ? 256u : 512u);
   static constexpr int SMEM = W_BYTES + 2 * PT_BYTES + PH_BYTES + A_BYTES + 1024 + 128;
+  // 8 warps: two per TMEM lane quadrant, each taking 32 of a chunk's 64 columns (and half of
+  // At's BC columns at the end), so every SM sub-partition runs two independent epilogue warps
+  static constexpr int THREADS = 256;
 };
 
 template <int BC, int MGROUP>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(PmCfg<BC>::THREADS, 1)
 permute_mask_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmPth,
                        const __grid_constant__ CUtensorMap tmPtl, const __grid_constant__ CUtensorMap tmPh,
                        uint32_t* __restrict__ mask, __nv_bfloat16* __restrict__ At,
@@ -68,8 +71,9 @@ permute_mask_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
   const uint32_t tmem = *holder;
   pdl_wait();
   pdl_trigger();
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-  const int row = warp * 32 + lane, grow = r0 + row;
+  const int q = warp & 3, h = warp >> 2;   // TMEM lane quadrant, column half
+  const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+  const int row = q * 32 + lane, grow = r0 + row;
   const int words = cin / 32;
   constexpr uint32_t idesc1 = idesc_bf16(128, 64, false, false);
   constexpr uint32_t idesc2 = idesc_bf16(128, BC, false, false);
@@ -127,39 +131,29 @@ permute_mask_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
     // the first product of chunk c has read Pt: the next chunk's transposed images may load
     if (tid == 0 && c + 1 < C::NCH) load_pt(c + 1);
     tc_fence_after();
-    uint32_t v0[32], v1[32];
-    tmem_ld32(tmem + lane_off + 0, v0);
-    tmem_ld32(tmem + lane_off + 32, v1);
+    // this thread's 32 columns h * 32 .. of the chunk
+    uint32_t v[32];
+    tmem_ld32(tmem + lane_off + h * 32, v);
     tmem_ld_wait();
-    const uint32_t w0 = MGROUP == 4 ? nm4_keep<32>(v0, n) : nm_word<MGROUP>(v0, n);
-    const uint32_t w1 = MGROUP == 4 ? nm4_keep<32>(v1, n) : nm_word<MGROUP>(v1, n);
+    const uint32_t w = MGROUP == 4 ? nm4_keep<32>(v, n) : nm_word<MGROUP>(v, n);
     if (grow < cout) {
-      const int wi = (col0 + c * 64) / 32;
-      mask[(size_t)grow * words + wi] = w0;
-      mask[(size_t)grow * words + wi + 1] = w1;
+      mask[(size_t)grow * words + (col0 + c * 64) / 32 + h] = w;
       if (Wp_out) {
-        float4* o = reinterpret_cast<float4*>(Wp_out + (size_t)grow * cin + col0 + c * 64);
+        float4* o = reinterpret_cast<float4*>(Wp_out + (size_t)grow * cin + col0 + c * 64 + h * 32);
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
-          o[q] = make_float4(__uint_as_float(v0[4 * q]), __uint_as_float(v0[4 * q + 1]),
-                             __uint_as_float(v0[4 * q + 2]), __uint_as_float(v0[4 * q + 3]));
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-          o[8 + q] = make_float4(__uint_as_float(v1[4 * q]), __uint_as_float(v1[4 * q + 1]),
-                                 __uint_as_float(v1[4 * q + 2]), __uint_as_float(v1[4 * q + 3]));
+        for (int qq = 0; qq < 8; ++qq)
+          o[qq] = make_float4(__uint_as_float(v[4 * qq]), __uint_as_float(v[4 * qq + 1]),
+                              __uint_as_float(v[4 * qq + 2]), __uint_as_float(v[4 * qq + 3]));
       }
     }
-    // A_c = M . W'_c as bf16 into the K-major SW128 operand tile
+    // A_c = M . W'_c as bf16 into the K-major SW128 operand tile (16-byte chunks 4 h .. 4 h + 3)
 #pragma unroll
-    for (int ch = 0; ch < 8; ++ch) {
-      const uint32_t* v = ch < 4 ? v0 : v1;
-      const uint32_t w = ch < 4 ? w0 : w1;
-      const int b0 = (ch & 3) * 8;
+    for (int ch = 0; ch < 4; ++ch) {
       float f[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) f[e] = ((w >> (b0 + e)) & 1u) ? __uint_as_float(v[b0 + e]) : 0.f;
-      st_sw128(sA, row, ch, make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
-                                       pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7])));
+      for (int e = 0; e < 8; ++e) f[e] = ((w >> (8 * ch + e)) & 1u) ? __uint_as_float(v[8 * ch + e]) : 0.f;
+      st_sw128(sA, row, 4 * h + ch, make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                                               pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7])));
     }
     fence_async_smem();
     tc_fence_before();
@@ -181,8 +175,9 @@ permute_mask_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
   if (ok) ok = __syncthreads_and(mbar_wait(bar_mma2, (uint32_t)(C::NCH - 1) & 1u, abort_flag, 24));
   if (ok) {
     tc_fence_after();
+    // At columns: this warp's half of the BC
 #pragma unroll 1
-    for (int cc = 0; cc < BC / 32; ++cc) {
+    for (int cc = h * (BC / 64); cc < (h + 1) * (BC / 64); ++cc) {
       uint32_t r[32];
       tmem_ld32(tmem + lane_off + 64 + cc * 32, r);
       tmem_ld_wait();
@@ -910,7 +905,8 @@ lcp_status permute_mask_bc(const CUtensorMap& mW, const CUtensorMap& mPth, const
   auto k = permute_mask_tc_kernel<BC, MG>;
   TC_TRY(set_smem(k, PmCfg<BC>::SMEM, "permute_mask_tc"));
   const dim3 grid(cdiv(cout, 128), cin / BC);
-  return launch_kernel(k, grid, dim3(128), PmCfg<BC>::SMEM, st, 1, true, "permute_mask_tc", mW, mPth, mPtl, mPh, mask,
+  return launch_kernel(k, grid, dim3(PmCfg<BC>::THREADS), PmCfg<BC>::SMEM, st, 1, true, "permute_mask_tc", mW, mPth,
+                       mPtl, mPh, mask,
                        At, Wp, cout, cin, n);
 }
 
