@@ -521,8 +521,9 @@ block_bwd_ws128_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
 // images would not fit beside the tiles.  TMEM: W' 128 | dA 128 | dP 128.
 constexpr int Q_T_BYTES = 16384;                  // 128 rows x 64 bf16: one column quarter
 constexpr int Q_SMEM = 12 * Q_T_BYTES + 1024 + 128;
+constexpr int Q_THREADS = 256;   // eight warps (two per TMEM lane quadrant)
 
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(Q_THREADS, 1)
 block_bwd_q_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmDAt,
                    const __grid_constant__ CUtensorMap tmPth, const uint32_t* __restrict__ mask,
                    float* __restrict__ dP, int cout, int cin, int rows_per_split) {
@@ -566,8 +567,10 @@ block_bwd_q_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
   const uint32_t tmem = *holder;
   pdl_wait();
   pdl_trigger();
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-  const int row = warp * 32 + lane;
+  // eight warps: two per TMEM lane quadrant, each taking 64 of the quadrant's 128 columns
+  const int qd = warp & 3, h = warp >> 2;
+  const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
+  const int row = qd * 32 + lane;
   const int words = cin / 32;
   uint32_t pending = 0;   // thread 0: quarters with a load not yet seen complete (parity pending_par)
   uint32_t pending_par = 0;
@@ -614,7 +617,7 @@ block_bwd_q_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
     const int grow = r0 + row;
     const bool valid = grow < rend;
 #pragma unroll 1
-    for (int cc = 0; cc < 4; ++cc) {
+    for (int cc = 2 * h; cc < 2 * h + 2; ++cc) {
       uint32_t wv[32], dv[32];
       tmem_ld32(tW + lane_off + cc * 32, wv);
       tmem_ld32(tDA + lane_off + cc * 32, dv);
@@ -662,7 +665,7 @@ block_bwd_q_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
     // thread `row` holds dP row i = 128 qr + row of the quadrant, columns 128 qc + (0..127)
     float* o = dP + (size_t)s * nb * B * B + ((size_t)t * B + qr * 128 + row) * B + qc * 128;
 #pragma unroll 1
-    for (int cc = 0; cc < 4; ++cc) {
+    for (int cc = 2 * h; cc < 2 * h + 2; ++cc) {
       uint32_t r[32];
       tmem_ld32(tDP + lane_off + cc * 32, r);
       tmem_ld_wait();
@@ -724,7 +727,7 @@ lcp_status launch_block_bwd_tc(const __nv_bfloat16* W, const __nv_bfloat16* dAt,
     // the 128 transposed-image rows of one quadrant's columns, in 64-column K quarters
     TC_TRY(make_map(&mPth, img_pt_hi, BC, cin, 64, 128, "block_bwd Pt_hi"));
     TC_TRY(set_smem(block_bwd_q_kernel, Q_SMEM, "block_bwd_q"));
-    return launch_kernel(block_bwd_q_kernel, dim3((cin / 256) * 4, splits), dim3(128), Q_SMEM, st, 1, true,
+    return launch_kernel(block_bwd_q_kernel, dim3((cin / 256) * 4, splits), dim3(Q_THREADS), Q_SMEM, st, 1, true,
                          "block_bwd_q", mW, mD, mPth, mask, dP_partials, cout, cin, rows);
   }
   TC_TRY(make_map(&mPth, img_pt_hi, BC, cin, 64, BC, "block_bwd Pt_hi"));
