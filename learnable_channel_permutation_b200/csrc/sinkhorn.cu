@@ -89,20 +89,20 @@ template <int B> struct SkCfg {
   static_assert(R * TPR == NT && B * TPC == NT, "bad Sinkhorn configuration");
 };
 
-// The forward kernel's threads: for B <= 64 a 128-thread CTA (one warp per SM sub-partition,
-// 32 elements of a row and 32 of a column a thread: one shuffle per reduction and a four-warp
-// barrier per step, the step's latency being what bounds a block); the clusters of B = 128 and
-// B = 256 keep 1024 threads a CTA.
+// The B <= 64 forward kernel's threads: a 128-thread CTA (one warp per SM sub-partition, 32
+// elements of a row and 32 of a column a thread for B = 64: one shuffle per reduction and a
+// four-warp barrier per step, the step's latency being what bounds a block).
 template <int B> struct SkFwdCfg {
-  static constexpr int CS = SkCfg<B>::CS;
-  static constexpr int NT = (B <= 64) ? 128 : 1024;
-  static constexpr int R = B / CS;
+  static_assert(B <= 64, "the cluster sizes run sinkhorn_fwd_cluster_kernel");
+  static constexpr int CS = 1;
+  static constexpr int NT = 128;
+  static constexpr int R = B;
   static constexpr int TPR = NT / R;
   static constexpr int EPR = B / TPR;
   static constexpr int TPC = NT / B;
   static constexpr int EPC = R / TPC;
   static constexpr int NW = NT / 32;
-  static constexpr int MINB = (B <= 64) ? 4 : 1;   // CTAs an SM (register bound 128 / 64)
+  static constexpr int MINB = 4;   // CTAs an SM (register bound 128)
   static_assert(TPR >= 1 && TPR <= 32 && (32 % TPR) == 0, "row slices must sit inside a warp");
   static_assert(TPC >= 1 && TPC <= 32 && (32 % TPC) == 0, "column slices must sit inside a warp");
   static_assert(R * TPR == NT && B * TPC == NT, "bad Sinkhorn configuration");
@@ -216,11 +216,11 @@ __device__ __forceinline__ void block_range(float mx, float mn, float* red, floa
 // operands in the same order: the same values).  Z_0 is staged with a row pitch of B + 4
 // (16-byte rows).  The range of Z_0 is reduced from the staged registers under the barrier
 // that publishes the tile.
-// Shared memory (floats): tile[R*(B+4)] rv[R] cv[B] xm[2B] xs[2B] red[66]
+// Shared memory (floats): tile[B*(B+4)] rv[B] cv[B] red[66]
 template <int B> __host__ __device__ constexpr int fwd_ld() { return B + 4; }
 template <int B> constexpr size_t fwd_smem_base() {
   using C = SkFwdCfg<B>;
-  return sizeof(float) * (C::R * fwd_ld<B>() + C::R + B + 4 * B + 66);
+  return sizeof(float) * (C::R * fwd_ld<B>() + C::R + B + 66);
 }
 
 template <int B>
@@ -238,9 +238,7 @@ sinkhorn_fwd_kernel(const __grid_constant__ SkFwdBatch batch, float tau, int ite
   float* tile = sm;
   float* rv = tile + R * LD;   // per row of this CTA: a_i (linear) or R_i (log domain)
   float* cv = rv + R;          // per column: b_j (linear) or C_j (log domain)
-  float* xm = cv + B;          // this CTA's column partials, double-buffered by iteration parity
-  float* xs = xm + 2 * B;
-  float* red = xs + 2 * B;
+  float* red = cv + B;
 
   const int rank = cta_rank<CS>();
   const int row0 = rank * R;
@@ -310,22 +308,6 @@ sinkhorn_fwd_kernel(const __grid_constant__ SkFwdBatch batch, float tau, int ite
     zmax = fmaxf(zmax, red[w]);
     zmin = fminf(zmin, red[32 + w]);
   }
-  if constexpr (CS > 1) {
-    if (tid == 0) {
-      red[64] = zmax;
-      red[65] = zmin;
-    }
-    cluster_barrier<CS>();
-    float a = -CUDART_INF_F, bmin = CUDART_INF_F;
-#pragma unroll
-    for (int q = 0; q < CS; ++q) {
-      const float* pr = peer<CS>(red, q);
-      a = fmaxf(a, pr[64]);
-      bmin = fminf(bmin, pr[65]);
-    }
-    zmax = a;
-    zmin = bmin;
-  }
   float zr[EPR], zc[EPC];
 #pragma unroll
   for (int e = 0; e < EPR; e += 4) {
@@ -381,22 +363,9 @@ sinkhorn_fwd_kernel(const __grid_constant__ SkFwdBatch batch, float tau, int ite
           s3 = fmaf(zc[e + 3], a4.w, s3);
         }
         const float s = group_sum<TPC>((s0 + s1) + (s2 + s3));
-        if constexpr (CS == 1) {
-          if (g == 0) {
-            cv[j] = __fdividef(1.f, s);
-            if (ckpt) ck_col(k, s);
-          }
-        } else {
-          float* bs = xs + (k & 1) * B;
-          if (g == 0) bs[j] = s;
-          cluster_barrier<CS>();
-          if (g == 0) {
-            float S = 0.f;
-#pragma unroll
-            for (int q = 0; q < CS; ++q) S += peer<CS>(bs, q)[j];
-            cv[j] = __fdividef(1.f, S);
-            if (ckpt && rank == 0) ck_col(k, S);
-          }
+        if (g == 0) {
+          cv[j] = __fdividef(1.f, s);
+          if (ckpt) ck_col(k, s);
         }
         __syncthreads();
       }
@@ -441,31 +410,12 @@ sinkhorn_fwd_kernel(const __grid_constant__ SkFwdBatch batch, float tau, int ite
         }
         float m, s;
         lse_parts<EPC, TPC>(x, m, s);
-        if constexpr (CS == 1) {
-          if (g == 0) {
-            const float v = m + __logf(s);
-            cv[j] = v;
-            if (ckpt) ck_col(k, v);
-          }
-          __syncthreads();
-        } else {
-          float* bm = xm + (k & 1) * B;
-          float* bs = xs + (k & 1) * B;
-          if (g == 0) { bm[j] = m; bs[j] = s; }
-          cluster_barrier<CS>();
-          if (g == 0) {
-            float M = -CUDART_INF_F;
-#pragma unroll
-            for (int q = 0; q < CS; ++q) M = fmaxf(M, peer<CS>(bm, q)[j]);
-            float S = 0.f;
-#pragma unroll
-            for (int q = 0; q < CS; ++q) S += peer<CS>(bs, q)[j] * __expf(peer<CS>(bm, q)[j] - M);
-            const float v = M + __logf(S);
-            cv[j] = v;
-            if (ckpt && rank == 0) ck_col(k, v);
-          }
-          __syncthreads();
+        if (g == 0) {
+          const float v = m + __logf(s);
+          cv[j] = v;
+          if (ckpt) ck_col(k, v);
         }
+        __syncthreads();
       }
     }
     // P = exp(Z_0 - R - C)
@@ -541,10 +491,8 @@ sinkhorn_fwd_kernel(const __grid_constant__ SkFwdBatch batch, float tau, int ite
       }
     }
   }
-  // every thread (and every CTA of the cluster) is done with this block's shared
-  // memory before the next block overwrites it
-  if constexpr (CS > 1) cluster_barrier<CS>();
-  else __syncthreads();
+  // every thread is done with this block's shared memory before the next block overwrites it
+  __syncthreads();
   }
 }
 
@@ -1588,7 +1536,6 @@ int grid_blocks(K kernel, int nt, size_t smem, int cs, int blocks) {
 
 template <int B>
 lcp_status fwd_b(const SkFwdBatch& batch, int blocks, float tau, int iters, cudaStream_t st) {
-  using C = SkFwdCfg<B>;
   if (B == 64 && blocks >= LCP_SINKHORN_WARP_MIN_BLOCKS) {
     // one warp a block: enough blocks to keep every SM's warps busy
     const int g = grid_blocks(sinkhorn_fwd_warp_kernel, 32 * kSkWarpWarps, 0, 1,
@@ -1596,7 +1543,8 @@ lcp_status fwd_b(const SkFwdBatch& batch, int blocks, float tau, int iters, cuda
     return launch_kernel(sinkhorn_fwd_warp_kernel, dim3(g), dim3(32 * kSkWarpWarps), 0, st, 1, true, "sinkhorn_fwd",
                          batch, tau, iters);
   }
-  if constexpr (C::CS > 1) {
+  if constexpr (SkCfg<B>::CS > 1) {
+    using C = SkCfg<B>;
     const size_t smem = fwd_cluster_smem<B>();
     const lcp_status s0 = ensure_smem_limit(reinterpret_cast<const void*>(sinkhorn_fwd_cluster_kernel<B>),
                                             (int)smem, "sinkhorn_fwd");
@@ -1605,6 +1553,7 @@ lcp_status fwd_b(const SkFwdBatch& batch, int blocks, float tau, int iters, cuda
     return launch_kernel(sinkhorn_fwd_cluster_kernel<B>, dim3(g * C::CS), dim3(C::NT), smem, st, C::CS, true,
                          "sinkhorn_fwd", batch, tau, iters);
   } else {
+    using C = SkFwdCfg<B>;
     const size_t smem = fwd_smem_base<B>();
     const lcp_status s0 =
         ensure_smem_limit(reinterpret_cast<const void*>(sinkhorn_fwd_kernel<B>), (int)smem, "sinkhorn_fwd");
