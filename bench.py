@@ -527,11 +527,22 @@ def extras(args, b, synth, wl, li, layer, step, flush, pk, dev):
         del g
         ms_h = timed(lambda: b.harden(layer["P"], layer["perm"]), K)
         layer.pop("perm")
+        # the large blocks (auction solver) on the 4096 x 4096 sweep layer's initial P
+        large = {}
+        for Bl in (128, 256):
+            wl_l = synth.sweep_4096(Bl, 5, 1.0, 2, 4)
+            Ll = torch.from_numpy(synth.make_inputs(wl_l)[0].L).to(dev)
+            Pl = torch.empty_like(Ll)
+            b.sinkhorn_fwd(Ll, Pl, None, wl_l.tau, wl_l.iters)
+            perm_l = torch.empty(Ll.shape[0], Bl, dtype=torch.int32, device=dev)
+            large[f"B{Bl}"] = {"harden_kernel_ms": timed(lambda: b.harden(Pl, perm_l), min(K, 20)),
+                               "blocks": int(Ll.shape[0]), "tau": wl_l.tau}
         out["hard_step"] = {"value": 1e3 / ms, "unit": UNIT, "ms_per_step": ms, "steps": K,
-                            "harden_kernel_ms": ms_h, "blocks": nb,
+                            "harden_kernel_ms": ms_h, "blocks": nb, "large_blocks": large,
                             "note": "LCP_FLAG_HARD: the forward pass uses the per-block maximum-weight "
-                                    "assignment of the Sinkhorn output (one warp per block), the backward "
-                                    "pass is straight-through; not the headline"}
+                                    "assignment of the Sinkhorn output (B <= 64: shortest augmenting paths, "
+                                    "one warp per block; B = 128, 256: epsilon-scaling auction, one CTA per "
+                                    "block), the backward pass is straight-through; not the headline"}
 
     if want("score_step"):
         # mask from Wanda scores (LCP_FLAG_SCORE): S computed once, S_hat = S P_B ranked each step

@@ -234,8 +234,11 @@ LCP_API lcp_status lcp_score(const void* W, const void* X, void* S, float* stats
 
 /* Hardening ("Method" 2: P = argmax over permutations of Tr(P^T P_hat), the
  * Hungarian algorithm): for each of `nblocks` B x B blocks of P_hat (float32,
- * [nblocks, B, B]) the permutation maximising sum_i P_hat[i, perm[i]], solved
- * exactly (shortest augmenting paths; float32 potentials).  perm: int32
+ * [nblocks, B, B]) the permutation maximising sum_i P_hat[i, perm[i]].  B = 32
+ * and 64: solved exactly (shortest augmenting paths, float32 potentials).
+ * B = 128 and 256: an epsilon-scaling auction on P_hat quantised to 2^28..2^29
+ * levels of each block's range, whose result is within B (max - min) 2^-27 of
+ * the maximum (max, min: the block's extreme values).  perm: int32
  * [nblocks, B] (required); P_hard: float32 [nblocks, B, B] 0/1 matrices
  * (optional, NULL = not written).  B in {32, 64, 128, 256}.  When several
  * permutations attain the maximum, the result is one of them (deterministic). */

@@ -6,8 +6,12 @@
 // the hard matrix in the operand images and hand their dP to the Sinkhorn
 // reverse pass of the soft matrix.
 //
-// Solver: the Hungarian method in its shortest-augmenting-path form, exact up
-// to float32 rounding of the potentials.  Costs c[i][j] = -P_hat[i][j].  Start
+// Two solvers, chosen by block size (measured on a B200: the single-warp search
+// is the faster one for B = 32 and 64, the auction below for B = 128 and 256,
+// where the search's step count grows with B^2).
+//
+// B = 32 and 64: the Hungarian method in its shortest-augmenting-path form,
+// exact up to float32 rounding of the potentials.  Costs c[i][j] = -P_hat[i][j].  Start
 // from v[j] = min_i c[i][j] (feasible), and match every column to the row of
 // its minimum when no lower-numbered column claims that row (tight edges).
 // Then each still-free row i0 runs a Dijkstra search over reduced costs with
@@ -18,14 +22,14 @@
 // Once a free column is reached at distance D, each scanned column's
 // potential moves by d[j] - D and the matching flips along the path.
 //
-// One warp per block.  Lane l owns columns l, l + 32, ...: their potential v,
-// matched row, tentative distance, predecessor row and scanned flag live in
-// registers; the row -> column matching sits in shared memory next to the
-// block's costs (B <= 128; for B = 256 the first 216 of its 256 rows, the rest
-// read from global memory).  A
-// search step is one scan of the owned columns, one warp-wide argmin (ties:
-// lowest column) and two shuffles from the scanned column's owner, so the
-// result is deterministic.
+// One warp per block (B = 32 and 64).  Lane l owns columns l, l + 32, ...: their
+// potential v, matched row, tentative distance, predecessor row and scanned flag
+// live in registers; the row -> column matching sits in shared memory next to
+// the block's costs.  A search step is one scan of the owned columns, one
+// warp-wide argmin (ties: lowest column) and two shuffles from the scanned
+// column's owner, so the result is deterministic.
+
+#include <climits>
 
 #include <math_constants.h>
 
@@ -40,12 +44,10 @@ constexpr int kFree = -1;
 constexpr int kRoot = -2;   // the virtual column the tree of the current row grows from
 
 template <int B> struct HdCfg {
+  static_assert(B <= 64, "the shortest-path solver serves B <= 64; larger blocks use the auction");
   static constexpr int CPL = B / 32;                        // columns per lane
-  static constexpr bool SMEM_COST = B <= 128;
-  // B = 256: the first CROWS cost rows in shared memory, the rest read from global memory
-  static constexpr int CROWS = SMEM_COST ? B : 216;
-  static constexpr int WARPS = B <= 64 ? 4 : 1;             // blocks per CTA
-  static constexpr int COST_FLOATS = CROWS * B;
+  static constexpr int WARPS = 4;                           // blocks per CTA
+  static constexpr int COST_FLOATS = B * B;
   static constexpr int PER_WARP = COST_FLOATS + 3 * B;      // costs, row -> column, match, claims (4-byte words)
   static constexpr size_t SMEM = (size_t)WARPS * PER_WARP * 4;
 };
@@ -88,15 +90,12 @@ harden_kernel(const float* __restrict__ P, int* __restrict__ perm, float* __rest
   const float* Pb = P + (size_t)blk * B * B;
 
   {
-    for (int q = lane; q < C::CROWS * B / 4; q += 32) {
+    for (int q = lane; q < B * B / 4; q += 32) {
       const float4 x = reinterpret_cast<const float4*>(Pb)[q];
       cost[4 * q + 0] = -x.x; cost[4 * q + 1] = -x.y; cost[4 * q + 2] = -x.z; cost[4 * q + 3] = -x.w;
     }
   }
-  auto c_at = [&](int i, int j) -> float {
-    if constexpr (C::SMEM_COST) return cost[i * B + j];
-    else return i < C::CROWS ? cost[i * B + j] : -__ldg(Pb + (size_t)i * B + j);
-  };
+  auto c_at = [&](int i, int j) -> float { return cost[i * B + j]; };
   for (int i = lane; i < B; i += 32) { u[i] = 0.f; match[i] = kFree; way[i] = kRoot; }
   __syncwarp();
 
@@ -266,6 +265,277 @@ harden_kernel(const float* __restrict__ P, int* __restrict__ perm, float* __rest
   }
 }
 
+// ---------------------------------------------------------------------------
+// B = 128 and 256: Bertsekas' forward auction with epsilon-scaling, in Jacobi
+// rounds.  One CTA of 32 warps per block.  The benefits P_hat[i][j] are mapped
+// onto integers a_ij = rint((P_hat[i][j] - min) 2^k) over the block's own range,
+// 2^k the power of two with (max - min) 2^k in [2^28, 2^29).  Every unassigned row ("person") i bids for the column ("object")
+// j* of largest value a_ij - p_j, raising its price to
+// p_j* + (best - second best value) + eps; each column goes to its highest bid
+// (lowest row on equal bids) and displaces its previous owner.  Phases run with
+// eps a fixed fraction of the block's integer range, then divided by a fixed
+// factor down to 1; between phases a row keeps its column only while it is
+// within eps of its best value.  The final phase
+// (eps = 1) ends with every row within one unit of its best value, so the
+// assignment is within B units of the integer problem's maximum; with every
+// a_ij within half a unit of (P_hat[i][j] - min) 2^k, it is within 2 B 2^-k
+// <= B (max - min) 2^-27 of the maximum of P_hat itself.
+//
+// Each column's price and owner share one 64-bit word, price << 32 | (2^32 - 1
+// - row), so a bid is a single shared-memory atomicMax and a row knows it still
+// holds its column by reading that word.  A round reads (prices, owners) under
+// one barrier and lands its bids under the next, so the result does not depend
+// on the warps' timing.  Warp w handles rows w, w + WARPS, ...; lane l holds
+// the CPL consecutive columns l CPL, ..., and a bid is one pass over them, two
+// warp-wide integer maximum reductions and a ballot (ties: lowest column).
+// ---------------------------------------------------------------------------
+
+constexpr int kAuScaleLog2 = 29;               // benefits span [0, 2^29)
+constexpr int kAuMaxRounds = 1 << 16;          // the sizes here need ~100 to ~1200
+constexpr int kAuPriceLimit = 0x60000000;      // prices stay below ~2^29 by far; checked
+
+template <int B> struct AuCfg {
+  static_assert(B == 128 || B == 256, "the auction serves B = 128 and 256");
+  static constexpr int WARPS = 32;
+  // epsilon schedule: the first phase at the block's integer range / EPS_DIV,
+  // each next one THETA times smaller (the fastest of the schedules measured,
+  // over near-uniform, intermediate and spread Sinkhorn outputs)
+  static constexpr int EPS_DIV = B == 128 ? 128 : 512;
+  static constexpr int THETA = B == 128 ? 16 : 32;
+  static constexpr int THREADS = 32 * WARPS;
+  static constexpr int PPW = B / WARPS;                     // rows per warp
+  static constexpr int CPL = B / 32;                        // columns per lane
+  static constexpr int SROWS = B == 128 ? B : 192;          // benefit rows in shared memory
+  static constexpr int SSLOTS = SROWS / WARPS;              // a warp's rows k < SSLOTS read them there
+  static constexpr int RSLOTS = PPW - SSLOTS;               // the rest live in registers
+  static constexpr size_t BEN_BYTES = (size_t)SROWS * B * 4;
+  static constexpr size_t SMEM = BEN_BYTES + (size_t)B * 8 + 2 * 32 * 4 + 16;
+};
+
+__device__ __forceinline__ unsigned au_code(int i) { return 0xffffffffu - (unsigned)i; }
+
+// CPL consecutive ints / 64-bit words from shared memory, vectorised
+template <int CPL> __device__ __forceinline__ void au_load_ints(const int* src, int (&v)[CPL]) {
+#pragma unroll
+  for (int q = 0; q < CPL / 4; ++q) {
+    const int4 t = reinterpret_cast<const int4*>(src)[q];
+    v[4 * q] = t.x; v[4 * q + 1] = t.y; v[4 * q + 2] = t.z; v[4 * q + 3] = t.w;
+  }
+}
+template <int CPL> __device__ __forceinline__ void au_load_prices(const unsigned long long* w, int (&p)[CPL]) {
+#pragma unroll
+  for (int q = 0; q < CPL / 2; ++q) {
+    const ulonglong2 t = reinterpret_cast<const ulonglong2*>(w)[q];
+    p[2 * q] = (int)(t.x >> 32); p[2 * q + 1] = (int)(t.y >> 32);
+  }
+}
+
+template <int B>
+__global__ void __launch_bounds__(AuCfg<B>::THREADS)
+harden_auction_kernel(const float* __restrict__ P, int* __restrict__ perm, float* __restrict__ P_hard,
+                      __nv_bfloat16* __restrict__ pt_hi, __nv_bfloat16* __restrict__ pt_lo,
+                      __nv_bfloat16* __restrict__ p_hi, int nblocks) {
+  using C = AuCfg<B>;
+  constexpr int CPL = C::CPL, PPW = C::PPW, NW = C::WARPS, NT = C::THREADS;
+  pdl_wait();
+  pdl_trigger();
+  extern __shared__ __align__(16) unsigned char au_smem[];
+  int* ben = reinterpret_cast<int*>(au_smem);                                        // [SROWS][B]
+  unsigned long long* word = reinterpret_cast<unsigned long long*>(au_smem + C::BEN_BYTES);   // [B]
+  unsigned* red = reinterpret_cast<unsigned*>(word + B);                              // [2][32]
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int blk = blockIdx.x;
+  if (blk >= nblocks) return;
+  const float* Pb = P + (size_t)blk * B * B;
+
+  // the block's range: order-preserving keys, minimum and maximum over the CTA
+  unsigned kmin = 0xffffffffu, kmax = 0u;
+  for (int q = threadIdx.x; q < B * B / 4; q += NT) {
+    const float4 x = __ldg(reinterpret_cast<const float4*>(Pb) + q);
+    const unsigned k0 = sort_key(x.x), k1 = sort_key(x.y), k2 = sort_key(x.z), k3 = sort_key(x.w);
+    kmin = min(kmin, min(min(k0, k1), min(k2, k3)));
+    kmax = max(kmax, max(max(k0, k1), max(k2, k3)));
+  }
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  if (lane == 0) { red[warp] = kmin; red[32 + warp] = kmax; }
+  for (int j = threadIdx.x; j < B; j += NT) word[j] = 0ull;   // price 0, no owner
+  __syncthreads();
+  kmin = __reduce_min_sync(0xffffffffu, lane < NW ? red[lane] : 0xffffffffu);
+  kmax = __reduce_max_sync(0xffffffffu, lane < NW ? red[32 + lane] : 0u);
+  // a_ij = rint((P_ij - min) 2^k), 2^k the power of two with (max - min) 2^k in
+  // [2^28, 2^29): the difference of two floats is exact in double and so is the
+  // scaling, so every benefit is within half a unit of the exact value
+  const double lo = (double)key_value(kmin), hi = (double)key_value(kmax);
+  int ex = 0;
+  if (hi > lo) frexp(hi - lo, &ex);
+  const double scale = hi > lo ? ldexp(1.0, kAuScaleLog2 - ex) : 0.0;
+  auto quant = [&](float x) { return (int)rint(((double)x - lo) * scale); };
+  for (int q = threadIdx.x; q < C::SROWS * B / 4; q += NT) {
+    const float4 x = __ldg(reinterpret_cast<const float4*>(Pb) + q);
+    reinterpret_cast<int4*>(ben)[q] = make_int4(quant(x.x), quant(x.y), quant(x.z), quant(x.w));
+  }
+  int rben[C::RSLOTS > 0 ? C::RSLOTS : 1][CPL];
+#pragma unroll
+  for (int r = 0; r < C::RSLOTS; ++r) {
+    const int i = warp + NW * (C::SSLOTS + r);
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) rben[r][c] = quant(__ldg(Pb + (size_t)i * B + lane * CPL + c));
+  }
+  __syncthreads();
+
+  auto benefits = [&](int k, int (&a)[CPL]) {
+    if (k < C::SSLOTS) {
+      au_load_ints<CPL>(ben + (size_t)(warp + NW * k) * B + lane * CPL, a);
+    } else {
+#pragma unroll
+      for (int r = 0; r < C::RSLOTS; ++r)
+        if (k == C::SSLOTS + r) {
+#pragma unroll
+          for (int c = 0; c < CPL; ++c) a[c] = rben[r][c];
+        }
+    }
+  };
+
+  int myobj[PPW];
+#pragma unroll
+  for (int k = 0; k < PPW; ++k) myobj[k] = 0;   // word[0] has no owner yet: every row starts free
+  int eps = max(1, (int)rint((hi - lo) * scale) / C::EPS_DIV);
+  int rounds = 0;
+  bool ok = true;
+  int over = 0;   // a bid reached the price limit (clamped; reported after the search)
+  for (int phase = 0; ok; ++phase) {
+    if (phase > 0) {
+      // a row keeps its column only while its value there is within eps of its best value
+#pragma unroll
+      for (int k = 0; k < PPW; ++k) {
+        const int i = warp + NW * k;
+        const unsigned long long wo = word[myobj[k]];
+        if ((unsigned)wo == au_code(i)) {
+          int a[CPL], p[CPL];
+          benefits(k, a);
+          au_load_prices<CPL>(word + lane * CPL, p);
+          int v1 = a[0] - p[0];
+#pragma unroll
+          for (int c = 1; c < CPL; ++c) v1 = max(v1, a[c] - p[c]);
+          const int m1 = __reduce_max_sync(0xffffffffu, v1);
+          const int ol = myobj[k] / CPL, oc = myobj[k] % CPL;
+          int vo = a[0] - p[0];
+#pragma unroll
+          for (int c = 1; c < CPL; ++c)
+            if (c == oc) vo = a[c] - p[c];
+          vo = __shfl_sync(0xffffffffu, vo, ol);
+          if (m1 - vo > eps && lane == 0) word[myobj[k]] = wo & 0xffffffff00000000ull;   // release, price kept
+        }
+      }
+      __syncthreads();
+    }
+    for (;;) {
+      if (++rounds > kAuMaxRounds) { ok = false; break; }
+      unsigned pend = 0;
+      int bidv[PPW];
+      unsigned held[PPW];   // owner codes of the rows' columns, loaded together before any branch
+#pragma unroll
+      for (int k = 0; k < PPW; ++k) held[k] = (unsigned)word[myobj[k]];
+#pragma unroll
+      for (int k = 0; k < PPW; ++k) {
+        const int i = warp + NW * k;
+        bidv[k] = 0;
+        if (held[k] != au_code(i)) {   // free: bid
+          int a[CPL], p[CPL];
+          benefits(k, a);
+          au_load_prices<CPL>(word + lane * CPL, p);
+          int v1 = INT_MIN, v2 = INT_MIN, c1 = 0;
+#pragma unroll
+          for (int c = 0; c < CPL; ++c) {
+            const int v = a[c] - p[c];
+            if (v > v1) { v2 = v1; v1 = v; c1 = c; }
+            else if (v > v2) v2 = v;
+          }
+          const int m1 = __reduce_max_sync(0xffffffffu, v1);
+          const int wl = __ffs(__ballot_sync(0xffffffffu, v1 == m1)) - 1;   // lowest column attaining it
+          const int m2 = __reduce_max_sync(0xffffffffu, lane == wl ? v2 : v1);
+          int pc = p[0];
+#pragma unroll
+          for (int c = 1; c < CPL; ++c)
+            if (c == c1) pc = p[c];
+          const int cw = __shfl_sync(0xffffffffu, c1, wl);
+          const int pw = __shfl_sync(0xffffffffu, pc, wl);
+          const long long bid = (long long)pw + ((long long)m1 - m2) + eps;
+          if (bid >= kAuPriceLimit) over = 1;
+          bidv[k] = (int)min(bid, (long long)kAuPriceLimit);
+          myobj[k] = wl * CPL + cw;
+          pend |= 1u << k;
+        }
+      }
+      __syncthreads();   // every read of this round precedes every bid
+      if (lane == 0) {
+#pragma unroll
+        for (int k = 0; k < PPW; ++k)
+          if (pend & (1u << k))
+            atomicMax(&word[myobj[k]], ((unsigned long long)(unsigned)bidv[k] << 32) | au_code(warp + NW * k));
+      }
+      if (!__syncthreads_or(pend != 0u)) break;
+    }
+    if (eps == 1) break;
+    eps = max(1, eps / C::THETA);
+  }
+  if (__syncthreads_or(over)) ok = false;
+  if (!ok) {
+    if (threadIdx.x == 0) atomicCAS(&g_harden_error, 0, 202);
+    return;
+  }
+
+  // outputs: pi(i) = the column row i holds; the column -> row table for the matrices
+  int* pb = perm + (size_t)blk * B;
+  if (lane == 0) {
+#pragma unroll
+    for (int k = 0; k < PPW; ++k) pb[warp + NW * k] = myobj[k];
+  }
+  int* row_of = ben;   // the benefits are no longer read
+  __syncthreads();
+  for (int j = threadIdx.x; j < B; j += NT) row_of[j] = (int)(0xffffffffu - (unsigned)word[j]);
+  __syncthreads();
+  if (P_hard) {
+    float* H = P_hard + (size_t)blk * B * B;
+    for (int q = threadIdx.x; q < B * B / 4; q += NT) reinterpret_cast<float4*>(H)[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+    __syncthreads();
+    for (int j = threadIdx.x; j < B; j += NT)
+      if ((unsigned)row_of[j] < (unsigned)B) H[(size_t)row_of[j] * B + j] = 1.f;
+  }
+  if (pt_hi) {
+    constexpr int BC = B < 64 ? 64 : B;
+    const int gcol0 = blk * B;
+    const size_t tb = (size_t)(gcol0 / BC) * BC * BC;
+    const int q0 = gcol0 % BC;
+    const __nv_bfloat16 one = __float2bfloat16_rn(1.f), zero = __float2bfloat16_rn(0.f);
+    for (int q = threadIdx.x; q < B * B; q += NT) {
+      const int a = q / B, bcol = q % B;
+      pt_hi[tb + (size_t)(q0 + a) * BC + q0 + bcol] = zero;
+      pt_lo[tb + (size_t)(q0 + a) * BC + q0 + bcol] = zero;
+      p_hi[tb + (size_t)(q0 + a) * BC + q0 + bcol] = zero;
+    }
+    __syncthreads();
+    for (int j = threadIdx.x; j < B; j += NT) {
+      const int i = row_of[j];
+      if ((unsigned)i >= (unsigned)B) continue;   // cannot happen: every column has an owner
+      pt_hi[tb + (size_t)(q0 + j) * BC + q0 + i] = one;
+      p_hi[tb + (size_t)(q0 + i) * BC + q0 + j] = one;
+    }
+  }
+}
+
+template <int B>
+lcp_status harden_auction_b(const float* P, int* perm, float* P_hard, __nv_bfloat16* a, __nv_bfloat16* b,
+                            __nv_bfloat16* c, int nblocks, cudaStream_t st) {
+  using C = AuCfg<B>;
+  const lcp_status s0 =
+      ensure_smem_limit(reinterpret_cast<const void*>(harden_auction_kernel<B>), (int)C::SMEM, "harden");
+  if (s0 != LCP_OK) return s0;
+  return launch_kernel(harden_auction_kernel<B>, dim3(nblocks), dim3(C::THREADS), C::SMEM, st, 1, true, "harden",
+                       P, perm, P_hard, a, b, c, nblocks);
+}
+
 template <int B>
 lcp_status harden_b(const float* P, int* perm, float* P_hard, __nv_bfloat16* a, __nv_bfloat16* b,
                     __nv_bfloat16* c, int nblocks, cudaStream_t st) {
@@ -282,11 +552,11 @@ lcp_status harden_b(const float* P, int* perm, float* P_hard, __nv_bfloat16* a, 
 lcp_status launch_harden(const float* P, int* perm, float* P_hard, __nv_bfloat16* img_pt_hi,
                          __nv_bfloat16* img_pt_lo, __nv_bfloat16* img_p_hi, int nblocks, int B, cudaStream_t st) {
   if (nblocks == 0) return LCP_OK;
-  switch (B) {
+  switch (B) {   // shortest augmenting paths for the small blocks, the auction for the large ones
     case 32: return harden_b<32>(P, perm, P_hard, img_pt_hi, img_pt_lo, img_p_hi, nblocks, st);
     case 64: return harden_b<64>(P, perm, P_hard, img_pt_hi, img_pt_lo, img_p_hi, nblocks, st);
-    case 128: return harden_b<128>(P, perm, P_hard, img_pt_hi, img_pt_lo, img_p_hi, nblocks, st);
-    case 256: return harden_b<256>(P, perm, P_hard, img_pt_hi, img_pt_lo, img_p_hi, nblocks, st);
+    case 128: return harden_auction_b<128>(P, perm, P_hard, img_pt_hi, img_pt_lo, img_p_hi, nblocks, st);
+    case 256: return harden_auction_b<256>(P, perm, P_hard, img_pt_hi, img_pt_lo, img_p_hi, nblocks, st);
   }
   return fail(LCP_ERR_SHAPE, "harden: unsupported block size %d", B);
 }

@@ -38,11 +38,17 @@ def _check_valid(perm, Ph):
 
 
 @pytest.mark.parametrize("B", [32, 64, 128, 256])
-@pytest.mark.parametrize("kind", ["spread", "init_scale", "peaked"])
+@pytest.mark.parametrize("kind", ["spread", "init_scale", "peaked", "few_large"])
 def test_harden_reaches_the_maximum(gpu_lib, B, kind):
     rng = np.random.default_rng(B + len(kind))
     nb = 6
-    if kind == "peaked":
+    if kind == "few_large":
+        # a wide range (0 .. 0.6) but a maximum near 2, set by many near-tied small entries
+        P = rng.uniform(0, 1e-3, (nb, B, B))
+        for k in range(nb):
+            P[k].flat[rng.choice(B * B, size=4, replace=False)] = rng.uniform(0.3, 0.6, 4)
+        P = P.astype(np.float32)
+    elif kind == "peaked":
         pis = np.stack([rng.permutation(B) for _ in range(nb)])
         P = (0.7 * O.perm_matrix(pis) + 0.3 / B + rng.uniform(0, 1e-4, (nb, B, B))).astype(np.float32)
     else:
