@@ -756,8 +756,8 @@ def config_runs(b, synth, pk, dev, flush, K):
         del layers, inputs
         torch.cuda.empty_cache()
     out["sweep_4096"] = {"points": points, "shape": [4096, 4096, 2048],
-                         "note": "B=256 runs the block backward on CUDA cores (its 256 x 256 dP accumulator "
-                                 "does not fit the fused kernel's tensor memory)"}
+                         "note": "every point runs only tensor-core contractions; at B = 256 four CTAs "
+                                 "share a block in the block backward, each owning a 128 x 128 quadrant of dP"}
     return out
 
 
