@@ -292,7 +292,7 @@ harden_kernel(const float* __restrict__ P, int* __restrict__ perm, float* __rest
 
 constexpr int kAuScaleLog2 = 29;               // benefits span [0, 2^29)
 constexpr int kAuMaxRounds = 1 << 16;          // the sizes here need ~100 to ~1200
-constexpr int kAuPriceLimit = 0x60000000;      // prices stay below ~2^29 by far; checked
+constexpr int kAuPriceLimit = 0x60000000;      // prices stayed below 2^29 in every case measured; checked
 
 template <int B> struct AuCfg {
   static_assert(B == 128 || B == 256, "the auction serves B = 128 and 256");
@@ -309,7 +309,7 @@ template <int B> struct AuCfg {
   static constexpr int SSLOTS = SROWS / WARPS;              // a warp's rows k < SSLOTS read them there
   static constexpr int RSLOTS = PPW - SSLOTS;               // the rest live in registers
   static constexpr size_t BEN_BYTES = (size_t)SROWS * B * 4;
-  static constexpr size_t SMEM = BEN_BYTES + (size_t)B * 8 + 2 * 32 * 4 + 16;
+  static constexpr size_t SMEM = BEN_BYTES + (size_t)B * 8 + 2 * 32 * 4;   // benefits, words, range scratch
 };
 
 __device__ __forceinline__ unsigned au_code(int i) { return 0xffffffffu - (unsigned)i; }
