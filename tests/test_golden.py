@@ -3,20 +3,20 @@
 The toy fixture (tests/golden/toy_step.json, written by make_golden.py from the
 oracle) is checked two ways: the oracle replays it bit for bit, which guards
 against regressions only; and an independent float64 restatement of the pages'
-forward equations (linear-domain Sinkhorn-Knopp, a top-k N:M mask, torch's
-cosine similarity) differentiated by torch autograd reproduces its loss, P, mask
-and dL within rounding, which pins the stored values, the oracle's hand-written
-reverse pass included, to something other than the oracle.
+forward equations differentiated by torch autograd (tests/autograd_reference.py)
+reproduces its loss, P, mask and dL within rounding, which pins the stored
+values, the oracle's hand-written reverse pass included, to something other
+than the oracle.
 """
 import json
 import os
 
 import numpy as np
-import torch
-import torch.nn.functional as F
 
 from oracle import lcp_oracle as O
 from learnable_channel_permutation_b200 import synth
+
+import autograd_reference as AR
 
 HERE = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
 
@@ -30,33 +30,9 @@ def _toy():
     return g, wl, li, L
 
 
-def _autograd_step(W, X_tokens, L, tau, iters, n, m):
-    """One soft step of [PermLLM] Method 2-3 written with torch float64 ops;
-    the gradient to the logits comes from autograd, the mask is held constant."""
-    Lt = torch.tensor(L, dtype=torch.float64, requires_grad=True)
-    K = torch.exp(Lt / tau)
-    for _ in range(iters):              # Sinkhorn-Knopp on exp(L / tau): rows, then columns
-        K = K / K.sum(dim=2, keepdim=True)
-        K = K / K.sum(dim=1, keepdim=True)
-    PB = torch.block_diag(*K)
-    Wt = torch.tensor(W, dtype=torch.float64)
-    Xt = torch.tensor(X_tokens, dtype=torch.float64)          # [T, C_in]
-    Wp = Wt @ PB
-    groups = Wp.detach().abs().reshape(Wp.shape[0], -1, m)
-    top = groups.topk(n, dim=2)
-    M = torch.zeros_like(groups, dtype=torch.bool).scatter_(2, top.indices, True).reshape(Wp.shape)
-    Ys = (Xt @ PB) @ torch.where(M, Wp, 0.0).T                  # permuted inputs times the pruned W'
-    Yd = Xt @ Wt.T
-    loss = (1.0 - F.cosine_similarity(Yd, Ys, dim=1)).mean()
-    loss.backward()
-    dropped = torch.where(M.reshape(groups.shape), -torch.inf, groups).amax(dim=2)
-    gap = float((top.values[..., -1] - dropped).min())         # > 0: the mask is unique
-    return dict(loss=float(loss.detach()), P=K.detach().numpy(), mask=M.numpy(), dL=Lt.grad.numpy(), gap=gap)
-
-
 def test_toy_fixture_matches_an_autograd_restatement():
     g, wl, li, L = _toy()
-    ref = _autograd_step(li.W, li.X, L, wl.tau, wl.iters, wl.n, wl.m)
+    ref = AR.autograd_step(li.W, li.X, L, wl.tau, wl.iters, wl.n, wl.m)
     assert ref["gap"] > 1e-9          # the two W' agree to ~1e-16: rounding cannot flip the mask
     P = np.array([float(v) for v in g["P"]]).reshape(ref["P"].shape)
     dL = np.array([float(v) for v in g["dL"]]).reshape(ref["dL"].shape)

@@ -16,6 +16,8 @@ import pytest
 
 from oracle import lcp_oracle as O
 
+import autograd_reference as AR
+
 
 def rand(shape, seed, scale=1.0):
     return np.random.default_rng(seed).standard_normal(shape) * scale
@@ -725,3 +727,50 @@ def test_sparse24_mm_by_explicit_loops():
         for o in range(3):
             ref = sum(vals[o, k] * X[t, src[4 * (k // 2) + idx[o, k]]] for k in range(8))
             assert math.isclose(Y[t, o], ref, rel_tol=1e-12, abs_tol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# The reverse pass against autograd of an independent torch restatement
+# ---------------------------------------------------------------------------
+
+def _small(seed, B, cin_blocks=2, cout=12, T=10, lscale=0.5):
+    rng = np.random.default_rng(seed)
+    W = rng.standard_normal((cout, cin_blocks * B)) * 0.02
+    X = rng.standard_normal((T, cin_blocks * B))
+    L = rng.standard_normal((cin_blocks, B, B)) * lscale
+    return W, X, L
+
+
+def _agree(out, ref):
+    assert ref["gap"] > 1e-9                       # the mask is unique: rounding cannot flip it
+    assert np.array_equal(out["mask"], ref["mask"])
+    assert abs(out["loss"] - ref["loss"]) <= 1e-12 * abs(ref["loss"])
+    nrm = np.linalg.norm(ref["dL"])
+    assert nrm > 0 and np.linalg.norm(out["dL"] - ref["dL"]) <= 1e-12 * nrm
+
+
+@pytest.mark.parametrize("B,n,m,iters,tau", [(8, 2, 4, 1, 1.0), (8, 2, 4, 5, 0.5), (16, 4, 8, 3, 0.2),
+                                             (16, 2, 4, 20, 0.1)])
+def test_dL_equals_autograd_of_a_torch_restatement(B, n, m, iters, tau):
+    W, X, L = _small(40 + B + iters, B)
+    ref = AR.autograd_step(W, X, L, tau, iters, n, m)
+    out = O.step(W, X, L, tau, iters, n, m)
+    assert np.max(np.abs(out["P"] - ref["P"])) <= 1e-13
+    _agree(out, ref)
+
+
+def test_hardened_step_equals_autograd_with_a_straight_through_estimator():
+    W, X, L = _small(51, 16, lscale=1.0)
+    out = O.step_hard(W, X, L, 0.5, 5, 2, 4)
+    ref = AR.autograd_step(W, X, L, 0.5, 5, 2, 4, hard_perm=out["perm"])
+    assert np.max(np.abs(out["P_soft"] - ref["P"])) <= 1e-13
+    _agree(out, ref)
+
+
+@pytest.mark.parametrize("kind", ["wanda", "ria"])
+def test_score_ranked_mask_step_equals_autograd(kind):
+    W, X, L = _small(52, 8)
+    S = O.importance(W, X, kind)
+    out = O.step(W, X, L, 0.5, 5, 2, 4, score=S)
+    ref = AR.autograd_step(W, X, L, 0.5, 5, 2, 4, score=S)
+    _agree(out, ref)
