@@ -125,7 +125,9 @@ LCP_API lcp_status lcp_workspace_size(const lcp_layer* layers, int nlayers, cons
                               size_t* bytes);
 
 /* One forward + backward step for each of `nlayers` independent layers
- * (each with its own W, L, P, dL and loss; X may be shared).  `ws` is a device
+ * (each with its own W, L, P, dL and loss; X may be shared).  Cites: the whole
+ * "Method" section and its "optimization objective" (the loss above and its
+ * gradient to L).  `ws` is a device
  * buffer of at least lcp_workspace_size() bytes, 256-byte aligned, owned by the
  * caller and not used concurrently by another call.  nlayers == 0 is a no-op. */
 LCP_API lcp_status lcp_step(const lcp_layer* layers, int nlayers, const lcp_hparams* hp, void* ws,
@@ -174,7 +176,9 @@ LCP_API lcp_status lcp_step_launches(const lcp_layer* layers, int nlayers, const
 LCP_API lcp_status lcp_sinkhorn_fwd(const float* L, float* P, float* ckpt, int nblocks, int B, float tau,
                             int iters, cudaStream_t stream);
 
-/* Reverse pass of lcp_sinkhorn_fwd: dL = d loss / d L given d loss / d P.
+/* Reverse pass of lcp_sinkhorn_fwd ("Method", 1: the gradient flows back
+ * through every row and column normalisation): dL = d loss / d L given
+ * d loss / d P.
  * dP holds dP_splits partial gradients [dP_splits, nblocks, B, B] that are
  * summed in index order (deterministic).  ckpt from lcp_sinkhorn_fwd with the
  * same L, tau and iters. */
@@ -199,7 +203,8 @@ typedef struct {
   float* v;
 } lcp_adamw_state;
 
-/* One AdamW update of n float32 parameters in place (g = dL; n a multiple of 4;
+/* One AdamW update ("Implementation details": AdamW on the logits) of n float32
+ * parameters in place (g = dL; n a multiple of 4;
  * every pointer 16-byte aligned).  t >= 1. */
 LCP_API lcp_status lcp_adamw(float* L, const float* dL, float* m, float* v, long long n,
                              const lcp_adamw_params* opt, int t, cudaStream_t stream);
@@ -266,7 +271,8 @@ LCP_API lcp_status nm_mask(const void* Wp, uint32_t* mask_bits, int rows, int co
 LCP_API lcp_status lcp_loss_fwd(const float* Yd, const float* Ys, float* loss, float* stats, int cout,
                         int tokens, cudaStream_t stream);
 
-/* G = d loss / d Ys for the loss above, written in `dtype` ([tokens, cout]);
+/* G = d loss / d Ys for the loss above ("optimization objective": the gradient
+ * of 1 - cos(y_d, y_s) with respect to y_s), written in `dtype` ([tokens, cout]);
  * stats from lcp_loss_fwd on the same Yd, Ys. */
 LCP_API lcp_status lcp_loss_bwd(const float* Yd, const float* Ys, const float* stats, void* G, int cout,
                         int tokens, lcp_dtype dtype, cudaStream_t stream);
@@ -294,7 +300,8 @@ LCP_API lcp_status lcp_calib_gemm(const void* X, const void* W, const void* At, 
 LCP_API lcp_status lcp_calib_gemm_loss(const void* X, const void* W, const void* At, void* D, void* Ys,
                                        float* partials, int tokens, int cout, int cin, cudaStream_t stream);
 
-/* The token-averaged cosine loss and G = d loss / d Ys (bf16 [T, C_out]) from
+/* ("optimization objective") The token-averaged cosine loss and G = d loss / d Ys
+ * (bf16 [T, C_out]) from
  * lcp_calib_gemm_loss's outputs: the slot partials of each token, summed in a
  * fixed order, give c_t = <y_d,y_s> / max(|y_d||y_s|, 1e-8) and the loss
  * (1/T) sum_t (1 - c_t); G_t = -(1/T)(y_d / (|y_d||y_s|) - c_t y_s / |y_s|^2)
@@ -304,7 +311,8 @@ LCP_API lcp_status lcp_calib_gemm_loss(const void* X, const void* W, const void*
 LCP_API lcp_status lcp_loss_pair(const void* D, const void* Ys, const float* partials, float* loss, float* stats,
                                  void* G, unsigned* counter, int cout, int tokens, cudaStream_t stream);
 
-/* Weight gradient of the sparse output on the tensor cores: dAt = G^T X with
+/* Weight gradient of the sparse output on the tensor cores ("optimization
+ * objective" with "Method", 3: y_s = At x, so d loss / d At = G^T X): dAt = G^T X with
  * G [T, C_out] and X [T, C_in] bf16 and dAt [C_out, C_in] bf16 (float32
  * accumulation over the T tokens). */
 LCP_API lcp_status lcp_grad_gemm(const void* G, const void* X, void* dAt, int tokens, int cout,
@@ -325,7 +333,8 @@ LCP_API lcp_status lcp_grad_gemm(const void* G, const void* X, void* dAt, int to
  * and recorded in lcp_device_error (302); a perm that is not a permutation of
  * its block gives unspecified (in-bounds) results. */
 
-/* Compressed weight from W [C_out, C_in] (original column order, `dtype`), perm
+/* ("Effect on inference acceleration": the 2:4 weight stored for sparse
+ * tensor cores) Compressed weight from W [C_out, C_in] (original column order, `dtype`), perm
  * (NULL: identity, B then only needs to divide C_in; 0 is accepted) and the
  * mask bits of M [C_out, C_in/32] in permuted order (as lcp_step writes them
  * for LCP_FLAG_HARD).  A group without exactly two kept bits is written as
@@ -340,7 +349,8 @@ LCP_API lcp_status lcp_pack24(const void* W, const int32_t* perm, const uint32_t
 LCP_API lcp_status lcp_gather(const void* X, const int32_t* perm, void* Xp, int tokens, int cin, int B,
                               lcp_dtype dtype, cudaStream_t stream);
 
-/* The deployed product Y = x_pi A^T for every token: X [T, C_in] in `dtype`
+/* ("Effect on inference acceleration": the permuted, 2:4-sparse layer at run
+ * time) The deployed product Y = x_pi A^T for every token: X [T, C_in] in `dtype`
  * (original channel order when perm is given, already permuted when perm is
  * NULL), values / meta as above, Y [T, C_out] float32 (float32 accumulation).
  * Built for decode-sized T (tiles of up to 16 tokens; larger T runs tile by
@@ -364,7 +374,7 @@ LCP_API lcp_status lcp_device_error(int* site, int reset);
 LCP_API lcp_status lcp_selftest_bounded_wait(int* site);
 
 /* Allocation-free variant of lcp_loss_fwd (the paper has no counterpart; this
- * is a library convenience).  Same loss, same arguments minus the scratch
+ * is a library convenience).  Same loss ("optimization objective"), same arguments minus the scratch
  * buffer: the per-token scratch lives in a static __device__ array of
  * LCP_STATIC_MAX_TOKENS * 4 floats (1 MiB) that every GPU loading the library
  * holds until exit.  For callers that cannot allocate device memory: embedders
