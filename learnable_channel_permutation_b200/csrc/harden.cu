@@ -288,6 +288,13 @@ harden_kernel(const float* __restrict__ P, int* __restrict__ perm, float* __rest
 // on the warps' timing.  Warp w handles rows w, w + WARPS, ...; lane l holds
 // the CPL consecutive columns l CPL, ..., and a bid is one pass over them, two
 // warp-wide integer maximum reductions and a ballot (ties: lowest column).
+//
+// Every thread tracks how many rows are free (a bid that finds its column
+// without an owner leaves one fewer; a release one more).  When a single row
+// is free, the rest of the phase is that row's chain of displacements: warp 0
+// runs it alone, writing each bid directly (no barrier, no atomic), until a bid
+// takes a column nobody holds -- the same bids the Jacobi rounds would make,
+// one a round, without two CTA barriers each.
 // ---------------------------------------------------------------------------
 
 constexpr int kAuScaleLog2 = 29;               // benefits span [0, 2^29)
@@ -309,7 +316,8 @@ template <int B> struct AuCfg {
   static constexpr int SSLOTS = SROWS / WARPS;              // a warp's rows k < SSLOTS read them there
   static constexpr int RSLOTS = PPW - SSLOTS;               // the rest live in registers
   static constexpr size_t BEN_BYTES = (size_t)SROWS * B * 4;
-  static constexpr size_t SMEM = BEN_BYTES + (size_t)B * 8 + 2 * 32 * 4;   // benefits, words, range scratch
+  // benefits, words, range scratch, row -> column table
+  static constexpr size_t SMEM = BEN_BYTES + (size_t)B * 8 + 2 * 32 * 4 + (size_t)B * 4;
 };
 
 __device__ __forceinline__ unsigned au_code(int i) { return 0xffffffffu - (unsigned)i; }
@@ -343,6 +351,7 @@ harden_auction_kernel(const float* __restrict__ P, int* __restrict__ perm, float
   int* ben = reinterpret_cast<int*>(au_smem);                                        // [SROWS][B]
   unsigned long long* word = reinterpret_cast<unsigned long long*>(au_smem + C::BEN_BYTES);   // [B]
   unsigned* red = reinterpret_cast<unsigned*>(word + B);                              // [2][32]
+  int* obj_of = reinterpret_cast<int*>(red + 64);                                     // [B]
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int blk = blockIdx.x;
   if (blk >= nblocks) return;
@@ -397,9 +406,19 @@ harden_auction_kernel(const float* __restrict__ P, int* __restrict__ perm, float
     }
   };
 
+  auto any_row = [&](int i, int (&a)[CPL]) {   // rows past SROWS from global memory, quantised alike
+    if (i < C::SROWS) {
+      au_load_ints<CPL>(ben + (size_t)i * B + lane * CPL, a);
+    } else {
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) a[c] = quant(__ldg(Pb + (size_t)i * B + lane * CPL + c));
+    }
+  };
+
   int myobj[PPW];
 #pragma unroll
   for (int k = 0; k < PPW; ++k) myobj[k] = 0;   // word[0] has no owner yet: every row starts free
+  int nfree = B;   // rows without a column, the same in every thread
   int eps = max(1, (int)rint((hi - lo) * scale) / C::EPS_DIV);
   int rounds = 0;
   bool ok = true;
@@ -407,6 +426,7 @@ harden_auction_kernel(const float* __restrict__ P, int* __restrict__ perm, float
   for (int phase = 0; ok; ++phase) {
     if (phase > 0) {
       // a row keeps its column only while its value there is within eps of its best value
+      unsigned rel = 0;
 #pragma unroll
       for (int k = 0; k < PPW; ++k) {
         const int i = warp + NW * k;
@@ -425,13 +445,83 @@ harden_auction_kernel(const float* __restrict__ P, int* __restrict__ perm, float
           for (int c = 1; c < CPL; ++c)
             if (c == oc) vo = a[c] - p[c];
           vo = __shfl_sync(0xffffffffu, vo, ol);
-          if (m1 - vo > eps && lane == 0) word[myobj[k]] = wo & 0xffffffff00000000ull;   // release, price kept
+          if (m1 - vo > eps) {
+            if (lane == 0) word[myobj[k]] = wo & 0xffffffff00000000ull;   // release, price kept
+            rel |= 1u << k;
+          }
         }
       }
-      __syncthreads();
+      nfree += __syncthreads_count(lane < PPW && ((rel >> lane) & 1u));
     }
     for (;;) {
       if (++rounds > kAuMaxRounds) { ok = false; break; }
+      if (nfree == 0) break;
+      if (nfree == 1) {
+        // one free row: its chain of displacements runs on warp 0 alone, each bid
+        // written directly (no barrier, no atomic), until a bid takes a free column
+        if (lane == 0) {
+#pragma unroll
+          for (int k = 0; k < PPW; ++k) obj_of[warp + NW * k] = myobj[k];
+        }
+        if (threadIdx.x == 0) red[0] = 0u;
+        __syncthreads();
+        if (warp == 0) {
+          int f = -1;
+          for (int i0 = 0; i0 < B; i0 += 32) {
+            const unsigned bal =
+                __ballot_sync(0xffffffffu, (unsigned)word[obj_of[i0 + lane]] != au_code(i0 + lane));
+            if (f < 0 && bal != 0u) f = i0 + __ffs(bal) - 1;
+          }
+          for (int chain = 0; f >= 0; ++chain) {
+            if (chain >= kAuMaxRounds) {
+              if (lane == 0) red[0] = 1u;
+              break;
+            }
+            int a[CPL], p[CPL];
+            unsigned own[CPL];
+            any_row(f, a);
+#pragma unroll
+            for (int q = 0; q < CPL / 2; ++q) {
+              const ulonglong2 t = reinterpret_cast<const ulonglong2*>(word + lane * CPL)[q];
+              p[2 * q] = (int)(t.x >> 32); own[2 * q] = (unsigned)t.x;
+              p[2 * q + 1] = (int)(t.y >> 32); own[2 * q + 1] = (unsigned)t.y;
+            }
+            int v1 = INT_MIN, v2 = INT_MIN, c1 = 0;
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) {
+              const int v = a[c] - p[c];
+              if (v > v1) { v2 = v1; v1 = v; c1 = c; }
+              else if (v > v2) v2 = v;
+            }
+            const int m1 = __reduce_max_sync(0xffffffffu, v1);
+            const int wl = __ffs(__ballot_sync(0xffffffffu, v1 == m1)) - 1;
+            const int m2 = __reduce_max_sync(0xffffffffu, lane == wl ? v2 : v1);
+            int pc = p[0];
+            unsigned oc = own[0];
+#pragma unroll
+            for (int c = 1; c < CPL; ++c)
+              if (c == c1) { pc = p[c]; oc = own[c]; }
+            const int cw = __shfl_sync(0xffffffffu, c1, wl);
+            const int pw = __shfl_sync(0xffffffffu, pc, wl);
+            const unsigned prev = __shfl_sync(0xffffffffu, oc, wl);
+            const long long bid = (long long)pw + ((long long)m1 - m2) + eps;
+            if (bid >= kAuPriceLimit) over = 1;
+            const int j = wl * CPL + cw;
+            if (lane == 0) {
+              word[j] = ((unsigned long long)(unsigned)min(bid, (long long)kAuPriceLimit) << 32) | au_code(f);
+              obj_of[f] = j;
+            }
+            __syncwarp();
+            f = prev != 0u ? (int)(0xffffffffu - prev) : -1;   // the displaced owner bids next
+          }
+        }
+        __syncthreads();
+        if (red[0] != 0u) { ok = false; break; }
+#pragma unroll
+        for (int k = 0; k < PPW; ++k) myobj[k] = obj_of[warp + NW * k];
+        nfree = 0;
+        break;
+      }
       unsigned pend = 0;
       int bidv[PPW];
       unsigned held[PPW];   // owner codes of the rows' columns, loaded together before any branch
@@ -469,13 +559,17 @@ harden_auction_kernel(const float* __restrict__ P, int* __restrict__ perm, float
         }
       }
       __syncthreads();   // every read of this round precedes every bid
-      if (lane == 0) {
+      // lane k lands bid k; a bid that finds its column without an owner leaves one row
+      // fewer free (exactly one bid on such a column sees that, whichever wins)
+      bool took = false;
 #pragma unroll
-        for (int k = 0; k < PPW; ++k)
-          if (pend & (1u << k))
-            atomicMax(&word[myobj[k]], ((unsigned long long)(unsigned)bidv[k] << 32) | au_code(warp + NW * k));
-      }
-      if (!__syncthreads_or(pend != 0u)) break;
+      for (int k = 0; k < PPW; ++k)
+        if (lane == k && (pend & (1u << k))) {
+          const unsigned long long old =
+              atomicMax(&word[myobj[k]], ((unsigned long long)(unsigned)bidv[k] << 32) | au_code(warp + NW * k));
+          took = (unsigned)old == 0u;
+        }
+      nfree -= __syncthreads_count(took);
     }
     if (eps == 1) break;
     eps = max(1, eps / C::THETA);
