@@ -302,17 +302,17 @@ constexpr int kAuMaxRounds = 1 << 16;          // the sizes here need ~100 to ~1
 constexpr int kAuPriceLimit = 0x60000000;      // prices stayed below 2^29 in every case measured; checked
 
 template <int B> struct AuCfg {
-  static_assert(B == 128 || B == 256, "the auction serves B = 128 and 256");
-  static constexpr int WARPS = 32;
+  static_assert(B == 64 || B == 128 || B == 256, "the auction serves B = 64, 128 and 256");
+  static constexpr int WARPS = B == 64 ? 16 : 32;
   // epsilon schedule: the first phase at the block's integer range / EPS_DIV,
   // each next one THETA times smaller (the fastest of the schedules measured,
   // over near-uniform, intermediate and spread Sinkhorn outputs)
-  static constexpr int EPS_DIV = B == 128 ? 128 : 512;
-  static constexpr int THETA = B == 128 ? 16 : 32;
+  static constexpr int EPS_DIV = B == 64 ? 256 : (B == 128 ? 128 : 512);
+  static constexpr int THETA = B == 64 ? 64 : (B == 128 ? 16 : 32);
   static constexpr int THREADS = 32 * WARPS;
   static constexpr int PPW = B / WARPS;                     // rows per warp
   static constexpr int CPL = B / 32;                        // columns per lane
-  static constexpr int SROWS = B == 128 ? B : 192;          // benefit rows in shared memory
+  static constexpr int SROWS = B <= 128 ? B : 192;          // benefit rows in shared memory
   static constexpr int SSLOTS = SROWS / WARPS;              // a warp's rows k < SSLOTS read them there
   static constexpr int RSLOTS = PPW - SSLOTS;               // the rest live in registers
   static constexpr size_t BEN_BYTES = (size_t)SROWS * B * 4;
@@ -324,6 +324,11 @@ __device__ __forceinline__ unsigned au_code(int i) { return 0xffffffffu - (unsig
 
 // CPL consecutive ints / 64-bit words from shared memory, vectorised
 template <int CPL> __device__ __forceinline__ void au_load_ints(const int* src, int (&v)[CPL]) {
+  if constexpr (CPL == 2) {
+    const int2 t = *reinterpret_cast<const int2*>(src);
+    v[0] = t.x; v[1] = t.y;
+    return;
+  }
 #pragma unroll
   for (int q = 0; q < CPL / 4; ++q) {
     const int4 t = reinterpret_cast<const int4*>(src)[q];
@@ -648,7 +653,12 @@ lcp_status launch_harden(const float* P, int* perm, float* P_hard, __nv_bfloat16
   if (nblocks == 0) return LCP_OK;
   switch (B) {   // shortest augmenting paths for the small blocks, the auction for the large ones
     case 32: return harden_b<32>(P, perm, P_hard, img_pt_hi, img_pt_lo, img_p_hi, nblocks, st);
-    case 64: return harden_b<64>(P, perm, P_hard, img_pt_hi, img_pt_lo, img_p_hi, nblocks, st);
+#ifndef LCP_HARDEN_AUCTION_64
+#define LCP_HARDEN_AUCTION_64 0   // 1: the auction at B = 64 (faster on spread P, slower near the initialisation)
+#endif
+    case 64:
+      if (LCP_HARDEN_AUCTION_64) return harden_auction_b<64>(P, perm, P_hard, img_pt_hi, img_pt_lo, img_p_hi, nblocks, st);
+      return harden_b<64>(P, perm, P_hard, img_pt_hi, img_pt_lo, img_p_hi, nblocks, st);
     case 128: return harden_auction_b<128>(P, perm, P_hard, img_pt_hi, img_pt_lo, img_p_hi, nblocks, st);
     case 256: return harden_auction_b<256>(P, perm, P_hard, img_pt_hi, img_pt_lo, img_p_hi, nblocks, st);
   }
